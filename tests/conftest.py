@@ -1,0 +1,19 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 and the built CUDA library")
+    config.addinivalue_line("markers", "slow: full-size workload (minutes)")
+
+
+def pytest_collection_modifyitems(config, items):
+    # GPU tests never pass silently on a machine without a GPU: if one is
+    # selected there, it fails in its fixture with a clear message.
+    pass

@@ -1,0 +1,143 @@
+"""Pins of the oracle's softmax-gated pooling and requantisation: printed
+entry counts, identity at pool = stride = 1, closed forms for uniform gates,
+the bias-to-slot mapping, the gate's source vector, convexity.  CPU only."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_entry_counts_match_stated_workloads():
+    n = 0
+    for line in open(os.path.join(GOLDEN, "entry_counts.txt")):
+        line = line.split("#")[0].strip()
+        if line:
+            t, s, e = map(int, line.split())
+            assert O.n_entries(t, s) == e
+            n += 1
+    assert n >= 4
+
+
+def test_pool_positions_overlap_previous_group():
+    # CSA: window 8, stride 4 -> previous group + own group
+    assert list(O.pool_positions(0, 8, 4)) == [-4, -3, -2, -1, 0, 1, 2, 3]
+    assert list(O.pool_positions(5, 8, 4)) == list(range(16, 24))
+    # HCA: window = stride = 128 -> disjoint blocks
+    assert list(O.pool_positions(2, 128, 128)) == list(range(256, 384))
+
+
+def _scalar_tokens(D=3):
+    # token p carries the value p in every dim
+    return lambda p: np.full(D, float(p))
+
+
+def test_identity_when_pool_equals_stride_equals_one():
+    rng = np.random.default_rng(0)
+    X = rng.standard_normal((37, 6))
+    src = lambda p: X[p]
+    (out,), w = O.pool_entries(src, [src], rng.standard_normal(6), rng.standard_normal(1), 1, 1,
+                               range(37))
+    assert np.array_equal(out, X)
+    assert np.all(w == 1.0)
+
+
+def test_uniform_gates_give_window_mean_csa():
+    src = _scalar_tokens()
+    (out,), w = O.pool_entries(src, [src], np.zeros(3), np.zeros(8), 8, 4, range(6))
+    # entry 0 sees positions 0..3 only (left edge), entry j>=1 sees 4j-4..4j+3
+    assert np.allclose(out[0], 1.5, rtol=0, atol=1e-15)
+    for j in range(1, 6):
+        assert np.allclose(out[j], 4 * j - 0.5, rtol=0, atol=1e-13)
+    assert np.allclose(w[0], [0, 0, 0, 0, 0.25, 0.25, 0.25, 0.25])
+
+
+def test_uniform_gates_give_window_mean_hca():
+    src = _scalar_tokens()
+    (out,), _ = O.pool_entries(src, [src], np.zeros(3), np.zeros(128), 128, 128, range(3))
+    for j in range(3):
+        assert np.allclose(out[j], 128 * j + 63.5, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("slot", [0, 3, 4, 7])
+def test_positional_bias_selects_slot(slot):
+    src = _scalar_tokens()
+    b = np.zeros(8)
+    b[slot] = 60.0       # e^60 dominates every other slot
+    (out,), _ = O.pool_entries(src, [src], np.zeros(3), b, 8, 4, [3])
+    assert np.allclose(out[0], 4 * 3 - 4 + slot, rtol=1e-12)
+
+
+def test_gate_reads_the_key_not_the_value():
+    rng = np.random.default_rng(1)
+    K = rng.standard_normal((16, 4)) * 0.01
+    V = rng.standard_normal((16, 4))
+    K[9, 2] = 40.0                      # token 9 has a large key component on dim 2
+    w = np.zeros(4); w[2] = 1.0         # the gate looks at key dim 2 only
+    (ok, ov), _ = O.pool_entries(lambda p: K[p], [lambda p: K[p], lambda p: V[p]], w,
+                                 np.zeros(8), 8, 4, [2, 3])
+    # token 9 lies in the windows of entries 2 (4..11) and 3 (8..15)
+    for row in (0, 1):
+        assert np.allclose(ov[row], V[9], rtol=1e-12, atol=1e-12)
+
+
+def test_weights_sum_to_one_and_convexity():
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((64, 5))
+    src = lambda p: X[p]
+    (out,), w = O.pool_entries(src, [src], rng.standard_normal(5), rng.standard_normal(8),
+                               8, 4, range(16))
+    assert np.allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    for j in range(16):
+        pos = O.pool_positions(j, 8, 4)
+        pos = pos[pos >= 0]
+        assert np.all(out[j] <= X[pos].max(axis=0) + 1e-14)
+        assert np.all(out[j] >= X[pos].min(axis=0) - 1e-14)
+
+
+def test_requantize_roundtrip_and_amax():
+    rng = np.random.default_rng(3)
+    # values already on the E4M3 grid at scale s = amax/448 quantise to themselves
+    codes = rng.integers(0, 0x7E, size=(10, 128)).astype(np.uint8)
+    codes[:, 0] = 0x7E                      # force the block amax to 448 * s
+    codes[:, 64] = 0xFE
+    s = rng.uniform(0.5, 2.0, size=(10, 2))
+    c = O.e4m3_decode(codes) * np.repeat(s, 64, axis=1)
+    c = np.concatenate([c, rng.standard_normal((10, 64))], axis=1)
+    qc, qs, qr = O.requantize(c, 128)
+    assert np.array_equal(qc, codes)
+    assert np.allclose(qs, s, rtol=1e-15, atol=0)
+    assert np.array_equal(qr, O.bf16_encode(c[:, 128:]))
+
+
+def test_requantize_zero_block_and_codes_match_torch():
+    rng = np.random.default_rng(4)
+    c = rng.standard_normal((50, 448 + 64)) * 3
+    c[7, 64:128] = 0.0
+    qc, qs, _ = O.requantize(c, 448)
+    assert qs[7, 1] == 1.0 and np.all(qc[7, 64:128] == 0)
+    assert np.all(np.abs(O.e4m3_decode(qc)) <= 448)
+    # every block's largest magnitude lands on 448 exactly
+    for b in range(7):
+        blk = np.abs(O.e4m3_decode(qc[:, 64 * b:64 * (b + 1)])).max(axis=1)
+        assert np.all((blk == 448) | (qs[:, b] == 1.0))
+    ref = torch.from_numpy(c[:, :448] / np.repeat(qs, 64, axis=1)).clamp(-448, 448)
+    ref = ref.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ref, qc)
+
+
+def test_layer_compress_tiny_uniform_gate_equals_mean():
+    wl = W.get("tiny")
+    L = W.make_csa_layer(wl)
+    L["gate_w"] = torch.zeros_like(L["gate_w"])
+    L["gate_b"] = torch.zeros_like(L["gate_b"])
+    res = O.layer_compress(L, [wl.T - 12], [wl.T])[0]
+    ring = L["ring_k"]["data"][0].double().numpy()
+    for j, row in zip(res["j"], res["k"]):
+        pos = O.pool_positions(int(j), 8, 4)
+        assert np.allclose(row, ring[pos % ring.shape[0]].mean(axis=0), rtol=1e-13, atol=1e-13)

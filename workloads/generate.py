@@ -1,0 +1,232 @@
+"""Seeded synthetic layer inputs.
+
+Recipe (all draws from one `torch.Generator` seeded per layer):
+  * FP8 planes (raw tokens, compressed entries, indexer keys, indexer queries):
+    x ~ N(0,1) per element, per-64-element block scale s ~ U[0.5, 2], stored
+    code = E4M3(clamp(x / s, +-448)), stored scale = s.  The dequantised input
+    is therefore E4M3(code) * s.
+  * BF16 RoPE dims: N(0,1) rounded to BF16.   fp32 planes: N(0,1).
+  * q: N(0,1) as BF16 (fp32 and pre-scaled by 1/sqrt(D) for the tiny workload).
+  * indexer head weights: N(0,1)/sqrt(H_I).   gate w, b: N(0, 0.1^2).
+  * needles: at a needle position p the CSA entry p // stride gets, as its
+    indexer key, the query's indexer head with the largest weight scaled by 4,
+    and as its KV entry the first head's query (E4M3-encoded); the HCA entry
+    p // 128 gets the same KV needle.
+  * ring slots that hold no live position carry NaN scales / NaN values, so a
+    kernel that reads one produces NaN.
+
+Nothing here pools, scores, selects or attends: this module only produces
+inputs.  Tensors are created on `device` from a generator on that device.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from .configs import Workload
+
+_E4M3_MAX = 448.0
+
+
+def e4m3_from_float(x: torch.Tensor) -> torch.Tensor:
+    """Encode fp32 values as E4M3 codes (uint8) with torch's cast, clamped first
+    because torch maps out-of-range values to NaN."""
+    return x.clamp(-_E4M3_MAX, _E4M3_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def _n_slots(t: int, stride: int) -> int:
+    # number of compressed entries a cache must hold for t tokens
+    return t // stride
+
+
+class _Rng:
+    def __init__(self, seed: int, device):
+        self.device = torch.device(device)
+        self.g = torch.Generator(device=self.device)
+        self.g.manual_seed(seed)
+
+    def normal(self, *shape, std=1.0):
+        return torch.randn(*shape, generator=self.g, device=self.device, dtype=torch.float32) * std
+
+    def uniform(self, lo, hi, *shape):
+        return lo + (hi - lo) * torch.rand(*shape, generator=self.g, device=self.device,
+                                           dtype=torch.float32)
+
+    def integers(self, lo, hi, *shape):
+        return torch.randint(lo, hi, shape, generator=self.g, device=self.device)
+
+
+def _scale_cols(d_nope: int, pad: int) -> int:
+    nb = (d_nope + 63) // 64
+    return ((nb + pad - 1) // pad) * pad
+
+
+def _fp8_planes(rng: _Rng, lead, d_nope: int, scale_pad: int):
+    """codes uint8 [*lead, d_nope], scales f32 [*lead, cols] (pad columns NaN)."""
+    nb = (d_nope + 63) // 64
+    x = rng.normal(*lead, d_nope)
+    s = rng.uniform(0.5, 2.0, *lead, nb)
+    s_el = s.repeat_interleave(64, dim=-1)[..., :d_nope]
+    codes = e4m3_from_float(x / s_el)
+    cols = _scale_cols(d_nope, scale_pad)
+    scale = torch.full((*lead, cols), float("nan"), device=rng.device, dtype=torch.float32)
+    scale[..., :nb] = s
+    return codes, scale
+
+
+def _cache(rng: _Rng, wl: Workload, B: int, n: int, *, d_nope: int, d_rope: int,
+           fmt: str, scale_pad: int, ring: bool):
+    """A cache of n slots per sequence in the workload's storage format."""
+    c = {"fmt": fmt, "d_nope": d_nope, "d_rope": d_rope, "ring": ring, "cap": n}
+    if fmt == "f32":
+        c["data"] = rng.normal(B, n, d_nope + d_rope)
+    else:
+        c["data"], c["scale"] = _fp8_planes(rng, (B, n), d_nope, scale_pad)
+        if d_rope:
+            c["rope"] = rng.normal(B, n, d_rope).to(torch.bfloat16)
+    return c
+
+
+def _poison_ring(c: dict, t_end: int):
+    """Mark slots that hold no live position (pos < 0) with NaN."""
+    cap = c["cap"]
+    live = min(cap, t_end)
+    if live == cap:
+        return
+    dead = torch.arange(live, cap)  # slots p % cap for p in [t_end-cap, 0) map here when t_end < cap
+    if c["fmt"] == "f32":
+        c["data"][:, dead] = float("nan")
+    else:
+        c["scale"][:, dead] = float("nan")
+        if "rope" in c:
+            c["rope"][:, dead] = float("nan")
+
+
+def _needle_positions(rng: _Rng, wl: Workload, t: int):
+    if wl.needles == 0 or wl.prefill:
+        return torch.zeros(wl.B, 0, dtype=torch.int64)
+    if wl.needle_mode == "loguniform":
+        u = rng.uniform(0.0, math.log(t), wl.B, wl.needles)
+        d = torch.floor(torch.exp(u)).to(torch.int64).clamp_(0, t - 1)
+        return (t - 1 - d).cpu()
+    return rng.integers(0, t, wl.B, wl.needles).cpu()
+
+
+def _queries(rng: _Rng, wl: Workload):
+    B, Tq = wl.B, wl.Tq
+    if wl.fmt == "f32":
+        q = rng.normal(B, Tq, wl.Hq, wl.D)
+        if wl.q_prescale:
+            q = q * (1.0 / math.sqrt(wl.D))
+        return q
+    return rng.normal(B, Tq, wl.Hq, wl.D).to(torch.bfloat16)
+
+
+def _positions(wl: Workload, device):
+    """q_pos [B][Tq] int64 and ctx_len [B] int64 (tokens incl. the last query)."""
+    if wl.prefill:
+        pos = torch.arange(wl.T, wl.T + wl.Tq, device=device, dtype=torch.int64)
+        pos = pos.unsqueeze(0).expand(wl.B, wl.Tq).contiguous()
+    else:
+        pos = torch.full((wl.B, 1), wl.T - 1, device=device, dtype=torch.int64)
+    return pos, pos[:, -1] + 1
+
+
+def _plant_kv_needle(cache: dict, b: int, j: int, q_head0: torch.Tensor, rng: _Rng):
+    d_nope = cache["d_nope"]
+    if cache["fmt"] == "f32":
+        cache["data"][b, j, :d_nope] = q_head0[:d_nope].float()
+        return
+    v = q_head0[:d_nope].float() * 0.5
+    s = cache["scale"][b, j, : (d_nope + 63) // 64]
+    cache["data"][b, j] = e4m3_from_float(v / s.repeat_interleave(64)[:d_nope])
+
+
+def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap: int | None = None):
+    """Inputs of one CSA layer: raw KV / indexer-key rings, the compressed CSA
+    cache and indexer-key cache, queries, indexer queries and weights, gates."""
+    rng = _Rng(wl.seed * 7919 + 11 if seed is None else seed, device)
+    t_end = wl.t_end
+    n_c = _n_slots(t_end, wl.csa_stride)
+    cap = ring_cap or _default_ring(wl, wl.csa_pool, wl.csa_stride)
+    L = {"kind": "csa", "wl": wl, "t_end": t_end}
+    kw = dict(d_nope=wl.d_nope, d_rope=wl.d_rope, fmt=wl.fmt, scale_pad=8)
+    L["ring_k"] = _cache(rng, wl, wl.B, cap, ring=True, **kw)
+    L["ring_v"] = _cache(rng, wl, wl.B, cap, ring=True, **kw) if wl.separate_v else None
+    ik_kw = dict(d_nope=wl.d_I, d_rope=0, fmt=wl.fmt, scale_pad=2)
+    L["ring_ik"] = _cache(rng, wl, wl.B, cap, ring=True, **ik_kw)
+    for key in ("ring_k", "ring_v", "ring_ik"):
+        if L[key] is not None:
+            _poison_ring(L[key], t_end)
+    L["comp_k"] = _cache(rng, wl, wl.B, max(n_c, 1), ring=False, **kw)
+    L["comp_v"] = _cache(rng, wl, wl.B, max(n_c, 1), ring=False, **kw) if wl.separate_v else None
+    L["comp_ik"] = _cache(rng, wl, wl.B, max(n_c, 1), ring=False, **ik_kw)
+    L["n_comp"] = n_c
+    L["q"] = _queries(rng, wl)
+    if wl.fmt == "f32":
+        L["q_ik"] = rng.normal(wl.B, wl.Tq, wl.H_I, wl.d_I)
+        L["q_ik_scale"] = None
+    else:
+        L["q_ik"], L["q_ik_scale"] = _fp8_planes(rng, (wl.B, wl.Tq, wl.H_I), wl.d_I, 1)
+    L["head_w"] = rng.normal(wl.B, wl.Tq, wl.H_I) / math.sqrt(wl.H_I)
+    L["gate_w"] = rng.normal(wl.D, std=0.1)
+    L["gate_b"] = rng.normal(wl.csa_pool, std=0.1)
+    L["pool"], L["stride"] = wl.csa_pool, wl.csa_stride
+    L["q_pos"], L["ctx_len"] = _positions(wl, device)
+    L["needles"] = _needle_positions(rng, wl, t_end)
+    for b in range(wl.B):
+        hstar = int(torch.argmax(L["head_w"][b, 0]).item())
+        for p in L["needles"][b].tolist():
+            j = p // wl.csa_stride
+            if j >= n_c:
+                continue
+            if wl.fmt == "f32":
+                L["comp_ik"]["data"][b, j] = L["q_ik"][b, 0, hstar] * 4.0
+            else:
+                L["comp_ik"]["data"][b, j] = L["q_ik"][b, 0, hstar]
+                L["comp_ik"]["scale"][b, j, :] = L["q_ik_scale"][b, 0, hstar, :2] * 4.0
+            _plant_kv_needle(L["comp_k"], b, j, L["q"][b, 0, 0], rng)
+    return L
+
+
+def make_hca_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap: int | None = None):
+    """Inputs of one HCA layer: raw KV ring, the compressed HCA cache, queries, gates."""
+    rng = _Rng(wl.seed * 7919 + 23 if seed is None else seed, device)
+    t_end = wl.t_end
+    n_h = _n_slots(t_end, wl.hca_stride)
+    cap = ring_cap or _default_ring(wl, wl.hca_pool, wl.hca_stride)
+    L = {"kind": "hca", "wl": wl, "t_end": t_end}
+    kw = dict(d_nope=wl.d_nope, d_rope=wl.d_rope, fmt=wl.fmt, scale_pad=8)
+    L["ring_k"] = _cache(rng, wl, wl.B, cap, ring=True, **kw)
+    L["ring_v"] = _cache(rng, wl, wl.B, cap, ring=True, **kw) if wl.separate_v else None
+    for key in ("ring_k", "ring_v"):
+        if L[key] is not None:
+            _poison_ring(L[key], t_end)
+    L["comp_k"] = _cache(rng, wl, wl.B, max(n_h, 1), ring=False, **kw)
+    L["comp_v"] = _cache(rng, wl, wl.B, max(n_h, 1), ring=False, **kw) if wl.separate_v else None
+    L["n_comp"] = n_h
+    L["q"] = _queries(rng, wl)
+    L["gate_w"] = rng.normal(wl.D, std=0.1)
+    L["gate_b"] = rng.normal(wl.hca_pool, std=0.1)
+    L["pool"], L["stride"] = wl.hca_pool, wl.hca_stride
+    L["q_pos"], L["ctx_len"] = _positions(wl, device)
+    L["needles"] = _needle_positions(rng, wl, t_end)
+    for b in range(wl.B):
+        for p in L["needles"][b].tolist():
+            j = p // wl.hca_stride
+            if j < n_h:
+                _plant_kv_needle(L["comp_k"], b, j, L["q"][b, 0, 0], rng)
+    return L
+
+
+def _default_ring(wl: Workload, pool: int, stride: int) -> int:
+    """Smallest power of two holding the window and, for a prefill chunk, every
+    position the chunk's queries and pooling windows can reach."""
+    need = max(wl.window, pool)
+    if wl.prefill:
+        need = wl.Tq + max(wl.window, pool)
+    cap = 1
+    while cap < need:
+        cap *= 2
+    return cap
