@@ -1,0 +1,515 @@
+#!/usr/bin/env python3
+"""Benchmark: CSA+HCA hybrid-attention decode at a 1,048,576-token context.
+
+One step is one decode token through one CSA layer and one HCA layer of every
+sequence, at a position where both compressors fire (T = 2^20 is a multiple of
+4 and of 128):
+  CSA layer: csa_compress (new entry) -> indexer_topk (score 262,144 entries,
+             keep 1,024) -> hybrid_attn_decode (1,024 selected + 128 window)
+  HCA layer: hca_compress (new entry) -> hybrid_attn_decode (8,192 dense + 128)
+The metric is decode queries/s (one query = one token through both layers).
+
+Inputs are seeded synthetic tensors resident in HBM.  R replicas of every
+layer's inputs rotate between steps; their per-step bytes total more than 4x
+the 126 MB L2, so each step reads HBM.  The timed region replays a CUDA graph
+of G steps ceil(K/G) times (exactly K steps).  The dominant call
+(indexer_topk) is bracketed by event records inside the graph.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own sequences (weak scaling, no data-path
+collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "CSA+HCA decode queries/s at 1M ctx; achieved HBM GB/s vs B200 peak"
+UNIT = "queries/s"
+
+
+# ------------------------------------------------------------------ helpers
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the GPU is loaded."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1])); mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our path
+
+class Replica:
+    """One sequence batch's CSA and HCA layer inputs on the device."""
+
+    def __init__(self, wl, seed, dev):
+        from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
+        self.csa_L = W.make_csa_layer(wl, device=dev, seed=seed)
+        self.hca_L = W.make_hca_layer(wl, device=dev, seed=seed + 500_000)
+        self.csa = CSALayer(self.csa_L)
+        self.hca = HCALayer(self.hca_L)
+        T = wl.T
+        self.t_begin = torch.full((wl.B,), T - 1, dtype=torch.int64, device=dev)
+        self.t_end = torch.full((wl.B,), T, dtype=torch.int64, device=dev)
+
+    def step(self, mark=None):
+        """Enqueue one decode step on the current stream; mark(i) records an
+        event between calls (i = 0 before indexer_topk, 1 after)."""
+        self.csa.compress(self.t_begin, self.t_end, 1)
+        if mark:
+            mark(0)
+        self.csa.select()
+        if mark:
+            mark(1)
+        self.csa.attend()
+        self.hca.compress(self.t_begin, self.t_end, 1)
+        self.hca.attend()
+
+
+def _rt():
+    from cuda.bindings import runtime as rt
+    return rt
+
+
+def _ok(res, what):
+    err = res[0] if isinstance(res, tuple) else res
+    if int(err) != 0:
+        raise RuntimeError(f"{what}: {err}")
+    return res[1] if isinstance(res, tuple) and len(res) == 2 else res
+
+
+class StepGraph:
+    """CUDA graph of G consecutive steps over rotating replicas, with external
+    event records around every indexer_topk call."""
+
+    def __init__(self, replicas, G, stream, r0=0):
+        rt = _rt()
+        self.G = G
+        self.events = [[_ok(rt.cudaEventCreate(), "event") for _ in range(2)] for _ in range(G)]
+        sh = rt.cudaStream_t(stream.cuda_stream)
+        with torch.cuda.stream(stream):
+            _ok(rt.cudaStreamBeginCapture(
+                sh, rt.cudaStreamCaptureMode.cudaStreamCaptureModeThreadLocal), "capture")
+            for i in range(G):
+                rep = replicas[(r0 + i) % len(replicas)]
+                ev = self.events[i]
+                rep.step(mark=lambda m, ev=ev: _ok(rt.cudaEventRecordWithFlags(
+                    ev[m], sh, rt.cudaEventRecordExternal), "record"))
+            self.graph = _ok(rt.cudaStreamEndCapture(sh), "end capture")
+        self.exec = _ok(rt.cudaGraphInstantiate(self.graph, 0), "instantiate")
+        self.kernels = self._count_kernels()
+        self.sh = sh
+
+    def _count_kernels(self):
+        rt = _rt()
+        res = rt.cudaGraphGetNodes(self.graph)
+        n = res[-1]
+        res = rt.cudaGraphGetNodes(self.graph, n)
+        nodes = res[1]
+        kern = 0
+        for nd in nodes:
+            t = _ok(rt.cudaGraphNodeGetType(nd), "node type")
+            if t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kern += 1
+        return kern
+
+    def launch(self):
+        _ok(_rt().cudaGraphLaunch(self.exec, self.sh), "graph launch")
+
+    def indexer_ms(self):
+        rt = _rt()
+        return [_ok(rt.cudaEventElapsedTime(a, b), "elapsed") for a, b in self.events]
+
+
+def indexer_bytes(wl):
+    """Algorithmic bytes of one indexer_topk call: every visible CSA entry's
+    FP8 indexer key (d_I bytes) and its d_I/64 fp32 scales, the FP8 query
+    heads with scales, head weights, and the selected indices written."""
+    n_c = wl.T // wl.csa_stride
+    per_entry = wl.d_I + 4 * (wl.d_I // 64)
+    q = wl.H_I * wl.d_I + 4 * wl.H_I * (wl.d_I // 64) + 4 * wl.H_I
+    return wl.B * (n_c * per_entry + q + 4 * wl.k)
+
+
+def step_bytes(wl):
+    """Algorithmic HBM bytes of one full decode step (both layers)."""
+    entry = wl.d_nope + 2 * wl.d_rope + 4 * (wl.d_nope // 64)
+    n_h = wl.T // wl.hca_stride
+    q = wl.Hq * wl.D * 2
+    out = wl.Hq * wl.D * 4 + wl.Hq * 4
+    csa = indexer_bytes(wl) + wl.B * ((wl.k + wl.window) * entry + q + out)
+    hca = wl.B * ((n_h + wl.window) * entry + q + out)
+    compress = wl.B * ((wl.csa_pool + wl.hca_pool) * entry + 2 * entry
+                       + wl.csa_pool * (wl.d_I + 8) + (wl.d_I + 8))
+    return csa + hca + compress
+
+
+def run_ours(args, rank, world, dev):
+    import compressed_sparse_kv_softmax_b200 as C  # noqa: F401  (fails loudly without the .so)
+    wl = W.get(args.workload)
+    torch.cuda.set_device(dev)
+    per_rep_bytes = step_bytes(wl)
+    R = max(args.replicas, math.ceil(4 * 126e6 / per_rep_bytes) + 1)
+    replicas = [Replica(wl, 1000 + r + 7919 * rank, dev) for r in range(R)]
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    # warm-up: W steps eagerly through the public API (also performs the
+    # library's one-time kernel attribute set-up outside any graph capture)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            replicas[i % R].step()
+    stream.synchronize()
+    G = max(1, min(args.graph_steps, args.steps))
+    graph = StepGraph(replicas, G, stream)
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    time.sleep(0.3)
+    # untimed graph replays so the clock sampler sees the GPU under load
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, int(0.2 / max(1e-6, 30e-6 * G)))):
+            graph.launch()
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    n_launch = math.ceil(args.steps / G)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(n_launch):
+            graph.launch()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    steps_done = n_launch * G
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    idx_ms = float(np.mean(graph.indexer_ms()))
+    total_q = wl.B * steps_done * world
+    value = total_q / (ms / 1e3)
+
+    peak, peak_kind = _peaks()
+    ib = indexer_bytes(wl)
+    achieved = ib / (idx_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "indexer_topk (lightning-indexer scoring + top-k)",
+                "peak_kind": f"{peak_kind} HBM copy bandwidth (burst)",
+                "algorithmic_bytes_per_launch": ib, "avg_launch_us": round(idx_ms * 1e3, 3)}
+    traffic = _profile_traffic(args.workload)
+    if traffic is not None:
+        roofline["traffic"] = traffic
+
+    res = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+           "steps": steps_done, "warmup": args.warmup, "ms_per_step": ms / steps_done,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3/bf16 storage, fp32 math",
+           "data": "synthetic (seeded Gaussian FP8 E4M3 + BF16 caches with needles)",
+           "config": {"workload": f"{wl.name}: 1 CSA + 1 HCA layer decode, B={wl.B}/GPU, "
+                                  f"ctx={wl.T}, Hq={wl.Hq}, D={wl.d_nope}+{wl.d_rope}, "
+                                  f"H_I={wl.H_I}x{wl.d_I}, k={wl.k}, window={wl.window}",
+                      "global_batch": wl.B * world, "seq_len": wl.T,
+                      "parallelism": f"replicas x{world} (weak)",
+                      "l2": f"{R} rotating input replicas, {R * per_rep_bytes / 1e6:.0f} MB "
+                            f"touched per cycle (> 4x L2)",
+                      "step_bytes": per_rep_bytes},
+           "roofline": roofline,
+           "gpu_launches": graph.kernels * n_launch,
+           "clocks": clocks}
+    return res, replicas, wl
+
+
+def _profile_traffic(workload):
+    """DRAM bytes per indexer launch from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+    if os.path.exists(p):
+        try:
+            return json.load(open(p)).get("indexer_dram_bytes_per_launch")
+        except (ValueError, OSError):
+            return None
+    return None
+
+
+def run_e2e(args, replicas, wl, dev, world):
+    """Same metric through the public API with per-step host<->device copies:
+    the new token's raw KV and indexer key, q, the indexer query, head weights
+    and positions go in from pinned host memory; out and lse come back."""
+    K = max(3, min(args.steps, args.e2e_steps))
+    rep = replicas[0]
+    cl, hl = rep.csa_L, rep.hca_L
+    ins = []
+    slot = (wl.T - 1) % cl["ring_k"]["cap"]
+    for Ld in (cl, hl):
+        for key in ("data", "scale", "rope"):
+            ins.append(Ld["ring_k"][key][:, slot])
+        ins.append(Ld["q"])
+    ins += [cl["ring_ik"]["data"][:, slot], cl["ring_ik"]["scale"][:, slot], cl["q_ik"],
+            cl["q_ik_scale"], cl["head_w"], cl["q_pos"], cl["ctx_len"], hl["ctx_len"],
+            rep.t_begin, rep.t_end]
+    host_in = [t.detach().cpu().pin_memory() for t in ins]
+    outs = [rep.csa.out, rep.csa.lse, rep.hca.out, rep.hca.lse]
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    bi = sum(t.numel() * t.element_size() for t in host_in)
+    bo = sum(t.numel() * t.element_size() for t in host_out)
+    stream = torch.cuda.Stream(device=dev)
+
+    def one():
+        for d, h in zip(ins, host_in):
+            d.copy_(h, non_blocking=True)
+        rep.step()
+        for h, d in zip(host_out, outs):
+            h.copy_(d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(K):
+            one()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(wl.B * K * world / (ms / 1e3), 2), "unit": UNIT,
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": K,
+            "path": "eager public API calls (no graph), single replica"}
+
+
+# ------------------------------------------------------------- the oracle
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _cpu_layer(L):
+    out = {}
+    for k, v in L.items():
+        if isinstance(v, torch.Tensor):
+            out[k] = v.detach().cpu()
+        elif isinstance(v, dict):
+            out[k] = {kk: (vv.detach().cpu() if isinstance(vv, torch.Tensor) else vv)
+                      for kk, vv in v.items()}
+        else:
+            out[k] = v
+    return out
+
+
+def oracle_query(Lc, Lh, frac=1.0):
+    """One decode query through the oracle: CSA indexer + top-k + sparse
+    attention, HCA dense attention.  frac < 1 runs the same steps over the
+    first frac of the compressed entries (a bounded sample of the query)."""
+    import oracle as O
+    from oracle.layer import as_numpy_cache, _q, _q_ik
+    wl = Lc["wl"]
+    res = []
+    for b in range(wl.B):
+        pos = int(Lc["q_pos"][b, 0])
+        n_c = max(1, int(O.n_entries(pos + 1, wl.csa_stride) * frac))
+        ik = as_numpy_cache(Lc["comp_ik"])
+        s = O.indexer_scores(_q_ik(Lc, b, 0), Lc["head_w"][b, 0].double().numpy(),
+                             O.dequant_slots(ik, b, np.arange(n_c)))
+        k = max(1, int(round(wl.k * frac)))
+        idx = O.topk(s, n_c, k)
+        ck = as_numpy_cache(Lc["comp_k"])
+        sel = idx[idx >= 0]
+        rk = as_numpy_cache(Lc["ring_k"])
+        wlen = max(1, int(round(wl.window * frac)))
+        wpos = O.window_positions(pos, wlen)
+        win = O.dequant_slots(rk, b, O.ring_slots(wpos, rk["cap"]))
+        comp = O.dequant_slots(ck, b, sel)
+        res.append(O.hybrid_attention(_q(Lc, b, 0), comp, comp, win, win, wl.sm_scale))
+        n_h = max(1, int(O.n_entries(pos + 1, wl.hca_stride) * frac))
+        hk = as_numpy_cache(Lh["comp_k"])
+        hr = as_numpy_cache(Lh["ring_k"])
+        comp = O.dequant_slots(hk, b, np.arange(n_h))
+        win = O.dequant_slots(hr, b, O.ring_slots(wpos, hr["cap"]))
+        res.append(O.hybrid_attention(_q(Lh, b, 0), comp, comp, win, win, wl.sm_scale))
+    return res
+
+
+def cpu_baseline(Lc, Lh, budget_s=12.0):
+    """The oracle as it stands on the host cores, whole queries until the
+    budget is spent (at least one)."""
+    Lc, Lh = _cpu_layer(Lc), _cpu_layer(Lh)
+    wl = Lc["wl"]
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_query(Lc, Lh)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(wl.B * n / dt, 4), "unit": UNIT, "cores": _threads(),
+            "kind": "oracle",
+            "sample": f"{n} whole decode queries (B={wl.B}) of the same workload, "
+                      f"numpy float64, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step is one decode query over a
+    bounded sample (the first `frac` of the compressed entries), sized so the
+    whole run ends within a few minutes."""
+    if rank != 0:
+        return None
+    wl = W.get(args.workload)
+    Lc = _cpu_layer(W.make_csa_layer(wl, seed=1000))
+    Lh = _cpu_layer(W.make_hca_layer(wl, seed=501_000))
+    t = time.perf_counter()
+    oracle_query(Lc, Lh, frac=1 / 64)
+    t_small = max(1e-4, time.perf_counter() - t) * 64    # rough cost of one whole query
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    frac = min(1.0, max(1 / 4096, budget / t_small))
+    for _ in range(args.warmup):
+        oracle_query(Lc, Lh, frac)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_query(Lc, Lh, frac)
+    dt = time.perf_counter() - t0
+    value = wl.B * frac * args.steps / dt
+    cores = _threads()
+    return {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{wl.name}: 1 CSA + 1 HCA layer decode, B={wl.B}, ctx={wl.T}"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"each step: one decode query over the first "
+                                       f"{frac:.5f} of the compressed entries; value scaled "
+                                       f"by that fraction"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="long")
+    ap.add_argument("--replicas", type=int, default=4)
+    ap.add_argument("--graph-steps", type=int, default=250)
+    ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    res, replicas, wl = run_ours(args, rank, world, dev)
+    res["e2e"] = run_e2e(args, replicas, wl, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(replicas[0].csa_L, replicas[0].hca_L, args.cpu_budget)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

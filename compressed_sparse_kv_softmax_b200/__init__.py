@@ -1,0 +1,189 @@
+"""Python binding of libcskv.so (hybrid compressed sparse KV attention for B200).
+
+Argument marshalling only: torch tensors become device pointers and byte
+strides, the current torch CUDA stream becomes the launch stream, and every
+non-zero status raises `CskvError`.  All computation runs in the library's
+CUDA kernels; there is no CPU fallback.  Importing the package without a
+built libcskv.so raises ImportError.
+
+Cache planes follow the C descriptor (include/cskv.h): for B sequences of
+`cap` slots, `data` is [B, cap, ...] with one slot per row; E4M3_BF16 caches
+add `scale` [B, cap, >= d_nope/64] fp32 and `rope` [B, cap, d_rope] bf16.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcskv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m compressed_sparse_kv_softmax_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, -1, -2, -3, -4
+FMT_F32, FMT_E4M3_BF16 = 0, 1
+
+
+class CskvCache(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("d_nope", ctypes.c_int32), ("d_rope", ctypes.c_int32),
+                ("ring", ctypes.c_int32), ("cap", ctypes.c_int64),
+                ("data", ctypes.c_void_p), ("data_stride", ctypes.c_int64),
+                ("scale", ctypes.c_void_p), ("scale_stride", ctypes.c_int64),
+                ("rope", ctypes.c_void_p), ("rope_stride", ctypes.c_int64)]
+
+
+_P = ctypes.c_void_p
+_PC = ctypes.POINTER(CskvCache)
+_I, _I64, _F, _SZ = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+_lib.csa_compress.argtypes = [_I, _P, _P, _I64, _PC, _PC, _PC, _P, _P, _I, _I, _PC, _PC, _PC, _P]
+_lib.hca_compress.argtypes = [_I, _P, _P, _I64, _PC, _PC, _P, _P, _I, _I, _PC, _PC, _P]
+_lib.indexer_topk.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC, _I, _I, _I64, _P, _P, _P,
+                              _SZ, _P]
+_lib.hybrid_attn_decode.argtypes = [_I, _P, _P, _I, _F, _PC, _PC, _I, _P, _I, _I64, _PC, _PC,
+                                    _I, _P, _P, _P, _SZ, _P]
+_lib.hybrid_attn_prefill.argtypes = [_I, _I, _P, _P, _I, _F, _PC, _PC, _I, _P, _I, _I64, _PC,
+                                     _PC, _I, _P, _P, _P, _SZ, _P]
+_lib.cskv_indexer_workspace_size.argtypes = [_I, _I, _I64, _I]
+_lib.cskv_indexer_workspace_size.restype = _SZ
+_lib.cskv_attn_workspace_size.argtypes = [_I, _I, _I, _I, _I64, _I]
+_lib.cskv_attn_workspace_size.restype = _SZ
+_lib.cskv_error_string.argtypes = [_I]
+_lib.cskv_error_string.restype = ctypes.c_char_p
+_lib.cskv_version.restype = _I
+for _name in ("csa_compress", "hca_compress", "indexer_topk", "hybrid_attn_decode",
+              "hybrid_attn_prefill"):
+    getattr(_lib, _name).restype = _I
+
+
+class CskvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.cskv_error_string(status).decode()} (status {status})")
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise CskvError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _slot_bytes(t):
+    # bytes between consecutive slots of a [B, cap, ...] plane
+    return t.stride(1) * t.element_size()
+
+
+def cache_struct(c):
+    """C descriptor for a cache given as a dict of planes
+    {"fmt": "f32"|"e4m3", "d_nope", "d_rope", "ring", "cap", "data", "scale", "rope"}
+    (or None)."""
+    if c is None:
+        return None
+    s = CskvCache()
+    s.fmt = FMT_F32 if c["fmt"] == "f32" else FMT_E4M3_BF16
+    s.d_nope, s.d_rope = int(c["d_nope"]), int(c["d_rope"])
+    s.ring, s.cap = int(bool(c["ring"])), int(c["cap"])
+    s.data, s.data_stride = c["data"].data_ptr(), _slot_bytes(c["data"])
+    sc, rp = c.get("scale"), c.get("rope")
+    if sc is not None:
+        s.scale, s.scale_stride = sc.data_ptr(), _slot_bytes(sc)
+    if rp is not None:
+        s.rope, s.rope_stride = rp.data_ptr(), _slot_bytes(rp)
+    return s
+
+
+def _ref(s):
+    return None if s is None else ctypes.byref(s)
+
+
+def _stream(stream):
+    if stream is not None:
+        return ctypes.c_void_p(stream)
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def indexer_workspace_size(B, Tq, max_entries, k) -> int:
+    return int(_lib.cskv_indexer_workspace_size(B, Tq, max_entries, k))
+
+
+def attn_workspace_size(B, Tq, Hq, Dv, max_entries, window) -> int:
+    return int(_lib.cskv_attn_workspace_size(B, Tq, Hq, Dv, max_entries, window))
+
+
+def workspace(nbytes: int, device="cuda"):
+    """A 256-byte-aligned uint8 device buffer of at least nbytes."""
+    import torch
+    return torch.empty(max(int(nbytes), 1) + 256, dtype=torch.uint8, device=device)
+
+
+def _ws(ws):
+    # returns (aligned pointer, usable bytes)
+    p = ws.data_ptr()
+    ap = (p + 255) & ~255
+    return ctypes.c_void_p(ap), ws.numel() - (ap - p)
+
+
+def csa_compress(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride,
+                 out_k, out_v, out_ik, stream=None):
+    cs = [cache_struct(c) for c in (raw_k, raw_v, raw_ik, out_k, out_v, out_ik)]
+    _check(_lib.csa_compress(B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]),
+                             _ref(cs[1]), _ref(cs[2]), _ptr(gate_w), _ptr(gate_b), pool, stride,
+                             _ref(cs[3]), _ref(cs[4]), _ref(cs[5]), _stream(stream)),
+           "csa_compress")
+
+
+def hca_compress(B, t_begin, t_end, max_new, raw_k, raw_v, gate_w, gate_b, pool, stride,
+                 out_k, out_v, stream=None):
+    cs = [cache_struct(c) for c in (raw_k, raw_v, out_k, out_v)]
+    _check(_lib.hca_compress(B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]),
+                             _ref(cs[1]), _ptr(gate_w), _ptr(gate_b), pool, stride, _ref(cs[2]),
+                             _ref(cs[3]), _stream(stream)), "hca_compress")
+
+
+def indexer_topk(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
+                 out_idx, out_score, ws, stream=None):
+    c = cache_struct(ik)
+    wp, wn = _ws(ws)
+    _check(_lib.indexer_topk(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
+                             H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
+                             _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
+           "indexer_topk")
+
+
+def hybrid_attn_decode(B, ctx_len, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
+                       max_entries, win_k, win_v, window, out, lse, ws, stream=None):
+    cs = [cache_struct(c) for c in (comp_k, comp_v, win_k, win_v)]
+    wp, wn = _ws(ws)
+    _check(_lib.hybrid_attn_decode(B, _ptr(ctx_len), _ptr(q), Hq, sm_scale, _ref(cs[0]),
+                                   _ref(cs[1]), comp_stride, _ptr(sel), k, int(max_entries),
+                                   _ref(cs[2]), _ref(cs[3]), window, _ptr(out), _ptr(lse), wp,
+                                   wn, _stream(stream)), "hybrid_attn_decode")
+
+
+def hybrid_attn_prefill(B, Tq, q_pos, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
+                        max_entries, win_k, win_v, window, out, lse, ws, stream=None):
+    cs = [cache_struct(c) for c in (comp_k, comp_v, win_k, win_v)]
+    wp, wn = _ws(ws)
+    _check(_lib.hybrid_attn_prefill(B, Tq, _ptr(q_pos), _ptr(q), Hq, sm_scale, _ref(cs[0]),
+                                    _ref(cs[1]), comp_stride, _ptr(sel), k, int(max_entries),
+                                    _ref(cs[2]), _ref(cs[3]), window, _ptr(out), _ptr(lse), wp,
+                                    wn, _stream(stream)), "hybrid_attn_prefill")
+
+
+def error_string(status: int) -> str:
+    return _lib.cskv_error_string(status).decode()
+
+
+def version() -> int:
+    return int(_lib.cskv_version())
+
+
+lib = _lib

@@ -1,0 +1,126 @@
+// Internal device/host helpers shared by the kernels of libcskv.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cskv.h"
+
+namespace cskv {
+
+// Device-side view of a cskv_cache (passed to kernels by value).
+struct Cache {
+  int fmt, d_nope, d_rope, ring;
+  long long cap;
+  uint8_t *data; long long data_stride;
+  uint8_t *scale; long long scale_stride;   // bytes
+  uint8_t *rope; long long rope_stride;
+
+  __host__ __device__ int dims() const { return d_nope + d_rope; }
+  __host__ __device__ long long row(int b, long long slot) const {
+    return (long long)b * cap + slot;
+  }
+  // slot holding token position p (ring) or entry j (compressed cache)
+  __host__ __device__ long long slot_of(long long p) const { return ring ? (p % cap) : p; }
+  __device__ const uint8_t *data_ptr(int b, long long slot) const {
+    return data + row(b, slot) * data_stride;
+  }
+  __device__ const float *scale_ptr(int b, long long slot) const {
+    return reinterpret_cast<const float *>(scale + row(b, slot) * scale_stride);
+  }
+  __device__ const __nv_bfloat16 *rope_ptr(int b, long long slot) const {
+    return reinterpret_cast<const __nv_bfloat16 *>(rope + row(b, slot) * rope_stride);
+  }
+  // dequantised value of dim d of a slot (scalar path)
+  __device__ float value(int b, long long slot, int d) const {
+    if (fmt == CSKV_FMT_F32)
+      return reinterpret_cast<const float *>(data_ptr(b, slot))[d];
+    if (d < d_nope) {
+      __nv_fp8_e4m3 c;
+      c.__x = data_ptr(b, slot)[d];
+      return float(c) * scale_ptr(b, slot)[d >> 6];
+    }
+    return __bfloat162float(rope_ptr(b, slot)[d - d_nope]);
+  }
+};
+
+inline Cache to_dev(const cskv_cache *c) {
+  Cache v{};
+  if (!c) return v;
+  v.fmt = c->fmt; v.d_nope = c->d_nope; v.d_rope = c->d_rope; v.ring = c->ring;
+  v.cap = c->cap;
+  v.data = (uint8_t *)c->data; v.data_stride = c->data_stride;
+  v.scale = (uint8_t *)c->scale; v.scale_stride = c->scale_stride;
+  v.rope = (uint8_t *)c->rope; v.rope_stride = c->rope_stride;
+  return v;
+}
+
+// E4M3 encode: round to nearest even, saturate to +-448 (finite-only format).
+__device__ __forceinline__ uint8_t e4m3_encode(float x) {
+  return (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float e4m3_decode(uint8_t code) {
+  __nv_fp8_e4m3 c;
+  c.__x = code;
+  return float(c);
+}
+
+// Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// host-side launch helpers (defined in the kernel files)
+int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
+                    const Cache &raw_k, const Cache &raw_v, const Cache &raw_ik,
+                    const float *gate_w, const float *gate_b, int pool, int stride,
+                    const Cache &out_k, const Cache &out_v, const Cache &out_ik,
+                    cudaStream_t st);
+
+struct IndexerArgs {
+  int B, Tq, H_I, d_I, stride, k;
+  long long max_entries;
+  const int64_t *q_pos;
+  const void *q_ik; const float *q_ik_scale; const float *head_w;
+  Cache ik;
+  int32_t *out_idx; float *out_score;
+  void *ws; size_t ws_bytes;
+};
+size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k);
+int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st);
+
+struct AttnArgs {
+  int B, Tq, Hq, D, Dv;
+  float sm_scale;
+  const int64_t *pos;      // q_pos [B][Tq] or ctx_len [B] (decode)
+  int pos_is_ctx_len;      // 1: pos[b] = tokens incl. the query (decode)
+  const void *q;
+  Cache comp_k, comp_v;    // comp_k.data == nullptr -> window only
+  int has_comp, comp_stride;
+  const int32_t *sel; int k;
+  long long max_entries;
+  Cache win_k, win_v;
+  int window;
+  float *out, *lse;
+  void *ws; size_t ws_bytes;
+};
+size_t attn_ws_bytes(int B, int Tq, int Hq, int Dv, long long max_entries, int window);
+int launch_attention(const AttnArgs &a, cudaStream_t st);
+
+}  // namespace cskv

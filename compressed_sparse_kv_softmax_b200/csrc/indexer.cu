@@ -1,0 +1,109 @@
+// Lightning-indexer scoring (generic CUDA-core path) and the indexer_topk driver.
+//
+// The indexer scores every compressed CSA entry per query at low precision
+// («DeepSeek V4-Pro: Architektur, KV-Cache-Kompression und Hyper-Connections
+// im Detail», "Kompression und Selektion"; «DeepSeek-V4: 1 Million Token
+// Context endlich nutzbar», "Hybrid Attention: CSA und HCA").  Score of entry j
+// for one query row:  s_j = sum_h w[h] * max(0, q[h] . k[j])  with q and k
+// the dequantised FP8 (or fp32) vectors.
+//
+// This file holds the path for any (H_I, d_I) and both formats: one thread
+// per entry, the query's heads dequantised once per CTA into shared memory.
+// The 64-head x 128-dim FP8 layout at scale goes through the tensor-core
+// kernel in indexer_tc.cu.
+#include "cskv_internal.cuh"
+
+namespace cskv {
+
+void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,
+                      long long max_entries, int k, int rows, int32_t *out_idx,
+                      float *out_score, cudaStream_t st);
+bool indexer_tc_supported(const IndexerArgs &a);
+int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, cudaStream_t st);
+
+namespace {
+
+constexpr int kKeys = 128;   // entries per CTA (one per thread)
+
+__global__ void __launch_bounds__(kKeys)
+indexer_score_kernel(IndexerArgs a, float *__restrict__ scores, long long ld) {
+  extern __shared__ float sm[];
+  const int H = a.H_I, dI = a.d_I;
+  float *q = sm;                       // [H][dI]
+  float *w = q + H * dI;               // [H]
+  float *kt = w + H;                   // [kKeys][dI + 1]
+  const int row = blockIdx.y;
+  const int b = row / a.Tq;
+  long long n = (a.q_pos[row] + 1) / a.stride;
+  if (n > a.max_entries) n = a.max_entries;
+  const long long j0 = (long long)blockIdx.x * kKeys;
+  if (j0 >= n) return;
+  const int tid = threadIdx.x;
+  const long long qoff = (long long)row * H * dI;
+  for (int i = tid; i < H * dI; i += blockDim.x) {
+    if (a.ik.fmt == CSKV_FMT_F32) {
+      q[i] = reinterpret_cast<const float *>(a.q_ik)[qoff + i];
+    } else {
+      const int h = i / dI, d = i % dI;
+      const float sc = a.q_ik_scale[((long long)row * H + h) * (dI >> 6) + (d >> 6)];
+      q[i] = e4m3_decode(reinterpret_cast<const uint8_t *>(a.q_ik)[qoff + i]) * sc;
+    }
+  }
+  for (int h = tid; h < H; h += blockDim.x) w[h] = a.head_w[(long long)row * H + h];
+  // dequantise this CTA's keys (coalesced over dims)
+  for (int i = tid; i < kKeys * dI; i += blockDim.x) {
+    const int r = i / dI, d = i % dI;
+    const long long j = j0 + r;
+    kt[r * (dI + 1) + d] = j < n ? a.ik.value(b, j, d) : 0.f;
+  }
+  __syncthreads();
+  const long long j = j0 + tid;
+  if (j >= n) return;
+  const float *kr = kt + tid * (dI + 1);
+  float s = 0.f;
+  for (int h = 0; h < H; ++h) {
+    const float *qh = q + h * dI;
+    float dot = 0.f;
+    for (int d = 0; d < dI; ++d) dot = fmaf(qh[d], kr[d], dot);
+    s = fmaf(w[h], fmaxf(dot, 0.f), s);
+  }
+  scores[(long long)row * ld + j] = s;
+}
+
+}  // namespace
+
+size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k) {
+  (void)k;
+  const long long ld = (max_entries + 3) & ~3LL;
+  return (size_t)B * Tq * ld * sizeof(float) + 256;
+}
+
+int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
+  const int rows = a.B * a.Tq;
+  if (rows == 0) return CSKV_OK;
+  const long long ld = (a.max_entries + 3) & ~3LL;
+  float *scores = reinterpret_cast<float *>(a.ws);
+  if (a.max_entries > 0) {
+    if (indexer_tc_supported(a)) {
+      const int rc = launch_indexer_tc(a, scores, ld, st);
+      if (rc != CSKV_OK) return rc;
+    } else {
+      const size_t smem = sizeof(float) * ((size_t)a.H_I * a.d_I + a.H_I +
+                                           (size_t)kKeys * (a.d_I + 1));
+      static bool smem_set = false;   // one-time opt-in to the full shared memory
+      if (smem > 48 * 1024 && !smem_set) {
+        cudaFuncSetAttribute(indexer_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024);
+        smem_set = true;
+      }
+      dim3 grid((unsigned)((a.max_entries + kKeys - 1) / kKeys), (unsigned)rows);
+      indexer_score_kernel<<<grid, kKeys, smem, st>>>(a, scores, ld);
+      if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
+    }
+  }
+  launch_topk_rows(scores, ld, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
+                   a.out_score, st);
+  return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
+}
+
+}  // namespace cskv

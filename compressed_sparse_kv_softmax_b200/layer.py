@@ -1,0 +1,116 @@
+"""Per-layer drivers over device buffers (marshalling around the C ABI).
+
+A CSA layer step is: csa_compress of the newly arrived tokens, indexer_topk,
+hybrid attention over the selected entries plus the window.  An HCA layer step
+is: hca_compress, hybrid attention over every visible entry plus the window.
+A window-only layer (the first two layers of the model) is hybrid attention
+with no compressed cache.  Buffers are torch tensors on one CUDA device; the
+caches are dicts of planes as described in the package docstring.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (attn_workspace_size, csa_compress, hca_compress, hybrid_attn_decode,
+               hybrid_attn_prefill, indexer_topk, indexer_workspace_size, workspace)
+
+
+def _dims(c):
+    return int(c["d_nope"]) + int(c["d_rope"])
+
+
+class CSALayer:
+    """One CSA layer: raw rings, compressed caches, the indexer and attention.
+
+    L: dict with ring_k, ring_v (or None), ring_ik, comp_k, comp_v (or None),
+    comp_ik, q, q_ik, q_ik_scale, head_w, gate_w, gate_b, pool, stride, q_pos,
+    ctx_len and the shape fields of `wl` (B, Tq, Hq, H_I, d_I, k, window,
+    prefill, sm_scale)."""
+
+    def __init__(self, L, k=None, max_entries=None):
+        wl = L["wl"]
+        self.L, self.wl = L, wl
+        self.B, self.Tq, self.Hq = wl.B, wl.Tq, wl.Hq
+        self.k = int(k if k is not None else wl.k)
+        self.max_entries = int(max_entries if max_entries is not None else L["comp_ik"]["cap"])
+        dev = L["q"].device
+        self.Dv = _dims(L["comp_v"] or L["comp_k"])
+        self.idx = torch.empty(self.B, self.Tq, self.k, dtype=torch.int32, device=dev)
+        self.score = torch.empty(self.B, self.Tq, self.k, dtype=torch.float32, device=dev)
+        self.out = torch.empty(self.B, self.Tq, self.Hq, self.Dv, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(self.B, self.Tq, self.Hq, dtype=torch.float32, device=dev)
+        self.ws_idx = workspace(indexer_workspace_size(self.B, self.Tq, self.max_entries, self.k),
+                                dev)
+        self.ws_attn = workspace(attn_workspace_size(self.B, self.Tq, self.Hq, self.Dv, self.k,
+                                                     wl.window), dev)
+
+    def compress(self, t_begin, t_end, max_new):
+        L = self.L
+        csa_compress(self.B, t_begin, t_end, max_new, L["ring_k"], L["ring_v"], L["ring_ik"],
+                     L["gate_w"], L["gate_b"], L["pool"], L["stride"], L["comp_k"], L["comp_v"],
+                     L["comp_ik"])
+
+    def select(self):
+        L, wl = self.L, self.wl
+        indexer_topk(self.B, self.Tq, L["q_pos"], L["q_ik"], L["q_ik_scale"], L["head_w"],
+                     wl.H_I, wl.d_I, L["comp_ik"], L["stride"], self.k, self.max_entries,
+                     self.idx, self.score, self.ws_idx)
+        return self.idx
+
+    def attend(self, sel=None):
+        L, wl = self.L, self.wl
+        sel = self.idx if sel is None else sel
+        if wl.prefill:
+            hybrid_attn_prefill(self.B, self.Tq, L["q_pos"], L["q"], self.Hq, wl.sm_scale,
+                                L["comp_k"], L["comp_v"], L["stride"], sel, self.k, self.k,
+                                L["ring_k"], L["ring_v"], wl.window, self.out, self.lse,
+                                self.ws_attn)
+        else:
+            hybrid_attn_decode(self.B, L["ctx_len"], L["q"], self.Hq, wl.sm_scale, L["comp_k"],
+                               L["comp_v"], L["stride"], sel, self.k, self.k, L["ring_k"],
+                               L["ring_v"], wl.window, self.out, self.lse, self.ws_attn)
+        return self.out, self.lse
+
+    def step(self):
+        self.select()
+        return self.attend()
+
+
+class HCALayer:
+    """One HCA layer: raw ring, compressed cache, dense attention plus window.
+    With dense=False (no compressed cache) it is a window-only layer."""
+
+    def __init__(self, L, max_entries=None, dense=True):
+        wl = L["wl"]
+        self.L, self.wl, self.dense = L, wl, dense
+        self.B, self.Tq, self.Hq = wl.B, wl.Tq, wl.Hq
+        self.max_entries = int(max_entries if max_entries is not None else L["comp_k"]["cap"])
+        dev = L["q"].device
+        self.Dv = _dims(L["comp_v"] or L["comp_k"])
+        self.out = torch.empty(self.B, self.Tq, self.Hq, self.Dv, dtype=torch.float32, device=dev)
+        self.lse = torch.empty(self.B, self.Tq, self.Hq, dtype=torch.float32, device=dev)
+        self.ws_attn = workspace(attn_workspace_size(self.B, self.Tq, self.Hq, self.Dv,
+                                                     self.max_entries if dense else 0,
+                                                     wl.window), dev)
+
+    def compress(self, t_begin, t_end, max_new):
+        L = self.L
+        hca_compress(self.B, t_begin, t_end, max_new, L["ring_k"], L["ring_v"], L["gate_w"],
+                     L["gate_b"], L["pool"], L["stride"], L["comp_k"], L["comp_v"])
+
+    def attend(self):
+        L, wl = self.L, self.wl
+        ck = L["comp_k"] if self.dense else None
+        cv = L["comp_v"] if self.dense else None
+        me = self.max_entries if self.dense else 0
+        if wl.prefill:
+            hybrid_attn_prefill(self.B, self.Tq, L["q_pos"], L["q"], self.Hq, wl.sm_scale, ck, cv,
+                                L["stride"], None, 0, me, L["ring_k"], L["ring_v"], wl.window,
+                                self.out, self.lse, self.ws_attn)
+        else:
+            hybrid_attn_decode(self.B, L["ctx_len"], L["q"], self.Hq, wl.sm_scale, ck, cv,
+                               L["stride"], None, 0, me, L["ring_k"], L["ring_v"], wl.window,
+                               self.out, self.lse, self.ws_attn)
+        return self.out, self.lse
+
+    step = attend

@@ -1,0 +1,204 @@
+/*
+ * cskv.h - C ABI of the B200 (sm_100a) hybrid compressed sparse KV attention
+ * library (libcskv.so).
+ *
+ * What it computes (DeepSeek-V4 hybrid attention as described on the pages):
+ *  - CSA compresses the KV sequence 4x by softmax-gated pooling with a learned
+ *    positional bias, over windows that overlap across group boundaries; a
+ *    lightning indexer scores every CSA entry at low precision and the top-k
+ *    (512 for V4-Flash, 1,024 for V4-Pro) are attended sparsely.
+ *    («DeepSeek-V4: 1 Million Token Context endlich nutzbar», section "Hybrid
+ *    Attention: CSA und HCA"; «DeepSeek V4-Pro: Architektur,
+ *    KV-Cache-Kompression und Hyper-Connections im Detail», section
+ *    "Kompression und Selektion"; «Chinas KI-Unabhaengigkeit?: Bei Deepseek V4
+ *    haben kleine Aenderungen grosse Wirkung», section "Komprimierte
+ *    Erinnerung fuer laengere Kontexte".)
+ *  - HCA compresses 128x and attends densely over all compressed entries
+ *    (same sections).
+ *  - Both add the raw last-128-token sliding window, merged with the
+ *    compressed part through log-sum-exp into one softmax over the union
+ *    (golem.de section above; webconsulting.at "Das Wichtigste").
+ *  - Cache entries store the non-RoPE dims as FP8 E4M3 and the last 64 (RoPE)
+ *    dims as BF16 (chaosnode.de and golem.de sections above).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates nothing, keeps no state between calls and never synchronises
+ *    the stream; work is enqueued on `stream` (NULL = legacy default stream).
+ *  - Per-step sizes that change from step to step (token counts, positions)
+ *    are DEVICE int64 arrays, so a decode step can be captured in a CUDA graph.
+ *    Host-side bounds (max_new, max_entries) size the launch grids.
+ *  - Arguments are checked on the host before anything is enqueued; on an
+ *    argument error nothing is launched and a negative status is returned.
+ *  - Scratch memory comes from the caller's workspace `ws` of `ws_bytes`
+ *    bytes (256-byte aligned), sized with the matching *_workspace_size().
+ *  - Return value: CSKV_OK or a negative CSKV_ERR_* status; the text of a
+ *    status is cskv_error_string(status).  CSKV_ERR_CUDA reports a launch
+ *    error (the CUDA error is left pending for the caller to query).
+ *  - Every call is thread-safe; concurrent calls must not share outputs or
+ *    workspaces.
+ */
+#ifndef CSKV_H
+#define CSKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared opaquely so the header needs no CUDA include. */
+typedef struct CUstream_st *cskv_stream_t;
+
+enum {
+  CSKV_OK = 0,
+  CSKV_ERR_ARG = -1,          /* null pointer, bad shape, misalignment, size bound */
+  CSKV_ERR_UNSUPPORTED = -2,  /* valid but not implemented combination of formats/dims */
+  CSKV_ERR_CUDA = -3,         /* a kernel launch failed */
+  CSKV_ERR_WORKSPACE = -4     /* ws is NULL, misaligned or smaller than required */
+};
+
+enum {
+  CSKV_FMT_F32 = 0,        /* fp32 values, d_nope + d_rope per slot (no scale/rope planes) */
+  CSKV_FMT_E4M3_BF16 = 1   /* d_nope E4M3 codes + d_nope/64 fp32 scales + d_rope BF16 */
+};
+
+/*
+ * A cache of `cap` slots per sequence, for B sequences stored back to back.
+ * Slot s of sequence b starts at  plane + (b * cap + s) * plane_stride  in
+ * each plane (strides in BYTES).
+ *  - Compressed cache (ring = 0): entry j lives in slot j.
+ *  - Raw-token ring   (ring = 1): token position p lives in slot p % cap.
+ * E4M3_BF16 layout: value[d] = E4M3(data[d]) * scale[d / 64]  for d < d_nope,
+ *                   value[d_nope + r] = BF16(rope[r])          for r < d_rope.
+ * The lightning-indexer key cache uses the same descriptor with d_rope = 0.
+ * Alignment: data and rope pointers and strides are multiples of 16 bytes;
+ * scale pointer 16-byte aligned, scale stride a multiple of 4 bytes and at
+ * least 4 * ceil(d_nope / 64).  F32: data pointer and stride multiples of 16.
+ */
+typedef struct cskv_cache {
+  int32_t fmt;            /* CSKV_FMT_* */
+  int32_t d_nope;         /* E4M3 dims (multiple of 64) or leading fp32 dims */
+  int32_t d_rope;         /* BF16 dims, or trailing fp32 dims */
+  int32_t ring;           /* 0: slot = entry index; 1: slot = position % cap */
+  int64_t cap;            /* slots per sequence */
+  void *data;   int64_t data_stride;
+  float *scale; int64_t scale_stride;
+  void *rope;   int64_t rope_stride;
+} cskv_cache;
+
+/*
+ * csa_compress - CSA softmax-gated pooling (4x, overlapping windows).
+ * Entry j pools the `pool` raw tokens at positions
+ *     stride*(j+1) - pool + r,  r = 0 .. pool-1   (positions < 0 absent),
+ * i.e. the previous group and group j for pool = 8, stride = 4.  Gate logits
+ *     g_r = gate_w . k_{p_r} + gate_b[r]
+ * (gate_w [D] fp32 over the dequantised key, gate_b [pool] fp32 per slot),
+ * a = softmax(g) over present slots, entry = sum_r a_r x_{p_r} for the key,
+ * the value (raw_v, separate-V layout only) and the raw indexer key (raw_ik)
+ * alike.  E4M3 outputs are re-quantised per 64-element block with
+ * scale = amax / 448 (1 for an all-zero block), codes rounded to nearest even
+ * and saturated; BF16 dims rounded to nearest even.
+ * Writes every entry j with n(t_begin[b]) <= j < n(t_end[b]), n(t) = t / stride,
+ * at most max_new per sequence (the host bound that sizes the grid).
+ *   t_begin, t_end : [B] device int64; tokens [t_begin, t_end) just arrived.
+ *   raw_k, raw_v, raw_ik : rings (ring = 1) holding every position the new
+ *       entries read; raw_v and raw_ik may be NULL (K = V; no indexer keys).
+ *   out_k, out_v, out_ik : compressed caches (ring = 0) with cap >= n(t_end).
+ * Requirements: pool >= stride; cap of each ring >= (max_new - 1) * stride + pool,
+ * the span of positions that max_new consecutive entries read.
+ */
+int csa_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
+                 const cskv_cache *raw_k, const cskv_cache *raw_v, const cskv_cache *raw_ik,
+                 const float *gate_w, const float *gate_b, int pool, int stride,
+                 const cskv_cache *out_k, const cskv_cache *out_v, const cskv_cache *out_ik,
+                 cskv_stream_t stream);
+
+/*
+ * hca_compress - HCA pooling of 128 tokens into one entry by learned weights
+ * (pool = stride = 128 on the pages).  Same definition and arguments as
+ * csa_compress without the indexer keys.
+ */
+int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
+                 const cskv_cache *raw_k, const cskv_cache *raw_v,
+                 const float *gate_w, const float *gate_b, int pool, int stride,
+                 const cskv_cache *out_k, const cskv_cache *out_v, cskv_stream_t stream);
+
+/*
+ * indexer_topk - lightning-indexer scores of every visible CSA entry and the
+ * top-k selection per query row.
+ *   s_j = sum_h head_w[h] * max(0, q_ik[h] . k_ik[j])       (per query row)
+ * over visible entries j < n(q_pos + 1) = (q_pos + 1) / stride, then the k
+ * highest scores, ties to the lower index; fewer than k visible -> all of
+ * them, remaining slots -1.  The indices of one row are written in ascending
+ * entry order.
+ *   q_pos    : [B][Tq] device int64, position of each query token.
+ *   q_ik     : [B][Tq][H_I][d_I]; E4M3 codes when ik->fmt is E4M3_BF16 (with
+ *              q_ik_scale [B][Tq][H_I][d_I/64] fp32), fp32 when ik->fmt is F32
+ *              (q_ik_scale NULL).
+ *   head_w   : [B][Tq][H_I] fp32.
+ *   ik       : indexer-key cache (ring = 0, d_nope = d_I, d_rope = 0).
+ *   k        : selections per row, 1 <= k <= 4096.
+ *   max_entries : host bound on visible entries per row (<= ik->cap).
+ *   out_idx  : [B][Tq][k] int32.   out_score : [B][Tq][k] fp32 or NULL.
+ *   ws       : cskv_indexer_workspace_size(B, Tq, max_entries, k) bytes.
+ */
+int indexer_topk(int B, int Tq, const int64_t *q_pos,
+                 const void *q_ik, const float *q_ik_scale, const float *head_w,
+                 int H_I, int d_I, const cskv_cache *ik, int stride, int k,
+                 int64_t max_entries, int32_t *out_idx, float *out_score,
+                 void *ws, size_t ws_bytes, cskv_stream_t stream);
+
+size_t cskv_indexer_workspace_size(int B, int Tq, int64_t max_entries, int k);
+
+/*
+ * hybrid_attn_decode - one query token per sequence at position ctx_len-1.
+ * Keys: the compressed entries (sel != NULL: the k listed CSA entries, -1
+ * skipped; sel == NULL: every visible entry j < ctx_len / comp_stride, HCA)
+ * plus the raw window positions max(0, pos-window+1) .. pos, all under one
+ * softmax per head:
+ *   l = sm_scale * q_h . K,  out_h = sum softmax(l) V,  lse_h = log sum e^l.
+ * MQA: all Hq heads share one KV head; K = V = the whole entry unless comp_v /
+ * win_v are given (separate-V layout).  comp_k == NULL: window only.
+ *   ctx_len : [B] device int64, tokens including the query token.
+ *   q       : [B][Hq][D] BF16 for E4M3_BF16 caches, fp32 for F32 caches.
+ *   sel     : [B][k] int32 or NULL.   max_entries: host bound on compressed
+ *             keys per row (k when sel != NULL; visible entries otherwise).
+ *   win_k   : raw ring (ring = 1), cap >= window.
+ *   out     : [B][Hq][Dv] fp32.   lse : [B][Hq] fp32 (natural log).
+ *   ws      : cskv_attn_workspace_size(B, 1, Hq, Dv, max_entries, window) bytes.
+ */
+int hybrid_attn_decode(int B, const int64_t *ctx_len, const void *q, int Hq, float sm_scale,
+                       const cskv_cache *comp_k, const cskv_cache *comp_v, int comp_stride,
+                       const int32_t *sel, int k, int64_t max_entries,
+                       const cskv_cache *win_k, const cskv_cache *win_v, int window,
+                       float *out, float *lse, void *ws, size_t ws_bytes, cskv_stream_t stream);
+
+/*
+ * hybrid_attn_prefill - Tq query tokens per sequence at positions q_pos
+ * (chunked prefill); every row uses its own visibility: compressed entries
+ * j < (q_pos + 1) / comp_stride (dense) or its own sel row (sparse), and the
+ * window max(0, q_pos-window+1) .. q_pos, which makes attention causal inside
+ * the chunk.  Same definition and layouts as hybrid_attn_decode with a Tq
+ * axis: q [B][Tq][Hq][D], sel [B][Tq][k], out [B][Tq][Hq][Dv], lse [B][Tq][Hq].
+ * The ring must hold every position the chunk's windows reach.
+ */
+int hybrid_attn_prefill(int B, int Tq, const int64_t *q_pos, const void *q, int Hq,
+                        float sm_scale, const cskv_cache *comp_k, const cskv_cache *comp_v,
+                        int comp_stride, const int32_t *sel, int k, int64_t max_entries,
+                        const cskv_cache *win_k, const cskv_cache *win_v, int window,
+                        float *out, float *lse, void *ws, size_t ws_bytes, cskv_stream_t stream);
+
+size_t cskv_attn_workspace_size(int B, int Tq, int Hq, int Dv, int64_t max_entries, int window);
+
+/* Static text for a status code. */
+const char *cskv_error_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int cskv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSKV_H */

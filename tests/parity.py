@@ -1,0 +1,105 @@
+"""Comparison rules between the CUDA path and the oracle.
+
+  * top-k: the GPU set G and the oracle set R (entries >= 0) have equal size;
+    G lists distinct visible entries in ascending order, then -1 padding; any
+    entry in G\\R or R\\G has an oracle score within 1e-3 * |s_(k)| of the
+    oracle's k-th score s_(k) (a near-tie swap); otherwise the sets are equal.
+  * attention: max |o - o_ref| <= 2e-3 * RMS(o_ref) over the call's output,
+    and |lse - lse_ref| <= LSE_TOL.
+  * re-quantised entries: every stored code / BF16 pattern is one that exact
+    rounding produces for some input within a relative REL_EPS of the oracle's
+    float64 value; at least 99.9% equal the oracle's own rounding.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+
+TOPK_REL = 1e-3
+ATTN_REL = 2e-3
+# Natural-log units.  The tensor-core path rounds dequantised K/V and the
+# probabilities to fp16 (unit roundoff 2^-11); a logit over D = 512 dims then
+# carries an error of about sm_scale * 2^-11 * ||q|| * ||K|| / sqrt(D) ~ 5e-4,
+# and lse inherits at most the largest logit error.
+LSE_TOL = 2e-3
+# Relative perturbation of the pooled value covered by float32 evaluation of
+# the gate dot product (D terms), the softmax and the pooled sum.
+REL_EPS = 2e-5
+
+
+def check_topk(gpu_idx, ref_idx, ref_scores, where=""):
+    gpu_idx = np.asarray(gpu_idx, dtype=np.int64)
+    ref_idx = np.asarray(ref_idx, dtype=np.int64)
+    n_vis = ref_scores.shape[0]
+    R = ref_idx[ref_idx >= 0]
+    G = gpu_idx[gpu_idx >= 0]
+    assert G.size == R.size, f"{where}: {G.size} selected, oracle {R.size}"
+    assert np.all(gpu_idx[: G.size] >= 0) and np.all(gpu_idx[G.size:] == -1), f"{where}: padding"
+    assert np.all(np.diff(G) > 0), f"{where}: not strictly ascending"
+    assert np.all(G < n_vis), f"{where}: entry beyond the visible range"
+    gs, rs = set(G.tolist()), set(R.tolist())
+    if gs == rs:
+        return 0
+    sk = ref_scores[R[-1]]
+    tol = TOPK_REL * abs(sk)
+    diff = (gs - rs) | (rs - gs)
+    bad = [j for j in diff if abs(ref_scores[j] - sk) > tol]
+    assert not bad, (f"{where}: {len(bad)} swaps beyond the near-tie band, e.g. entry {bad[0]} "
+                     f"score {ref_scores[bad[0]]} vs k-th {sk}")
+    return len(gs - rs)
+
+
+def check_attention(out, lse, ref_o, ref_lse, where=""):
+    out = np.asarray(out, dtype=np.float64)
+    ref_o = np.asarray(ref_o, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref_o ** 2))
+    err = np.max(np.abs(out - ref_o))
+    assert np.all(np.isfinite(out)), f"{where}: non-finite output"
+    assert err <= ATTN_REL * rms, f"{where}: max|o-ref| = {err:.3e} > {ATTN_REL} * RMS {rms:.3e}"
+    lerr = np.max(np.abs(np.asarray(lse, dtype=np.float64) - ref_lse))
+    assert lerr <= LSE_TOL, f"{where}: max|lse-ref| = {lerr:.3e}"
+    return err / rms, lerr
+
+
+def _allowed(encode, y, eps):
+    y = np.asarray(y, dtype=np.float64)
+    d = eps * np.abs(y)
+    return encode(y), encode(y - d), encode(y + d)
+
+
+def check_codes(got, y, encode, eps=REL_EPS, min_exact=0.999, where=""):
+    """got: stored codes; y: oracle values in code units (float64)."""
+    got = np.asarray(got)
+    ref, lo, hi = _allowed(encode, y, eps)
+    ok = (got == ref) | (got == lo) | (got == hi)
+    assert np.all(ok), (f"{where}: {np.sum(~ok)} codes outside the rounding band, e.g. got "
+                        f"{got[~ok][:4]} want {ref[~ok][:4]} for {y[~ok][:4]}")
+    exact = np.mean(got == ref)
+    assert exact >= min_exact, f"{where}: only {exact:.5f} of codes equal the oracle's"
+    return exact
+
+
+def bf16_bits(t):
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def check_compressed_e4m3(cache, b, js, ref_vals, d_nope, where=""):
+    """cache: GPU planes (torch); ref_vals: oracle pooled float64 [n][D]."""
+    js = np.asarray(js)
+    codes = cache["data"][b, js].cpu().numpy()
+    nb = d_nope // 64
+    scales = cache["scale"][b, js][:, :nb].cpu().double().numpy()
+    amax = np.stack([np.max(np.abs(ref_vals[:, 64 * i:64 * (i + 1)]), axis=1)
+                     for i in range(nb)], axis=1)
+    ref_s = np.where(amax > 0, amax / 448.0, 1.0)
+    serr = np.max(np.abs(scales / ref_s - 1.0)) if scales.size else 0.0
+    assert serr <= REL_EPS, f"{where}: scale rel err {serr:.3e}"
+    y = ref_vals[:, :d_nope] / np.repeat(scales, 64, axis=1)
+    exact = check_codes(codes, y, O.e4m3_encode, where=where + " e4m3")
+    d_rope = ref_vals.shape[1] - d_nope
+    if d_rope:
+        rope = bf16_bits(cache["rope"][b, js])
+        check_codes(rope, ref_vals[:, d_nope:], O.bf16_encode, where=where + " bf16")
+    return exact, serr

@@ -1,0 +1,127 @@
+"""The C-ABI library loads, exports every entry point declared in
+include/cskv.h, and rejects bad arguments on the host before launching
+anything (CPU only: no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cskv.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "for")))
+
+
+@pytest.fixture(scope="module")
+def C():
+    import compressed_sparse_kv_softmax_b200 as C
+    return C
+
+
+def test_header_declares_the_five_calls():
+    d = _declared()
+    for n in ("csa_compress", "hca_compress", "indexer_topk", "hybrid_attn_decode",
+              "hybrid_attn_prefill"):
+        assert n in d
+
+
+def test_every_declared_symbol_is_exported(C):
+    lib = ctypes.CDLL(C.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), f"{name} declared in cskv.h but not exported"
+
+
+def test_error_strings_and_version(C):
+    assert C.error_string(0) == "ok"
+    for s in (-1, -2, -3, -4):
+        assert C.error_string(s) and C.error_string(s) != "unknown status"
+    assert C.version() >= 100
+
+
+def test_workspace_sizes(C):
+    assert C.attn_workspace_size(1, 1, 64, 512, 8192, 128) >= 64 * 513 * 4 * (8192 // 128)
+    assert C.indexer_workspace_size(1, 1, 262144, 1024) >= 262144 * 4
+    assert C.attn_workspace_size(0, 1, 64, 512, 8192, 128) == 0
+    assert C.indexer_workspace_size(1, 1, -1, 8) == 0
+
+
+def _fake_cache(ring, cap=256, fmt=1, d_nope=448, d_rope=64, ptr=1 << 20):
+    from compressed_sparse_kv_softmax_b200 import CskvCache
+    c = CskvCache()
+    c.fmt, c.d_nope, c.d_rope, c.ring, c.cap = fmt, d_nope, d_rope, ring, cap
+    c.data, c.data_stride = ptr, 448
+    c.scale, c.scale_stride = ptr + (1 << 24), 32
+    c.rope, c.rope_stride = ptr + (1 << 25), 128
+    return c
+
+
+def test_argument_errors_are_caught_on_the_host(C):
+    lib = C.lib
+    ERR_ARG, ERR_UNSUP, ERR_WS = C.ERR_ARG, C.ERR_UNSUPPORTED, C.ERR_WORKSPACE
+    P = ctypes.c_void_p
+    ring, comp = _fake_cache(1), _fake_cache(0, cap=8192)
+    q = P(1 << 26)
+    ctx = P(1 << 27)
+    out = P(1 << 28)
+    lse = P(1 << 29)
+    ws = P(1 << 30)
+    big = 1 << 34
+    R = ctypes.byref
+    # null query
+    assert lib.hybrid_attn_decode(1, ctx, None, 64, 0.04, R(comp), None, 128, None, 0, 8192,
+                                  R(ring), None, 128, out, lse, ws, big, None) == ERR_ARG
+    # window ring smaller than the window
+    small = _fake_cache(1, cap=64)
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(comp), None, 128, None, 0, 8192,
+                                  R(small), None, 128, out, lse, ws, big, None) == ERR_ARG
+    # compressed cache given as a ring
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(ring), None, 128, None, 0, 8192,
+                                  R(ring), None, 128, out, lse, ws, big, None) == ERR_ARG
+    # max_entries beyond the cache
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(comp), None, 128, None, 0, 9000,
+                                  R(ring), None, 128, out, lse, ws, big, None) == ERR_ARG
+    # sparse with k > max_entries
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(comp), None, 4, P(1 << 31), 1024, 512,
+                                  R(ring), None, 128, out, lse, ws, big, None) == ERR_ARG
+    # workspace too small / misaligned
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(comp), None, 128, None, 0, 8192,
+                                  R(ring), None, 128, out, lse, ws, 16, None) == ERR_WS
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(comp), None, 128, None, 0, 8192,
+                                  R(ring), None, 128, out, lse, P((1 << 30) + 8), big,
+                                  None) == ERR_WS
+    # misaligned plane stride
+    bad = _fake_cache(0, cap=8192)
+    bad.data_stride = 450
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(bad), None, 128, None, 0, 8192,
+                                  R(ring), None, 128, out, lse, ws, big, None) == ERR_ARG
+    # d_nope not a multiple of 64 in the FP8 layout
+    odd = _fake_cache(0, cap=8192, d_nope=100)
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(odd), None, 128, None, 0, 8192,
+                                  R(ring), None, 128, out, lse, ws, big, None) == ERR_UNSUP
+    # indexer: k out of range, key cache with rope dims, missing scales
+    ik = _fake_cache(0, cap=262144, d_nope=128, d_rope=0)
+    ik.data_stride, ik.scale_stride = 128, 8
+    args = (1, 1, ctx, q, P(1 << 32), P(1 << 33), 64, 128)
+    assert lib.indexer_topk(*args, R(ik), 4, 0, 262144, out, None, ws, big, None) == ERR_ARG
+    assert lib.indexer_topk(*args, R(ik), 4, 5000, 262144, out, None, ws, big, None) == ERR_ARG
+    assert lib.indexer_topk(1, 1, ctx, q, None, P(1 << 33), 64, 128, R(ik), 4, 1024, 262144,
+                            out, None, ws, big, None) == ERR_ARG
+    assert lib.indexer_topk(*args, R(ik), 4, 1024, 262145, out, None, ws, big, None) == ERR_ARG
+    assert lib.indexer_topk(*args, R(comp), 4, 1024, 8192, out, None, ws, big, None) == ERR_ARG
+    # compress: ring too small for the entries requested, pool < stride
+    gate = P(1 << 35)
+    assert lib.csa_compress(1, ctx, ctx, 100, R(ring), None, None, gate, gate, 8, 4, R(comp),
+                            None, None, None) == ERR_ARG
+    assert lib.hca_compress(1, ctx, ctx, 1, R(ring), None, gate, gate, 64, 128, R(comp), None,
+                            None) == ERR_ARG
+    # zero-sized work is a no-op success without touching the device
+    assert lib.csa_compress(1, ctx, ctx, 0, R(ring), None, None, gate, gate, 8, 4, R(comp),
+                            None, None, None) == 0
+    assert lib.hybrid_attn_prefill(1, 0, ctx, q, 64, 0.04, R(comp), None, 128, None, 0, 8192,
+                                   R(ring), None, 128, out, lse, ws, big, None) == 0

@@ -1,0 +1,260 @@
+"""GPU-vs-oracle parity of every stage, through the C ABI, on seeded inputs:
+CSA/HCA compression, indexer top-k, sparse/dense hybrid attention with the
+window, decode and chunked prefill, fp32 and FP8+BF16 layouts, edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from gpu_common import require_gpu, sample_rows, to_device
+from parity import check_attention, check_compressed_e4m3, check_topk
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def C():
+    return require_gpu()
+
+
+# ------------------------------------------------------------------ compress
+
+def _run_compress(C, L, Ld, t_begin, t_end, kind):
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
+    B = len(t_begin)
+    tb = torch.tensor(t_begin, dtype=torch.int64, device="cuda")
+    te = torch.tensor(t_end, dtype=torch.int64, device="cuda")
+    S = Ld["stride"]
+    max_new = max(e // S - b // S for b, e in zip(t_begin, t_end))
+    layer = CSALayer(Ld) if kind == "csa" else HCALayer(Ld)
+    layer.compress(tb, te, max(max_new, 1))
+    torch.cuda.synchronize()
+    return O.layer_compress(L, t_begin, t_end)
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+@pytest.mark.parametrize("span", [1, 4, 300])
+def test_compress_f32_tiny(C, kind, span):
+    wl = W.get("tiny").with_(T=4096 + 7)
+    mk = W.make_csa_layer if kind == "csa" else W.make_hca_layer
+    L = mk(wl, ring_cap=1024)
+    Ld = to_device(L)
+    T = wl.T
+    ref = _run_compress(C, L, Ld, [T - span], [T], kind)[0]
+    for name, key in (("k", "comp_k"), ("v", "comp_v"), ("ik", "comp_ik")):
+        if name not in ref or not len(ref["j"]):
+            continue
+        got = Ld[key]["data"][0, ref["j"]].double().cpu().numpy()
+        want = ref[name]
+        err = np.max(np.abs(got - want) / (1e-3 + np.abs(want)))
+        assert err <= 2e-5, (name, err)
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_compress_e4m3_parity_decode(C, kind):
+    wl = W.get("parity_decode")
+    mk = W.make_csa_layer if kind == "csa" else W.make_hca_layer
+    L = mk(wl, ring_cap=1024)
+    Ld = to_device(L)
+    T = wl.T
+    t_begin = [T - 600, T - 1, T - 257]
+    t_end = [T, T, T - 1]
+    res = _run_compress(C, L, Ld, t_begin, t_end, kind)
+    n_checked = 0
+    for b, r in enumerate(res):
+        if not len(r["j"]):
+            continue
+        check_compressed_e4m3(Ld["comp_k"], b, r["j"], r["k"], wl.d_nope, where=f"{kind} b{b} kv")
+        if "ik" in r:
+            check_compressed_e4m3(Ld["comp_ik"], b, r["j"], r["ik"], wl.d_I, where=f"b{b} ik")
+        n_checked += len(r["j"])
+    assert n_checked > 0
+
+
+def test_compress_first_entries_left_edge(C):
+    # the first CSA entries see positions < 0 (absent slots)
+    wl = W.get("parity_decode").with_(T=40, B=1)
+    L = W.make_csa_layer(wl, ring_cap=64)
+    Ld = to_device(L)
+    ref = _run_compress(C, L, Ld, [0], [40], "csa")[0]
+    assert list(ref["j"]) == list(range(10))
+    check_compressed_e4m3(Ld["comp_k"], 0, ref["j"], ref["k"], wl.d_nope, where="left edge")
+
+
+# ------------------------------------------------------------------- indexer
+
+def _run_indexer(C, Ld, k=None):
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    layer = CSALayer(Ld, k=k)
+    layer.select()
+    torch.cuda.synchronize()
+    return layer
+
+
+@pytest.mark.parametrize("name", ["tiny", "parity_decode", "parity_prefill"])
+def test_indexer_topk(C, name):
+    wl = W.get(name)
+    L = W.make_csa_layer(wl)
+    Ld = to_device(L)
+    layer = _run_indexer(C, Ld)
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_indexer_topk(L, wl.k, rows=rows)
+    idx = layer.idx.cpu().numpy()
+    sc = layer.score.cpu().numpy()
+    for (b, t), (ridx, rs) in ref.items():
+        check_topk(idx[b, t], ridx, rs, where=f"{name} row {(b, t)}")
+        sel = idx[b, t][idx[b, t] >= 0]
+        assert np.allclose(sc[b, t][: sel.size], rs[sel], rtol=1e-4, atol=1e-4 * np.abs(rs).max())
+
+
+@pytest.mark.parametrize("T,k", [(3, 8), (4, 8), (64, 16), (64, 100), (517, 129)])
+def test_indexer_edge_sizes(C, T, k):
+    wl = W.get("parity_decode").with_(T=T, B=2, k=k)
+    L = W.make_csa_layer(wl)
+    Ld = to_device(L)
+    layer = _run_indexer(C, Ld)
+    ref = O.layer_indexer_topk(L, k)
+    idx = layer.idx.cpu().numpy()
+    for (b, t), (ridx, rs) in ref.items():
+        check_topk(idx[b, t], ridx, rs, where=f"T={T} k={k} row {(b, t)}")
+
+
+# ----------------------------------------------------------------- attention
+
+def _sel_from_oracle(L, k):
+    wl = L["wl"]
+    ref = O.layer_indexer_topk(L, k)
+    sel = np.full((wl.B, wl.Tq, k), -1, dtype=np.int32)
+    for (b, t), (idx, _) in ref.items():
+        sel[b, t] = idx
+    return sel
+
+
+@pytest.mark.parametrize("name", ["tiny", "parity_decode", "parity_prefill"])
+def test_csa_attention_given_selection(C, name):
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    wl = W.get(name)
+    L = W.make_csa_layer(wl)
+    Ld = to_device(L)
+    sel = _sel_from_oracle(L, wl.k)
+    layer = CSALayer(Ld)
+    out, lse = layer.attend(torch.from_numpy(sel).cuda())
+    torch.cuda.synchronize()
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_attention(L, sel=sel, rows=rows)
+    got_o = np.stack([out[b, t].cpu().numpy() for b, t in rows])
+    got_l = np.stack([lse[b, t].cpu().numpy() for b, t in rows])
+    check_attention(got_o, got_l, np.stack([ref[r][0] for r in rows]),
+                    np.stack([ref[r][1] for r in rows]), where=name)
+
+
+@pytest.mark.parametrize("name", ["tiny", "parity_decode", "parity_prefill"])
+def test_hca_dense_attention(C, name):
+    from compressed_sparse_kv_softmax_b200.layer import HCALayer
+    wl = W.get(name)
+    L = W.make_hca_layer(wl)
+    Ld = to_device(L)
+    layer = HCALayer(Ld)
+    out, lse = layer.attend()
+    torch.cuda.synchronize()
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_attention(L, sel=None, rows=rows)
+    got_o = np.stack([out[b, t].cpu().numpy() for b, t in rows])
+    got_l = np.stack([lse[b, t].cpu().numpy() for b, t in rows])
+    check_attention(got_o, got_l, np.stack([ref[r][0] for r in rows]),
+                    np.stack([ref[r][1] for r in rows]), where=name)
+
+
+@pytest.mark.parametrize("T", [1, 2, 77, 128, 129, 300])
+def test_window_only_layer(C, T):
+    from compressed_sparse_kv_softmax_b200.layer import HCALayer
+    wl = W.get("parity_decode").with_(T=T, B=2)
+    L = W.make_hca_layer(wl)
+    Ld = to_device(L)
+    layer = HCALayer(Ld, dense=False)
+    out, lse = layer.attend()
+    torch.cuda.synchronize()
+    for b in range(wl.B):
+        q, _, _, wk, wv = O.layer_attention_dense_keys(L, b, 0)
+        ro, rl = O.attend(q, wk, wv, wl.sm_scale)
+        check_attention(out[b, 0].cpu().numpy(), lse[b, 0].cpu().numpy(), ro, rl, where=f"T={T}")
+
+
+@pytest.mark.parametrize("T", [3, 5, 130, 1000])
+def test_dense_small_contexts(C, T):
+    from compressed_sparse_kv_softmax_b200.layer import HCALayer
+    for mk in (W.make_hca_layer, W.make_csa_layer):
+        wl = W.get("parity_decode").with_(T=T, B=2)
+        L = mk(wl)
+        Ld = to_device(L)
+        layer = HCALayer(Ld)
+        out, lse = layer.attend()
+        torch.cuda.synchronize()
+        ref = O.layer_attention(L, sel=None)
+        for (b, t), (ro, rl) in ref.items():
+            check_attention(out[b, t].cpu().numpy(), lse[b, t].cpu().numpy(), ro, rl,
+                            where=f"T={T}")
+
+
+def test_sparse_with_holes_and_k_above_entries(C):
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    wl = W.get("parity_decode").with_(T=201, B=2, k=64)     # 50 entries visible, k = 64
+    L = W.make_csa_layer(wl)
+    Ld = to_device(L)
+    sel = _sel_from_oracle(L, wl.k)
+    assert np.sum(sel[0, 0] == -1) == 14
+    layer = CSALayer(Ld)
+    out, lse = layer.attend(torch.from_numpy(sel).cuda())
+    torch.cuda.synchronize()
+    ref = O.layer_attention(L, sel=sel)
+    dense = O.layer_attention(L, sel=None)
+    for key, (ro, rl) in ref.items():
+        check_attention(out[key].cpu().numpy(), lse[key].cpu().numpy(), ro, rl, where="holes")
+        # k >= entries: the sparse result equals dense attention over all entries
+        check_attention(out[key].cpu().numpy(), lse[key].cpu().numpy(), *dense[key],
+                        where="k>=n")
+
+
+# ---------------------------------------------------------------- end to end
+
+def test_end_to_end_tiny_pipeline(C):
+    """GPU compress -> GPU indexer -> GPU attention against the oracle's own
+    pipeline on the same raw tokens (no GPU value enters the oracle)."""
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
+    wl = W.get("tiny").with_(T=2048 + 3)
+    for kind in ("csa", "hca"):
+        mk = W.make_csa_layer if kind == "csa" else W.make_hca_layer
+        L = mk(wl, ring_cap=4096)
+        Ld = to_device(L)
+        T = wl.T
+        S = L["stride"]
+        tb = torch.zeros(1, dtype=torch.int64, device="cuda")
+        te = torch.full((1,), T, dtype=torch.int64, device="cuda")
+        layer = CSALayer(Ld) if kind == "csa" else HCALayer(Ld)
+        layer.compress(tb, te, T // S)
+        # oracle pipeline: its own compression of the same ring
+        comp = O.layer_compress(L, [0], [T])[0]
+        Lo = dict(L)
+        for name, key in (("k", "comp_k"), ("v", "comp_v"), ("ik", "comp_ik")):
+            if name in comp:
+                c = dict(L[key])
+                c["data"] = torch.from_numpy(comp[name][None].astype(np.float32))
+                Lo[key] = c
+        if kind == "csa":
+            layer.select()
+            torch.cuda.synchronize()
+            (ridx, rs), = O.layer_indexer_topk(Lo, wl.k).values()
+            n_swaps = check_topk(layer.idx[0, 0].cpu().numpy(), ridx, rs, where="e2e")
+            out, lse = layer.attend()
+            torch.cuda.synchronize()
+            if n_swaps == 0:
+                (ro, rl), = O.layer_attention(Lo, sel=ridx[None, None]).values()
+                check_attention(out[0, 0].cpu().numpy(), lse[0, 0].cpu().numpy(), ro, rl,
+                                where="e2e csa")
+        else:
+            out, lse = layer.attend()
+            torch.cuda.synchronize()
+            (ro, rl), = O.layer_attention(Lo, sel=None).values()
+            check_attention(out[0, 0].cpu().numpy(), lse[0, 0].cpu().numpy(), ro, rl,
+                            where="e2e hca")
