@@ -224,13 +224,7 @@ int launch_attention(const AttnArgs &a, cudaStream_t st) {
     const size_t smem = sizeof(float) * ((size_t)a.Hq * a.D + (size_t)kChunk * (a.D + 1) +
                                          (sep_v ? (size_t)kChunk * (a.Dv + 1) : 0) +
                                          (size_t)a.Hq * kChunk);
-    if (smem > 227 * 1024) return CSKV_ERR_UNSUPPORTED;
-    static int smem_set = 0;   // largest dynamic smem opted in so far (one-time set-up)
-    if ((int)smem > smem_set) {
-      cudaFuncSetAttribute(attn_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           227 * 1024);
-      smem_set = 227 * 1024;
-    }
+    if (!ensure_dynamic_smem(attn_chunk_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
     attn_chunk_kernel<<<dim3(nc, rows), kThreads, smem, st>>>(a, ncc, nc, part_o, part_lse);
     if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
   }

@@ -86,6 +86,30 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Opt a kernel in to `bytes` of dynamic shared memory (host, idempotent).
+// Returns false when the request does not fit next to the kernel's static
+// shared memory.  Clears the error it may leave behind.
+template <typename K>
+inline bool ensure_dynamic_smem(K kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return true;
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if ((size_t)attr.maxDynamicSharedSizeBytes >= bytes) return true;
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (bytes + attr.sharedSizeBytes > (size_t)optin) return false;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+
 // host-side launch helpers (defined in the kernel files)
 int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
                     const Cache &raw_k, const Cache &raw_v, const Cache &raw_ik,

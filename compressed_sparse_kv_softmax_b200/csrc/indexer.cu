@@ -90,12 +90,7 @@ int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
     } else {
       const size_t smem = sizeof(float) * ((size_t)a.H_I * a.d_I + a.H_I +
                                            (size_t)kKeys * (a.d_I + 1));
-      static bool smem_set = false;   // one-time opt-in to the full shared memory
-      if (smem > 48 * 1024 && !smem_set) {
-        cudaFuncSetAttribute(indexer_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             200 * 1024);
-        smem_set = true;
-      }
+      if (!ensure_dynamic_smem(indexer_score_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
       dim3 grid((unsigned)((a.max_entries + kKeys - 1) / kKeys), (unsigned)rows);
       indexer_score_kernel<<<grid, kKeys, smem, st>>>(a, scores, ld);
       if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;

@@ -77,6 +77,12 @@ def layer_compress(L, t_begin, t_end):
         r = {"j": np.asarray(js, dtype=np.int64), "weights": w}
         for name, arr in zip(names, pooled):
             r[name] = arr
+        # sum_r a_r |x_{p_r}|: the magnitude scale of each pooled sum, which
+        # bounds its floating-point evaluation error
+        absvals = [(lambda f: (lambda p: np.abs(f(p))))(v) for v in vals]
+        mags, _ = pool_entries(reader(ring_k), absvals, gw, gb, pool, stride, js)
+        for name, arr in zip(names, mags):
+            r[name + "_mag"] = arr
         if ring_k["fmt"] != "f32":
             for name, d_nope in (("k", ring_k["d_nope"]),
                                  ("ik", ring_ik["d_nope"] if ring_ik else None)):

@@ -8,7 +8,7 @@ import torch
 import oracle as O
 import workloads as W
 from gpu_common import require_gpu, sample_rows, to_device
-from parity import check_attention, check_compressed_e4m3, check_topk
+from parity import check_attention, check_compressed_e4m3, check_pooled_f32, check_topk
 
 pytestmark = pytest.mark.gpu
 
@@ -46,9 +46,7 @@ def test_compress_f32_tiny(C, kind, span):
         if name not in ref or not len(ref["j"]):
             continue
         got = Ld[key]["data"][0, ref["j"]].double().cpu().numpy()
-        want = ref[name]
-        err = np.max(np.abs(got - want) / (1e-3 + np.abs(want)))
-        assert err <= 2e-5, (name, err)
+        check_pooled_f32(got, ref[name], ref[name + "_mag"], where=f"{kind} {name}")
 
 
 @pytest.mark.parametrize("kind", ["csa", "hca"])
@@ -65,9 +63,11 @@ def test_compress_e4m3_parity_decode(C, kind):
     for b, r in enumerate(res):
         if not len(r["j"]):
             continue
-        check_compressed_e4m3(Ld["comp_k"], b, r["j"], r["k"], wl.d_nope, where=f"{kind} b{b} kv")
+        check_compressed_e4m3(Ld["comp_k"], b, r["j"], r["k"], r["k_mag"], wl.d_nope,
+                              where=f"{kind} b{b} kv")
         if "ik" in r:
-            check_compressed_e4m3(Ld["comp_ik"], b, r["j"], r["ik"], wl.d_I, where=f"b{b} ik")
+            check_compressed_e4m3(Ld["comp_ik"], b, r["j"], r["ik"], r["ik_mag"], wl.d_I,
+                                  where=f"b{b} ik")
         n_checked += len(r["j"])
     assert n_checked > 0
 
@@ -79,7 +79,8 @@ def test_compress_first_entries_left_edge(C):
     Ld = to_device(L)
     ref = _run_compress(C, L, Ld, [0], [40], "csa")[0]
     assert list(ref["j"]) == list(range(10))
-    check_compressed_e4m3(Ld["comp_k"], 0, ref["j"], ref["k"], wl.d_nope, where="left edge")
+    check_compressed_e4m3(Ld["comp_k"], 0, ref["j"], ref["k"], ref["k_mag"], wl.d_nope,
+                          where="left edge")
 
 
 # ------------------------------------------------------------------- indexer
