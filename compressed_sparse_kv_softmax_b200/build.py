@@ -1,6 +1,9 @@
 """Build libcskv.so in-tree for sm_100a with nvcc.
 
-    python -m compressed_sparse_kv_softmax_b200.build [-v]
+    python compressed_sparse_kv_softmax_b200/build.py [-v]
+
+(Run it as a script: importing it through the package would first load the
+library it builds.)
 
 Each csrc/*.cu compiles to an object under _build/ (in parallel), then the
 objects link into compressed_sparse_kv_softmax_b200/libcskv.so.
