@@ -24,7 +24,7 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, -1, -2, -3, -4
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_SCRATCH_LIMIT = 0, -1, -2, -3, -4, -5
 FMT_F32, FMT_E4M3_BF16 = 0, 1
 
 
@@ -52,6 +52,10 @@ _lib.cskv_indexer_workspace_size.argtypes = [_I, _I, _I64, _I]
 _lib.cskv_indexer_workspace_size.restype = _SZ
 _lib.cskv_attn_workspace_size.argtypes = [_I, _I, _I, _I, _I64, _I]
 _lib.cskv_attn_workspace_size.restype = _SZ
+_lib.indexer_topk_noalloc.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC, _I, _I, _I64, _P,
+                                      _P, _P]
+_lib.indexer_topk_noalloc.restype = _I
+_lib.cskv_noalloc_scratch_bytes.restype = _SZ
 _lib.cskv_error_string.argtypes = [_I]
 _lib.cskv_error_string.restype = ctypes.c_char_p
 _lib.cskv_version.restype = _I
@@ -156,6 +160,22 @@ def indexer_topk(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k
                              H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
                              _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
            "indexer_topk")
+
+
+def indexer_topk_noalloc(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k,
+                         max_entries, out_idx, out_score, stream=None):
+    """indexer_topk without a workspace, for callers that cannot allocate one:
+    the library's fixed device scratch array is used instead (see cskv.h).
+    Calls that overlap on the GPU share that array and must be serialised."""
+    c = cache_struct(ik)
+    _check(_lib.indexer_topk_noalloc(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale),
+                                     _ptr(head_w), H_I, d_I, ctypes.byref(c), stride, k,
+                                     int(max_entries), _ptr(out_idx), _ptr(out_score),
+                                     _stream(stream)), "indexer_topk_noalloc")
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(_lib.cskv_noalloc_scratch_bytes())
 
 
 def hybrid_attn_decode(B, ctx_len, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,

@@ -224,6 +224,8 @@ const char *cskv_error_string(int status) {
     case CSKV_ERR_UNSUPPORTED: return "unsupported format or dimension combination";
     case CSKV_ERR_CUDA: return "CUDA kernel launch failed";
     case CSKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case CSKV_ERR_SCRATCH_LIMIT:
+      return "request needs more scratch than indexer_topk_noalloc's fixed array holds";
     default: return "unknown status";
   }
 }

@@ -56,7 +56,8 @@ enum {
   CSKV_ERR_ARG = -1,          /* null pointer, bad shape, misalignment, size bound */
   CSKV_ERR_UNSUPPORTED = -2,  /* valid but not implemented combination of formats/dims */
   CSKV_ERR_CUDA = -3,         /* a kernel launch failed */
-  CSKV_ERR_WORKSPACE = -4     /* ws is NULL, misaligned or smaller than required */
+  CSKV_ERR_WORKSPACE = -4,    /* ws is NULL, misaligned or smaller than required */
+  CSKV_ERR_SCRATCH_LIMIT = -5 /* request larger than indexer_topk_noalloc's fixed scratch */
 };
 
 enum {
@@ -151,6 +152,35 @@ int indexer_topk(int B, int Tq, const int64_t *q_pos,
                  void *ws, size_t ws_bytes, cskv_stream_t stream);
 
 size_t cskv_indexer_workspace_size(int B, int Tq, int64_t max_entries, int k);
+
+/*
+ * indexer_topk_noalloc - indexer_topk for callers that cannot provide a
+ * workspace (no counterpart on the pages: it is a deployment convenience).
+ * Callers that may not allocate device memory themselves - a host framework
+ * that owns every device allocation through its own pool and passes plug-ins
+ * no scratch, a real-time loop that forbids allocation after start-up, an
+ * op interface without a workspace argument - use this variant.  Same
+ * arguments and results as indexer_topk minus ws/ws_bytes; the scratch is a
+ * fixed array of cskv_noalloc_scratch_bytes() (8 MiB) in the library's device
+ * memory, held on every GPU that loads the library until the process exits.
+ *  - The first call on a device looks the array's address up (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - Requests whose workspace (cskv_indexer_workspace_size) exceeds the array
+ *    return CSKV_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *  - All calls share the array: calls that may overlap on the GPU (other
+ *    streams or host threads on the same device) race and must be serialised
+ *    by the caller.  Nothing in the array needs to start at zero.
+ *  - It allocates nothing (no cudaMalloc / cudaFree or allocating library call).
+ */
+int indexer_topk_noalloc(int B, int Tq, const int64_t *q_pos,
+                         const void *q_ik, const float *q_ik_scale, const float *head_w,
+                         int H_I, int d_I, const cskv_cache *ik, int stride, int k,
+                         int64_t max_entries, int32_t *out_idx, float *out_score,
+                         cskv_stream_t stream);
+
+/* Size in bytes of indexer_topk_noalloc's fixed scratch array. */
+size_t cskv_noalloc_scratch_bytes(void);
 
 /*
  * hybrid_attn_decode - one query token per sequence at position ctx_len-1.
