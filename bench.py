@@ -217,7 +217,8 @@ def run_ours(args, rank, world, dev):
     wl = W.get(args.workload)
     torch.cuda.set_device(dev)
     per_rep_bytes = step_bytes(wl)
-    R = max(args.replicas, math.ceil(4 * 126e6 / per_rep_bytes) + 1)
+    # enough replicas that one rotation touches > 4x the 126 MB L2 (unless set)
+    R = args.replicas if args.replicas > 0 else math.ceil(4 * 126e6 / per_rep_bytes) + 1
     replicas = [Replica(wl, 1000 + r + 7919 * rank, dev) for r in range(R)]
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
@@ -479,7 +480,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="long")
-    ap.add_argument("--replicas", type=int, default=4)
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="input replicas to rotate (0: enough to exceed 4x L2)")
     ap.add_argument("--graph-steps", type=int, default=250)
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--cpu-budget", type=float, default=12.0)

@@ -12,14 +12,19 @@
 // The 64-head x 128-dim FP8 layout at scale goes through the tensor-core
 // kernel in indexer_tc.cu.
 #include "cskv_internal.cuh"
+#include "topk_common.cuh"
 
 namespace cskv {
 
 void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,
                       long long max_entries, int k, int rows, int32_t *out_idx,
                       float *out_score, cudaStream_t st);
+int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
+                       long long max_entries, int k, int rows, int32_t *out_idx,
+                       float *out_score, cudaStream_t st);
 bool indexer_tc_supported(const IndexerArgs &a);
-int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, cudaStream_t st);
+int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
+                      int *err, cudaStream_t st);
 
 namespace {
 
@@ -73,30 +78,32 @@ indexer_score_kernel(IndexerArgs a, float *__restrict__ scores, long long ld) {
 }  // namespace
 
 size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k) {
-  (void)k;
-  const long long ld = (max_entries + 3) & ~3LL;
-  return (size_t)B * Tq * ld * sizeof(float) + 256;
+  size_t total = 0;
+  indexer_ws_layout(nullptr, (long long)B * Tq, max_entries, k, &total);
+  return total;
 }
 
 int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
   const int rows = a.B * a.Tq;
   if (rows == 0) return CSKV_OK;
-  const long long ld = (a.max_entries + 3) & ~3LL;
-  float *scores = reinterpret_cast<float *>(a.ws);
-  if (a.max_entries > 0) {
-    if (indexer_tc_supported(a)) {
-      const int rc = launch_indexer_tc(a, scores, ld, st);
-      if (rc != CSKV_OK) return rc;
-    } else {
-      const size_t smem = sizeof(float) * ((size_t)a.H_I * a.d_I + a.H_I +
-                                           (size_t)kKeys * (a.d_I + 1));
-      if (!ensure_dynamic_smem(indexer_score_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
-      dim3 grid((unsigned)((a.max_entries + kKeys - 1) / kKeys), (unsigned)rows);
-      indexer_score_kernel<<<grid, kKeys, smem, st>>>(a, scores, ld);
-      if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
-    }
+  const IndexerWs w = indexer_ws_layout(a.ws, rows, a.max_entries, a.k, nullptr);
+  if (a.max_entries > 0 && indexer_tc_supported(a)) {
+    // tensor-core scoring builds the score histogram the multi-CTA selection uses
+    if (cudaMemsetAsync(w.hist, 0, w.zero_bytes, st) != cudaSuccess) return CSKV_ERR_CUDA;
+    int rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
+    if (rc != CSKV_OK) return rc;
+    return launch_topk_select(w, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
+                              a.out_score, st);
   }
-  launch_topk_rows(scores, ld, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
+  if (a.max_entries > 0) {
+    const size_t smem = sizeof(float) * ((size_t)a.H_I * a.d_I + a.H_I +
+                                         (size_t)kKeys * (a.d_I + 1));
+    if (!ensure_dynamic_smem(indexer_score_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)((a.max_entries + kKeys - 1) / kKeys), (unsigned)rows);
+    indexer_score_kernel<<<grid, kKeys, smem, st>>>(a, w.scores, w.ld);
+    if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
+  }
+  launch_topk_rows(w.scores, w.ld, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
                    a.out_score, st);
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }

@@ -1,13 +1,294 @@
-// Tensor-core (tcgen05) lightning-indexer scoring for the FP8 64-head x 128-dim layout.
+// Lightning-indexer scoring on the 5th-generation tensor cores (tcgen05) for
+// the FP8 layout with 64 indexer heads of dim 128.
+//
+// The indexer scores every compressed CSA entry per query at low precision
+// («DeepSeek V4-Pro: Architektur, KV-Cache-Kompression und Hyper-Connections
+// im Detail», "Kompression und Selektion"; «DeepSeek-V4: 1 Million Token
+// Context endlich nutzbar», "Hybrid Attention: CSA und HCA"):
+//   s_j = sum_h w_h * max(0, q_h . k_j),   q_h . k_j = sum_b sq_{h,b} sk_{j,b} (Q_h,b . K_j,b)
+// where b indexes the two 64-element scale blocks of the 128-dim FP8 vectors.
+//
+// Per query row the entries are a [n x 128] FP8 matrix: each 128-entry tile
+// is one MMA of M = 128 entries x N = 64 heads, with the two scale blocks
+// accumulated separately (K = 64 each) so the per-entry and per-head block
+// scales can be applied in fp32 afterwards.
+//
+// CTA roles (persistent over the row's tiles assigned to the CTA):
+//   warp 0      TMA producer: key tiles (128 rows x 128 B, 128-byte swizzle)
+//               into a kStages-deep shared-memory ring
+//   warp 1      MMA issuer (one thread): 4 tcgen05.mma per tile into one of
+//               kAcc TMEM accumulator slots (2 x 64 fp32 columns each)
+//   warp 2      TMEM allocation
+//   warps 4-11  two epilogue warpgroups taking alternate tiles: tcgen05.ld,
+//               block scales, per-head ReLU, head weights -> score; score
+//               histogram (top 12 bits of the order-preserving key) for the
+//               selection kernel
+// HBM traffic is the key tile stream (128 B + the 8 B of scales per entry);
+// scores (4 B per entry) go to the workspace and stay in L2.
+#include <cudaTypedefs.h>
+
 #include "cskv_internal.cuh"
+#include "sm100.cuh"
+#include "topk_common.cuh"
 
 namespace cskv {
 
-bool indexer_tc_supported(const IndexerArgs &a) { (void)a; return false; }
+namespace {
 
-int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, cudaStream_t st) {
-  (void)a; (void)scores; (void)ld; (void)st;
-  return CSKV_ERR_UNSUPPORTED;
+using namespace sm100;
+
+constexpr int kTile = 128;          // entries per tile (MMA M)
+constexpr int kHeads = 64;          // MMA N
+constexpr int kDim = 128;           // bytes per key (FP8 dims)
+constexpr int kStages = 8;
+constexpr int kAcc = 4;             // TMEM accumulator slots, 128 columns each
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (4 + kEpiWarps);
+constexpr uint32_t kTileBytes = kTile * kDim;
+constexpr uint32_t kIdesc = idesc(kFmtE4M3, kFmtE4M3, 0, 0, kTile, kHeads);
+
+struct __align__(1024) Smem {
+  uint8_t keys[kStages][kTileBytes];      // 1024-aligned tiles
+  uint8_t q[kHeads * kDim];               // B operand, K-major, 128-byte swizzle
+  float4 qc[kHeads];                      // (sq0, sq1, w, 0) per head
+  uint32_t hist[kTopkBins];
+  uint64_t full[kStages], empty[kStages], acc_full[kAcc], acc_empty[kAcc], mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void record_abort(Smem &sm, int *err, int code) {
+  sm.abort = 1;
+  if (err) atomicOr(err, code);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
+                  float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
+                  int *__restrict__ err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem &sm = *reinterpret_cast<Smem *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.y;
+  const int b = row / a.Tq;
+  long long n = (a.q_pos[row] + 1) / a.stride;
+  if (n > a.max_entries) n = a.max_entries;
+  if (n < 0) n = 0;
+  const int tiles = (int)((n + kTile - 1) / kTile);
+  const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
+    for (int s = 0; s < kAcc; ++s) {
+      mbar_init(&sm.acc_full[s], 1);
+      mbar_init(&sm.acc_empty[s], 32 * kEpiWarps / 2);
+    }
+    mbar_init(&sm.mma_done, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmap);
+  if (warp == 2) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  // query heads -> B operand (K-major, 128-byte swizzle: 16-byte chunk c of
+  // head h lands at chunk c ^ (h & 7) of its 128-byte row)
+  {
+    const uint8_t *qsrc = reinterpret_cast<const uint8_t *>(a.q_ik) + (size_t)row * kHeads * kDim;
+    for (int i = tid; i < kHeads * kDim / 16; i += kThreads) {
+      const int h = i >> 3, c = i & 7;
+      const uint4 v = *reinterpret_cast<const uint4 *>(qsrc + h * kDim + c * 16);
+      *reinterpret_cast<uint4 *>(&sm.q[h * kDim + ((c ^ (h & 7)) << 4)]) = v;
+    }
+    for (int h = tid; h < kHeads; h += kThreads) {
+      const float *qs = a.q_ik_scale + ((size_t)row * kHeads + h) * 2;
+      sm.qc[h] = make_float4(qs[0], qs[1], a.head_w[(size_t)row * kHeads + h], 0.f);
+    }
+    for (int i = tid; i < kTopkBins; i += kThreads) sm.hist[i] = 0;
+  }
+  fence_proxy_async_shared();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (elect_one()) {
+      int issued = 0;
+      for (int i = 0; i < my_tiles && !sm.abort; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (i >= kStages && !mbar_wait(&sm.empty[s], ph ^ 1)) {
+          record_abort(sm, err, 1);
+          break;
+        }
+        const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
+        mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+        tma_load_2d(sm.keys[s], &tmap, &sm.full[s], 0, (int32_t)((long long)b * a.ik.cap + j0));
+        ++issued;
+      }
+      // never leave while a copy into this CTA's shared memory is in flight
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_wait(&sm.full[i % kStages], (i / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (elect_one()) {
+      int done = 0;
+      for (int i = 0; i < my_tiles && !sm.abort; ++i) {
+        const int s = i % kStages, acc = i % kAcc;
+        if (i >= kAcc && !mbar_wait(&sm.acc_empty[acc], ((i / kAcc) & 1) ^ 1)) {
+          record_abort(sm, err, 2);
+          break;
+        }
+        if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
+          record_abort(sm, err, 2);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ka = smem_addr(sm.keys[s]), qa = smem_addr(sm.q);
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint32_t off = kb * 64 + kk * 32;
+            mma_f8(tmem + acc * 128 + kb * 64, desc_kmajor_sw128(ka + off),
+                   desc_kmajor_sw128(qa + off), kIdesc, kk);
+          }
+        }
+        mma_commit(&sm.empty[s]);
+        mma_commit(&sm.acc_full[acc]);
+        ++done;
+      }
+      // every MMA of this CTA has finished before TMEM is released
+      mma_commit(&sm.mma_done);
+      if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm, err, 4);
+    }
+  } else if (warp >= 4) {
+    // ---------------- epilogue: two warpgroups take alternate tiles
+    const int grp = (warp - 4) >> 2;          // 0 or 1
+    const int quad = warp & 3;                // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;           // entry within the tile
+    float *srow = scores + (size_t)row * ld;
+    const uint8_t *scale_base = reinterpret_cast<const uint8_t *>(a.ik.scale);
+    for (int i = grp; i < my_tiles; i += 2) {
+      const int acc = i % kAcc;
+      const long long j = (long long)(blockIdx.x + i * gridDim.x) * kTile + r;
+      float sk0 = 0.f, sk1 = 0.f;
+      if (j < n) {
+        const float *sp = reinterpret_cast<const float *>(
+            scale_base + ((long long)b * a.ik.cap + j) * a.ik.scale_stride);
+        sk0 = __ldg(sp);
+        sk1 = __ldg(sp + 1);
+      }
+      if (!mbar_wait(&sm.acc_full[acc], (i / kAcc) & 1)) {
+        record_abort(sm, err, 8);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * 128;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float a0[32], a1[32];
+        tmem_ld32(taddr + half * 32, a0);        // block 0, heads 32*half ..
+        tmem_ld32(taddr + 64 + half * 32, a1);   // block 1
+        tmem_wait_ld();
+        if (half == 1) {
+          // both halves are in registers: hand the accumulator slot back
+          tc_fence_before();
+          mbar_arrive(&sm.acc_empty[acc]);
+        }
+#pragma unroll
+        for (int h = 0; h < 32; h += 4) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 c = sm.qc[half * 32 + h + u];
+            const float x = fmaf(a0[h + u] * c.x, sk0, (a1[h + u] * c.y) * sk1);
+            const float t = c.z * fmaxf(x, 0.f);
+            if (u == 0) s0 += t; else if (u == 1) s1 += t; else if (u == 2) s2 += t; else s3 += t;
+          }
+        }
+      }
+      const float sc = (s0 + s1) + (s2 + s3);
+      if (j < n) {
+        srow[j] = sc;
+        atomicAdd(&sm.hist[score_key(sc) >> kTopkShift], 1u);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // fold this CTA's histogram into the row's
+  uint32_t *hg = hist_g + (size_t)row * kTopkBins;
+  for (int i = tid; i < kTopkBins; i += kThreads) {
+    const uint32_t v = sm.hist[i];
+    if (v) atomicAdd(&hg[i], v);
+  }
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool indexer_tc_supported(const IndexerArgs &a) {
+  if (a.ik.fmt != CSKV_FMT_E4M3_BF16 || a.d_I != kDim || a.H_I != kHeads) return false;
+  if ((long long)a.B * a.ik.cap >= (1LL << 31)) return false;
+  if (((uintptr_t)a.ik.data & 15) || (a.ik.data_stride & 15)) return false;
+  if ((uintptr_t)a.q_ik & 15) return false;
+  int dev = 0, major = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  return major == 10 && encode_fn() != nullptr;
+}
+
+int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
+                      int *err, cudaStream_t st) {
+  auto fn = encode_fn();
+  if (!fn) return CSKV_ERR_UNSUPPORTED;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)((long long)a.B * a.ik.cap)};
+  cuuint64_t strides[1] = {(cuuint64_t)a.ik.data_stride};
+  cuuint32_t box[2] = {(cuuint32_t)kDim, (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.ik.data, dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return CSKV_ERR_UNSUPPORTED;
+  const size_t smem = sizeof(Smem) + 1024;
+  if (!ensure_dynamic_smem(indexer_tc_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int rows = a.B * a.Tq;
+  const long long tiles = (a.max_entries + kTile - 1) / kTile;
+  long long splits = (sms + rows - 1) / rows;
+  if (splits > tiles) splits = tiles;
+  if (splits < 1) splits = 1;
+  dim3 grid((unsigned)splits, (unsigned)rows);
+  indexer_tc_kernel<<<grid, kThreads, smem, st>>>(a, map, scores, ld, hist, err);
+  return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 
 }  // namespace cskv

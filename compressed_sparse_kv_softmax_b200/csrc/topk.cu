@@ -5,22 +5,33 @@
 // haben kleine Aenderungen grosse Wirkung», "Komprimierte Erinnerung fuer
 // laengere Kontexte").  Selection here is exact: the k largest scores of the
 // row's visible entries, ties to the lower entry index, written in ascending
-// entry order (deterministic), -1 / -inf padding when fewer than k are visible.
+// entry order, -1 / -inf padding when fewer than k are visible.  Scores are
+// compared through an order-preserving uint32 key.
 //
-// Method: scores are mapped to order-preserving uint32 keys; a 4-pass 8-bit
-// radix select finds the k-th largest key `thr` and how many entries equal
-// to it are taken (`take_eq`); a final pass in index order keeps every key
-// above thr and the first take_eq keys equal to it, placing each at its rank
-// via a block-wide prefix sum.
+// Two kernels:
+//  * topk_rows_kernel - one CTA per row: a 4-pass 8-bit radix select finds
+//    the k-th largest key and how many equal keys to take, then an ordered
+//    compaction in index order writes the result.  Used after the generic
+//    scoring kernel and as the fall-back for pathological rows.
+//  * topk_select_kernel - several CTAs per row, after the tensor-core scoring
+//    kernel has built a histogram of the top 12 key bits:
+//      1. every CTA finds the bucket b* holding the k-th largest key;
+//      2. every CTA scans its slice of the row, appending entries above b*
+//         (sure winners) and entries in b* (candidates);
+//      3. the last CTA to finish (atomic ticket, nobody waits) selects the
+//         missing candidates by the low 20 key bits, breaks exact ties by the
+//         lower index, and sorts the k indices.
+#include <climits>
+
 #include "cskv_internal.cuh"
+#include "topk_common.cuh"
 
 namespace cskv {
 
 namespace {
 
-constexpr int kTopkThreads = 1024;
-
-// exclusive prefix sum over the block; returns the block total in *total
+// exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024);
+// returns the block total in *total
 __device__ __forceinline__ int block_exclusive_scan(int x, int *scratch, int *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = blockDim.x >> 5;
@@ -50,25 +61,14 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *scratch, int *to
   return res;
 }
 
-}  // namespace
-
-// scores: [rows][ld] fp32, n_vis per row from q_pos; out_idx/out_score: [rows][k]
-__global__ void __launch_bounds__(kTopkThreads)
-topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *__restrict__ q_pos,
-                 int stride, long long max_entries, int k, int32_t *__restrict__ out_idx,
-                 float *__restrict__ out_score) {
+// Whole-row exact top-k by one CTA (any blockDim multiple of 32).
+__device__ void topk_row_single_cta(const float *__restrict__ s, long long n, int k,
+                                    int32_t *__restrict__ oi, float *__restrict__ os) {
   __shared__ int hist[256];
   __shared__ int scan_scratch[33];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
-  const int row = blockIdx.x;
   const int tid = threadIdx.x;
-  long long n = (q_pos[row] + 1) / stride;
-  if (n > max_entries) n = max_entries;
-  const float *s = scores + (long long)row * ld;
-  int32_t *oi = out_idx + (long long)row * k;
-  float *os = out_score ? out_score + (long long)row * k : nullptr;
-
   uint32_t thr = 0;
   int take_eq = 0;
   const bool all = n <= k;
@@ -102,8 +102,6 @@ topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *
     thr = prefix;
     take_eq = remaining;
   }
-
-  // ordered compaction in index order
   int base_gt = 0, base_eq = 0;
   for (long long j0 = 0; j0 < n; j0 += blockDim.x) {
     const long long j = j0 + tid;
@@ -135,11 +133,268 @@ topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *
   }
 }
 
+__device__ __forceinline__ long long visible(const int64_t *q_pos, int row, int stride,
+                                             long long max_entries) {
+  long long n = (q_pos[row] + 1) / stride;
+  if (n > max_entries) n = max_entries;
+  return n < 0 ? 0 : n;
+}
+
+// Ascending bitonic sort of v[0..m) in shared memory, m a power of two.
+__device__ void bitonic_sort_smem(int32_t *v, int m) {
+  for (int size = 2; size <= m; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < (m >> 1); i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const int32_t a = v[lo], b = v[hi];
+        if ((a > b) == up) { v[lo] = b; v[hi] = a; }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+constexpr int kSelThreads = 512;
+constexpr int kCandSmem = kCandCap; // candidates the last CTA refines in shared memory
+constexpr int kMaxK = 4096;
+
+struct SelSmem {
+  uint32_t hist[kTopkBins];         // row histogram, later the refine histograms
+  uint32_t ckey[kCandSmem];
+  int32_t cidx[kCandSmem];
+  int32_t out[kMaxK];
+  int scan[33];
+  int bstar, above, is_last, thr2, take_eq, n_eq, fallback;
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(1024)
+topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *__restrict__ q_pos,
+                 int stride, long long max_entries, int k, int32_t *__restrict__ out_idx,
+                 float *__restrict__ out_score) {
+  const int row = blockIdx.x;
+  const long long n = visible(q_pos, row, stride, max_entries);
+  topk_row_single_cta(scores + (long long)row * ld, n, k, out_idx + (long long)row * k,
+                      out_score ? out_score + (long long)row * k : nullptr);
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int stride,
+                   long long max_entries, int k, int32_t *__restrict__ out_idx,
+                   float *__restrict__ out_score) {
+  extern __shared__ __align__(16) uint8_t sel_smem_raw[];
+  SelSmem &sm = *reinterpret_cast<SelSmem *>(sel_smem_raw);
+  const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const long long n = visible(q_pos, row, stride, max_entries);
+  const float *s = w.scores + (long long)row * w.ld;
+  int32_t *oi = out_idx + (long long)row * k;
+  float *os = out_score ? out_score + (long long)row * k : nullptr;
+
+  if (n <= k) {            // every visible entry is selected, already in order
+    if (blockIdx.x == 0) {
+      for (int i = tid; i < k; i += blockDim.x) {
+        oi[i] = i < n ? i : -1;
+        if (os) os[i] = i < n ? s[i] : -__int_as_float(0x7f800000);
+      }
+    }
+    return;
+  }
+
+  if (tid == 0) { sm.bstar = 0; sm.above = -1; }
+  // 1. threshold bucket b*: the bucket holding the k-th largest key
+  const uint32_t *hrow = w.hist + (size_t)row * kTopkBins;
+  constexpr int kPer = kTopkBins / kSelThreads;            // bins per thread, from the top
+  uint32_t local[kPer];
+  int lsum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    local[i] = hrow[kTopkBins - 1 - (tid * kPer + i)];
+    lsum += (int)local[i];
+  }
+  int total;
+  const int before = block_exclusive_scan(lsum, sm.scan, &total);
+  if (before < k && before + lsum >= k) {
+    int cum = before;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      if (cum + (int)local[i] >= k) {
+        sm.bstar = kTopkBins - 1 - (tid * kPer + i);
+        sm.above = cum;
+        break;
+      }
+      cum += (int)local[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t bstar = (uint32_t)sm.bstar;
+  const int above = sm.above;
+
+  // 2. this CTA's slice: sure winners and candidates
+  uint32_t *ctr = w.ctr + (size_t)row * 4;
+  int32_t *selrow = w.sel + (size_t)row * k;
+  int32_t *candrow = w.cand + (size_t)row * kCandCap;
+  const long long per = ((n + gridDim.x - 1) / gridDim.x + 31) & ~31LL;
+  const long long j_lo = (long long)blockIdx.x * per;
+  const long long j_hi = min(n, j_lo + per);
+  for (long long j0 = j_lo; j0 < j_hi; j0 += blockDim.x) {
+    const long long j = j0 + tid;
+    uint32_t bkt = 0;
+    bool valid = j < j_hi;
+    if (valid) bkt = score_key(s[j]) >> kTopkShift;
+    const bool gt = valid && bkt > bstar;
+    const bool eq = valid && bkt == bstar;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const unsigned mg = __ballot_sync(0xffffffffu, gt);
+    const unsigned me = __ballot_sync(0xffffffffu, eq);
+    uint32_t bg = 0, be = 0;
+    if (lane == 0) {
+      if (mg) bg = atomicAdd(&ctr[0], (uint32_t)__popc(mg));
+      if (me) be = atomicAdd(&ctr[1], (uint32_t)__popc(me));
+    }
+    bg = __shfl_sync(0xffffffffu, bg, 0);
+    be = __shfl_sync(0xffffffffu, be, 0);
+    if (gt) {
+      const uint32_t p = bg + __popc(mg & lt_mask);
+      if (p < (uint32_t)k) selrow[p] = (int32_t)j;
+    }
+    if (eq) {
+      const uint32_t p = be + __popc(me & lt_mask);
+      if (p < (uint32_t)kCandCap) candrow[p] = (int32_t)j;
+    }
+  }
+
+  // 3. the last CTA of the row finishes the selection
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sm.is_last = atomicAdd(&ctr[2], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+  const int n_cand = (int)atomicAdd(&ctr[1], 0u);
+  const int r = k - above;                 // candidates still to take, 1 <= r <= n_cand
+  // any inconsistency between the histogram and the scores (never expected)
+  // sends the row to the single-CTA path instead of indexing out of range
+  if (tid == 0)
+    sm.fallback = above < 0 || above >= k || r < 1 || r > n_cand || n_cand > kCandSmem ||
+                  atomicAdd(&ctr[0], 0u) != (uint32_t)above;
+  __syncthreads();
+  if (!sm.fallback) {
+    for (int i = tid; i < n_cand; i += blockDim.x) {
+      const int32_t j = candrow[i];
+      sm.cidx[i] = j;
+      sm.ckey[i] = score_key(s[j]);
+    }
+    // radix select of the r-th largest candidate key on bits 19..10, then 9..0
+    uint32_t prefix = bstar << kTopkShift, mask = 0xFFFu << kTopkShift;
+    int remaining = r;
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = 10 - 10 * pass;
+      for (int i = tid; i < 1024; i += blockDim.x) sm.hist[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < n_cand; i += blockDim.x) {
+        const uint32_t key = sm.ckey[i];
+        if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int cum = 0, bkt = 1023;
+        for (; bkt > 0; --bkt) {
+          if (cum + (int)sm.hist[bkt] >= remaining) break;
+          cum += (int)sm.hist[bkt];
+        }
+        sm.thr2 = (int)(prefix | ((uint32_t)bkt << shift));
+        sm.take_eq = remaining - cum;
+      }
+      __syncthreads();
+      prefix = (uint32_t)sm.thr2;
+      remaining = sm.take_eq;
+      mask |= 1023u << shift;
+      __syncthreads();
+    }
+    const uint32_t thr2 = (uint32_t)sm.thr2;
+    const int take_eq = sm.take_eq;
+    // sure winners, then candidates above thr2, then the take_eq lowest
+    // indices among candidates equal to thr2 (gathered at the end of `out`)
+    for (int i = tid; i < above; i += blockDim.x) sm.out[i] = selrow[i];
+    if (tid == 0) { sm.is_last = 0; sm.n_eq = 0; }
+    __syncthreads();
+    int *cnt_gt = &sm.is_last;     // reuse as a counter
+    for (int i = tid; i < n_cand; i += blockDim.x) {
+      const uint32_t key = sm.ckey[i];
+      if (key > thr2) {
+        const int p = atomicAdd(cnt_gt, 1);
+        if (above + p < k) sm.out[above + p] = sm.cidx[i];
+      }
+    }
+    __syncthreads();
+    const int n_gt = *cnt_gt;                 // == r - take_eq
+    // equal keys: collect into the cand key array (no longer needed)
+    int32_t *eqv = reinterpret_cast<int32_t *>(sm.hist);   // up to kTopkBins entries
+    for (int i = tid; i < n_cand; i += blockDim.x) {
+      if (sm.ckey[i] == thr2) {
+        const int p = atomicAdd(&sm.n_eq, 1);
+        if (p < kTopkBins) eqv[p] = sm.cidx[i];
+      }
+    }
+    __syncthreads();
+    const int n_eq = sm.n_eq;
+    if (n_eq > kTopkBins || above + n_gt + take_eq != k || take_eq > n_eq) {
+      if (tid == 0) sm.fallback = 1;
+    } else {
+      if (n_eq > take_eq) {
+        int m = 1;
+        while (m < n_eq) m <<= 1;
+        for (int i = n_eq + tid; i < m; i += blockDim.x) eqv[i] = INT_MAX;
+        __syncthreads();
+        bitonic_sort_smem(eqv, m);
+      }
+      for (int i = tid; i < take_eq; i += blockDim.x) sm.out[above + n_gt + i] = eqv[i];
+    }
+    __syncthreads();
+    if (!sm.fallback) {
+      int m = 1;
+      while (m < k) m <<= 1;
+      for (int i = k + tid; i < m; i += blockDim.x) sm.out[i] = INT_MAX;
+      __syncthreads();
+      bitonic_sort_smem(sm.out, m);
+      for (int i = tid; i < k; i += blockDim.x) {
+        const int32_t j = sm.out[i];
+        oi[i] = j;
+        if (os) os[i] = s[j];
+      }
+    }
+  }
+  __syncthreads();
+  if (sm.fallback) topk_row_single_cta(s, n, k, oi, os);
+}
+
 void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,
                       long long max_entries, int k, int rows, int32_t *out_idx,
                       float *out_score, cudaStream_t st) {
-  topk_rows_kernel<<<rows, kTopkThreads, 0, st>>>(scores, ld, q_pos, stride, max_entries, k,
-                                                  out_idx, out_score);
+  topk_rows_kernel<<<rows, 1024, 0, st>>>(scores, ld, q_pos, stride, max_entries, k, out_idx,
+                                          out_score);
+}
+
+int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
+                       long long max_entries, int k, int rows, int32_t *out_idx,
+                       float *out_score, cudaStream_t st) {
+  if (k > kMaxK) return CSKV_ERR_UNSUPPORTED;
+  const size_t smem = sizeof(SelSmem);
+  if (!ensure_dynamic_smem(topk_select_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // slices of at least 4096 scores; enough CTAs to cover the SMs at one row
+  long long splits = (max_entries + 4095) / 4096;
+  const long long cap = (sms + rows - 1) / rows;
+  if (splits > cap) splits = cap;
+  if (splits < 1) splits = 1;
+  topk_select_kernel<<<dim3((unsigned)splits, (unsigned)rows), kSelThreads, smem, st>>>(
+      w, q_pos, stride, max_entries, k, out_idx, out_score);
+  return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 
 }  // namespace cskv

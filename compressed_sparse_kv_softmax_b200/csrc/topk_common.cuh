@@ -1,0 +1,56 @@
+// Shared constants of the score histogram the indexer builds for the top-k.
+#pragma once
+
+#include <stdint.h>
+
+namespace cskv {
+
+// Histogram over the top 12 bits of the order-preserving score key (sign,
+// exponent and 3 mantissa bits): 4096 buckets, each 1/8 of an octave wide.
+constexpr int kTopkBins = 4096;
+constexpr int kTopkShift = 20;
+// Candidates (entries inside the threshold bucket) kept per row; the final
+// refinement runs in shared memory up to this count and falls back to the
+// single-CTA selection of the whole row beyond it.
+constexpr int kCandCap = 8192;
+
+// Indexer workspace layout, one section after another, each 256-byte aligned:
+//   err      4 int                 device status words
+//   scores   rows x ld fp32
+//   hist     rows x kTopkBins u32  (zeroed before scoring)
+//   ctr      rows x 4 u32          selected count, candidate count, ticket (zeroed)
+//   sel      rows x k int32        entries above the threshold bucket
+//   cand     rows x kCandCap int32 entries inside the threshold bucket
+struct IndexerWs {
+  int *err;
+  float *scores;
+  uint32_t *hist;
+  uint32_t *ctr;
+  int32_t *sel;
+  int32_t *cand;
+  long long ld;
+  size_t zero_bytes;   // bytes from `hist` that must be zero before the call
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline IndexerWs indexer_ws_layout(void *base, long long rows, long long max_entries, int k,
+                                   size_t *total) {
+  IndexerWs w{};
+  w.ld = (max_entries + 3) & ~3LL;
+  if (w.ld < 4) w.ld = 4;
+  uint8_t *p = static_cast<uint8_t *>(base);
+  size_t off = 0;
+  w.err = reinterpret_cast<int *>(p + off);           off = align256(off + 16);
+  w.scores = reinterpret_cast<float *>(p + off);      off = align256(off + rows * w.ld * 4);
+  const size_t zero_begin = off;
+  w.hist = reinterpret_cast<uint32_t *>(p + off);     off = align256(off + rows * kTopkBins * 4);
+  w.ctr = reinterpret_cast<uint32_t *>(p + off);      off = align256(off + rows * 16);
+  w.zero_bytes = off - zero_begin;
+  w.sel = reinterpret_cast<int32_t *>(p + off);       off = align256(off + rows * (size_t)k * 4);
+  w.cand = reinterpret_cast<int32_t *>(p + off);      off = align256(off + rows * (size_t)kCandCap * 4);
+  if (total) *total = off;
+  return w;
+}
+
+}  // namespace cskv

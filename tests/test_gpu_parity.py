@@ -109,7 +109,8 @@ def test_indexer_topk(C, name):
         assert np.allclose(sc[b, t][: sel.size], rs[sel], rtol=1e-4, atol=1e-4 * np.abs(rs).max())
 
 
-@pytest.mark.parametrize("T,k", [(3, 8), (4, 8), (64, 16), (64, 100), (517, 129)])
+@pytest.mark.parametrize("T,k", [(3, 8), (4, 8), (64, 16), (64, 100), (517, 129), (1000, 100),
+                                 (2100, 500), (40000, 4096)])
 def test_indexer_edge_sizes(C, T, k):
     wl = W.get("parity_decode").with_(T=T, B=2, k=k)
     L = W.make_csa_layer(wl)
