@@ -151,42 +151,56 @@ attn_chunk_kernel(AttnArgs a, int n_comp_chunks, int n_chunks, float *__restrict
 }
 
 // out[row][h][:] = sum_i e^{lse_i - L} o_i,  lse[row][h] = L = log sum_i e^{lse_i}
-__global__ void __launch_bounds__(128)
+// CTA (row * Hq + head, d-block of 128); 4 groups of 128 threads split the chunks,
+// each thread one output dim; a shared-memory sum joins the groups.
+constexpr int kMergeD = 128, kMergeGroups = 4;
+
+__global__ void __launch_bounds__(kMergeD * kMergeGroups)
 attn_merge_kernel(int Hq, int Dv, int n_chunks, const float *__restrict__ part_o,
                   const float *__restrict__ part_lse, float *__restrict__ out,
                   float *__restrict__ lse) {
   extern __shared__ float wts[];          // [n_chunks]
-  const int row = blockIdx.x, h = blockIdx.y;
-  const float *pl = part_lse + (long long)row * n_chunks * Hq + h;
+  __shared__ float red[kMergeGroups][kMergeD];
   __shared__ float s_L;
-  if (threadIdx.x < 32) {
+  const int row = blockIdx.x / Hq, h = blockIdx.x % Hq;
+  const int tid = threadIdx.x, grp = tid / kMergeD, dl = tid % kMergeD;
+  const int d = blockIdx.y * kMergeD + dl;
+  const float *pl = part_lse + (long long)row * n_chunks * Hq + h;
+  for (int i = tid; i < n_chunks; i += blockDim.x) wts[i] = __ldg(pl + (long long)i * Hq);
+  __syncthreads();
+  if (tid < 32) {
     float m = -CUDART_INF_F;
-    for (int i = threadIdx.x; i < n_chunks; i += 32) m = fmaxf(m, pl[(long long)i * Hq]);
+    for (int i = tid; i < n_chunks; i += 32) m = fmaxf(m, wts[i]);
     m = warp_max(m);
     float s = 0.f;
-    for (int i = threadIdx.x; i < n_chunks; i += 32) {
-      const float l = pl[(long long)i * Hq];
-      s += l == -CUDART_INF_F ? 0.f : expf(l - m);
-    }
+    for (int i = tid; i < n_chunks; i += 32) s += wts[i] == -CUDART_INF_F ? 0.f : expf(wts[i] - m);
     s = warp_sum(s);
     const float L = m + logf(s);
-    for (int i = threadIdx.x; i < n_chunks; i += 32) {
-      const float l = pl[(long long)i * Hq];
-      wts[i] = l == -CUDART_INF_F ? 0.f : expf(l - L);
-    }
-    if (threadIdx.x == 0) s_L = L;
+    __syncwarp();
+    for (int i = tid; i < n_chunks; i += 32)
+      wts[i] = wts[i] == -CUDART_INF_F ? 0.f : expf(wts[i] - L);
+    if (tid == 0) s_L = L;
   }
   __syncthreads();
-  const float *po = part_o + (long long)row * n_chunks * Hq * Dv + (long long)h * Dv;
-  for (int d = threadIdx.x; d < Dv; d += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < n_chunks; ++i) {
+  float acc = 0.f;
+  if (d < Dv) {
+    const float *po = part_o + (long long)row * n_chunks * Hq * Dv + (long long)h * Dv + d;
+    const long long cstride = (long long)Hq * Dv;
+#pragma unroll 8
+    for (int i = grp; i < n_chunks; i += kMergeGroups) {
       const float w = wts[i];
-      if (w != 0.f) acc = fmaf(w, po[(long long)i * Hq * Dv + d], acc);
+      if (w != 0.f) acc = fmaf(w, __ldg(po + i * cstride), acc);
     }
-    out[((long long)row * Hq + h) * Dv + d] = acc;
   }
-  if (threadIdx.x == 0) lse[(long long)row * Hq + h] = s_L;
+  red[grp][dl] = acc;
+  __syncthreads();
+  if (grp == 0 && d < Dv) {
+    float t = red[0][dl];
+#pragma unroll
+    for (int g = 1; g < kMergeGroups; ++g) t += red[g][dl];
+    out[((long long)row * Hq + h) * Dv + d] = t;
+  }
+  if (blockIdx.y == 0 && tid == 0) lse[(long long)row * Hq + h] = s_L;
 }
 
 int chunk_keys(const AttnArgs &a) { return attn_tc_supported(a) ? attn_tc_chunk_keys() : kChunk; }
@@ -228,8 +242,10 @@ int launch_attention(const AttnArgs &a, cudaStream_t st) {
     attn_chunk_kernel<<<dim3(nc, rows), kThreads, smem, st>>>(a, ncc, nc, part_o, part_lse);
     if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
   }
-  attn_merge_kernel<<<dim3(rows, a.Hq), 128, sizeof(float) * nc, st>>>(
-      a.Hq, a.Dv, nc, part_o, part_lse, a.out, a.lse);
+  const size_t msmem = sizeof(float) * nc;
+  if (!ensure_dynamic_smem(attn_merge_kernel, msmem)) return CSKV_ERR_UNSUPPORTED;
+  attn_merge_kernel<<<dim3((unsigned)(rows * a.Hq), (a.Dv + kMergeD - 1) / kMergeD), kMergeD * kMergeGroups,
+                      msmem, st>>>(a.Hq, a.Dv, nc, part_o, part_lse, a.out, a.lse);
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 

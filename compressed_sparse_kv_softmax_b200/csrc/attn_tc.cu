@@ -1,15 +1,442 @@
-// Tensor-core (tcgen05) hybrid attention for the 64-head x 512-dim FP8+BF16 layout.
+// Hybrid attention on the 5th-generation tensor cores (tcgen05) for the MQA
+// layout with 64 query heads over one 512-dim FP8+BF16 KV entry (K = V).
+//
+// CSA attends its selected entries, HCA every compressed entry, both plus the
+// raw 128-token window («DeepSeek-V4: 1 Million Token Context endlich
+// nutzbar», "Hybrid Attention: CSA und HCA»; «Chinas KI-Unabhaengigkeit?: Bei
+// Deepseek V4 haben kleine Aenderungen grosse Wirkung», "Komprimierte
+// Erinnerung fuer laengere Kontexte").  The cache stores 448 dims as E4M3 with
+// one fp32 scale per 64 dims and the last 64 dims as BF16.
+//
+// One CTA computes the partial softmax (o, lse) of one query row over one
+// unit of at most 64 keys of the row's key list (compressed part first, then
+// the window); attn_merge_kernel combines the units through log-sum-exp.
+//
+// Precision: the outputs must agree with float64 to 2e-3 of the output's RMS,
+// which is ~0.1 while single values of V are O(1): a few units in 2^-14.  A
+// single FP16 rounding of K, V or P alone already misses that, so every
+// tensor-core operand that is not exact in FP16 is split into two FP16 terms,
+// x = hi + lo with hi = fp16(x), lo = fp16(x - hi) (about 22 bits together):
+//   S = K_hi Q^T + K_lo Q^T           (Q is BF16, exact in FP16)
+//   O = V_hi P_hi + V_lo P_hi + V_hi P_lo   (V = K; the lo x lo term is 2^-22)
+// with fp32 accumulation in TMEM.
+//
+//   1. gather: each warp converts 8 keys per batch (all loads first); lanes
+//      0-27 take 16 FP8 codes each (x block scale), lanes 28-31 16 BF16 RoPE
+//      values each; hi and lo parts land in two K-major 128-byte-swizzled
+//      tiles [8 chunks of 64 dims][64 keys][128 B].  Q becomes FP16 in the
+//      same layout [8 chunks][64 heads][128 B].
+//   2. S^T with keys on the MMA M axis (M = 128, rows 64..127 masked;
+//      N = 64 heads; K = 512 in 32 steps per part), fp32 in TMEM cols 0..63.
+//   3. softmax over keys per head: each thread owns one key row; a warp
+//      reduce-scatter butterfly (32+16+8+4+2 shuffles) leaves lane L with
+//      heads 2L, 2L+1 over the warp's keys, shared memory joins the warps.
+//      P = exp2(S * scale * log2 e - m) goes as hi/lo MN-major tiles
+//      [keys][64 heads]; the per-head sums use the same butterfly.
+//   4. O^T = V^T P^T reading the key tiles MN-major (M = 128 dims x 4,
+//      N = 64 heads, K = keys), fp32 in TMEM columns 64..319.
+//   5. each thread owns one dim: o[h][d] / l_h and lse_h = ln2 (m_h + log2 l_h)
+//      go to the partial buffers.
+#include <math_constants.h>
+
 #include "cskv_internal.cuh"
+#include "sm100.cuh"
 
 namespace cskv {
 
-bool attn_tc_supported(const AttnArgs &a) { (void)a; return false; }
-int attn_tc_chunk_keys() { return 128; }
+namespace {
+
+using namespace sm100;
+
+constexpr int kHeads = 64, kD = 512, kDn = 448, kDr = 64;
+constexpr int kKeys = 64;                          // keys per unit (valid MMA rows)
+constexpr int kM = 128;                            // MMA M (rows kKeys..127 are masked)
+constexpr int kThreads = 128;
+constexpr uint32_t kChunkK = kKeys * 128;          // bytes per 64-dim chunk of a key tile
+constexpr uint32_t kChunkQ = kHeads * 128;         // bytes per 64-dim chunk of Q
+constexpr uint32_t kIdescQK = idesc(kFmtF16, kFmtF16, 0, 0, kM, kHeads);
+constexpr uint32_t kIdescPV = idesc(kFmtF16, kFmtF16, 1, 1, 128, kHeads);
+
+struct __align__(1024) Smem {
+  // key tiles, hi and lo parts (K-major view: K; MN-major view: V^T).  An
+  // M = 128 read of a chunk runs 64 rows into the next buffer: masked rows.
+  uint8_t khi[8 * kChunkK];         // 64 KB
+  uint8_t klo[8 * kChunkK];         // 64 KB
+  uint8_t q[8 * kChunkQ];           // 64 KB
+  uint8_t phi[kKeys * 128];         // 8 KB: P^T hi, MN-major [keys][64 heads]
+  uint8_t plo[kKeys * 128];         // 8 KB
+  float red[4][kHeads];
+  float m[kHeads], l[kHeads];
+  long long slot[kM];
+  uint64_t bar;
+  uint32_t tmem_base;
+};
+
+// byte offset of 16-byte unit u of row r in a 128-byte-swizzled K-major
+// chunk (8-row atoms of 1024 bytes)
+__device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t u) {
+  return r * 128u + ((u ^ (r & 7u)) << 4);
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// split two fp32 values into FP16 hi and lo parts (x = hi + lo to ~2^-22)
+__device__ __forceinline__ void split_h2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// Warp reduce-scatter of 64 per-lane values: afterwards lane L holds the
+// combination over the warp of values 2L and 2L+1 (in out[0], out[1]).
+template <bool kMax>
+__device__ __forceinline__ void butterfly64(float (&v)[64], float &o0, float &o1) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int step = 0; step < 5; ++step) {
+    const int half = 32 >> step;             // values kept after this step
+    const int bit = 16 >> step;              // partner lane distance
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = upper ? v[i + half] : v[i];
+      const float send = upper ? v[i] : v[i + half];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, bit);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  o0 = v[0];
+  o1 = v[1];
+}
+
+struct Row {
+  long long pos, n_comp, w_lo;
+  int n_win;
+};
+
+__device__ __forceinline__ Row row_of(const AttnArgs &a, int row) {
+  Row r;
+  const int b = row / a.Tq;
+  r.pos = a.pos_is_ctx_len ? a.pos[b] - 1 : a.pos[row];
+  if (!a.has_comp) r.n_comp = 0;
+  else if (a.sel) r.n_comp = a.k;
+  else {
+    const long long n = (r.pos + 1) / a.comp_stride;
+    r.n_comp = n < a.max_entries ? n : a.max_entries;
+  }
+  r.w_lo = r.pos - a.window + 1;
+  if (r.w_lo < 0) r.w_lo = 0;
+  r.n_win = (int)(r.pos - r.w_lo + 1);
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
+               float *__restrict__ part_o, float *__restrict__ part_lse) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                       ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.y, unit = blockIdx.x;
+  const int b = row / a.Tq;
+  const Row R = row_of(a, row);
+
+  if (tid == 0) {
+    mbar_init(&sm.bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+
+  // ---- Q: BF16 -> FP16, K-major swizzled
+  {
+    const __nv_bfloat16 *qg =
+        reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD;
+    // 32 16-byte units per thread, loaded 16 at a time before any is used
+    constexpr int kPer = kHeads * kD / 8 / kThreads, kBatch = 16;
+#pragma unroll
+    for (int i0 = 0; i0 < kPer; i0 += kBatch) {
+      uint4 raw[kBatch];
+#pragma unroll
+      for (int e = 0; e < kBatch; ++e) {
+        const int i = tid + (i0 + e) * kThreads;
+        raw[e] = __ldg(reinterpret_cast<const uint4 *>(qg) + i);
+      }
+#pragma unroll
+      for (int e = 0; e < kBatch; ++e) {
+        const int i = tid + (i0 + e) * kThreads;
+        const int h = i >> 6, c = (i >> 3) & 7, u = i & 7;  // 8 dims per unit
+        const __nv_bfloat162 *bp = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
+        uint4 o;
+        uint32_t *op = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(bp[q]);
+          op[q] = pack_h2(f.x, f.y);
+        }
+        *reinterpret_cast<uint4 *>(sm.q + c * kChunkQ + swz(h, u)) = o;
+      }
+    }
+  }
+
+  // ---- resolve this unit's key slots (one per thread), then gather
+  const bool comp_unit = unit < n_comp_units;
+  const long long base = comp_unit ? (long long)unit * unit_keys
+                                   : (long long)(unit - n_comp_units) * unit_keys;
+  const long long avail = comp_unit ? R.n_comp - base : (long long)R.n_win - base;
+  const int nkeys = (int)(avail < 0 ? 0 : (avail < unit_keys ? avail : unit_keys));
+  const int ksteps = (nkeys + 15) >> 4;            // 16-key MMA steps of the P V product
+  const Cache &src = comp_unit ? a.comp_k : a.win_k;
+  {
+    long long slot = -1;
+    if (tid < nkeys) {          // nkeys <= kKeys: rows kKeys..kM-1 stay invalid
+      const long long i = base + tid;
+      if (comp_unit) {
+        const long long j = a.sel ? (long long)a.sel[(long long)row * a.k + i] : i;
+        if (j >= 0 && j < src.cap) slot = j;
+      } else {
+        slot = src.slot_of(R.w_lo + i);
+      }
+    }
+    sm.slot[tid] = slot;
+  }
+  // (the barrier also publishes the slots) any key at all in this unit?
+  const bool any = __syncthreads_or(sm.slot[tid] >= 0) != 0;
+  const bool my_valid = sm.slot[tid] >= 0;          // validity of key row `tid`
+  // each warp converts 8 consecutive key rows per batch, loads first
+  for (int r0 = warp * 8; r0 < ksteps * 16; r0 += 32) {
+    uint4 raw[8], raw2[8];
+    float sc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const long long slot = sm.slot[r0 + e];
+      raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
+      sc[e] = 0.f;
+      if (slot < 0) continue;
+      if (lane < 28) {
+        raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
+        sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
+      } else {
+        const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
+        raw[e] = __ldg(rp);
+        raw2[e] = __ldg(rp + 1);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int r = r0 + e;
+      uint4 h0, h1, l0, l1;
+      uint32_t *ph0 = reinterpret_cast<uint32_t *>(&h0), *ph1 = reinterpret_cast<uint32_t *>(&h1);
+      uint32_t *pl0 = reinterpret_cast<uint32_t *>(&l0), *pl1 = reinterpret_cast<uint32_t *>(&l1);
+      int d0;
+      if (lane < 28) {
+        // 16 FP8 codes: dims 16*lane .. +15, block scale lane/4 (absent key: zeros)
+        const uint8_t *cb = reinterpret_cast<const uint8_t *>(&raw[e]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          split_h2(e4m3_decode(cb[2 * q]) * sc[e], e4m3_decode(cb[2 * q + 1]) * sc[e], ph0[q],
+                   pl0[q]);
+          split_h2(e4m3_decode(cb[8 + 2 * q]) * sc[e], e4m3_decode(cb[8 + 2 * q + 1]) * sc[e],
+                   ph1[q], pl1[q]);
+        }
+        d0 = lane * 16;
+      } else {
+        // 16 BF16 RoPE dims: 448 + 16 * (lane - 28) ..
+        const __nv_bfloat162 *b0 = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
+        const __nv_bfloat162 *b1 = reinterpret_cast<const __nv_bfloat162 *>(&raw2[e]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f0 = __bfloat1622float2(b0[q]), f1 = __bfloat1622float2(b1[q]);
+          split_h2(f0.x, f0.y, ph0[q], pl0[q]);
+          split_h2(f1.x, f1.y, ph1[q], pl1[q]);
+        }
+        d0 = kDn + (lane - 28) * 16;
+      }
+      const int c = d0 >> 6, u = (d0 & 63) >> 3;
+      const uint32_t o0 = c * kChunkK + swz(r, u), o1 = c * kChunkK + swz(r, u + 1);
+      *reinterpret_cast<uint4 *>(sm.khi + o0) = h0;
+      *reinterpret_cast<uint4 *>(sm.khi + o1) = h1;
+      *reinterpret_cast<uint4 *>(sm.klo + o0) = l0;
+      *reinterpret_cast<uint4 *>(sm.klo + o1) = l1;
+    }
+  }
+  fence_proxy_async_shared();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  float *po = part_o + ((size_t)row * n_units + unit) * kHeads * kD;
+  float *pl = part_lse + ((size_t)row * n_units + unit) * kHeads;
+
+  if (!any) {
+    // no key in this unit: a partial that the merge weighs with zero
+    for (int i = tid; i < kHeads * kD; i += kThreads) po[i] = 0.f;
+    if (tid < kHeads) pl[tid] = -CUDART_INF_F;
+  } else {
+    // ---- S^T = K Q^T
+    if (tid == 0) {
+      const uint32_t qa = smem_addr(sm.q);
+      for (int part = 0; part < 2; ++part) {          // K_hi Q^T, then + K_lo Q^T
+        const uint32_t ka = smem_addr(part ? sm.klo : sm.khi);
+#pragma unroll 4
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t off = (ks & 3) << 5;         // 16 dims = 32 bytes per step
+          mma_f16(tmem, desc_kmajor_sw128(ka + (ks >> 2) * kChunkK + off),
+                  desc_kmajor_sw128(qa + (ks >> 2) * kChunkQ + off), kIdescQK,
+                  (part | ks) != 0);
+        }
+      }
+      mma_commit(&sm.bar);
+    }
+    bool ok = mbar_wait(&sm.bar, 0);
+    tc_fence_after();
+    // ---- softmax over keys, per head
+    float s[64];
+    {
+      float t[32];
+      const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
+      tmem_ld32(ta, t);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] = t[i];
+      tmem_ld32(ta + 32, t);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[32 + i] = t[i];
+      tmem_wait_ld();
+    }
+    const float c2 = a.sm_scale * 1.4426950408889634f;   // logits in log2 units
+#pragma unroll
+    for (int i = 0; i < 64; ++i) s[i] = my_valid ? s[i] * c2 : -CUDART_INF_F;
+    {
+      float v[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) v[i] = s[i];
+      float m0, m1;
+      butterfly64<true>(v, m0, m1);
+      sm.red[warp][2 * lane] = m0;
+      sm.red[warp][2 * lane + 1] = m1;
+    }
+    __syncthreads();
+    if (tid < kHeads)
+      sm.m[tid] = fmaxf(fmaxf(sm.red[0][tid], sm.red[1][tid]), fmaxf(sm.red[2][tid], sm.red[3][tid]));
+    __syncthreads();
+    {
+      float v[64];
+#pragma unroll
+      for (int h = 0; h < 64; h += 8) {
+        uint4 wh, wl;
+        uint32_t *whp = reinterpret_cast<uint32_t *>(&wh), *wlp = reinterpret_cast<uint32_t *>(&wl);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int hh = h + 2 * e;
+          const float p0 = my_valid ? exp2f(s[hh] - sm.m[hh]) : 0.f;
+          const float p1 = my_valid ? exp2f(s[hh + 1] - sm.m[hh + 1]) : 0.f;
+          split_h2(p0, p1, whp[e], wlp[e]);
+          v[hh] = p0;
+          v[hh + 1] = p1;
+        }
+        if (tid < kKeys) {
+          *reinterpret_cast<uint4 *>(sm.phi + swz(tid, h >> 3)) = wh;
+          *reinterpret_cast<uint4 *>(sm.plo + swz(tid, h >> 3)) = wl;
+        }
+      }
+      float l0, l1;
+      butterfly64<false>(v, l0, l1);
+      sm.red[warp][2 * lane] = l0;
+      sm.red[warp][2 * lane + 1] = l1;
+    }
+    fence_proxy_async_shared();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid < kHeads) sm.l[tid] = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
+    // ---- O^T = V^T P^T
+    if (tid == 0) {
+      const uint32_t vh = smem_addr(sm.khi), vl = smem_addr(sm.klo);
+      const uint32_t ph = smem_addr(sm.phi), pl = smem_addr(sm.plo);
+      for (int mt = 0; mt < 4; ++mt) {
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint32_t voff = (2 * mt) * kChunkK + ks * 2048, poff = ks * 2048;
+          const uint32_t d = tmem + 64 + mt * 64;
+          // V_hi P_hi + V_lo P_hi + V_hi P_lo
+          mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkK, 1024),
+                  desc_mnmajor_sw128(ph + poff, kChunkK, 1024), kIdescPV, ks > 0);
+          mma_f16(d, desc_mnmajor_sw128(vl + voff, kChunkK, 1024),
+                  desc_mnmajor_sw128(ph + poff, kChunkK, 1024), kIdescPV, 1);
+          mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkK, 1024),
+                  desc_mnmajor_sw128(pl + poff, kChunkK, 1024), kIdescPV, 1);
+        }
+      }
+      mma_commit(&sm.bar);
+    }
+    ok = mbar_wait(&sm.bar, 1) && ok;
+    tc_fence_after();
+    __syncthreads();
+    // ---- epilogue: thread = dim within each 128-dim tile
+    const float inv_ln = 0.6931471805599453f;
+    if (tid < kHeads) pl[tid] = ok ? (sm.m[tid] + log2f(sm.l[tid])) * inv_ln : CUDART_NAN_F;
+    for (int mt = 0; mt < 4; ++mt) {
+      const int d = mt * 128 + tid;
+      const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + 64 + mt * 64;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float o[32];
+        tmem_ld32(ta + half * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int h = half * 32 + i;
+          po[(size_t)h * kD + d] = o[i] / sm.l[h];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool attn_tc_supported(const AttnArgs &a) {
+  if (a.win_k.fmt != CSKV_FMT_E4M3_BF16 || a.win_v.data) return false;
+  if (a.Hq != kHeads || a.D != kD || a.Dv != kD) return false;
+  if (a.win_k.d_nope != kDn || a.win_k.d_rope != kDr) return false;
+  auto aligned = [](const Cache &c) {
+    return !(((uintptr_t)c.data | (uintptr_t)c.rope | (uintptr_t)c.data_stride |
+              (uintptr_t)c.rope_stride) & 15) &&
+           !(((uintptr_t)c.scale | (uintptr_t)c.scale_stride) & 3);
+  };
+  if (!aligned(a.win_k) || (a.has_comp && !aligned(a.comp_k))) return false;
+  if ((uintptr_t)a.q & 15) return false;
+  int dev = 0, major = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  return major == 10;
+}
+
+int attn_tc_chunk_keys() { return kKeys; }
 
 int launch_attn_tc(const AttnArgs &a, float *part_o, float *part_lse, int n_chunks,
                    cudaStream_t st) {
-  (void)a; (void)part_o; (void)part_lse; (void)n_chunks; (void)st;
-  return CSKV_ERR_UNSUPPORTED;
+  const long long max_comp = a.has_comp ? (a.sel ? a.k : a.max_entries) : 0;
+  const int ncc = (int)((max_comp + kKeys - 1) / kKeys);
+  if (n_chunks != ncc + (a.window + kKeys - 1) / kKeys) return CSKV_ERR_ARG;
+  const size_t smem = sizeof(Smem) + 1024;
+  if (!ensure_dynamic_smem(attn_tc_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+  const int rows = a.B * a.Tq;
+  attn_tc_kernel<<<dim3((unsigned)n_chunks, (unsigned)rows), kThreads, smem, st>>>(
+      a, kKeys, ncc, n_chunks, part_o, part_lse);
+  return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 
 }  // namespace cskv

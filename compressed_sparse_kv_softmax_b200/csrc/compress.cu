@@ -11,9 +11,13 @@
 // Detail», "Kompression und Selektion".)
 //
 // One CTA per (new entry, sequence).  The work is a few KB per entry and runs
-// once per 4 (CSA) or 128 (HCA) tokens, so the kernel is written for clarity:
-// one warp per slot for the gate dot products, one thread per dim for the
-// pooled sums, one warp per 64-element block for the re-quantisation.
+// once per 4 (CSA) or 128 (HCA) tokens.  At decode a single entry is written,
+// so the latency of the loads decides the time: the staged kernel copies the
+// whole pooling window into shared memory with one round of 16-byte loads,
+// then computes the gates (one warp per slot), the pooled sums (one thread
+// per dim) and the re-quantisation (one warp per 64-element block) from
+// shared memory.  Windows too large for shared memory use compress_kernel,
+// which reads global memory directly.
 #include <math_constants.h>
 
 #include "cskv_internal.cuh"
@@ -127,6 +131,171 @@ compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__
   }
 }
 
+// ---------------------------------------------------------------------------
+// Shared-memory variant: the whole pooling window of every plane is first
+// copied into shared memory with 16-byte loads issued by all threads at once,
+// then the gates and pooled sums read shared memory only.
+
+struct SlotLayout {       // bytes of one staged slot and the offsets of its parts
+  int data_bytes, scale_off, rope_off, bytes;
+};
+
+__host__ __device__ inline int round16(int x) { return (x + 15) & ~15; }
+
+__host__ __device__ inline SlotLayout slot_layout(const Cache &c) {
+  SlotLayout l;
+  if (c.fmt == CSKV_FMT_F32) {
+    l.data_bytes = 4 * c.dims();
+    l.scale_off = l.rope_off = l.bytes = round16(l.data_bytes);
+    return l;
+  }
+  l.data_bytes = c.d_nope;
+  l.scale_off = round16(c.d_nope);
+  l.rope_off = l.scale_off + round16(4 * (c.d_nope >> 6));
+  l.bytes = l.rope_off + round16(2 * c.d_rope);
+  return l;
+}
+
+// asynchronous global -> shared copies (no register round trip), so every
+// copy a thread issues is in flight at once; completed by cp.async.wait_all
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// copy n bytes (a multiple of 4) from global to shared memory, 16 bytes at a
+// time when both ends allow it
+__device__ inline void stage_bytes(uint8_t *dst, const uint8_t *src, int n, int t, int nt) {
+  if ((((uintptr_t)src | (uintptr_t)dst) & 15) == 0 && (n & 15) == 0) {
+    for (int i = t; i < (n >> 4); i += nt) cp_async16(dst + 16 * i, src + 16 * i);
+  } else {
+    for (int i = t; i < (n >> 2); i += nt) cp_async4(dst + 4 * i, src + 4 * i);
+  }
+}
+
+// stage `pool` slots of plane set `c` for positions first .. first+pool-1
+__device__ void stage_window(const Cache &c, const SlotLayout &l, int b, long long first,
+                             int pool, uint8_t *buf) {
+  const int nt = blockDim.x;
+  for (int r = 0; r < pool; ++r) {
+    const long long p = first + r;
+    if (p < 0) continue;
+    const long long slot = c.slot_of(p);
+    uint8_t *dst = buf + (size_t)r * l.bytes;
+    stage_bytes(dst, c.data + c.row(b, slot) * c.data_stride, l.data_bytes, threadIdx.x, nt);
+    if (c.fmt != CSKV_FMT_F32) {
+      stage_bytes(dst + l.scale_off, c.scale + c.row(b, slot) * c.scale_stride,
+                  4 * (c.d_nope >> 6), threadIdx.x, nt);
+      if (c.d_rope)
+        stage_bytes(dst + l.rope_off, c.rope + c.row(b, slot) * c.rope_stride, 2 * c.d_rope,
+                    threadIdx.x, nt);
+    }
+  }
+}
+
+__device__ __forceinline__ float staged_value(const Cache &c, const SlotLayout &l,
+                                              const uint8_t *slot, int d) {
+  if (c.fmt == CSKV_FMT_F32) return reinterpret_cast<const float *>(slot)[d];
+  if (d < c.d_nope)
+    return e4m3_decode(slot[d]) * reinterpret_cast<const float *>(slot + l.scale_off)[d >> 6];
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(slot + l.rope_off)[d - c.d_nope]);
+}
+
+__device__ void pool_staged(const Cache &c, const SlotLayout &l, const uint8_t *buf,
+                            long long first, int pool, const float *a, float *pooled) {
+  const int D = c.dims();
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < pool; ++r) {
+      if (first + r < 0) continue;
+      acc = fmaf(a[r], staged_value(c, l, buf + (size_t)r * l.bytes, d), acc);
+    }
+    pooled[d] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__ t_end,
+                       Cache raw_k, Cache raw_v, Cache raw_ik, const float *__restrict__ gate_w,
+                       const float *__restrict__ gate_b, int pool, int stride, Cache out_k,
+                       Cache out_v, Cache out_ik) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  const int b = blockIdx.y;
+  const long long j = t_begin[b] / stride + blockIdx.x;
+  if (j >= t_end[b] / stride || j < 0) return;
+  if (j >= out_k.cap || (raw_v.data && j >= out_v.cap) || (raw_ik.data && j >= out_ik.cap))
+    return;
+  const long long first = (long long)stride * (j + 1) - pool;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const SlotLayout lk = slot_layout(raw_k);
+  const SlotLayout lv = raw_v.data ? slot_layout(raw_v) : lk;
+  const SlotLayout li = raw_ik.data ? slot_layout(raw_ik) : lk;
+  uint8_t *bk = csm;
+  uint8_t *bv = bk + (size_t)pool * lk.bytes;
+  uint8_t *bi = bv + (raw_v.data ? (size_t)pool * lv.bytes : 0);
+  float *a = reinterpret_cast<float *>(bi + (raw_ik.data ? (size_t)pool * li.bytes : 0));
+  float *pooled = a + pool;
+  const int D = raw_k.dims();
+
+  stage_window(raw_k, lk, b, first, pool, bk);
+  if (raw_v.data) stage_window(raw_v, lv, b, first, pool, bv);
+  if (raw_ik.data) stage_window(raw_ik, li, b, first, pool, bi);
+  cp_async_wait_all();
+  __syncthreads();
+
+  // gate logits g_r = gate_w . k_{p_r} + gate_b[r]
+  for (int r = warp; r < pool; r += kWarps) {
+    const long long p = first + r;
+    float acc = 0.f;
+    if (p >= 0) {
+      const uint8_t *slot = bk + (size_t)r * lk.bytes;
+      for (int d = lane; d < D; d += 32) acc = fmaf(__ldg(gate_w + d), staged_value(raw_k, lk, slot, d), acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) a[r] = p >= 0 ? acc + gate_b[r] : -CUDART_INF_F;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float m = -CUDART_INF_F;
+    for (int r = lane; r < pool; r += 32) m = fmaxf(m, a[r]);
+    m = warp_max(m);
+    float s = 0.f;
+    for (int r = lane; r < pool; r += 32) s += (a[r] == -CUDART_INF_F) ? 0.f : expf(a[r] - m);
+    s = warp_sum(s);
+    __syncwarp();
+    for (int r = lane; r < pool; r += 32)
+      a[r] = (a[r] == -CUDART_INF_F) ? 0.f : expf(a[r] - m) / s;
+  }
+  __syncthreads();
+
+  pool_staged(raw_k, lk, bk, first, pool, a, pooled);
+  __syncthreads();
+  store_entry(out_k, b, j, pooled, D);
+  __syncthreads();
+  if (raw_v.data) {
+    pool_staged(raw_v, lv, bv, first, pool, a, pooled);
+    __syncthreads();
+    store_entry(out_v, b, j, pooled, raw_v.dims());
+    __syncthreads();
+  }
+  if (raw_ik.data) {
+    pool_staged(raw_ik, li, bi, first, pool, a, pooled);
+    __syncthreads();
+    store_entry(out_ik, b, j, pooled, raw_ik.dims());
+  }
+}
+
 }  // namespace
 
 int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
@@ -138,10 +307,19 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
   int dmax = raw_k.dims();
   if (raw_v.data && raw_v.dims() > dmax) dmax = raw_v.dims();
   if (raw_ik.data && raw_ik.dims() > dmax) dmax = raw_ik.dims();
-  const size_t smem = sizeof(float) * (size_t)(pool + dmax);
   dim3 grid((unsigned)max_new, (unsigned)B);
-  compress_kernel<<<grid, kThreads, smem, st>>>(t_begin, t_end, raw_k, raw_v, raw_ik, gate_w,
-                                                gate_b, pool, stride, out_k, out_v, out_ik);
+  size_t staged = (size_t)pool * slot_layout(raw_k).bytes;
+  if (raw_v.data) staged += (size_t)pool * slot_layout(raw_v).bytes;
+  if (raw_ik.data) staged += (size_t)pool * slot_layout(raw_ik).bytes;
+  const size_t smem_staged = staged + sizeof(float) * (size_t)(pool + dmax);
+  if (smem_staged <= 200 * 1024 && ensure_dynamic_smem(compress_staged_kernel, smem_staged)) {
+    compress_staged_kernel<<<grid, kThreads, smem_staged, st>>>(
+        t_begin, t_end, raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride, out_k, out_v, out_ik);
+  } else {
+    const size_t smem = sizeof(float) * (size_t)(pool + dmax);
+    compress_kernel<<<grid, kThreads, smem, st>>>(t_begin, t_end, raw_k, raw_v, raw_ik, gate_w,
+                                                  gate_b, pool, stride, out_k, out_v, out_ik);
+  }
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 

@@ -89,7 +89,7 @@ int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
   const IndexerWs w = indexer_ws_layout(a.ws, rows, a.max_entries, a.k, nullptr);
   if (a.max_entries > 0 && indexer_tc_supported(a)) {
     // tensor-core scoring builds the score histogram the multi-CTA selection uses
-    if (cudaMemsetAsync(w.hist, 0, w.zero_bytes, st) != cudaSuccess) return CSKV_ERR_CUDA;
+    if (cudaMemsetAsync(w.err, 0, w.zero_bytes, st) != cudaSuccess) return CSKV_ERR_CUDA;
     int rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
     if (rc != CSKV_OK) return rc;
     return launch_topk_select(w, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,

@@ -61,13 +61,43 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *scratch, int *to
   return res;
 }
 
+// Bins are counts of keys sharing a digit; this finds the bin holding the
+// `target`-th largest key: scanning bins from the top (bin nbins-1 down), the
+// first bin at which the running count reaches `target`.  Thread t owns
+// `per` consecutive bins from the top; a block-wide prefix sum of the owners'
+// totals locates the owner, which walks its own bins.  Results land in
+// *out_bin and *out_above (count of keys in higher bins); every thread must
+// call it, and it ends with a block barrier.
+template <typename Bins>
+__device__ void find_threshold_bin(const Bins &bins, int nbins, int target, int *scan_scratch,
+                                   int *out_bin, int *out_above) {
+  const int per = (nbins + blockDim.x - 1) / blockDim.x;
+  const int top = nbins - 1 - (int)threadIdx.x * per;
+  int lsum = 0;
+  for (int i = 0; i < per; ++i)
+    if (top - i >= 0) lsum += (int)bins(top - i);
+  int total;
+  const int before = block_exclusive_scan(lsum, scan_scratch, &total);
+  if (before < target && before + lsum >= target) {
+    int cum = before;
+    for (int i = 0; i < per && top - i >= 0; ++i) {
+      const int c = (int)bins(top - i);
+      if (cum + c >= target) {
+        *out_bin = top - i;
+        *out_above = cum;
+        break;
+      }
+      cum += c;
+    }
+  }
+  __syncthreads();
+}
+
 // Whole-row exact top-k by one CTA (any blockDim multiple of 32).
 __device__ void topk_row_single_cta(const float *__restrict__ s, long long n, int k,
                                     int32_t *__restrict__ oi, float *__restrict__ os) {
   __shared__ int hist[256];
   __shared__ int scan_scratch[33];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_remaining;
   const int tid = threadIdx.x;
   uint32_t thr = 0;
   int take_eq = 0;
@@ -84,18 +114,12 @@ __device__ void topk_row_single_cta(const float *__restrict__ s, long long n, in
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
       }
       __syncthreads();
-      if (tid == 0) {
-        int cum = 0, bkt = 255;
-        for (; bkt > 0; --bkt) {
-          if (cum + hist[bkt] >= remaining) break;
-          cum += hist[bkt];
-        }
-        s_prefix = prefix | ((uint32_t)bkt << shift);
-        s_remaining = remaining - cum;
-      }
-      __syncthreads();
-      prefix = s_prefix;
-      remaining = s_remaining;
+      __shared__ int s_bin, s_above;
+      if (tid == 0) { s_bin = 0; s_above = 0; }
+      find_threshold_bin([&](int i) { return hist[i]; }, 256, remaining, scan_scratch, &s_bin,
+                         &s_above);
+      prefix = prefix | ((uint32_t)s_bin << shift);
+      remaining = remaining - s_above;
       mask |= 255u << shift;
       __syncthreads();
     }
@@ -206,29 +230,10 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   if (tid == 0) { sm.bstar = 0; sm.above = -1; }
   // 1. threshold bucket b*: the bucket holding the k-th largest key
   const uint32_t *hrow = w.hist + (size_t)row * kTopkBins;
-  constexpr int kPer = kTopkBins / kSelThreads;            // bins per thread, from the top
-  uint32_t local[kPer];
-  int lsum = 0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    local[i] = hrow[kTopkBins - 1 - (tid * kPer + i)];
-    lsum += (int)local[i];
-  }
-  int total;
-  const int before = block_exclusive_scan(lsum, sm.scan, &total);
-  if (before < k && before + lsum >= k) {
-    int cum = before;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      if (cum + (int)local[i] >= k) {
-        sm.bstar = kTopkBins - 1 - (tid * kPer + i);
-        sm.above = cum;
-        break;
-      }
-      cum += (int)local[i];
-    }
-  }
+  for (int i = tid; i < kTopkBins; i += blockDim.x) sm.hist[i] = hrow[i];
   __syncthreads();
+  find_threshold_bin([&](int i) { return sm.hist[i]; }, kTopkBins, k, sm.scan, &sm.bstar,
+                     &sm.above);
   const uint32_t bstar = (uint32_t)sm.bstar;
   const int above = sm.above;
 
@@ -299,21 +304,17 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
         if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
       }
       __syncthreads();
-      if (tid == 0) {
-        int cum = 0, bkt = 1023;
-        for (; bkt > 0; --bkt) {
-          if (cum + (int)sm.hist[bkt] >= remaining) break;
-          cum += (int)sm.hist[bkt];
-        }
-        sm.thr2 = (int)(prefix | ((uint32_t)bkt << shift));
-        sm.take_eq = remaining - cum;
-      }
+      if (tid == 0) { sm.thr2 = 0; sm.take_eq = 0; }
+      find_threshold_bin([&](int i) { return sm.hist[i]; }, 1024, remaining, sm.scan, &sm.thr2,
+                         &sm.take_eq);
+      prefix = prefix | ((uint32_t)sm.thr2 << shift);
+      remaining = remaining - sm.take_eq;
       __syncthreads();
-      prefix = (uint32_t)sm.thr2;
-      remaining = sm.take_eq;
+      if (tid == 0) { sm.thr2 = (int)prefix; sm.take_eq = remaining; }
       mask |= 1023u << shift;
       __syncthreads();
     }
+    __syncthreads();
     const uint32_t thr2 = (uint32_t)sm.thr2;
     const int take_eq = sm.take_eq;
     // sure winners, then candidates above thr2, then the take_eq lowest

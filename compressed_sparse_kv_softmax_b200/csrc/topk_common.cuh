@@ -15,8 +15,8 @@ constexpr int kTopkShift = 20;
 constexpr int kCandCap = 8192;
 
 // Indexer workspace layout, one section after another, each 256-byte aligned:
-//   err      4 int                 device status words
 //   scores   rows x ld fp32
+//   err      4 int                 device status words (zeroed before scoring)
 //   hist     rows x kTopkBins u32  (zeroed before scoring)
 //   ctr      rows x 4 u32          selected count, candidate count, ticket (zeroed)
 //   sel      rows x k int32        entries above the threshold bucket
@@ -41,9 +41,9 @@ inline IndexerWs indexer_ws_layout(void *base, long long rows, long long max_ent
   if (w.ld < 4) w.ld = 4;
   uint8_t *p = static_cast<uint8_t *>(base);
   size_t off = 0;
-  w.err = reinterpret_cast<int *>(p + off);           off = align256(off + 16);
   w.scores = reinterpret_cast<float *>(p + off);      off = align256(off + rows * w.ld * 4);
   const size_t zero_begin = off;
+  w.err = reinterpret_cast<int *>(p + off);           off = align256(off + 16);
   w.hist = reinterpret_cast<uint32_t *>(p + off);     off = align256(off + rows * kTopkBins * 4);
   w.ctr = reinterpret_cast<uint32_t *>(p + off);      off = align256(off + rows * 16);
   w.zero_bytes = off - zero_begin;

@@ -69,3 +69,21 @@ def test_decode_attention_full_size(C, name):
                     np.stack([lse[r].cpu().numpy() for r in rows]),
                     np.stack([ref[r][0] for r in rows]), np.stack([ref[r][1] for r in rows]),
                     where=f"{name} hca")
+
+
+def test_prefill_sparse_attention_full_size(C):
+    """8,192 query rows on a 1,048,576-token context, each with its own 1,024
+    selected entries plus its causal window; 64 sampled rows checked."""
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    wl = W.get("prefill")
+    L = W.make_csa_layer(wl, device="cuda")
+    sel = W.random_selection(wl, wl.k, device="cuda")
+    layer = CSALayer(L)
+    out, lse = layer.attend(sel)
+    torch.cuda.synchronize()
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_attention(L, sel=sel.cpu().numpy(), rows=rows)
+    check_attention(np.stack([out[r].cpu().numpy() for r in rows]),
+                    np.stack([lse[r].cpu().numpy() for r in rows]),
+                    np.stack([ref[r][0] for r in rows]), np.stack([ref[r][1] for r in rows]),
+                    where="prefill csa")

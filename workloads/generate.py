@@ -230,3 +230,27 @@ def _default_ring(wl: Workload, pool: int, stride: int) -> int:
     while cap < need:
         cap *= 2
     return cap
+
+
+def random_selection(wl: Workload, k: int, seed: int = 17, device="cpu"):
+    """A seeded stand-in for an indexer selection: for every query row, k
+    distinct visible CSA entries in ascending order (all visible entries when
+    fewer than k), -1 padded.  int32 [B][Tq][k]."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    pos, _ = _positions(wl, "cpu")
+    out = torch.full((wl.B, wl.Tq, k), -1, dtype=torch.int32)
+    for b in range(wl.B):
+        for t in range(wl.Tq):
+            n = int(pos[b, t] + 1) // wl.csa_stride
+            if n <= k:
+                out[b, t, :n] = torch.arange(n, dtype=torch.int32)
+            else:
+                # oversample, de-duplicate, keep k at random, sort
+                u = torch.empty(0, dtype=torch.int64)
+                while u.numel() < k:
+                    u = torch.unique(torch.cat([u, torch.randint(0, n, (2 * k,), generator=g)]))
+                pick = u[torch.randperm(u.numel(), generator=g)[:k]].sort().values
+                out[b, t] = pick.to(torch.int32)
+    return out.to(device)
+
