@@ -294,15 +294,27 @@ def run_ours(args, rank, world, dev):
     return res, replicas, wl
 
 
+_TRAFFIC_SOURCES = ["indexer.cu", "indexer_tc.cu", "topk.cu", "topk_common.cuh", "sm100.cuh"]
+
+
 def _profile_traffic(workload):
-    """DRAM bytes per indexer launch from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
-    if os.path.exists(p):
-        try:
-            return json.load(open(p)).get("indexer_dram_bytes_per_launch")
-        except (ValueError, OSError):
-            return None
-    return None
+    """DRAM bytes per indexer_topk call from the committed ncu summary, when
+    the kernel sources still hash to the ones the counters were taken on
+    (null otherwise: the counters describe another build)."""
+    import hashlib
+    import re
+    p = os.path.join(ROOT, "profiles", f"indexer_tc_{workload}_decode.md")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
+    m_h = re.search(r"^traffic_sources_sha256_16:\s*([0-9a-f]+)", text, re.M)
+    if not (m_t and m_h):
+        return None
+    h = hashlib.sha256()
+    for f in _TRAFFIC_SOURCES:
+        h.update(open(os.path.join(ROOT, "compressed_sparse_kv_softmax_b200", "csrc", f), "rb").read())
+    return int(m_t.group(1)) if h.hexdigest()[:16] == m_h.group(1) else None
 
 
 def run_e2e(args, replicas, wl, dev, world):

@@ -51,7 +51,7 @@ using namespace sm100;
 constexpr int kHeads = 64, kD = 512, kDn = 448, kDr = 64;
 constexpr int kKeys = 64;                          // keys per unit (valid MMA rows)
 constexpr int kM = 128;                            // MMA M (rows kKeys..127 are masked)
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;                      // warps w, w+4 share TMEM lanes
 constexpr uint32_t kChunkK = kKeys * 128;          // bytes per 64-dim chunk of a key tile
 constexpr uint32_t kChunkQ = kHeads * 128;         // bytes per 64-dim chunk of Q
 constexpr uint32_t kIdescQK = idesc(kFmtF16, kFmtF16, 0, 0, kM, kHeads);
@@ -66,7 +66,7 @@ struct __align__(1024) Smem {
   uint8_t phi[kKeys * 128];         // 8 KB: P^T hi, MN-major [keys][64 heads]
   uint8_t plo[kKeys * 128];         // 8 KB
   float red[4][kHeads];
-  float m[kHeads], l[kHeads];
+  float m[kHeads], l[kHeads], inv_l[kHeads];
   long long slot[kM];
   uint64_t bar;
   uint32_t tmem_base;
@@ -92,14 +92,14 @@ __device__ __forceinline__ void split_h2(float a, float b, uint32_t &hi, uint32_
   lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
-// Warp reduce-scatter of 64 per-lane values: afterwards lane L holds the
-// combination over the warp of values 2L and 2L+1 (in out[0], out[1]).
+// Warp reduce-scatter of 32 per-lane values: afterwards lane L holds the
+// combination over the warp's lanes of value L (16+8+4+2+1 shuffles).
 template <bool kMax>
-__device__ __forceinline__ void butterfly64(float (&v)[64], float &o0, float &o1) {
+__device__ __forceinline__ float butterfly32(float (&v)[32]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int step = 0; step < 5; ++step) {
-    const int half = 32 >> step;             // values kept after this step
+    const int half = 16 >> step;             // values kept after this step
     const int bit = 16 >> step;              // partner lane distance
     const bool upper = (lane & bit) != 0;
 #pragma unroll
@@ -110,8 +110,13 @@ __device__ __forceinline__ void butterfly64(float (&v)[64], float &o0, float &o1
       v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
     }
   }
-  o0 = v[0];
-  o1 = v[1];
+  return v[0];
+}
+
+// two E4M3 codes (low byte first) -> float2
+__device__ __forceinline__ float2 e4m3x2(uint32_t pair) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)pair, __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2 *>(&h));
 }
 
 struct Row {
@@ -159,7 +164,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
   {
     const __nv_bfloat16 *qg =
         reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD;
-    // 32 16-byte units per thread, loaded 16 at a time before any is used
+    // 16-byte units per thread, loaded 16 at a time before any is used
     constexpr int kPer = kHeads * kD / 8 / kThreads, kBatch = 16;
 #pragma unroll
     for (int i0 = 0; i0 < kPer; i0 += kBatch) {
@@ -194,7 +199,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
   const int nkeys = (int)(avail < 0 ? 0 : (avail < unit_keys ? avail : unit_keys));
   const int ksteps = (nkeys + 15) >> 4;            // 16-key MMA steps of the P V product
   const Cache &src = comp_unit ? a.comp_k : a.win_k;
-  {
+  if (tid < kM) {
     long long slot = -1;
     if (tid < nkeys) {          // nkeys <= kKeys: rows kKeys..kM-1 stay invalid
       const long long i = base + tid;
@@ -208,10 +213,12 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
     sm.slot[tid] = slot;
   }
   // (the barrier also publishes the slots) any key at all in this unit?
-  const bool any = __syncthreads_or(sm.slot[tid] >= 0) != 0;
-  const bool my_valid = sm.slot[tid] >= 0;          // validity of key row `tid`
+  const bool any = __syncthreads_or(tid < kM && sm.slot[tid] >= 0) != 0;
+  const int quad = warp & 3, colh = warp >> 2;      // TMEM lane quadrant, head half
+  const int krow = tid & 127;                       // key row = TMEM lane of this thread
+  const bool my_valid = sm.slot[krow] >= 0;
   // each warp converts 8 consecutive key rows per batch, loads first
-  for (int r0 = warp * 8; r0 < ksteps * 16; r0 += 32) {
+  for (int r0 = warp * 8; r0 < ksteps * 16; r0 += 8 * kThreads / 32) {
     uint4 raw[8], raw2[8];
     float sc[8];
 #pragma unroll
@@ -238,13 +245,17 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
       int d0;
       if (lane < 28) {
         // 16 FP8 codes: dims 16*lane .. +15, block scale lane/4 (absent key: zeros)
-        const uint8_t *cb = reinterpret_cast<const uint8_t *>(&raw[e]);
+        const uint32_t *cw = reinterpret_cast<const uint32_t *>(&raw[e]);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          split_h2(e4m3_decode(cb[2 * q]) * sc[e], e4m3_decode(cb[2 * q + 1]) * sc[e], ph0[q],
-                   pl0[q]);
-          split_h2(e4m3_decode(cb[8 + 2 * q]) * sc[e], e4m3_decode(cb[8 + 2 * q + 1]) * sc[e],
-                   ph1[q], pl1[q]);
+          const float2 a = e4m3x2(cw[q] & 0xffffu), c = e4m3x2(cw[q] >> 16);
+          if (q < 2) {
+            split_h2(a.x * sc[e], a.y * sc[e], ph0[2 * q], pl0[2 * q]);
+            split_h2(c.x * sc[e], c.y * sc[e], ph0[2 * q + 1], pl0[2 * q + 1]);
+          } else {
+            split_h2(a.x * sc[e], a.y * sc[e], ph1[2 * q - 4], pl1[2 * q - 4]);
+            split_h2(c.x * sc[e], c.y * sc[e], ph1[2 * q - 3], pl1[2 * q - 3]);
+          }
         }
         d0 = lane * 16;
       } else {
@@ -297,65 +308,55 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
     }
     bool ok = mbar_wait(&sm.bar, 0);
     tc_fence_after();
-    // ---- softmax over keys, per head
-    float s[64];
-    {
-      float t[32];
-      const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
-      tmem_ld32(ta, t);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s[i] = t[i];
-      tmem_ld32(ta + 32, t);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s[32 + i] = t[i];
-      tmem_wait_ld();
-    }
+    // ---- softmax over keys, per head (this thread: key krow, heads 32*colh ..)
+    float sv[32];
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    tmem_ld32(tl + colh * 32, sv);
+    tmem_wait_ld();
     const float c2 = a.sm_scale * 1.4426950408889634f;   // logits in log2 units
 #pragma unroll
-    for (int i = 0; i < 64; ++i) s[i] = my_valid ? s[i] * c2 : -CUDART_INF_F;
+    for (int i = 0; i < 32; ++i) sv[i] = my_valid ? sv[i] * c2 : -CUDART_INF_F;
     {
-      float v[64];
+      float v[32];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) v[i] = s[i];
-      float m0, m1;
-      butterfly64<true>(v, m0, m1);
-      sm.red[warp][2 * lane] = m0;
-      sm.red[warp][2 * lane + 1] = m1;
+      for (int i = 0; i < 32; ++i) v[i] = sv[i];
+      sm.red[quad][colh * 32 + lane] = butterfly32<true>(v);
     }
     __syncthreads();
     if (tid < kHeads)
       sm.m[tid] = fmaxf(fmaxf(sm.red[0][tid], sm.red[1][tid]), fmaxf(sm.red[2][tid], sm.red[3][tid]));
     __syncthreads();
     {
-      float v[64];
+      float v[32];
 #pragma unroll
-      for (int h = 0; h < 64; h += 8) {
+      for (int h = 0; h < 32; h += 8) {
         uint4 wh, wl;
         uint32_t *whp = reinterpret_cast<uint32_t *>(&wh), *wlp = reinterpret_cast<uint32_t *>(&wl);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int hh = h + 2 * e;
-          const float p0 = my_valid ? exp2f(s[hh] - sm.m[hh]) : 0.f;
-          const float p1 = my_valid ? exp2f(s[hh + 1] - sm.m[hh + 1]) : 0.f;
+          const int hh = h + 2 * e, hg = colh * 32 + hh;
+          const float p0 = my_valid ? exp2f(sv[hh] - sm.m[hg]) : 0.f;
+          const float p1 = my_valid ? exp2f(sv[hh + 1] - sm.m[hg + 1]) : 0.f;
           split_h2(p0, p1, whp[e], wlp[e]);
           v[hh] = p0;
           v[hh + 1] = p1;
         }
-        if (tid < kKeys) {
-          *reinterpret_cast<uint4 *>(sm.phi + swz(tid, h >> 3)) = wh;
-          *reinterpret_cast<uint4 *>(sm.plo + swz(tid, h >> 3)) = wl;
+        if (krow < kKeys) {
+          const uint32_t u = (colh * 32 + h) >> 3;
+          *reinterpret_cast<uint4 *>(sm.phi + swz(krow, u)) = wh;
+          *reinterpret_cast<uint4 *>(sm.plo + swz(krow, u)) = wl;
         }
       }
-      float l0, l1;
-      butterfly64<false>(v, l0, l1);
-      sm.red[warp][2 * lane] = l0;
-      sm.red[warp][2 * lane + 1] = l1;
+      sm.red[quad][colh * 32 + lane] = butterfly32<false>(v);
     }
     fence_proxy_async_shared();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid < kHeads) sm.l[tid] = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
+    if (tid < kHeads) {
+      sm.l[tid] = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
+      sm.inv_l[tid] = 1.f / sm.l[tid];
+    }
     // ---- O^T = V^T P^T
     if (tid == 0) {
       const uint32_t vh = smem_addr(sm.khi), vl = smem_addr(sm.klo);
@@ -378,22 +379,18 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
     ok = mbar_wait(&sm.bar, 1) && ok;
     tc_fence_after();
     __syncthreads();
-    // ---- epilogue: thread = dim within each 128-dim tile
+    // ---- epilogue: thread = dim within each 128-dim tile, heads 32*colh ..
     const float inv_ln = 0.6931471805599453f;
     if (tid < kHeads) pl[tid] = ok ? (sm.m[tid] + log2f(sm.l[tid])) * inv_ln : CUDART_NAN_F;
     for (int mt = 0; mt < 4; ++mt) {
-      const int d = mt * 128 + tid;
-      const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + 64 + mt * 64;
+      const int d = mt * 128 + quad * 32 + lane;
+      float o[32];
+      tmem_ld32(tl + 64 + mt * 64 + colh * 32, o);
+      tmem_wait_ld();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float o[32];
-        tmem_ld32(ta + half * 32, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int h = half * 32 + i;
-          po[(size_t)h * kD + d] = o[i] / sm.l[h];
-        }
+      for (int i = 0; i < 32; ++i) {
+        const int h = colh * 32 + i;
+        po[(size_t)h * kD + d] = o[i] * sm.inv_l[h];
       }
     }
   }

@@ -184,22 +184,23 @@ __device__ inline void stage_bytes(uint8_t *dst, const uint8_t *src, int n, int 
   }
 }
 
-// stage `pool` slots of plane set `c` for positions first .. first+pool-1
-__device__ void stage_window(const Cache &c, const SlotLayout &l, int b, long long first,
+// stage `pool` slots of plane set `c` for positions first .. first+pool-1;
+// rows[r] is the precomputed slot row (b * cap + slot) of position first + r,
+// or -1 when that position does not exist.  One warp per slot: the 16-byte
+// copies of a slot are spread over its lanes.
+__device__ void stage_window(const Cache &c, const SlotLayout &l, const long long *rows,
                              int pool, uint8_t *buf) {
-  const int nt = blockDim.x;
-  for (int r = 0; r < pool; ++r) {
-    const long long p = first + r;
-    if (p < 0) continue;
-    const long long slot = c.slot_of(p);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int r = warp; r < pool; r += nw) {
+    const long long row = rows[r];
+    if (row < 0) continue;
     uint8_t *dst = buf + (size_t)r * l.bytes;
-    stage_bytes(dst, c.data + c.row(b, slot) * c.data_stride, l.data_bytes, threadIdx.x, nt);
+    stage_bytes(dst, c.data + row * c.data_stride, l.data_bytes, lane, 32);
     if (c.fmt != CSKV_FMT_F32) {
-      stage_bytes(dst + l.scale_off, c.scale + c.row(b, slot) * c.scale_stride,
-                  4 * (c.d_nope >> 6), threadIdx.x, nt);
+      stage_bytes(dst + l.scale_off, c.scale + row * c.scale_stride, 4 * (c.d_nope >> 6), lane,
+                  32);
       if (c.d_rope)
-        stage_bytes(dst + l.rope_off, c.rope + c.row(b, slot) * c.rope_stride, 2 * c.d_rope,
-                    threadIdx.x, nt);
+        stage_bytes(dst + l.rope_off, c.rope + row * c.rope_stride, 2 * c.d_rope, lane, 32);
     }
   }
 }
@@ -247,10 +248,25 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   float *a = reinterpret_cast<float *>(bi + (raw_ik.data ? (size_t)pool * li.bytes : 0));
   float *pooled = a + pool;
   const int D = raw_k.dims();
+  int dmax = D;
+  if (raw_v.data && raw_v.dims() > dmax) dmax = raw_v.dims();
+  if (raw_ik.data && raw_ik.dims() > dmax) dmax = raw_ik.dims();
+  long long *rows = reinterpret_cast<long long *>(
+      (reinterpret_cast<uintptr_t>(pooled + dmax) + 7) & ~uintptr_t(7));
+  long long *rows_v = rows + pool;
+  long long *rows_i = rows_v + pool;
 
-  stage_window(raw_k, lk, b, first, pool, bk);
-  if (raw_v.data) stage_window(raw_v, lv, b, first, pool, bv);
-  if (raw_ik.data) stage_window(raw_ik, li, b, first, pool, bi);
+  // slot rows of the window's positions, one modulo per position
+  for (int r = tid; r < pool; r += blockDim.x) {
+    const long long p = first + r;
+    rows[r] = p < 0 ? -1 : raw_k.row(b, raw_k.slot_of(p));
+    if (raw_v.data) rows_v[r] = p < 0 ? -1 : raw_v.row(b, raw_v.slot_of(p));
+    if (raw_ik.data) rows_i[r] = p < 0 ? -1 : raw_ik.row(b, raw_ik.slot_of(p));
+  }
+  __syncthreads();
+  stage_window(raw_k, lk, rows, pool, bk);
+  if (raw_v.data) stage_window(raw_v, lv, rows_v, pool, bv);
+  if (raw_ik.data) stage_window(raw_ik, li, rows_i, pool, bi);
   cp_async_wait_all();
   __syncthreads();
 
@@ -311,7 +327,8 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
   size_t staged = (size_t)pool * slot_layout(raw_k).bytes;
   if (raw_v.data) staged += (size_t)pool * slot_layout(raw_v).bytes;
   if (raw_ik.data) staged += (size_t)pool * slot_layout(raw_ik).bytes;
-  const size_t smem_staged = staged + sizeof(float) * (size_t)(pool + dmax);
+  const size_t smem_staged = staged + sizeof(float) * (size_t)(pool + dmax + 1) +
+                             3 * sizeof(long long) * (size_t)pool + 16;
   if (smem_staged <= 200 * 1024 && ensure_dynamic_smem(compress_staged_kernel, smem_staged)) {
     compress_staged_kernel<<<grid, kThreads, smem_staged, st>>>(
         t_begin, t_end, raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride, out_k, out_v, out_ik);

@@ -165,14 +165,15 @@ __device__ __forceinline__ long long visible(const int64_t *q_pos, int row, int 
 }
 
 // Ascending bitonic sort of v[0..m) in shared memory, m a power of two.
-__device__ void bitonic_sort_smem(int32_t *v, int m) {
+template <typename T>
+__device__ void bitonic_sort_smem(T *v, int m) {
   for (int size = 2; size <= m; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       for (int i = threadIdx.x; i < (m >> 1); i += blockDim.x) {
         const int lo = 2 * i - (i & (stride - 1));
         const int hi = lo + stride;
         const bool up = (lo & size) == 0;
-        const int32_t a = v[lo], b = v[hi];
+        const T a = v[lo], b = v[hi];
         if ((a > b) == up) { v[lo] = b; v[hi] = a; }
       }
       __syncthreads();
@@ -180,17 +181,30 @@ __device__ void bitonic_sort_smem(int32_t *v, int m) {
   }
 }
 
+// inverse of score_key
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+__device__ __forceinline__ uint64_t pack_entry(long long j, uint32_t key) {
+  return ((uint64_t)(uint32_t)j << 32) | key;
+}
+
 constexpr int kSelThreads = 512;
 constexpr int kCandSmem = kCandCap; // candidates the last CTA refines in shared memory
 constexpr int kMaxK = 4096;
+constexpr int kScanBatch = 8;       // scores a thread loads before processing any
+// rows of up to this many entries are ordered through a bitmap plus word
+// prefix counts, both held in the (by then unused) candidate buffer
+constexpr int kBitmapWords = kCandSmem;                 // 8192 words x 2 arrays = 64 KB
+constexpr long long kBitmapEntries = 32LL * kBitmapWords;
 
 struct SelSmem {
-  uint32_t hist[kTopkBins];         // row histogram, later the refine histograms
-  uint32_t ckey[kCandSmem];
-  int32_t cidx[kCandSmem];
-  int32_t out[kMaxK];
+  uint32_t hist[kTopkBins];         // row histogram, later refine histograms / tie list
+  uint64_t cand[kCandSmem];         // (index << 32) | key
+  uint64_t out[kMaxK];              // (index << 32) | key of the selection
   int scan[33];
-  int bstar, above, is_last, thr2, take_eq, n_eq, fallback;
+  int bstar, above, is_last, thr2, take_eq, n_eq, n_gt, fallback, n_cand, n_sel;
 };
 
 }  // namespace
@@ -227,70 +241,118 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     return;
   }
 
-  if (tid == 0) { sm.bstar = 0; sm.above = -1; }
   // 1. threshold bucket b*: the bucket holding the k-th largest key
-  const uint32_t *hrow = w.hist + (size_t)row * kTopkBins;
-  for (int i = tid; i < kTopkBins; i += blockDim.x) sm.hist[i] = hrow[i];
+  if (tid == 0) { sm.bstar = 0; sm.above = -1; }
+  {
+    const uint32_t *hrow = w.hist + (size_t)row * kTopkBins;
+    constexpr int kPer = kTopkBins / kSelThreads;
+    uint32_t v[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) v[e] = __ldcg(hrow + tid + e * kSelThreads);
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) sm.hist[tid + e * kSelThreads] = v[e];
+  }
   __syncthreads();
   find_threshold_bin([&](int i) { return sm.hist[i]; }, kTopkBins, k, sm.scan, &sm.bstar,
                      &sm.above);
   const uint32_t bstar = (uint32_t)sm.bstar;
   const int above = sm.above;
 
-  // 2. this CTA's slice: sure winners and candidates
+  // 2. this CTA's slice: sure winners (above b*) and candidates (in b*),
+  //    appended as (index, key) pairs; one atomic per warp and batch
   uint32_t *ctr = w.ctr + (size_t)row * 4;
-  int32_t *selrow = w.sel + (size_t)row * k;
-  int32_t *candrow = w.cand + (size_t)row * kCandCap;
+  uint64_t *selrow = w.sel + (size_t)row * k;
+  uint64_t *candrow = w.cand + (size_t)row * kCandCap;
   const long long per = ((n + gridDim.x - 1) / gridDim.x + 31) & ~31LL;
   const long long j_lo = (long long)blockIdx.x * per;
   const long long j_hi = min(n, j_lo + per);
-  for (long long j0 = j_lo; j0 < j_hi; j0 += blockDim.x) {
-    const long long j = j0 + tid;
-    uint32_t bkt = 0;
-    bool valid = j < j_hi;
-    if (valid) bkt = score_key(s[j]) >> kTopkShift;
-    const bool gt = valid && bkt > bstar;
-    const bool eq = valid && bkt == bstar;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    const unsigned mg = __ballot_sync(0xffffffffu, gt);
-    const unsigned me = __ballot_sync(0xffffffffu, eq);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (long long j0 = j_lo; j0 < j_hi; j0 += (long long)kScanBatch * kSelThreads) {
+    uint32_t key[kScanBatch];
+#pragma unroll
+    for (int e = 0; e < kScanBatch; ++e) {
+      const long long j = j0 + e * kSelThreads + tid;
+      key[e] = j < j_hi ? score_key(__ldcg(s + j)) : 0u;
+    }
+    unsigned mg[kScanBatch], me[kScanBatch];
+    int cg = 0, ce = 0;
+#pragma unroll
+    for (int e = 0; e < kScanBatch; ++e) {
+      const long long j = j0 + e * kSelThreads + tid;
+      const uint32_t bkt = key[e] >> kTopkShift;
+      mg[e] = __ballot_sync(0xffffffffu, j < j_hi && bkt > bstar);
+      me[e] = __ballot_sync(0xffffffffu, j < j_hi && bkt == bstar);
+      cg += __popc(mg[e]);
+      ce += __popc(me[e]);
+    }
     uint32_t bg = 0, be = 0;
     if (lane == 0) {
-      if (mg) bg = atomicAdd(&ctr[0], (uint32_t)__popc(mg));
-      if (me) be = atomicAdd(&ctr[1], (uint32_t)__popc(me));
+      if (cg) bg = atomicAdd(&ctr[0], (uint32_t)cg);
+      if (ce) be = atomicAdd(&ctr[1], (uint32_t)ce);
     }
     bg = __shfl_sync(0xffffffffu, bg, 0);
     be = __shfl_sync(0xffffffffu, be, 0);
-    if (gt) {
-      const uint32_t p = bg + __popc(mg & lt_mask);
-      if (p < (uint32_t)k) selrow[p] = (int32_t)j;
-    }
-    if (eq) {
-      const uint32_t p = be + __popc(me & lt_mask);
-      if (p < (uint32_t)kCandCap) candrow[p] = (int32_t)j;
+#pragma unroll
+    for (int e = 0; e < kScanBatch; ++e) {
+      const long long j = j0 + e * kSelThreads + tid;
+      if (mg[e] >> lane & 1u) {
+        const uint32_t p = bg + __popc(mg[e] & lt_mask);
+        if (p < (uint32_t)k) selrow[p] = pack_entry(j, key[e]);
+      }
+      if (me[e] >> lane & 1u) {
+        const uint32_t p = be + __popc(me[e] & lt_mask);
+        if (p < (uint32_t)kCandCap) candrow[p] = pack_entry(j, key[e]);
+      }
+      bg += __popc(mg[e]);
+      be += __popc(me[e]);
     }
   }
 
   // 3. the last CTA of the row finishes the selection
   __threadfence();
   __syncthreads();
-  if (tid == 0) sm.is_last = atomicAdd(&ctr[2], 1u) == gridDim.x - 1;
+  if (tid == 0) {
+    sm.is_last = atomicAdd(&ctr[2], 1u) == gridDim.x - 1;
+    if (sm.is_last) {
+      __threadfence();
+      sm.n_sel = (int)atomicAdd(&ctr[0], 0u);
+      sm.n_cand = (int)atomicAdd(&ctr[1], 0u);
+    }
+  }
   __syncthreads();
   if (!sm.is_last) return;
-  __threadfence();
-  const int n_cand = (int)atomicAdd(&ctr[1], 0u);
+  const int n_cand = sm.n_cand;
   const int r = k - above;                 // candidates still to take, 1 <= r <= n_cand
   // any inconsistency between the histogram and the scores (never expected)
   // sends the row to the single-CTA path instead of indexing out of range
   if (tid == 0)
     sm.fallback = above < 0 || above >= k || r < 1 || r > n_cand || n_cand > kCandSmem ||
-                  atomicAdd(&ctr[0], 0u) != (uint32_t)above;
+                  sm.n_sel != above;
   __syncthreads();
   if (!sm.fallback) {
-    for (int i = tid; i < n_cand; i += blockDim.x) {
-      const int32_t j = candrow[i];
-      sm.cidx[i] = j;
-      sm.ckey[i] = score_key(s[j]);
+    {  // candidates and sure winners into shared memory, loads first
+      constexpr int kC = kCandSmem / kSelThreads, kS = kMaxK / kSelThreads;
+      uint64_t v[kC], u[kS];
+#pragma unroll
+      for (int e = 0; e < kC; ++e) {
+        const int i = tid + e * kSelThreads;
+        v[e] = i < n_cand ? __ldcg(candrow + i) : 0ull;
+      }
+#pragma unroll
+      for (int e = 0; e < kS; ++e) {
+        const int i = tid + e * kSelThreads;
+        u[e] = i < above ? __ldcg(selrow + i) : 0ull;
+      }
+#pragma unroll
+      for (int e = 0; e < kC; ++e) {
+        const int i = tid + e * kSelThreads;
+        if (i < n_cand) sm.cand[i] = v[e];
+      }
+#pragma unroll
+      for (int e = 0; e < kS; ++e) {
+        const int i = tid + e * kSelThreads;
+        if (i < above) sm.out[i] = u[e];
+      }
     }
     // radix select of the r-th largest candidate key on bits 19..10, then 9..0
     uint32_t prefix = bstar << kTopkShift, mask = 0xFFFu << kTopkShift;
@@ -300,7 +362,7 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
       for (int i = tid; i < 1024; i += blockDim.x) sm.hist[i] = 0;
       __syncthreads();
       for (int i = tid; i < n_cand; i += blockDim.x) {
-        const uint32_t key = sm.ckey[i];
+        const uint32_t key = (uint32_t)sm.cand[i];
         if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
       }
       __syncthreads();
@@ -309,62 +371,90 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
                          &sm.take_eq);
       prefix = prefix | ((uint32_t)sm.thr2 << shift);
       remaining = remaining - sm.take_eq;
-      __syncthreads();
-      if (tid == 0) { sm.thr2 = (int)prefix; sm.take_eq = remaining; }
       mask |= 1023u << shift;
       __syncthreads();
     }
+    const uint32_t thr2 = prefix;
+    const int take_eq = remaining;
+    // candidates above thr2 follow the sure winners; the indices of candidates
+    // equal to thr2 go to a tie list (the lowest take_eq of them are taken)
+    if (tid == 0) { sm.n_gt = 0; sm.n_eq = 0; }
     __syncthreads();
-    const uint32_t thr2 = (uint32_t)sm.thr2;
-    const int take_eq = sm.take_eq;
-    // sure winners, then candidates above thr2, then the take_eq lowest
-    // indices among candidates equal to thr2 (gathered at the end of `out`)
-    for (int i = tid; i < above; i += blockDim.x) sm.out[i] = selrow[i];
-    if (tid == 0) { sm.is_last = 0; sm.n_eq = 0; }
-    __syncthreads();
-    int *cnt_gt = &sm.is_last;     // reuse as a counter
+    uint32_t *eqv = sm.hist;                 // up to kTopkBins entries
     for (int i = tid; i < n_cand; i += blockDim.x) {
-      const uint32_t key = sm.ckey[i];
+      const uint64_t c = sm.cand[i];
+      const uint32_t key = (uint32_t)c;
       if (key > thr2) {
-        const int p = atomicAdd(cnt_gt, 1);
-        if (above + p < k) sm.out[above + p] = sm.cidx[i];
-      }
-    }
-    __syncthreads();
-    const int n_gt = *cnt_gt;                 // == r - take_eq
-    // equal keys: collect into the cand key array (no longer needed)
-    int32_t *eqv = reinterpret_cast<int32_t *>(sm.hist);   // up to kTopkBins entries
-    for (int i = tid; i < n_cand; i += blockDim.x) {
-      if (sm.ckey[i] == thr2) {
+        const int p = atomicAdd(&sm.n_gt, 1);
+        if (above + p < k) sm.out[above + p] = c;
+      } else if (key == thr2) {
         const int p = atomicAdd(&sm.n_eq, 1);
-        if (p < kTopkBins) eqv[p] = sm.cidx[i];
+        if (p < kTopkBins) eqv[p] = (uint32_t)(c >> 32);
       }
     }
     __syncthreads();
-    const int n_eq = sm.n_eq;
+    const int n_gt = sm.n_gt, n_eq = sm.n_eq;
     if (n_eq > kTopkBins || above + n_gt + take_eq != k || take_eq > n_eq) {
       if (tid == 0) sm.fallback = 1;
     } else {
       if (n_eq > take_eq) {
         int m = 1;
         while (m < n_eq) m <<= 1;
-        for (int i = n_eq + tid; i < m; i += blockDim.x) eqv[i] = INT_MAX;
+        for (int i = n_eq + tid; i < m; i += blockDim.x) eqv[i] = 0xffffffffu;
         __syncthreads();
         bitonic_sort_smem(eqv, m);
       }
-      for (int i = tid; i < take_eq; i += blockDim.x) sm.out[above + n_gt + i] = eqv[i];
+      for (int i = tid; i < take_eq; i += blockDim.x)
+        sm.out[above + n_gt + i] = ((uint64_t)eqv[i] << 32) | thr2;
     }
     __syncthreads();
     if (!sm.fallback) {
-      int m = 1;
-      while (m < k) m <<= 1;
-      for (int i = k + tid; i < m; i += blockDim.x) sm.out[i] = INT_MAX;
-      __syncthreads();
-      bitonic_sort_smem(sm.out, m);
-      for (int i = tid; i < k; i += blockDim.x) {
-        const int32_t j = sm.out[i];
-        oi[i] = j;
-        if (os) os[i] = s[j];
+      if (n <= kBitmapEntries) {
+        // ascending order by rank: the selected entries are distinct indices
+        // below n; mark them in a bitmap, prefix-count the words, and each
+        // entry's rank is the count of marked indices below it
+        uint32_t *bits = reinterpret_cast<uint32_t *>(sm.cand);
+        uint32_t *wpre = bits + kBitmapWords;
+        const int nw = (int)((n + 31) >> 5);
+        for (int i = tid; i < nw; i += blockDim.x) bits[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < k; i += blockDim.x) {
+          const uint32_t j = (uint32_t)(sm.out[i] >> 32);
+          atomicOr(&bits[j >> 5], 1u << (j & 31));
+        }
+        __syncthreads();
+        const int per_t = (nw + blockDim.x - 1) / blockDim.x;
+        const int w0 = tid * per_t;
+        int cnt = 0;
+        for (int i = 0; i < per_t; ++i)
+          if (w0 + i < nw) cnt += __popc(bits[w0 + i]);
+        int tot;
+        int run = block_exclusive_scan(cnt, sm.scan, &tot);
+        for (int i = 0; i < per_t; ++i) {
+          if (w0 + i < nw) {
+            wpre[w0 + i] = (uint32_t)run;
+            run += __popc(bits[w0 + i]);
+          }
+        }
+        __syncthreads();
+        for (int i = tid; i < k; i += blockDim.x) {
+          const uint64_t e = sm.out[i];
+          const uint32_t j = (uint32_t)(e >> 32);
+          const int rank = (int)wpre[j >> 5] + __popc(bits[j >> 5] & ((1u << (j & 31)) - 1u));
+          oi[rank] = (int32_t)j;
+          if (os) os[rank] = key_score((uint32_t)e);
+        }
+      } else {
+        int m = 1;
+        while (m < k) m <<= 1;
+        for (int i = k + tid; i < m; i += blockDim.x) sm.out[i] = ~0ull;
+        __syncthreads();
+        bitonic_sort_smem(sm.out, m);        // ascending entry index
+        for (int i = tid; i < k; i += blockDim.x) {
+          const uint64_t e = sm.out[i];
+          oi[i] = (int32_t)(e >> 32);
+          if (os) os[i] = key_score((uint32_t)e);
+        }
       }
     }
   }

@@ -19,15 +19,15 @@ constexpr int kCandCap = 8192;
 //   err      4 int                 device status words (zeroed before scoring)
 //   hist     rows x kTopkBins u32  (zeroed before scoring)
 //   ctr      rows x 4 u32          selected count, candidate count, ticket (zeroed)
-//   sel      rows x k int32        entries above the threshold bucket
-//   cand     rows x kCandCap int32 entries inside the threshold bucket
+//   sel      rows x k u64          entries above the threshold bucket, (index << 32) | key
+//   cand     rows x kCandCap u64   entries inside the threshold bucket, same packing
 struct IndexerWs {
   int *err;
   float *scores;
   uint32_t *hist;
   uint32_t *ctr;
-  int32_t *sel;
-  int32_t *cand;
+  uint64_t *sel;
+  uint64_t *cand;
   long long ld;
   size_t zero_bytes;   // bytes from `hist` that must be zero before the call
 };
@@ -47,8 +47,8 @@ inline IndexerWs indexer_ws_layout(void *base, long long rows, long long max_ent
   w.hist = reinterpret_cast<uint32_t *>(p + off);     off = align256(off + rows * kTopkBins * 4);
   w.ctr = reinterpret_cast<uint32_t *>(p + off);      off = align256(off + rows * 16);
   w.zero_bytes = off - zero_begin;
-  w.sel = reinterpret_cast<int32_t *>(p + off);       off = align256(off + rows * (size_t)k * 4);
-  w.cand = reinterpret_cast<int32_t *>(p + off);      off = align256(off + rows * (size_t)kCandCap * 4);
+  w.sel = reinterpret_cast<uint64_t *>(p + off);      off = align256(off + rows * (size_t)k * 8);
+  w.cand = reinterpret_cast<uint64_t *>(p + off);     off = align256(off + rows * (size_t)kCandCap * 8);
   if (total) *total = off;
   return w;
 }
