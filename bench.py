@@ -1,19 +1,22 @@
 #!/usr/bin/env python3
 """Benchmark: CSA+HCA hybrid-attention decode at a 1,048,576-token context.
 
-One step is one decode token through one CSA layer and one HCA layer of every
-sequence, at a position where both compressors fire (T = 2^20 is a multiple of
-4 and of 128):
-  CSA layer: csa_compress (new entry) -> indexer_topk (score 262,144 entries,
-             keep 1,024) -> hybrid_attn_decode (1,024 selected + 128 window)
-  HCA layer: hca_compress (new entry) -> hybrid_attn_decode (8,192 dense + 128)
+One step is one decode token of every sequence through one CSA layer and one
+HCA layer.  Steps walk through a window of 128 consecutive positions centred
+on 1,048,576 (contexts 1,048,513 .. 1,048,640), one HCA period, so that the
+compressors run exactly where an entry completes: CSA compression on the 32
+tokens that close a 4-token group, HCA compression on the one token that
+closes a 128-token block.  Every step runs
+  CSA layer: [csa_compress] -> indexer_topk (score the ~262,144 visible
+             entries, keep 1,024) -> hybrid_attn_decode (1,024 + 128 window)
+  HCA layer: [hca_compress] -> hybrid_attn_decode (8,192 dense + 128 window)
 The metric is decode queries/s (one query = one token through both layers).
 
 Inputs are seeded synthetic tensors resident in HBM.  R replicas of every
 layer's inputs rotate between steps; their per-step bytes total more than 4x
-the 126 MB L2, so each step reads HBM.  The timed region replays a CUDA graph
-of G steps ceil(K/G) times (exactly K steps).  The dominant call
-(indexer_topk) is bracketed by event records inside the graph.
+the 126 MB L2, so each step reads HBM.  The timed region replays CUDA graphs
+of 128 steps (plus one graph of the remaining steps), exactly K steps.  The
+dominant call (indexer_topk) is bracketed by event records inside the graph.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -107,31 +110,59 @@ class ClockSampler:
 
 # ------------------------------------------------------------- our path
 
-class Replica:
-    """One sequence batch's CSA and HCA layer inputs on the device."""
+PERIOD = 128       # one HCA block: every compression pattern of the window repeats
 
-    def __init__(self, wl, seed, dev):
+
+class Schedule:
+    """Positions of the decode window: step s queries position T0 + s with
+    ctx_len T0 + s + 1 (T0 = T - 64, T the workload context)."""
+
+    def __init__(self, wl, dev):
+        self.T0 = wl.T - PERIOD // 2
+        self.q_pos, self.ctx, self.tb, self.te = [], [], [], []
+        self.csa_fires, self.hca_fires = [], []
+        for step in range(PERIOD):
+            p = self.T0 + step
+            self.q_pos.append(torch.full((wl.B, 1), p, dtype=torch.int64, device=dev))
+            self.ctx.append(torch.full((wl.B,), p + 1, dtype=torch.int64, device=dev))
+            self.tb.append(torch.full((wl.B,), p, dtype=torch.int64, device=dev))
+            self.te.append(torch.full((wl.B,), p + 1, dtype=torch.int64, device=dev))
+            self.csa_fires.append((p + 1) // wl.csa_stride > p // wl.csa_stride)
+            self.hca_fires.append((p + 1) // wl.hca_stride > p // wl.hca_stride)
+
+    @property
+    def t_end(self):
+        return self.T0 + PERIOD
+
+
+class Replica:
+    """One sequence batch's CSA and HCA layer inputs on the device, holding
+    every position of the decode window."""
+
+    def __init__(self, wl, sched, seed, dev):
         from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
-        self.csa_L = W.make_csa_layer(wl, device=dev, seed=seed)
-        self.hca_L = W.make_hca_layer(wl, device=dev, seed=seed + 500_000)
+        wlw = wl.with_(T=sched.t_end)
+        self.csa_L = W.make_csa_layer(wlw, device=dev, seed=seed)
+        self.hca_L = W.make_hca_layer(wlw, device=dev, seed=seed + 500_000)
         self.csa = CSALayer(self.csa_L)
         self.hca = HCALayer(self.hca_L)
-        T = wl.T
-        self.t_begin = torch.full((wl.B,), T - 1, dtype=torch.int64, device=dev)
-        self.t_end = torch.full((wl.B,), T, dtype=torch.int64, device=dev)
+        self.sched = sched
 
-    def step(self, mark=None):
-        """Enqueue one decode step on the current stream; mark(i) records an
-        event between calls (i = 0 before indexer_topk, 1 after)."""
-        self.csa.compress(self.t_begin, self.t_end, 1)
+    def step(self, s, mark=None):
+        """Enqueue decode step s of the window on the current stream; mark(i)
+        records an event between calls (i = 0 before indexer_topk, 1 after)."""
+        sc = self.sched
+        if sc.csa_fires[s]:
+            self.csa.compress(sc.tb[s], sc.te[s], 1)
         if mark:
             mark(0)
-        self.csa.select()
+        self.csa.select(sc.q_pos[s])
         if mark:
             mark(1)
-        self.csa.attend()
-        self.hca.compress(self.t_begin, self.t_end, 1)
-        self.hca.attend()
+        self.csa.attend(pos=sc.ctx[s])
+        if sc.hca_fires[s]:
+            self.hca.compress(sc.tb[s], sc.te[s], 1)
+        self.hca.attend(pos=sc.ctx[s])
 
 
 def _rt():
@@ -147,10 +178,11 @@ def _ok(res, what):
 
 
 class StepGraph:
-    """CUDA graph of G consecutive steps over rotating replicas, with external
-    event records around every indexer_topk call."""
+    """CUDA graph of G consecutive decode steps (step i of the timed sequence
+    uses replica i % R and window position i % PERIOD), with external event
+    records around every indexer_topk call."""
 
-    def __init__(self, replicas, G, stream, r0=0):
+    def __init__(self, replicas, G, stream, i0=0):
         rt = _rt()
         self.G = G
         self.events = [[_ok(rt.cudaEventCreate(), "event") for _ in range(2)] for _ in range(G)]
@@ -159,9 +191,9 @@ class StepGraph:
             _ok(rt.cudaStreamBeginCapture(
                 sh, rt.cudaStreamCaptureMode.cudaStreamCaptureModeThreadLocal), "capture")
             for i in range(G):
-                rep = replicas[(r0 + i) % len(replicas)]
+                rep = replicas[(i0 + i) % len(replicas)]
                 ev = self.events[i]
-                rep.step(mark=lambda m, ev=ev: _ok(rt.cudaEventRecordWithFlags(
+                rep.step((i0 + i) % PERIOD, mark=lambda m, ev=ev: _ok(rt.cudaEventRecordWithFlags(
                     ev[m], sh, rt.cudaEventRecordExternal), "record"))
             self.graph = _ok(rt.cudaStreamEndCapture(sh), "end capture")
         self.exec = _ok(rt.cudaGraphInstantiate(self.graph, 0), "instantiate")
@@ -200,16 +232,18 @@ def indexer_bytes(wl):
 
 
 def step_bytes(wl):
-    """Algorithmic HBM bytes of one full decode step (both layers)."""
+    """Algorithmic HBM bytes of one decode step (both layers), compression
+    averaged over the 128-step window (32 CSA entries and 1 HCA entry)."""
     entry = wl.d_nope + 2 * wl.d_rope + 4 * (wl.d_nope // 64)
+    ik = wl.d_I + 4 * (wl.d_I // 64)
     n_h = wl.T // wl.hca_stride
     q = wl.Hq * wl.D * 2
     out = wl.Hq * wl.D * 4 + wl.Hq * 4
     csa = indexer_bytes(wl) + wl.B * ((wl.k + wl.window) * entry + q + out)
     hca = wl.B * ((n_h + wl.window) * entry + q + out)
-    compress = wl.B * ((wl.csa_pool + wl.hca_pool) * entry + 2 * entry
-                       + wl.csa_pool * (wl.d_I + 8) + (wl.d_I + 8))
-    return csa + hca + compress
+    compress = wl.B * ((PERIOD // wl.csa_stride) * (wl.csa_pool * (entry + ik) + entry + ik)
+                       + (PERIOD // wl.hca_stride) * (wl.hca_pool * entry + entry)) / PERIOD
+    return int(csa + hca + compress)
 
 
 def run_ours(args, rank, world, dev):
@@ -219,17 +253,20 @@ def run_ours(args, rank, world, dev):
     per_rep_bytes = step_bytes(wl)
     # enough replicas that one rotation touches > 4x the 126 MB L2 (unless set)
     R = args.replicas if args.replicas > 0 else math.ceil(4 * 126e6 / per_rep_bytes) + 1
-    replicas = [Replica(wl, 1000 + r + 7919 * rank, dev) for r in range(R)]
+    sched = Schedule(wl, dev)
+    replicas = [Replica(wl, sched, 1000 + r + 7919 * rank, dev) for r in range(R)]
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
     # warm-up: W steps eagerly through the public API (also performs the
     # library's one-time kernel attribute set-up outside any graph capture)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            replicas[i % R].step()
+            replicas[i % R].step(i % PERIOD)
     stream.synchronize()
     G = max(1, min(args.graph_steps, args.steps))
     graph = StepGraph(replicas, G, stream)
+    rest = args.steps % G
+    tail = StepGraph(replicas, rest, stream, i0=(args.steps // G) * G) if rest else None
 
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()
@@ -244,18 +281,20 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    n_launch = math.ceil(args.steps / G)
+    n_launch = args.steps // G
     with torch.cuda.stream(stream):
         t0.record(stream)
         for _ in range(n_launch):
             graph.launch()
+        if tail:
+            tail.launch()
         t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
     ms = t0.elapsed_time(t1)
-    steps_done = n_launch * G
+    steps_done = n_launch * G + rest
     if world > 1:
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -281,15 +320,17 @@ def run_ours(args, rank, world, dev):
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3/bf16 storage, fp32 math",
            "data": "synthetic (seeded Gaussian FP8 E4M3 + BF16 caches with needles)",
            "config": {"workload": f"{wl.name}: 1 CSA + 1 HCA layer decode, B={wl.B}/GPU, "
-                                  f"ctx={wl.T}, Hq={wl.Hq}, D={wl.d_nope}+{wl.d_rope}, "
-                                  f"H_I={wl.H_I}x{wl.d_I}, k={wl.k}, window={wl.window}",
+                                  f"ctx {sched.T0 + 1}..{sched.T0 + PERIOD} (128-token window "
+                                  f"around {wl.T}: 32 CSA + 1 HCA compressions), Hq={wl.Hq}, "
+                                  f"D={wl.d_nope}+{wl.d_rope}, H_I={wl.H_I}x{wl.d_I}, k={wl.k}, "
+                                  f"window={wl.window}",
                       "global_batch": wl.B * world, "seq_len": wl.T,
                       "parallelism": f"replicas x{world} (weak)",
                       "l2": f"{R} rotating input replicas, {R * per_rep_bytes / 1e6:.0f} MB "
                             f"touched per cycle (> 4x L2)",
                       "step_bytes": per_rep_bytes},
            "roofline": roofline,
-           "gpu_launches": graph.kernels * n_launch,
+           "gpu_launches": graph.kernels * n_launch + (tail.kernels if tail else 0),
            "clocks": clocks}
     return res, replicas, wl
 
@@ -319,37 +360,46 @@ def _profile_traffic(workload):
 
 def run_e2e(args, replicas, wl, dev, world):
     """Same metric through the public API with per-step host<->device copies:
-    the new token's raw KV and indexer key, q, the indexer query, head weights
-    and positions go in from pinned host memory; out and lse come back."""
+    the new token's raw KV and indexer key (into their ring slots), q, the
+    indexer query and scales, head weights and the step's positions go in from
+    pinned host memory; out and lse of both layers come back."""
     K = max(3, min(args.steps, args.e2e_steps))
     rep = replicas[0]
+    sc = rep.sched
     cl, hl = rep.csa_L, rep.hca_L
-    ins = []
-    slot = (wl.T - 1) % cl["ring_k"]["cap"]
-    for Ld in (cl, hl):
-        for key in ("data", "scale", "rope"):
-            ins.append(Ld["ring_k"][key][:, slot])
-        ins.append(Ld["q"])
-    ins += [cl["ring_ik"]["data"][:, slot], cl["ring_ik"]["scale"][:, slot], cl["q_ik"],
-            cl["q_ik_scale"], cl["head_w"], cl["q_pos"], cl["ctx_len"], hl["ctx_len"],
-            rep.t_begin, rep.t_end]
-    host_in = [t.detach().cpu().pin_memory() for t in ins]
+    cap = cl["ring_k"]["cap"]
+
+    def step_inputs(s):
+        p = sc.T0 + s
+        slot = p % cap
+        ins = []
+        for Ld in (cl, hl):
+            for key in ("data", "scale", "rope"):
+                ins.append(Ld["ring_k"][key][:, slot])
+            ins.append(Ld["q"])
+        ins += [cl["ring_ik"]["data"][:, slot], cl["ring_ik"]["scale"][:, slot], cl["q_ik"],
+                cl["q_ik_scale"], cl["head_w"], sc.q_pos[s], sc.ctx[s], sc.tb[s], sc.te[s]]
+        return ins
+
+    dev_in = [step_inputs(s) for s in range(PERIOD)]
+    host_in = [[t.detach().cpu().pin_memory() for t in ins] for ins in dev_in]
     outs = [rep.csa.out, rep.csa.lse, rep.hca.out, rep.hca.lse]
     host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    bi = sum(t.numel() * t.element_size() for t in host_in)
+    bi = sum(t.numel() * t.element_size() for t in host_in[0])
     bo = sum(t.numel() * t.element_size() for t in host_out)
     stream = torch.cuda.Stream(device=dev)
 
-    def one():
-        for d, h in zip(ins, host_in):
+    def one(i):
+        s = i % PERIOD
+        for d, h in zip(dev_in[s], host_in[s]):
             d.copy_(h, non_blocking=True)
-        rep.step()
+        rep.step(s)
         for h, d in zip(host_out, outs):
             h.copy_(d, non_blocking=True)
 
     with torch.cuda.stream(stream):
-        for _ in range(3):
-            one()
+        for i in range(3):
+            one(i)
     stream.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -357,8 +407,8 @@ def run_e2e(args, replicas, wl, dev, world):
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for _ in range(K):
-            one()
+        for i in range(K):
+            one(i)
         e1.record(stream)
     stream.synchronize()
     ms = e0.elapsed_time(e1)
@@ -368,7 +418,7 @@ def run_e2e(args, replicas, wl, dev, world):
         ms = float(t.item())
     return {"value": round(wl.B * K * world / (ms / 1e3), 2), "unit": UNIT,
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": K,
-            "path": "eager public API calls (no graph), single replica"}
+            "path": "eager public API calls (no graph), single replica, same decode window"}
 
 
 # ------------------------------------------------------------- the oracle
@@ -494,7 +544,7 @@ def main():
     ap.add_argument("--workload", default="long")
     ap.add_argument("--replicas", type=int, default=0,
                     help="input replicas to rotate (0: enough to exceed 4x L2)")
-    ap.add_argument("--graph-steps", type=int, default=250)
+    ap.add_argument("--graph-steps", type=int, default=PERIOD)
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -50,25 +50,30 @@ class CSALayer:
                      L["gate_w"], L["gate_b"], L["pool"], L["stride"], L["comp_k"], L["comp_v"],
                      L["comp_ik"])
 
-    def select(self):
+    def select(self, q_pos=None):
+        """indexer_topk; q_pos [B][Tq] (device) overrides the layer's positions."""
         L, wl = self.L, self.wl
-        indexer_topk(self.B, self.Tq, L["q_pos"], L["q_ik"], L["q_ik_scale"], L["head_w"],
+        q_pos = L["q_pos"] if q_pos is None else q_pos
+        indexer_topk(self.B, self.Tq, q_pos, L["q_ik"], L["q_ik_scale"], L["head_w"],
                      wl.H_I, wl.d_I, L["comp_ik"], L["stride"], self.k, self.max_entries,
                      self.idx, self.score, self.ws_idx)
         return self.idx
 
-    def attend(self, sel=None):
+    def attend(self, sel=None, pos=None):
+        """Hybrid attention over `sel` (default: the last selection); pos
+        overrides q_pos (prefill) or ctx_len (decode)."""
         L, wl = self.L, self.wl
         sel = self.idx if sel is None else sel
         if wl.prefill:
-            hybrid_attn_prefill(self.B, self.Tq, L["q_pos"], L["q"], self.Hq, wl.sm_scale,
-                                L["comp_k"], L["comp_v"], L["stride"], sel, self.k, self.k,
-                                L["ring_k"], L["ring_v"], wl.window, self.out, self.lse,
-                                self.ws_attn)
+            hybrid_attn_prefill(self.B, self.Tq, L["q_pos"] if pos is None else pos, L["q"],
+                                self.Hq, wl.sm_scale, L["comp_k"], L["comp_v"], L["stride"], sel,
+                                self.k, self.k, L["ring_k"], L["ring_v"], wl.window, self.out,
+                                self.lse, self.ws_attn)
         else:
-            hybrid_attn_decode(self.B, L["ctx_len"], L["q"], self.Hq, wl.sm_scale, L["comp_k"],
-                               L["comp_v"], L["stride"], sel, self.k, self.k, L["ring_k"],
-                               L["ring_v"], wl.window, self.out, self.lse, self.ws_attn)
+            hybrid_attn_decode(self.B, L["ctx_len"] if pos is None else pos, L["q"], self.Hq,
+                               wl.sm_scale, L["comp_k"], L["comp_v"], L["stride"], sel, self.k,
+                               self.k, L["ring_k"], L["ring_v"], wl.window, self.out, self.lse,
+                               self.ws_attn)
         return self.out, self.lse
 
     def step(self):
@@ -98,19 +103,21 @@ class HCALayer:
         hca_compress(self.B, t_begin, t_end, max_new, L["ring_k"], L["ring_v"], L["gate_w"],
                      L["gate_b"], L["pool"], L["stride"], L["comp_k"], L["comp_v"])
 
-    def attend(self):
+    def attend(self, pos=None):
+        """Dense hybrid attention; pos overrides q_pos (prefill) or ctx_len (decode)."""
         L, wl = self.L, self.wl
         ck = L["comp_k"] if self.dense else None
         cv = L["comp_v"] if self.dense else None
         me = self.max_entries if self.dense else 0
         if wl.prefill:
-            hybrid_attn_prefill(self.B, self.Tq, L["q_pos"], L["q"], self.Hq, wl.sm_scale, ck, cv,
-                                L["stride"], None, 0, me, L["ring_k"], L["ring_v"], wl.window,
-                                self.out, self.lse, self.ws_attn)
+            hybrid_attn_prefill(self.B, self.Tq, L["q_pos"] if pos is None else pos, L["q"],
+                                self.Hq, wl.sm_scale, ck, cv, L["stride"], None, 0, me,
+                                L["ring_k"], L["ring_v"], wl.window, self.out, self.lse,
+                                self.ws_attn)
         else:
-            hybrid_attn_decode(self.B, L["ctx_len"], L["q"], self.Hq, wl.sm_scale, ck, cv,
-                               L["stride"], None, 0, me, L["ring_k"], L["ring_v"], wl.window,
-                               self.out, self.lse, self.ws_attn)
+            hybrid_attn_decode(self.B, L["ctx_len"] if pos is None else pos, L["q"], self.Hq,
+                               wl.sm_scale, ck, cv, L["stride"], None, 0, me, L["ring_k"],
+                               L["ring_v"], wl.window, self.out, self.lse, self.ws_attn)
         return self.out, self.lse
 
     step = attend
