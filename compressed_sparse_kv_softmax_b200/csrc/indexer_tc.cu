@@ -50,12 +50,34 @@ constexpr uint32_t kIdesc = idesc(kFmtE4M3, kFmtE4M3, 0, 0, kTile, kHeads);
 struct __align__(1024) Smem {
   uint8_t keys[kStages][kTileBytes];      // 1024-aligned tiles
   uint8_t q[kHeads * kDim];               // B operand, K-major, 128-byte swizzle
-  float4 qc[kHeads];                      // (sq0, sq1, w, 0) per head
+  float c0[kHeads], c1[kHeads], w[kHeads]; // per head: block-0 and block-1 query scale, weight
   uint32_t hist[kTopkBins];
   uint64_t full[kStages], empty[kStages], acc_full[kAcc], acc_empty[kAcc], mma_done;
   uint32_t tmem_base;
   int abort;
 };
+
+// packed fp32 pairs (sm_100 f32x2 arithmetic)
+__device__ __forceinline__ unsigned long long f2u(float2 v) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+  return r;
+}
+__device__ __forceinline__ float2 u2f(unsigned long long r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(r);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2u(a)), "l"(f2u(b)), "l"(f2u(c)));
+  return u2f(r);
+}
 
 __device__ __forceinline__ void record_abort(Smem &sm, int *err, int code) {
   sm.abort = 1;
@@ -93,26 +115,31 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
-  // query heads -> B operand (K-major, 128-byte swizzle: 16-byte chunk c of
-  // head h lands at chunk c ^ (h & 7) of its 128-byte row)
-  {
+  tc_fence_before();
+  __syncthreads();                 // barriers initialised, TMEM address published
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (warp != 0) {
+    // query heads -> B operand (K-major, 128-byte swizzle: 16-byte chunk c of
+    // head h lands at chunk c ^ (h & 7) of its 128-byte row); the producer
+    // warp streams keys meanwhile
+    const int t = tid - 32, nt = kThreads - 32;
     const uint8_t *qsrc = reinterpret_cast<const uint8_t *>(a.q_ik) + (size_t)row * kHeads * kDim;
-    for (int i = tid; i < kHeads * kDim / 16; i += kThreads) {
+    for (int i = t; i < kHeads * kDim / 16; i += nt) {
       const int h = i >> 3, c = i & 7;
       const uint4 v = *reinterpret_cast<const uint4 *>(qsrc + h * kDim + c * 16);
       *reinterpret_cast<uint4 *>(&sm.q[h * kDim + ((c ^ (h & 7)) << 4)]) = v;
     }
-    for (int h = tid; h < kHeads; h += kThreads) {
+    for (int h = t; h < kHeads; h += nt) {
       const float *qs = a.q_ik_scale + ((size_t)row * kHeads + h) * 2;
-      sm.qc[h] = make_float4(qs[0], qs[1], a.head_w[(size_t)row * kHeads + h], 0.f);
+      sm.c0[h] = qs[0];
+      sm.c1[h] = qs[1];
+      sm.w[h] = a.head_w[(size_t)row * kHeads + h];
     }
-    for (int i = tid; i < kTopkBins; i += kThreads) sm.hist[i] = 0;
+    for (int i = t; i < kTopkBins; i += nt) sm.hist[i] = 0;
+    fence_proxy_async_shared();
+    asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");   // all warps but the producer
   }
-  fence_proxy_async_shared();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -190,7 +217,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       }
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * 128;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      const float2 k0 = make_float2(sk0, sk0), k1 = make_float2(sk1, sk1);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         float a0[32], a1[32];
@@ -204,16 +232,22 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
         }
 #pragma unroll
         for (int h = 0; h < 32; h += 4) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float4 c = sm.qc[half * 32 + h + u];
-            const float x = fmaf(a0[h + u] * c.x, sk0, (a1[h + u] * c.y) * sk1);
-            const float t = c.z * fmaxf(x, 0.f);
-            if (u == 0) s0 += t; else if (u == 1) s1 += t; else if (u == 2) s2 += t; else s3 += t;
-          }
+          const int hg = half * 32 + h;
+          const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
+          const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
+          const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
+          // x = sk0 sq0 a0 + sk1 sq1 a1 for heads (h, h+1) and (h+2, h+3)
+          float2 x = fma2(mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)), k0,
+                          mul2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), k1));
+          float2 y = fma2(mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)), k0,
+                          mul2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), k1));
+          x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
+          y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
+          acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
+          acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
         }
       }
-      const float sc = (s0 + s1) + (s2 + s3);
+      const float sc = (acc0.x + acc0.y) + (acc1.x + acc1.y);
       if (j < n) {
         srow[j] = sc;
         atomicAdd(&sm.hist[score_key(sc) >> kTopkShift], 1u);

@@ -423,18 +423,29 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
           atomicOr(&bits[j >> 5], 1u << (j & 31));
         }
         __syncthreads();
-        const int per_t = (nw + blockDim.x - 1) / blockDim.x;
-        const int w0 = tid * per_t;
+        // warp w owns words [w * span, (w + 1) * span), read lane-contiguous
+        // (conflict-free); a warp scan inside, a block scan across warps
+        const int nwarps = blockDim.x >> 5, warp = tid >> 5;
+        const int span = (((nw + nwarps - 1) / nwarps) + 31) & ~31;
+        const int wb = warp * span;
         int cnt = 0;
-        for (int i = 0; i < per_t; ++i)
-          if (w0 + i < nw) cnt += __popc(bits[w0 + i]);
+        for (int i = lane; i < span; i += 32)
+          if (wb + i < nw) cnt += __popc(bits[wb + i]);
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
         int tot;
-        int run = block_exclusive_scan(cnt, sm.scan, &tot);
-        for (int i = 0; i < per_t; ++i) {
-          if (w0 + i < nw) {
-            wpre[w0 + i] = (uint32_t)run;
-            run += __popc(bits[w0 + i]);
+        int run = block_exclusive_scan(lane == 0 ? cnt : 0, sm.scan, &tot);
+        run = __shfl_sync(0xffffffffu, run, 0);
+        for (int i0 = 0; i0 < span; i0 += 32) {
+          const int wi = wb + i0 + lane;
+          const int c = wi < nw ? __popc(bits[wi]) : 0;
+          int incl = c;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
           }
+          if (wi < nw) wpre[wi] = (uint32_t)(run + incl - c);
+          run += __shfl_sync(0xffffffffu, incl, 31);
         }
         __syncthreads();
         for (int i = tid; i < k; i += blockDim.x) {
