@@ -91,6 +91,7 @@ int attention_common(int B, int Tq, const int64_t *pos, int pos_is_ctx_len, cons
                      float *lse, void *ws, size_t ws_bytes, cskv_stream_t stream) {
   if (B < 0 || Tq < 0 || (int64_t)B * Tq > 0x7fffffffLL) return CSKV_ERR_ARG;
   if (Hq < 1 || Hq > 65535 || window < 1) return CSKV_ERR_ARG;
+  if ((int64_t)B * Tq * Hq > 0x7fffffffLL) return CSKV_ERR_ARG;
   if (B == 0 || Tq == 0) return CSKV_OK;
   if (!pos || !q || !out || !lse || !aligned16(q)) return CSKV_ERR_ARG;
   CSKV_TRY(check_cache(win_k, 1));

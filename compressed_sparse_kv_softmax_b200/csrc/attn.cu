@@ -23,14 +23,15 @@
 namespace cskv {
 
 bool attn_tc_supported(const AttnArgs &a);
-int launch_attn_tc(const AttnArgs &a, float *part_o, float *part_lse, int n_chunks,
+int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *part_lse,
                    cudaStream_t st);
-int attn_tc_chunk_keys();
+int attn_tc_unit_keys();
 
 namespace {
 
-constexpr int kChunk = 32;        // keys per CTA in the CUDA-core path
+constexpr int kChunk = 32;        // keys per unit in the CUDA-core path (one per lane)
 constexpr int kThreads = 256;
+constexpr int kTargetCtas = 296;  // splits aim at two CTAs per SM of a 148-SM part
 
 struct RowInfo {
   long long pos;          // query position
@@ -57,97 +58,121 @@ __device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int row) {
   return r;
 }
 
+// CUDA-core path: a split runs its units (kChunk keys each) with an online
+// softmax, the running output in shared memory.
 __global__ void __launch_bounds__(kThreads)
-attn_chunk_kernel(AttnArgs a, int n_comp_chunks, int n_chunks, float *__restrict__ part_o,
+attn_units_kernel(AttnArgs a, AttnPlan p, float *__restrict__ part_o,
                   float *__restrict__ part_lse) {
   extern __shared__ float sm[];
+  pdl_wait();
+  pdl_trigger();
   const int Hq = a.Hq, D = a.D, Dv = a.Dv;
   const bool sep_v = a.win_v.data != nullptr;
-  float *q = sm;                          // [Hq][D]
-  float *kt = q + Hq * D;                 // [kChunk][D+1]
+  float *q = sm;                                    // [Hq][D]
+  float *kt = q + Hq * D;                           // [kChunk][D+1]
   float *vt = sep_v ? kt + kChunk * (D + 1) : kt;   // [kChunk][Dv+1]
-  float *p = (sep_v ? vt + kChunk * (Dv + 1) : kt + kChunk * (D + 1));  // [Hq][kChunk]
+  float *pt = (sep_v ? vt + kChunk * (Dv + 1) : kt + kChunk * (D + 1));  // [Hq][kChunk]
+  float *o = pt + Hq * kChunk;                      // [Hq][Dv] running output
+  float *mrun = o + Hq * Dv, *lrun = mrun + Hq, *alpha = lrun + Hq;
   __shared__ long long key_slot[kChunk];
-  __shared__ int key_src[kChunk];         // 0 none, 1 compressed, 2 window
+  __shared__ int key_src[kChunk];                   // 0 none, 1 compressed, 2 window
 
-  const int row = blockIdx.y, chunk = blockIdx.x;
+  const int row = blockIdx.x, split = blockIdx.y;
   const int b = row / a.Tq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const RowInfo ri = row_info(a, row);
-
-  if (tid < kChunk) {
-    int src = 0;
-    long long slot = 0;
-    if (chunk < n_comp_chunks) {
-      const long long i = (long long)chunk * kChunk + tid;
-      if (i < ri.n_comp) {
-        long long j = a.sel ? (long long)a.sel[(long long)row * a.k + i] : i;
-        if (j >= 0 && j < a.comp_k.cap && j < a.comp_v.cap) { src = 1; slot = j; }
-      }
-    } else {
-      const long long i = (long long)(chunk - n_comp_chunks) * kChunk + tid;
-      if (i < ri.n_win) { src = 2; slot = a.win_k.slot_of(ri.w_lo + i); }
-    }
-    key_src[tid] = src;
-    key_slot[tid] = slot;
-  }
-  // query row -> fp32
   const long long qoff = (long long)row * Hq * D;
   for (int i = tid; i < Hq * D; i += kThreads) {
     q[i] = a.win_k.fmt == CSKV_FMT_F32
                ? reinterpret_cast<const float *>(a.q)[qoff + i]
                : __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(a.q)[qoff + i]);
   }
-  __syncthreads();
-  for (int i = tid; i < kChunk * D; i += kThreads) {
-    const int r = i / D, d = i % D;
-    const int src = key_src[r];
-    float v = 0.f;
-    if (src == 1) v = a.comp_k.value(b, key_slot[r], d);
-    else if (src == 2) v = a.win_k.value(b, key_slot[r], d);
-    kt[r * (D + 1) + d] = v;
+  for (int i = tid; i < Hq * Dv; i += kThreads) o[i] = 0.f;
+  for (int h = tid; h < Hq; h += kThreads) {
+    mrun[h] = -CUDART_INF_F;
+    lrun[h] = 0.f;
   }
-  if (sep_v) {
-    for (int i = tid; i < kChunk * Dv; i += kThreads) {
-      const int r = i / Dv, d = i % Dv;
+  const int u_begin = split * p.per_cta;
+  const int u_end = min(p.n_units, u_begin + p.per_cta);
+  for (int unit = u_begin; unit < u_end; ++unit) {
+    if (tid < kChunk) {
+      int src = 0;
+      long long slot = 0;
+      if (unit < p.n_comp_units) {
+        const long long i = (long long)unit * kChunk + tid;
+        if (i < ri.n_comp) {
+          const long long j = a.sel ? (long long)a.sel[(long long)row * a.k + i] : i;
+          if (j >= 0 && j < a.comp_k.cap && j < a.comp_v.cap) { src = 1; slot = j; }
+        }
+      } else {
+        const long long i = (long long)(unit - p.n_comp_units) * kChunk + tid;
+        if (i < ri.n_win) { src = 2; slot = a.win_k.slot_of(ri.w_lo + i); }
+      }
+      key_src[tid] = src;
+      key_slot[tid] = slot;
+    }
+    __syncthreads();
+    for (int i = tid; i < kChunk * D; i += kThreads) {
+      const int r = i / D, d = i % D;
       const int src = key_src[r];
       float v = 0.f;
-      if (src == 1) v = a.comp_v.value(b, key_slot[r], d);
-      else if (src == 2) v = a.win_v.value(b, key_slot[r], d);
-      vt[r * (Dv + 1) + d] = v;
+      if (src == 1) v = a.comp_k.value(b, key_slot[r], d);
+      else if (src == 2) v = a.win_k.value(b, key_slot[r], d);
+      kt[r * (D + 1) + d] = v;
     }
-  }
-  __syncthreads();
-  // logits: warp <-> head, lane <-> key
-  for (int h = warp; h < Hq; h += kThreads / 32) {
-    float l = -CUDART_INF_F;
-    if (key_src[lane]) {
-      const float *qh = q + h * D;
-      const float *kr = kt + lane * (D + 1);
-      float dot = 0.f;
-      for (int d = 0; d < D; ++d) dot = fmaf(qh[d], kr[d], dot);
-      l = a.sm_scale * dot;
+    if (sep_v) {
+      for (int i = tid; i < kChunk * Dv; i += kThreads) {
+        const int r = i / Dv, d = i % Dv;
+        const int src = key_src[r];
+        float v = 0.f;
+        if (src == 1) v = a.comp_v.value(b, key_slot[r], d);
+        else if (src == 2) v = a.win_v.value(b, key_slot[r], d);
+        vt[r * (Dv + 1) + d] = v;
+      }
     }
-    const float m = warp_max(l);
-    const float e = (m == -CUDART_INF_F || l == -CUDART_INF_F) ? 0.f : expf(l - m);
-    const float s = warp_sum(e);
-    p[h * kChunk + lane] = s > 0.f ? e / s : 0.f;
-    if (lane == 0)
-      part_lse[((long long)row * n_chunks + chunk) * Hq + h] =
-          s > 0.f ? m + logf(s) : -CUDART_INF_F;
-  }
-  __syncthreads();
-  // partial output o_h = sum_c p[h][c] V[c]
-  const int vstride = sep_v ? Dv + 1 : D + 1;
-  float *po = part_o + ((long long)row * n_chunks + chunk) * Hq * Dv;
-  for (int i = tid; i < Hq * Dv; i += kThreads) {
-    const int h = i / Dv, d = i % Dv;
-    const float *ph = p + h * kChunk;
-    float acc = 0.f;
+    __syncthreads();
+    // logits and softmax update: warp <-> head, lane <-> key
+    for (int h = warp; h < Hq; h += kThreads / 32) {
+      float l = -CUDART_INF_F;
+      if (key_src[lane]) {
+        const float *qh = q + h * D;
+        const float *kr = kt + lane * (D + 1);
+        float dot = 0.f;
+        for (int d = 0; d < D; ++d) dot = fmaf(qh[d], kr[d], dot);
+        l = a.sm_scale * dot;
+      }
+      const float mold = mrun[h];
+      const float mnew = fmaxf(mold, warp_max(l));
+      const float e = l == -CUDART_INF_F ? 0.f : expf(l - mnew);
+      const float s = warp_sum(e);
+      pt[h * kChunk + lane] = e;
+      if (lane == 0) {
+        const float al = mold == -CUDART_INF_F ? 0.f : expf(mold - mnew);
+        alpha[h] = al;
+        lrun[h] = lrun[h] * al + s;
+        mrun[h] = mnew;
+      }
+    }
+    __syncthreads();
+    const int vstride = sep_v ? Dv + 1 : D + 1;
+    for (int i = tid; i < Hq * Dv; i += kThreads) {
+      const int h = i / Dv, d = i % Dv;
+      const float *ph = pt + h * kChunk;
+      float acc = o[i] * alpha[h];
 #pragma unroll 8
-    for (int c = 0; c < kChunk; ++c) acc = fmaf(ph[c], vt[c * vstride + d], acc);
-    po[i] = acc;
+      for (int c = 0; c < kChunk; ++c) acc = fmaf(ph[c], vt[c * vstride + d], acc);
+      o[i] = acc;
+    }
+    __syncthreads();
   }
+  float *po = part_o + ((long long)row * p.splits + split) * Hq * Dv;
+  for (int i = tid; i < Hq * Dv; i += kThreads) {
+    const float l = lrun[i / Dv];
+    po[i] = l > 0.f ? o[i] / l : 0.f;
+  }
+  for (int h = tid; h < Hq; h += kThreads)
+    part_lse[((long long)row * p.splits + split) * Hq + h] =
+        lrun[h] > 0.f ? mrun[h] + logf(lrun[h]) : -CUDART_INF_F;
 }
 
 // out[row][h][:] = sum_i e^{lse_i - L} o_i,  lse[row][h] = L = log sum_i e^{lse_i}
@@ -161,6 +186,8 @@ attn_merge_kernel(int Hq, int Dv, int n_chunks, const float *__restrict__ part_o
                   float *__restrict__ lse) {
   extern __shared__ float wts[];          // [n_chunks]
   __shared__ float red[kMergeGroups][kMergeD];
+  pdl_wait();
+  pdl_trigger();
   __shared__ float s_L;
   const int row = blockIdx.x / Hq, h = blockIdx.x % Hq;
   const int tid = threadIdx.x, grp = tid / kMergeD, dl = tid % kMergeD;
@@ -203,50 +230,70 @@ attn_merge_kernel(int Hq, int Dv, int n_chunks, const float *__restrict__ part_o
   if (blockIdx.y == 0 && tid == 0) lse[(long long)row * Hq + h] = s_L;
 }
 
-int chunk_keys(const AttnArgs &a) { return attn_tc_supported(a) ? attn_tc_chunk_keys() : kChunk; }
-
 }  // namespace
 
-static void plan_chunks(long long max_comp, int window, int chunk, int *n_comp_chunks,
-                        int *n_chunks) {
-  *n_comp_chunks = (int)((max_comp + chunk - 1) / chunk);
-  *n_chunks = *n_comp_chunks + (window + chunk - 1) / chunk;
+AttnPlan attn_plan(long long rows, long long max_comp, int window, int unit) {
+  AttnPlan p;
+  p.unit = unit;
+  p.n_comp_units = (int)((max_comp + unit - 1) / unit);
+  p.n_units = p.n_comp_units + (window + unit - 1) / unit;
+  long long splits = (kTargetCtas + rows - 1) / rows;
+  if (splits > p.n_units) splits = p.n_units;
+  if (splits < 1) splits = 1;
+  p.per_cta = (int)((p.n_units + splits - 1) / splits);
+  p.splits = (p.n_units + p.per_cta - 1) / p.per_cta;
+  return p;
+}
+
+static size_t partial_bytes(const AttnPlan &p, long long rows, int Hq, int Dv) {
+  if (p.splits <= 1) return 0;   // one split per row writes the output directly
+  return (size_t)rows * p.splits * Hq * ((size_t)Dv + 1) * sizeof(float) + 512;
 }
 
 size_t attn_ws_bytes(int B, int Tq, int Hq, int Dv, long long max_entries, int window) {
-  // sized for the smaller chunk of the two paths (more partials)
-  int ncc, nc;
-  plan_chunks(max_entries, window, kChunk, &ncc, &nc);
-  const size_t rows = (size_t)B * Tq;
-  return rows * nc * Hq * ((size_t)Dv + 1) * sizeof(float) + 512;
+  // either path may run: the larger of the two plans
+  const long long rows = (long long)B * Tq;
+  const size_t a = partial_bytes(attn_plan(rows, max_entries, window, kChunk), rows, Hq, Dv);
+  const size_t b =
+      partial_bytes(attn_plan(rows, max_entries, window, attn_tc_unit_keys()), rows, Hq, Dv);
+  return a > b ? a : b;
 }
 
 int launch_attention(const AttnArgs &a, cudaStream_t st) {
   const int rows = a.B * a.Tq;
   if (rows == 0) return CSKV_OK;
-  const int chunk = chunk_keys(a);
-  int ncc, nc;
-  plan_chunks(a.has_comp ? (a.sel ? a.k : a.max_entries) : 0, a.window, chunk, &ncc, &nc);
-  float *part_o = reinterpret_cast<float *>(a.ws);
-  float *part_lse = part_o + (size_t)rows * nc * a.Hq * a.Dv;
-  part_lse = reinterpret_cast<float *>(((uintptr_t)part_lse + 255) & ~(uintptr_t)255);
-  if (attn_tc_supported(a)) {
-    const int rc = launch_attn_tc(a, part_o, part_lse, nc, st);
+  const bool tc = attn_tc_supported(a);
+  const long long max_comp = a.has_comp ? (a.sel ? a.k : a.max_entries) : 0;
+  const AttnPlan p = attn_plan(rows, max_comp, a.window, tc ? attn_tc_unit_keys() : kChunk);
+  const bool direct = p.splits == 1;
+  float *part_o = direct ? a.out : reinterpret_cast<float *>(a.ws);
+  float *part_lse = a.lse;
+  if (!direct) {
+    part_lse = part_o + (size_t)rows * p.splits * a.Hq * a.Dv;
+    part_lse = reinterpret_cast<float *>(((uintptr_t)part_lse + 255) & ~(uintptr_t)255);
+  }
+  if (tc) {
+    const int rc = launch_attn_tc(a, p, part_o, part_lse, st);
     if (rc != CSKV_OK) return rc;
   } else {
     const bool sep_v = a.win_v.data != nullptr;
     const size_t smem = sizeof(float) * ((size_t)a.Hq * a.D + (size_t)kChunk * (a.D + 1) +
                                          (sep_v ? (size_t)kChunk * (a.Dv + 1) : 0) +
-                                         (size_t)a.Hq * kChunk);
-    if (!ensure_dynamic_smem(attn_chunk_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
-    attn_chunk_kernel<<<dim3(nc, rows), kThreads, smem, st>>>(a, ncc, nc, part_o, part_lse);
-    if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
+                                         (size_t)a.Hq * kChunk + (size_t)a.Hq * a.Dv +
+                                         3 * (size_t)a.Hq);
+    if (!ensure_dynamic_smem(attn_units_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+    if (launch_pdl(attn_units_kernel, dim3(rows, p.splits), dim3(kThreads), smem, st, a, p,
+                   part_o, part_lse) != cudaSuccess)
+      return CSKV_ERR_CUDA;
   }
-  const size_t msmem = sizeof(float) * nc;
+  if (direct) return CSKV_OK;
+  const size_t msmem = sizeof(float) * p.splits;
   if (!ensure_dynamic_smem(attn_merge_kernel, msmem)) return CSKV_ERR_UNSUPPORTED;
-  attn_merge_kernel<<<dim3((unsigned)(rows * a.Hq), (a.Dv + kMergeD - 1) / kMergeD), kMergeD * kMergeGroups,
-                      msmem, st>>>(a.Hq, a.Dv, nc, part_o, part_lse, a.out, a.lse);
-  return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
+  if (launch_pdl(attn_merge_kernel, dim3((unsigned)(rows * a.Hq), (a.Dv + kMergeD - 1) / kMergeD),
+                 dim3(kMergeD * kMergeGroups), msmem, st, a.Hq, a.Dv, p.splits,
+                 (const float *)part_o, (const float *)part_lse, a.out, a.lse) != cudaSuccess)
+    return CSKV_ERR_CUDA;
+  return CSKV_OK;
 }
 
 }  // namespace cskv

@@ -66,7 +66,7 @@ struct __align__(1024) Smem {
   uint8_t phi[kKeys * 128];         // 8 KB: P^T hi, MN-major [keys][64 heads]
   uint8_t plo[kKeys * 128];         // 8 KB
   float red[4][kHeads];
-  float m[kHeads], l[kHeads], inv_l[kHeads];
+  float m[kHeads], l[kHeads], inv_l[kHeads], alpha[kHeads];
   long long slot[kM];
   uint64_t bar;
   uint32_t tmem_base;
@@ -141,15 +141,14 @@ __device__ __forceinline__ Row row_of(const AttnArgs &a, int row) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
-               float *__restrict__ part_o, float *__restrict__ part_lse) {
+attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, int units_per_cta,
+               int n_splits, float *__restrict__ part_o, float *__restrict__ part_lse) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row = blockIdx.y, unit = blockIdx.x;
+  const int row = blockIdx.x, split = blockIdx.y;
   const int b = row / a.Tq;
-  const Row R = row_of(a, row);
 
   if (tid == 0) {
     mbar_init(&sm.bar, 1);
@@ -159,6 +158,14 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
+  if (tid < kHeads) {
+    sm.m[tid] = -CUDART_INF_F;
+    sm.l[tid] = 0.f;
+  }
+
+  pdl_wait();                      // global memory from here on
+  pdl_trigger();
+  const Row R = row_of(a, row);
 
   // ---- Q: BF16 -> FP16, K-major swizzled
   {
@@ -191,114 +198,118 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
     }
   }
 
-  // ---- resolve this unit's key slots (one per thread), then gather
-  const bool comp_unit = unit < n_comp_units;
-  const long long base = comp_unit ? (long long)unit * unit_keys
-                                   : (long long)(unit - n_comp_units) * unit_keys;
-  const long long avail = comp_unit ? R.n_comp - base : (long long)R.n_win - base;
-  const int nkeys = (int)(avail < 0 ? 0 : (avail < unit_keys ? avail : unit_keys));
-  const int ksteps = (nkeys + 15) >> 4;            // 16-key MMA steps of the P V product
-  const Cache &src = comp_unit ? a.comp_k : a.win_k;
-  if (tid < kM) {
-    long long slot = -1;
-    if (tid < nkeys) {          // nkeys <= kKeys: rows kKeys..kM-1 stay invalid
-      const long long i = base + tid;
-      if (comp_unit) {
-        const long long j = a.sel ? (long long)a.sel[(long long)row * a.k + i] : i;
-        if (j >= 0 && j < src.cap) slot = j;
-      } else {
-        slot = src.slot_of(R.w_lo + i);
-      }
-    }
-    sm.slot[tid] = slot;
-  }
-  // (the barrier also publishes the slots) any key at all in this unit?
-  const bool any = __syncthreads_or(tid < kM && sm.slot[tid] >= 0) != 0;
   const int quad = warp & 3, colh = warp >> 2;      // TMEM lane quadrant, head half
   const int krow = tid & 127;                       // key row = TMEM lane of this thread
-  const bool my_valid = sm.slot[krow] >= 0;
-  // each warp converts 8 consecutive key rows per batch, loads first
-  for (int r0 = warp * 8; r0 < ksteps * 16; r0 += 8 * kThreads / 32) {
-    uint4 raw[8], raw2[8];
-    float sc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const long long slot = sm.slot[r0 + e];
-      raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
-      sc[e] = 0.f;
-      if (slot < 0) continue;
-      if (lane < 28) {
-        raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
-        sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
-      } else {
-        const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
-        raw[e] = __ldg(rp);
-        raw2[e] = __ldg(rp + 1);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int r = r0 + e;
-      uint4 h0, h1, l0, l1;
-      uint32_t *ph0 = reinterpret_cast<uint32_t *>(&h0), *ph1 = reinterpret_cast<uint32_t *>(&h1);
-      uint32_t *pl0 = reinterpret_cast<uint32_t *>(&l0), *pl1 = reinterpret_cast<uint32_t *>(&l1);
-      int d0;
-      if (lane < 28) {
-        // 16 FP8 codes: dims 16*lane .. +15, block scale lane/4 (absent key: zeros)
-        const uint32_t *cw = reinterpret_cast<const uint32_t *>(&raw[e]);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 a = e4m3x2(cw[q] & 0xffffu), c = e4m3x2(cw[q] >> 16);
-          if (q < 2) {
-            split_h2(a.x * sc[e], a.y * sc[e], ph0[2 * q], pl0[2 * q]);
-            split_h2(c.x * sc[e], c.y * sc[e], ph0[2 * q + 1], pl0[2 * q + 1]);
-          } else {
-            split_h2(a.x * sc[e], a.y * sc[e], ph1[2 * q - 4], pl1[2 * q - 4]);
-            split_h2(c.x * sc[e], c.y * sc[e], ph1[2 * q - 3], pl1[2 * q - 3]);
-          }
-        }
-        d0 = lane * 16;
-      } else {
-        // 16 BF16 RoPE dims: 448 + 16 * (lane - 28) ..
-        const __nv_bfloat162 *b0 = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
-        const __nv_bfloat162 *b1 = reinterpret_cast<const __nv_bfloat162 *>(&raw2[e]);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f0 = __bfloat1622float2(b0[q]), f1 = __bfloat1622float2(b1[q]);
-          split_h2(f0.x, f0.y, ph0[q], pl0[q]);
-          split_h2(f1.x, f1.y, ph1[q], pl1[q]);
-        }
-        d0 = kDn + (lane - 28) * 16;
-      }
-      const int c = d0 >> 6, u = (d0 & 63) >> 3;
-      const uint32_t o0 = c * kChunkK + swz(r, u), o1 = c * kChunkK + swz(r, u + 1);
-      *reinterpret_cast<uint4 *>(sm.khi + o0) = h0;
-      *reinterpret_cast<uint4 *>(sm.khi + o1) = h1;
-      *reinterpret_cast<uint4 *>(sm.klo + o0) = l0;
-      *reinterpret_cast<uint4 *>(sm.klo + o1) = l1;
-    }
-  }
-  fence_proxy_async_shared();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
-  float *po = part_o + ((size_t)row * n_units + unit) * kHeads * kD;
-  float *pl = part_lse + ((size_t)row * n_units + unit) * kHeads;
+  const uint32_t tmem_tl = ((uint32_t)(quad * 32) << 16);
+  const float c2 = a.sm_scale * 1.4426950408889634f;   // logits in log2 units
+  uint32_t phase = 0;                               // parity of the next completion of sm.bar
+  bool started = false;                             // O^T in TMEM holds a partial sum
+  bool ok = true;
+  uint32_t tmem = 0;
+  const int u_begin = split * units_per_cta;
+  const int u_end = min(n_units, u_begin + units_per_cta);
 
-  if (!any) {
-    // no key in this unit: a partial that the merge weighs with zero
-    for (int i = tid; i < kHeads * kD; i += kThreads) po[i] = 0.f;
-    if (tid < kHeads) pl[tid] = -CUDART_INF_F;
-  } else {
-    // ---- S^T = K Q^T
+  for (int unit = u_begin; unit < u_end; ++unit) {
+    // ---- resolve this unit's key slots (one per thread)
+    const bool comp_unit = unit < n_comp_units;
+    const long long base = comp_unit ? (long long)unit * unit_keys
+                                     : (long long)(unit - n_comp_units) * unit_keys;
+    const long long avail = comp_unit ? R.n_comp - base : (long long)R.n_win - base;
+    const int nkeys = (int)(avail < 0 ? 0 : (avail < unit_keys ? avail : unit_keys));
+    const int ksteps = (nkeys + 15) >> 4;          // 16-key MMA steps of the P V product
+    const Cache &src = comp_unit ? a.comp_k : a.win_k;
+    if (tid < kM) {
+      long long slot = -1;
+      if (tid < nkeys) {        // nkeys <= kKeys: rows kKeys..kM-1 stay invalid
+        const long long i = base + tid;
+        if (comp_unit) {
+          const long long j = a.sel ? (long long)a.sel[(long long)row * a.k + i] : i;
+          if (j >= 0 && j < src.cap) slot = j;
+        } else {
+          slot = src.slot_of(R.w_lo + i);
+        }
+      }
+      sm.slot[tid] = slot;
+    }
+    // (the barrier also publishes the slots) any key at all in this unit?
+    if (!__syncthreads_or(tid < kM && sm.slot[tid] >= 0)) continue;
+    const bool my_valid = sm.slot[krow] >= 0;
+
+    // ---- gather: each warp converts 8 consecutive key rows per batch, loads first
+    for (int r0 = warp * 8; r0 < ksteps * 16; r0 += 8 * kThreads / 32) {
+      uint4 raw[8], raw2[8];
+      float sc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const long long slot = sm.slot[r0 + e];
+        raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
+        sc[e] = 0.f;
+        if (slot < 0) continue;
+        if (lane < 28) {
+          raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
+          sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
+        } else {
+          const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
+          raw[e] = __ldg(rp);
+          raw2[e] = __ldg(rp + 1);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int r = r0 + e;
+        uint4 h0, h1, l0, l1;
+        uint32_t *ph0 = reinterpret_cast<uint32_t *>(&h0), *ph1 = reinterpret_cast<uint32_t *>(&h1);
+        uint32_t *pl0 = reinterpret_cast<uint32_t *>(&l0), *pl1 = reinterpret_cast<uint32_t *>(&l1);
+        int d0;
+        if (lane < 28) {
+          // 16 FP8 codes: dims 16*lane .. +15, block scale lane/4 (absent key: zeros)
+          const uint32_t *cw = reinterpret_cast<const uint32_t *>(&raw[e]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 x = e4m3x2(cw[q] & 0xffffu), y = e4m3x2(cw[q] >> 16);
+            if (q < 2) {
+              split_h2(x.x * sc[e], x.y * sc[e], ph0[2 * q], pl0[2 * q]);
+              split_h2(y.x * sc[e], y.y * sc[e], ph0[2 * q + 1], pl0[2 * q + 1]);
+            } else {
+              split_h2(x.x * sc[e], x.y * sc[e], ph1[2 * q - 4], pl1[2 * q - 4]);
+              split_h2(y.x * sc[e], y.y * sc[e], ph1[2 * q - 3], pl1[2 * q - 3]);
+            }
+          }
+          d0 = lane * 16;
+        } else {
+          // 16 BF16 RoPE dims: 448 + 16 * (lane - 28) ..
+          const __nv_bfloat162 *b0 = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
+          const __nv_bfloat162 *b1 = reinterpret_cast<const __nv_bfloat162 *>(&raw2[e]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f0 = __bfloat1622float2(b0[q]), f1 = __bfloat1622float2(b1[q]);
+            split_h2(f0.x, f0.y, ph0[q], pl0[q]);
+            split_h2(f1.x, f1.y, ph1[q], pl1[q]);
+          }
+          d0 = kDn + (lane - 28) * 16;
+        }
+        const int c = d0 >> 6, u = (d0 & 63) >> 3;
+        const uint32_t o0 = c * kChunkK + swz(r, u), o1 = c * kChunkK + swz(r, u + 1);
+        *reinterpret_cast<uint4 *>(sm.khi + o0) = h0;
+        *reinterpret_cast<uint4 *>(sm.khi + o1) = h1;
+        *reinterpret_cast<uint4 *>(sm.klo + o0) = l0;
+        *reinterpret_cast<uint4 *>(sm.klo + o1) = l1;
+      }
+    }
+    fence_proxy_async_shared();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tmem = sm.tmem_base;
+
+    // ---- S^T = K Q^T  (hi and lo parts of K)
     if (tid == 0) {
       const uint32_t qa = smem_addr(sm.q);
-      for (int part = 0; part < 2; ++part) {          // K_hi Q^T, then + K_lo Q^T
+      for (int part = 0; part < 2; ++part) {
         const uint32_t ka = smem_addr(part ? sm.klo : sm.khi);
 #pragma unroll 4
         for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t off = (ks & 3) << 5;         // 16 dims = 32 bytes per step
+          const uint32_t off = (ks & 3) << 5;       // 16 dims = 32 bytes per step
           mma_f16(tmem, desc_kmajor_sw128(ka + (ks >> 2) * kChunkK + off),
                   desc_kmajor_sw128(qa + (ks >> 2) * kChunkQ + off), kIdescQK,
                   (part | ks) != 0);
@@ -306,14 +317,14 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
       }
       mma_commit(&sm.bar);
     }
-    bool ok = mbar_wait(&sm.bar, 0);
+    ok = mbar_wait(&sm.bar, phase) && ok;
+    phase ^= 1;
     tc_fence_after();
-    // ---- softmax over keys, per head (this thread: key krow, heads 32*colh ..)
+
+    // ---- softmax over this unit's keys with the running per-head max
     float sv[32];
-    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    tmem_ld32(tl + colh * 32, sv);
+    tmem_ld32(tmem + tmem_tl + colh * 32, sv);
     tmem_wait_ld();
-    const float c2 = a.sm_scale * 1.4426950408889634f;   // logits in log2 units
 #pragma unroll
     for (int i = 0; i < 32; ++i) sv[i] = my_valid ? sv[i] * c2 : -CUDART_INF_F;
     {
@@ -323,8 +334,16 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
       sm.red[quad][colh * 32 + lane] = butterfly32<true>(v);
     }
     __syncthreads();
-    if (tid < kHeads)
-      sm.m[tid] = fmaxf(fmaxf(sm.red[0][tid], sm.red[1][tid]), fmaxf(sm.red[2][tid], sm.red[3][tid]));
+    if (tid < kHeads) {
+      // lazy rescaling: keep the running max unless the unit's max exceeds it
+      // by more than 8 (P stays <= 2^8, fine in FP16 hi/lo parts)
+      const float tmax = fmaxf(fmaxf(sm.red[0][tid], sm.red[1][tid]),
+                               fmaxf(sm.red[2][tid], sm.red[3][tid]));
+      const float mold = sm.m[tid];
+      const float mnew = (mold == -CUDART_INF_F || tmax > mold + 8.f) ? tmax : mold;
+      sm.alpha[tid] = mold == -CUDART_INF_F ? 0.f : exp2f(mold - mnew);
+      sm.m[tid] = mnew;
+    }
     __syncthreads();
     {
       float v[32];
@@ -349,15 +368,38 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
       }
       sm.red[quad][colh * 32 + lane] = butterfly32<false>(v);
     }
+    // ---- rescale the running O^T where a head's max moved (rare)
+    if (started) {
+      bool need = false;
+      float al[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        al[i] = sm.alpha[colh * 32 + i];
+        need |= al[i] != 1.f;
+      }
+      if (__syncthreads_or(need)) {
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+          float o[32];
+          const uint32_t ta = tmem + tmem_tl + 64 + mt * 64 + colh * 32;
+          tmem_ld32(ta, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= al[i];
+          tmem_st32(ta, o);
+        }
+        tmem_wait_st();
+      }
+    }
     fence_proxy_async_shared();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid < kHeads) {
-      sm.l[tid] = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
-      sm.inv_l[tid] = 1.f / sm.l[tid];
-    }
-    // ---- O^T = V^T P^T
+    if (tid < kHeads)
+      sm.l[tid] = sm.l[tid] * sm.alpha[tid] +
+                  ((sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]));
+
+    // ---- O^T (+)= V^T P^T
     if (tid == 0) {
       const uint32_t vh = smem_addr(sm.khi), vl = smem_addr(sm.klo);
       const uint32_t ph = smem_addr(sm.phi), pl = smem_addr(sm.plo);
@@ -367,7 +409,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
           const uint32_t d = tmem + 64 + mt * 64;
           // V_hi P_hi + V_lo P_hi + V_hi P_lo
           mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkK, 1024),
-                  desc_mnmajor_sw128(ph + poff, kChunkK, 1024), kIdescPV, ks > 0);
+                  desc_mnmajor_sw128(ph + poff, kChunkK, 1024), kIdescPV, started || ks > 0);
           mma_f16(d, desc_mnmajor_sw128(vl + voff, kChunkK, 1024),
                   desc_mnmajor_sw128(ph + poff, kChunkK, 1024), kIdescPV, 1);
           mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkK, 1024),
@@ -376,16 +418,29 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
       }
       mma_commit(&sm.bar);
     }
-    ok = mbar_wait(&sm.bar, 1) && ok;
+    ok = mbar_wait(&sm.bar, phase) && ok;
+    phase ^= 1;
     tc_fence_after();
+    started = true;
+  }
+
+  // ---- epilogue: thread = dim within each 128-dim tile, heads 32*colh ..
+  __syncthreads();
+  float *po = part_o + ((size_t)row * n_splits + split) * kHeads * kD;
+  float *pl = part_lse + ((size_t)row * n_splits + split) * kHeads;
+  if (!started) {
+    // no key in this split: a partial that the merge weighs with zero
+    for (int i = tid; i < kHeads * kD; i += kThreads) po[i] = 0.f;
+    if (tid < kHeads) pl[tid] = -CUDART_INF_F;
+  } else {
+    if (tid < kHeads) sm.inv_l[tid] = 1.f / sm.l[tid];
     __syncthreads();
-    // ---- epilogue: thread = dim within each 128-dim tile, heads 32*colh ..
     const float inv_ln = 0.6931471805599453f;
     if (tid < kHeads) pl[tid] = ok ? (sm.m[tid] + log2f(sm.l[tid])) * inv_ln : CUDART_NAN_F;
     for (int mt = 0; mt < 4; ++mt) {
       const int d = mt * 128 + quad * 32 + lane;
       float o[32];
-      tmem_ld32(tl + 64 + mt * 64 + colh * 32, o);
+      tmem_ld32(tmem + tmem_tl + 64 + mt * 64 + colh * 32, o);
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -398,7 +453,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units,
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(sm.tmem_base, 512);
   }
 }
 
@@ -421,19 +476,18 @@ bool attn_tc_supported(const AttnArgs &a) {
   return major == 10;
 }
 
-int attn_tc_chunk_keys() { return kKeys; }
+int attn_tc_unit_keys() { return kKeys; }
 
-int launch_attn_tc(const AttnArgs &a, float *part_o, float *part_lse, int n_chunks,
+int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *part_lse,
                    cudaStream_t st) {
-  const long long max_comp = a.has_comp ? (a.sel ? a.k : a.max_entries) : 0;
-  const int ncc = (int)((max_comp + kKeys - 1) / kKeys);
-  if (n_chunks != ncc + (a.window + kKeys - 1) / kKeys) return CSKV_ERR_ARG;
   const size_t smem = sizeof(Smem) + 1024;
   if (!ensure_dynamic_smem(attn_tc_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   const int rows = a.B * a.Tq;
-  attn_tc_kernel<<<dim3((unsigned)n_chunks, (unsigned)rows), kThreads, smem, st>>>(
-      a, kKeys, ncc, n_chunks, part_o, part_lse);
-  return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
+  return launch_pdl(attn_tc_kernel, dim3((unsigned)rows, (unsigned)p.splits), dim3(kThreads),
+                    smem, st, a, p.unit, p.n_comp_units, p.n_units, p.per_cta, p.splits, part_o,
+                    part_lse) == cudaSuccess
+             ? CSKV_OK
+             : CSKV_ERR_CUDA;
 }
 
 }  // namespace cskv

@@ -76,6 +76,8 @@ compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__
                 const float *__restrict__ gate_b, int pool, int stride, Cache out_k,
                 Cache out_v, Cache out_ik) {
   extern __shared__ float smem[];
+  pdl_wait();
+  pdl_trigger();
   float *a = smem;                 // [pool] gate logits, then weights
   float *pooled = smem + pool;     // [max dims]
   const int b = blockIdx.y;
@@ -232,6 +234,8 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
                        const float *__restrict__ gate_b, int pool, int stride, Cache out_k,
                        Cache out_v, Cache out_ik) {
   extern __shared__ __align__(16) uint8_t csm[];
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   const long long j = t_begin[b] / stride + blockIdx.x;
   if (j >= t_end[b] / stride || j < 0) return;
@@ -330,12 +334,15 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
   const size_t smem_staged = staged + sizeof(float) * (size_t)(pool + dmax + 1) +
                              3 * sizeof(long long) * (size_t)pool + 16;
   if (smem_staged <= 200 * 1024 && ensure_dynamic_smem(compress_staged_kernel, smem_staged)) {
-    compress_staged_kernel<<<grid, kThreads, smem_staged, st>>>(
-        t_begin, t_end, raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride, out_k, out_v, out_ik);
+    if (launch_pdl(compress_staged_kernel, grid, dim3(kThreads), smem_staged, st, t_begin, t_end,
+                   raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride, out_k, out_v,
+                   out_ik) != cudaSuccess)
+      return CSKV_ERR_CUDA;
   } else {
     const size_t smem = sizeof(float) * (size_t)(pool + dmax);
-    compress_kernel<<<grid, kThreads, smem, st>>>(t_begin, t_end, raw_k, raw_v, raw_ik, gate_w,
-                                                  gate_b, pool, stride, out_k, out_v, out_ik);
+    if (launch_pdl(compress_kernel, grid, dim3(kThreads), smem, st, t_begin, t_end, raw_k, raw_v,
+                   raw_ik, gate_w, gate_b, pool, stride, out_k, out_v, out_ik) != cudaSuccess)
+      return CSKV_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }

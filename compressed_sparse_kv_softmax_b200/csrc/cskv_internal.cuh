@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "cskv.h"
 
 namespace cskv {
@@ -110,6 +112,34 @@ inline bool ensure_dynamic_smem(K kernel, size_t bytes) {
   return true;
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation: it may start while the previous
+// kernel on the stream is finishing, runs only on-chip set-up (shared memory,
+// barriers, TMEM, descriptor prefetch) before pdl_wait(), and touches global
+// memory only after it.  pdl_wait() returns once every preceding grid has
+// completed and its writes are visible; without a programmatic predecessor it
+// returns at once.  pdl_trigger() lets the next kernel begin launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // host-side launch helpers (defined in the kernel files)
 int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
                     const Cache &raw_k, const Cache &raw_v, const Cache &raw_ik,
@@ -144,6 +174,18 @@ struct AttnArgs {
   float *out, *lse;
   void *ws; size_t ws_bytes;
 };
+// How one query row's key list is cut into units and units into splits (one
+// CTA per split).  A split runs its units with an online softmax; with one
+// split per row the kernel writes the final output, otherwise each split
+// writes a partial (o, lse) that attn_merge_kernel combines.
+struct AttnPlan {
+  int unit;           // keys per unit
+  int n_comp_units;   // units of the compressed part (the window's follow)
+  int n_units;
+  int per_cta;        // units per split
+  int splits;         // splits per row
+};
+AttnPlan attn_plan(long long rows, long long max_comp, int window, int unit);
 size_t attn_ws_bytes(int B, int Tq, int Hq, int Dv, long long max_entries, int window);
 int launch_attention(const AttnArgs &a, cudaStream_t st);
 

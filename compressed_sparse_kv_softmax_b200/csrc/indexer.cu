@@ -33,6 +33,8 @@ constexpr int kKeys = 128;   // entries per CTA (one per thread)
 __global__ void __launch_bounds__(kKeys)
 indexer_score_kernel(IndexerArgs a, float *__restrict__ scores, long long ld) {
   extern __shared__ float sm[];
+  pdl_wait();
+  pdl_trigger();
   const int H = a.H_I, dI = a.d_I;
   float *q = sm;                       // [H][dI]
   float *w = q + H * dI;               // [H]
@@ -75,6 +77,15 @@ indexer_score_kernel(IndexerArgs a, float *__restrict__ scores, long long ld) {
   scores[(long long)row * ld + j] = s;
 }
 
+// zeroes n 32-bit words (the histogram and counters of the selection)
+__global__ void __launch_bounds__(256) zero_words_kernel(uint32_t *__restrict__ p, long long n) {
+  pdl_wait();
+  pdl_trigger();
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    p[i] = 0u;
+}
+
 }  // namespace
 
 size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k) {
@@ -89,7 +100,12 @@ int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
   const IndexerWs w = indexer_ws_layout(a.ws, rows, a.max_entries, a.k, nullptr);
   if (a.max_entries > 0 && indexer_tc_supported(a)) {
     // tensor-core scoring builds the score histogram the multi-CTA selection uses
-    if (cudaMemsetAsync(w.err, 0, w.zero_bytes, st) != cudaSuccess) return CSKV_ERR_CUDA;
+    const long long words = (long long)(w.zero_bytes / 4);
+    long long blocks = (words + 255) / 256;
+    if (blocks > 1184) blocks = 1184;
+    if (launch_pdl(zero_words_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                   reinterpret_cast<uint32_t *>(w.err), words) != cudaSuccess)
+      return CSKV_ERR_CUDA;
     int rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
     if (rc != CSKV_OK) return rc;
     return launch_topk_select(w, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
@@ -100,7 +116,9 @@ int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
                                          (size_t)kKeys * (a.d_I + 1));
     if (!ensure_dynamic_smem(indexer_score_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
     dim3 grid((unsigned)((a.max_entries + kKeys - 1) / kKeys), (unsigned)rows);
-    indexer_score_kernel<<<grid, kKeys, smem, st>>>(a, w.scores, w.ld);
+    if (launch_pdl(indexer_score_kernel, grid, dim3(kKeys), smem, st, a, w.scores, w.ld) !=
+        cudaSuccess)
+      return CSKV_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
   }
   launch_topk_rows(w.scores, w.ld, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,

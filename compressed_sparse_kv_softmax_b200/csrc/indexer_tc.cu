@@ -94,11 +94,6 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row = blockIdx.y;
   const int b = row / a.Tq;
-  long long n = (a.q_pos[row] + 1) / a.stride;
-  if (n > a.max_entries) n = a.max_entries;
-  if (n < 0) n = 0;
-  const int tiles = (int)((n + kTile - 1) / kTile);
-  const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / gridDim.x + 1 : 0;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
@@ -119,6 +114,13 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   __syncthreads();                 // barriers initialised, TMEM address published
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  pdl_wait();                      // global memory from here on
+  pdl_trigger();
+  long long n = (a.q_pos[row] + 1) / a.stride;
+  if (n > a.max_entries) n = a.max_entries;
+  if (n < 0) n = 0;
+  const int tiles = (int)((n + kTile - 1) / kTile);
+  const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / gridDim.x + 1 : 0;
   if (warp != 0) {
     // query heads -> B operand (K-major, 128-byte swizzle: 16-byte chunk c of
     // head h lands at chunk c ^ (h & 7) of its 128-byte row); the producer
@@ -321,8 +323,10 @@ int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_
   if (splits > tiles) splits = tiles;
   if (splits < 1) splits = 1;
   dim3 grid((unsigned)splits, (unsigned)rows);
-  indexer_tc_kernel<<<grid, kThreads, smem, st>>>(a, map, scores, ld, hist, err);
-  return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
+  return launch_pdl(indexer_tc_kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist,
+                    err) == cudaSuccess
+             ? CSKV_OK
+             : CSKV_ERR_CUDA;
 }
 
 }  // namespace cskv

@@ -213,6 +213,8 @@ __global__ void __launch_bounds__(1024)
 topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *__restrict__ q_pos,
                  int stride, long long max_entries, int k, int32_t *__restrict__ out_idx,
                  float *__restrict__ out_score) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x;
   const long long n = visible(q_pos, row, stride, max_entries);
   topk_row_single_cta(scores + (long long)row * ld, n, k, out_idx + (long long)row * k,
@@ -225,6 +227,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
                    float *__restrict__ out_score) {
   extern __shared__ __align__(16) uint8_t sel_smem_raw[];
   SelSmem &sm = *reinterpret_cast<SelSmem *>(sel_smem_raw);
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
   const long long n = visible(q_pos, row, stride, max_entries);
   const float *s = w.scores + (long long)row * w.ld;
@@ -476,8 +480,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
 void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,
                       long long max_entries, int k, int rows, int32_t *out_idx,
                       float *out_score, cudaStream_t st) {
-  topk_rows_kernel<<<rows, 1024, 0, st>>>(scores, ld, q_pos, stride, max_entries, k, out_idx,
-                                          out_score);
+  launch_pdl(topk_rows_kernel, dim3(rows), dim3(1024), 0, st, scores, ld, q_pos, stride,
+             max_entries, k, out_idx, out_score);
 }
 
 int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
@@ -494,8 +498,8 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
   const long long cap = (sms + rows - 1) / rows;
   if (splits > cap) splits = cap;
   if (splits < 1) splits = 1;
-  topk_select_kernel<<<dim3((unsigned)splits, (unsigned)rows), kSelThreads, smem, st>>>(
-      w, q_pos, stride, max_entries, k, out_idx, out_score);
+  launch_pdl(topk_select_kernel, dim3((unsigned)splits, (unsigned)rows), dim3(kSelThreads), smem,
+             st, w, q_pos, stride, max_entries, k, out_idx, out_score);
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 

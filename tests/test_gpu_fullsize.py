@@ -87,3 +87,21 @@ def test_prefill_sparse_attention_full_size(C):
                     np.stack([lse[r].cpu().numpy() for r in rows]),
                     np.stack([ref[r][0] for r in rows]), np.stack([ref[r][1] for r in rows]),
                     where="prefill csa")
+
+
+def test_prefill_dense_attention_full_size(C):
+    """HCA over the same 8,192-token chunk: each row attends every compressed
+    entry it can see (about 8,200) plus its causal window, so every row runs
+    its whole key list through one CTA's online softmax; 64 sampled rows."""
+    from compressed_sparse_kv_softmax_b200.layer import HCALayer
+    wl = W.get("prefill")
+    L = W.make_hca_layer(wl, device="cuda")
+    layer = HCALayer(L)
+    out, lse = layer.attend()
+    torch.cuda.synchronize()
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_attention(L, sel=None, rows=rows)
+    check_attention(np.stack([out[r].cpu().numpy() for r in rows]),
+                    np.stack([lse[r].cpu().numpy() for r in rows]),
+                    np.stack([ref[r][0] for r in rows]), np.stack([ref[r][1] for r in rows]),
+                    where="prefill hca")
