@@ -13,14 +13,19 @@
 //    the k-th largest key and how many equal keys to take, then an ordered
 //    compaction in index order writes the result.  Used after the generic
 //    scoring kernel and as the fall-back for pathological rows.
-//  * topk_select_kernel - several CTAs per row, after the tensor-core scoring
-//    kernel has built a histogram of the top 12 key bits:
-//      1. every CTA finds the bucket b* holding the k-th largest key;
-//      2. every CTA scans its slice of the row, appending entries above b*
-//         (sure winners) and entries in b* (candidates);
-//      3. the last CTA to finish (atomic ticket, nobody waits) selects the
-//         missing candidates by the low 20 key bits, breaks exact ties by the
-//         lower index, and sorts the k indices.
+//  * topk_select_kernel - several CTAs per row, each owning a contiguous
+//    slice of the row, after the tensor-core scoring kernel has built a
+//    histogram of the top 12 key bits:
+//      1. every CTA finds the bucket b* holding the k-th largest key, counts
+//         its slice's entries above b* and appends the entries inside b*
+//         (candidates) to the row's list;
+//      2. the row's CTAs meet once at a bounded barrier;
+//      3. every CTA reads the whole candidate list (a few thousand entries)
+//         and resolves the exact k-th key and the ties to take, so all of
+//         them hold the same decision; per-slice counts give each CTA the
+//         offset of its slice in the output;
+//      4. every CTA writes its slice's selected entries in index order, so
+//         the output comes out ascending without a sort.
 #include <climits>
 
 #include "cskv_internal.cuh"
@@ -181,31 +186,48 @@ __device__ void bitonic_sort_smem(T *v, int m) {
   }
 }
 
-// inverse of score_key
-__device__ __forceinline__ float key_score(uint32_t key) {
-  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
-}
-
 __device__ __forceinline__ uint64_t pack_entry(long long j, uint32_t key) {
   return ((uint64_t)(uint32_t)j << 32) | key;
 }
 
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 constexpr int kSelThreads = 512;
-constexpr int kCandSmem = kCandCap; // candidates the last CTA refines in shared memory
+constexpr int kSelPer = 8;                        // consecutive entries per thread and pass
+constexpr int kSelChunk = kSelThreads * kSelPer;  // entries per CTA and pass
 constexpr int kMaxK = 4096;
-constexpr int kScanBatch = 8;       // scores a thread loads before processing any
-// rows of up to this many entries are ordered through a bitmap plus word
-// prefix counts, both held in the (by then unused) candidate buffer
-constexpr int kBitmapWords = kCandSmem;                 // 8192 words x 2 arrays = 64 KB
-constexpr long long kBitmapEntries = 32LL * kBitmapWords;
+constexpr int kTieCap = kTopkBins;                // exact ties held in the histogram's space
+// Spins of the row barrier before it gives up (each backs off ~0.1-1 us, so
+// the limit is seconds: far beyond any legitimate wait, which is microseconds).
+constexpr uint32_t kBarrierSpins = 1u << 22;
 
 struct SelSmem {
-  uint32_t hist[kTopkBins];         // row histogram, later refine histograms / tie list
-  uint64_t cand[kCandSmem];         // (index << 32) | key
-  uint64_t out[kMaxK];              // (index << 32) | key of the selection
+  uint32_t hist[kTopkBins];   // row histogram, then refine bins, then the tie list
+  uint64_t cand[kCandCap];    // (index << 32) | key of every candidate of the row
+  int cnt[kMaxSplits];        // selected entries per slice of the row
   int scan[33];
-  int bstar, above, is_last, thr2, take_eq, n_eq, n_gt, fallback, n_cand, n_sel;
+  int bstar, above, thr_bin, take, n_eq, state, n_cand, base, total, wins;
+  uint32_t tie_cut;
 };
+
+// scores j0 .. j0+7 of a row (entries at or beyond j_hi read as -inf)
+__device__ __forceinline__ void load8(const float *__restrict__ s, long long j0, long long j_hi,
+                                      float (&v)[kSelPer]) {
+  if (j0 + kSelPer <= j_hi) {
+    const float4 a = __ldcg(reinterpret_cast<const float4 *>(s + j0));
+    const float4 b = __ldcg(reinterpret_cast<const float4 *>(s + j0) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e)
+      v[e] = j0 + e < j_hi ? __ldcg(s + j0 + e) : -__int_as_float(0x7f800000);
+  }
+}
 
 }  // namespace
 
@@ -229,14 +251,15 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   SelSmem &sm = *reinterpret_cast<SelSmem *>(sel_smem_raw);
   pdl_wait();
   pdl_trigger();
-  const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nsplit = gridDim.x, me = blockIdx.x;
   const long long n = visible(q_pos, row, stride, max_entries);
   const float *s = w.scores + (long long)row * w.ld;
   int32_t *oi = out_idx + (long long)row * k;
   float *os = out_score ? out_score + (long long)row * k : nullptr;
 
   if (n <= k) {            // every visible entry is selected, already in order
-    if (blockIdx.x == 0) {
+    if (me == 0) {
       for (int i = tid; i < k; i += blockDim.x) {
         oi[i] = i < n ? i : -1;
         if (os) os[i] = i < n ? s[i] : -__int_as_float(0x7f800000);
@@ -245,8 +268,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     return;
   }
 
-  // 1. threshold bucket b*: the bucket holding the k-th largest key
-  if (tid == 0) { sm.bstar = 0; sm.above = -1; }
+  // ---- 1. threshold bucket b*, this slice's winners and candidates
+  if (tid == 0) { sm.bstar = 0; sm.above = -1; sm.wins = 0; }
   {
     const uint32_t *hrow = w.hist + (size_t)row * kTopkBins;
     constexpr int kPer = kTopkBins / kSelThreads;
@@ -262,100 +285,94 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   const uint32_t bstar = (uint32_t)sm.bstar;
   const int above = sm.above;
 
-  // 2. this CTA's slice: sure winners (above b*) and candidates (in b*),
-  //    appended as (index, key) pairs; one atomic per warp and batch
+  const long long per = ((n + nsplit - 1) / nsplit + kSelPer - 1) / kSelPer * kSelPer;
+  const long long j_lo = (long long)me * per;
+  const long long j_hi = j_lo + per < n ? j_lo + per : n;
   uint32_t *ctr = w.ctr + (size_t)row * 4;
-  uint64_t *selrow = w.sel + (size_t)row * k;
   uint64_t *candrow = w.cand + (size_t)row * kCandCap;
-  const long long per = ((n + gridDim.x - 1) / gridDim.x + 31) & ~31LL;
-  const long long j_lo = (long long)blockIdx.x * per;
-  const long long j_hi = min(n, j_lo + per);
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (long long j0 = j_lo; j0 < j_hi; j0 += (long long)kScanBatch * kSelThreads) {
-    uint32_t key[kScanBatch];
+  float keep[kSelPer];                 // the first pass's scores, reused in step 4
+  int wins = 0;
+  for (long long c0 = j_lo; c0 < j_hi; c0 += kSelChunk) {
+    const long long j0 = c0 + (long long)tid * kSelPer;
+    float v[kSelPer];
+    load8(s, j0, j_hi, v);
+    if (c0 == j_lo) {
 #pragma unroll
-    for (int e = 0; e < kScanBatch; ++e) {
-      const long long j = j0 + e * kSelThreads + tid;
-      key[e] = j < j_hi ? score_key(__ldcg(s + j)) : 0u;
+      for (int e = 0; e < kSelPer; ++e) keep[e] = v[e];
     }
-    unsigned mg[kScanBatch], me[kScanBatch];
-    int cg = 0, ce = 0;
+    int nc = 0;
+    uint32_t cmask = 0;
 #pragma unroll
-    for (int e = 0; e < kScanBatch; ++e) {
-      const long long j = j0 + e * kSelThreads + tid;
-      const uint32_t bkt = key[e] >> kTopkShift;
-      mg[e] = __ballot_sync(0xffffffffu, j < j_hi && bkt > bstar);
-      me[e] = __ballot_sync(0xffffffffu, j < j_hi && bkt == bstar);
-      cg += __popc(mg[e]);
-      ce += __popc(me[e]);
-    }
-    uint32_t bg = 0, be = 0;
-    if (lane == 0) {
-      if (cg) bg = atomicAdd(&ctr[0], (uint32_t)cg);
-      if (ce) be = atomicAdd(&ctr[1], (uint32_t)ce);
-    }
-    bg = __shfl_sync(0xffffffffu, bg, 0);
-    be = __shfl_sync(0xffffffffu, be, 0);
-#pragma unroll
-    for (int e = 0; e < kScanBatch; ++e) {
-      const long long j = j0 + e * kSelThreads + tid;
-      if (mg[e] >> lane & 1u) {
-        const uint32_t p = bg + __popc(mg[e] & lt_mask);
-        if (p < (uint32_t)k) selrow[p] = pack_entry(j, key[e]);
+    for (int e = 0; e < kSelPer; ++e) {
+      if (j0 + e < j_hi) {
+        const uint32_t bkt = score_key(v[e]) >> kTopkShift;
+        wins += bkt > bstar;
+        if (bkt == bstar) { cmask |= 1u << e; ++nc; }
       }
-      if (me[e] >> lane & 1u) {
-        const uint32_t p = be + __popc(me[e] & lt_mask);
-        if (p < (uint32_t)kCandCap) candrow[p] = pack_entry(j, key[e]);
+    }
+    // warp-aggregated append of the candidates
+    int incl = nc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t base = 0;
+    if (lane == 31 && incl) base = atomicAdd(&ctr[0], (uint32_t)incl);
+    base = __shfl_sync(0xffffffffu, base, 31);
+    uint32_t p = base + (uint32_t)(incl - nc);
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e) {
+      if (cmask >> e & 1u) {
+        if (p < (uint32_t)kCandCap) candrow[p] = pack_entry(j0 + e, score_key(v[e]));
+        ++p;
       }
-      bg += __popc(mg[e]);
-      be += __popc(me[e]);
     }
   }
+  wins = __reduce_add_sync(0xffffffffu, wins);
+  if (lane == 0 && wins) atomicAdd(&sm.wins, wins);
 
-  // 3. the last CTA of the row finishes the selection
+  // ---- 2. row barrier: every slice's candidates and winner count are visible
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    sm.is_last = atomicAdd(&ctr[2], 1u) == gridDim.x - 1;
-    if (sm.is_last) {
-      __threadfence();
-      sm.n_sel = (int)atomicAdd(&ctr[0], 0u);
-      sm.n_cand = (int)atomicAdd(&ctr[1], 0u);
+    w.wins[(size_t)row * kMaxSplits + me] = (uint32_t)sm.wins;
+    __threadfence();
+    atomicAdd(&ctr[1], 1u);
+    int state = 0;
+    uint32_t spins = 0;
+    while (ld_acquire_u32(&ctr[1]) < (uint32_t)nsplit) {
+      if (++spins > kBarrierSpins) {
+        state = 1;
+        atomicOr(w.err, 2);
+        break;
+      }
+      __nanosleep(64);
     }
+    sm.state = state;
+    sm.n_cand = (int)ld_acquire_u32(&ctr[0]);
   }
   __syncthreads();
-  if (!sm.is_last) return;
   const int n_cand = sm.n_cand;
-  const int r = k - above;                 // candidates still to take, 1 <= r <= n_cand
-  // any inconsistency between the histogram and the scores (never expected)
-  // sends the row to the single-CTA path instead of indexing out of range
-  if (tid == 0)
-    sm.fallback = above < 0 || above >= k || r < 1 || r > n_cand || n_cand > kCandSmem ||
-                  sm.n_sel != above;
-  __syncthreads();
-  if (!sm.fallback) {
-    {  // candidates and sure winners into shared memory, loads first
-      constexpr int kC = kCandSmem / kSelThreads, kS = kMaxK / kSelThreads;
-      uint64_t v[kC], u[kS];
+  const int r = k - above;             // candidates still to take
+  bool fallback = sm.state != 0 || above < 0 || above >= k || r < 1 || r > n_cand ||
+                  n_cand > kCandCap;
+
+  // ---- 3. the exact k-th key among the candidates (same result in every CTA)
+  uint32_t thr = 0, tie_cut = 0xffffffffu;
+  if (!fallback) {
+    {
+      constexpr int kC = kCandCap / kSelThreads;
+      uint64_t v[kC];
 #pragma unroll
       for (int e = 0; e < kC; ++e) {
         const int i = tid + e * kSelThreads;
         v[e] = i < n_cand ? __ldcg(candrow + i) : 0ull;
       }
 #pragma unroll
-      for (int e = 0; e < kS; ++e) {
-        const int i = tid + e * kSelThreads;
-        u[e] = i < above ? __ldcg(selrow + i) : 0ull;
-      }
-#pragma unroll
       for (int e = 0; e < kC; ++e) {
         const int i = tid + e * kSelThreads;
         if (i < n_cand) sm.cand[i] = v[e];
-      }
-#pragma unroll
-      for (int e = 0; e < kS; ++e) {
-        const int i = tid + e * kSelThreads;
-        if (i < above) sm.out[i] = u[e];
       }
     }
     // radix select of the r-th largest candidate key on bits 19..10, then 9..0
@@ -370,111 +387,104 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
         if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
       }
       __syncthreads();
-      if (tid == 0) { sm.thr2 = 0; sm.take_eq = 0; }
-      find_threshold_bin([&](int i) { return sm.hist[i]; }, 1024, remaining, sm.scan, &sm.thr2,
-                         &sm.take_eq);
-      prefix = prefix | ((uint32_t)sm.thr2 << shift);
-      remaining = remaining - sm.take_eq;
+      if (tid == 0) { sm.thr_bin = 0; sm.take = 0; }
+      find_threshold_bin([&](int i) { return sm.hist[i]; }, 1024, remaining, sm.scan, &sm.thr_bin,
+                         &sm.take);
+      prefix |= (uint32_t)sm.thr_bin << shift;
+      remaining -= sm.take;
       mask |= 1023u << shift;
       __syncthreads();
     }
-    const uint32_t thr2 = prefix;
-    const int take_eq = remaining;
-    // candidates above thr2 follow the sure winners; the indices of candidates
-    // equal to thr2 go to a tie list (the lowest take_eq of them are taken)
-    if (tid == 0) { sm.n_gt = 0; sm.n_eq = 0; }
+    thr = prefix;
+    const int take_eq = remaining;     // keys equal to thr to take, lowest indices first
+    // exact ties: when more keys equal thr than are taken, the cut is the
+    // take_eq-th smallest of their indices
+    if (tid == 0) sm.n_eq = 0;
     __syncthreads();
-    uint32_t *eqv = sm.hist;                 // up to kTopkBins entries
+    uint32_t *eqv = sm.hist;
     for (int i = tid; i < n_cand; i += blockDim.x) {
       const uint64_t c = sm.cand[i];
-      const uint32_t key = (uint32_t)c;
-      if (key > thr2) {
-        const int p = atomicAdd(&sm.n_gt, 1);
-        if (above + p < k) sm.out[above + p] = c;
-      } else if (key == thr2) {
+      if ((uint32_t)c == thr) {
         const int p = atomicAdd(&sm.n_eq, 1);
-        if (p < kTopkBins) eqv[p] = (uint32_t)(c >> 32);
+        if (p < kTieCap) eqv[p] = (uint32_t)(c >> 32);
       }
     }
     __syncthreads();
-    const int n_gt = sm.n_gt, n_eq = sm.n_eq;
-    if (n_eq > kTopkBins || above + n_gt + take_eq != k || take_eq > n_eq) {
-      if (tid == 0) sm.fallback = 1;
-    } else {
-      if (n_eq > take_eq) {
-        int m = 1;
-        while (m < n_eq) m <<= 1;
-        for (int i = n_eq + tid; i < m; i += blockDim.x) eqv[i] = 0xffffffffu;
-        __syncthreads();
-        bitonic_sort_smem(eqv, m);
-      }
-      for (int i = tid; i < take_eq; i += blockDim.x)
-        sm.out[above + n_gt + i] = ((uint64_t)eqv[i] << 32) | thr2;
-    }
-    __syncthreads();
-    if (!sm.fallback) {
-      if (n <= kBitmapEntries) {
-        // ascending order by rank: the selected entries are distinct indices
-        // below n; mark them in a bitmap, prefix-count the words, and each
-        // entry's rank is the count of marked indices below it
-        uint32_t *bits = reinterpret_cast<uint32_t *>(sm.cand);
-        uint32_t *wpre = bits + kBitmapWords;
-        const int nw = (int)((n + 31) >> 5);
-        for (int i = tid; i < nw; i += blockDim.x) bits[i] = 0u;
-        __syncthreads();
-        for (int i = tid; i < k; i += blockDim.x) {
-          const uint32_t j = (uint32_t)(sm.out[i] >> 32);
-          atomicOr(&bits[j >> 5], 1u << (j & 31));
-        }
-        __syncthreads();
-        // warp w owns words [w * span, (w + 1) * span), read lane-contiguous
-        // (conflict-free); a warp scan inside, a block scan across warps
-        const int nwarps = blockDim.x >> 5, warp = tid >> 5;
-        const int span = (((nw + nwarps - 1) / nwarps) + 31) & ~31;
-        const int wb = warp * span;
-        int cnt = 0;
-        for (int i = lane; i < span; i += 32)
-          if (wb + i < nw) cnt += __popc(bits[wb + i]);
-        cnt = __reduce_add_sync(0xffffffffu, cnt);
-        int tot;
-        int run = block_exclusive_scan(lane == 0 ? cnt : 0, sm.scan, &tot);
-        run = __shfl_sync(0xffffffffu, run, 0);
-        for (int i0 = 0; i0 < span; i0 += 32) {
-          const int wi = wb + i0 + lane;
-          const int c = wi < nw ? __popc(bits[wi]) : 0;
-          int incl = c;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          if (wi < nw) wpre[wi] = (uint32_t)(run + incl - c);
-          run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        __syncthreads();
-        for (int i = tid; i < k; i += blockDim.x) {
-          const uint64_t e = sm.out[i];
-          const uint32_t j = (uint32_t)(e >> 32);
-          const int rank = (int)wpre[j >> 5] + __popc(bits[j >> 5] & ((1u << (j & 31)) - 1u));
-          oi[rank] = (int32_t)j;
-          if (os) os[rank] = key_score((uint32_t)e);
-        }
-      } else {
-        int m = 1;
-        while (m < k) m <<= 1;
-        for (int i = k + tid; i < m; i += blockDim.x) sm.out[i] = ~0ull;
-        __syncthreads();
-        bitonic_sort_smem(sm.out, m);        // ascending entry index
-        for (int i = tid; i < k; i += blockDim.x) {
-          const uint64_t e = sm.out[i];
-          oi[i] = (int32_t)(e >> 32);
-          if (os) os[i] = key_score((uint32_t)e);
-        }
-      }
+    const int n_eq = sm.n_eq;
+    if (take_eq < 1 || n_eq < take_eq || n_eq > kTieCap) {
+      fallback = true;
+    } else if (n_eq > take_eq) {
+      int m = 1;
+      while (m < n_eq) m <<= 1;
+      for (int i = n_eq + tid; i < m; i += blockDim.x) eqv[i] = 0xffffffffu;
+      __syncthreads();
+      bitonic_sort_smem(eqv, m);
+      tie_cut = eqv[take_eq - 1];
     }
   }
-  __syncthreads();
-  if (sm.fallback) topk_row_single_cta(s, n, k, oi, os);
+
+  // ---- per-slice counts of the selection, and this slice's output offset
+  if (!fallback) {
+    for (int c = tid; c < nsplit; c += blockDim.x)
+      sm.cnt[c] = (int)__ldcg(w.wins + (size_t)row * kMaxSplits + c);
+    __syncthreads();
+    for (int i = tid; i < n_cand; i += blockDim.x) {
+      const uint64_t c = sm.cand[i];
+      const uint32_t key = (uint32_t)c, j = (uint32_t)(c >> 32);
+      if (key > thr || (key == thr && j <= tie_cut)) atomicAdd(&sm.cnt[j / per], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int tot = 0, before = 0;
+      for (int c0 = 0; c0 < nsplit; c0 += 32) {
+        const int c = c0 + lane;
+        const int v = c < nsplit ? sm.cnt[c] : 0;
+        tot += __reduce_add_sync(0xffffffffu, v);
+        before += __reduce_add_sync(0xffffffffu, c < me ? v : 0);
+      }
+      if (lane == 0) { sm.total = tot; sm.base = before; }
+    }
+    __syncthreads();
+    fallback = sm.total != k;
+  }
+
+  // ---- 4. this slice's selected entries, in index order, at its offset
+  if (!fallback) {
+    int base = sm.base;
+    for (long long c0 = j_lo; c0 < j_hi; c0 += kSelChunk) {
+      const long long j0 = c0 + (long long)tid * kSelPer;
+      float v[kSelPer];
+      if (c0 == j_lo) {
+#pragma unroll
+        for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
+      } else {
+        load8(s, j0, j_hi, v);
+      }
+      uint32_t fl = 0;
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) {
+        const uint32_t key = score_key(v[e]);
+        const bool take = j0 + e < j_hi &&
+                          (key > thr || (key == thr && (uint32_t)(j0 + e) <= tie_cut));
+        fl |= (uint32_t)take << e;
+      }
+      int tot;
+      int p = base + block_exclusive_scan(__popc(fl), sm.scan, &tot);
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) {
+        if ((fl >> e & 1u) && p < k) {
+          oi[p] = (int32_t)(j0 + e);
+          if (os) os[p] = v[e];
+        }
+        p += fl >> e & 1u;
+      }
+      base += tot;
+    }
+    return;
+  }
+  // inconsistent histogram or candidate overflow (never expected with the
+  // scoring kernel's histogram): the row's first CTA selects the whole row
+  if (me == 0) topk_row_single_cta(s, n, k, oi, os);
 }
 
 void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,
@@ -493,10 +503,13 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // slices of at least 4096 scores; enough CTAs to cover the SMs at one row
-  long long splits = (max_entries + 4095) / 4096;
-  const long long cap = (sms + rows - 1) / rows;
+  // one pass of kSelChunk scores per CTA; the CTAs of a row wait for one
+  // another once, so a row's CTAs must all be resident at the same time:
+  // at most one CTA per SM over the whole grid, else one CTA per row
+  long long splits = (max_entries + kSelChunk - 1) / kSelChunk;
+  const long long cap = sms / rows;
   if (splits > cap) splits = cap;
+  if (splits > kMaxSplits) splits = kMaxSplits;
   if (splits < 1) splits = 1;
   launch_pdl(topk_select_kernel, dim3((unsigned)splits, (unsigned)rows), dim3(kSelThreads), smem,
              st, w, q_pos, stride, max_entries, k, out_idx, out_score);

@@ -9,33 +9,35 @@ namespace cskv {
 // exponent and 3 mantissa bits): 4096 buckets, each 1/8 of an octave wide.
 constexpr int kTopkBins = 4096;
 constexpr int kTopkShift = 20;
-// Candidates (entries inside the threshold bucket) kept per row; the final
-// refinement runs in shared memory up to this count and falls back to the
-// single-CTA selection of the whole row beyond it.
+// Candidates (entries inside the threshold bucket) kept per row; rows with
+// more fall back to the single-CTA selection of the whole row.
 constexpr int kCandCap = 8192;
+// Most CTAs that share one row in the multi-CTA selection.
+constexpr int kMaxSplits = 256;
 
 // Indexer workspace layout, one section after another, each 256-byte aligned:
 //   scores   rows x ld fp32
 //   err      4 int                 device status words (zeroed before scoring)
 //   hist     rows x kTopkBins u32  (zeroed before scoring)
-//   ctr      rows x 4 u32          selected count, candidate count, ticket (zeroed)
-//   sel      rows x k u64          entries above the threshold bucket, (index << 32) | key
-//   cand     rows x kCandCap u64   entries inside the threshold bucket, same packing
+//   ctr      rows x 4 u32          candidate count, barrier arrivals (zeroed)
+//   wins     rows x kMaxSplits u32 entries above the threshold bucket per CTA
+//   cand     rows x kCandCap u64   entries inside the threshold bucket, (index << 32) | key
 struct IndexerWs {
   int *err;
   float *scores;
   uint32_t *hist;
   uint32_t *ctr;
-  uint64_t *sel;
+  uint32_t *wins;
   uint64_t *cand;
   long long ld;
-  size_t zero_bytes;   // bytes from `hist` that must be zero before the call
+  size_t zero_bytes;   // bytes from `err` that must be zero before the call
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 inline IndexerWs indexer_ws_layout(void *base, long long rows, long long max_entries, int k,
                                    size_t *total) {
+  (void)k;
   IndexerWs w{};
   w.ld = (max_entries + 3) & ~3LL;
   if (w.ld < 4) w.ld = 4;
@@ -47,7 +49,7 @@ inline IndexerWs indexer_ws_layout(void *base, long long rows, long long max_ent
   w.hist = reinterpret_cast<uint32_t *>(p + off);     off = align256(off + rows * kTopkBins * 4);
   w.ctr = reinterpret_cast<uint32_t *>(p + off);      off = align256(off + rows * 16);
   w.zero_bytes = off - zero_begin;
-  w.sel = reinterpret_cast<uint64_t *>(p + off);      off = align256(off + rows * (size_t)k * 8);
+  w.wins = reinterpret_cast<uint32_t *>(p + off);     off = align256(off + rows * (size_t)kMaxSplits * 4);
   w.cand = reinterpret_cast<uint64_t *>(p + off);     off = align256(off + rows * (size_t)kCandCap * 8);
   if (total) *total = off;
   return w;

@@ -122,6 +122,49 @@ def test_indexer_edge_sizes(C, T, k):
         check_topk(idx[b, t], ridx, rs, where=f"T={T} k={k} row {(b, t)}")
 
 
+def _tied_keys(wl, needles, every):
+    """Indexer keys that all repeat the key of the row's best entry: every
+    `every`-th entry at its scale (equal scores), the others at half scale
+    (half the score, a lower histogram bucket) and the `needles` at twice
+    the scale."""
+    L = W.make_csa_layer(wl)
+    j0 = int(np.argmax(O.layer_indexer_topk(L, 1)[(0, 0)][1]))
+    ik = L["comp_ik"]
+    ik["data"][0, :] = ik["data"][0, j0].clone()
+    sc0 = ik["scale"][0, j0].clone()
+    ik["scale"][0, :] = sc0 * 0.5
+    ik["scale"][0, 0::every] = sc0
+    ik["scale"][0, needles] = sc0 * 2.0
+    return L
+
+
+@pytest.mark.parametrize("T,k,every", [(18000, 300, 3), (40000, 300, 1)])
+def test_indexer_exact_ties_take_lower_indices(C, T, k, every):
+    # exact score ties at the k-th score: the lowest indices are taken, and the
+    # output is ascending.  T=18000 keeps the tied candidates in the multi-CTA
+    # path; every=1 (all entries tied) overflows the candidate list and takes
+    # the single-CTA path.
+    wl = W.get("parity_decode").with_(T=T, B=1, k=k)
+    rng = np.random.default_rng(5)
+    n = T // 4
+    needles = np.sort(rng.choice(np.arange(1, n), 37, replace=False))
+    L = _tied_keys(wl, needles, every)
+    sc = O.layer_indexer_topk(L, k)[(0, 0)][1]
+    ties = np.array([j for j in range(0, n, every) if j not in set(needles.tolist())])
+    rest = np.setdiff1d(np.arange(n), np.concatenate([needles, ties]))
+    # the oracle's scores (to its own rounding: BLAS may sum identical rows in
+    # different orders) show the intended structure: the needles, then a tie
+    # group holding the k-th score, then the rest
+    assert sc[ties[0]] > 0
+    assert np.allclose(sc[ties], sc[ties[0]], rtol=1e-12, atol=0)
+    assert np.allclose(sc[needles], 2 * sc[ties[0]], rtol=1e-12, atol=0)
+    assert rest.size == 0 or sc[rest].max() < 0.6 * sc[ties[0]]
+    expect = np.sort(np.concatenate([needles, ties[: k - len(needles)]]))
+    layer = _run_indexer(C, to_device(L))
+    got = layer.idx.cpu().numpy()[0, 0]
+    assert np.array_equal(got, expect)
+
+
 # ----------------------------------------------------------------- attention
 
 def _sel_from_oracle(L, k):
