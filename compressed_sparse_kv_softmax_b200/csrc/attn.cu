@@ -176,58 +176,121 @@ attn_units_kernel(AttnArgs a, AttnPlan p, float *__restrict__ part_o,
 }
 
 // out[row][h][:] = sum_i e^{lse_i - L} o_i,  lse[row][h] = L = log sum_i e^{lse_i}
-// CTA (row * Hq + head, d-block of 128); 4 groups of 128 threads split the chunks,
-// each thread one output dim; a shared-memory sum joins the groups.
-constexpr int kMergeD = 128, kMergeGroups = 4;
+// CTA (row * Hq + head, half of the dims), 1024 threads: thread t takes 4
+// consecutive dims (t % 64) and the partials i = t / 64, t / 64 + 16, ..;
+// every partial a thread reads is requested before any is used, together
+// with the LSEs, whose weights one warp computes; shared memory sums the 16
+// groups.
+constexpr int kMergeThreads = 1024, kMergeQuads = 64;            // 4-dim columns per CTA
+constexpr int kMergeGroups = kMergeThreads / kMergeQuads;        // 16
+constexpr int kMergeBatch = 9;      // partials per thread and batch (144 per CTA)
+constexpr int kMergeLse = 2048;     // LSE weights held in shared memory
 
-__global__ void __launch_bounds__(kMergeD * kMergeGroups)
+// four consecutive values p[0..3] of which the first n exist (16-byte load when
+// vec and all four exist)
+__device__ __forceinline__ float4 load4(const float *p, int n, bool vec) {
+  if (vec && n >= 4) return __ldcg(reinterpret_cast<const float4 *>(p));
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (n > 0) r.x = __ldcg(p);
+  if (n > 1) r.y = __ldcg(p + 1);
+  if (n > 2) r.z = __ldcg(p + 2);
+  if (n > 3) r.w = __ldcg(p + 3);
+  return r;
+}
+
+__global__ void __launch_bounds__(kMergeThreads)
 attn_merge_kernel(int Hq, int Dv, int n_chunks, const float *__restrict__ part_o,
                   const float *__restrict__ part_lse, float *__restrict__ out,
                   float *__restrict__ lse) {
-  extern __shared__ float wts[];          // [n_chunks]
-  __shared__ float red[kMergeGroups][kMergeD];
+  __shared__ float4 red[kMergeGroups][kMergeQuads];
+  __shared__ float wts[kMergeLse];
+  __shared__ float s_L;
   pdl_wait();
   pdl_trigger();
-  __shared__ float s_L;
   const int row = blockIdx.x / Hq, h = blockIdx.x % Hq;
-  const int tid = threadIdx.x, grp = tid / kMergeD, dl = tid % kMergeD;
-  const int d = blockIdx.y * kMergeD + dl;
+  const int tid = threadIdx.x, q = tid % kMergeQuads, g = tid / kMergeQuads;
+  const int d = (blockIdx.y * kMergeQuads + q) * 4;
+  const bool dv = d < Dv;
+  const int nd = Dv - d;                   // dims of this thread's four that exist
+  const bool vec = (Dv & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
   const float *pl = part_lse + (long long)row * n_chunks * Hq + h;
-  for (int i = tid; i < n_chunks; i += blockDim.x) wts[i] = __ldg(pl + (long long)i * Hq);
+  const float *po = part_o + (long long)row * n_chunks * Hq * Dv + (long long)h * Dv + d;
+  const long long cstride = (long long)Hq * Dv;
+  // the first batch of partials and the LSEs, all in flight at once
+  float4 v[kMergeBatch];
+#pragma unroll
+  for (int k = 0; k < kMergeBatch; ++k) {
+    const int i = g + k * kMergeGroups;
+    v[k] = (i < n_chunks && dv) ? load4(po + i * cstride, nd, vec) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const int nw = n_chunks < kMergeLse ? n_chunks : kMergeLse;
+  for (int i = tid; i < nw; i += kMergeThreads) wts[i] = __ldcg(pl + (long long)i * Hq);
   __syncthreads();
   if (tid < 32) {
     float m = -CUDART_INF_F;
-    for (int i = tid; i < n_chunks; i += 32) m = fmaxf(m, wts[i]);
-    m = warp_max(m);
-    float s = 0.f;
-    for (int i = tid; i < n_chunks; i += 32) s += wts[i] == -CUDART_INF_F ? 0.f : expf(wts[i] - m);
-    s = warp_sum(s);
-    const float L = m + logf(s);
-    __syncwarp();
     for (int i = tid; i < n_chunks; i += 32)
+      m = fmaxf(m, i < kMergeLse ? wts[i] : __ldcg(pl + (long long)i * Hq));
+    m = warp_max(m);
+    float ssum = 0.f;
+    if (m != -CUDART_INF_F)
+      for (int i = tid; i < n_chunks; i += 32)
+        ssum += expf((i < kMergeLse ? wts[i] : __ldcg(pl + (long long)i * Hq)) - m);
+    ssum = warp_sum(ssum);
+    const float L = m != -CUDART_INF_F ? m + logf(ssum) : -CUDART_INF_F;
+    __syncwarp();
+    for (int i = tid; i < nw; i += 32)
       wts[i] = wts[i] == -CUDART_INF_F ? 0.f : expf(wts[i] - L);
     if (tid == 0) s_L = L;
   }
   __syncthreads();
-  float acc = 0.f;
-  if (d < Dv) {
-    const float *po = part_o + (long long)row * n_chunks * Hq * Dv + (long long)h * Dv + d;
-    const long long cstride = (long long)Hq * Dv;
-#pragma unroll 8
-    for (int i = grp; i < n_chunks; i += kMergeGroups) {
-      const float w = wts[i];
-      if (w != 0.f) acc = fmaf(w, __ldg(po + i * cstride), acc);
+  const float L = s_L;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int b0 = 0; b0 < n_chunks; b0 += kMergeGroups * kMergeBatch) {
+    if (b0 > 0) {
+#pragma unroll
+      for (int k = 0; k < kMergeBatch; ++k) {
+        const int i = b0 + g + k * kMergeGroups;
+        v[k] = (i < n_chunks && dv) ? load4(po + i * cstride, nd, vec)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      const int i = b0 + g + k * kMergeGroups;
+      if (i < n_chunks) {
+        const float li = i < kMergeLse ? 0.f : __ldcg(pl + (long long)i * Hq);
+        const float w = i < kMergeLse ? wts[i] : (li == -CUDART_INF_F ? 0.f : expf(li - L));
+        acc.x = fmaf(w, v[k].x, acc.x);
+        acc.y = fmaf(w, v[k].y, acc.y);
+        acc.z = fmaf(w, v[k].z, acc.z);
+        acc.w = fmaf(w, v[k].w, acc.w);
+      }
     }
   }
-  red[grp][dl] = acc;
+  red[g][q] = acc;
   __syncthreads();
-  if (grp == 0 && d < Dv) {
-    float t = red[0][dl];
+  // every partial has been read (the values were used before the barrier):
+  // their 128-byte lines leave L2 without being written back to HBM
+  if ((q & 7) == 0 && dv && (Dv & 31) == 0)
+    for (int i = g; i < n_chunks; i += kMergeGroups) discard_l2_line(po + i * cstride);
+  if (g == 0 && dv) {
+    float4 t = red[0][q];
 #pragma unroll
-    for (int g = 1; g < kMergeGroups; ++g) t += red[g][dl];
-    out[((long long)row * Hq + h) * Dv + d] = t;
+    for (int k = 1; k < kMergeGroups; ++k) {
+      const float4 u = red[k][q];
+      t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+    }
+    float *o = out + ((long long)row * Hq + h) * Dv + d;
+    if (vec) {
+      *reinterpret_cast<float4 *>(o) = t;
+    } else {
+      o[0] = t.x;
+      if (nd > 1) o[1] = t.y;
+      if (nd > 2) o[2] = t.z;
+      if (nd > 3) o[3] = t.w;
+    }
   }
-  if (blockIdx.y == 0 && tid == 0) lse[(long long)row * Hq + h] = s_L;
+  if (blockIdx.y == 0 && tid == 0) lse[(long long)row * Hq + h] = L;
 }
 
 }  // namespace
@@ -287,11 +350,10 @@ int launch_attention(const AttnArgs &a, cudaStream_t st) {
       return CSKV_ERR_CUDA;
   }
   if (direct) return CSKV_OK;
-  const size_t msmem = sizeof(float) * p.splits;
-  if (!ensure_dynamic_smem(attn_merge_kernel, msmem)) return CSKV_ERR_UNSUPPORTED;
-  if (launch_pdl(attn_merge_kernel, dim3((unsigned)(rows * a.Hq), (a.Dv + kMergeD - 1) / kMergeD),
-                 dim3(kMergeD * kMergeGroups), msmem, st, a.Hq, a.Dv, p.splits,
-                 (const float *)part_o, (const float *)part_lse, a.out, a.lse) != cudaSuccess)
+  if (launch_pdl(attn_merge_kernel,
+                 dim3((unsigned)(rows * a.Hq), (a.Dv + 4 * kMergeQuads - 1) / (4 * kMergeQuads)),
+                 dim3(kMergeThreads), 0, st, a.Hq, a.Dv, p.splits, (const float *)part_o,
+                 (const float *)part_lse, a.out, a.lse) != cudaSuccess)
     return CSKV_ERR_CUDA;
   return CSKV_OK;
 }

@@ -17,17 +17,20 @@
 // single FP16 rounding of K, V or P alone already misses that, so every
 // tensor-core operand that is not exact in FP16 is split into two FP16 terms,
 // x = hi + lo with hi = fp16(x), lo = fp16(x - hi) (about 22 bits together):
-//   S = K_hi Q^T + K_lo Q^T           (Q is BF16, exact in FP16)
+//   S = K_hi Q^T + K_lo Q^T           (Q is BF16, exact in FP16; one MMA chain
+//                                      over the hi and lo rows stacked on M)
 //   O = V_hi P_hi + V_lo P_hi + V_hi P_lo   (V = K; the lo x lo term is 2^-22)
 // with fp32 accumulation in TMEM.
 //
-//   1. gather: each warp converts 8 keys per batch (all loads first); lanes
-//      0-27 take 16 FP8 codes each (x block scale), lanes 28-31 16 BF16 RoPE
-//      values each; hi and lo parts land in two K-major 128-byte-swizzled
-//      tiles [8 chunks of 64 dims][64 keys][128 B].  Q becomes FP16 in the
-//      same layout [8 chunks][64 heads][128 B].
-//   2. S^T with keys on the MMA M axis (M = 128, rows 64..127 masked;
-//      N = 64 heads; K = 512 in 32 steps per part), fp32 in TMEM cols 0..63.
+//   1. gather: each warp loads 8 keys (all loads first; the first unit stages
+//      Q meanwhile), then converts them: lanes 0-27 take 16 FP8 codes each
+//      (x block scale), lanes 28-31 16 BF16 RoPE values each.  Per 64-dim
+//      chunk the key tile holds 64 rows of hi parts then 64 rows of lo parts
+//      (K-major, 128-byte swizzle).  Q becomes FP16 in the same layout
+//      [8 chunks][64 heads][128 B].
+//   2. [K_hi; K_lo] Q^T with the 128 stacked rows on the MMA M axis (N = 64
+//      heads, K = 512 in 32 steps), fp32 in TMEM cols 0..63; lanes 64..127
+//      (lo parts) are added to lanes 0..63 through shared memory.
 //   3. softmax over keys per head: each thread owns one key row; a warp
 //      reduce-scatter butterfly (32+16+8+4+2 shuffles) leaves lane L with
 //      heads 2L, 2L+1 over the warp's keys, shared memory joins the warps.
@@ -52,7 +55,8 @@ constexpr int kHeads = 64, kD = 512, kDn = 448, kDr = 64;
 constexpr int kKeys = 64;                          // keys per unit (valid MMA rows)
 constexpr int kM = 128;                            // MMA M (rows kKeys..127 are masked)
 constexpr int kThreads = 256;                      // warps w, w+4 share TMEM lanes
-constexpr uint32_t kChunkK = kKeys * 128;          // bytes per 64-dim chunk of a key tile
+constexpr uint32_t kChunkK = kKeys * 128;          // bytes per 64-dim chunk of the hi (or lo) rows
+constexpr uint32_t kChunkKK = 2 * kChunkK;         // bytes per 64-dim chunk: hi rows, then lo rows
 constexpr uint32_t kChunkQ = kHeads * 128;         // bytes per 64-dim chunk of Q
 constexpr uint32_t kIdescQK = idesc(kFmtF16, kFmtF16, 0, 0, kM, kHeads);
 constexpr uint32_t kIdescPV = idesc(kFmtF16, kFmtF16, 1, 1, 128, kHeads);
@@ -60,8 +64,7 @@ constexpr uint32_t kIdescPV = idesc(kFmtF16, kFmtF16, 1, 1, 128, kHeads);
 struct __align__(1024) Smem {
   // key tiles, hi and lo parts (K-major view: K; MN-major view: V^T).  An
   // M = 128 read of a chunk runs 64 rows into the next buffer: masked rows.
-  uint8_t khi[8 * kChunkK];         // 64 KB
-  uint8_t klo[8 * kChunkK];         // 64 KB
+  uint8_t kt[8 * kChunkKK];         // 128 KB: per 64-dim chunk, 64 hi rows then 64 lo rows
   uint8_t q[8 * kChunkQ];           // 64 KB
   uint8_t phi[kKeys * 128];         // 8 KB: P^T hi, MN-major [keys][64 heads]
   uint8_t plo[kKeys * 128];         // 8 KB
@@ -119,6 +122,36 @@ __device__ __forceinline__ float2 e4m3x2(uint32_t pair) {
   return __half22float2(*reinterpret_cast<const __half2 *>(&h));
 }
 
+// Q [64 heads][512] BF16 -> FP16 in the K-major 128-byte-swizzled layout
+// [8 chunks of 64 dims][64 heads][128 B], loads batched before any is used
+__device__ __forceinline__ void stage_q(const __nv_bfloat16 *__restrict__ qg, uint8_t *q) {
+  constexpr int kPer = kHeads * kD / 8 / kThreads, kBatch = 8;
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int i0 = 0; i0 < kPer; i0 += kBatch) {
+    uint4 raw[kBatch];
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e) {
+      const int i = tid + (i0 + e) * kThreads;
+      raw[e] = __ldg(reinterpret_cast<const uint4 *>(qg) + i);
+    }
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e) {
+      const int i = tid + (i0 + e) * kThreads;
+      const int h = i >> 6, c = (i >> 3) & 7, u = i & 7;  // 8 dims per unit
+      const __nv_bfloat162 *bp = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
+      uint4 o;
+      uint32_t *op = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(bp[k]);
+        op[k] = pack_h2(f.x, f.y);
+      }
+      *reinterpret_cast<uint4 *>(q + c * kChunkQ + swz(h, u)) = o;
+    }
+  }
+}
+
 struct Row {
   long long pos, n_comp, w_lo;
   int n_win;
@@ -167,37 +200,6 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
   pdl_trigger();
   const Row R = row_of(a, row);
 
-  // ---- Q: BF16 -> FP16, K-major swizzled
-  {
-    const __nv_bfloat16 *qg =
-        reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD;
-    // 16-byte units per thread, loaded 16 at a time before any is used
-    constexpr int kPer = kHeads * kD / 8 / kThreads, kBatch = 16;
-#pragma unroll
-    for (int i0 = 0; i0 < kPer; i0 += kBatch) {
-      uint4 raw[kBatch];
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e) {
-        const int i = tid + (i0 + e) * kThreads;
-        raw[e] = __ldg(reinterpret_cast<const uint4 *>(qg) + i);
-      }
-#pragma unroll
-      for (int e = 0; e < kBatch; ++e) {
-        const int i = tid + (i0 + e) * kThreads;
-        const int h = i >> 6, c = (i >> 3) & 7, u = i & 7;  // 8 dims per unit
-        const __nv_bfloat162 *bp = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
-        uint4 o;
-        uint32_t *op = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(bp[q]);
-          op[q] = pack_h2(f.x, f.y);
-        }
-        *reinterpret_cast<uint4 *>(sm.q + c * kChunkQ + swz(h, u)) = o;
-      }
-    }
-  }
-
   const int quad = warp & 3, colh = warp >> 2;      // TMEM lane quadrant, head half
   const int krow = tid & 127;                       // key row = TMEM lane of this thread
   const uint32_t tmem_tl = ((uint32_t)(quad * 32) << 16);
@@ -205,6 +207,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
   uint32_t phase = 0;                               // parity of the next completion of sm.bar
   bool started = false;                             // O^T in TMEM holds a partial sum
   bool ok = true;
+  bool q_ready = false;                             // Q staged in shared memory
   uint32_t tmem = 0;
   const int u_begin = split * units_per_cta;
   const int u_end = min(n_units, u_begin + units_per_cta);
@@ -235,25 +238,33 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     if (!__syncthreads_or(tid < kM && sm.slot[tid] >= 0)) continue;
     const bool my_valid = sm.slot[krow] >= 0;
 
-    // ---- gather: each warp converts 8 consecutive key rows per batch, loads first
-    for (int r0 = warp * 8; r0 < ksteps * 16; r0 += 8 * kThreads / 32) {
-      uint4 raw[8], raw2[8];
-      float sc[8];
+    // ---- gather: each warp takes 8 consecutive key rows; all loads are
+    // issued first, then (first unit only) Q is staged while they are in
+    // flight, then the rows are converted
+    const int r0 = warp * 8;
+    const bool has_rows = r0 < ksteps * 16;   // kKeys = 8 warps x 8 rows
+    uint4 raw[8], raw2[8];
+    float sc[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const long long slot = sm.slot[r0 + e];
-        raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
-        sc[e] = 0.f;
-        if (slot < 0) continue;
-        if (lane < 28) {
-          raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
-          sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
-        } else {
-          const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
-          raw[e] = __ldg(rp);
-          raw2[e] = __ldg(rp + 1);
-        }
+    for (int e = 0; e < 8; ++e) {
+      raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
+      sc[e] = 0.f;
+      const long long slot = has_rows ? sm.slot[r0 + e] : -1;
+      if (slot < 0) continue;
+      if (lane < 28) {
+        raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
+        sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
+      } else {
+        const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
+        raw[e] = __ldg(rp);
+        raw2[e] = __ldg(rp + 1);
       }
+    }
+    if (!q_ready) {
+      stage_q(reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD, sm.q);
+      q_ready = true;
+    }
+    if (has_rows) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int r = r0 + e;
@@ -289,11 +300,12 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
           d0 = kDn + (lane - 28) * 16;
         }
         const int c = d0 >> 6, u = (d0 & 63) >> 3;
-        const uint32_t o0 = c * kChunkK + swz(r, u), o1 = c * kChunkK + swz(r, u + 1);
-        *reinterpret_cast<uint4 *>(sm.khi + o0) = h0;
-        *reinterpret_cast<uint4 *>(sm.khi + o1) = h1;
-        *reinterpret_cast<uint4 *>(sm.klo + o0) = l0;
-        *reinterpret_cast<uint4 *>(sm.klo + o1) = l1;
+        // hi part in row r, lo part in row 64 + r of the chunk (same swizzle phase)
+        const uint32_t o0 = c * kChunkKK + swz(r, u), o1 = c * kChunkKK + swz(r, u + 1);
+        *reinterpret_cast<uint4 *>(sm.kt + o0) = h0;
+        *reinterpret_cast<uint4 *>(sm.kt + o1) = h1;
+        *reinterpret_cast<uint4 *>(sm.kt + kChunkK + o0) = l0;
+        *reinterpret_cast<uint4 *>(sm.kt + kChunkK + o1) = l1;
       }
     }
     fence_proxy_async_shared();
@@ -302,18 +314,15 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     tc_fence_after();
     tmem = sm.tmem_base;
 
-    // ---- S^T = K Q^T  (hi and lo parts of K)
+    // ---- [K_hi; K_lo] Q^T: M = 128 rows (hi parts of the unit's keys, then
+    // their lo parts), N = 64 heads, K = 512 in 32 steps
     if (tid == 0) {
-      const uint32_t qa = smem_addr(sm.q);
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t ka = smem_addr(part ? sm.klo : sm.khi);
+      const uint32_t qa = smem_addr(sm.q), ka = smem_addr(sm.kt);
 #pragma unroll 4
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t off = (ks & 3) << 5;       // 16 dims = 32 bytes per step
-          mma_f16(tmem, desc_kmajor_sw128(ka + (ks >> 2) * kChunkK + off),
-                  desc_kmajor_sw128(qa + (ks >> 2) * kChunkQ + off), kIdescQK,
-                  (part | ks) != 0);
-        }
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        const uint32_t off = (ks & 3) << 5;       // 16 dims = 32 bytes per step
+        mma_f16(tmem, desc_kmajor_sw128(ka + (ks >> 2) * kChunkKK + off),
+                desc_kmajor_sw128(qa + (ks >> 2) * kChunkQ + off), kIdescQK, ks != 0);
       }
       mma_commit(&sm.bar);
     }
@@ -325,6 +334,22 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     float sv[32];
     tmem_ld32(tmem + tmem_tl + colh * 32, sv);
     tmem_wait_ld();
+    {
+      // S = hi rows + lo rows: TMEM lanes 64..127 hand their values to lanes
+      // 0..63 through the P buffers (free until P is written), head-major so
+      // that the lanes of a warp touch consecutive words
+      float *scr = reinterpret_cast<float *>(sm.phi);   // [64 heads][64 keys]
+      if (krow >= kKeys) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) scr[(colh * 32 + i) * kKeys + (krow - kKeys)] = sv[i];
+      }
+      __syncthreads();
+      if (krow < kKeys) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[i] += scr[(colh * 32 + i) * kKeys + krow];
+      }
+      __syncthreads();
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) sv[i] = my_valid ? sv[i] * c2 : -CUDART_INF_F;
     {
@@ -401,18 +426,18 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
 
     // ---- O^T (+)= V^T P^T
     if (tid == 0) {
-      const uint32_t vh = smem_addr(sm.khi), vl = smem_addr(sm.klo);
+      const uint32_t vh = smem_addr(sm.kt), vl = vh + kChunkK;
       const uint32_t ph = smem_addr(sm.phi), pl = smem_addr(sm.plo);
       for (int mt = 0; mt < 4; ++mt) {
         for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t voff = (2 * mt) * kChunkK + ks * 2048, poff = ks * 2048;
+          const uint32_t voff = (2 * mt) * kChunkKK + ks * 2048, poff = ks * 2048;
           const uint32_t d = tmem + 64 + mt * 64;
           // V_hi P_hi + V_lo P_hi + V_hi P_lo
-          mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkK, 1024),
+          mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkKK, 1024),
                   desc_mnmajor_sw128(ph + poff, kChunkK, 1024), kIdescPV, started || ks > 0);
-          mma_f16(d, desc_mnmajor_sw128(vl + voff, kChunkK, 1024),
+          mma_f16(d, desc_mnmajor_sw128(vl + voff, kChunkKK, 1024),
                   desc_mnmajor_sw128(ph + poff, kChunkK, 1024), kIdescPV, 1);
-          mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkK, 1024),
+          mma_f16(d, desc_mnmajor_sw128(vh + voff, kChunkKK, 1024),
                   desc_mnmajor_sw128(pl + poff, kChunkK, 1024), kIdescPV, 1);
         }
       }

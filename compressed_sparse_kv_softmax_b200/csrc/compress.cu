@@ -237,28 +237,38 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   pdl_wait();
   pdl_trigger();
   const int b = blockIdx.y;
-  const long long j = t_begin[b] / stride + blockIdx.x;
-  if (j >= t_end[b] / stride || j < 0) return;
-  if (j >= out_k.cap || (raw_v.data && j >= out_v.cap) || (raw_ik.data && j >= out_ik.cap))
-    return;
-  const long long first = (long long)stride * (j + 1) - pool;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const SlotLayout lk = slot_layout(raw_k);
   const SlotLayout lv = raw_v.data ? slot_layout(raw_v) : lk;
   const SlotLayout li = raw_ik.data ? slot_layout(raw_ik) : lk;
+  const int D = raw_k.dims();
+  const int Dv = raw_v.data ? raw_v.dims() : 0, Di = raw_ik.data ? raw_ik.dims() : 0;
   uint8_t *bk = csm;
   uint8_t *bv = bk + (size_t)pool * lk.bytes;
   uint8_t *bi = bv + (raw_v.data ? (size_t)pool * lv.bytes : 0);
-  float *a = reinterpret_cast<float *>(bi + (raw_ik.data ? (size_t)pool * li.bytes : 0));
-  float *pooled = a + pool;
-  const int D = raw_k.dims();
-  int dmax = D;
-  if (raw_v.data && raw_v.dims() > dmax) dmax = raw_v.dims();
-  if (raw_ik.data && raw_ik.dims() > dmax) dmax = raw_ik.dims();
-  long long *rows = reinterpret_cast<long long *>(
-      (reinterpret_cast<uintptr_t>(pooled + dmax) + 7) & ~uintptr_t(7));
+  float *gw = reinterpret_cast<float *>(bi + (raw_ik.data ? (size_t)pool * li.bytes : 0));
+  float *gb = gw + round16(D);
+  float *a = gb + round16(pool);
+  float *pk = a + round16(pool);           // pooled key, value, indexer key
+  float *pv = pk + round16(D);
+  float *pi = pv + round16(Dv);
+  long long *rows = reinterpret_cast<long long *>(pi + round16(Di));
   long long *rows_v = rows + pool;
   long long *rows_i = rows_v + pool;
+
+  // the gate weights and biases travel while the token counts load
+  stage_bytes(reinterpret_cast<uint8_t *>(gw), reinterpret_cast<const uint8_t *>(gate_w), 4 * D,
+              tid, kThreads);
+  stage_bytes(reinterpret_cast<uint8_t *>(gb), reinterpret_cast<const uint8_t *>(gate_b),
+              4 * pool, tid, kThreads);
+  const long long j = t_begin[b] / stride + blockIdx.x;
+  // never write past a cache's capacity, whatever the device-side token counts say
+  if (j >= t_end[b] / stride || j < 0 || j >= out_k.cap || (raw_v.data && j >= out_v.cap) ||
+      (raw_ik.data && j >= out_ik.cap)) {
+    cp_async_wait_all();
+    return;
+  }
+  const long long first = (long long)stride * (j + 1) - pool;
 
   // slot rows of the window's positions, one modulo per position
   for (int r = tid; r < pool; r += blockDim.x) {
@@ -280,10 +290,10 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
     float acc = 0.f;
     if (p >= 0) {
       const uint8_t *slot = bk + (size_t)r * lk.bytes;
-      for (int d = lane; d < D; d += 32) acc = fmaf(__ldg(gate_w + d), staged_value(raw_k, lk, slot, d), acc);
+      for (int d = lane; d < D; d += 32) acc = fmaf(gw[d], staged_value(raw_k, lk, slot, d), acc);
     }
     acc = warp_sum(acc);
-    if (lane == 0) a[r] = p >= 0 ? acc + gate_b[r] : -CUDART_INF_F;
+    if (lane == 0) a[r] = p >= 0 ? acc + gb[r] : -CUDART_INF_F;
   }
   __syncthreads();
   if (warp == 0) {
@@ -299,21 +309,15 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   }
   __syncthreads();
 
-  pool_staged(raw_k, lk, bk, first, pool, a, pooled);
+  // pooled sums of every plane (no barrier between the planes)
+  pool_staged(raw_k, lk, bk, first, pool, a, pk);
+  if (raw_v.data) pool_staged(raw_v, lv, bv, first, pool, a, pv);
+  if (raw_ik.data) pool_staged(raw_ik, li, bi, first, pool, a, pi);
   __syncthreads();
-  store_entry(out_k, b, j, pooled, D);
-  __syncthreads();
-  if (raw_v.data) {
-    pool_staged(raw_v, lv, bv, first, pool, a, pooled);
-    __syncthreads();
-    store_entry(out_v, b, j, pooled, raw_v.dims());
-    __syncthreads();
-  }
-  if (raw_ik.data) {
-    pool_staged(raw_ik, li, bi, first, pool, a, pooled);
-    __syncthreads();
-    store_entry(out_ik, b, j, pooled, raw_ik.dims());
-  }
+  // re-quantisation and stores (no shared memory is written from here on)
+  store_entry(out_k, b, j, pk, D);
+  if (raw_v.data) store_entry(out_v, b, j, pv, Dv);
+  if (raw_ik.data) store_entry(out_ik, b, j, pi, Di);
 }
 
 }  // namespace
@@ -331,8 +335,12 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
   size_t staged = (size_t)pool * slot_layout(raw_k).bytes;
   if (raw_v.data) staged += (size_t)pool * slot_layout(raw_v).bytes;
   if (raw_ik.data) staged += (size_t)pool * slot_layout(raw_ik).bytes;
-  const size_t smem_staged = staged + sizeof(float) * (size_t)(pool + dmax + 1) +
-                             3 * sizeof(long long) * (size_t)pool + 16;
+  const int Dk = raw_k.dims(), Dv = raw_v.data ? raw_v.dims() : 0;
+  const int Di = raw_ik.data ? raw_ik.dims() : 0;
+  const size_t smem_staged =
+      staged +
+      sizeof(float) * (size_t)(2 * round16(Dk) + 2 * round16(pool) + round16(Dv) + round16(Di)) +
+      3 * sizeof(long long) * (size_t)pool + 16;
   if (smem_staged <= 200 * 1024 && ensure_dynamic_smem(compress_staged_kernel, smem_staged)) {
     if (launch_pdl(compress_staged_kernel, grid, dim3(kThreads), smem_staged, st, t_begin, t_end,
                    raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride, out_k, out_v,

@@ -88,6 +88,12 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Drop a dead 128-byte line of scratch memory from L2 without writing it back
+// to HBM (its contents become undefined).  `p` is 128-byte aligned.
+__device__ __forceinline__ void discard_l2_line(const void *p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 // Opt a kernel in to `bytes` of dynamic shared memory (host, idempotent).
 // Returns false when the request does not fit next to the kernel's static
 // shared memory.  Clears the error it may leave behind.

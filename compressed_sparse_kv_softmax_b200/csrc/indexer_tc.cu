@@ -19,7 +19,7 @@
 //   warp 1      MMA issuer (one thread): 4 tcgen05.mma per tile into one of
 //               kAcc TMEM accumulator slots (2 x 64 fp32 columns each)
 //   warp 2      TMEM allocation
-//   warps 4-11  two epilogue warpgroups taking alternate tiles: tcgen05.ld,
+//   warps 4-15  three epilogue warpgroups taking tiles in turn: tcgen05.ld,
 //               block scales, per-head ReLU, head weights -> score; score
 //               histogram (top 12 bits of the order-preserving key) for the
 //               selection kernel
@@ -42,13 +42,15 @@ constexpr int kHeads = 64;          // MMA N
 constexpr int kDim = 128;           // bytes per key (FP8 dims)
 constexpr int kStages = 8;
 constexpr int kAcc = 4;             // TMEM accumulator slots, 128 columns each
-constexpr int kEpiWarps = 8;
+constexpr int kEpiGroups = 3;       // epilogue warpgroups, taking tiles in turn
+constexpr int kEpiWarps = 4 * kEpiGroups;
 constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr uint32_t kTileBytes = kTile * kDim;
 constexpr uint32_t kIdesc = idesc(kFmtE4M3, kFmtE4M3, 0, 0, kTile, kHeads);
 
 struct __align__(1024) Smem {
   uint8_t keys[kStages][kTileBytes];      // 1024-aligned tiles
+  float2 kscale[kStages][kTile];          // the tiles' per-entry block scales
   uint8_t q[kHeads * kDim];               // B operand, K-major, 128-byte swizzle
   float c0[kHeads], c1[kHeads], w[kHeads]; // per head: block-0 and block-1 query scale, weight
   uint32_t hist[kTopkBins];
@@ -96,10 +98,15 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   const int b = row / a.Tq;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
+    // a stage is free again once its MMAs have completed (one commit) and
+    // the epilogue warpgroup of its tile has read the scales (128 arrivals)
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1 + 128);
+    }
     for (int s = 0; s < kAcc; ++s) {
       mbar_init(&sm.acc_full[s], 1);
-      mbar_init(&sm.acc_empty[s], 32 * kEpiWarps / 2);
+      mbar_init(&sm.acc_empty[s], 128);
     }
     mbar_init(&sm.mma_done, 1);
     sm.abort = 0;
@@ -145,6 +152,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
 
   if (warp == 0) {
     // ---------------- TMA producer
+    const long long total_rows = (long long)a.B * a.ik.cap;
     if (elect_one()) {
       int issued = 0;
       for (int i = 0; i < my_tiles && !sm.abort; ++i) {
@@ -155,8 +163,17 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
           break;
         }
         const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
-        mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
-        tma_load_2d(sm.keys[s], &tmap, &sm.full[s], 0, (int32_t)((long long)b * a.ik.cap + j0));
+        const long long g0 = (long long)b * a.ik.cap + j0;    // first row of the tile
+        // scales of the rows that exist (the key TMA zero-fills past the end;
+        // a bulk copy must not read past it): whole 16-byte pairs of rows
+        long long rows = total_rows - g0;
+        rows = rows < kTile ? rows : kTile;
+        const uint32_t sbytes = (uint32_t)(rows * 8) & ~15u;
+        mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
+        tma_load_2d(sm.keys[s], &tmap, &sm.full[s], 0, (int32_t)g0);
+        if (sbytes)
+          bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + g0 * 8, sbytes,
+                    &sm.full[s]);
         ++issued;
       }
       // never leave while a copy into this CTA's shared memory is in flight
@@ -197,27 +214,42 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm, err, 4);
     }
   } else if (warp >= 4) {
-    // ---------------- epilogue: two warpgroups take alternate tiles
-    const int grp = (warp - 4) >> 2;          // 0 or 1
+    // ---------------- epilogue: the warpgroups take tiles in turn
+    const int grp = (warp - 4) >> 2;          // 0 .. kEpiGroups-1
     const int quad = warp & 3;                // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;           // entry within the tile
     float *srow = scores + (size_t)row * ld;
     const uint8_t *scale_base = reinterpret_cast<const uint8_t *>(a.ik.scale);
-    for (int i = grp; i < my_tiles; i += 2) {
+    const long long total_rows = (long long)a.B * a.ik.cap;
+    for (int i = grp; i < my_tiles; i += kEpiGroups) {
       const int acc = i % kAcc;
+      const int s = i % kStages;
       const long long j = (long long)(blockIdx.x + i * gridDim.x) * kTile + r;
-      float sk0 = 0.f, sk1 = 0.f;
-      if (j < n) {
-        const float *sp = reinterpret_cast<const float *>(
-            scale_base + ((long long)b * a.ik.cap + j) * a.ik.scale_stride);
-        sk0 = __ldg(sp);
-        sk1 = __ldg(sp + 1);
-      }
       if (!mbar_wait(&sm.acc_full[acc], (i / kAcc) & 1)) {
         record_abort(sm, err, 8);
         break;
       }
       tc_fence_after();
+      // the tile's scales arrived with its keys; the stage cannot be refilled
+      // before this warpgroup arrives on its empty barrier, so the wait on
+      // the stage's full barrier (for visibility of the copy) returns at once.
+      // An odd last row of the whole cache came without them: plain load.
+      mbar_wait(&sm.full[s], (i / kStages) & 1);
+      float sk0 = 0.f, sk1 = 0.f;
+      if (j < n) {
+        const long long g = (long long)b * a.ik.cap + j;
+        const long long tile_rows = total_rows - (g - r);   // rows from the tile's first
+        if (!(g == total_rows - 1 && tile_rows < kTile && (tile_rows & 1))) {
+          const float2 v = sm.kscale[s][r];
+          sk0 = v.x;
+          sk1 = v.y;
+        } else {
+          const float *sp = reinterpret_cast<const float *>(scale_base + g * 8);
+          sk0 = __ldg(sp);
+          sk1 = __ldg(sp + 1);
+        }
+      }
+      mbar_arrive(&sm.empty[s]);
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * 128;
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
       const float2 k0 = make_float2(sk0, sk0), k1 = make_float2(sk1, sk1);
@@ -250,9 +282,13 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
         }
       }
       const float sc = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+      // histogram: one shared-memory atomic per distinct bucket of the warp
+      const unsigned live = __ballot_sync(0xffffffffu, j < n);
       if (j < n) {
         srow[j] = sc;
-        atomicAdd(&sm.hist[score_key(sc) >> kTopkShift], 1u);
+        const uint32_t bin = score_key(sc) >> kTopkShift;
+        const unsigned peers = __match_any_sync(live, bin);
+        if ((peers & ((1u << lane) - 1u)) == 0u) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
       }
     }
   }
@@ -292,6 +328,9 @@ bool indexer_tc_supported(const IndexerArgs &a) {
   if (a.ik.fmt != CSKV_FMT_E4M3_BF16 || a.d_I != kDim || a.H_I != kHeads) return false;
   if ((long long)a.B * a.ik.cap >= (1LL << 31)) return false;
   if (((uintptr_t)a.ik.data & 15) || (a.ik.data_stride & 15)) return false;
+  // scales: two fp32 per entry back to back, each tile's block 16-byte aligned
+  if (a.ik.scale_stride != 8 || ((uintptr_t)a.ik.scale & 15)) return false;
+  if (a.B > 1 && (a.ik.cap & 1)) return false;
   if ((uintptr_t)a.q_ik & 15) return false;
   int dev = 0, major = 0;
   cudaGetDevice(&dev);

@@ -253,10 +253,27 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   pdl_trigger();
   const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nsplit = gridDim.x, me = blockIdx.x;
-  const long long n = visible(q_pos, row, stride, max_entries);
   const float *s = w.scores + (long long)row * w.ld;
   int32_t *oi = out_idx + (long long)row * k;
   float *os = out_score ? out_score + (long long)row * k : nullptr;
+  // slices follow the host bound, so this CTA's first scores, the histogram
+  // and the row's position are all requested before any of them is used
+  const long long per = ((max_entries + nsplit - 1) / nsplit + kSelPer - 1) / kSelPer * kSelPer;
+  const long long j_lo = (long long)me * per;
+  const long long j_cap = j_lo + per < max_entries ? j_lo + per : max_entries;
+  const long long pos = q_pos[row];
+  constexpr int kHPer = kTopkBins / kSelThreads;
+  uint32_t hv[kHPer];
+  {
+    const uint32_t *hrow = w.hist + (size_t)row * kTopkBins;
+#pragma unroll
+    for (int e = 0; e < kHPer; ++e) hv[e] = __ldcg(hrow + tid + e * kSelThreads);
+  }
+  float keep[kSelPer];                 // the first pass's scores
+  load8(s, j_lo + (long long)tid * kSelPer, j_cap, keep);
+  long long n = (pos + 1) / stride;
+  if (n > max_entries) n = max_entries;
+  if (n < 0) n = 0;
 
   if (n <= k) {            // every visible entry is selected, already in order
     if (me == 0) {
@@ -270,35 +287,26 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
 
   // ---- 1. threshold bucket b*, this slice's winners and candidates
   if (tid == 0) { sm.bstar = 0; sm.above = -1; sm.wins = 0; }
-  {
-    const uint32_t *hrow = w.hist + (size_t)row * kTopkBins;
-    constexpr int kPer = kTopkBins / kSelThreads;
-    uint32_t v[kPer];
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) v[e] = __ldcg(hrow + tid + e * kSelThreads);
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) sm.hist[tid + e * kSelThreads] = v[e];
-  }
+  for (int e = 0; e < kHPer; ++e) sm.hist[tid + e * kSelThreads] = hv[e];
   __syncthreads();
   find_threshold_bin([&](int i) { return sm.hist[i]; }, kTopkBins, k, sm.scan, &sm.bstar,
                      &sm.above);
   const uint32_t bstar = (uint32_t)sm.bstar;
   const int above = sm.above;
 
-  const long long per = ((n + nsplit - 1) / nsplit + kSelPer - 1) / kSelPer * kSelPer;
-  const long long j_lo = (long long)me * per;
   const long long j_hi = j_lo + per < n ? j_lo + per : n;
   uint32_t *ctr = w.ctr + (size_t)row * 4;
   uint64_t *candrow = w.cand + (size_t)row * kCandCap;
-  float keep[kSelPer];                 // the first pass's scores, reused in step 4
   int wins = 0;
   for (long long c0 = j_lo; c0 < j_hi; c0 += kSelChunk) {
     const long long j0 = c0 + (long long)tid * kSelPer;
     float v[kSelPer];
-    load8(s, j0, j_hi, v);
     if (c0 == j_lo) {
 #pragma unroll
-      for (int e = 0; e < kSelPer; ++e) keep[e] = v[e];
+      for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
+    } else {
+      load8(s, j0, j_hi, v);
     }
     int nc = 0;
     uint32_t cmask = 0;
@@ -360,6 +368,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
 
   // ---- 3. the exact k-th key among the candidates (same result in every CTA)
   uint32_t thr = 0, tie_cut = 0xffffffffu;
+  // per-slice winner counts, requested now and used after the refinement
+  const int wins_c = tid < nsplit ? (int)__ldcg(w.wins + (size_t)row * kMaxSplits + tid) : 0;
   if (!fallback) {
     {
       constexpr int kC = kCandCap / kSelThreads;
@@ -375,25 +385,62 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
         if (i < n_cand) sm.cand[i] = v[e];
       }
     }
-    // radix select of the r-th largest candidate key on bits 19..10, then 9..0
-    uint32_t prefix = bstar << kTopkShift, mask = 0xFFFu << kTopkShift;
+    // radix select of the r-th largest candidate key (all candidates share
+    // the bucket bits): bits 19..8 in one 4096-bin pass, then the few
+    // candidates left in the chosen bin by one warp (up to 32 of them) or by
+    // a 256-bin pass over bits 7..0
+    uint32_t prefix = bstar << kTopkShift;
     int remaining = r;
-    for (int pass = 0; pass < 2; ++pass) {
-      const int shift = 10 - 10 * pass;
-      for (int i = tid; i < 1024; i += blockDim.x) sm.hist[i] = 0;
+    for (int i = tid; i < kTopkBins; i += blockDim.x) sm.hist[i] = 0;
+    if (tid == 0) { sm.thr_bin = 0; sm.take = 0; sm.n_eq = 0; }
+    __syncthreads();
+    for (int i = tid; i < n_cand; i += blockDim.x)
+      atomicAdd(&sm.hist[((uint32_t)sm.cand[i] >> 8) & 4095u], 1u);
+    __syncthreads();
+    find_threshold_bin([&](int i) { return sm.hist[i]; }, kTopkBins, remaining, sm.scan,
+                       &sm.thr_bin, &sm.take);
+    prefix |= (uint32_t)sm.thr_bin << 8;
+    remaining -= sm.take;
+    const int in_bin = (int)sm.hist[sm.thr_bin];
+    __syncthreads();
+    if (in_bin <= 32) {
+      uint32_t *lst = sm.hist;           // keys of the bin's candidates
+      if (tid == 0) sm.take = 0;         // stays 0 (-> fall-back) if no rank matches
+      for (int i = tid; i < n_cand; i += blockDim.x) {
+        const uint32_t key = (uint32_t)sm.cand[i];
+        if ((key >> 8) == (prefix >> 8)) lst[atomicAdd(&sm.n_eq, 1)] = key;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        const int cnt = sm.n_eq;
+        const uint32_t mine = lane < cnt ? lst[lane] : 0u;
+        int gt = 0, ge = 0;
+        for (int m = 0; m < cnt; ++m) {
+          const uint32_t o = __shfl_sync(0xffffffffu, mine, m);
+          gt += o > mine;
+          ge += o >= mine;
+        }
+        // the key whose rank range covers `remaining`; equal keys agree
+        if (lane < cnt && gt < remaining && remaining <= ge) {
+          sm.thr_bin = (int)(mine & 255u);
+          sm.take = remaining - gt;
+        }
+      }
+      __syncthreads();
+      prefix |= (uint32_t)sm.thr_bin;
+      remaining = sm.take;
+    } else {
+      for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
       __syncthreads();
       for (int i = tid; i < n_cand; i += blockDim.x) {
         const uint32_t key = (uint32_t)sm.cand[i];
-        if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 1023u], 1u);
+        if ((key >> 8) == (prefix >> 8)) atomicAdd(&sm.hist[key & 255u], 1u);
       }
       __syncthreads();
-      if (tid == 0) { sm.thr_bin = 0; sm.take = 0; }
-      find_threshold_bin([&](int i) { return sm.hist[i]; }, 1024, remaining, sm.scan, &sm.thr_bin,
+      find_threshold_bin([&](int i) { return sm.hist[i]; }, 256, remaining, sm.scan, &sm.thr_bin,
                          &sm.take);
-      prefix |= (uint32_t)sm.thr_bin << shift;
+      prefix |= (uint32_t)sm.thr_bin;
       remaining -= sm.take;
-      mask |= 1023u << shift;
-      __syncthreads();
     }
     thr = prefix;
     const int take_eq = remaining;     // keys equal to thr to take, lowest indices first
@@ -425,8 +472,7 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
 
   // ---- per-slice counts of the selection, and this slice's output offset
   if (!fallback) {
-    for (int c = tid; c < nsplit; c += blockDim.x)
-      sm.cnt[c] = (int)__ldcg(w.wins + (size_t)row * kMaxSplits + c);
+    if (tid < nsplit) sm.cnt[tid] = wins_c;
     __syncthreads();
     for (int i = tid; i < n_cand; i += blockDim.x) {
       const uint64_t c = sm.cand[i];
