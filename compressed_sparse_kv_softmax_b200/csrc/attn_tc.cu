@@ -71,7 +71,7 @@ struct __align__(1024) Smem {
   float red[4][kHeads];
   float m[kHeads], l[kHeads], inv_l[kHeads], alpha[kHeads];
   long long slot[kM];
-  uint64_t bar;
+  uint64_t bar, gbar;
   uint32_t tmem_base;
 };
 
@@ -152,6 +152,84 @@ __device__ __forceinline__ void stage_q(const __nv_bfloat16 *__restrict__ qg, ui
   }
 }
 
+// Raw key rows of one unit staged in the (not yet used) Q buffer: FP8 codes
+// [64][448], block scales [64][32 B], RoPE [64][128 B].  Used for units whose
+// keys are consecutive cache slots (dense compressed entries, the window) in
+// a cache whose planes have exactly these row pitches: each run of slots
+// then arrives with three bulk copies.
+constexpr uint32_t kStgScale = kKeys * kDn, kStgRope = kStgScale + kKeys * 32;
+constexpr uint32_t kRowBytes = kDn + 32 + 2 * kDr;    // bytes one row brings
+static_assert(kStgRope + kKeys * 2 * kDr <= 8 * kChunkQ, "staging fits the Q buffer");
+
+__host__ __device__ inline bool dense_rows(const Cache &c) {
+  return c.data_stride == kDn && c.scale_stride == 32 && c.rope_stride == 2 * kDr &&
+         !(((uintptr_t)c.data | (uintptr_t)c.scale | (uintptr_t)c.rope) & 15);
+}
+
+__device__ __forceinline__ void load_q(const __nv_bfloat16 *__restrict__ qg, uint4 (&raw)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    raw[e] = __ldg(reinterpret_cast<const uint4 *>(qg) + threadIdx.x + e * kThreads);
+}
+__device__ __forceinline__ void store_q(const uint4 (&raw)[16], uint8_t *q) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int i = threadIdx.x + e * kThreads;
+    const int h = i >> 6, c = (i >> 3) & 7, u = i & 7;  // 8 dims per unit
+    const __nv_bfloat162 *bp = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
+    uint4 o;
+    uint32_t *op = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(bp[k]);
+      op[k] = pack_h2(f.x, f.y);
+    }
+    *reinterpret_cast<uint4 *>(q + c * kChunkQ + swz(h, u)) = o;
+  }
+}
+
+// Convert key row r (16 FP8 codes x block scale on lanes 0-27, 16 BF16 RoPE
+// values on lanes 28-31) into its hi and lo FP16 parts in the key tile.
+__device__ __forceinline__ void convert_row(uint8_t *kt, int r, int lane, const uint4 &raw,
+                                            const uint4 &raw2, float sc) {
+  uint4 h0, h1, l0, l1;
+  uint32_t *ph0 = reinterpret_cast<uint32_t *>(&h0), *ph1 = reinterpret_cast<uint32_t *>(&h1);
+  uint32_t *pl0 = reinterpret_cast<uint32_t *>(&l0), *pl1 = reinterpret_cast<uint32_t *>(&l1);
+  int d0;
+  if (lane < 28) {
+    const uint32_t *cw = reinterpret_cast<const uint32_t *>(&raw);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 x = e4m3x2(cw[q] & 0xffffu), y = e4m3x2(cw[q] >> 16);
+      if (q < 2) {
+        split_h2(x.x * sc, x.y * sc, ph0[2 * q], pl0[2 * q]);
+        split_h2(y.x * sc, y.y * sc, ph0[2 * q + 1], pl0[2 * q + 1]);
+      } else {
+        split_h2(x.x * sc, x.y * sc, ph1[2 * q - 4], pl1[2 * q - 4]);
+        split_h2(y.x * sc, y.y * sc, ph1[2 * q - 3], pl1[2 * q - 3]);
+      }
+    }
+    d0 = lane * 16;
+  } else {
+    const __nv_bfloat162 *b0 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    const __nv_bfloat162 *b1 = reinterpret_cast<const __nv_bfloat162 *>(&raw2);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f0 = __bfloat1622float2(b0[q]), f1 = __bfloat1622float2(b1[q]);
+      split_h2(f0.x, f0.y, ph0[q], pl0[q]);
+      split_h2(f1.x, f1.y, ph1[q], pl1[q]);
+    }
+    d0 = kDn + (lane - 28) * 16;
+  }
+  // hi part in row r, lo part in row 64 + r of the chunk (same swizzle phase)
+  const int c = d0 >> 6, u = (d0 & 63) >> 3;
+  const uint32_t o0 = c * kChunkKK + swz(r, u), o1 = c * kChunkKK + swz(r, u + 1);
+  *reinterpret_cast<uint4 *>(kt + o0) = h0;
+  *reinterpret_cast<uint4 *>(kt + o1) = h1;
+  *reinterpret_cast<uint4 *>(kt + kChunkK + o0) = l0;
+  *reinterpret_cast<uint4 *>(kt + kChunkK + o1) = l1;
+}
+
 struct Row {
   long long pos, n_comp, w_lo;
   int n_win;
@@ -185,6 +263,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
 
   if (tid == 0) {
     mbar_init(&sm.bar, 1);
+    mbar_init(&sm.gbar, 1);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -238,74 +317,91 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     if (!__syncthreads_or(tid < kM && sm.slot[tid] >= 0)) continue;
     const bool my_valid = sm.slot[krow] >= 0;
 
-    // ---- gather: each warp takes 8 consecutive key rows; all loads are
-    // issued first, then (first unit only) Q is staged while they are in
-    // flight, then the rows are converted
+    // ---- gather: warp w converts key rows 8w .. 8w+7 into the key tile
     const int r0 = warp * 8;
     const bool has_rows = r0 < ksteps * 16;   // kKeys = 8 warps x 8 rows
-    uint4 raw[8], raw2[8];
-    float sc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
-      sc[e] = 0.f;
-      const long long slot = has_rows ? sm.slot[r0 + e] : -1;
-      if (slot < 0) continue;
-      if (lane < 28) {
-        raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
-        sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
-      } else {
-        const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
-        raw[e] = __ldg(rp);
-        raw2[e] = __ldg(rp + 1);
+    const __nv_bfloat16 *qg =
+        reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD;
+    // consecutive slots: the window's positions (one or two runs around the
+    // ring) or dense compressed entries (one run)
+    const bool runs_ok = !q_ready && dense_rows(src) && !(comp_unit && a.sel);
+    if (runs_ok) {
+      // first unit: bulk copies bring the rows into the still unused Q buffer
+      // while Q itself is loaded into registers; the rows are converted from
+      // shared memory, then Q takes its buffer
+      if (tid == 0) {
+        long long s0, len0;
+        if (comp_unit) {
+          s0 = base;
+          len0 = nkeys;
+        } else {
+          s0 = src.slot_of(R.w_lo + base);
+          len0 = src.cap - s0 < nkeys ? src.cap - s0 : nkeys;
+        }
+        mbar_arrive_expect_tx(&sm.gbar, (uint32_t)nkeys * kRowBytes);
+        const long long s_run[2] = {s0, 0};
+        const int r_run[2] = {0, (int)len0}, n_run[2] = {(int)len0, nkeys - (int)len0};
+        for (int k = 0; k < 2; ++k) {
+          if (n_run[k] <= 0) continue;
+          const int r = r_run[k], n = n_run[k];
+          bulk_load(sm.q + r * kDn, src.data_ptr(b, s_run[k]), n * kDn, &sm.gbar);
+          bulk_load(sm.q + kStgScale + r * 32, src.scale_ptr(b, s_run[k]), n * 32, &sm.gbar);
+          bulk_load(sm.q + kStgRope + r * 2 * kDr, src.rope_ptr(b, s_run[k]), n * 2 * kDr,
+                    &sm.gbar);
+        }
       }
-    }
-    if (!q_ready) {
-      stage_q(reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD, sm.q);
-      q_ready = true;
-    }
-    if (has_rows) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int r = r0 + e;
-        uint4 h0, h1, l0, l1;
-        uint32_t *ph0 = reinterpret_cast<uint32_t *>(&h0), *ph1 = reinterpret_cast<uint32_t *>(&h1);
-        uint32_t *pl0 = reinterpret_cast<uint32_t *>(&l0), *pl1 = reinterpret_cast<uint32_t *>(&l1);
-        int d0;
-        if (lane < 28) {
-          // 16 FP8 codes: dims 16*lane .. +15, block scale lane/4 (absent key: zeros)
-          const uint32_t *cw = reinterpret_cast<const uint32_t *>(&raw[e]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 x = e4m3x2(cw[q] & 0xffffu), y = e4m3x2(cw[q] >> 16);
-            if (q < 2) {
-              split_h2(x.x * sc[e], x.y * sc[e], ph0[2 * q], pl0[2 * q]);
-              split_h2(y.x * sc[e], y.y * sc[e], ph0[2 * q + 1], pl0[2 * q + 1]);
+      uint4 qraw[16];
+      load_q(qg, qraw);
+      ok = mbar_wait(&sm.gbar, 0) && ok;     // used once per CTA: phase 0
+      if (has_rows) {
+        for (int e = 0; e < 8; ++e) {
+          const int r = r0 + e;
+          uint4 raw = make_uint4(0, 0, 0, 0), raw2 = make_uint4(0, 0, 0, 0);
+          float sc = 0.f;
+          if (r < nkeys) {
+            if (lane < 28) {
+              raw = *reinterpret_cast<const uint4 *>(sm.q + r * kDn + 16 * lane);
+              sc = *reinterpret_cast<const float *>(sm.q + kStgScale + r * 32 + 4 * (lane >> 2));
             } else {
-              split_h2(x.x * sc[e], x.y * sc[e], ph1[2 * q - 4], pl1[2 * q - 4]);
-              split_h2(y.x * sc[e], y.y * sc[e], ph1[2 * q - 3], pl1[2 * q - 3]);
+              const uint4 *rp =
+                  reinterpret_cast<const uint4 *>(sm.q + kStgRope + r * 2 * kDr) + 2 * (lane - 28);
+              raw = rp[0];
+              raw2 = rp[1];
             }
           }
-          d0 = lane * 16;
-        } else {
-          // 16 BF16 RoPE dims: 448 + 16 * (lane - 28) ..
-          const __nv_bfloat162 *b0 = reinterpret_cast<const __nv_bfloat162 *>(&raw[e]);
-          const __nv_bfloat162 *b1 = reinterpret_cast<const __nv_bfloat162 *>(&raw2[e]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f0 = __bfloat1622float2(b0[q]), f1 = __bfloat1622float2(b1[q]);
-            split_h2(f0.x, f0.y, ph0[q], pl0[q]);
-            split_h2(f1.x, f1.y, ph1[q], pl1[q]);
-          }
-          d0 = kDn + (lane - 28) * 16;
+          convert_row(sm.kt, r, lane, raw, raw2, sc);
         }
-        const int c = d0 >> 6, u = (d0 & 63) >> 3;
-        // hi part in row r, lo part in row 64 + r of the chunk (same swizzle phase)
-        const uint32_t o0 = c * kChunkKK + swz(r, u), o1 = c * kChunkKK + swz(r, u + 1);
-        *reinterpret_cast<uint4 *>(sm.kt + o0) = h0;
-        *reinterpret_cast<uint4 *>(sm.kt + o1) = h1;
-        *reinterpret_cast<uint4 *>(sm.kt + kChunkK + o0) = l0;
-        *reinterpret_cast<uint4 *>(sm.kt + kChunkK + o1) = l1;
+      }
+      __syncthreads();                        // every staged row has been read
+      store_q(qraw, sm.q);
+      q_ready = true;
+    } else {
+      // all loads are issued first, then (first unit only) Q is staged while
+      // they are in flight, then the rows are converted
+      uint4 raw[8], raw2[8];
+      float sc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
+        sc[e] = 0.f;
+        const long long slot = has_rows ? sm.slot[r0 + e] : -1;
+        if (slot < 0) continue;
+        if (lane < 28) {
+          raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
+          sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
+        } else {
+          const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
+          raw[e] = __ldg(rp);
+          raw2[e] = __ldg(rp + 1);
+        }
+      }
+      if (!q_ready) {
+        stage_q(qg, sm.q);
+        q_ready = true;
+      }
+      if (has_rows) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) convert_row(sm.kt, r0 + e, lane, raw[e], raw2[e], sc[e]);
       }
     }
     fence_proxy_async_shared();

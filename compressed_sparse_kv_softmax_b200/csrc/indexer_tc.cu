@@ -123,11 +123,19 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   const uint32_t tmem = sm.tmem_base;
   pdl_wait();                      // global memory from here on
   pdl_trigger();
-  long long n = (a.q_pos[row] + 1) / a.stride;
-  if (n > a.max_entries) n = a.max_entries;
-  if (n < 0) n = 0;
-  const int tiles = (int)((n + kTile - 1) / kTile);
-  const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / gridDim.x + 1 : 0;
+  const long long qpos = a.q_pos[row];
+  // tiles of this CTA for n visible entries (tile t goes to CTA t % grid)
+  auto tiles_of = [&](long long nn) {
+    const int tl = (int)((nn + kTile - 1) / kTile);
+    return tl > (int)blockIdx.x ? (tl - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  };
+  // visible entries of the row (each role asks for it only where it needs it,
+  // so the producer is not held up by the position's load)
+  auto visible_n = [&]() {
+    long long nn = (qpos + 1) / a.stride;
+    if (nn > a.max_entries) nn = a.max_entries;
+    return nn < 0 ? 0LL : nn;
+  };
   if (warp != 0) {
     // query heads -> B operand (K-major, 128-byte swizzle: 16-byte chunk c of
     // head h lands at chunk c ^ (h & 7) of its 128-byte row); the producer
@@ -154,14 +162,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
     // ---------------- TMA producer
     const long long total_rows = (long long)a.B * a.ik.cap;
     if (elect_one()) {
-      int issued = 0;
-      for (int i = 0; i < my_tiles && !sm.abort; ++i) {
+      auto issue = [&](int i) {
         const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
-        if (i >= kStages && !mbar_wait(&sm.empty[s], ph ^ 1)) {
-          record_abort(sm, err, 1);
-          break;
-        }
         const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
         const long long g0 = (long long)b * a.ik.cap + j0;    // first row of the tile
         // scales of the rows that exist (the key TMA zero-fills past the end;
@@ -174,6 +176,21 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
         if (sbytes)
           bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + g0 * 8, sbytes,
                     &sm.full[s]);
+      };
+      // the first stages are filled from the host bound before the row's
+      // position has arrived (tiles past the visible ones are loaded, never used)
+      const int spec = min(kStages, tiles_of(a.max_entries));
+      int issued = 0;
+      for (; issued < spec; ++issued) issue(issued);
+      const int my_tiles = tiles_of(visible_n());
+      for (int i = spec; i < my_tiles && !sm.abort; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!mbar_wait(&sm.empty[s], ph ^ 1)) {
+          record_abort(sm, err, 1);
+          break;
+        }
+        issue(i);
         ++issued;
       }
       // never leave while a copy into this CTA's shared memory is in flight
@@ -183,6 +200,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (elect_one()) {
+      const int my_tiles = tiles_of(visible_n());
       int done = 0;
       for (int i = 0; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages, acc = i % kAcc;
@@ -215,6 +233,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: the warpgroups take tiles in turn
+    const long long n = visible_n();
+    const int my_tiles = tiles_of(n);
     const int grp = (warp - 4) >> 2;          // 0 .. kEpiGroups-1
     const int quad = warp & 3;                // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;           // entry within the tile
@@ -235,7 +255,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       // the stage's full barrier (for visibility of the copy) returns at once.
       // An odd last row of the whole cache came without them: plain load.
       mbar_wait(&sm.full[s], (i / kStages) & 1);
-      float sk0 = 0.f, sk1 = 0.f;
+      float sk0 = 1.f, sk1 = 0.f;            // (rows past n: score not stored)
       if (j < n) {
         const long long g = (long long)b * a.ik.cap + j;
         const long long tile_rows = total_rows - (g - r);   // rows from the tile's first
@@ -252,7 +272,14 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       mbar_arrive(&sm.empty[s]);
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * 128;
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      // x_h = sk0 (sq0_h a0_h + rho sq1_h a1_h) with rho = sk1 / sk0, and since
+      // sk0 > 0, w_h max(0, x_h) = sk0 w_h max(0, sq0_h a0_h + rho sq1_h a1_h):
+      // sk0 leaves the head loop.  A warp with an entry whose sk0 is not a
+      // positive number (or whose rho overflows) takes the direct form.
+      const float rho = sk1 / sk0;
+      const bool factored = __all_sync(0xffffffffu, j >= n || (sk0 > 0.f && fabsf(rho) <= 3.0e38f));
       const float2 k0 = make_float2(sk0, sk0), k1 = make_float2(sk1, sk1);
+      const float2 rr = make_float2(rho, rho);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         float a0[32], a1[32];
@@ -264,24 +291,42 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
           tc_fence_before();
           mbar_arrive(&sm.acc_empty[acc]);
         }
+        if (factored) {
 #pragma unroll
-        for (int h = 0; h < 32; h += 4) {
-          const int hg = half * 32 + h;
-          const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
-          const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
-          const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
-          // x = sk0 sq0 a0 + sk1 sq1 a1 for heads (h, h+1) and (h+2, h+3)
-          float2 x = fma2(mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)), k0,
-                          mul2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), k1));
-          float2 y = fma2(mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)), k0,
-                          mul2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), k1));
-          x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
-          y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
-          acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
-          acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+          for (int h = 0; h < 32; h += 4) {
+            const int hg = half * 32 + h;
+            const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
+            const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
+            const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
+            float2 x = fma2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), rr,
+                            mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)));
+            float2 y = fma2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), rr,
+                            mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)));
+            x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
+            y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
+            acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
+            acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 32; h += 4) {
+            const int hg = half * 32 + h;
+            const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
+            const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
+            const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
+            // x = sk0 sq0 a0 + sk1 sq1 a1 for heads (h, h+1) and (h+2, h+3)
+            float2 x = fma2(mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)), k0,
+                            mul2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), k1));
+            float2 y = fma2(mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)), k0,
+                            mul2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), k1));
+            x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
+            y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
+            acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
+            acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+          }
         }
       }
-      const float sc = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+      const float sc = ((acc0.x + acc0.y) + (acc1.x + acc1.y)) * (factored ? sk0 : 1.f);
       // histogram: one shared-memory atomic per distinct bucket of the warp
       const unsigned live = __ballot_sync(0xffffffffu, j < n);
       if (j < n) {
