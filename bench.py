@@ -7,8 +7,9 @@ on 1,048,576 (contexts 1,048,513 .. 1,048,640), one HCA period, so that the
 compressors run exactly where an entry completes: CSA compression on the 32
 tokens that close a 4-token group, HCA compression on the one token that
 closes a 128-token block.  Every step runs
-  CSA layer: [csa_compress] -> indexer_topk (score the ~262,144 visible
-             entries, keep 1,024) -> hybrid_attn_decode (1,024 + 128 window)
+  CSA layer: [csa_compress] -> indexer_score + indexer_select (= indexer_topk:
+             score the ~262,144 visible entries, keep 1,024)
+             -> hybrid_attn_decode (1,024 + 128 window)
   HCA layer: [hca_compress] -> hybrid_attn_decode (8,192 dense + 128 window)
 The metric is decode queries/s (one query = one token through both layers).
 
@@ -16,7 +17,8 @@ Inputs are seeded synthetic tensors resident in HBM.  R replicas of every
 layer's inputs rotate between steps; their per-step bytes total more than 4x
 the 126 MB L2, so each step reads HBM.  The timed region replays CUDA graphs
 of 128 steps (plus one graph of the remaining steps), exactly K steps.  The
-dominant call (indexer_topk) is bracketed by event records inside the graph.
+dominant kernel, the indexer's HBM scan (the indexer_score call), is
+bracketed by event records inside the graph.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -48,12 +50,19 @@ UNIT = "queries/s"
 
 # ------------------------------------------------------------------ helpers
 
-def _peaks():
+_FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks(kind="hbm_gbs"):
+    """A measured peak from MEASURED_PEAKS.json (HBM copy GB/s, or cuBLAS bf16
+    TFLOP/s as a burst or sustained), else the earlier measurement on this
+    pool that stands in for it."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        if kind in d:
+            return float(d[kind]), "measured"
+    return _FALLBACK_PEAKS[kind], "fallback"
 
 
 class ClockSampler:
@@ -150,15 +159,17 @@ class Replica:
 
     def step(self, s, mark=None):
         """Enqueue decode step s of the window on the current stream; mark(i)
-        records an event between calls (i = 0 before indexer_topk, 1 after)."""
+        records an event between calls (i = 0 before indexer_score, 1 after
+        it).  indexer_score + indexer_select is the indexer_topk call."""
         sc = self.sched
         if sc.csa_fires[s]:
             self.csa.compress(sc.tb[s], sc.te[s], 1)
         if mark:
             mark(0)
-        self.csa.select(sc.q_pos[s])
+        self.csa.select(sc.q_pos[s], phase="score")
         if mark:
             mark(1)
+        self.csa.select(sc.q_pos[s], phase="pick")
         self.csa.attend(pos=sc.ctx[s])
         if sc.hca_fires[s]:
             self.hca.compress(sc.tb[s], sc.te[s], 1)
@@ -183,7 +194,7 @@ EVENT_EVERY = 16  # steps between in-graph event pairs (each record node stalls 
 class StepGraph:
     """CUDA graph of G consecutive decode steps (step i of the timed sequence
     uses replica i % R and window position i % PERIOD), with external event
-    records around the indexer_topk call of every EVENT_EVERY-th step."""
+    records around the indexer scoring call of every EVENT_EVERY-th step."""
 
     def __init__(self, replicas, G, stream, i0=0):
         rt = _rt()
@@ -229,13 +240,14 @@ class StepGraph:
 
 
 def indexer_bytes(wl):
-    """Algorithmic bytes of one indexer_topk call: every visible CSA entry's
-    FP8 indexer key (d_I bytes) and its d_I/64 fp32 scales, the FP8 query
-    heads with scales, head weights, and the selected indices written."""
+    """Algorithmic HBM bytes of one indexer scoring launch: every visible CSA
+    entry's FP8 indexer key (d_I bytes) and its d_I/64 fp32 scales, the FP8
+    query heads with their scales and the head weights.  (The scores, 4 bytes
+    per entry, stay in L2 for the selection.)"""
     n_c = wl.T // wl.csa_stride
     per_entry = wl.d_I + 4 * (wl.d_I // 64)
     q = wl.H_I * wl.d_I + 4 * wl.H_I * (wl.d_I // 64) + 4 * wl.H_I
-    return wl.B * (n_c * per_entry + q + 4 * wl.k)
+    return wl.B * (n_c * per_entry + q)
 
 
 def step_bytes(wl):
@@ -246,7 +258,7 @@ def step_bytes(wl):
     n_h = wl.T // wl.hca_stride
     q = wl.Hq * wl.D * 2
     out = wl.Hq * wl.D * 4 + wl.Hq * 4
-    csa = indexer_bytes(wl) + wl.B * ((wl.k + wl.window) * entry + q + out)
+    csa = indexer_bytes(wl) + wl.B * (4 * wl.k + (wl.k + wl.window) * entry + q + out)
     hca = wl.B * ((n_h + wl.window) * entry + q + out)
     compress = wl.B * ((PERIOD // wl.csa_stride) * (wl.csa_pool * (entry + ik) + entry + ik)
                        + (PERIOD // wl.hca_stride) * (wl.hca_pool * entry + entry)) / PERIOD
@@ -315,7 +327,8 @@ def run_ours(args, rank, world, dev):
     achieved = ib / (idx_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": None,
-                "kernel": "indexer_topk (lightning-indexer scoring + top-k)",
+                "kernel": "indexer_tc_kernel (lightning-indexer scoring: the indexer_score "
+                          "call, histogram zeroing included)",
                 "peak_kind": f"{peak_kind} HBM copy bandwidth (burst)",
                 "algorithmic_bytes_per_launch": ib, "avg_launch_us": round(idx_ms * 1e3, 3),
                 "timed_launches": f"every {EVENT_EVERY}th step of the last graph replay"}
@@ -343,11 +356,11 @@ def run_ours(args, rank, world, dev):
     return res, replicas, wl
 
 
-_TRAFFIC_SOURCES = ["indexer.cu", "indexer_tc.cu", "topk.cu", "topk_common.cuh", "sm100.cuh"]
+_TRAFFIC_SOURCES = ["indexer.cu", "indexer_tc.cu", "topk_common.cuh", "sm100.cuh"]
 
 
 def _profile_traffic(workload):
-    """DRAM bytes per indexer_topk call from the committed ncu summary, when
+    """DRAM bytes per indexer scoring launch from the committed ncu summary, when
     the kernel sources still hash to the ones the counters were taken on
     (null otherwise: the counters describe another build)."""
     import hashlib
@@ -541,6 +554,102 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------- chunked prefill
+
+def run_prefill(args, rank, world, dev):
+    """Chunked prefill (--workload prefill): Tq new tokens per sequence on a
+    cached context.  One step = CSA layer (csa_compress of the chunk's
+    entries, indexer_score + indexer_select for every new token,
+    hybrid_attn_prefill) + HCA layer (hca_compress, hybrid_attn_prefill).
+    The step's tensors (queries, outputs, the score workspace) are far larger
+    than L2.  The metric is prefill tokens/s; the roofline object reports the
+    indexer scoring's tensor FLOP rate against the FP8 peak."""
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
+    wl = W.get(args.workload)
+    torch.cuda.set_device(dev)
+    csa = CSALayer(W.make_csa_layer(wl, device=dev, seed=1000 + 7919 * rank))
+    hca = HCALayer(W.make_hca_layer(wl, device=dev, seed=501000 + 7919 * rank))
+    tb = torch.full((wl.B,), wl.T, dtype=torch.int64, device=dev)
+    te = torch.full((wl.B,), wl.T + wl.Tq, dtype=torch.int64, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    names = ["csa_compress", "indexer_score", "indexer_select", "hybrid_attn_prefill (CSA)",
+             "hca_compress", "hybrid_attn_prefill (HCA)"]
+
+    def step(ev=None):
+        calls = [lambda: csa.compress(tb, te, wl.Tq // wl.csa_stride),
+                 lambda: csa.select(phase="score"), lambda: csa.select(phase="pick"),
+                 lambda: csa.attend(), lambda: hca.compress(tb, te, wl.Tq // wl.hca_stride),
+                 lambda: hca.attend()]
+        for i, c in enumerate(calls):
+            if ev:
+                ev[i].record(stream)
+            c()
+        if ev:
+            ev[-1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    K = max(1, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            step(evs[k])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    per_call = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(len(names))] for e in evs])
+    ms = float(sum(e[0].elapsed_time(e[-1]) for e in evs)) / K
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+    calls_ms = {n: round(float(v), 4) for n, v in zip(names, per_call.mean(axis=0))}
+    # FLOPs: visible entries differ per token of the chunk (causal)
+    pos = np.arange(wl.T, wl.T + wl.Tq)
+    n_c = ((pos + 1) // wl.csa_stride).astype(np.float64)
+    n_h = ((pos + 1) // wl.hca_stride).astype(np.float64)
+    win = np.minimum(pos + 1, wl.window)
+    idx_flop = wl.B * 2.0 * wl.H_I * wl.d_I * n_c.sum()
+    csa_flop = wl.B * 4.0 * wl.Hq * wl.D * (wl.k + win).sum()
+    hca_flop = wl.B * 4.0 * wl.Hq * wl.D * (n_h + win).sum()
+    # a step lasts far longer than a burst: the sustained GEMM figure
+    peak, peak_kind = _peaks(kind="bf16_tflops_sustained")
+    fp8_peak = 2.0 * peak            # the nominal FP8 : BF16 dense ratio
+    idx_tflops = idx_flop / (calls_ms["indexer_score"] / 1e3) / 1e12
+    tokens = wl.B * wl.Tq * world
+    res = {"metric": "chunked-prefill tokens/s (CSA+HCA layers, 8,192 new tokens on a "
+                     "1,048,576-token context)",
+           "value": round(tokens / (ms / 1e3), 2), "unit": "tokens/s", "n_gpus": world,
+           "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3/bf16 storage, fp32 math",
+           "data": "synthetic (seeded Gaussian FP8 E4M3 + BF16 caches)",
+           "config": {"workload": f"{wl.name}: B={wl.B}, {wl.Tq} new tokens at positions "
+                                  f"{wl.T}..{wl.T + wl.Tq - 1}, Hq={wl.Hq}, "
+                                  f"D={wl.d_nope}+{wl.d_rope}, H_I={wl.H_I}x{wl.d_I}, "
+                                  f"k={wl.k}, window={wl.window}",
+                      "l2": "per-step tensors (queries 0.5 GB, outputs 2 GB, scores 8.6 GB) "
+                            "far above L2"},
+           "roofline": {"bound": "tensor", "achieved": round(idx_tflops, 2),
+                        "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                        "frac": round(idx_tflops / fp8_peak, 4), "traffic": None,
+                        "kernel": "indexer_tc_kernel (indexer_score: FP8 scoring of every "
+                                  "visible entry for each new token)",
+                        "peak_kind": f"{peak_kind} sustained bf16 GEMM x 2 (nominal FP8/BF16 "
+                                     f"ratio)",
+                        "algorithmic_flop_per_launch": idx_flop},
+           "flop": {"indexer": idx_flop, "csa_attention": csa_flop, "hca_attention": hca_flop},
+           "calls_ms": calls_ms, "clocks": clocks, "e2e": None}
+    return res
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -572,6 +681,13 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
+    if W.get(args.workload).prefill:
+        res = run_prefill(args, rank, world, dev)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     res, replicas, wl = run_ours(args, rank, world, dev)
     res["e2e"] = run_e2e(args, replicas, wl, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -42,6 +42,8 @@ _I, _I64, _F, _SZ = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_
 
 _lib.csa_compress.argtypes = [_I, _P, _P, _I64, _PC, _PC, _PC, _P, _P, _I, _I, _PC, _PC, _PC, _P]
 _lib.hca_compress.argtypes = [_I, _P, _P, _I64, _PC, _PC, _P, _P, _I, _I, _PC, _PC, _P]
+_lib.indexer_score.argtypes = _lib.indexer_select.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC,
+                                                             _I, _I, _I64, _P, _P, _P, _SZ, _P]
 _lib.indexer_topk.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC, _I, _I, _I64, _P, _P, _P,
                               _SZ, _P]
 _lib.hybrid_attn_decode.argtypes = [_I, _P, _P, _I, _F, _PC, _PC, _I, _P, _I, _I64, _PC, _PC,
@@ -59,8 +61,8 @@ _lib.cskv_noalloc_scratch_bytes.restype = _SZ
 _lib.cskv_error_string.argtypes = [_I]
 _lib.cskv_error_string.restype = ctypes.c_char_p
 _lib.cskv_version.restype = _I
-for _name in ("csa_compress", "hca_compress", "indexer_topk", "hybrid_attn_decode",
-              "hybrid_attn_prefill"):
+for _name in ("csa_compress", "hca_compress", "indexer_topk", "indexer_score", "indexer_select",
+              "hybrid_attn_decode", "hybrid_attn_prefill"):
     getattr(_lib, _name).restype = _I
 
 
@@ -160,6 +162,28 @@ def indexer_topk(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k
                              H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
                              _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
            "indexer_topk")
+
+
+def indexer_score(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
+                  out_idx, out_score, ws, stream=None):
+    """First half of indexer_topk: scores and histogram into the workspace."""
+    c = cache_struct(ik)
+    wp, wn = _ws(ws)
+    _check(_lib.indexer_score(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
+                              H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
+                              _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
+           "indexer_score")
+
+
+def indexer_select(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
+                   out_idx, out_score, ws, stream=None):
+    """Second half of indexer_topk: the top-k from the workspace's scores."""
+    c = cache_struct(ik)
+    wp, wn = _ws(ws)
+    _check(_lib.indexer_select(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
+                               H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
+                               _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
+           "indexer_select")
 
 
 def indexer_topk_noalloc(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k,

@@ -139,6 +139,36 @@ int attention_common(int B, int Tq, const int64_t *pos, int pos_is_ctx_len, cons
   return launch_attention(a, (cudaStream_t)stream);
 }
 
+int indexer_common(int phases, int B, int Tq, const int64_t *q_pos, const void *q_ik,
+                   const float *q_ik_scale, const float *head_w, int H_I, int d_I,
+                   const cskv_cache *ik, int stride, int k, int64_t max_entries,
+                   int32_t *out_idx, float *out_score, void *ws, size_t ws_bytes,
+                   cskv_stream_t stream) {
+  if (B < 0 || Tq < 0 || (int64_t)B * Tq > 0x7fffffffLL) return CSKV_ERR_ARG;
+  if (k < 1 || k > 4096 || stride < 1 || H_I < 1 || d_I < 1 || max_entries < 0)
+    return CSKV_ERR_ARG;
+  if (B == 0 || Tq == 0) return CSKV_OK;
+  if (!q_pos || !q_ik || !head_w || !out_idx) return CSKV_ERR_ARG;
+  CSKV_TRY(check_cache(ik, 0));
+  if (ik->d_rope != 0 || ik->d_nope != d_I || max_entries > ik->cap) return CSKV_ERR_ARG;
+  if (ik->fmt == CSKV_FMT_E4M3_BF16) {
+    if (!q_ik_scale) return CSKV_ERR_ARG;
+  } else if (q_ik_scale) {
+    return CSKV_ERR_ARG;
+  }
+  if ((size_t)H_I * d_I * 4 + (size_t)H_I * 4 + 128ull * (d_I + 1) * 4 > 200 * 1024)
+    return CSKV_ERR_UNSUPPORTED;
+  CSKV_TRY(check_ws(ws, ws_bytes, indexer_ws_bytes(B, Tq, max_entries, k)));
+  IndexerArgs a{};
+  a.B = B; a.Tq = Tq; a.H_I = H_I; a.d_I = d_I; a.stride = stride; a.k = k;
+  a.max_entries = max_entries;
+  a.q_pos = q_pos; a.q_ik = q_ik; a.q_ik_scale = q_ik_scale; a.head_w = head_w;
+  a.ik = to_dev(ik);
+  a.out_idx = out_idx; a.out_score = out_score;
+  a.ws = ws; a.ws_bytes = ws_bytes;
+  return launch_indexer_topk(a, phases, (cudaStream_t)stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -169,29 +199,25 @@ int indexer_topk(int B, int Tq, const int64_t *q_pos, const void *q_ik, const fl
                  const float *head_w, int H_I, int d_I, const cskv_cache *ik, int stride, int k,
                  int64_t max_entries, int32_t *out_idx, float *out_score, void *ws,
                  size_t ws_bytes, cskv_stream_t stream) {
-  if (B < 0 || Tq < 0 || (int64_t)B * Tq > 0x7fffffffLL) return CSKV_ERR_ARG;
-  if (k < 1 || k > 4096 || stride < 1 || H_I < 1 || d_I < 1 || max_entries < 0)
-    return CSKV_ERR_ARG;
-  if (B == 0 || Tq == 0) return CSKV_OK;
-  if (!q_pos || !q_ik || !head_w || !out_idx) return CSKV_ERR_ARG;
-  CSKV_TRY(check_cache(ik, 0));
-  if (ik->d_rope != 0 || ik->d_nope != d_I || max_entries > ik->cap) return CSKV_ERR_ARG;
-  if (ik->fmt == CSKV_FMT_E4M3_BF16) {
-    if (!q_ik_scale) return CSKV_ERR_ARG;
-  } else if (q_ik_scale) {
-    return CSKV_ERR_ARG;
-  }
-  if ((size_t)H_I * d_I * 4 + (size_t)H_I * 4 + 128ull * (d_I + 1) * 4 > 200 * 1024)
-    return CSKV_ERR_UNSUPPORTED;
-  CSKV_TRY(check_ws(ws, ws_bytes, indexer_ws_bytes(B, Tq, max_entries, k)));
-  IndexerArgs a{};
-  a.B = B; a.Tq = Tq; a.H_I = H_I; a.d_I = d_I; a.stride = stride; a.k = k;
-  a.max_entries = max_entries;
-  a.q_pos = q_pos; a.q_ik = q_ik; a.q_ik_scale = q_ik_scale; a.head_w = head_w;
-  a.ik = to_dev(ik);
-  a.out_idx = out_idx; a.out_score = out_score;
-  a.ws = ws; a.ws_bytes = ws_bytes;
-  return launch_indexer_topk(a, (cudaStream_t)stream);
+  return indexer_common(kIndexerScore | kIndexerSelect, B, Tq, q_pos, q_ik, q_ik_scale, head_w,
+                        H_I, d_I, ik, stride, k, max_entries, out_idx, out_score, ws, ws_bytes,
+                        stream);
+}
+
+int indexer_score(int B, int Tq, const int64_t *q_pos, const void *q_ik, const float *q_ik_scale,
+                  const float *head_w, int H_I, int d_I, const cskv_cache *ik, int stride, int k,
+                  int64_t max_entries, int32_t *out_idx, float *out_score, void *ws,
+                  size_t ws_bytes, cskv_stream_t stream) {
+  return indexer_common(kIndexerScore, B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik,
+                        stride, k, max_entries, out_idx, out_score, ws, ws_bytes, stream);
+}
+
+int indexer_select(int B, int Tq, const int64_t *q_pos, const void *q_ik, const float *q_ik_scale,
+                   const float *head_w, int H_I, int d_I, const cskv_cache *ik, int stride, int k,
+                   int64_t max_entries, int32_t *out_idx, float *out_score, void *ws,
+                   size_t ws_bytes, cskv_stream_t stream) {
+  return indexer_common(kIndexerSelect, B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik,
+                        stride, k, max_entries, out_idx, out_score, ws, ws_bytes, stream);
 }
 
 size_t cskv_attn_workspace_size(int B, int Tq, int Hq, int Dv, int64_t max_entries, int window) {

@@ -163,7 +163,10 @@ struct IndexerArgs {
   void *ws; size_t ws_bytes;
 };
 size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k);
-int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st);
+// phases of an indexer call: scoring (with the selection histogram) and the
+// top-k selection from the scores in the workspace
+constexpr int kIndexerScore = 1, kIndexerSelect = 2;
+int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st);
 
 struct AttnArgs {
   int B, Tq, Hq, D, Dv;

@@ -94,24 +94,28 @@ size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k) {
   return total;
 }
 
-int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
+int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st) {
   const int rows = a.B * a.Tq;
   if (rows == 0) return CSKV_OK;
   const IndexerWs w = indexer_ws_layout(a.ws, rows, a.max_entries, a.k, nullptr);
+  const bool score = phases & kIndexerScore, select = phases & kIndexerSelect;
   if (a.max_entries > 0 && indexer_tc_supported(a)) {
     // tensor-core scoring builds the score histogram the multi-CTA selection uses
-    const long long words = (long long)(w.zero_bytes / 4);
-    long long blocks = (words + 255) / 256;
-    if (blocks > 1184) blocks = 1184;
-    if (launch_pdl(zero_words_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
-                   reinterpret_cast<uint32_t *>(w.err), words) != cudaSuccess)
-      return CSKV_ERR_CUDA;
-    int rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
-    if (rc != CSKV_OK) return rc;
+    if (score) {
+      const long long words = (long long)(w.zero_bytes / 4);
+      long long blocks = (words + 255) / 256;
+      if (blocks > 1184) blocks = 1184;
+      if (launch_pdl(zero_words_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                     reinterpret_cast<uint32_t *>(w.err), words) != cudaSuccess)
+        return CSKV_ERR_CUDA;
+      const int rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
+      if (rc != CSKV_OK) return rc;
+    }
+    if (!select) return CSKV_OK;
     return launch_topk_select(w, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
                               a.out_score, st);
   }
-  if (a.max_entries > 0) {
+  if (score && a.max_entries > 0) {
     const size_t smem = sizeof(float) * ((size_t)a.H_I * a.d_I + a.H_I +
                                          (size_t)kKeys * (a.d_I + 1));
     if (!ensure_dynamic_smem(indexer_score_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
@@ -121,8 +125,9 @@ int launch_indexer_topk(const IndexerArgs &a, cudaStream_t st) {
       return CSKV_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return CSKV_ERR_CUDA;
   }
-  launch_topk_rows(w.scores, w.ld, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
-                   a.out_score, st);
+  if (select)
+    launch_topk_rows(w.scores, w.ld, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
+                     a.out_score, st);
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 

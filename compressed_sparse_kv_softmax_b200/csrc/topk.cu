@@ -98,6 +98,41 @@ __device__ void find_threshold_bin(const Bins &bins, int nbins, int target, int 
   __syncthreads();
 }
 
+// Same search with two block barriers: thread t owns `per` consecutive bins
+// from the top (nbins = blockDim.x * per), a warp scan gives the counts
+// inside a warp, shared memory the counts of the warps above.
+template <typename Bins>
+__device__ void find_threshold_bin2(const Bins &bins, int nbins, int target, int *wsum,
+                                    int *out_bin, int *out_above) {
+  const int per = nbins / blockDim.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int top = nbins - 1 - (int)threadIdx.x * per;
+  int lsum = 0;
+  for (int i = 0; i < per; ++i) lsum += (int)bins(top - i);
+  int incl = lsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int before = incl - lsum;
+  for (int w = 0; w < warp; ++w) before += wsum[w];
+  if (before < target && before + lsum >= target) {
+    int cum = before;
+    for (int i = 0; i < per; ++i) {
+      const int c = (int)bins(top - i);
+      if (cum + c >= target) {
+        *out_bin = top - i;
+        *out_above = cum;
+        break;
+      }
+      cum += c;
+    }
+  }
+  __syncthreads();
+}
+
 // Whole-row exact top-k by one CTA (any blockDim multiple of 32).
 __device__ void topk_row_single_cta(const float *__restrict__ s, long long n, int k,
                                     int32_t *__restrict__ oi, float *__restrict__ os) {
@@ -290,8 +325,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
 #pragma unroll
   for (int e = 0; e < kHPer; ++e) sm.hist[tid + e * kSelThreads] = hv[e];
   __syncthreads();
-  find_threshold_bin([&](int i) { return sm.hist[i]; }, kTopkBins, k, sm.scan, &sm.bstar,
-                     &sm.above);
+  find_threshold_bin2([&](int i) { return sm.hist[i]; }, kTopkBins, k, sm.scan, &sm.bstar,
+                      &sm.above);
   const uint32_t bstar = (uint32_t)sm.bstar;
   const int above = sm.above;
 
@@ -341,7 +376,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   if (lane == 0 && wins) atomicAdd(&sm.wins, wins);
 
   // ---- 2. row barrier: every slice's candidates and winner count are visible
-  __threadfence();
+  // (the block barrier orders the CTA's writes before thread 0's fence and
+  // release; the acquiring load and the next block barrier order the reads)
   __syncthreads();
   if (tid == 0) {
     w.wins[(size_t)row * kMaxSplits + me] = (uint32_t)sm.wins;
@@ -397,8 +433,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     for (int i = tid; i < n_cand; i += blockDim.x)
       atomicAdd(&sm.hist[((uint32_t)sm.cand[i] >> 8) & 4095u], 1u);
     __syncthreads();
-    find_threshold_bin([&](int i) { return sm.hist[i]; }, kTopkBins, remaining, sm.scan,
-                       &sm.thr_bin, &sm.take);
+    find_threshold_bin2([&](int i) { return sm.hist[i]; }, kTopkBins, remaining, sm.scan,
+                        &sm.thr_bin, &sm.take);
     prefix |= (uint32_t)sm.thr_bin << 8;
     remaining -= sm.take;
     const int in_bin = (int)sm.hist[sm.thr_bin];

@@ -12,7 +12,8 @@ from __future__ import annotations
 import torch
 
 from . import (attn_workspace_size, csa_compress, hca_compress, hybrid_attn_decode,
-               hybrid_attn_prefill, indexer_topk, indexer_workspace_size, workspace)
+               hybrid_attn_prefill, indexer_score, indexer_select, indexer_topk,
+               indexer_workspace_size, workspace)
 
 
 def _dims(c):
@@ -50,13 +51,14 @@ class CSALayer:
                      L["gate_w"], L["gate_b"], L["pool"], L["stride"], L["comp_k"], L["comp_v"],
                      L["comp_ik"])
 
-    def select(self, q_pos=None):
-        """indexer_topk; q_pos [B][Tq] (device) overrides the layer's positions."""
+    def select(self, q_pos=None, phase="both"):
+        """indexer_topk; q_pos [B][Tq] (device) overrides the layer's positions.
+        phase "score" / "pick" runs only indexer_score / indexer_select."""
         L, wl = self.L, self.wl
         q_pos = L["q_pos"] if q_pos is None else q_pos
-        indexer_topk(self.B, self.Tq, q_pos, L["q_ik"], L["q_ik_scale"], L["head_w"],
-                     wl.H_I, wl.d_I, L["comp_ik"], L["stride"], self.k, self.max_entries,
-                     self.idx, self.score, self.ws_idx)
+        fn = {"both": indexer_topk, "score": indexer_score, "pick": indexer_select}[phase]
+        fn(self.B, self.Tq, q_pos, L["q_ik"], L["q_ik_scale"], L["head_w"], wl.H_I, wl.d_I,
+           L["comp_ik"], L["stride"], self.k, self.max_entries, self.idx, self.score, self.ws_idx)
         return self.idx
 
     def attend(self, sel=None, pos=None):

@@ -151,6 +151,31 @@ int indexer_topk(int B, int Tq, const int64_t *q_pos,
                  int64_t max_entries, int32_t *out_idx, float *out_score,
                  void *ws, size_t ws_bytes, cskv_stream_t stream);
 
+/*
+ * indexer_score / indexer_select - the two halves of indexer_topk, for callers
+ * that time or schedule the scoring (the HBM stream over every indexer key)
+ * apart from the selection (an L2-resident pass over the scores).  Both take
+ * exactly indexer_topk's arguments; indexer_score followed by indexer_select
+ * on the same stream with the same arguments and workspace is indexer_topk.
+ *  - indexer_score writes the scores of every visible entry, and the
+ *    histogram the selection starts from, into the workspace; out_idx and
+ *    out_score are not written.
+ *  - indexer_select reads them and writes out_idx / out_score.  The
+ *    workspace must not be used by another call in between.
+ * (The pages describe the indexer and the top-k as one step; the split is an
+ * interface convenience with no counterpart there.)
+ */
+int indexer_score(int B, int Tq, const int64_t *q_pos,
+                  const void *q_ik, const float *q_ik_scale, const float *head_w,
+                  int H_I, int d_I, const cskv_cache *ik, int stride, int k,
+                  int64_t max_entries, int32_t *out_idx, float *out_score,
+                  void *ws, size_t ws_bytes, cskv_stream_t stream);
+int indexer_select(int B, int Tq, const int64_t *q_pos,
+                   const void *q_ik, const float *q_ik_scale, const float *head_w,
+                   int H_I, int d_I, const cskv_cache *ik, int stride, int k,
+                   int64_t max_entries, int32_t *out_idx, float *out_score,
+                   void *ws, size_t ws_bytes, cskv_stream_t stream);
+
 size_t cskv_indexer_workspace_size(int B, int Tq, int64_t max_entries, int k);
 
 /*

@@ -108,12 +108,14 @@ def test_argument_errors_are_caught_on_the_host(C):
     ik = _fake_cache(0, cap=262144, d_nope=128, d_rope=0)
     ik.data_stride, ik.scale_stride = 128, 8
     args = (1, 1, ctx, q, P(1 << 32), P(1 << 33), 64, 128)
-    assert lib.indexer_topk(*args, R(ik), 4, 0, 262144, out, None, ws, big, None) == ERR_ARG
-    assert lib.indexer_topk(*args, R(ik), 4, 5000, 262144, out, None, ws, big, None) == ERR_ARG
-    assert lib.indexer_topk(1, 1, ctx, q, None, P(1 << 33), 64, 128, R(ik), 4, 1024, 262144,
-                            out, None, ws, big, None) == ERR_ARG
-    assert lib.indexer_topk(*args, R(ik), 4, 1024, 262145, out, None, ws, big, None) == ERR_ARG
-    assert lib.indexer_topk(*args, R(comp), 4, 1024, 8192, out, None, ws, big, None) == ERR_ARG
+    # (indexer_score / indexer_select check exactly what indexer_topk checks)
+    for fn in (lib.indexer_topk, lib.indexer_score, lib.indexer_select):
+        assert fn(*args, R(ik), 4, 0, 262144, out, None, ws, big, None) == ERR_ARG
+        assert fn(*args, R(ik), 4, 5000, 262144, out, None, ws, big, None) == ERR_ARG
+        assert fn(1, 1, ctx, q, None, P(1 << 33), 64, 128, R(ik), 4, 1024, 262144,
+                  out, None, ws, big, None) == ERR_ARG
+        assert fn(*args, R(ik), 4, 1024, 262145, out, None, ws, big, None) == ERR_ARG
+        assert fn(*args, R(comp), 4, 1024, 8192, out, None, ws, big, None) == ERR_ARG
     # compress: ring too small for the entries requested, pool < stride
     gate = P(1 << 35)
     assert lib.csa_compress(1, ctx, ctx, 100, R(ring), None, None, gate, gate, 8, 4, R(comp),
@@ -125,3 +127,11 @@ def test_argument_errors_are_caught_on_the_host(C):
                             None, None, None) == 0
     assert lib.hybrid_attn_prefill(1, 0, ctx, q, 64, 0.04, R(comp), None, 128, None, 0, 8192,
                                    R(ring), None, 128, out, lse, ws, big, None) == 0
+
+
+def test_layer_phases_name_the_split_calls(C):
+    # CSALayer.select(phase=...) dispatches to the two halves of indexer_topk
+    from compressed_sparse_kv_softmax_b200 import layer
+    assert layer.indexer_score is C.indexer_score
+    assert layer.indexer_select is C.indexer_select
+    assert layer.indexer_topk is C.indexer_topk

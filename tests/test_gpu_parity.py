@@ -109,6 +109,21 @@ def test_indexer_topk(C, name):
         assert np.allclose(sc[b, t][: sel.size], rs[sel], rtol=1e-4, atol=1e-4 * np.abs(rs).max())
 
 
+@pytest.mark.parametrize("name", ["tiny", "parity_decode"])
+def test_indexer_score_then_select_is_indexer_topk(C, name):
+    # the two halves called in turn give indexer_topk's results bit for bit
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    Ld = to_device(W.make_csa_layer(W.get(name)))
+    whole = CSALayer(Ld)
+    whole.select()
+    split = CSALayer(Ld)
+    split.select(phase="score")
+    split.select(phase="pick")
+    torch.cuda.synchronize()
+    assert torch.equal(whole.idx, split.idx)
+    assert torch.equal(whole.score, split.score)
+
+
 @pytest.mark.parametrize("T,k", [(3, 8), (4, 8), (64, 16), (64, 100), (517, 129), (1000, 100),
                                  (2100, 500), (40000, 4096)])
 def test_indexer_edge_sizes(C, T, k):
