@@ -25,7 +25,7 @@ namespace cskv {
 bool attn_tc_supported(const AttnArgs &a);
 int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *part_lse,
                    cudaStream_t st);
-int attn_tc_unit_keys();
+int attn_tc_unit_keys(long long rows, long long keys);
 
 namespace {
 
@@ -317,8 +317,9 @@ size_t attn_ws_bytes(int B, int Tq, int Hq, int Dv, long long max_entries, int w
   // either path may run: the larger of the two plans
   const long long rows = (long long)B * Tq;
   const size_t a = partial_bytes(attn_plan(rows, max_entries, window, kChunk), rows, Hq, Dv);
-  const size_t b =
-      partial_bytes(attn_plan(rows, max_entries, window, attn_tc_unit_keys()), rows, Hq, Dv);
+  const size_t b = partial_bytes(
+      attn_plan(rows, max_entries, window, attn_tc_unit_keys(rows, max_entries + window)), rows,
+      Hq, Dv);
   return a > b ? a : b;
 }
 
@@ -327,7 +328,8 @@ int launch_attention(const AttnArgs &a, cudaStream_t st) {
   if (rows == 0) return CSKV_OK;
   const bool tc = attn_tc_supported(a);
   const long long max_comp = a.has_comp ? (a.sel ? a.k : a.max_entries) : 0;
-  const AttnPlan p = attn_plan(rows, max_comp, a.window, tc ? attn_tc_unit_keys() : kChunk);
+  const AttnPlan p =
+      attn_plan(rows, max_comp, a.window, tc ? attn_tc_unit_keys(rows, max_comp + a.window) : kChunk);
   const bool direct = p.splits == 1;
   float *part_o = direct ? a.out : reinterpret_cast<float *>(a.ws);
   float *part_lse = a.lse;

@@ -318,8 +318,9 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     const bool my_valid = sm.slot[krow] >= 0;
 
     // ---- gather: warp w converts key rows 8w .. 8w+7 into the key tile
-    const int r0 = warp * 8;
-    const bool has_rows = r0 < ksteps * 16;   // kKeys = 8 warps x 8 rows
+    const int rpw = unit_keys >> 3;           // key rows per warp: the unit over 8 warps
+    const int r0 = warp * rpw;
+    const bool has_rows = r0 < ksteps * 16;
     const __nv_bfloat16 *qg =
         reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD;
     // consecutive slots: the window's positions (one or two runs around the
@@ -354,7 +355,8 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
       load_q(qg, qraw);
       ok = mbar_wait(&sm.gbar, 0) && ok;     // used once per CTA: phase 0
       if (has_rows) {
-        for (int e = 0; e < 8; ++e) {
+#pragma unroll 1
+        for (int e = 0; e < rpw; ++e) {
           const int r = r0 + e;
           uint4 raw = make_uint4(0, 0, 0, 0), raw2 = make_uint4(0, 0, 0, 0);
           float sc = 0.f;
@@ -384,7 +386,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
       for (int e = 0; e < 8; ++e) {
         raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
         sc[e] = 0.f;
-        const long long slot = has_rows ? sm.slot[r0 + e] : -1;
+        const long long slot = has_rows && e < rpw ? sm.slot[r0 + e] : -1;
         if (slot < 0) continue;
         if (lane < 28) {
           raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
@@ -401,7 +403,8 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
       }
       if (has_rows) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) convert_row(sm.kt, r0 + e, lane, raw[e], raw2[e], sc[e]);
+        for (int e = 0; e < 8; ++e)
+          if (e < rpw) convert_row(sm.kt, r0 + e, lane, raw[e], raw2[e], sc[e]);
       }
     }
     fence_proxy_async_shared();
@@ -597,7 +600,17 @@ bool attn_tc_supported(const AttnArgs &a) {
   return major == 10;
 }
 
-int attn_tc_unit_keys() { return kKeys; }
+// Keys per unit: the smallest of 16, 32, 64 whose units, one CTA each, all fit
+// on the SMs at once (one CTA per SM), else 64.  Short key lists (a decode
+// row's top-k) then spread over more SMs; long ones keep the full tile.
+int attn_tc_unit_keys(long long rows, long long keys) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  for (int u = 16; u < kKeys; u *= 2)
+    if (rows * ((keys + u - 1) / u) <= sms) return u;
+  return kKeys;
+}
 
 int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *part_lse,
                    cudaStream_t st) {
