@@ -216,15 +216,25 @@ attn_merge_kernel(int Hq, int Dv, int n_chunks, const float *__restrict__ part_o
   const float *pl = part_lse + (long long)row * n_chunks * Hq + h;
   const float *po = part_o + (long long)row * n_chunks * Hq * Dv + (long long)h * Dv + d;
   const long long cstride = (long long)Hq * Dv;
-  // the first batch of partials and the LSEs, all in flight at once
+  // the LSEs (needed first) and the first batch of partials, all in flight at once
+  const int nw = n_chunks < kMergeLse ? n_chunks : kMergeLse;
+  float lv[kMergeLse / kMergeThreads];
+#pragma unroll
+  for (int e = 0; e < kMergeLse / kMergeThreads; ++e) {
+    const int i = tid + e * kMergeThreads;
+    lv[e] = i < nw ? __ldcg(pl + (long long)i * Hq) : 0.f;
+  }
   float4 v[kMergeBatch];
 #pragma unroll
   for (int k = 0; k < kMergeBatch; ++k) {
     const int i = g + k * kMergeGroups;
     v[k] = (i < n_chunks && dv) ? load4(po + i * cstride, nd, vec) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const int nw = n_chunks < kMergeLse ? n_chunks : kMergeLse;
-  for (int i = tid; i < nw; i += kMergeThreads) wts[i] = __ldcg(pl + (long long)i * Hq);
+#pragma unroll
+  for (int e = 0; e < kMergeLse / kMergeThreads; ++e) {
+    const int i = tid + e * kMergeThreads;
+    if (i < nw) wts[i] = lv[e];
+  }
   __syncthreads();
   if (tid < 32) {
     float m = -CUDART_INF_F;

@@ -561,6 +561,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     __syncthreads();
     const float inv_ln = 0.6931471805599453f;
     if (tid < kHeads) pl[tid] = ok ? (sm.m[tid] + log2f(sm.l[tid])) * inv_ln : CUDART_NAN_F;
+#pragma unroll 1
     for (int mt = 0; mt < 4; ++mt) {
       const int d = mt * 128 + quad * 32 + lane;
       float o[32];

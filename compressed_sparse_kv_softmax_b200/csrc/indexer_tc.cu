@@ -19,7 +19,7 @@
 //   warp 1      MMA issuer (one thread): 4 tcgen05.mma per tile into one of
 //               kAcc TMEM accumulator slots (2 x 64 fp32 columns each)
 //   warp 2      TMEM allocation
-//   warps 4-15  three epilogue warpgroups taking tiles in turn: tcgen05.ld,
+//   warps 4-19  four epilogue warpgroups taking tiles in turn: tcgen05.ld,
 //               block scales, per-head ReLU, head weights -> score; score
 //               histogram (top 12 bits of the order-preserving key) for the
 //               selection kernel
@@ -42,11 +42,17 @@ constexpr int kHeads = 64;          // MMA N
 constexpr int kDim = 128;           // bytes per key (FP8 dims)
 constexpr int kStages = 8;
 constexpr int kAcc = 4;             // TMEM accumulator slots, 128 columns each
-constexpr int kEpiGroups = 3;       // epilogue warpgroups, taking tiles in turn
+constexpr int kEpiGroups = 4;       // epilogue warpgroups, taking tiles in turn
+constexpr int kHeadChunk = 16;      // heads per TMEM load in the epilogue (16 or 32)
 constexpr int kEpiWarps = 4 * kEpiGroups;
 constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr uint32_t kTileBytes = kTile * kDim;
 constexpr uint32_t kIdesc = idesc(kFmtE4M3, kFmtE4M3, 0, 0, kTile, kHeads);
+// Tile i uses accumulator slot i % kAcc, and the group that takes tile i + kAcc
+// waits on that slot's barrier with the next phase's parity.  That wait is
+// only sound once tile i's phase has completed, which holds when the group's
+// previous tile is tile i itself or a later one: at most kAcc groups.
+static_assert(kEpiGroups <= kAcc, "more epilogue groups than accumulator slots");
 
 struct __align__(1024) Smem {
   uint8_t keys[kStages][kTileBytes];      // 1024-aligned tiles
@@ -280,21 +286,22 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       const bool factored = __all_sync(0xffffffffu, j >= n || (sk0 > 0.f && fabsf(rho) <= 3.0e38f));
       const float2 k0 = make_float2(sk0, sk0), k1 = make_float2(sk1, sk1);
       const float2 rr = make_float2(rho, rho);
+      // kHeadChunk heads per TMEM load (block 0 at column h, block 1 at 64 + h)
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float a0[32], a1[32];
-        tmem_ld32(taddr + half * 32, a0);        // block 0, heads 32*half ..
-        tmem_ld32(taddr + 64 + half * 32, a1);   // block 1
+      for (int c0 = 0; c0 < kHeads; c0 += kHeadChunk) {
+        float a0[kHeadChunk], a1[kHeadChunk];
+        tmem_ld(taddr + c0, a0);
+        tmem_ld(taddr + 64 + c0, a1);
         tmem_wait_ld();
-        if (half == 1) {
-          // both halves are in registers: hand the accumulator slot back
+        if (c0 + kHeadChunk == kHeads) {
+          // the last heads are in registers: hand the accumulator slot back
           tc_fence_before();
           mbar_arrive(&sm.acc_empty[acc]);
         }
         if (factored) {
 #pragma unroll
-          for (int h = 0; h < 32; h += 4) {
-            const int hg = half * 32 + h;
+          for (int h = 0; h < kHeadChunk; h += 4) {
+            const int hg = c0 + h;
             const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
             const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
             const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
@@ -309,8 +316,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
           }
         } else {
 #pragma unroll
-          for (int h = 0; h < 32; h += 4) {
-            const int hg = half * 32 + h;
+          for (int h = 0; h < kHeadChunk; h += 4) {
+            const int hg = c0 + h;
             const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
             const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
             const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
