@@ -66,6 +66,29 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *scratch, int *to
   return res;
 }
 
+// Exclusive prefix sum over the block with one block barrier: a warp scan,
+// then each thread adds the totals of the warps before its own (read from
+// `wsum`).  A following call must be separated from this one by a barrier.
+__device__ __forceinline__ int block_exclusive_scan1(int x, int *wsum, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int before = incl - x, tot = 0;
+  for (int w = 0; w < nw; ++w) {
+    const int t = wsum[w];
+    before += w < warp ? t : 0;
+    tot += t;
+  }
+  *total = tot;
+  return before;
+}
+
 // Bins are counts of keys sharing a digit; this finds the bin holding the
 // `target`-th largest key: scanning bins from the top (bin nbins-1 down), the
 // first bin at which the running count reaches `target`.  Thread t owns
@@ -246,7 +269,7 @@ struct SelSmem {
   int cnt[kMaxSplits];        // selected entries per slice of the row
   int scan[33];
   int bstar, above, thr_bin, take, n_eq, state, n_cand, base, total, wins;
-  uint32_t tie_cut;
+  uint32_t tie_cut, thr_full;
 };
 
 // scores j0 .. j0+7 of a row (entries at or beyond j_hi read as -inf)
@@ -278,7 +301,7 @@ topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *
                       out_score ? out_score + (long long)row * k : nullptr);
 }
 
-__global__ void __launch_bounds__(kSelThreads)
+__global__ void __launch_bounds__(kSelThreads, 1)
 topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int stride,
                    long long max_entries, int k, int32_t *__restrict__ out_idx,
                    float *__restrict__ out_score) {
@@ -415,21 +438,23 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
         const int i = tid + e * kSelThreads;
         v[e] = i < n_cand ? __ldcg(candrow + i) : 0ull;
       }
+      // the next histogram's bins and the per-slice counts start meanwhile
+      for (int i = tid; i < kTopkBins; i += blockDim.x) sm.hist[i] = 0;
+      if (tid < nsplit) sm.cnt[tid] = wins_c;
+      if (tid == 0) { sm.thr_bin = 0; sm.take = 0; sm.n_eq = 0; }
 #pragma unroll
       for (int e = 0; e < kC; ++e) {
         const int i = tid + e * kSelThreads;
         if (i < n_cand) sm.cand[i] = v[e];
       }
     }
+    __syncthreads();
     // radix select of the r-th largest candidate key (all candidates share
     // the bucket bits): bits 19..8 in one 4096-bin pass, then the few
-    // candidates left in the chosen bin by one warp (up to 32 of them) or by
-    // a 256-bin pass over bits 7..0
+    // candidates left in the chosen bin by one warp (up to 32 of them, ties
+    // included) or by a 256-bin pass over bits 7..0
     uint32_t prefix = bstar << kTopkShift;
     int remaining = r;
-    for (int i = tid; i < kTopkBins; i += blockDim.x) sm.hist[i] = 0;
-    if (tid == 0) { sm.thr_bin = 0; sm.take = 0; sm.n_eq = 0; }
-    __syncthreads();
     for (int i = tid; i < n_cand; i += blockDim.x)
       atomicAdd(&sm.hist[((uint32_t)sm.cand[i] >> 8) & 4095u], 1u);
     __syncthreads();
@@ -440,31 +465,48 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     const int in_bin = (int)sm.hist[sm.thr_bin];
     __syncthreads();
     if (in_bin <= 32) {
-      uint32_t *lst = sm.hist;           // keys of the bin's candidates
-      if (tid == 0) sm.take = 0;         // stays 0 (-> fall-back) if no rank matches
+      uint64_t *lst = reinterpret_cast<uint64_t *>(sm.hist);   // the bin's candidates
       for (int i = tid; i < n_cand; i += blockDim.x) {
-        const uint32_t key = (uint32_t)sm.cand[i];
-        if ((key >> 8) == (prefix >> 8)) lst[atomicAdd(&sm.n_eq, 1)] = key;
+        const uint64_t c = sm.cand[i];
+        if (((uint32_t)c >> 8) == (prefix >> 8)) lst[atomicAdd(&sm.n_eq, 1)] = c;
       }
       __syncthreads();
       if (warp == 0) {
         const int cnt = sm.n_eq;
-        const uint32_t mine = lane < cnt ? lst[lane] : 0u;
+        const uint64_t c = lane < cnt ? lst[lane] : 0ull;
+        const uint32_t key = (uint32_t)c, idx = (uint32_t)(c >> 32);
         int gt = 0, ge = 0;
         for (int m = 0; m < cnt; ++m) {
-          const uint32_t o = __shfl_sync(0xffffffffu, mine, m);
-          gt += o > mine;
-          ge += o >= mine;
+          const uint32_t o = __shfl_sync(0xffffffffu, key, m);
+          gt += o > key;
+          ge += o >= key;
         }
-        // the key whose rank range covers `remaining`; equal keys agree
-        if (lane < cnt && gt < remaining && remaining <= ge) {
-          sm.thr_bin = (int)(mine & 255u);
-          sm.take = remaining - gt;
+        // the key whose rank range covers `remaining` (equal keys agree)
+        const unsigned hit = __ballot_sync(0xffffffffu, lane < cnt && gt < remaining && remaining <= ge);
+        const int src = hit ? __ffs(hit) - 1 : 0;
+        const uint32_t tkey = __shfl_sync(0xffffffffu, key, src);
+        const int take = remaining - __shfl_sync(0xffffffffu, gt, src);
+        // exact ties: the take-th smallest index among the keys equal to tkey
+        const bool eq = lane < cnt && key == tkey;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        int rank = 0;
+        for (int m = 0; m < cnt; ++m) {
+          const uint32_t oi = __shfl_sync(0xffffffffu, idx, m);
+          rank += (eqm >> m & 1u) && oi < idx;
+        }
+        const unsigned cut = __ballot_sync(0xffffffffu, eq && rank == take - 1);
+        const uint32_t cut_idx = __shfl_sync(0xffffffffu, idx, cut ? __ffs(cut) - 1 : 0);
+        if (lane == 0) {
+          sm.thr_full = tkey;
+          sm.take = hit ? take : 0;       // 0: no rank matched -> fall-back
+          // all equal keys taken: no cut; otherwise the take-th smallest index
+          sm.tie_cut = (__popc(eqm) > take && cut) ? cut_idx : 0xffffffffu;
         }
       }
       __syncthreads();
-      prefix |= (uint32_t)sm.thr_bin;
-      remaining = sm.take;
+      thr = sm.thr_full;
+      tie_cut = sm.tie_cut;
+      if (sm.take < 1) fallback = true;
     } else {
       for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
       __syncthreads();
@@ -477,39 +519,37 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
                          &sm.take);
       prefix |= (uint32_t)sm.thr_bin;
       remaining -= sm.take;
-    }
-    thr = prefix;
-    const int take_eq = remaining;     // keys equal to thr to take, lowest indices first
-    // exact ties: when more keys equal thr than are taken, the cut is the
-    // take_eq-th smallest of their indices
-    if (tid == 0) sm.n_eq = 0;
-    __syncthreads();
-    uint32_t *eqv = sm.hist;
-    for (int i = tid; i < n_cand; i += blockDim.x) {
-      const uint64_t c = sm.cand[i];
-      if ((uint32_t)c == thr) {
-        const int p = atomicAdd(&sm.n_eq, 1);
-        if (p < kTieCap) eqv[p] = (uint32_t)(c >> 32);
-      }
-    }
-    __syncthreads();
-    const int n_eq = sm.n_eq;
-    if (take_eq < 1 || n_eq < take_eq || n_eq > kTieCap) {
-      fallback = true;
-    } else if (n_eq > take_eq) {
-      int m = 1;
-      while (m < n_eq) m <<= 1;
-      for (int i = n_eq + tid; i < m; i += blockDim.x) eqv[i] = 0xffffffffu;
+      thr = prefix;
+      const int take_eq = remaining;     // keys equal to thr to take, lowest indices first
+      // exact ties: when more keys equal thr than are taken, the cut is the
+      // take_eq-th smallest of their indices
+      if (tid == 0) sm.n_eq = 0;
       __syncthreads();
-      bitonic_sort_smem(eqv, m);
-      tie_cut = eqv[take_eq - 1];
+      uint32_t *eqv = sm.hist;
+      for (int i = tid; i < n_cand; i += blockDim.x) {
+        const uint64_t c = sm.cand[i];
+        if ((uint32_t)c == thr) {
+          const int p = atomicAdd(&sm.n_eq, 1);
+          if (p < kTieCap) eqv[p] = (uint32_t)(c >> 32);
+        }
+      }
+      __syncthreads();
+      const int n_eq = sm.n_eq;
+      if (take_eq < 1 || n_eq < take_eq || n_eq > kTieCap) {
+        fallback = true;
+      } else if (n_eq > take_eq) {
+        int m = 1;
+        while (m < n_eq) m <<= 1;
+        for (int i = n_eq + tid; i < m; i += blockDim.x) eqv[i] = 0xffffffffu;
+        __syncthreads();
+        bitonic_sort_smem(eqv, m);
+        tie_cut = eqv[take_eq - 1];
+      }
     }
   }
 
   // ---- per-slice counts of the selection, and this slice's output offset
   if (!fallback) {
-    if (tid < nsplit) sm.cnt[tid] = wins_c;
-    __syncthreads();
     for (int i = tid; i < n_cand; i += blockDim.x) {
       const uint64_t c = sm.cand[i];
       const uint32_t key = (uint32_t)c, j = (uint32_t)(c >> 32);
@@ -551,7 +591,8 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
         fl |= (uint32_t)take << e;
       }
       int tot;
-      int p = base + block_exclusive_scan(__popc(fl), sm.scan, &tot);
+      if (c0 != j_lo) __syncthreads();      // the previous pass has read sm.scan
+      int p = base + block_exclusive_scan1(__popc(fl), sm.scan, &tot);
 #pragma unroll
       for (int e = 0; e < kSelPer; ++e) {
         if ((fl >> e & 1u) && p < k) {

@@ -153,16 +153,18 @@ def _tied_keys(wl, needles, every):
     return L
 
 
-@pytest.mark.parametrize("T,k,every", [(18000, 300, 3), (40000, 300, 1)])
-def test_indexer_exact_ties_take_lower_indices(C, T, k, every):
+@pytest.mark.parametrize("T,k,every,n_needles", [(18000, 300, 3, 37), (40000, 300, 1, 37),
+                                                 (18000, 5, 3, 10)])
+def test_indexer_exact_ties_take_lower_indices(C, T, k, every, n_needles):
     # exact score ties at the k-th score: the lowest indices are taken, and the
     # output is ascending.  T=18000 keeps the tied candidates in the multi-CTA
-    # path; every=1 (all entries tied) overflows the candidate list and takes
-    # the single-CTA path.
+    # path (1,500 tied keys: the 256-bin pass and the sorted tie list; 10
+    # tied needles with k=5: the warp that ranks a small bin); every=1 (all
+    # entries tied) overflows the candidate list and takes the single-CTA path.
     wl = W.get("parity_decode").with_(T=T, B=1, k=k)
     rng = np.random.default_rng(5)
     n = T // 4
-    needles = np.sort(rng.choice(np.arange(1, n), 37, replace=False))
+    needles = np.sort(rng.choice(np.arange(1, n), n_needles, replace=False))
     L = _tied_keys(wl, needles, every)
     sc = O.layer_indexer_topk(L, k)[(0, 0)][1]
     ties = np.array([j for j in range(0, n, every) if j not in set(needles.tolist())])
@@ -174,7 +176,10 @@ def test_indexer_exact_ties_take_lower_indices(C, T, k, every):
     assert np.allclose(sc[ties], sc[ties[0]], rtol=1e-12, atol=0)
     assert np.allclose(sc[needles], 2 * sc[ties[0]], rtol=1e-12, atol=0)
     assert rest.size == 0 or sc[rest].max() < 0.6 * sc[ties[0]]
-    expect = np.sort(np.concatenate([needles, ties[: k - len(needles)]]))
+    if k <= len(needles):
+        expect = needles[:k]
+    else:
+        expect = np.sort(np.concatenate([needles, ties[: k - len(needles)]]))
     layer = _run_indexer(C, to_device(L))
     got = layer.idx.cpu().numpy()[0, 0]
     assert np.array_equal(got, expect)
