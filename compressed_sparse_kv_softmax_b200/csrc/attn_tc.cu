@@ -22,20 +22,24 @@
 //   O = V_hi P_hi + V_lo P_hi + V_hi P_lo   (V = K; the lo x lo term is 2^-22)
 // with fp32 accumulation in TMEM.
 //
-//   1. gather: each warp loads 8 keys (all loads first; the first unit stages
-//      Q meanwhile), then converts them: lanes 0-27 take 16 FP8 codes each
-//      (x block scale), lanes 28-31 16 BF16 RoPE values each.  Per 64-dim
-//      chunk the key tile holds 64 rows of hi parts then 64 rows of lo parts
-//      (K-major, 128-byte swizzle).  Q becomes FP16 in the same layout
-//      [8 chunks][64 heads][128 B].
+//   1. gather: a unit holds 16, 32 or 64 keys; each warp takes 1/8 of them.
+//      The first unit of a CTA whose keys are consecutive slots (dense
+//      entries, the window) arrives by bulk copies into the still unused Q
+//      buffer while Q is loaded into registers; otherwise each lane loads its
+//      part of the rows (all loads first, Q staged meanwhile).  Conversion:
+//      lanes 0-27 take 16 FP8 codes each (x block scale), lanes 28-31 16
+//      BF16 RoPE values each.  Per 64-dim chunk the key tile holds 64 rows of
+//      hi parts then 64 rows of lo parts (K-major, 128-byte swizzle).  Q
+//      becomes FP16 in the same layout [8 chunks][64 heads][128 B].
 //   2. [K_hi; K_lo] Q^T with the 128 stacked rows on the MMA M axis (N = 64
-//      heads, K = 512 in 32 steps), fp32 in TMEM cols 0..63; lanes 64..127
-//      (lo parts) are added to lanes 0..63 through shared memory.
-//   3. softmax over keys per head: each thread owns one key row; a warp
-//      reduce-scatter butterfly (32+16+8+4+2 shuffles) leaves lane L with
-//      heads 2L, 2L+1 over the warp's keys, shared memory joins the warps.
-//      P = exp2(S * scale * log2 e - m) goes as hi/lo MN-major tiles
-//      [keys][64 heads]; the per-head sums use the same butterfly.
+//      heads, K = 512 in 32 steps), fp32 in TMEM cols 0..63.
+//   3. softmax over keys per head: the four threads of key row r (TMEM lanes
+//      r and 64 + r, each with one half of the heads) trade S parts through
+//      shared memory so that each holds hi + lo for 16 heads; a warp
+//      reduce-scatter butterfly (8+4+2+1 shuffles and the lane pair) gives
+//      each head's max and sum over the warp's 32 keys, shared memory joins
+//      the two warps of a head.  P = exp2(S * scale * log2 e - m) goes as
+//      hi/lo MN-major tiles [keys][64 heads].
 //   4. O^T = V^T P^T reading the key tiles MN-major (M = 128 dims x 4,
 //      N = 64 heads, K = keys), fp32 in TMEM columns 64..319.
 //   5. each thread owns one dim: o[h][d] / l_h and lse_h = ln2 (m_h + log2 l_h)
@@ -114,6 +118,28 @@ __device__ __forceinline__ float butterfly32(float (&v)[32]) {
     }
   }
   return v[0];
+}
+
+// Warp reduction of 16 per-lane values: afterwards lanes 2i and 2i+1 hold the
+// combination over all 32 lanes of value i (8+4+2+1 exchanges, then the pair).
+template <bool kMax>
+__device__ __forceinline__ float butterfly16(float (&v)[16]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int step = 0; step < 4; ++step) {
+    const int half = 8 >> step;              // values kept after this step
+    const int bit = 16 >> step;              // partner lane distance
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = upper ? v[i + half] : v[i];
+      const float send = upper ? v[i] : v[i + half];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, bit);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, v[0], 1);
+  return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
 // two E4M3 codes (low byte first) -> float2
@@ -315,7 +341,6 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     }
     // (the barrier also publishes the slots) any key at all in this unit?
     if (!__syncthreads_or(tid < kM && sm.slot[tid] >= 0)) continue;
-    const bool my_valid = sm.slot[krow] >= 0;
 
     // ---- gather: warp w converts key rows 8w .. 8w+7 into the key tile
     const int rpw = unit_keys >> 3;           // key rows per warp: the unit over 8 warps
@@ -429,40 +454,45 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     phase ^= 1;
     tc_fence_after();
 
-    // ---- softmax over this unit's keys with the running per-head max
-    float sv[32];
-    tmem_ld32(tmem + tmem_tl + colh * 32, sv);
-    tmem_wait_ld();
+    // ---- softmax over this unit's keys with the running per-head max.  The
+    // four threads of a key row r (TMEM lanes r and 64 + r, two head halves)
+    // split its 64 heads 16 each: lane r keeps heads h0 .. h0+15 and lane
+    // 64 + r heads h0+16 .. h0+31 of its half, after trading the other
+    // sixteen S parts (hi or lo) through the P buffers (free until P is
+    // written), head-major so that a warp's lanes touch consecutive words.
+    const bool lo_row = krow >= kKeys;
+    const int r = krow & (kKeys - 1);                  // this thread's key row
+    const int h0 = colh * 32 + (lo_row ? 16 : 0);      // first of its 16 heads
+    const bool r_valid = sm.slot[r] >= 0;
+    float sv[16];
     {
-      // S = hi rows + lo rows: TMEM lanes 64..127 hand their values to lanes
-      // 0..63 through the P buffers (free until P is written), head-major so
-      // that the lanes of a warp touch consecutive words
+      float t[32];
+      tmem_ld32(tmem + tmem_tl + colh * 32, t);
+      tmem_wait_ld();
       float *scr = reinterpret_cast<float *>(sm.phi);   // [64 heads][64 keys]
-      if (krow >= kKeys) {
+      const int give = lo_row ? colh * 32 : colh * 32 + 16;   // heads the partner keeps
 #pragma unroll
-        for (int i = 0; i < 32; ++i) scr[(colh * 32 + i) * kKeys + (krow - kKeys)] = sv[i];
-      }
+      for (int i = 0; i < 16; ++i) scr[(give + i) * kKeys + r] = lo_row ? t[i] : t[16 + i];
       __syncthreads();
-      if (krow < kKeys) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[i] += scr[(colh * 32 + i) * kKeys + krow];
-      }
+      for (int i = 0; i < 16; ++i)
+        sv[i] = (lo_row ? t[16 + i] : t[i]) + scr[(h0 + i) * kKeys + r];
       __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) sv[i] = my_valid ? sv[i] * c2 : -CUDART_INF_F;
+    for (int i = 0; i < 16; ++i) sv[i] = r_valid ? sv[i] * c2 : -CUDART_INF_F;
     {
-      float v[32];
+      float v[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = sv[i];
-      sm.red[quad][colh * 32 + lane] = butterfly32<true>(v);
+      for (int i = 0; i < 16; ++i) v[i] = sv[i];
+      const float mx = butterfly16<true>(v);
+      if (!(lane & 1)) sm.red[quad & 1][h0 + (lane >> 1)] = mx;
     }
     __syncthreads();
     if (tid < kHeads) {
       // lazy rescaling: keep the running max unless the unit's max exceeds it
       // by more than 8 (P stays <= 2^8, fine in FP16 hi/lo parts)
-      const float tmax = fmaxf(fmaxf(sm.red[0][tid], sm.red[1][tid]),
-                               fmaxf(sm.red[2][tid], sm.red[3][tid]));
+      const float tmax = fmaxf(sm.red[0][tid], sm.red[1][tid]);
       const float mold = sm.m[tid];
       const float mnew = (mold == -CUDART_INF_F || tmax > mold + 8.f) ? tmax : mold;
       sm.alpha[tid] = mold == -CUDART_INF_F ? 0.f : exp2f(mold - mnew);
@@ -470,27 +500,26 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     }
     __syncthreads();
     {
-      float v[32];
+      float v[16];
 #pragma unroll
-      for (int h = 0; h < 32; h += 8) {
+      for (int h = 0; h < 16; h += 8) {
         uint4 wh, wl;
         uint32_t *whp = reinterpret_cast<uint32_t *>(&wh), *wlp = reinterpret_cast<uint32_t *>(&wl);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int hh = h + 2 * e, hg = colh * 32 + hh;
-          const float p0 = my_valid ? exp2f(sv[hh] - sm.m[hg]) : 0.f;
-          const float p1 = my_valid ? exp2f(sv[hh + 1] - sm.m[hg + 1]) : 0.f;
+          const int hh = h + 2 * e, hg = h0 + hh;
+          const float p0 = r_valid ? exp2f(sv[hh] - sm.m[hg]) : 0.f;
+          const float p1 = r_valid ? exp2f(sv[hh + 1] - sm.m[hg + 1]) : 0.f;
           split_h2(p0, p1, whp[e], wlp[e]);
           v[hh] = p0;
           v[hh + 1] = p1;
         }
-        if (krow < kKeys) {
-          const uint32_t u = (colh * 32 + h) >> 3;
-          *reinterpret_cast<uint4 *>(sm.phi + swz(krow, u)) = wh;
-          *reinterpret_cast<uint4 *>(sm.plo + swz(krow, u)) = wl;
-        }
+        const uint32_t u = (h0 + h) >> 3;
+        *reinterpret_cast<uint4 *>(sm.phi + swz(r, u)) = wh;
+        *reinterpret_cast<uint4 *>(sm.plo + swz(r, u)) = wl;
       }
-      sm.red[quad][colh * 32 + lane] = butterfly32<false>(v);
+      const float sum = butterfly16<false>(v);
+      if (!(lane & 1)) sm.red[quad & 1][h0 + (lane >> 1)] = sum;
     }
     // ---- rescale the running O^T where a head's max moved (rare)
     if (started) {
@@ -519,9 +548,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid < kHeads)
-      sm.l[tid] = sm.l[tid] * sm.alpha[tid] +
-                  ((sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]));
+    if (tid < kHeads) sm.l[tid] = sm.l[tid] * sm.alpha[tid] + (sm.red[0][tid] + sm.red[1][tid]);
 
     // ---- O^T (+)= V^T P^T
     if (tid == 0) {

@@ -217,18 +217,39 @@ __device__ __forceinline__ float staged_value(const Cache &c, const SlotLayout &
 
 __device__ void pool_staged(const Cache &c, const SlotLayout &l, const uint8_t *buf,
                             long long first, int pool, const float *a, float *pooled) {
-  const int D = c.dims();
+  // the format and the slots present (positions >= 0) are fixed per entry: the
+  // per-dim loops below carry no per-value branches
+  const int D = c.dims(), dn = c.d_nope, bytes = l.bytes;
+  const int r0 = first < 0 ? (int)-first : 0;
+  if (c.fmt == CSKV_FMT_F32) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      float acc = 0.f;
+      for (int r = r0; r < pool; ++r)
+        acc = fmaf(a[r], reinterpret_cast<const float *>(buf + (size_t)r * bytes)[d], acc);
+      pooled[d] = acc;
+    }
+    return;
+  }
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float acc = 0.f;
-    for (int r = 0; r < pool; ++r) {
-      if (first + r < 0) continue;
-      acc = fmaf(a[r], staged_value(c, l, buf + (size_t)r * l.bytes, d), acc);
+    if (d < dn) {
+      const int so = l.scale_off + 4 * (d >> 6);
+      for (int r = r0; r < pool; ++r) {
+        const uint8_t *slot = buf + (size_t)r * bytes;
+        acc = fmaf(a[r] * *reinterpret_cast<const float *>(slot + so), e4m3_decode(slot[d]), acc);
+      }
+    } else {
+      const int ro = l.rope_off + 2 * (d - dn);
+      for (int r = r0; r < pool; ++r)
+        acc = fmaf(a[r],
+                   __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(buf + (size_t)r * bytes + ro)),
+                   acc);
     }
     pooled[d] = acc;
   }
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
 compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__ t_end,
                        Cache raw_k, Cache raw_v, Cache raw_ik, const float *__restrict__ gate_w,
                        const float *__restrict__ gate_b, int pool, int stride, Cache out_k,
