@@ -258,14 +258,20 @@ class StepGraph:
         return [_ok(rt.cudaEventElapsedTime(a, b), "elapsed") for a, b in self.events]
 
 
+def _ik_scales(wl):
+    """fp32 scales per indexer key or query head: one per vector in the
+    per-vector layout, else one per 64 dims."""
+    return 1 if wl.ik_fmt == "e4m3vec" else wl.d_I // 64
+
+
 def indexer_bytes(wl):
     """Algorithmic HBM bytes of one indexer scoring launch: every visible CSA
-    entry's FP8 indexer key (d_I bytes) and its d_I/64 fp32 scales, the FP8
-    query heads with their scales and the head weights.  (The scores, 4 bytes
-    per entry, stay in L2 for the selection.)"""
+    entry's FP8 indexer key (d_I bytes) and its fp32 scale(s), the FP8 query
+    heads with their scales and the head weights.  (The scores, 4 bytes per
+    entry, stay in L2 for the selection.)"""
     n_c = wl.T // wl.csa_stride
-    per_entry = wl.d_I + 4 * (wl.d_I // 64)
-    q = wl.H_I * wl.d_I + 4 * wl.H_I * (wl.d_I // 64) + 4 * wl.H_I
+    per_entry = wl.d_I + 4 * _ik_scales(wl)
+    q = wl.H_I * wl.d_I + 4 * wl.H_I * _ik_scales(wl) + 4 * wl.H_I
     return wl.B * (n_c * per_entry + q)
 
 
@@ -273,7 +279,7 @@ def step_bytes(wl):
     """Algorithmic HBM bytes of one decode step (both layers), compression
     averaged over the 128-step window (32 CSA entries and 1 HCA entry)."""
     entry = wl.d_nope + 2 * wl.d_rope + 4 * (wl.d_nope // 64)
-    ik = wl.d_I + 4 * (wl.d_I // 64)
+    ik = wl.d_I + 4 * _ik_scales(wl)
     n_h = wl.T // wl.hca_stride
     q = wl.Hq * wl.D * 2
     out = wl.Hq * wl.D * 4 + wl.Hq * 4
@@ -365,6 +371,8 @@ def run_ours(args, rank, world, dev):
                                   f"around {wl.T}: 32 CSA + 1 HCA compressions), Hq={wl.Hq}, "
                                   f"D={wl.d_nope}+{wl.d_rope}, H_I={wl.H_I}x{wl.d_I}, k={wl.k}, "
                                   f"window={wl.window}",
+                      "indexer_scales": "one fp32 per key / query head"
+                                        if wl.ik_fmt == "e4m3vec" else "one fp32 per 64 dims",
                       "global_batch": wl.B * world, "seq_len": wl.T,
                       "parallelism": f"replicas x{world} (weak)",
                       "l2": f"{R} rotating input replicas, {R * per_rep_bytes / 1e6:.0f} MB "

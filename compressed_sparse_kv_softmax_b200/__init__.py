@@ -25,7 +25,8 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_SCRATCH_LIMIT = 0, -1, -2, -3, -4, -5
-FMT_F32, FMT_E4M3_BF16 = 0, 1
+FMT_F32, FMT_E4M3_BF16, FMT_E4M3_VEC = 0, 1, 2
+_FMT = {"f32": FMT_F32, "e4m3": FMT_E4M3_BF16, "e4m3vec": FMT_E4M3_VEC}
 
 
 class CskvCache(ctypes.Structure):
@@ -88,12 +89,13 @@ def _slot_bytes(t):
 
 def cache_struct(c):
     """C descriptor for a cache given as a dict of planes
-    {"fmt": "f32"|"e4m3", "d_nope", "d_rope", "ring", "cap", "data", "scale", "rope"}
+    {"fmt": "f32"|"e4m3"|"e4m3vec", "d_nope", "d_rope", "ring", "cap", "data", "scale",
+    "rope"}
     (or None)."""
     if c is None:
         return None
     s = CskvCache()
-    s.fmt = FMT_F32 if c["fmt"] == "f32" else FMT_E4M3_BF16
+    s.fmt = _FMT[c["fmt"]]
     s.d_nope, s.d_rope = int(c["d_nope"]), int(c["d_rope"])
     s.ring, s.cap = int(bool(c["ring"])), int(c["cap"])
     s.data, s.data_stride = c["data"].data_ptr(), _slot_bytes(c["data"])

@@ -21,11 +21,12 @@ int check_cache(const cskv_cache *c, int ring) {
     if (c->data_stride < 4LL * (c->d_nope + c->d_rope)) return CSKV_ERR_ARG;
     return CSKV_OK;
   }
-  if (c->fmt != CSKV_FMT_E4M3_BF16) return CSKV_ERR_UNSUPPORTED;
+  if (c->fmt != CSKV_FMT_E4M3_BF16 && c->fmt != CSKV_FMT_E4M3_VEC) return CSKV_ERR_UNSUPPORTED;
   if (c->d_nope < 64 || c->d_nope % 64) return CSKV_ERR_UNSUPPORTED;
+  if (c->fmt == CSKV_FMT_E4M3_VEC && c->d_rope) return CSKV_ERR_UNSUPPORTED;
   if (c->data_stride < c->d_nope) return CSKV_ERR_ARG;
-  if (!c->scale || !aligned16(c->scale) || c->scale_stride % 4 ||
-      c->scale_stride < 4LL * (c->d_nope / 64))
+  const long long n_scales = c->fmt == CSKV_FMT_E4M3_VEC ? 1 : c->d_nope / 64;
+  if (!c->scale || !aligned16(c->scale) || c->scale_stride % 4 || c->scale_stride < 4LL * n_scales)
     return CSKV_ERR_ARG;
   if (c->d_rope) {
     if (c->d_rope % 8) return CSKV_ERR_UNSUPPORTED;
@@ -72,7 +73,12 @@ int compress_common(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
     if (!rings[i]) continue;
     CSKV_TRY(check_cache(rings[i], 1));
     CSKV_TRY(check_cache(outs[i], 0));
-    if (!same_layout(rings[i], outs[i]) || rings[i]->fmt != raw_k->fmt) return CSKV_ERR_ARG;
+    if (!same_layout(rings[i], outs[i])) return CSKV_ERR_ARG;
+    // V shares K's format; the indexer keys may take either E4M3 layout
+    // beside an E4M3 KV cache, fp32 beside an fp32 one
+    if (i == 1 ? rings[i]->fmt != raw_k->fmt
+               : (rings[i]->fmt == CSKV_FMT_F32) != (raw_k->fmt == CSKV_FMT_F32))
+      return CSKV_ERR_ARG;
   }
   for (int i = 0; i < 3; ++i) {
     if (!rings[i]) continue;
@@ -151,7 +157,7 @@ int indexer_common(int phases, int B, int Tq, const int64_t *q_pos, const void *
   if (!q_pos || !q_ik || !head_w || !out_idx) return CSKV_ERR_ARG;
   CSKV_TRY(check_cache(ik, 0));
   if (ik->d_rope != 0 || ik->d_nope != d_I || max_entries > ik->cap) return CSKV_ERR_ARG;
-  if (ik->fmt == CSKV_FMT_E4M3_BF16) {
+  if (ik->fmt == CSKV_FMT_E4M3_BF16 || ik->fmt == CSKV_FMT_E4M3_VEC) {
     if (!q_ik_scale) return CSKV_ERR_ARG;
   } else if (q_ik_scale) {
     return CSKV_ERR_ARG;

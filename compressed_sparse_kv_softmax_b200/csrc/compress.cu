@@ -38,6 +38,18 @@ __device__ void store_entry(const Cache &out, int b, long long j, const float *p
   }
   uint8_t *codes = out.data + out.row(b, j) * out.data_stride;
   float *scales = reinterpret_cast<float *>(out.scale + out.row(b, j) * out.scale_stride);
+  if (out.fmt == CSKV_FMT_E4M3_VEC) {
+    // one scale for the whole vector: warp 0 finds its amax and encodes
+    if (warp == 0) {
+      float amax = 0.f;
+      for (int d = lane; d < out.d_nope; d += 32) amax = fmaxf(amax, fabsf(pooled[d]));
+      amax = warp_max(amax);
+      const float s = amax > 0.f ? amax / 448.f : 1.f;
+      for (int d = lane; d < out.d_nope; d += 32) codes[d] = e4m3_encode(pooled[d] / s);
+      if (lane == 0) scales[0] = s;
+    }
+    return;
+  }
   const int nb = out.d_nope >> 6;
   for (int blk = warp; blk < nb; blk += kWarps) {
     const float v0 = pooled[blk * 64 + lane];
@@ -153,7 +165,7 @@ __host__ __device__ inline SlotLayout slot_layout(const Cache &c) {
   }
   l.data_bytes = c.d_nope;
   l.scale_off = round16(c.d_nope);
-  l.rope_off = l.scale_off + round16(4 * (c.d_nope >> 6));
+  l.rope_off = l.scale_off + round16(4 * c.n_scales());
   l.bytes = l.rope_off + round16(2 * c.d_rope);
   return l;
 }
@@ -199,7 +211,7 @@ __device__ void stage_window(const Cache &c, const SlotLayout &l, const long lon
     uint8_t *dst = buf + (size_t)r * l.bytes;
     stage_bytes(dst, c.data + row * c.data_stride, l.data_bytes, lane, 32);
     if (c.fmt != CSKV_FMT_F32) {
-      stage_bytes(dst + l.scale_off, c.scale + row * c.scale_stride, 4 * (c.d_nope >> 6), lane,
+      stage_bytes(dst + l.scale_off, c.scale + row * c.scale_stride, 4 * c.n_scales(), lane,
                   32);
       if (c.d_rope)
         stage_bytes(dst + l.rope_off, c.rope + row * c.rope_stride, 2 * c.d_rope, lane, 32);
@@ -211,7 +223,8 @@ __device__ __forceinline__ float staged_value(const Cache &c, const SlotLayout &
                                               const uint8_t *slot, int d) {
   if (c.fmt == CSKV_FMT_F32) return reinterpret_cast<const float *>(slot)[d];
   if (d < c.d_nope)
-    return e4m3_decode(slot[d]) * reinterpret_cast<const float *>(slot + l.scale_off)[d >> 6];
+    return e4m3_decode(slot[d]) *
+           reinterpret_cast<const float *>(slot + l.scale_off)[c.fmt == CSKV_FMT_E4M3_VEC ? 0 : d >> 6];
   return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(slot + l.rope_off)[d - c.d_nope]);
 }
 
@@ -233,7 +246,7 @@ __device__ void pool_staged(const Cache &c, const SlotLayout &l, const uint8_t *
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float acc = 0.f;
     if (d < dn) {
-      const int so = l.scale_off + 4 * (d >> 6);
+      const int so = l.scale_off + (c.fmt == CSKV_FMT_E4M3_VEC ? 0 : 4 * (d >> 6));
       for (int r = r0; r < pool; ++r) {
         const uint8_t *slot = buf + (size_t)r * bytes;
         acc = fmaf(a[r] * *reinterpret_cast<const float *>(slot + so), e4m3_decode(slot[d]), acc);

@@ -22,6 +22,9 @@ struct Cache {
   uint8_t *rope; long long rope_stride;
 
   __host__ __device__ int dims() const { return d_nope + d_rope; }
+  // fp32 scales per slot and the dims each covers
+  __host__ __device__ int n_scales() const { return fmt == CSKV_FMT_E4M3_VEC ? 1 : d_nope >> 6; }
+  __host__ __device__ int scale_block() const { return fmt == CSKV_FMT_E4M3_VEC ? d_nope : 64; }
   __host__ __device__ long long row(int b, long long slot) const {
     return (long long)b * cap + slot;
   }
@@ -43,7 +46,7 @@ struct Cache {
     if (d < d_nope) {
       __nv_fp8_e4m3 c;
       c.__x = data_ptr(b, slot)[d];
-      return float(c) * scale_ptr(b, slot)[d >> 6];
+      return float(c) * scale_ptr(b, slot)[fmt == CSKV_FMT_E4M3_VEC ? 0 : d >> 6];
     }
     return __bfloat162float(rope_ptr(b, slot)[d - d_nope]);
   }

@@ -52,7 +52,10 @@ indexer_score_kernel(IndexerArgs a, float *__restrict__ scores, long long ld) {
       q[i] = reinterpret_cast<const float *>(a.q_ik)[qoff + i];
     } else {
       const int h = i / dI, d = i % dI;
-      const float sc = a.q_ik_scale[((long long)row * H + h) * (dI >> 6) + (d >> 6)];
+      // query scales follow the keys' layout: per 64 dims, or one per head
+      const float sc = a.ik.fmt == CSKV_FMT_E4M3_VEC
+                           ? a.q_ik_scale[(long long)row * H + h]
+                           : a.q_ik_scale[((long long)row * H + h) * (dI >> 6) + (d >> 6)];
       q[i] = e4m3_decode(reinterpret_cast<const uint8_t *>(a.q_ik)[qoff + i]) * sc;
     }
   }

@@ -1,29 +1,30 @@
 // Lightning-indexer scoring on the 5th-generation tensor cores (tcgen05) for
-// the FP8 layout with 64 indexer heads of dim 128.
+// FP8 indexer keys and queries with 64 heads of dim 128.
 //
 // The indexer scores every compressed CSA entry per query at low precision
 // («DeepSeek V4-Pro: Architektur, KV-Cache-Kompression und Hyper-Connections
 // im Detail», "Kompression und Selektion"; «DeepSeek-V4: 1 Million Token
 // Context endlich nutzbar», "Hybrid Attention: CSA und HCA"):
-//   s_j = sum_h w_h * max(0, q_h . k_j),   q_h . k_j = sum_b sq_{h,b} sk_{j,b} (Q_h,b . K_j,b)
-// where b indexes the two 64-element scale blocks of the 128-dim FP8 vectors.
+//   s_j = sum_h w_h * max(0, q_h . k_j)
+// with q and k dequantised FP8 vectors.  Two scale layouts:
+//   per vector (E4M3_VEC):  q_h . k_j = sq_h sk_j (Q_h . K_j)
+//   per 64 dims (E4M3_BF16): q_h . k_j = sum_b sq_{h,b} sk_{j,b} (Q_h,b . K_j,b)
 //
 // Per query row the entries are a [n x 128] FP8 matrix: each 128-entry tile
-// is one MMA of M = 128 entries x N = 64 heads, with the two scale blocks
-// accumulated separately (K = 64 each) so the per-entry and per-head block
-// scales can be applied in fp32 afterwards.
+// is one MMA chain of M = 128 entries x N = 64 heads (4 steps of K = 32),
+// into one accumulator (per-vector scales) or one per 64-dim block, so that
+// the scales can be applied in fp32 afterwards.
 //
 // CTA roles (persistent over the row's tiles assigned to the CTA):
 //   warp 0      TMA producer: key tiles (128 rows x 128 B, 128-byte swizzle)
-//               into a kStages-deep shared-memory ring
+//               and their scales (bulk copy) into a kStages-deep ring
 //   warp 1      MMA issuer (one thread): 4 tcgen05.mma per tile into one of
-//               kAcc TMEM accumulator slots (2 x 64 fp32 columns each)
+//               the TMEM accumulator slots (64 or 128 fp32 columns each)
 //   warp 2      TMEM allocation
 //   warps 4-19  four epilogue warpgroups taking tiles in turn: tcgen05.ld,
-//               block scales, per-head ReLU, head weights -> score; score
-//               histogram (top 12 bits of the order-preserving key) for the
-//               selection kernel
-// HBM traffic is the key tile stream (128 B + the 8 B of scales per entry);
+//               scales, per-head ReLU, head weights -> score; score histogram
+//               (top 12 bits of the order-preserving key) for the selection
+// HBM traffic is the key tile stream (128 B + 4 or 8 B of scales per entry);
 // scores (4 B per entry) go to the workspace and stay in L2.
 #include <cudaTypedefs.h>
 
@@ -41,28 +42,42 @@ constexpr int kTile = 128;          // entries per tile (MMA M)
 constexpr int kHeads = 64;          // MMA N
 constexpr int kDim = 128;           // bytes per key (FP8 dims)
 constexpr int kStages = 8;
-constexpr int kAcc = 4;             // TMEM accumulator slots, 128 columns each
 constexpr int kEpiGroups = 4;       // epilogue warpgroups, taking tiles in turn
 constexpr int kHeadChunk = 16;      // heads per TMEM load in the epilogue (16 or 32)
 constexpr int kEpiWarps = 4 * kEpiGroups;
 constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr uint32_t kTileBytes = kTile * kDim;
 constexpr uint32_t kIdesc = idesc(kFmtE4M3, kFmtE4M3, 0, 0, kTile, kHeads);
-// Tile i uses accumulator slot i % kAcc, and the group that takes tile i + kAcc
-// waits on that slot's barrier with the next phase's parity.  That wait is
-// only sound once tile i's phase has completed, which holds when the group's
-// previous tile is tile i itself or a later one: at most kAcc groups.
-static_assert(kEpiGroups <= kAcc, "more epilogue groups than accumulator slots");
+constexpr int kMaxAcc = 8;
+
+// The two key / query scale layouts: kVec = one fp32 scale per vector (one
+// accumulator of 64 columns per tile), else one per 64-dim block (an
+// accumulator per block, 128 columns per tile).
+template <bool kVec>
+struct Lay {
+  static constexpr int kAccCols = kVec ? 64 : 128;
+  static constexpr int kAcc = 512 / kAccCols;        // TMEM accumulator slots
+  static constexpr int kScaleBytes = kVec ? 4 : 8;   // key scales per entry
+  // Tile i uses accumulator slot i % kAcc, and the group that takes tile i +
+  // kAcc waits on that slot's barrier with the next phase's parity.  That
+  // wait is only sound once tile i's phase has completed, which holds when
+  // the group's previous tile is tile i itself or a later one: at most kAcc
+  // groups.
+  static_assert(kEpiGroups <= kAcc, "more epilogue groups than accumulator slots");
+  static_assert(kAcc <= kMaxAcc, "barrier arrays");
+};
 
 struct __align__(1024) Smem {
   uint8_t keys[kStages][kTileBytes];      // 1024-aligned tiles
-  float2 kscale[kStages][kTile];          // the tiles' per-entry block scales
+  float kscale[kStages][2 * kTile];       // the tiles' per-entry scales (1 or 2 each)
   uint8_t q[kHeads * kDim];               // B operand, K-major, 128-byte swizzle
-  float c0[kHeads], c1[kHeads], w[kHeads]; // per head: block-0 and block-1 query scale, weight
+  // per head: per-64 layout: block-0 / block-1 query scale and the weight;
+  // per-vector layout: query scale, scale x weight, weight
+  float c0[kHeads], c1[kHeads], w[kHeads];
   uint32_t hist[kTopkBins];
-  uint64_t full[kStages], empty[kStages], acc_full[kAcc], acc_empty[kAcc], mma_done;
+  uint64_t full[kStages], empty[kStages], acc_full[kMaxAcc], acc_empty[kMaxAcc], mma_done;
   uint32_t tmem_base;
-  int abort;
+  int abort, qscale_pos;
 };
 
 // packed fp32 pairs (sm_100 f32x2 arithmetic)
@@ -92,6 +107,7 @@ __device__ __forceinline__ void record_abort(Smem &sm, int *err, int code) {
   if (err) atomicOr(err, code);
 }
 
+template <bool kVec>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                   float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
@@ -102,6 +118,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row = blockIdx.y;
   const int b = row / a.Tq;
+  constexpr int kAcc = Lay<kVec>::kAcc, kAccCols = Lay<kVec>::kAccCols;
+  constexpr int kScaleBytes = Lay<kVec>::kScaleBytes;
 
   if (tid == 0) {
     // a stage is free again once its MMAs have completed (one commit) and
@@ -153,11 +171,21 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       const uint4 v = *reinterpret_cast<const uint4 *>(qsrc + h * kDim + c * 16);
       *reinterpret_cast<uint4 *>(&sm.q[h * kDim + ((c ^ (h & 7)) << 4)]) = v;
     }
+    if (t == 0) sm.qscale_pos = 1;
+    asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");
     for (int h = t; h < kHeads; h += nt) {
-      const float *qs = a.q_ik_scale + ((size_t)row * kHeads + h) * 2;
-      sm.c0[h] = qs[0];
-      sm.c1[h] = qs[1];
-      sm.w[h] = a.head_w[(size_t)row * kHeads + h];
+      const float wh = a.head_w[(size_t)row * kHeads + h];
+      if (kVec) {
+        const float c = a.q_ik_scale[(size_t)row * kHeads + h];
+        sm.c0[h] = c;
+        sm.c1[h] = c * wh;      // scale x weight, for the factored form
+        if (!(c > 0.f)) sm.qscale_pos = 0;
+      } else {
+        const float *qs = a.q_ik_scale + ((size_t)row * kHeads + h) * 2;
+        sm.c0[h] = qs[0];
+        sm.c1[h] = qs[1];
+      }
+      sm.w[h] = wh;
     }
     for (int i = t; i < kTopkBins; i += nt) sm.hist[i] = 0;
     fence_proxy_async_shared();
@@ -176,12 +204,12 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
         // a bulk copy must not read past it): whole 16-byte pairs of rows
         long long rows = total_rows - g0;
         rows = rows < kTile ? rows : kTile;
-        const uint32_t sbytes = (uint32_t)(rows * 8) & ~15u;
+        const uint32_t sbytes = (uint32_t)(rows * kScaleBytes) & ~15u;
         mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
         tma_load_2d(sm.keys[s], &tmap, &sm.full[s], 0, (int32_t)g0);
         if (sbytes)
-          bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + g0 * 8, sbytes,
-                    &sm.full[s]);
+          bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + g0 * kScaleBytes,
+                    sbytes, &sm.full[s]);
       };
       // the first stages are filled from the host bound before the row's
       // position has arrived (tiles past the visible ones are loaded, never used)
@@ -224,9 +252,11 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
         for (int kb = 0; kb < 2; ++kb) {
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
+            // per-vector scales: one accumulator over all 128 dims; per-64
+            // scales: one accumulator per 64-dim block
             const uint32_t off = kb * 64 + kk * 32;
-            mma_f8(tmem + acc * 128 + kb * 64, desc_kmajor_sw128(ka + off),
-                   desc_kmajor_sw128(qa + off), kIdesc, kk);
+            mma_f8(tmem + acc * kAccCols + (kVec ? 0 : kb * 64), desc_kmajor_sw128(ka + off),
+                   desc_kmajor_sw128(qa + off), kIdesc, kVec ? (kb | kk) : kk);
           }
         }
         mma_commit(&sm.empty[s]);
@@ -265,75 +295,124 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       if (j < n) {
         const long long g = (long long)b * a.ik.cap + j;
         const long long tile_rows = total_rows - (g - r);   // rows from the tile's first
-        if (!(g == total_rows - 1 && tile_rows < kTile && (tile_rows & 1))) {
-          const float2 v = sm.kscale[s][r];
-          sk0 = v.x;
-          sk1 = v.y;
+        // entries whose scales the stage's bulk copy brought (whole 16-byte
+        // groups); the rest (at most three at the very end of the cache)
+        // come by plain loads
+        const long long copied =
+            ((tile_rows < kTile ? tile_rows : kTile) * kScaleBytes & ~15LL) / kScaleBytes;
+        if (r < copied) {
+          sk0 = sm.kscale[s][kVec ? r : 2 * r];
+          if (!kVec) sk1 = sm.kscale[s][2 * r + 1];
         } else {
-          const float *sp = reinterpret_cast<const float *>(scale_base + g * 8);
+          const float *sp = reinterpret_cast<const float *>(scale_base + g * kScaleBytes);
           sk0 = __ldg(sp);
-          sk1 = __ldg(sp + 1);
+          if (!kVec) sk1 = __ldg(sp + 1);
         }
       }
       mbar_arrive(&sm.empty[s]);
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * 128;
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * kAccCols;
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-      // x_h = sk0 (sq0_h a0_h + rho sq1_h a1_h) with rho = sk1 / sk0, and since
-      // sk0 > 0, w_h max(0, x_h) = sk0 w_h max(0, sq0_h a0_h + rho sq1_h a1_h):
-      // sk0 leaves the head loop.  A warp with an entry whose sk0 is not a
-      // positive number (or whose rho overflows) takes the direct form.
-      const float rho = sk1 / sk0;
-      const bool factored = __all_sync(0xffffffffu, j >= n || (sk0 > 0.f && fabsf(rho) <= 3.0e38f));
-      const float2 k0 = make_float2(sk0, sk0), k1 = make_float2(sk1, sk1);
-      const float2 rr = make_float2(rho, rho);
-      // kHeadChunk heads per TMEM load (block 0 at column h, block 1 at 64 + h)
+      float fac = 1.f;                       // applied to the head sum
+      if constexpr (kVec) {
+        // x_h = sk c_h a_h; with sk > 0 and every c_h > 0,
+        // w_h max(0, x_h) = sk (c_h w_h) max(0, a_h): sk leaves the head loop
+        // and c_h w_h is one constant per head.  Otherwise the direct form.
+        const bool factored = sm.qscale_pos && __all_sync(0xffffffffu, j >= n || sk0 > 0.f);
+        const float2 kk = make_float2(sk0, sk0);
 #pragma unroll
-      for (int c0 = 0; c0 < kHeads; c0 += kHeadChunk) {
-        float a0[kHeadChunk], a1[kHeadChunk];
-        tmem_ld(taddr + c0, a0);
-        tmem_ld(taddr + 64 + c0, a1);
-        tmem_wait_ld();
-        if (c0 + kHeadChunk == kHeads) {
-          // the last heads are in registers: hand the accumulator slot back
-          tc_fence_before();
-          mbar_arrive(&sm.acc_empty[acc]);
-        }
-        if (factored) {
-#pragma unroll
-          for (int h = 0; h < kHeadChunk; h += 4) {
-            const int hg = c0 + h;
-            const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
-            const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
-            const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
-            float2 x = fma2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), rr,
-                            mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)));
-            float2 y = fma2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), rr,
-                            mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)));
-            x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
-            y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
-            acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
-            acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+        for (int c0 = 0; c0 < kHeads; c0 += kHeadChunk) {
+          float a0[kHeadChunk];
+          tmem_ld(taddr + c0, a0);
+          tmem_wait_ld();
+          if (c0 + kHeadChunk == kHeads) {
+            // the last heads are in registers: hand the accumulator slot back
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty[acc]);
           }
-        } else {
+          if (factored) {
 #pragma unroll
-          for (int h = 0; h < kHeadChunk; h += 4) {
-            const int hg = c0 + h;
-            const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
-            const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
-            const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
-            // x = sk0 sq0 a0 + sk1 sq1 a1 for heads (h, h+1) and (h+2, h+3)
-            float2 x = fma2(mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)), k0,
-                            mul2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), k1));
-            float2 y = fma2(mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)), k0,
-                            mul2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), k1));
-            x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
-            y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
-            acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
-            acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+            for (int h = 0; h < kHeadChunk; h += 4) {
+              const float4 D = *reinterpret_cast<const float4 *>(&sm.c1[c0 + h]);
+              const float2 x = make_float2(fmaxf(a0[h], 0.f), fmaxf(a0[h + 1], 0.f));
+              const float2 y = make_float2(fmaxf(a0[h + 2], 0.f), fmaxf(a0[h + 3], 0.f));
+              acc0 = fma2(make_float2(D.x, D.y), x, acc0);
+              acc1 = fma2(make_float2(D.z, D.w), y, acc1);
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < kHeadChunk; h += 4) {
+              const float4 C = *reinterpret_cast<const float4 *>(&sm.c0[c0 + h]);
+              const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[c0 + h]);
+              float2 x = mul2(mul2(make_float2(a0[h], a0[h + 1]), make_float2(C.x, C.y)), kk);
+              float2 y = mul2(mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C.z, C.w)), kk);
+              x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
+              y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
+              acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
+              acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+            }
           }
         }
+        fac = factored ? sk0 : 1.f;
+      } else {
+        // x_h = sk0 (sq0_h a0_h + rho sq1_h a1_h) with rho = sk1 / sk0, and
+        // since sk0 > 0, w_h max(0, x_h) = sk0 w_h max(0, sq0_h a0_h + rho
+        // sq1_h a1_h): sk0 leaves the head loop.  A warp with an entry whose
+        // sk0 is not a positive number (or whose rho overflows) takes the
+        // direct form.
+        const float rho = sk1 / sk0;
+        const bool factored =
+            __all_sync(0xffffffffu, j >= n || (sk0 > 0.f && fabsf(rho) <= 3.0e38f));
+        const float2 k0 = make_float2(sk0, sk0), k1 = make_float2(sk1, sk1);
+        const float2 rr = make_float2(rho, rho);
+        // kHeadChunk heads per TMEM load (block 0 at column h, block 1 at 64 + h)
+#pragma unroll
+        for (int c0 = 0; c0 < kHeads; c0 += kHeadChunk) {
+          float a0[kHeadChunk], a1[kHeadChunk];
+          tmem_ld(taddr + c0, a0);
+          tmem_ld(taddr + 64 + c0, a1);
+          tmem_wait_ld();
+          if (c0 + kHeadChunk == kHeads) {
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty[acc]);
+          }
+          if (factored) {
+#pragma unroll
+            for (int h = 0; h < kHeadChunk; h += 4) {
+              const int hg = c0 + h;
+              const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
+              const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
+              const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
+              float2 x = fma2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), rr,
+                              mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)));
+              float2 y = fma2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), rr,
+                              mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)));
+              x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
+              y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
+              acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
+              acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < kHeadChunk; h += 4) {
+              const int hg = c0 + h;
+              const float4 C0 = *reinterpret_cast<const float4 *>(&sm.c0[hg]);
+              const float4 C1 = *reinterpret_cast<const float4 *>(&sm.c1[hg]);
+              const float4 Wv = *reinterpret_cast<const float4 *>(&sm.w[hg]);
+              // x = sk0 sq0 a0 + sk1 sq1 a1 for heads (h, h+1) and (h+2, h+3)
+              float2 x = fma2(mul2(make_float2(a0[h], a0[h + 1]), make_float2(C0.x, C0.y)), k0,
+                              mul2(mul2(make_float2(a1[h], a1[h + 1]), make_float2(C1.x, C1.y)), k1));
+              float2 y = fma2(mul2(make_float2(a0[h + 2], a0[h + 3]), make_float2(C0.z, C0.w)), k0,
+                              mul2(mul2(make_float2(a1[h + 2], a1[h + 3]), make_float2(C1.z, C1.w)), k1));
+              x.x = fmaxf(x.x, 0.f); x.y = fmaxf(x.y, 0.f);
+              y.x = fmaxf(y.x, 0.f); y.y = fmaxf(y.y, 0.f);
+              acc0 = fma2(make_float2(Wv.x, Wv.y), x, acc0);
+              acc1 = fma2(make_float2(Wv.z, Wv.w), y, acc1);
+            }
+          }
+        }
+        fac = factored ? sk0 : 1.f;
       }
-      const float sc = ((acc0.x + acc0.y) + (acc1.x + acc1.y)) * (factored ? sk0 : 1.f);
+      const float sc = ((acc0.x + acc0.y) + (acc1.x + acc1.y)) * fac;
       // histogram: one shared-memory atomic per distinct bucket of the warp
       const unsigned live = __ballot_sync(0xffffffffu, j < n);
       if (j < n) {
@@ -377,12 +456,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 bool indexer_tc_supported(const IndexerArgs &a) {
-  if (a.ik.fmt != CSKV_FMT_E4M3_BF16 || a.d_I != kDim || a.H_I != kHeads) return false;
+  const bool vec = a.ik.fmt == CSKV_FMT_E4M3_VEC;
+  if ((a.ik.fmt != CSKV_FMT_E4M3_BF16 && !vec) || a.d_I != kDim || a.H_I != kHeads) return false;
   if ((long long)a.B * a.ik.cap >= (1LL << 31)) return false;
   if (((uintptr_t)a.ik.data & 15) || (a.ik.data_stride & 15)) return false;
-  // scales: two fp32 per entry back to back, each tile's block 16-byte aligned
-  if (a.ik.scale_stride != 8 || ((uintptr_t)a.ik.scale & 15)) return false;
-  if (a.B > 1 && (a.ik.cap & 1)) return false;
+  // scales: 8 (per-64) or 4 (per-vector) bytes per entry back to back, each
+  // tile's block 16-byte aligned
+  const long long sb = vec ? 4 : 8;
+  if (a.ik.scale_stride != sb || ((uintptr_t)a.ik.scale & 15)) return false;
+  if (a.B > 1 && (a.ik.cap * sb) % 16) return false;
   if ((uintptr_t)a.q_ik & 15) return false;
   int dev = 0, major = 0;
   cudaGetDevice(&dev);
@@ -404,7 +486,9 @@ int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(Smem) + 1024;
-  if (!ensure_dynamic_smem(indexer_tc_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+  const bool vec = a.ik.fmt == CSKV_FMT_E4M3_VEC;
+  auto kernel = vec ? indexer_tc_kernel<true> : indexer_tc_kernel<false>;
+  if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -414,8 +498,8 @@ int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_
   if (splits > tiles) splits = tiles;
   if (splits < 1) splits = 1;
   dim3 grid((unsigned)splits, (unsigned)rows);
-  return launch_pdl(indexer_tc_kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist,
-                    err) == cudaSuccess
+  return launch_pdl(kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist, err) ==
+                 cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;
 }

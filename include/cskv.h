@@ -62,7 +62,8 @@ enum {
 
 enum {
   CSKV_FMT_F32 = 0,        /* fp32 values, d_nope + d_rope per slot (no scale/rope planes) */
-  CSKV_FMT_E4M3_BF16 = 1   /* d_nope E4M3 codes + d_nope/64 fp32 scales + d_rope BF16 */
+  CSKV_FMT_E4M3_BF16 = 1,  /* d_nope E4M3 codes + d_nope/64 fp32 scales + d_rope BF16 */
+  CSKV_FMT_E4M3_VEC = 2    /* d_nope E4M3 codes + ONE fp32 scale per slot; d_rope = 0 */
 };
 
 /*
@@ -73,10 +74,14 @@ enum {
  *  - Raw-token ring   (ring = 1): token position p lives in slot p % cap.
  * E4M3_BF16 layout: value[d] = E4M3(data[d]) * scale[d / 64]  for d < d_nope,
  *                   value[d_nope + r] = BF16(rope[r])          for r < d_rope.
- * The lightning-indexer key cache uses the same descriptor with d_rope = 0.
+ * E4M3_VEC layout:  value[d] = E4M3(data[d]) * scale[0]        for d < d_nope
+ *                   (one scale per vector, no RoPE plane).
+ * The lightning-indexer key cache uses either E4M3 layout with d_rope = 0;
+ * E4M3_VEC is the one the tensor-core scoring path reads fastest (one
+ * accumulator per key and head).
  * Alignment: data and rope pointers and strides are multiples of 16 bytes;
  * scale pointer 16-byte aligned, scale stride a multiple of 4 bytes and at
- * least 4 * ceil(d_nope / 64).  F32: data pointer and stride multiples of 16.
+ * least 4 * ceil(d_nope / 64) (E4M3_BF16) or 4 (E4M3_VEC).  F32: data pointer and stride multiples of 16.
  */
 typedef struct cskv_cache {
   int32_t fmt;            /* CSKV_FMT_* */
@@ -98,9 +103,11 @@ typedef struct cskv_cache {
  * (gate_w [D] fp32 over the dequantised key, gate_b [pool] fp32 per slot),
  * a = softmax(g) over present slots, entry = sum_r a_r x_{p_r} for the key,
  * the value (raw_v, separate-V layout only) and the raw indexer key (raw_ik)
- * alike.  E4M3 outputs are re-quantised per 64-element block with
- * scale = amax / 448 (1 for an all-zero block), codes rounded to nearest even
- * and saturated; BF16 dims rounded to nearest even.
+ * alike.  E4M3 outputs are re-quantised per 64-element block (E4M3_BF16) or
+ * per vector (E4M3_VEC) with scale = amax / 448 (1 for an all-zero block),
+ * codes rounded to nearest even and saturated; BF16 dims rounded to nearest
+ * even.  Each ring has its output's layout; raw_v has raw_k's format; raw_ik
+ * is fp32 beside an fp32 raw_k and either E4M3 layout beside an E4M3 one.
  * Writes every entry j with n(t_begin[b]) <= j < n(t_end[b]), n(t) = t / stride,
  * at most max_new per sequence (the host bound that sizes the grid).
  *   t_begin, t_end : [B] device int64; tokens [t_begin, t_end) just arrived.
@@ -136,8 +143,9 @@ int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
  * entry order.
  *   q_pos    : [B][Tq] device int64, position of each query token.
  *   q_ik     : [B][Tq][H_I][d_I]; E4M3 codes when ik->fmt is E4M3_BF16 (with
- *              q_ik_scale [B][Tq][H_I][d_I/64] fp32), fp32 when ik->fmt is F32
- *              (q_ik_scale NULL).
+ *              q_ik_scale [B][Tq][H_I][d_I/64] fp32) or E4M3_VEC (with
+ *              q_ik_scale [B][Tq][H_I], one fp32 scale per head), fp32 when
+ *              ik->fmt is F32 (q_ik_scale NULL).
  *   head_w   : [B][Tq][H_I] fp32.
  *   ik       : indexer-key cache (ring = 0, d_nope = d_I, d_rope = 0).
  *   k        : selections per row, 1 <= k <= 4096.

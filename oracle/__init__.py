@@ -6,7 +6,7 @@ calls it and shares no code with it.
 """
 from .formats import (e4m3_decode, e4m3_encode, e4m3_value_table, bf16_decode,
                       bf16_encode)
-from .method import (n_entries, pool_positions, pool_entries, requantize,
+from .method import (n_entries, pool_positions, pool_entries, requantize, scale_block,
                      indexer_scores, topk, attend, window_positions,
                      hybrid_attention, dequant_slots, ring_slots)
 from .layer import (layer_compress, layer_indexer_topk, layer_attention,
@@ -14,7 +14,7 @@ from .layer import (layer_compress, layer_indexer_topk, layer_attention,
 
 __all__ = [
     "e4m3_decode", "e4m3_encode", "e4m3_value_table", "bf16_decode", "bf16_encode",
-    "n_entries", "pool_positions", "pool_entries", "requantize", "indexer_scores",
+    "n_entries", "pool_positions", "pool_entries", "requantize", "scale_block", "indexer_scores",
     "topk", "attend", "window_positions", "hybrid_attention", "dequant_slots",
     "ring_slots", "layer_compress", "layer_indexer_topk", "layer_attention",
     "layer_attention_dense_keys",

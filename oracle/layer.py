@@ -9,7 +9,7 @@ from __future__ import annotations
 import numpy as np
 
 from .method import (attend, dequant_slots, indexer_scores, n_entries, pool_entries,
-                     requantize, ring_slots, topk, window_positions)
+                     requantize, ring_slots, scale_block, topk, window_positions)
 
 
 def _np(t):
@@ -38,7 +38,10 @@ def _q_ik(L, b, t):
     from .formats import e4m3_decode
     sc = _np(L["q_ik_scale"])[b, t].astype(np.float64)       # [H_I][cols]
     d_I = q.shape[-1]
-    return e4m3_decode(_np(L["q_ik"])[b, t]) * np.repeat(sc[:, : (d_I + 63) // 64], 64, axis=1)[:, :d_I]
+    # the indexer queries share the indexer keys' scale layout
+    block = scale_block(L["comp_ik"]["fmt"], d_I)
+    nb = (d_I + block - 1) // block
+    return e4m3_decode(_np(L["q_ik"])[b, t]) * np.repeat(sc[:, :nb], block, axis=1)[:, :d_I]
 
 
 def _q(L, b, t):
@@ -84,10 +87,11 @@ def layer_compress(L, t_begin, t_end):
         for name, arr in zip(names, mags):
             r[name + "_mag"] = arr
         if ring_k["fmt"] != "f32":
-            for name, d_nope in (("k", ring_k["d_nope"]),
-                                 ("ik", ring_ik["d_nope"] if ring_ik else None)):
-                if name in r and d_nope is not None and len(js):
-                    codes, scales, rope = requantize(r[name], d_nope)
+            for name, cache in (("k", ring_k), ("ik", ring_ik)):
+                if name in r and cache is not None and len(js):
+                    d_nope = cache["d_nope"]
+                    codes, scales, rope = requantize(r[name], d_nope,
+                                                     scale_block(cache["fmt"], d_nope))
                     r[name + "_codes"], r[name + "_scales"], r[name + "_rope"] = codes, scales, rope
         res.append(r)
     return res

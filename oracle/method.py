@@ -79,10 +79,18 @@ def pool_entries(gate_src, values, gate_w, gate_b, pool: int, stride: int, j_lis
     return [np.asarray(o) for o in outs], np.asarray(weights)
 
 
-def requantize(c: np.ndarray, d_nope: int):
+def scale_block(fmt: str, d_nope: int) -> int:
+    """Dims per fp32 scale: 64 for the KV-cache layout ("e4m3"), the whole
+    vector for the indexer layout ("e4m3vec": one scale per key or query
+    head)."""
+    return d_nope if fmt == "e4m3vec" else 64
+
+
+def requantize(c: np.ndarray, d_nope: int, block: int = 64):
     """Store pooled entries in the cache format: FP8 E4M3 for the first d_nope
-    dims with one fp32 scale per 64-element block, BF16 for the rest
-    [chaosnode; golem: the last 64 values carry RoPE and stay BF16].
+    dims with one fp32 scale per `block`-element block, BF16 for the rest
+    [chaosnode; golem: the last 64 values carry RoPE and stay BF16].  The KV
+    cache uses 64-element blocks; the indexer keys one block per vector.
 
     READING: scale = amax/448 over the block (1 when the block is all zero),
     code = E4M3(c / scale) rounded to nearest-even and saturated.
@@ -90,15 +98,15 @@ def requantize(c: np.ndarray, d_nope: int):
     """
     c = np.asarray(c, dtype=np.float64)
     n = c.shape[0]
-    nb = (d_nope + 63) // 64
+    nb = (d_nope + block - 1) // block
     codes = np.empty((n, d_nope), dtype=np.uint8)
     scales = np.empty((n, nb), dtype=np.float64)
     for b in range(nb):
-        blk = c[:, 64 * b: min(64 * (b + 1), d_nope)]
+        blk = c[:, block * b: min(block * (b + 1), d_nope)]
         amax = np.max(np.abs(blk), axis=1)
         s = np.where(amax > 0, amax / E4M3_MAX, 1.0)
         scales[:, b] = s
-        codes[:, 64 * b: 64 * b + blk.shape[1]] = e4m3_encode(blk / s[:, None])
+        codes[:, block * b: block * b + blk.shape[1]] = e4m3_encode(blk / s[:, None])
     rope = bf16_encode(c[:, d_nope:])
     return codes, scales, rope
 
@@ -176,16 +184,18 @@ def dequant_slots(cache: dict, b: int, slots) -> np.ndarray:
     """Float64 values of the given slots of sequence b.
 
     cache: numpy planes {"fmt", "d_nope", "d_rope", "data", "scale", "rope"}.
-    E4M3 layout: x[d] = E4M3(code[d]) * scale[d // 64] for d < d_nope, and
-    x[d_nope + r] = BF16(rope[r]).  f32 layout: the stored values."""
+    E4M3 layouts: x[d] = E4M3(code[d]) * scale[d // block] for d < d_nope
+    (block 64, or the whole vector for "e4m3vec"), and x[d_nope + r] =
+    BF16(rope[r]).  f32 layout: the stored values."""
     slots = np.asarray(slots, dtype=np.int64)
     if cache["fmt"] == "f32":
         return cache["data"][b, slots].astype(np.float64)
     d_nope, d_rope = cache["d_nope"], cache["d_rope"]
-    nb = (d_nope + 63) // 64
+    block = scale_block(cache["fmt"], d_nope)
+    nb = (d_nope + block - 1) // block
     codes = cache["data"][b, slots]
     sc = cache["scale"][b, slots][:, :nb].astype(np.float64)
-    nope = e4m3_decode(codes) * np.repeat(sc, 64, axis=1)[:, :d_nope]
+    nope = e4m3_decode(codes) * np.repeat(sc, block, axis=1)[:, :d_nope]
     if d_rope == 0:
         return nope
     rope = bf16_decode(cache["rope"][b, slots])

@@ -100,12 +100,14 @@ def check_pooled_f32(got, ref_vals, ref_mag, where=""):
 
 def check_compressed_e4m3(cache, b, js, ref_vals, ref_mag, d_nope, where=""):
     """cache: GPU planes (torch); ref_vals: oracle pooled float64 [n][D];
-    ref_mag: sum_r a_r |x_r| per element (the error scale of each sum)."""
+    ref_mag: sum_r a_r |x_r| per element (the error scale of each sum).
+    The scale block is 64 elements, or the whole vector for "e4m3vec"."""
     js = np.asarray(js)
     codes = cache["data"][b, js].cpu().numpy()
-    nb = d_nope // 64
+    blk = O.scale_block(cache["fmt"], d_nope)
+    nb = d_nope // blk
     scales = cache["scale"][b, js][:, :nb].cpu().double().numpy()
-    blocks = [slice(64 * i, 64 * (i + 1)) for i in range(nb)]
+    blocks = [slice(blk * i, blk * (i + 1)) for i in range(nb)]
     amax = np.stack([np.max(np.abs(ref_vals[:, s_]), axis=1) for s_ in blocks], axis=1)
     mmax = np.stack([np.max(ref_mag[:, s_], axis=1) for s_ in blocks], axis=1)
     ref_s = np.where(amax > 0, amax / 448.0, 1.0)
@@ -113,7 +115,7 @@ def check_compressed_e4m3(cache, b, js, ref_vals, ref_mag, d_nope, where=""):
     s_tol = POOL_EPS * np.where(amax > 0, mmax / np.maximum(amax, 1e-300), 0.0) + 1e-7
     serr = np.abs(scales / ref_s - 1.0)
     assert np.all(serr <= s_tol), f"{where}: scale rel err {np.max(serr):.3e}"
-    s_el = np.repeat(scales, 64, axis=1)
+    s_el = np.repeat(scales, blk, axis=1)
     y = ref_vals[:, :d_nope] / s_el
     dy = POOL_EPS * ref_mag[:, :d_nope] / s_el
     exact = check_codes(codes, y, O.e4m3_encode, O.e4m3_decode, dy, where=where + " e4m3")

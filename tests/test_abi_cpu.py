@@ -122,6 +122,26 @@ def test_argument_errors_are_caught_on_the_host(C):
                             None, None, None) == ERR_ARG
     assert lib.hca_compress(1, ctx, ctx, 1, R(ring), None, gate, gate, 64, 128, R(comp), None,
                             None) == ERR_ARG
+    # compress formats: an fp32 indexer ring beside an FP8 KV ring, a per-vector
+    # V ring beside a per-64 K ring, a per-vector layout with RoPE dims
+    small_ring = _fake_cache(1, cap=16)
+    ik_f32 = _fake_cache(1, cap=16, fmt=C.FMT_F32, d_nope=128, d_rope=0)
+    ik_f32_out = _fake_cache(0, cap=8192, fmt=C.FMT_F32, d_nope=128, d_rope=0)
+    ik_f32.data_stride = ik_f32_out.data_stride = 512
+    assert lib.csa_compress(1, ctx, ctx, 1, R(small_ring), None, R(ik_f32), gate, gate, 8, 4,
+                            R(comp), None, R(ik_f32_out), None) == ERR_ARG
+    v_vec = _fake_cache(1, cap=16, fmt=C.FMT_E4M3_VEC, d_rope=0)
+    v_vec_out = _fake_cache(0, cap=8192, fmt=C.FMT_E4M3_VEC, d_rope=0)
+    assert lib.csa_compress(1, ctx, ctx, 1, R(small_ring), R(v_vec), None, gate, gate, 8, 4,
+                            R(comp), R(v_vec_out), None, None) == ERR_ARG
+    vec_rope = _fake_cache(0, cap=8192, fmt=C.FMT_E4M3_VEC)
+    assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(vec_rope), None, 128, None, 0, 8192,
+                                  R(ring), None, 128, out, lse, ws, big, None) == ERR_UNSUP
+    # per-vector indexer keys with a scale stride under 4 bytes
+    ik_vec = _fake_cache(0, cap=262144, fmt=C.FMT_E4M3_VEC, d_nope=128, d_rope=0)
+    ik_vec.data_stride, ik_vec.scale_stride = 128, 0
+    assert lib.indexer_topk(*args, R(ik_vec), 4, 1024, 262144, out, None, ws, big,
+                            None) == ERR_ARG
     # zero-sized work is a no-op success without touching the device
     assert lib.csa_compress(1, ctx, ctx, 0, R(ring), None, None, gate, gate, 8, 4, R(comp),
                             None, None, None) == 0

@@ -49,9 +49,9 @@ def test_compress_f32_tiny(C, kind, span):
         check_pooled_f32(got, ref[name], ref[name + "_mag"], where=f"{kind} {name}")
 
 
-@pytest.mark.parametrize("kind", ["csa", "hca"])
-def test_compress_e4m3_parity_decode(C, kind):
-    wl = W.get("parity_decode")
+@pytest.mark.parametrize("kind,ik_fmt", [("csa", "e4m3vec"), ("csa", "e4m3"), ("hca", "e4m3vec")])
+def test_compress_e4m3_parity_decode(C, kind, ik_fmt):
+    wl = W.get("parity_decode").with_(ik_fmt=ik_fmt)
     mk = W.make_csa_layer if kind == "csa" else W.make_hca_layer
     L = mk(wl, ring_cap=1024)
     Ld = to_device(L)
@@ -93,9 +93,14 @@ def _run_indexer(C, Ld, k=None):
     return layer
 
 
-@pytest.mark.parametrize("name", ["tiny", "parity_decode", "parity_prefill"])
-def test_indexer_topk(C, name):
+@pytest.mark.parametrize("name,ik_fmt", [("tiny", "f32"), ("parity_decode", "e4m3vec"),
+                                         ("parity_prefill", "e4m3vec"),
+                                         ("parity_decode", "e4m3"), ("parity_prefill", "e4m3")])
+def test_indexer_topk(C, name, ik_fmt):
+    # both FP8 indexer layouts: one scale per vector, and one per 64 dims
     wl = W.get(name)
+    if ik_fmt != "f32":
+        wl = wl.with_(ik_fmt=ik_fmt)
     L = W.make_csa_layer(wl)
     Ld = to_device(L)
     layer = _run_indexer(C, Ld)
@@ -124,17 +129,20 @@ def test_indexer_score_then_select_is_indexer_topk(C, name):
     assert torch.equal(whole.score, split.score)
 
 
-@pytest.mark.parametrize("T,k", [(3, 8), (4, 8), (64, 16), (64, 100), (517, 129), (1000, 100),
-                                 (2100, 500), (40000, 4096)])
-def test_indexer_edge_sizes(C, T, k):
-    wl = W.get("parity_decode").with_(T=T, B=2, k=k)
+@pytest.mark.parametrize("T,k,ik_fmt", [(3, 8, "e4m3vec"), (4, 8, "e4m3vec"), (64, 16, "e4m3vec"),
+                                        (64, 100, "e4m3vec"), (517, 129, "e4m3vec"),
+                                        (1000, 100, "e4m3vec"), (2100, 500, "e4m3vec"),
+                                        (40000, 4096, "e4m3vec"), (517, 129, "e4m3"),
+                                        (40000, 4096, "e4m3")])
+def test_indexer_edge_sizes(C, T, k, ik_fmt):
+    wl = W.get("parity_decode").with_(T=T, B=2, k=k, ik_fmt=ik_fmt)
     L = W.make_csa_layer(wl)
     Ld = to_device(L)
     layer = _run_indexer(C, Ld)
     ref = O.layer_indexer_topk(L, k)
     idx = layer.idx.cpu().numpy()
     for (b, t), (ridx, rs) in ref.items():
-        check_topk(idx[b, t], ridx, rs, where=f"T={T} k={k} row {(b, t)}")
+        check_topk(idx[b, t], ridx, rs, where=f"T={T} k={k} {ik_fmt} row {(b, t)}")
 
 
 def _tied_keys(wl, needles, every):

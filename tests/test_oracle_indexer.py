@@ -58,3 +58,48 @@ def test_topk_respects_visibility_and_prefers_lower_index():
     s = np.array([5.0, 5.0, 5.0, 9.0])
     assert list(O.topk(s, 3, 2)) == [0, 1]
     assert list(O.topk(s, 0, 2)) == [-1, -1]
+
+
+def _layer_scores_brute_force(L, b, n):
+    """Score of entries 0..n-1 for query row (b, 0) from the stored codes,
+    decoded through the E4M3 value table, with every scale applied to its
+    own dims: sum_h w_h max(0, sum_d q[h,d] sq[h, blk(d)] k[j,d] sk[j, blk(d)])."""
+    tab = O.e4m3_value_table()
+    blk = O.scale_block(L["comp_ik"]["fmt"], L["wl"].d_I)
+    q = L["q_ik"][b, 0].numpy()
+    sq = L["q_ik_scale"][b, 0].double().numpy()
+    kc = L["comp_ik"]["data"][b].numpy()
+    sk = L["comp_ik"]["scale"][b].double().numpy()
+    w = L["head_w"][b, 0].double().numpy()
+    H, d_I = q.shape
+    out = np.zeros(n)
+    for j in range(n):
+        tot = 0.0
+        for h in range(H):
+            dot = 0.0
+            for d in range(d_I):
+                dot += tab[q[h, d]] * sq[h, d // blk] * tab[kc[j, d]] * sk[j, d // blk]
+            tot += w[h] * max(dot, 0.0)
+        out[j] = tot
+    return out
+
+
+def test_layer_scores_follow_each_indexer_scale_layout():
+    # tiny FP8 layer, both indexer layouts: the query scales follow the keys'
+    import workloads as W
+    base = W.get("parity_decode").with_(B=1, T=163, H_I=3, d_I=64, k=8, needles=0)
+    for ik_fmt in ("e4m3vec", "e4m3"):
+        wl = base.with_(ik_fmt=ik_fmt)
+        L = W.make_csa_layer(wl)
+        (idx, s), = O.layer_indexer_topk(L, wl.k).values()
+        ref = _layer_scores_brute_force(L, 0, len(s))
+        assert np.allclose(s, ref, rtol=1e-12, atol=1e-12)
+    # the same codes under two scale layouts give different scores
+    wl = base.with_(ik_fmt="e4m3", d_I=128)
+    L = W.make_csa_layer(wl)
+    (idx, s), = O.layer_indexer_topk(L, wl.k).values()
+    assert np.allclose(s, _layer_scores_brute_force(L, 0, len(s)), rtol=1e-12, atol=1e-12)
+    L["comp_ik"]["fmt"] = "e4m3vec"
+    (idx2, s2), = O.layer_indexer_topk(L, wl.k).values()
+    assert np.allclose(s2, _layer_scores_brute_force(L, 0, len(s2)), rtol=1e-12, atol=1e-12)
+    assert not np.allclose(s, s2)

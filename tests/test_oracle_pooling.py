@@ -131,6 +131,42 @@ def test_requantize_zero_block_and_codes_match_torch():
     assert np.array_equal(ref, qc)
 
 
+def test_requantize_one_scale_per_vector():
+    # the indexer layout: one scale over all 128 dims, no BF16 part
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 0x7E, size=(12, 128)).astype(np.uint8)
+    codes[:, 77] = 0xFE                     # amax = 448 * s, sign negative
+    s = rng.uniform(0.01, 3.0, size=(12, 1))
+    c = O.e4m3_decode(codes) * s
+    qc, qs, qr = O.requantize(c, 128, O.scale_block("e4m3vec", 128))
+    assert qs.shape == (12, 1) and qr.shape[1] == 0
+    assert np.array_equal(qc, codes)
+    assert np.allclose(qs, s, rtol=1e-15, atol=0)
+    # a block-64 quantisation of the same rows keeps two scales, and differs
+    # wherever the two halves' maxima differ
+    qc64, qs64, _ = O.requantize(c, 128)
+    assert qs64.shape == (12, 2)
+    half = np.abs(O.e4m3_decode(codes)).reshape(12, 2, 64).max(axis=2) * s
+    assert np.allclose(qs64, half / 448.0, rtol=1e-15)
+    # the zero vector takes scale 1 and zero codes
+    z, zs, _ = O.requantize(np.zeros((1, 128)), 128, 128)
+    assert zs[0, 0] == 1.0 and not z.any()
+
+
+def test_dequant_slots_per_vector_brute_force():
+    rng = np.random.default_rng(6)
+    codes = rng.integers(0, 256, size=(2, 9, 32)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0      # no NaN codes
+    sc = rng.uniform(0.1, 2.0, size=(2, 9, 1))
+    cache = {"fmt": "e4m3vec", "d_nope": 32, "d_rope": 0, "data": codes, "scale": sc,
+             "rope": None}
+    tab = O.e4m3_value_table()
+    got = O.dequant_slots(cache, 1, [4, 0, 8])
+    for r, j in enumerate([4, 0, 8]):
+        for d in range(32):
+            assert got[r, d] == tab[codes[1, j, d]] * sc[1, j, 0]
+
+
 def test_layer_compress_tiny_uniform_gate_equals_mean():
     wl = W.get("tiny")
     L = W.make_csa_layer(wl)

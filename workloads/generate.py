@@ -57,19 +57,20 @@ class _Rng:
         return torch.randint(lo, hi, shape, generator=self.g, device=self.device)
 
 
-def _scale_cols(d_nope: int, pad: int) -> int:
-    nb = (d_nope + 63) // 64
+def _scale_cols(d_nope: int, pad: int, block: int = 64) -> int:
+    nb = (d_nope + block - 1) // block
     return ((nb + pad - 1) // pad) * pad
 
 
-def _fp8_planes(rng: _Rng, lead, d_nope: int, scale_pad: int):
-    """codes uint8 [*lead, d_nope], scales f32 [*lead, cols] (pad columns NaN)."""
-    nb = (d_nope + 63) // 64
+def _fp8_planes(rng: _Rng, lead, d_nope: int, scale_pad: int, block: int = 64):
+    """codes uint8 [*lead, d_nope], scales f32 [*lead, cols] (pad columns NaN);
+    one scale per `block` dims."""
+    nb = (d_nope + block - 1) // block
     x = rng.normal(*lead, d_nope)
     s = rng.uniform(0.5, 2.0, *lead, nb)
-    s_el = s.repeat_interleave(64, dim=-1)[..., :d_nope]
+    s_el = s.repeat_interleave(block, dim=-1)[..., :d_nope]
     codes = e4m3_from_float(x / s_el)
-    cols = _scale_cols(d_nope, scale_pad)
+    cols = _scale_cols(d_nope, scale_pad, block)
     scale = torch.full((*lead, cols), float("nan"), device=rng.device, dtype=torch.float32)
     scale[..., :nb] = s
     return codes, scale
@@ -82,7 +83,8 @@ def _cache(rng: _Rng, wl: Workload, B: int, n: int, *, d_nope: int, d_rope: int,
     if fmt == "f32":
         c["data"] = rng.normal(B, n, d_nope + d_rope)
     else:
-        c["data"], c["scale"] = _fp8_planes(rng, (B, n), d_nope, scale_pad)
+        block = d_nope if fmt == "e4m3vec" else 64
+        c["data"], c["scale"] = _fp8_planes(rng, (B, n), d_nope, scale_pad, block)
         if d_rope:
             c["rope"] = rng.normal(B, n, d_rope).to(torch.bfloat16)
     return c
@@ -154,7 +156,8 @@ def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
     kw = dict(d_nope=wl.d_nope, d_rope=wl.d_rope, fmt=wl.fmt, scale_pad=8)
     L["ring_k"] = _cache(rng, wl, wl.B, cap, ring=True, **kw)
     L["ring_v"] = _cache(rng, wl, wl.B, cap, ring=True, **kw) if wl.separate_v else None
-    ik_kw = dict(d_nope=wl.d_I, d_rope=0, fmt=wl.fmt, scale_pad=2)
+    ik_fmt = "f32" if wl.fmt == "f32" else wl.ik_fmt
+    ik_kw = dict(d_nope=wl.d_I, d_rope=0, fmt=ik_fmt, scale_pad=1 if ik_fmt == "e4m3vec" else 2)
     L["ring_ik"] = _cache(rng, wl, wl.B, cap, ring=True, **ik_kw)
     for key in ("ring_k", "ring_v", "ring_ik"):
         if L[key] is not None:
@@ -168,7 +171,8 @@ def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
         L["q_ik"] = rng.normal(wl.B, wl.Tq, wl.H_I, wl.d_I)
         L["q_ik_scale"] = None
     else:
-        L["q_ik"], L["q_ik_scale"] = _fp8_planes(rng, (wl.B, wl.Tq, wl.H_I), wl.d_I, 1)
+        L["q_ik"], L["q_ik_scale"] = _fp8_planes(rng, (wl.B, wl.Tq, wl.H_I), wl.d_I, 1,
+                                                 wl.d_I if ik_fmt == "e4m3vec" else 64)
     L["head_w"] = rng.normal(wl.B, wl.Tq, wl.H_I) / math.sqrt(wl.H_I)
     L["gate_w"] = rng.normal(wl.D, std=0.1)
     L["gate_b"] = rng.normal(wl.csa_pool, std=0.1)
@@ -185,7 +189,8 @@ def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
                 L["comp_ik"]["data"][b, j] = L["q_ik"][b, 0, hstar] * 4.0
             else:
                 L["comp_ik"]["data"][b, j] = L["q_ik"][b, 0, hstar]
-                L["comp_ik"]["scale"][b, j, :] = L["q_ik_scale"][b, 0, hstar, :2] * 4.0
+                nbq = L["q_ik_scale"].shape[-1]
+                L["comp_ik"]["scale"][b, j, :nbq] = L["q_ik_scale"][b, 0, hstar, :nbq] * 4.0
             _plant_kv_needle(L["comp_k"], b, j, L["q"][b, 0, 0], rng)
     return L
 
