@@ -384,7 +384,7 @@ def run_ours(args, rank, world, dev):
     return res, replicas, wl
 
 
-_TRAFFIC_SOURCES = ["indexer.cu", "indexer_tc.cu", "topk_common.cuh", "sm100.cuh"]
+_TRAFFIC_SOURCES = ["indexer.cu", "indexer_tc.cu", "topk_common.cuh", "sm100.cuh", "cskv_internal.cuh"]
 
 
 def _profile_traffic(workload):
