@@ -290,15 +290,14 @@ def step_bytes(wl):
     return int(csa + hca + compress)
 
 
-def run_ours(args, rank, world, dev):
-    import compressed_sparse_kv_softmax_b200 as C  # noqa: F401  (fails loudly without the .so)
-    wl = W.get(args.workload)
-    torch.cuda.set_device(dev)
+def _time_decode(args, wl, rank, world, dev, steps, seed0, clocks=True):
+    """Build the rotating replicas of `wl`, warm up, capture the step graph and
+    time exactly `steps` steps (max over ranks).  Returns the timing record."""
     per_rep_bytes = step_bytes(wl)
     # enough replicas that one rotation touches > 4x the 126 MB L2 (unless set)
     R = args.replicas if args.replicas > 0 else math.ceil(4 * 126e6 / per_rep_bytes) + 1
     sched = Schedule(wl, dev)
-    replicas = [Replica(wl, sched, 1000 + r + 7919 * rank, dev) for r in range(R)]
+    replicas = [Replica(wl, sched, seed0 + r + 7919 * rank, dev) for r in range(R)]
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
     # warm-up: W steps eagerly through the public API (also performs the
@@ -307,14 +306,15 @@ def run_ours(args, rank, world, dev):
         for i in range(args.warmup):
             replicas[i % R].step(i % PERIOD)
     stream.synchronize()
-    G = max(1, min(args.graph_steps, args.steps))
+    G = max(1, min(args.graph_steps, steps))
     graph = StepGraph(replicas, G, stream)
-    rest = args.steps % G
-    tail = StepGraph(replicas, rest, stream, i0=(args.steps // G) * G) if rest else None
+    rest = steps % G
+    tail = StepGraph(replicas, rest, stream, i0=(steps // G) * G) if rest else None
 
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
-    sampler.start()
-    time.sleep(0.3)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0) if clocks else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
     # untimed graph replays so the clock sampler sees the GPU under load
     with torch.cuda.stream(stream):
         for _ in range(max(1, int(0.2 / max(1e-6, 30e-6 * G)))):
@@ -325,7 +325,7 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    n_launch = args.steps // G
+    n_launch = steps // G
     with torch.cuda.stream(stream):
         t0.record(stream)
         for _ in range(n_launch):
@@ -336,14 +336,47 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
+    clk = sampler.stop() if sampler else None
     ms = t0.elapsed_time(t1)
-    steps_done = n_launch * G + rest
     if world > 1:
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    idx_ms = float(np.mean(graph.indexer_ms()))
+    return {"ms": ms, "steps": n_launch * G + rest, "idx_ms": float(np.mean(graph.indexer_ms())),
+            "clocks": clk, "replicas": replicas, "R": R, "sched": sched,
+            "per_rep_bytes": per_rep_bytes,
+            "launches": graph.kernels * n_launch + (tail.kernels if tail else 0)}
+
+
+def _other_layout(args, wl, rank, world, dev):
+    """The same step with the other FP8 indexer scale layout, timed briefly:
+    the layout comparison rides along with the headline number."""
+    other = wl.with_(ik_fmt="e4m3" if wl.ik_fmt == "e4m3vec" else "e4m3vec")
+    t = _time_decode(args, other, rank, world, dev, args.alt_steps, 5000, clocks=False)
+    ib = indexer_bytes(other)
+    peak, _ = _peaks()
+    achieved = ib / (t["idx_ms"] / 1e3) / 1e9
+    out = {"indexer_scales": _scales_text(other),
+           "value": round(other.B * t["steps"] * world / (t["ms"] / 1e3), 2), "unit": UNIT,
+           "steps": t["steps"], "ms_per_step": t["ms"] / t["steps"],
+           "indexer_score_us": round(t["idx_ms"] * 1e3, 3),
+           "indexer_algorithmic_bytes": ib, "indexer_frac": round(achieved / peak, 4)}
+    del t
+    torch.cuda.empty_cache()
+    return out
+
+
+def _scales_text(wl):
+    return "one fp32 per key / query head" if wl.ik_fmt == "e4m3vec" else "one fp32 per 64 dims"
+
+
+def run_ours(args, rank, world, dev):
+    import compressed_sparse_kv_softmax_b200 as C  # noqa: F401  (fails loudly without the .so)
+    wl = W.get(args.workload).with_(ik_fmt=args.ik_fmt)
+    torch.cuda.set_device(dev)
+    t = _time_decode(args, wl, rank, world, dev, args.steps, 1000)
+    replicas, R, sched, per_rep_bytes = t["replicas"], t["R"], t["sched"], t["per_rep_bytes"]
+    ms, steps_done, idx_ms, clocks = t["ms"], t["steps"], t["idx_ms"], t["clocks"]
     total_q = wl.B * steps_done * world
     value = total_q / (ms / 1e3)
 
@@ -358,7 +391,7 @@ def run_ours(args, rank, world, dev):
                 "algorithmic_bytes_per_launch": ib, "avg_launch_us": round(idx_ms * 1e3, 3),
                 "timed_launches": f"every {EVENT_EVERY}th step of the last graph replay, "
                                   f"events on a side stream (no serialisation of the step)"}
-    traffic = _profile_traffic(args.workload)
+    traffic = _profile_traffic(args.workload) if wl.ik_fmt == "e4m3vec" else None
     if traffic is not None:
         roofline["traffic"] = traffic
 
@@ -371,16 +404,18 @@ def run_ours(args, rank, world, dev):
                                   f"around {wl.T}: 32 CSA + 1 HCA compressions), Hq={wl.Hq}, "
                                   f"D={wl.d_nope}+{wl.d_rope}, H_I={wl.H_I}x{wl.d_I}, k={wl.k}, "
                                   f"window={wl.window}",
-                      "indexer_scales": "one fp32 per key / query head"
-                                        if wl.ik_fmt == "e4m3vec" else "one fp32 per 64 dims",
+                      "indexer_scales": _scales_text(wl),
                       "global_batch": wl.B * world, "seq_len": wl.T,
                       "parallelism": f"replicas x{world} (weak)",
                       "l2": f"{R} rotating input replicas, {R * per_rep_bytes / 1e6:.0f} MB "
                             f"touched per cycle (> 4x L2)",
                       "step_bytes": per_rep_bytes},
            "roofline": roofline,
-           "gpu_launches": graph.kernels * n_launch + (tail.kernels if tail else 0),
+           "gpu_launches": t["launches"],
            "clocks": clocks}
+    del t
+    if args.alt_steps > 0:
+        res["other_indexer_layout"] = _other_layout(args, wl, rank, world, dev)
     return res, replicas, wl
 
 
@@ -552,7 +587,7 @@ def run_reference(args, rank, world):
     whole run ends within a few minutes."""
     if rank != 0:
         return None
-    wl = W.get(args.workload)
+    wl = W.get(args.workload).with_(ik_fmt=args.ik_fmt)
     Lc = _cpu_layer(W.make_csa_layer(wl, seed=1000))
     Lh = _cpu_layer(W.make_hca_layer(wl, seed=501_000))
     t = time.perf_counter()
@@ -572,7 +607,8 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"{wl.name}: 1 CSA + 1 HCA layer decode, B={wl.B}, ctx={wl.T}"},
+            "config": {"workload": f"{wl.name}: 1 CSA + 1 HCA layer decode, B={wl.B}, ctx={wl.T}",
+                       "indexer_scales": _scales_text(wl)},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores,
                              "kind": "oracle",
                              "sample": f"each step: one decode query over the first "
@@ -593,7 +629,7 @@ def run_prefill(args, rank, world, dev):
     than L2.  The metric is prefill tokens/s; the roofline object reports the
     indexer scoring's tensor FLOP rate against the FP8 peak."""
     from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
-    wl = W.get(args.workload)
+    wl = W.get(args.workload).with_(ik_fmt=args.ik_fmt)
     torch.cuda.set_device(dev)
     csa = CSALayer(W.make_csa_layer(wl, device=dev, seed=1000 + 7919 * rank))
     hca = HCALayer(W.make_hca_layer(wl, device=dev, seed=501000 + 7919 * rank))
@@ -663,6 +699,7 @@ def run_prefill(args, rank, world, dev):
                                   f"{wl.T}..{wl.T + wl.Tq - 1}, Hq={wl.Hq}, "
                                   f"D={wl.d_nope}+{wl.d_rope}, H_I={wl.H_I}x{wl.d_I}, "
                                   f"k={wl.k}, window={wl.window}",
+                      "indexer_scales": _scales_text(wl),
                       "l2": "per-step tensors (queries 0.5 GB, outputs 2 GB, scores 8.6 GB) "
                             "far above L2"},
            "roofline": {"bound": "tensor", "achieved": round(idx_tflops, 2),
@@ -693,6 +730,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ik-fmt", default="e4m3vec", choices=["e4m3vec", "e4m3"],
+                    help="FP8 indexer scale layout: one scale per vector, or per 64 dims")
+    ap.add_argument("--alt-steps", type=int, default=4096,
+                    help="steps timed with the other indexer layout (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

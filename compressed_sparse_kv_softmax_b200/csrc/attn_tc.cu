@@ -27,8 +27,9 @@
 //      entries, the window) arrives by bulk copies into the still unused Q
 //      buffer while Q is loaded into registers; otherwise each lane loads its
 //      part of the rows (all loads first, Q staged meanwhile).  Conversion:
-//      lanes 0-27 take 16 FP8 codes each (x block scale), lanes 28-31 16
-//      BF16 RoPE values each.  Per 64-dim chunk the key tile holds 64 rows of
+//      a row is 28 units of 16 FP8 codes (x block scale) and 8 units of 8
+//      BF16 RoPE values; lane l of a warp with rpw rows takes row l % rpw
+//      and every (32 / rpw)-th unit.  Per 64-dim chunk the key tile holds 64 rows of
 //      hi parts then 64 rows of lo parts (K-major, 128-byte swizzle).  Q
 //      becomes FP16 in the same layout [8 chunks][64 heads][128 B].
 //   2. [K_hi; K_lo] Q^T with the 128 stacked rows on the MMA M axis (N = 64
@@ -214,46 +215,78 @@ __device__ __forceinline__ void store_q(const uint4 (&raw)[16], uint8_t *q) {
   }
 }
 
-// Convert key row r (16 FP8 codes x block scale on lanes 0-27, 16 BF16 RoPE
-// values on lanes 28-31) into its hi and lo FP16 parts in the key tile.
-__device__ __forceinline__ void convert_row(uint8_t *kt, int r, int lane, const uint4 &raw,
-                                            const uint4 &raw2, float sc) {
+// Key-row conversion work of one warp: its rpw rows (2, 4 or 8) hold 28
+// code units each (16 FP8 codes of one 64-dim block, x the block's scale)
+// and 8 RoPE units (8 BF16 values).  Lane l takes row l % rpw and the units
+// l / rpw + k * (32 / rpw): every lane converts, none diverges, and each
+// store of the warp covers every 16-byte bank group of the swizzled tile
+// exactly four times (four wavefronts per 512 bytes).
+constexpr int kCodeUnits = kDn / 16;                 // 28 per row
+constexpr int kRopeUnits = kDr / 8;                  // 8 per row
+constexpr int kCodeIt = 7, kRopeIt = 2;              // per lane at rpw = 8 (the most)
+
+struct RowParts {
+  uint4 code[kCodeIt];
+  float sc[kCodeIt];
+  uint4 rope[kRopeIt];
+};
+
+// code unit k / RoPE unit k of this lane (>= the per-row count: none)
+__device__ __forceinline__ int code_unit(int lane, int lg, int k) { return (lane >> lg) + (k << (5 - lg)); }
+
+// 16 codes x scale -> hi and lo FP16 parts at dims 16 j .. 16 j + 15 of row r
+__device__ __forceinline__ void convert_code_unit(uint8_t *kt, int r, int j, const uint4 &raw,
+                                                  float sc) {
   uint4 h0, h1, l0, l1;
   uint32_t *ph0 = reinterpret_cast<uint32_t *>(&h0), *ph1 = reinterpret_cast<uint32_t *>(&h1);
   uint32_t *pl0 = reinterpret_cast<uint32_t *>(&l0), *pl1 = reinterpret_cast<uint32_t *>(&l1);
-  int d0;
-  if (lane < 28) {
-    const uint32_t *cw = reinterpret_cast<const uint32_t *>(&raw);
+  const uint32_t *cw = reinterpret_cast<const uint32_t *>(&raw);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 x = e4m3x2(cw[q] & 0xffffu), y = e4m3x2(cw[q] >> 16);
-      if (q < 2) {
-        split_h2(x.x * sc, x.y * sc, ph0[2 * q], pl0[2 * q]);
-        split_h2(y.x * sc, y.y * sc, ph0[2 * q + 1], pl0[2 * q + 1]);
-      } else {
-        split_h2(x.x * sc, x.y * sc, ph1[2 * q - 4], pl1[2 * q - 4]);
-        split_h2(y.x * sc, y.y * sc, ph1[2 * q - 3], pl1[2 * q - 3]);
-      }
-    }
-    d0 = lane * 16;
-  } else {
-    const __nv_bfloat162 *b0 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-    const __nv_bfloat162 *b1 = reinterpret_cast<const __nv_bfloat162 *>(&raw2);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 f0 = __bfloat1622float2(b0[q]), f1 = __bfloat1622float2(b1[q]);
-      split_h2(f0.x, f0.y, ph0[q], pl0[q]);
-      split_h2(f1.x, f1.y, ph1[q], pl1[q]);
-    }
-    d0 = kDn + (lane - 28) * 16;
+  for (int q = 0; q < 4; ++q) {
+    const float2 x = e4m3x2(cw[q] & 0xffffu), y = e4m3x2(cw[q] >> 16);
+    uint32_t *ph = q < 2 ? ph0 : ph1, *pl = q < 2 ? pl0 : pl1;
+    const int o = 2 * (q & 1);
+    split_h2(x.x * sc, x.y * sc, ph[o], pl[o]);
+    split_h2(y.x * sc, y.y * sc, ph[o + 1], pl[o + 1]);
   }
   // hi part in row r, lo part in row 64 + r of the chunk (same swizzle phase)
-  const int c = d0 >> 6, u = (d0 & 63) >> 3;
+  const int c = j >> 2, u = (j & 3) << 1;
   const uint32_t o0 = c * kChunkKK + swz(r, u), o1 = c * kChunkKK + swz(r, u + 1);
   *reinterpret_cast<uint4 *>(kt + o0) = h0;
   *reinterpret_cast<uint4 *>(kt + o1) = h1;
   *reinterpret_cast<uint4 *>(kt + kChunkK + o0) = l0;
   *reinterpret_cast<uint4 *>(kt + kChunkK + o1) = l1;
+}
+
+// 8 BF16 RoPE values -> hi and lo FP16 parts at dims 448 + 8 v .. of row r
+__device__ __forceinline__ void convert_rope_unit(uint8_t *kt, int r, int v, const uint4 &raw) {
+  uint4 h, l;
+  uint32_t *ph = reinterpret_cast<uint32_t *>(&h), *pl = reinterpret_cast<uint32_t *>(&l);
+  const __nv_bfloat162 *bp = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(bp[q]);
+    split_h2(f.x, f.y, ph[q], pl[q]);
+  }
+  const uint32_t o = (kDn / 64) * kChunkKK + swz(r, v);
+  *reinterpret_cast<uint4 *>(kt + o) = h;
+  *reinterpret_cast<uint4 *>(kt + kChunkK + o) = l;
+}
+
+// convert the parts a lane holds for row r (r < rows_out: rows past the
+// unit's MMA steps are not written)
+__device__ __forceinline__ void convert_parts(uint8_t *kt, const RowParts &p, int r, int lane,
+                                              int lg) {
+#pragma unroll
+  for (int k = 0; k < kCodeIt; ++k) {
+    const int j = code_unit(lane, lg, k);
+    if (j < kCodeUnits) convert_code_unit(kt, r, j, p.code[k], p.sc[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < kRopeIt; ++k) {
+    const int v = code_unit(lane, lg, k);
+    if (v < kRopeUnits) convert_rope_unit(kt, r, v, p.rope[k]);
+  }
 }
 
 struct Row {
@@ -342,10 +375,13 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     // (the barrier also publishes the slots) any key at all in this unit?
     if (!__syncthreads_or(tid < kM && sm.slot[tid] >= 0)) continue;
 
-    // ---- gather: warp w converts key rows 8w .. 8w+7 into the key tile
+    // ---- gather: warp w converts key rows rpw w .. rpw w + rpw - 1 into the
+    // key tile (lane l: row l % rpw, see convert_parts)
     const int rpw = unit_keys >> 3;           // key rows per warp: the unit over 8 warps
+    const int lg = __ffs(rpw) - 1;
     const int r0 = warp * rpw;
-    const bool has_rows = r0 < ksteps * 16;
+    const int my_r = r0 + (lane & (rpw - 1));
+    const bool has_rows = r0 < ksteps * 16;   // (then all rpw rows are)
     const __nv_bfloat16 *qg =
         reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD;
     // consecutive slots: the window's positions (one or two runs around the
@@ -380,24 +416,26 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
       load_q(qg, qraw);
       ok = mbar_wait(&sm.gbar, 0) && ok;     // used once per CTA: phase 0
       if (has_rows) {
-#pragma unroll 1
-        for (int e = 0; e < rpw; ++e) {
-          const int r = r0 + e;
-          uint4 raw = make_uint4(0, 0, 0, 0), raw2 = make_uint4(0, 0, 0, 0);
-          float sc = 0.f;
-          if (r < nkeys) {
-            if (lane < 28) {
-              raw = *reinterpret_cast<const uint4 *>(sm.q + r * kDn + 16 * lane);
-              sc = *reinterpret_cast<const float *>(sm.q + kStgScale + r * 32 + 4 * (lane >> 2));
-            } else {
-              const uint4 *rp =
-                  reinterpret_cast<const uint4 *>(sm.q + kStgRope + r * 2 * kDr) + 2 * (lane - 28);
-              raw = rp[0];
-              raw2 = rp[1];
-            }
+        const bool live = my_r < nkeys;
+        RowParts p;
+#pragma unroll
+        for (int k = 0; k < kCodeIt; ++k) {
+          const int j = code_unit(lane, lg, k);
+          p.code[k] = make_uint4(0, 0, 0, 0);
+          p.sc[k] = 0.f;
+          if (live && j < kCodeUnits) {
+            p.code[k] = *reinterpret_cast<const uint4 *>(sm.q + my_r * kDn + 16 * j);
+            p.sc[k] = *reinterpret_cast<const float *>(sm.q + kStgScale + my_r * 32 + 4 * (j >> 2));
           }
-          convert_row(sm.kt, r, lane, raw, raw2, sc);
         }
+#pragma unroll
+        for (int k = 0; k < kRopeIt; ++k) {
+          const int v = code_unit(lane, lg, k);
+          p.rope[k] = make_uint4(0, 0, 0, 0);
+          if (live && v < kRopeUnits)
+            p.rope[k] = *reinterpret_cast<const uint4 *>(sm.q + kStgRope + my_r * 2 * kDr + 16 * v);
+        }
+        convert_parts(sm.kt, p, my_r, lane, lg);
       }
       __syncthreads();                        // every staged row has been read
       store_q(qraw, sm.q);
@@ -405,32 +443,30 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     } else {
       // all loads are issued first, then (first unit only) Q is staged while
       // they are in flight, then the rows are converted
-      uint4 raw[8], raw2[8];
-      float sc[8];
+      const long long slot = has_rows ? sm.slot[my_r] : -1;
+      RowParts p;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        raw[e] = raw2[e] = make_uint4(0, 0, 0, 0);
-        sc[e] = 0.f;
-        const long long slot = has_rows && e < rpw ? sm.slot[r0 + e] : -1;
-        if (slot < 0) continue;
-        if (lane < 28) {
-          raw[e] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + lane);
-          sc[e] = __ldg(src.scale_ptr(b, slot) + (lane >> 2));
-        } else {
-          const uint4 *rp = reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + 2 * (lane - 28);
-          raw[e] = __ldg(rp);
-          raw2[e] = __ldg(rp + 1);
+      for (int k = 0; k < kCodeIt; ++k) {
+        const int j = code_unit(lane, lg, k);
+        p.code[k] = make_uint4(0, 0, 0, 0);
+        p.sc[k] = 0.f;
+        if (slot >= 0 && j < kCodeUnits) {
+          p.code[k] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + j);
+          p.sc[k] = __ldg(src.scale_ptr(b, slot) + (j >> 2));
         }
+      }
+#pragma unroll
+      for (int k = 0; k < kRopeIt; ++k) {
+        const int v = code_unit(lane, lg, k);
+        p.rope[k] = make_uint4(0, 0, 0, 0);
+        if (slot >= 0 && v < kRopeUnits)
+          p.rope[k] = __ldg(reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + v);
       }
       if (!q_ready) {
         stage_q(qg, sm.q);
         q_ready = true;
       }
-      if (has_rows) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (e < rpw) convert_row(sm.kt, r0 + e, lane, raw[e], raw2[e], sc[e]);
-      }
+      if (has_rows) convert_parts(sm.kt, p, my_r, lane, lg);
     }
     fence_proxy_async_shared();
     tc_fence_before();
