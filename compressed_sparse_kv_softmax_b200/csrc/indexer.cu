@@ -25,6 +25,8 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
 bool indexer_tc_supported(const IndexerArgs &a);
 int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
                       int *err, cudaStream_t st);
+int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
+                        int *err, cudaStream_t st);
 
 namespace {
 
@@ -111,7 +113,9 @@ int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st) {
       if (launch_pdl(zero_words_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
                      reinterpret_cast<uint32_t *>(w.err), words) != cudaSuccess)
         return CSKV_ERR_CUDA;
-      const int rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
+      // several query rows per sequence share each key tile; one row streams alone
+      int rc = launch_indexer_rows(a, w.scores, w.ld, w.hist, w.err, st);
+      if (rc == CSKV_ERR_UNSUPPORTED) rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
       if (rc != CSKV_OK) return rc;
     }
     if (!select) return CSKV_OK;

@@ -80,28 +80,6 @@ struct __align__(1024) Smem {
   int abort, qscale_pos;
 };
 
-// packed fp32 pairs (sm_100 f32x2 arithmetic)
-__device__ __forceinline__ unsigned long long f2u(float2 v) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
-  return r;
-}
-__device__ __forceinline__ float2 u2f(unsigned long long r) {
-  float2 v;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
-  return v;
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  unsigned long long r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2u(a)), "l"(f2u(b)));
-  return u2f(r);
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  unsigned long long r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2u(a)), "l"(f2u(b)), "l"(f2u(c)));
-  return u2f(r);
-}
-
 __device__ __forceinline__ void record_abort(Smem &sm, int *err, int code) {
   sm.abort = 1;
   if (err) atomicOr(err, code);
@@ -472,19 +450,24 @@ bool indexer_tc_supported(const IndexerArgs &a) {
   return major == 10 && encode_fn() != nullptr;
 }
 
-int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                      int *err, cudaStream_t st) {
+bool make_key_tmap(const IndexerArgs &a, CUtensorMap *map) {
   auto fn = encode_fn();
-  if (!fn) return CSKV_ERR_UNSUPPORTED;
-  CUtensorMap map;
+  if (!fn) return false;
+  // all sequences' key rows as one [B * cap] x 128-byte matrix; 128 x 128 B
+  // boxes in the 128-byte swizzle the K-major operand descriptors expect
   cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)((long long)a.B * a.ik.cap)};
   cuuint64_t strides[1] = {(cuuint64_t)a.ik.data_stride};
   cuuint32_t box[2] = {(cuuint32_t)kDim, (cuuint32_t)kTile};
   cuuint32_t estr[2] = {1, 1};
-  if (fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.ik.data, dims, strides, box, estr,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return CSKV_ERR_UNSUPPORTED;
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.ik.data, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
+                      int *err, cudaStream_t st) {
+  CUtensorMap map;
+  if (!make_key_tmap(a, &map)) return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(Smem) + 1024;
   const bool vec = a.ik.fmt == CSKV_FMT_E4M3_VEC;
   auto kernel = vec ? indexer_tc_kernel<true> : indexer_tc_kernel<false>;

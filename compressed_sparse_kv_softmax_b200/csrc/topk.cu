@@ -357,14 +357,20 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   uint32_t *ctr = w.ctr + (size_t)row * 4;
   uint64_t *candrow = w.cand + (size_t)row * kCandCap;
   int wins = 0;
+  // rows longer than one pass (few rows per launch, or a CTA per row): the
+  // next two passes' scores are requested while this one is counted
+  float v[kSelPer], p1[kSelPer], p2[kSelPer];
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
+  if (j_lo + kSelChunk < j_hi) load8(s, j_lo + kSelChunk + (long long)tid * kSelPer, j_hi, p1);
+  if (j_lo + 2 * kSelChunk < j_hi)
+    load8(s, j_lo + 2 * kSelChunk + (long long)tid * kSelPer, j_hi, p2);
   for (long long c0 = j_lo; c0 < j_hi; c0 += kSelChunk) {
     const long long j0 = c0 + (long long)tid * kSelPer;
-    float v[kSelPer];
-    if (c0 == j_lo) {
+    if (c0 != j_lo) {
 #pragma unroll
-      for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
-    } else {
-      load8(s, j0, j_hi, v);
+      for (int e = 0; e < kSelPer; ++e) { v[e] = p1[e]; p1[e] = p2[e]; }
+      if (c0 + 2 * kSelChunk < j_hi) load8(s, j0 + 2 * kSelChunk, j_hi, p2);
     }
     int nc = 0;
     uint32_t cmask = 0;
@@ -573,14 +579,17 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   // ---- 4. this slice's selected entries, in index order, at its offset
   if (!fallback) {
     int base = sm.base;
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
+    if (j_lo + kSelChunk < j_hi) load8(s, j_lo + kSelChunk + (long long)tid * kSelPer, j_hi, p1);
+    if (j_lo + 2 * kSelChunk < j_hi)
+      load8(s, j_lo + 2 * kSelChunk + (long long)tid * kSelPer, j_hi, p2);
     for (long long c0 = j_lo; c0 < j_hi; c0 += kSelChunk) {
       const long long j0 = c0 + (long long)tid * kSelPer;
-      float v[kSelPer];
-      if (c0 == j_lo) {
+      if (c0 != j_lo) {
 #pragma unroll
-        for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
-      } else {
-        load8(s, j0, j_hi, v);
+        for (int e = 0; e < kSelPer; ++e) { v[e] = p1[e]; p1[e] = p2[e]; }
+        if (c0 + 2 * kSelChunk < j_hi) load8(s, j0 + 2 * kSelChunk, j_hi, p2);
       }
       uint32_t fl = 0;
 #pragma unroll

@@ -114,6 +114,26 @@ def test_indexer_topk(C, name, ik_fmt):
         assert np.allclose(sc[b, t][: sel.size], rs[sel], rtol=1e-4, atol=1e-4 * np.abs(rs).max())
 
 
+@pytest.mark.parametrize("B,T,Tq,k", [(2, 508, 2, 16), (2, 508, 5, 64), (1, 3001, 8, 128),
+                                      (3, 1200, 13, 100), (1, 66_000, 9, 1024)])
+def test_indexer_many_rows_per_sequence(C, B, T, Tq, k):
+    # several query rows of a sequence share each key tile (groups of 8 rows,
+    # the last group ragged); positions T .. T+Tq-1 cross tile boundaries of
+    # the visible entry counts inside a group
+    wl = W.get("parity_prefill").with_(B=B, T=T, Tq=Tq, k=k)
+    L = W.make_csa_layer(wl)
+    Ld = to_device(L)
+    layer = _run_indexer(C, Ld)
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_indexer_topk(L, wl.k, rows=rows)
+    idx = layer.idx.cpu().numpy()
+    sc = layer.score.cpu().numpy()
+    for (b, t), (ridx, rs) in ref.items():
+        check_topk(idx[b, t], ridx, rs, where=f"B={B} T={T} Tq={Tq} row {(b, t)}")
+        sel = idx[b, t][idx[b, t] >= 0]
+        assert np.allclose(sc[b, t][: sel.size], rs[sel], rtol=1e-4, atol=1e-4 * np.abs(rs).max())
+
+
 @pytest.mark.parametrize("name", ["tiny", "parity_decode"])
 def test_indexer_score_then_select_is_indexer_topk(C, name):
     # the two halves called in turn give indexer_topk's results bit for bit
