@@ -630,6 +630,8 @@ def run_prefill(args, rank, world, dev):
     indexer scoring's tensor FLOP rate against the FP8 peak."""
     from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
     wl = W.get(args.workload).with_(ik_fmt=args.ik_fmt)
+    if args.tq:
+        wl = wl.with_(Tq=args.tq)
     torch.cuda.set_device(dev)
     csa = CSALayer(W.make_csa_layer(wl, device=dev, seed=1000 + 7919 * rank))
     hca = HCALayer(W.make_hca_layer(wl, device=dev, seed=501000 + 7919 * rank))
@@ -689,8 +691,8 @@ def run_prefill(args, rank, world, dev):
     fp8_peak = 2.0 * peak            # the nominal FP8 : BF16 dense ratio
     idx_tflops = idx_flop / (calls_ms["indexer_score"] / 1e3) / 1e12
     tokens = wl.B * wl.Tq * world
-    res = {"metric": "chunked-prefill tokens/s (CSA+HCA layers, 8,192 new tokens on a "
-                     "1,048,576-token context)",
+    res = {"metric": f"chunked-prefill tokens/s (CSA+HCA layers, {wl.Tq:,} new tokens on a "
+                     f"{wl.T:,}-token context)",
            "value": round(tokens / (ms / 1e3), 2), "unit": "tokens/s", "n_gpus": world,
            "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3/bf16 storage, fp32 math",
@@ -732,6 +734,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ik-fmt", default="e4m3vec", choices=["e4m3vec", "e4m3"],
                     help="FP8 indexer scale layout: one scale per vector, or per 64 dims")
+    ap.add_argument("--tq", type=int, default=0,
+                    help="prefill: new tokens per sequence (0: the workload's chunk); a "
+                         "shorter chunk is a smaller case of the same step, for profiling")
     ap.add_argument("--alt-steps", type=int, default=4096,
                     help="steps timed with the other indexer layout (0: skip)")
     args = ap.parse_args()

@@ -301,6 +301,9 @@ topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *
                       out_score ? out_score + (long long)row * k : nullptr);
 }
 
+// kDeep: slices longer than one pass (a CTA per row of a long chunk); the
+// next two passes' scores are then requested while one is counted
+template <bool kDeep>
 __global__ void __launch_bounds__(kSelThreads, 1)
 topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int stride,
                    long long max_entries, int k, int32_t *__restrict__ out_idx,
@@ -357,20 +360,24 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   uint32_t *ctr = w.ctr + (size_t)row * 4;
   uint64_t *candrow = w.cand + (size_t)row * kCandCap;
   int wins = 0;
-  // rows longer than one pass (few rows per launch, or a CTA per row): the
-  // next two passes' scores are requested while this one is counted
   float v[kSelPer], p1[kSelPer], p2[kSelPer];
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
-  if (j_lo + kSelChunk < j_hi) load8(s, j_lo + kSelChunk + (long long)tid * kSelPer, j_hi, p1);
-  if (j_lo + 2 * kSelChunk < j_hi)
-    load8(s, j_lo + 2 * kSelChunk + (long long)tid * kSelPer, j_hi, p2);
+  if (kDeep) {
+    if (j_lo + kSelChunk < j_hi) load8(s, j_lo + kSelChunk + (long long)tid * kSelPer, j_hi, p1);
+    if (j_lo + 2 * kSelChunk < j_hi)
+      load8(s, j_lo + 2 * kSelChunk + (long long)tid * kSelPer, j_hi, p2);
+  }
   for (long long c0 = j_lo; c0 < j_hi; c0 += kSelChunk) {
     const long long j0 = c0 + (long long)tid * kSelPer;
     if (c0 != j_lo) {
+      if (kDeep) {
 #pragma unroll
-      for (int e = 0; e < kSelPer; ++e) { v[e] = p1[e]; p1[e] = p2[e]; }
-      if (c0 + 2 * kSelChunk < j_hi) load8(s, j0 + 2 * kSelChunk, j_hi, p2);
+        for (int e = 0; e < kSelPer; ++e) { v[e] = p1[e]; p1[e] = p2[e]; }
+        if (c0 + 2 * kSelChunk < j_hi) load8(s, j0 + 2 * kSelChunk, j_hi, p2);
+      } else {
+        load8(s, j0, j_hi, v);
+      }
     }
     int nc = 0;
     uint32_t cmask = 0;
@@ -581,15 +588,21 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     int base = sm.base;
 #pragma unroll
     for (int e = 0; e < kSelPer; ++e) v[e] = keep[e];
-    if (j_lo + kSelChunk < j_hi) load8(s, j_lo + kSelChunk + (long long)tid * kSelPer, j_hi, p1);
-    if (j_lo + 2 * kSelChunk < j_hi)
-      load8(s, j_lo + 2 * kSelChunk + (long long)tid * kSelPer, j_hi, p2);
+    if (kDeep) {
+      if (j_lo + kSelChunk < j_hi) load8(s, j_lo + kSelChunk + (long long)tid * kSelPer, j_hi, p1);
+      if (j_lo + 2 * kSelChunk < j_hi)
+        load8(s, j_lo + 2 * kSelChunk + (long long)tid * kSelPer, j_hi, p2);
+    }
     for (long long c0 = j_lo; c0 < j_hi; c0 += kSelChunk) {
       const long long j0 = c0 + (long long)tid * kSelPer;
       if (c0 != j_lo) {
+        if (kDeep) {
 #pragma unroll
-        for (int e = 0; e < kSelPer; ++e) { v[e] = p1[e]; p1[e] = p2[e]; }
-        if (c0 + 2 * kSelChunk < j_hi) load8(s, j0 + 2 * kSelChunk, j_hi, p2);
+          for (int e = 0; e < kSelPer; ++e) { v[e] = p1[e]; p1[e] = p2[e]; }
+          if (c0 + 2 * kSelChunk < j_hi) load8(s, j0 + 2 * kSelChunk, j_hi, p2);
+        } else {
+          load8(s, j0, j_hi, v);
+        }
       }
       uint32_t fl = 0;
 #pragma unroll
@@ -631,7 +644,6 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
                        float *out_score, cudaStream_t st) {
   if (k > kMaxK) return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(SelSmem);
-  if (!ensure_dynamic_smem(topk_select_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -643,8 +655,11 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
   if (splits > cap) splits = cap;
   if (splits > kMaxSplits) splits = kMaxSplits;
   if (splits < 1) splits = 1;
-  launch_pdl(topk_select_kernel, dim3((unsigned)splits, (unsigned)rows), dim3(kSelThreads), smem,
-             st, w, q_pos, stride, max_entries, k, out_idx, out_score);
+  const long long per = ((max_entries + splits - 1) / splits + kSelPer - 1) / kSelPer * kSelPer;
+  auto kernel = per > kSelChunk ? topk_select_kernel<true> : topk_select_kernel<false>;
+  if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+  launch_pdl(kernel, dim3((unsigned)splits, (unsigned)rows), dim3(kSelThreads), smem, st, w,
+             q_pos, stride, max_entries, k, out_idx, out_score);
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 
