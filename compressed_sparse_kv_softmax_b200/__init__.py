@@ -127,9 +127,11 @@ def attn_workspace_size(B, Tq, Hq, Dv, max_entries, window) -> int:
 
 
 def workspace(nbytes: int, device="cuda"):
-    """A 256-byte-aligned uint8 device buffer of at least nbytes."""
+    """A zero-filled uint8 device buffer with at least nbytes past its first
+    256-byte boundary (zero-filled so that the first indexer call already
+    finds a clean score histogram)."""
     import torch
-    return torch.empty(max(int(nbytes), 1) + 256, dtype=torch.uint8, device=device)
+    return torch.zeros(max(int(nbytes), 1) + 256, dtype=torch.uint8, device=device)
 
 
 def _ws(ws):

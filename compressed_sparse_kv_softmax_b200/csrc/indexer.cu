@@ -24,9 +24,9 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
                        float *out_score, cudaStream_t st);
 bool indexer_tc_supported(const IndexerArgs &a);
 int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                      int *err, cudaStream_t st);
+                      uint32_t *ctr, int *err, cudaStream_t st);
 int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                        int *err, cudaStream_t st);
+                        uint32_t *ctr, int *err, cudaStream_t st);
 
 namespace {
 
@@ -82,15 +82,6 @@ indexer_score_kernel(IndexerArgs a, float *__restrict__ scores, long long ld) {
   scores[(long long)row * ld + j] = s;
 }
 
-// zeroes n 32-bit words (the histogram and counters of the selection)
-__global__ void __launch_bounds__(256) zero_words_kernel(uint32_t *__restrict__ p, long long n) {
-  pdl_wait();
-  pdl_trigger();
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x)
-    p[i] = 0u;
-}
-
 }  // namespace
 
 size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k) {
@@ -105,17 +96,19 @@ int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st) {
   const IndexerWs w = indexer_ws_layout(a.ws, rows, a.max_entries, a.k, nullptr);
   const bool score = phases & kIndexerScore, select = phases & kIndexerSelect;
   if (a.max_entries > 0 && indexer_tc_supported(a)) {
-    // tensor-core scoring builds the score histogram the multi-CTA selection uses
+    // tensor-core scoring builds the score histogram the multi-CTA selection
+    // uses.  The histogram only guides the selection (every count it implies
+    // is checked against the scores, and a row whose counts disagree is
+    // selected from its scores alone), so it is not cleared before the call:
+    // the selection clears each row's histogram once it has read it, and a
+    // fresh workspace's first call at worst takes the slower path.  The
+    // scoring kernel clears the selection's counters.
     if (score) {
-      const long long words = (long long)(w.zero_bytes / 4);
-      long long blocks = (words + 255) / 256;
-      if (blocks > 1184) blocks = 1184;
-      if (launch_pdl(zero_words_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
-                     reinterpret_cast<uint32_t *>(w.err), words) != cudaSuccess)
-        return CSKV_ERR_CUDA;
       // several query rows per sequence share each key tile; one row streams alone
-      int rc = launch_indexer_rows(a, w.scores, w.ld, w.hist, w.err, st);
-      if (rc == CSKV_ERR_UNSUPPORTED) rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.err, st);
+      int rc = launch_indexer_rows(a, w.scores, w.ld, w.hist, w.ctr,
+                                   w.err, st);
+      if (rc == CSKV_ERR_UNSUPPORTED)
+        rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.ctr, w.err, st);
       if (rc != CSKV_OK) return rc;
     }
     if (!select) return CSKV_OK;

@@ -89,7 +89,7 @@ template <bool kVec>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                   float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
-                  int *__restrict__ err) {
+                  uint32_t *__restrict__ ctr, int *__restrict__ err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem &sm = *reinterpret_cast<Smem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,6 +125,10 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   const uint32_t tmem = sm.tmem_base;
   pdl_wait();                      // global memory from here on
   pdl_trigger();
+  // the selection's per-row counters start at zero (the selection runs after
+  // this grid); the row's score histogram was zeroed by the last selection
+  if (blockIdx.x == 0 && tid < 4) ctr[(size_t)row * 4 + tid] = 0u;
+  if (blockIdx.x == 0 && row == 0 && tid == 0) *err = 0;
   const long long qpos = a.q_pos[row];
   // tiles of this CTA for n visible entries (tile t goes to CTA t % grid)
   auto tiles_of = [&](long long nn) {
@@ -465,7 +469,7 @@ bool make_key_tmap(const IndexerArgs &a, CUtensorMap *map) {
 }
 
 int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                      int *err, cudaStream_t st) {
+                      uint32_t *ctr, int *err, cudaStream_t st) {
   CUtensorMap map;
   if (!make_key_tmap(a, &map)) return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(Smem) + 1024;
@@ -481,7 +485,7 @@ int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_
   if (splits > tiles) splits = tiles;
   if (splits < 1) splits = 1;
   dim3 grid((unsigned)splits, (unsigned)rows);
-  return launch_pdl(kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist, err) ==
+  return launch_pdl(kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist, ctr, err) ==
                  cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;

@@ -117,7 +117,7 @@ __device__ __forceinline__ float2 row_part(const float (&v)[32], const float *c1
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                     float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
-                    int *__restrict__ err, int groups_per_seq) {
+                    uint32_t *__restrict__ ctr, int *__restrict__ err, int groups_per_seq) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   RowsSmem &sm = *reinterpret_cast<RowsSmem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -154,6 +154,10 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
   const uint32_t tmem = sm.tmem_base;
   pdl_wait();                      // global memory from here on
   pdl_trigger();
+  // the selection's per-row counters start at zero (the selection runs after
+  // this grid); the rows' score histograms were zeroed by the last selection
+  if (blockIdx.x == 0 && tid < nrows * 4) ctr[(size_t)row0 * 4 + tid] = 0u;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *err = 0;
 
   // tiles of this CTA for n entries (tile t goes to split t % gridDim.x)
   auto tiles_of = [&](long long nn) {
@@ -389,7 +393,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
 // per-vector scale layout; returns CSKV_ERR_UNSUPPORTED, before launching
 // anything, where the grid does not fit.
 int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                        int *err, cudaStream_t st) {
+                        uint32_t *ctr, int *err, cudaStream_t st) {
   if (a.ik.fmt != CSKV_FMT_E4M3_VEC || a.Tq < 2) return CSKV_ERR_UNSUPPORTED;
   const int gps = (a.Tq + kRows - 1) / kRows;
   const long long groups = (long long)a.B * gps;
@@ -410,7 +414,7 @@ int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint3
   if (splits < 1) splits = 1;
   dim3 grid((unsigned)splits, (unsigned)groups);
   return launch_pdl(indexer_rows_kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld,
-                    hist, err, gps) == cudaSuccess
+                    hist, ctr, err, gps) == cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;
 }

@@ -336,12 +336,17 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   if (n > max_entries) n = max_entries;
   if (n < 0) n = 0;
 
+  // the row's histogram is cleared for the next scoring call once every CTA
+  // of the row has read it (here, or past the row barrier below)
+  uint4 *hclear = reinterpret_cast<uint4 *>(w.hist + (size_t)row * kTopkBins);
   if (n <= k) {            // every visible entry is selected, already in order
     if (me == 0) {
       for (int i = tid; i < k; i += blockDim.x) {
         oi[i] = i < n ? i : -1;
         if (os) os[i] = i < n ? s[i] : -__int_as_float(0x7f800000);
       }
+      // (the histogram is not read on this path)
+      for (int i = tid; i < kTopkBins / 4; i += blockDim.x) hclear[i] = make_uint4(0, 0, 0, 0);
     }
     return;
   }
@@ -433,6 +438,10 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     sm.n_cand = (int)ld_acquire_u32(&ctr[0]);
   }
   __syncthreads();
+  // every CTA of the row has read the histogram before arriving (a CTA that
+  // gave up waiting selects from the scores alone)
+  if (me == 0)
+    for (int i = tid; i < kTopkBins / 4; i += blockDim.x) hclear[i] = make_uint4(0, 0, 0, 0);
   const int n_cand = sm.n_cand;
   const int r = k - above;             // candidates still to take
   bool fallback = sm.state != 0 || above < 0 || above >= k || r < 1 || r > n_cand ||

@@ -17,9 +17,13 @@ constexpr int kMaxSplits = 256;
 
 // Indexer workspace layout, one section after another, each 256-byte aligned:
 //   scores   rows x ld fp32
-//   err      4 int                 device status words (zeroed before scoring)
-//   hist     rows x kTopkBins u32  (zeroed before scoring)
-//   ctr      rows x 4 u32          candidate count, barrier arrivals (zeroed)
+//   err      4 int                 device status words (cleared by the scoring kernel)
+//   hist     rows x kTopkBins u32  score histogram: built by the scoring kernel,
+//                                  cleared by the selection once read (it only
+//                                  guides the selection: a stale one costs time,
+//                                  not correctness)
+//   ctr      rows x 4 u32          candidate count, barrier arrivals (cleared by
+//                                  the scoring kernel)
 //   wins     rows x kMaxSplits u32 entries above the threshold bucket per CTA
 //   cand     rows x kCandCap u64   entries inside the threshold bucket, (index << 32) | key
 struct IndexerWs {
@@ -30,7 +34,7 @@ struct IndexerWs {
   uint32_t *wins;
   uint64_t *cand;
   long long ld;
-  size_t zero_bytes;   // bytes from `err` that must be zero before the call
+  size_t zero_bytes;   // bytes from `err` to the end of `ctr`
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

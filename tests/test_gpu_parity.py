@@ -149,6 +149,40 @@ def test_indexer_score_then_select_is_indexer_topk(C, name):
     assert torch.equal(whole.score, split.score)
 
 
+@pytest.mark.parametrize("how", ["random_workspace", "scored_twice"])
+@pytest.mark.parametrize("name", ["parity_decode", "parity_prefill"])
+def test_indexer_exact_with_stale_histogram(C, name, how):
+    # the score histogram only guides the selection: a workspace holding
+    # random bytes, or a histogram filled twice (indexer_score called twice
+    # before indexer_select), must still give the exact top-k
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    wl = W.get(name)
+    L = W.make_csa_layer(wl)
+    Ld = to_device(L)
+    layer = CSALayer(Ld)
+    if how == "random_workspace":
+        g = torch.Generator(device="cuda").manual_seed(5)
+        layer.ws_idx.copy_(torch.randint(0, 256, layer.ws_idx.shape, generator=g,
+                                         device="cuda", dtype=torch.int32).to(torch.uint8))
+        layer.select()
+    else:
+        layer.select(phase="score")
+        layer.select(phase="score")
+        layer.select(phase="pick")
+    torch.cuda.synchronize()
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_indexer_topk(L, wl.k, rows=rows)
+    idx = layer.idx.cpu().numpy()
+    for (b, t), (ridx, rs) in ref.items():
+        check_topk(idx[b, t], ridx, rs, where=f"{name} {how} row {(b, t)}")
+    # the selection left a clean histogram: the next call takes the fast path
+    # and agrees with this one
+    first = layer.idx.clone()
+    layer.select()
+    torch.cuda.synchronize()
+    assert torch.equal(first, layer.idx)
+
+
 @pytest.mark.parametrize("T,k,ik_fmt", [(3, 8, "e4m3vec"), (4, 8, "e4m3vec"), (64, 16, "e4m3vec"),
                                         (64, 100, "e4m3vec"), (517, 129, "e4m3vec"),
                                         (1000, 100, "e4m3vec"), (2100, 500, "e4m3vec"),
@@ -257,6 +291,35 @@ def test_hca_dense_attention(C, name):
     got_l = np.stack([lse[b, t].cpu().numpy() for b, t in rows])
     check_attention(got_o, got_l, np.stack([ref[r][0] for r in rows]),
                     np.stack([ref[r][1] for r in rows]), where=name)
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_decode_attention_repeated_calls_one_workspace(C, kind):
+    # several decode calls in a row on one layer (one workspace, partials of
+    # the previous call still in it), each with new queries, each match the
+    # oracle
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
+    wl = W.get("parity_decode")
+    L = (W.make_csa_layer if kind == "csa" else W.make_hca_layer)(wl)
+    Ld = to_device(L)
+    sel = _sel_from_oracle(L, wl.k) if kind == "csa" else None
+    layer = CSALayer(Ld) if kind == "csa" else HCALayer(Ld)
+    rng = np.random.default_rng(123)
+    rows = sample_rows(wl.B, wl.Tq)
+    for call in range(3):
+        q = torch.from_numpy(rng.standard_normal(L["q"].shape).astype(np.float32)).to(L["q"].dtype)
+        L["q"] = q
+        Ld["q"].copy_(q.to(Ld["q"].device))
+        if kind == "csa":
+            out, lse = layer.attend(torch.from_numpy(sel).cuda())
+        else:
+            out, lse = layer.attend()
+        torch.cuda.synchronize()
+        ref = O.layer_attention(L, sel=sel, rows=rows)
+        got_o = np.stack([out[b, t].cpu().numpy() for b, t in rows])
+        got_l = np.stack([lse[b, t].cpu().numpy() for b, t in rows])
+        check_attention(got_o, got_l, np.stack([ref[r][0] for r in rows]),
+                        np.stack([ref[r][1] for r in rows]), where=f"{kind} call {call}")
 
 
 @pytest.mark.parametrize("T", [1, 2, 77, 128, 129, 300])
