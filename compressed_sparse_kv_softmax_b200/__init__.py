@@ -91,9 +91,10 @@ def cache_struct(c):
     """C descriptor for a cache given as a dict of planes
     {"fmt": "f32"|"e4m3"|"e4m3vec", "d_nope", "d_rope", "ring", "cap", "data", "scale",
     "rope"}
-    (or None)."""
-    if c is None:
-        return None
+    (or None).  A CskvCache is returned as it is: callers that pass the same
+    cache every step can build its descriptor once."""
+    if c is None or isinstance(c, CskvCache):
+        return c
     s = CskvCache()
     s.fmt = _FMT[c["fmt"]]
     s.d_nope, s.d_rope = int(c["d_nope"]), int(c["d_rope"])
@@ -109,6 +110,10 @@ def cache_struct(c):
 
 def _ref(s):
     return None if s is None else ctypes.byref(s)
+
+
+def _ikref(c):
+    return ctypes.byref(cache_struct(c))
 
 
 def _stream(stream):
@@ -160,10 +165,9 @@ def hca_compress(B, t_begin, t_end, max_new, raw_k, raw_v, gate_w, gate_b, pool,
 
 def indexer_topk(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
                  out_idx, out_score, ws, stream=None):
-    c = cache_struct(ik)
     wp, wn = _ws(ws)
     _check(_lib.indexer_topk(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
-                             H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
+                             H_I, d_I, _ikref(ik), stride, k, int(max_entries),
                              _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
            "indexer_topk")
 
@@ -171,10 +175,9 @@ def indexer_topk(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k
 def indexer_score(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
                   out_idx, out_score, ws, stream=None):
     """First half of indexer_topk: scores and histogram into the workspace."""
-    c = cache_struct(ik)
     wp, wn = _ws(ws)
     _check(_lib.indexer_score(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
-                              H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
+                              H_I, d_I, _ikref(ik), stride, k, int(max_entries),
                               _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
            "indexer_score")
 
@@ -182,10 +185,9 @@ def indexer_score(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, 
 def indexer_select(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
                    out_idx, out_score, ws, stream=None):
     """Second half of indexer_topk: the top-k from the workspace's scores."""
-    c = cache_struct(ik)
     wp, wn = _ws(ws)
     _check(_lib.indexer_select(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
-                               H_I, d_I, ctypes.byref(c), stride, k, int(max_entries),
+                               H_I, d_I, _ikref(ik), stride, k, int(max_entries),
                                _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
            "indexer_select")
 
@@ -195,9 +197,8 @@ def indexer_topk_noalloc(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, s
     """indexer_topk without a workspace, for callers that cannot allocate one:
     the library's fixed device scratch array is used instead (see cskv.h).
     Calls that overlap on the GPU share that array and must be serialised."""
-    c = cache_struct(ik)
     _check(_lib.indexer_topk_noalloc(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale),
-                                     _ptr(head_w), H_I, d_I, ctypes.byref(c), stride, k,
+                                     _ptr(head_w), H_I, d_I, _ikref(ik), stride, k,
                                      int(max_entries), _ptr(out_idx), _ptr(out_score),
                                      _stream(stream)), "indexer_topk_noalloc")
 

@@ -11,13 +11,21 @@ from __future__ import annotations
 
 import torch
 
-from . import (attn_workspace_size, csa_compress, hca_compress, hybrid_attn_decode,
-               hybrid_attn_prefill, indexer_score, indexer_select, indexer_topk,
-               indexer_workspace_size, workspace)
+from . import (attn_workspace_size, cache_struct, csa_compress, hca_compress,
+               hybrid_attn_decode, hybrid_attn_prefill, indexer_score, indexer_select,
+               indexer_topk, indexer_workspace_size, workspace)
 
 
 def _dims(c):
     return int(c["d_nope"]) + int(c["d_rope"])
+
+
+_CACHES = ("ring_k", "ring_v", "ring_ik", "comp_k", "comp_v", "comp_ik")
+
+
+def _descriptors(L):
+    """C descriptors of the layer's caches, built once (the planes do not move)."""
+    return {key: cache_struct(L.get(key)) for key in _CACHES}
 
 
 class CSALayer:
@@ -44,12 +52,13 @@ class CSALayer:
                                 dev)
         self.ws_attn = workspace(attn_workspace_size(self.B, self.Tq, self.Hq, self.Dv, self.k,
                                                      wl.window), dev)
+        self.cs = _descriptors(L)
 
     def compress(self, t_begin, t_end, max_new):
-        L = self.L
-        csa_compress(self.B, t_begin, t_end, max_new, L["ring_k"], L["ring_v"], L["ring_ik"],
-                     L["gate_w"], L["gate_b"], L["pool"], L["stride"], L["comp_k"], L["comp_v"],
-                     L["comp_ik"])
+        L, c = self.L, self.cs
+        csa_compress(self.B, t_begin, t_end, max_new, c["ring_k"], c["ring_v"], c["ring_ik"],
+                     L["gate_w"], L["gate_b"], L["pool"], L["stride"], c["comp_k"], c["comp_v"],
+                     c["comp_ik"])
 
     def select(self, q_pos=None, phase="both"):
         """indexer_topk; q_pos [B][Tq] (device) overrides the layer's positions.
@@ -58,23 +67,24 @@ class CSALayer:
         q_pos = L["q_pos"] if q_pos is None else q_pos
         fn = {"both": indexer_topk, "score": indexer_score, "pick": indexer_select}[phase]
         fn(self.B, self.Tq, q_pos, L["q_ik"], L["q_ik_scale"], L["head_w"], wl.H_I, wl.d_I,
-           L["comp_ik"], L["stride"], self.k, self.max_entries, self.idx, self.score, self.ws_idx)
+           self.cs["comp_ik"], L["stride"], self.k, self.max_entries, self.idx, self.score,
+           self.ws_idx)
         return self.idx
 
     def attend(self, sel=None, pos=None):
         """Hybrid attention over `sel` (default: the last selection); pos
         overrides q_pos (prefill) or ctx_len (decode)."""
-        L, wl = self.L, self.wl
+        L, wl, c = self.L, self.wl, self.cs
         sel = self.idx if sel is None else sel
         if wl.prefill:
             hybrid_attn_prefill(self.B, self.Tq, L["q_pos"] if pos is None else pos, L["q"],
-                                self.Hq, wl.sm_scale, L["comp_k"], L["comp_v"], L["stride"], sel,
-                                self.k, self.k, L["ring_k"], L["ring_v"], wl.window, self.out,
+                                self.Hq, wl.sm_scale, c["comp_k"], c["comp_v"], L["stride"], sel,
+                                self.k, self.k, c["ring_k"], c["ring_v"], wl.window, self.out,
                                 self.lse, self.ws_attn)
         else:
             hybrid_attn_decode(self.B, L["ctx_len"] if pos is None else pos, L["q"], self.Hq,
-                               wl.sm_scale, L["comp_k"], L["comp_v"], L["stride"], sel, self.k,
-                               self.k, L["ring_k"], L["ring_v"], wl.window, self.out, self.lse,
+                               wl.sm_scale, c["comp_k"], c["comp_v"], L["stride"], sel, self.k,
+                               self.k, c["ring_k"], c["ring_v"], wl.window, self.out, self.lse,
                                self.ws_attn)
         return self.out, self.lse
 
@@ -99,27 +109,28 @@ class HCALayer:
         self.ws_attn = workspace(attn_workspace_size(self.B, self.Tq, self.Hq, self.Dv,
                                                      self.max_entries if dense else 0,
                                                      wl.window), dev)
+        self.cs = _descriptors(L)
 
     def compress(self, t_begin, t_end, max_new):
-        L = self.L
-        hca_compress(self.B, t_begin, t_end, max_new, L["ring_k"], L["ring_v"], L["gate_w"],
-                     L["gate_b"], L["pool"], L["stride"], L["comp_k"], L["comp_v"])
+        L, c = self.L, self.cs
+        hca_compress(self.B, t_begin, t_end, max_new, c["ring_k"], c["ring_v"], L["gate_w"],
+                     L["gate_b"], L["pool"], L["stride"], c["comp_k"], c["comp_v"])
 
     def attend(self, pos=None):
         """Dense hybrid attention; pos overrides q_pos (prefill) or ctx_len (decode)."""
-        L, wl = self.L, self.wl
-        ck = L["comp_k"] if self.dense else None
-        cv = L["comp_v"] if self.dense else None
+        L, wl, c = self.L, self.wl, self.cs
+        ck = c["comp_k"] if self.dense else None
+        cv = c["comp_v"] if self.dense else None
         me = self.max_entries if self.dense else 0
         if wl.prefill:
             hybrid_attn_prefill(self.B, self.Tq, L["q_pos"] if pos is None else pos, L["q"],
                                 self.Hq, wl.sm_scale, ck, cv, L["stride"], None, 0, me,
-                                L["ring_k"], L["ring_v"], wl.window, self.out, self.lse,
+                                c["ring_k"], c["ring_v"], wl.window, self.out, self.lse,
                                 self.ws_attn)
         else:
             hybrid_attn_decode(self.B, L["ctx_len"] if pos is None else pos, L["q"], self.Hq,
-                               wl.sm_scale, ck, cv, L["stride"], None, 0, me, L["ring_k"],
-                               L["ring_v"], wl.window, self.out, self.lse, self.ws_attn)
+                               wl.sm_scale, ck, cv, L["stride"], None, 0, me, c["ring_k"],
+                               c["ring_v"], wl.window, self.out, self.lse, self.ws_attn)
         return self.out, self.lse
 
     step = attend
