@@ -53,6 +53,25 @@ UNIT = "queries/s"
 _FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def max_over_ranks(ms, dev, world):
+    """The slowest rank's time (every rank takes this collective step)."""
+    if world <= 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], device=dev, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, ms, world):
+    """Units of all ranks per second over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
+
+
+def rank_seed(base, rank):
+    """Each rank's replicas draw their own inputs (independent sequences)."""
+    return base + 7919 * rank
+
+
 def _peaks(kind="hbm_gbs"):
     """A measured peak from MEASURED_PEAKS.json (HBM copy GB/s, or cuBLAS bf16
     TFLOP/s as a burst or sustained), else the earlier measurement on this
@@ -300,7 +319,7 @@ def _time_decode(args, wl, rank, world, dev, steps, seed0, clocks=True):
     # enough replicas that one rotation touches > 4x the 126 MB L2 (unless set)
     R = args.replicas if args.replicas > 0 else math.ceil(4 * 126e6 / per_rep_bytes) + 1
     sched = Schedule(wl, dev)
-    replicas = [Replica(wl, sched, seed0 + r + 7919 * rank, dev) for r in range(R)]
+    replicas = [Replica(wl, sched, rank_seed(seed0 + r, rank), dev) for r in range(R)]
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
     # warm-up: W steps eagerly through the public API (also performs the
@@ -340,11 +359,7 @@ def _time_decode(args, wl, rank, world, dev, steps, seed0, clocks=True):
     if world > 1:
         torch.distributed.barrier()
     clk = sampler.stop() if sampler else None
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
     return {"ms": ms, "steps": n_launch * G + rest, "idx_ms": float(np.mean(graph.indexer_ms())),
             "clocks": clk, "replicas": replicas, "R": R, "sched": sched,
             "per_rep_bytes": per_rep_bytes,
@@ -380,8 +395,7 @@ def run_ours(args, rank, world, dev):
     t = _time_decode(args, wl, rank, world, dev, args.steps, 1000)
     replicas, R, sched, per_rep_bytes = t["replicas"], t["R"], t["sched"], t["per_rep_bytes"]
     ms, steps_done, idx_ms, clocks = t["ms"], t["steps"], t["idx_ms"], t["clocks"]
-    total_q = wl.B * steps_done * world
-    value = total_q / (ms / 1e3)
+    value = whole_job_rate(wl.B * steps_done, ms, world)
 
     peak, peak_kind = _peaks()
     ib = indexer_bytes(wl)
@@ -524,12 +538,8 @@ def run_e2e(args, replicas, wl, dev, world):
             one(i)
         e1.record(stream)
     stream.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(wl.B * K * world / (ms / 1e3), 2), "unit": UNIT,
+    ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
+    return {"value": round(whole_job_rate(wl.B * K, ms, world), 2), "unit": UNIT,
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "steps": K,
             "path": "eager public API calls (no graph), single replica, same decode window; "
                     "per step one copy of the small inputs, 8 ring-slot copies, one copy of "
@@ -664,8 +674,8 @@ def run_prefill(args, rank, world, dev):
     if args.tq:
         wl = wl.with_(Tq=args.tq)
     torch.cuda.set_device(dev)
-    csa = CSALayer(W.make_csa_layer(wl, device=dev, seed=1000 + 7919 * rank))
-    hca = HCALayer(W.make_hca_layer(wl, device=dev, seed=501000 + 7919 * rank))
+    csa = CSALayer(W.make_csa_layer(wl, device=dev, seed=rank_seed(1000, rank)))
+    hca = HCALayer(W.make_hca_layer(wl, device=dev, seed=rank_seed(501000, rank)))
     tb = torch.full((wl.B,), wl.T, dtype=torch.int64, device=dev)
     te = torch.full((wl.B,), wl.T + wl.Tq, dtype=torch.int64, device=dev)
     stream = torch.cuda.Stream(device=dev)
@@ -702,11 +712,8 @@ def run_prefill(args, rank, world, dev):
     torch.cuda.synchronize()
     clocks = sampler.stop()
     per_call = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(len(names))] for e in evs])
-    ms = float(sum(e[0].elapsed_time(e[-1]) for e in evs)) / K
+    ms = max_over_ranks(float(sum(e[0].elapsed_time(e[-1]) for e in evs)) / K, dev, world)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
         torch.distributed.barrier()
     calls_ms = {n: round(float(v), 4) for n, v in zip(names, per_call.mean(axis=0))}
     # FLOPs: visible entries differ per token of the chunk (causal)
@@ -721,10 +728,11 @@ def run_prefill(args, rank, world, dev):
     peak, peak_kind = _peaks(kind="bf16_tflops_sustained")
     fp8_peak = 2.0 * peak            # the nominal FP8 : BF16 dense ratio
     idx_tflops = idx_flop / (calls_ms["indexer_score"] / 1e3) / 1e12
-    tokens = wl.B * wl.Tq * world
+    tokens_per_rank = wl.B * wl.Tq
     res = {"metric": f"chunked-prefill tokens/s (CSA+HCA layers, {wl.Tq:,} new tokens on a "
                      f"{wl.T:,}-token context)",
-           "value": round(tokens / (ms / 1e3), 2), "unit": "tokens/s", "n_gpus": world,
+           "value": round(whole_job_rate(tokens_per_rank, ms, world), 2), "unit": "tokens/s",
+           "n_gpus": world,
            "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3/bf16 storage, fp32 math",
            "data": "synthetic (seeded Gaussian FP8 E4M3 + BF16 caches)",
