@@ -115,11 +115,13 @@ def test_indexer_topk(C, name, ik_fmt):
 
 
 @pytest.mark.parametrize("B,T,Tq,k", [(2, 508, 2, 16), (2, 508, 5, 64), (1, 3001, 8, 128),
-                                      (3, 1200, 13, 100), (1, 66_000, 9, 1024)])
+                                      (3, 1200, 13, 100), (1, 66_000, 9, 1024),
+                                      (1, 100_000, 200, 512)])
 def test_indexer_many_rows_per_sequence(C, B, T, Tq, k):
     # several query rows of a sequence share each key tile (groups of 8 rows,
     # the last group ragged); positions T .. T+Tq-1 cross tile boundaries of
-    # the visible entry counts inside a group
+    # the visible entry counts inside a group.  200 rows of 25,000 entries:
+    # one selection CTA per row, 7 passes with the next two always in flight
     wl = W.get("parity_prefill").with_(B=B, T=T, Tq=Tq, k=k)
     L = W.make_csa_layer(wl)
     Ld = to_device(L)
