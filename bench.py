@@ -176,22 +176,26 @@ class Replica:
         self.hca = HCALayer(self.hca_L)
         self.sched = sched
 
-    def step(self, s, mark=None, pos=None):
+    def step(self, s, mark=None, pos=None, split_select=True):
         """Enqueue decode step s of the window on the current stream; mark(i)
         records an event between calls (i = 0 before indexer_score, 1 after
-        it).  indexer_score + indexer_select is the indexer_topk call.  pos =
-        (q_pos, ctx_len, t_begin, t_end) device tensors replace the schedule's."""
+        it).  indexer_score + indexer_select is the indexer_topk call (one call
+        when split_select is False).  pos = (q_pos, ctx_len, t_begin, t_end)
+        device tensors replace the schedule's."""
         sc = self.sched
         q_pos, ctx, tb, te = pos if pos is not None else (sc.q_pos[s], sc.ctx[s], sc.tb[s],
                                                           sc.te[s])
         if sc.csa_fires[s]:
             self.csa.compress(tb, te, 1)
-        if mark:
-            mark(0)
-        self.csa.select(q_pos, phase="score")
-        if mark:
-            mark(1)
-        self.csa.select(q_pos, phase="pick")
+        if split_select:
+            if mark:
+                mark(0)
+            self.csa.select(q_pos, phase="score")
+            if mark:
+                mark(1)
+            self.csa.select(q_pos, phase="pick")
+        else:
+            self.csa.select(q_pos)
         self.csa.attend(pos=ctx)
         if sc.hca_fires[s]:
             self.hca.compress(tb, te, 1)
@@ -521,7 +525,7 @@ def run_e2e(args, replicas, wl, dev, world):
         dev_buf.copy_(host_small[s], non_blocking=True)
         for d, h in zip(dev_ring[s], host_ring[s]):
             d.copy_(h, non_blocking=True)
-        rep.step(s, pos=pos)
+        rep.step(s, pos=pos, split_select=False)
         host_out.copy_(out_buf, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -541,9 +545,10 @@ def run_e2e(args, replicas, wl, dev, world):
     ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
     return {"value": round(whole_job_rate(wl.B * K, ms, world), 2), "unit": UNIT,
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "steps": K,
-            "path": "eager public API calls (no graph), single replica, same decode window; "
-                    "per step one copy of the small inputs, 8 ring-slot copies, one copy of "
-                    "both layers' outputs"}
+            "path": "eager public API calls (no graph: csa_compress, indexer_topk, "
+                    "hybrid_attn_decode, hca_compress, hybrid_attn_decode), single replica, "
+                    "same decode window; per step one copy of the small inputs, 8 ring-slot "
+                    "copies, one copy of both layers' outputs"}
 
 
 # ------------------------------------------------------------- the oracle
