@@ -26,6 +26,7 @@ bool attn_tc_supported(const AttnArgs &a);
 int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *part_lse,
                    cudaStream_t st);
 int attn_tc_unit_keys(long long rows, long long keys);
+size_t attn_tc_tile_bytes(int B, int Tq, long long max_entries);
 
 namespace {
 
@@ -324,13 +325,16 @@ static size_t partial_bytes(const AttnPlan &p, long long rows, int Hq, int Dv) {
 }
 
 size_t attn_ws_bytes(int B, int Tq, int Hq, int Dv, long long max_entries, int window) {
-  // either path may run: the larger of the two plans
+  // either path may run: the larger of the two plans, or of the converted
+  // key tiles of a dense prefill (used only when a row has one split)
   const long long rows = (long long)B * Tq;
   const size_t a = partial_bytes(attn_plan(rows, max_entries, window, kChunk), rows, Hq, Dv);
   const size_t b = partial_bytes(
       attn_plan(rows, max_entries, window, attn_tc_unit_keys(rows, max_entries + window)), rows,
       Hq, Dv);
-  return a > b ? a : b;
+  const size_t t = attn_tc_tile_bytes(B, Tq, max_entries);
+  const size_t m = a > b ? a : b;
+  return m > t ? m : t;
 }
 
 int launch_attention(const AttnArgs &a, cudaStream_t st) {

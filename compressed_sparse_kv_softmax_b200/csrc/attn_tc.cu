@@ -76,7 +76,7 @@ struct __align__(1024) Smem {
   float red[4][kHeads];
   float m[kHeads], l[kHeads], inv_l[kHeads], alpha[kHeads];
   long long slot[kM];
-  uint64_t bar, gbar;
+  uint64_t bar, gbar, tbar;
   uint32_t tmem_base;
 };
 
@@ -310,9 +310,66 @@ __device__ __forceinline__ Row row_of(const AttnArgs &a, int row) {
   return r;
 }
 
+// Dense compressed entries in the key-tile layout of attn_tc_kernel: the
+// 64 entries of unit u of sequence b become the 128 KB tile [8 chunks of 64
+// dims][64 hi rows, 64 lo rows][128 B, 128-byte swizzle], converted once per
+// call for all query rows of a chunk.  Entries at or past the furthest row's
+// visible count are zero (cache slots past it may hold anything).
+__global__ void __launch_bounds__(kThreads)
+key_tiles_kernel(const AttnArgs a, uint8_t *__restrict__ tiles, int tile_units) {
+  __shared__ long long s_max[kThreads / 32];
+  pdl_wait();
+  pdl_trigger();
+  const int unit = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  long long nmax = 0;
+  for (int t = tid; t < a.Tq; t += kThreads) {
+    const long long n = (a.pos[(size_t)b * a.Tq + t] + 1) / a.comp_stride;
+    nmax = n > nmax ? n : nmax;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const long long y = __shfl_xor_sync(0xffffffffu, nmax, o);
+    nmax = y > nmax ? y : nmax;
+  }
+  if (lane == 0) s_max[warp] = nmax;
+  __syncthreads();
+  nmax = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) nmax = s_max[w] > nmax ? s_max[w] : nmax;
+  if (nmax > a.max_entries) nmax = a.max_entries;
+  if (nmax > a.comp_k.cap) nmax = a.comp_k.cap;
+  // warp w converts rows 8w .. 8w+7 (lane l: row l % 8, see convert_parts)
+  constexpr int rpw = kKeys / 8, lg = 3;
+  const int my_r = warp * rpw + (lane & (rpw - 1));
+  const long long j = (long long)unit * kKeys + my_r;
+  const bool live = j < nmax;
+  const Cache &src = a.comp_k;
+  RowParts p;
+#pragma unroll
+  for (int k = 0; k < kCodeIt; ++k) {
+    const int c = code_unit(lane, lg, k);
+    p.code[k] = make_uint4(0, 0, 0, 0);
+    p.sc[k] = 0.f;
+    if (live && c < kCodeUnits) {
+      p.code[k] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, j)) + c);
+      p.sc[k] = __ldg(src.scale_ptr(b, j) + (c >> 2));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kRopeIt; ++k) {
+    const int v = code_unit(lane, lg, k);
+    p.rope[k] = make_uint4(0, 0, 0, 0);
+    if (live && v < kRopeUnits)
+      p.rope[k] = __ldg(reinterpret_cast<const uint4 *>(src.rope_ptr(b, j)) + v);
+  }
+  convert_parts(tiles + ((size_t)b * tile_units + unit) * (8 * kChunkKK), p, my_r, lane, lg);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, int units_per_cta,
-               int n_splits, float *__restrict__ part_o, float *__restrict__ part_lse) {
+               int n_splits, float *__restrict__ part_o, float *__restrict__ part_lse,
+               const uint8_t *__restrict__ tiles, int tile_units) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
@@ -323,6 +380,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
   if (tid == 0) {
     mbar_init(&sm.bar, 1);
     mbar_init(&sm.gbar, 1);
+    mbar_init(&sm.tbar, 1);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -343,6 +401,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
   const uint32_t tmem_tl = ((uint32_t)(quad * 32) << 16);
   const float c2 = a.sm_scale * 1.4426950408889634f;   // logits in log2 units
   uint32_t phase = 0;                               // parity of the next completion of sm.bar
+  uint32_t tphase = 0;                              // same for sm.tbar (converted key tiles)
   bool started = false;                             // O^T in TMEM holds a partial sum
   bool ok = true;
   bool q_ready = false;                             // Q staged in shared memory
@@ -387,7 +446,22 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     // consecutive slots: the window's positions (one or two runs around the
     // ring) or dense compressed entries (one run)
     const bool runs_ok = !q_ready && dense_rows(src) && !(comp_unit && a.sel);
-    if (runs_ok) {
+    if (tiles && comp_unit) {
+      // dense entries converted once for every row of the call: the unit's
+      // key tile arrives whole by bulk copies (the previous unit's MMAs, the
+      // last readers of sm.kt, completed before this point)
+      if (tid == 0) {
+        const uint8_t *t = tiles + ((size_t)b * tile_units + unit) * (8 * kChunkKK);
+        mbar_arrive_expect_tx(&sm.tbar, 8 * kChunkKK);
+        for (int c = 0; c < 8; ++c) bulk_load(sm.kt + c * kChunkKK, t + c * kChunkKK, kChunkKK, &sm.tbar);
+      }
+      if (!q_ready) {
+        stage_q(qg, sm.q);
+        q_ready = true;
+      }
+      ok = mbar_wait(&sm.tbar, tphase) && ok;
+      tphase ^= 1;
+    } else if (runs_ok) {
       // first unit: bulk copies bring the rows into the still unused Q buffer
       // while Q itself is loaded into registers; the rows are converted from
       // shared memory, then Q takes its buffer
@@ -676,14 +750,33 @@ int attn_tc_unit_keys(long long rows, long long keys) {
   return kKeys;
 }
 
+// Bytes of converted key tiles for dense prefill rows (0 when not used).
+size_t attn_tc_tile_bytes(int B, int Tq, long long max_entries) {
+  if (Tq < 2 || max_entries <= 0) return 0;
+  return (size_t)B * (size_t)((max_entries + kKeys - 1) / kKeys) * (8 * kChunkKK);
+}
+
 int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *part_lse,
                    cudaStream_t st) {
   const size_t smem = sizeof(Smem) + 1024;
   if (!ensure_dynamic_smem(attn_tc_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   const int rows = a.B * a.Tq;
+  // dense entries shared by many query rows of a sequence (chunked prefill,
+  // one split per row): convert them once into the workspace
+  const uint8_t *tiles = nullptr;
+  int tile_units = 0;
+  const size_t tb = attn_tc_tile_bytes(a.B, a.Tq, a.max_entries);
+  if (a.has_comp && !a.sel && p.splits == 1 && p.unit == kKeys && tb && a.ws &&
+      a.ws_bytes >= tb && !((uintptr_t)a.ws & 127)) {
+    tile_units = (int)((a.max_entries + kKeys - 1) / kKeys);
+    if (launch_pdl(key_tiles_kernel, dim3((unsigned)tile_units, (unsigned)a.B), dim3(kThreads), 0,
+                   st, a, reinterpret_cast<uint8_t *>(a.ws), tile_units) != cudaSuccess)
+      return CSKV_ERR_CUDA;
+    tiles = reinterpret_cast<const uint8_t *>(a.ws);
+  }
   return launch_pdl(attn_tc_kernel, dim3((unsigned)rows, (unsigned)p.splits), dim3(kThreads),
                     smem, st, a, p.unit, p.n_comp_units, p.n_units, p.per_cta, p.splits, part_o,
-                    part_lse) == cudaSuccess
+                    part_lse, tiles, tile_units) == cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;
 }

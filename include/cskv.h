@@ -246,6 +246,9 @@ int hybrid_attn_decode(int B, const int64_t *ctx_len, const void *q, int Hq, flo
  * the chunk.  Same definition and layouts as hybrid_attn_decode with a Tq
  * axis: q [B][Tq][Hq][D], sel [B][Tq][k], out [B][Tq][Hq][Dv], lse [B][Tq][Hq].
  * The ring must hold every position the chunk's windows reach.
+ * With comp_k dense (sel == NULL) and several rows per sequence, the call
+ * first converts the visible compressed entries once into the workspace
+ * (cskv_attn_workspace_size with Tq > 1 includes that space).
  */
 int hybrid_attn_prefill(int B, int Tq, const int64_t *q_pos, const void *q, int Hq,
                         float sm_scale, const cskv_cache *comp_k, const cskv_cache *comp_v,
