@@ -366,6 +366,9 @@ key_tiles_kernel(const AttnArgs a, uint8_t *__restrict__ tiles, int tile_units) 
   convert_parts(tiles + ((size_t)b * tile_units + unit) * (8 * kChunkKK), p, my_r, lane, lg);
 }
 
+// kTiles: dense entries come as pre-converted key tiles (chunked prefill);
+// a separate instantiation keeps that path out of the decode kernel's code.
+template <bool kTiles>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, int units_per_cta,
                int n_splits, float *__restrict__ part_o, float *__restrict__ part_lse,
@@ -401,7 +404,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
   const uint32_t tmem_tl = ((uint32_t)(quad * 32) << 16);
   const float c2 = a.sm_scale * 1.4426950408889634f;   // logits in log2 units
   uint32_t phase = 0;                               // parity of the next completion of sm.bar
-  uint32_t tphase = 0;                              // same for sm.tbar (converted key tiles)
+  uint32_t tphase = 0;                              // same for sm.tbar (kTiles)
   bool started = false;                             // O^T in TMEM holds a partial sum
   bool ok = true;
   bool q_ready = false;                             // Q staged in shared memory
@@ -446,7 +449,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
     // consecutive slots: the window's positions (one or two runs around the
     // ring) or dense compressed entries (one run)
     const bool runs_ok = !q_ready && dense_rows(src) && !(comp_unit && a.sel);
-    if (tiles && comp_unit) {
+    if (kTiles && comp_unit) {
       // dense entries converted once for every row of the call: the unit's
       // key tile arrives whole by bulk copies (the previous unit's MMAs, the
       // last readers of sm.kt, completed before this point)
@@ -759,24 +762,26 @@ size_t attn_tc_tile_bytes(int B, int Tq, long long max_entries) {
 int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *part_lse,
                    cudaStream_t st) {
   const size_t smem = sizeof(Smem) + 1024;
-  if (!ensure_dynamic_smem(attn_tc_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   const int rows = a.B * a.Tq;
   // dense entries shared by many query rows of a sequence (chunked prefill,
   // one split per row): convert them once into the workspace
+  const size_t tb = attn_tc_tile_bytes(a.B, a.Tq, a.max_entries);
+  const bool use_tiles = a.has_comp && !a.sel && p.splits == 1 && p.unit == kKeys && tb &&
+                         a.ws && a.ws_bytes >= tb && !((uintptr_t)a.ws & 127);
+  auto kernel = use_tiles ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   const uint8_t *tiles = nullptr;
   int tile_units = 0;
-  const size_t tb = attn_tc_tile_bytes(a.B, a.Tq, a.max_entries);
-  if (a.has_comp && !a.sel && p.splits == 1 && p.unit == kKeys && tb && a.ws &&
-      a.ws_bytes >= tb && !((uintptr_t)a.ws & 127)) {
+  if (use_tiles) {
     tile_units = (int)((a.max_entries + kKeys - 1) / kKeys);
     if (launch_pdl(key_tiles_kernel, dim3((unsigned)tile_units, (unsigned)a.B), dim3(kThreads), 0,
                    st, a, reinterpret_cast<uint8_t *>(a.ws), tile_units) != cudaSuccess)
       return CSKV_ERR_CUDA;
     tiles = reinterpret_cast<const uint8_t *>(a.ws);
   }
-  return launch_pdl(attn_tc_kernel, dim3((unsigned)rows, (unsigned)p.splits), dim3(kThreads),
-                    smem, st, a, p.unit, p.n_comp_units, p.n_units, p.per_cta, p.splits, part_o,
-                    part_lse, tiles, tile_units) == cudaSuccess
+  return launch_pdl(kernel, dim3((unsigned)rows, (unsigned)p.splits), dim3(kThreads), smem, st, a,
+                    p.unit, p.n_comp_units, p.n_units, p.per_cta, p.splits, part_o, part_lse,
+                    tiles, tile_units) == cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;
 }
