@@ -367,8 +367,10 @@ key_tiles_kernel(const AttnArgs a, uint8_t *__restrict__ tiles, int tile_units) 
 }
 
 // kTiles: dense entries come as pre-converted key tiles (chunked prefill);
-// a separate instantiation keeps that path out of the decode kernel's code.
-template <bool kTiles>
+// kMulti: a CTA runs several units (the running output may need rescaling).
+// Separate instantiations keep those paths out of the decode kernel's code
+// (one unit per CTA, gathered or bulk-copied rows).
+template <bool kTiles, bool kMulti>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, int units_per_cta,
                int n_splits, float *__restrict__ part_o, float *__restrict__ part_lse,
@@ -635,7 +637,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
       if (!(lane & 1)) sm.red[quad & 1][h0 + (lane >> 1)] = sum;
     }
     // ---- rescale the running O^T where a head's max moved (rare)
-    if (started) {
+    if (kMulti && started) {
       bool need = false;
       float al[32];
 #pragma unroll
@@ -768,7 +770,8 @@ int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *p
   const size_t tb = attn_tc_tile_bytes(a.B, a.Tq, a.max_entries);
   const bool use_tiles = a.has_comp && !a.sel && p.splits == 1 && p.unit == kKeys && tb &&
                          a.ws && a.ws_bytes >= tb && !((uintptr_t)a.ws & 127);
-  auto kernel = use_tiles ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  auto kernel = use_tiles ? attn_tc_kernel<true, true>
+                          : (p.per_cta > 1 ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>);
   if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   const uint8_t *tiles = nullptr;
   int tile_units = 0;
