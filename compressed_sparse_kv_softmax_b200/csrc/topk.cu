@@ -269,6 +269,7 @@ struct SelSmem {
   int cnt[kMaxSplits];        // selected entries per slice of the row
   int scan[33];
   int bstar, above, thr_bin, take, n_eq, state, n_cand, base, total, wins;
+  unsigned solo_cand;         // candidate count when one CTA owns the row
   uint32_t tie_cut, thr_full;
 };
 
@@ -352,7 +353,7 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   }
 
   // ---- 1. threshold bucket b*, this slice's winners and candidates
-  if (tid == 0) { sm.bstar = 0; sm.above = -1; sm.wins = 0; }
+  if (tid == 0) { sm.bstar = 0; sm.above = -1; sm.wins = 0; sm.solo_cand = 0u; }
 #pragma unroll
   for (int e = 0; e < kHPer; ++e) sm.hist[tid + e * kSelThreads] = hv[e];
   __syncthreads();
@@ -402,7 +403,11 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
       if (lane >= o) incl += y;
     }
     uint32_t base = 0;
-    if (lane == 31 && incl) base = atomicAdd(&ctr[0], (uint32_t)incl);
+    // (a CTA that owns the whole row counts in shared memory: no L2 round
+    // trip per pass)
+    if (lane == 31 && incl)
+      base = nsplit == 1 ? atomicAdd(&sm.solo_cand, (uint32_t)incl)
+                         : atomicAdd(&ctr[0], (uint32_t)incl);
     base = __shfl_sync(0xffffffffu, base, 31);
     uint32_t p = base + (uint32_t)(incl - nc);
 #pragma unroll
@@ -435,7 +440,7 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
       __nanosleep(64);
     }
     sm.state = state;
-    sm.n_cand = (int)ld_acquire_u32(&ctr[0]);
+    sm.n_cand = nsplit == 1 ? (int)sm.solo_cand : (int)ld_acquire_u32(&ctr[0]);
   }
   __syncthreads();
   // every CTA of the row has read the histogram before arriving (a CTA that
