@@ -10,6 +10,10 @@
 // «DeepSeek V4-Pro: Architektur, KV-Cache-Kompression und Hyper-Connections im
 // Detail», "Kompression und Selektion".)
 //
+// (The helpers below are not inlined: the kernel runs on a cold instruction
+// cache - once per 4 or 128 tokens - so its time follows the code it fetches,
+// and the planes of one entry share one copy of each helper.)
+//
 // One CTA per (new entry, sequence).  The work is a few KB per entry and runs
 // once per 4 (CSA) or 128 (HCA) tokens.  At decode a single entry is written,
 // so the latency of the loads decides the time: the staged kernel copies the
@@ -29,7 +33,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
-__device__ void store_entry(const Cache &out, int b, long long j, const float *pooled, int D) {
+__device__ __noinline__ void store_entry(const Cache &out, int b, long long j,
+                                        const float *pooled, int D) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (out.fmt == CSKV_FMT_F32) {
     float *dst = reinterpret_cast<float *>(out.data + out.row(b, j) * out.data_stride);
@@ -202,7 +207,7 @@ __device__ inline void stage_bytes(uint8_t *dst, const uint8_t *src, int n, int 
 // rows[r] is the precomputed slot row (b * cap + slot) of position first + r,
 // or -1 when that position does not exist.  One warp per slot: the 16-byte
 // copies of a slot are spread over its lanes.
-__device__ void stage_window(const Cache &c, const SlotLayout &l, const long long *rows,
+__device__ __noinline__ void stage_window(const Cache &c, const SlotLayout &l, const long long *rows,
                              int pool, uint8_t *buf) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int r = warp; r < pool; r += nw) {
@@ -228,7 +233,7 @@ __device__ __forceinline__ float staged_value(const Cache &c, const SlotLayout &
   return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(slot + l.rope_off)[d - c.d_nope]);
 }
 
-__device__ void pool_staged(const Cache &c, const SlotLayout &l, const uint8_t *buf,
+__device__ __noinline__ void pool_staged(const Cache &c, const SlotLayout &l, const uint8_t *buf,
                             long long first, int pool, const float *a, float *pooled) {
   // the format and the slots present (positions >= 0) are fixed per entry: the
   // per-dim loops below carry no per-value branches
