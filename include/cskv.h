@@ -152,6 +152,12 @@ int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
  *   max_entries : host bound on visible entries per row (<= ik->cap).
  *   out_idx  : [B][Tq][k] int32.   out_score : [B][Tq][k] fp32 or NULL.
  *   ws       : cskv_indexer_workspace_size(B, Tq, max_entries, k) bytes.
+ *              The scoring leaves a per-row score histogram in it that only
+ *              guides the selection (every count is checked against the
+ *              scores); the selection clears it for the next call.  A
+ *              workspace holding anything else (never zero-filled, or last
+ *              used with other shapes) costs its first call time, not
+ *              correctness.
  */
 int indexer_topk(int B, int Tq, const int64_t *q_pos,
                  const void *q_ik, const float *q_ik_scale, const float *head_w,
