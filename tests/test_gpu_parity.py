@@ -295,6 +295,40 @@ def test_hca_dense_attention(C, name):
                     np.stack([ref[r][1] for r in rows]), where=name)
 
 
+@pytest.mark.parametrize("Tq", [2, 3, 6])
+def test_multi_token_decode_layers(C, Tq):
+    # a few query tokens per sequence at the end of a long context (draft
+    # tokens of speculative decoding): the indexer scores the rows together
+    # and both layers attend row by row, each row with its own visibility
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer, HCALayer
+    wl = W.get("parity_prefill").with_(B=2, T=20_000 - Tq, Tq=Tq, k=256)
+    Lc = W.make_csa_layer(wl)
+    csa = CSALayer(to_device(Lc))
+    idx = csa.select()
+    out, lse = csa.attend()
+    torch.cuda.synchronize()
+    rows = sample_rows(wl.B, wl.Tq)
+    ref = O.layer_indexer_topk(Lc, wl.k, rows=rows)
+    sel = np.full((wl.B, wl.Tq, wl.k), -1, dtype=np.int32)
+    for (b, t), (ridx, rs) in ref.items():
+        check_topk(idx[b, t].cpu().numpy(), ridx, rs, where=f"Tq={Tq} row {(b, t)}")
+        sel[b, t] = idx[b, t].cpu().numpy()         # attend the GPU's own selection
+    refa = O.layer_attention(Lc, sel=sel, rows=rows)
+    check_attention(np.stack([out[b, t].cpu().numpy() for b, t in rows]),
+                    np.stack([lse[b, t].cpu().numpy() for b, t in rows]),
+                    np.stack([refa[r][0] for r in rows]), np.stack([refa[r][1] for r in rows]),
+                    where=f"csa Tq={Tq}")
+    Lh = W.make_hca_layer(wl)
+    hca = HCALayer(to_device(Lh))
+    out, lse = hca.attend()
+    torch.cuda.synchronize()
+    refh = O.layer_attention(Lh, sel=None, rows=rows)
+    check_attention(np.stack([out[b, t].cpu().numpy() for b, t in rows]),
+                    np.stack([lse[b, t].cpu().numpy() for b, t in rows]),
+                    np.stack([refh[r][0] for r in rows]), np.stack([refh[r][1] for r in rows]),
+                    where=f"hca Tq={Tq}")
+
+
 @pytest.mark.parametrize("kind", ["csa", "hca"])
 def test_decode_attention_repeated_calls_one_workspace(C, kind):
     # several decode calls in a row on one layer (one workspace, partials of
