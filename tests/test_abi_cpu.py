@@ -49,6 +49,11 @@ def test_workspace_sizes(C):
     assert C.indexer_workspace_size(1, 1, 262144, 1024) >= 262144 * 4
     assert C.attn_workspace_size(0, 1, 64, 512, 8192, 128) == 0
     assert C.indexer_workspace_size(1, 1, -1, 8) == 0
+    # chunked prefill: room for the dense entries converted once per call into
+    # FP16 hi/lo key tiles (128 KB per 64 entries per sequence)
+    tiles = 2 * ((8256 + 63) // 64) * 128 * 1024
+    assert C.attn_workspace_size(2, 8192, 64, 512, 8256, 128) >= tiles
+    assert C.attn_workspace_size(2, 2, 64, 512, 8256, 128) >= tiles
 
 
 def _fake_cache(ring, cap=256, fmt=1, d_nope=448, d_rope=64, ptr=1 << 20):
