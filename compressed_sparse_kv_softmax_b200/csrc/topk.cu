@@ -157,7 +157,9 @@ __device__ void find_threshold_bin2(const Bins &bins, int nbins, int target, int
 }
 
 // Whole-row exact top-k by one CTA (any blockDim multiple of 32).
-__device__ void topk_row_single_cta(const float *__restrict__ s, long long n, int k,
+// (not inlined: inside the multi-CTA selection it is the rarely taken
+// fall-back, kept out of the hot code's instruction stream)
+__device__ __noinline__ void topk_row_single_cta(const float *__restrict__ s, long long n, int k,
                                     int32_t *__restrict__ oi, float *__restrict__ os) {
   __shared__ int hist[256];
   __shared__ int scan_scratch[33];
