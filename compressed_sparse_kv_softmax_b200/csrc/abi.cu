@@ -6,6 +6,9 @@
 
 using namespace cskv;
 
+// most query rows (B x Tq) of one indexer call
+constexpr int64_t kMaxIndexerRows = 65535;
+
 namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -153,6 +156,9 @@ int indexer_common(int phases, int B, int Tq, const int64_t *q_pos, const void *
   if (B < 0 || Tq < 0 || (int64_t)B * Tq > 0x7fffffffLL) return CSKV_ERR_ARG;
   if (k < 1 || k > 4096 || stride < 1 || H_I < 1 || d_I < 1 || max_entries < 0)
     return CSKV_ERR_ARG;
+  // query rows run along a grid's y dimension in the scoring and selection
+  // kernels: at most 65,535 per call (larger batches are split by the caller)
+  if ((int64_t)B * Tq > kMaxIndexerRows) return CSKV_ERR_UNSUPPORTED;
   if (B == 0 || Tq == 0) return CSKV_OK;
   if (!q_pos || !q_ik || !head_w || !out_idx) return CSKV_ERR_ARG;
   CSKV_TRY(check_cache(ik, 0));

@@ -151,6 +151,8 @@ int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
  *   k        : selections per row, 1 <= k <= 4096.
  *   max_entries : host bound on visible entries per row (<= ik->cap).
  *   out_idx  : [B][Tq][k] int32.   out_score : [B][Tq][k] fp32 or NULL.
+ *   B * Tq   : at most 65,535 query rows per call (CSKV_ERR_UNSUPPORTED
+ *              otherwise, before anything is launched); split larger batches.
  *   ws       : cskv_indexer_workspace_size(B, Tq, max_entries, k) bytes.
  *              The scoring leaves a per-row score histogram in it that only
  *              guides the selection (every count is checked against the

@@ -121,6 +121,9 @@ def test_argument_errors_are_caught_on_the_host(C):
                   out, None, ws, big, None) == ERR_ARG
         assert fn(*args, R(ik), 4, 1024, 262145, out, None, ws, big, None) == ERR_ARG
         assert fn(*args, R(comp), 4, 1024, 8192, out, None, ws, big, None) == ERR_ARG
+        # more query rows than one call takes (B * Tq > 65,535): refused up front
+        assert fn(2, 40000, ctx, q, P(1 << 32), P(1 << 33), 64, 128, R(ik), 4, 1024, 262144,
+                  out, None, ws, big, None) == ERR_UNSUP
     # compress: ring too small for the entries requested, pool < stride
     gate = P(1 << 35)
     assert lib.csa_compress(1, ctx, ctx, 100, R(ring), None, None, gate, gate, 8, 4, R(comp),
