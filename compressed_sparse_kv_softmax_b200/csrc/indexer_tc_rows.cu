@@ -28,9 +28,15 @@
 //               (M = 128, N = 256, K = 32) into that half's accumulator
 //   warp 2      TMEM allocation (all 512 columns)
 //   warps 4-19  epilogue: warpgroup g reads row g of each half (64 heads of
-//               one query row for 32 entries per warp), applies ReLU, head
-//               weights and the key scale, stores the score (streaming
-//               store) and counts it in the row's score histogram
+//               one query row for 32 entries per warp, 32 heads per TMEM
+//               load), applies ReLU, head weights and the key scale, stores
+//               the score (streaming store) and counts it in the row's score
+//               histogram
+// Every (entry, row, head) product needs a ReLU and a weighted add in fp32,
+// about 1.5 issue slots per 64 MMA FLOP, so the epilogue's issue rate - not
+// the tensor pipe - sets the pace; waiting warps sleep in their mbarrier
+// waits (a suspend-time hint) rather than spin, leaving issue slots to the
+// working ones.
 // The histogram (top 12 bits of the order-preserving score key, as the
 // selection expects) is kept in shared memory as 16-bit counters, two per
 // word: a CTA covers at most kMaxTilesPerCta tiles of a row, i.e. fewer than
