@@ -653,8 +653,12 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"{wl.name}: 1 CSA + 1 HCA layer decode, B={wl.B}, ctx={wl.T}",
-                       "indexer_scales": _scales_text(wl)},
+            "config": {"workload": f"{wl.name}: 1 CSA + 1 HCA layer decode, B={wl.B}/GPU, "
+                                   f"ctx {wl.T}, Hq={wl.Hq}, D={wl.d_nope}+{wl.d_rope}, "
+                                   f"H_I={wl.H_I}x{wl.d_I}, k={wl.k}, window={wl.window}",
+                       "indexer_scales": _scales_text(wl),
+                       "global_batch": wl.B * world, "seq_len": wl.T,
+                       "parallelism": "oracle on the host cores, rank 0"},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores,
                              "kind": "oracle",
                              "sample": f"each step: one decode query over the first "
