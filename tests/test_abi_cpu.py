@@ -163,3 +163,33 @@ def test_layer_phases_name_the_split_calls(C):
     assert layer.indexer_score is C.indexer_score
     assert layer.indexer_select is C.indexer_select
     assert layer.indexer_topk is C.indexer_topk
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    # the boundary is a C ABI: the header compiles as C99 with warnings as
+    # errors, and a C program links against libcskv.so through it
+    import os
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.join(root, "compressed_sparse_kv_softmax_b200")
+    src = tmp_path / "use.c"
+    src.write_text('#include "cskv.h"\n'
+                   "#include <stdio.h>\n"
+                   "int main(void) {\n"
+                   '  printf("%d %s\\n", cskv_version(), cskv_error_string(0));\n'
+                   "  return cskv_indexer_workspace_size(1, 1, 1024, 64) == 0;\n"
+                   "}\n")
+    exe = tmp_path / "use"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+                        "-L", lib_dir, "-lcskv", "-Wl,-rpath," + lib_dir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.split()[1] == "ok"
+
