@@ -24,7 +24,10 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_SCRATCH_LIMIT = 0, -1, -2, -3, -4, -5
+OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_SCRATCH_LIMIT, ERR_DEVICE = (
+    0, -1, -2, -3, -4, -5, -6)
+# device-side events (bits of cskv_check_device_errors)
+DEV_INDEXER_WAIT, DEV_TOPK_BARRIER, DEV_ATTN_WAIT, DEV_ROW_FAILED = 1, 2, 4, 8
 FMT_F32, FMT_E4M3_BF16, FMT_E4M3_VEC = 0, 1, 2
 _FMT = {"f32": FMT_F32, "e4m3": FMT_E4M3_BF16, "e4m3vec": FMT_E4M3_VEC}
 
@@ -59,6 +62,10 @@ _lib.indexer_topk_noalloc.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC, _I, _
                                       _P, _P]
 _lib.indexer_topk_noalloc.restype = _I
 _lib.cskv_noalloc_scratch_bytes.restype = _SZ
+_lib.cskv_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
+_lib.cskv_check_device_errors.restype = _I
+_lib.cskv_debug_topk_barrier_spins.argtypes = [ctypes.c_uint32]
+_lib.cskv_debug_topk_barrier_spins.restype = ctypes.c_uint32
 _lib.cskv_error_string.argtypes = [_I]
 _lib.cskv_error_string.restype = ctypes.c_char_p
 _lib.cskv_version.restype = _I
@@ -225,6 +232,22 @@ def hybrid_attn_prefill(B, Tq, q_pos, q, Hq, sm_scale, comp_k, comp_v, comp_stri
                                     _ref(cs[1]), comp_stride, _ptr(sel), k, int(max_entries),
                                     _ref(cs[2]), _ref(cs[3]), window, _ptr(out), _ptr(lse), wp,
                                     wn, _stream(stream)), "hybrid_attn_prefill")
+
+
+def check_device_errors(stream=None) -> int:
+    """Waits for the stream, then reads and clears the device's sticky event
+    bits (DEV_*); returns them (0: nothing recorded).  Raises on a CUDA error."""
+    ev = ctypes.c_uint32(0)
+    st = _lib.cskv_check_device_errors(_stream(stream), ctypes.byref(ev))
+    if st not in (OK, ERR_DEVICE):
+        raise CskvError(st, "cskv_check_device_errors")
+    return int(ev.value)
+
+
+def debug_topk_barrier_spins(spins: int) -> int:
+    """Polls of the multi-CTA selection's row meeting point before a CTA
+    gives up (tests of the failure path); returns the previous setting."""
+    return int(_lib.cskv_debug_topk_barrier_spins(int(spins)))
 
 
 def error_string(status: int) -> str:

@@ -145,6 +145,8 @@ int attention_common(int B, int Tq, const int64_t *pos, int pos_is_ctx_len, cons
   a.window = window;
   a.out = out; a.lse = lse; a.ws = ws; a.ws_bytes = ws_bytes;
   CSKV_TRY(check_ws(ws, ws_bytes, attn_ws_bytes(B, Tq, Hq, a.Dv, max_comp, window)));
+  a.status = device_status_word();
+  if (!a.status) return CSKV_ERR_CUDA;
   return launch_attention(a, (cudaStream_t)stream);
 }
 
@@ -160,7 +162,7 @@ int indexer_common(int phases, int B, int Tq, const int64_t *q_pos, const void *
   // kernels: at most 65,535 per call (larger batches are split by the caller)
   if ((int64_t)B * Tq > kMaxIndexerRows) return CSKV_ERR_UNSUPPORTED;
   if (B == 0 || Tq == 0) return CSKV_OK;
-  if (!q_pos || !q_ik || !head_w || !out_idx) return CSKV_ERR_ARG;
+  if (!q_pos || !q_ik || !head_w || !out_idx || !aligned16(q_ik)) return CSKV_ERR_ARG;
   CSKV_TRY(check_cache(ik, 0));
   if (ik->d_rope != 0 || ik->d_nope != d_I || max_entries > ik->cap) return CSKV_ERR_ARG;
   if (ik->fmt == CSKV_FMT_E4M3_BF16 || ik->fmt == CSKV_FMT_E4M3_VEC) {
@@ -178,6 +180,8 @@ int indexer_common(int phases, int B, int Tq, const int64_t *q_pos, const void *
   a.ik = to_dev(ik);
   a.out_idx = out_idx; a.out_score = out_score;
   a.ws = ws; a.ws_bytes = ws_bytes;
+  a.status = device_status_word();
+  if (!a.status) return CSKV_ERR_CUDA;
   return launch_indexer_topk(a, phases, (cudaStream_t)stream);
 }
 
@@ -265,6 +269,8 @@ const char *cskv_error_string(int status) {
     case CSKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case CSKV_ERR_SCRATCH_LIMIT:
       return "request needs more scratch than indexer_topk_noalloc's fixed array holds";
+    case CSKV_ERR_DEVICE:
+      return "a kernel recorded a device-side event (a bounded wait ran out or a row failed)";
     default: return "unknown status";
   }
 }

@@ -691,7 +691,9 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
   }
 
   // ---- epilogue: thread = dim within each 128-dim tile, heads 32*colh ..
-  __syncthreads();
+  // (a wait that ran out anywhere in the CTA leaves the partial's lse NaN)
+  ok = __syncthreads_and(ok);
+  if (!ok && tid == 0) record_event(a.status, CSKV_DEV_ATTN_WAIT);
   float *po = part_o + ((size_t)row * n_splits + split) * kHeads * kD;
   float *pl = part_lse + ((size_t)row * n_splits + split) * kHeads;
   if (!started) {

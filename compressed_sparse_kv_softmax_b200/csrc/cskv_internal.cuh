@@ -74,6 +74,27 @@ __device__ __forceinline__ float e4m3_decode(uint8_t code) {
   return float(c);
 }
 
+// Bytes of a key tile's scales that one bulk copy brings: the 16-byte groups
+// of a packed scale plane (sb bytes per cache row) from the one holding the
+// tile's first row to the last one that lies entirely inside the plane.  The
+// copy starts `lead` bytes before the first row's scales; rows whose scales
+// the copy does not hold (at most three at the very end of the cache) are
+// read with plain loads.
+struct ScaleSpan {
+  long long src;       // first byte copied, from the plane's start
+  uint32_t lead;       // bytes before the tile's first row
+  uint32_t bytes;      // bytes copied (a multiple of 16, possibly 0)
+};
+__host__ __device__ inline ScaleSpan scale_span(long long g0, long long rows, int sb) {
+  const long long b0 = g0 * sb, b1 = (g0 + rows) * sb;
+  const long long a0 = b0 & ~15LL, a1 = b1 & ~15LL;
+  ScaleSpan sp;
+  sp.src = a0;
+  sp.lead = (uint32_t)(b0 - a0);
+  sp.bytes = a1 > a0 ? (uint32_t)(a1 - a0) : 0u;
+  return sp;
+}
+
 // Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
 __device__ __forceinline__ uint32_t score_key(float s) {
   uint32_t u = __float_as_uint(s);
@@ -149,6 +170,18 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Sticky per-device status word (status.cu): kernels OR CSKV_DEV_* bits into
+// it when a bounded wait runs out.  device_status_word() is its device
+// address on the current device (nullptr if the lookup failed).
+unsigned int *device_status_word();
+__device__ __forceinline__ void record_event(unsigned int *status, unsigned int bit) {
+  if (status) atomicOr(status, bit);
+}
+// Polls of the multi-CTA selection's row meeting point before a CTA gives up
+// (each poll backs off ~0.1-1 us, so the default is seconds).
+constexpr uint32_t kDefaultBarrierSpins = 1u << 22;
+uint32_t topk_barrier_spins();
+
 // host-side launch helpers (defined in the kernel files)
 int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
                     const Cache &raw_k, const Cache &raw_v, const Cache &raw_ik,
@@ -164,6 +197,7 @@ struct IndexerArgs {
   Cache ik;
   int32_t *out_idx; float *out_score;
   void *ws; size_t ws_bytes;
+  unsigned int *status;    // device status word
 };
 size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k);
 // phases of an indexer call: scoring (with the selection histogram) and the
@@ -185,6 +219,7 @@ struct AttnArgs {
   int window;
   float *out, *lse;
   void *ws; size_t ws_bytes;
+  unsigned int *status;    // device status word
 };
 // How one query row's key list is cut into units and units into splits (one
 // CTA per split).  A split runs its units with an online softmax; with one

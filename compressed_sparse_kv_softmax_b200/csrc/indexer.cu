@@ -18,15 +18,15 @@ namespace cskv {
 
 void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,
                       long long max_entries, int k, int rows, int32_t *out_idx,
-                      float *out_score, cudaStream_t st);
+                      float *out_score, unsigned int *status, cudaStream_t st);
 int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
                        long long max_entries, int k, int rows, int32_t *out_idx,
-                       float *out_score, cudaStream_t st);
+                       float *out_score, unsigned int *status, cudaStream_t st);
 bool indexer_tc_supported(const IndexerArgs &a);
 int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                      uint32_t *ctr, int *err, cudaStream_t st);
+                      uint32_t *ctr, cudaStream_t st);
 int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                        uint32_t *ctr, int *err, cudaStream_t st);
+                        uint32_t *ctr, cudaStream_t st);
 
 namespace {
 
@@ -105,15 +105,14 @@ int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st) {
     // scoring kernel clears the selection's counters.
     if (score) {
       // several query rows per sequence share each key tile; one row streams alone
-      int rc = launch_indexer_rows(a, w.scores, w.ld, w.hist, w.ctr,
-                                   w.err, st);
+      int rc = launch_indexer_rows(a, w.scores, w.ld, w.hist, w.ctr, st);
       if (rc == CSKV_ERR_UNSUPPORTED)
-        rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.ctr, w.err, st);
+        rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.ctr, st);
       if (rc != CSKV_OK) return rc;
     }
     if (!select) return CSKV_OK;
     return launch_topk_select(w, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
-                              a.out_score, st);
+                              a.out_score, a.status, st);
   }
   if (score && a.max_entries > 0) {
     const size_t smem = sizeof(float) * ((size_t)a.H_I * a.d_I + a.H_I +
@@ -127,7 +126,7 @@ int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st) {
   }
   if (select)
     launch_topk_rows(w.scores, w.ld, a.q_pos, a.stride, a.max_entries, a.k, rows, a.out_idx,
-                     a.out_score, st);
+                     a.out_score, a.status, st);
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 

@@ -80,16 +80,14 @@ struct __align__(1024) Smem {
   int abort, qscale_pos;
 };
 
-__device__ __forceinline__ void record_abort(Smem &sm, int *err, int code) {
-  sm.abort = 1;
-  if (err) atomicOr(err, code);
-}
+// A wait ran out: the CTA stops, and its scores are marked failed at the end.
+__device__ __forceinline__ void record_abort(Smem &sm) { sm.abort = 1; }
 
 template <bool kVec>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                   float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
-                  uint32_t *__restrict__ ctr, int *__restrict__ err) {
+                  uint32_t *__restrict__ ctr, bool packed) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem &sm = *reinterpret_cast<Smem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -128,7 +126,6 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   // the selection's per-row counters start at zero (the selection runs after
   // this grid); the row's score histogram was zeroed by the last selection
   if (blockIdx.x == 0 && tid < 4) ctr[(size_t)row * 4 + tid] = 0u;
-  if (blockIdx.x == 0 && row == 0 && tid == 0) *err = 0;
   const long long qpos = a.q_pos[row];
   // tiles of this CTA for n visible entries (tile t goes to CTA t % grid)
   auto tiles_of = [&](long long nn) {
@@ -183,15 +180,15 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
         const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
         const long long g0 = (long long)b * a.ik.cap + j0;    // first row of the tile
         // scales of the rows that exist (the key TMA zero-fills past the end;
-        // a bulk copy must not read past it): whole 16-byte pairs of rows
+        // a bulk copy must not read past it), when the plane is packed
         long long rows = total_rows - g0;
         rows = rows < kTile ? rows : kTile;
-        const uint32_t sbytes = (uint32_t)(rows * kScaleBytes) & ~15u;
-        mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
+        const ScaleSpan sp = packed ? scale_span(g0, rows, kScaleBytes) : ScaleSpan{0, 0, 0};
+        mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sp.bytes);
         tma_load_2d(sm.keys[s], &tmap, &sm.full[s], 0, (int32_t)g0);
-        if (sbytes)
-          bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + g0 * kScaleBytes,
-                    sbytes, &sm.full[s]);
+        if (sp.bytes)
+          bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + sp.src,
+                    sp.bytes, &sm.full[s]);
       };
       // the first stages are filled from the host bound before the row's
       // position has arrived (tiles past the visible ones are loaded, never used)
@@ -203,7 +200,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
         const int s = i % kStages;
         const uint32_t ph = (i / kStages) & 1;
         if (!mbar_wait(&sm.empty[s], ph ^ 1)) {
-          record_abort(sm, err, 1);
+          record_abort(sm);
           break;
         }
         issue(i);
@@ -221,11 +218,11 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       for (int i = 0; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages, acc = i % kAcc;
         if (i >= kAcc && !mbar_wait(&sm.acc_empty[acc], ((i / kAcc) & 1) ^ 1)) {
-          record_abort(sm, err, 2);
+          record_abort(sm);
           break;
         }
         if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
-          record_abort(sm, err, 2);
+          record_abort(sm);
           break;
         }
         tc_fence_after();
@@ -247,7 +244,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       }
       // every MMA of this CTA has finished before TMEM is released
       mma_commit(&sm.mma_done);
-      if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm, err, 4);
+      if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm);
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: the warpgroups take tiles in turn
@@ -264,7 +261,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       const int s = i % kStages;
       const long long j = (long long)(blockIdx.x + i * gridDim.x) * kTile + r;
       if (!mbar_wait(&sm.acc_full[acc], (i / kAcc) & 1)) {
-        record_abort(sm, err, 8);
+        record_abort(sm);
         break;
       }
       tc_fence_after();
@@ -276,19 +273,22 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       float sk0 = 1.f, sk1 = 0.f;            // (rows past n: score not stored)
       if (j < n) {
         const long long g = (long long)b * a.ik.cap + j;
-        const long long tile_rows = total_rows - (g - r);   // rows from the tile's first
-        // entries whose scales the stage's bulk copy brought (whole 16-byte
-        // groups); the rest (at most three at the very end of the cache)
-        // come by plain loads
-        const long long copied =
-            ((tile_rows < kTile ? tile_rows : kTile) * kScaleBytes & ~15LL) / kScaleBytes;
-        if (r < copied) {
-          sk0 = sm.kscale[s][kVec ? r : 2 * r];
-          if (!kVec) sk1 = sm.kscale[s][2 * r + 1];
+        const long long g0 = g - r, tile_rows = total_rows - g0;   // rows from the tile's first
+        // entries whose scales the stage's bulk copy brought; the rest come
+        // by plain loads
+        const ScaleSpan sp =
+            packed ? scale_span(g0, tile_rows < kTile ? tile_rows : kTile, kScaleBytes)
+                   : ScaleSpan{0, 0, 0};
+        const uint32_t off = sp.lead + (uint32_t)r * kScaleBytes;
+        if (off + kScaleBytes <= sp.bytes) {
+          const float *ss = reinterpret_cast<const float *>(
+              reinterpret_cast<const uint8_t *>(sm.kscale[s]) + off);
+          sk0 = ss[0];
+          if (!kVec) sk1 = ss[1];
         } else {
-          const float *sp = reinterpret_cast<const float *>(scale_base + g * kScaleBytes);
-          sk0 = __ldg(sp);
-          if (!kVec) sk1 = __ldg(sp + 1);
+          const float *sg = reinterpret_cast<const float *>(scale_base + g * a.ik.scale_stride);
+          sk0 = __ldg(sg);
+          if (!kVec) sk1 = __ldg(sg + 1);
         }
       }
       mbar_arrive(&sm.empty[s]);
@@ -408,8 +408,27 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
 
   tc_fence_before();
   __syncthreads();
-  // fold this CTA's histogram into the row's
   uint32_t *hg = hist_g + (size_t)row * kTopkBins;
+  if (sm.abort) {
+    // a wait ran out: every visible entry of this CTA's tiles reads NaN and
+    // is counted in the histogram's NaN bin, so the selection reports the
+    // row as failed instead of ranking stale scores
+    const long long n = visible_n();
+    const int my_tiles = tiles_of(n);
+    float *srow = scores + (size_t)row * ld;
+    uint32_t cnt = 0;
+    for (int i = 0; i < my_tiles; ++i)
+      for (int r = tid; r < kTile; r += kThreads) {
+        const long long j = (long long)(blockIdx.x + i * gridDim.x) * kTile + r;
+        if (j < n) {
+          srow[j] = __int_as_float(0x7fffffff);
+          ++cnt;
+        }
+      }
+    if (cnt) atomicAdd(&hg[kTopkNanBin], cnt);
+    if (tid == 0) record_event(a.status, CSKV_DEV_INDEXER_WAIT);
+  }
+  // fold this CTA's histogram into the row's
   for (int i = tid; i < kTopkBins; i += kThreads) {
     const uint32_t v = sm.hist[i];
     if (v) atomicAdd(&hg[i], v);
@@ -442,12 +461,8 @@ bool indexer_tc_supported(const IndexerArgs &a) {
   if ((a.ik.fmt != CSKV_FMT_E4M3_BF16 && !vec) || a.d_I != kDim || a.H_I != kHeads) return false;
   if ((long long)a.B * a.ik.cap >= (1LL << 31)) return false;
   if (((uintptr_t)a.ik.data & 15) || (a.ik.data_stride & 15)) return false;
-  // scales: 8 (per-64) or 4 (per-vector) bytes per entry back to back, each
-  // tile's block 16-byte aligned
-  const long long sb = vec ? 4 : 8;
-  if (a.ik.scale_stride != sb || ((uintptr_t)a.ik.scale & 15)) return false;
-  if (a.B > 1 && (a.ik.cap * sb) % 16) return false;
-  if ((uintptr_t)a.q_ik & 15) return false;
+  // (scales in any stride and alignment: packed planes arrive by bulk copy,
+  // others by plain loads; q_ik is 16-byte aligned by the ABI's checks)
   int dev = 0, major = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -469,7 +484,7 @@ bool make_key_tmap(const IndexerArgs &a, CUtensorMap *map) {
 }
 
 int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                      uint32_t *ctr, int *err, cudaStream_t st) {
+                      uint32_t *ctr, cudaStream_t st) {
   CUtensorMap map;
   if (!make_key_tmap(a, &map)) return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(Smem) + 1024;
@@ -485,7 +500,11 @@ int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_
   if (splits > tiles) splits = tiles;
   if (splits < 1) splits = 1;
   dim3 grid((unsigned)splits, (unsigned)rows);
-  return launch_pdl(kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist, ctr, err) ==
+  // a packed scale plane (one entry's scales after the other) comes by bulk
+  // copies with the key tiles
+  const bool packed = a.ik.scale_stride == (vec ? 4 : 8);
+  return launch_pdl(kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist, ctr,
+                    packed) ==
                  cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;

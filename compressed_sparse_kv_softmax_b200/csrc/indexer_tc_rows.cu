@@ -84,10 +84,8 @@ struct __align__(1024) RowsSmem {
   int qscale_pos[kRows];                       // every query scale of the row > 0
 };
 
-__device__ __forceinline__ void record_abort(RowsSmem &sm, int *err, int code) {
-  sm.abort = 1;
-  if (err) atomicOr(err, code);
-}
+// A wait ran out: the CTA stops, and its scores are marked failed at the end.
+__device__ __forceinline__ void record_abort(RowsSmem &sm) { sm.abort = 1; }
 
 // Part of a row's score over 32 heads, as two partial sums (factored: without
 // the key scale)
@@ -123,7 +121,7 @@ __device__ __forceinline__ float2 row_part(const float (&v)[32], const float *c1
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                     float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
-                    uint32_t *__restrict__ ctr, int *__restrict__ err, int groups_per_seq) {
+                    uint32_t *__restrict__ ctr, int groups_per_seq, bool packed) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   RowsSmem &sm = *reinterpret_cast<RowsSmem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -163,7 +161,6 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
   // the selection's per-row counters start at zero (the selection runs after
   // this grid); the rows' score histograms were zeroed by the last selection
   if (blockIdx.x == 0 && tid < nrows * 4) ctr[(size_t)row0 * 4 + tid] = 0u;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *err = 0;
 
   // tiles of this CTA for n entries (tile t goes to split t % gridDim.x)
   auto tiles_of = [&](long long nn) {
@@ -220,16 +217,16 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
         const int s = i % kStages;
         const long long j0 = ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile;
         const long long g0 = (long long)b * a.ik.cap + j0;     // first cache row of the tile
-        // scales of the rows that exist, in whole 16-byte groups (the key TMA
-        // zero-fills past the end; a bulk copy must not read past it)
+        // scales of the rows that exist (the key TMA zero-fills past the end;
+        // a bulk copy must not read past it), when the plane is packed
         long long rows = total_rows - g0;
         rows = rows < kTile ? rows : kTile;
-        const uint32_t sbytes = (uint32_t)(rows * 4) & ~15u;
-        mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sbytes);
+        const ScaleSpan sp = packed ? scale_span(g0, rows, 4) : ScaleSpan{0, 0, 0};
+        mbar_arrive_expect_tx(&sm.full[s], kTileBytes + sp.bytes);
         tma_load_2d_hint(sm.keys[s], &tmap, &sm.full[s], 0, (int32_t)g0, keep);
-        if (sbytes)
-          bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + g0 * 4, sbytes,
-                    &sm.full[s]);
+        if (sp.bytes)
+          bulk_load(sm.kscale[s], reinterpret_cast<const uint8_t *>(a.ik.scale) + sp.src,
+                    sp.bytes, &sm.full[s]);
       };
       // the first stages are filled from the host bound before the positions
       // are read (tiles past the visible ones are loaded, never used)
@@ -242,7 +239,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       for (int i = spec; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages;
         if (!mbar_wait_sleep(&sm.empty[s], ((i / kStages) & 1) ^ 1)) {
-          record_abort(sm, err, 1);
+          record_abort(sm);
           break;
         }
         issue(i);
@@ -262,7 +259,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       for (int i = 0; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages;
         if (!mbar_wait_sleep(&sm.full[s], (i / kStages) & 1)) {
-          record_abort(sm, err, 2);
+          record_abort(sm);
           break;
         }
         const uint32_t ka = smem_addr(sm.keys[s]);
@@ -270,7 +267,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
         for (int h = 0; h < halves; ++h) {
           // the epilogue has drained this half's accumulator of the last tile
           if (i > 0 && !mbar_wait_sleep(&sm.acc_empty[h], (i - 1) & 1)) {
-            record_abort(sm, err, 2);
+            record_abort(sm);
             ok = false;
             break;
           }
@@ -287,7 +284,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       }
       // every MMA of this CTA has finished before TMEM is released
       mma_commit(&sm.mma_done);
-      if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm, err, 4);
+      if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm);
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: warpgroup eg takes row eg of each half
@@ -300,12 +297,9 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
     nr[0] = (int)sm.n[eg];
     nr[1] = (int)sm.n[kHalfRows + eg];
     const int my_tiles = tiles_of(nmax);
-    // cache rows whose scales the stages' bulk copies bring (whole 16-byte
-    // groups: every row below the cache's row count rounded down to 4); the
-    // last few rows of the whole cache come by plain loads
-    const int copied_end = (int)(((long long)a.B * a.ik.cap) & ~3LL);
+    const long long total_rows = (long long)a.B * a.ik.cap;
     const int gb = b * (int)a.ik.cap;
-    const float *scale_base = reinterpret_cast<const float *>(a.ik.scale);
+    const uint8_t *scale_base = reinterpret_cast<const uint8_t *>(a.ik.scale);
     float *srow0 = scores + (row0 + eg) * ld;
     float *srow1 = scores + (row0 + kHalfRows + eg) * ld;
     const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + eg * kHeads;
@@ -317,17 +311,27 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       // the tile's scales arrived with its keys (the stage is not refilled
       // before this warp arrives on its empty barrier)
       if (!mbar_wait_sleep(&sm.full[s], (i / kStages) & 1)) {
-        record_abort(sm, err, 8);
+        record_abort(sm);
         break;
       }
       float sk = 1.f;
-      if (j < nmax) sk = gb + j < copied_end ? sm.kscale[s][r] : __ldg(scale_base + gb + j);
+      if (j < nmax) {
+        // the scales the stage's bulk copy brought, else a plain load
+        const long long g0 = (long long)gb + jt, tile_rows = total_rows - g0;
+        const ScaleSpan sp =
+            packed ? scale_span(g0, tile_rows < kTile ? tile_rows : kTile, 4) : ScaleSpan{0, 0, 0};
+        const uint32_t off = sp.lead + 4u * (uint32_t)r;
+        sk = off + 4 <= sp.bytes
+                 ? *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(sm.kscale[s]) + off)
+                 : __ldg(reinterpret_cast<const float *>(scale_base +
+                                                         ((long long)gb + j) * a.ik.scale_stride));
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
       bool stop = false;
       for (int h = 0; h < halves; ++h) {
         if (!mbar_wait_sleep(&sm.acc_full[h], i & 1)) {
-          record_abort(sm, err, 8);
+          record_abort(sm);
           stop = true;
           break;
         }
@@ -376,6 +380,28 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
 
   tc_fence_before();
   __syncthreads();
+  if (sm.abort) {
+    // a wait ran out: every visible entry of this CTA's tiles reads NaN in
+    // each of the group's rows and is counted in its histogram's NaN bin, so
+    // the selection reports those rows as failed
+    long long nmax = 0;
+    for (int q = 0; q < nrows; ++q) nmax = max(nmax, sm.n[q]);
+    const int my_tiles = tiles_of(nmax);
+    for (int q = 0; q < nrows; ++q) {
+      uint32_t cnt = 0;
+      float *srow = scores + (row0 + q) * ld;
+      for (int i = 0; i < my_tiles; ++i)
+        for (int r = tid; r < kTile; r += kThreads) {
+          const long long j = ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile + r;
+          if (j < sm.n[q]) {
+            srow[j] = __int_as_float(0x7fffffff);
+            ++cnt;
+          }
+        }
+      if (cnt) atomicAdd(hist_g + (size_t)(row0 + q) * kTopkBins + kTopkNanBin, cnt);
+    }
+    if (tid == 0) record_event(a.status, CSKV_DEV_INDEXER_WAIT);
+  }
   // fold the 16-bit counters into the rows' 32-bit histograms
   for (int i = tid; i < nrows * kHistWords; i += kThreads) {
     const int rr = i / kHistWords, wi = i % kHistWords;
@@ -399,7 +425,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
 // per-vector scale layout; returns CSKV_ERR_UNSUPPORTED, before launching
 // anything, where the grid does not fit.
 int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
-                        uint32_t *ctr, int *err, cudaStream_t st) {
+                        uint32_t *ctr, cudaStream_t st) {
   if (a.ik.fmt != CSKV_FMT_E4M3_VEC || a.Tq < 2) return CSKV_ERR_UNSUPPORTED;
   const int gps = (a.Tq + kRows - 1) / kRows;
   const long long groups = (long long)a.B * gps;
@@ -419,8 +445,9 @@ int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint3
   if (splits < fill) splits = fill < tiles ? fill : tiles;
   if (splits < 1) splits = 1;
   dim3 grid((unsigned)splits, (unsigned)groups);
+  const bool packed = a.ik.scale_stride == 4;
   return launch_pdl(indexer_rows_kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld,
-                    hist, ctr, err, gps) == cudaSuccess
+                    hist, ctr, gps, packed) == cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;
 }

@@ -13,16 +13,23 @@
 // that device; make that first call before any stream capture.  All calls
 // share the one array, so calls that overlap on the GPU (different streams,
 // or different host threads, on the same device) race on it and must be
-// serialised by the caller.  The indexer writes every score slot it later
-// reads, so nothing in the array has to start at zero.
+// serialised by the caller.  Nothing in it has to start at zero: each call's
+// scoring writes every score slot its selection reads (a scoring CTA whose
+// wait ran out writes NaN there, and the selection then reports the row as
+// failed), and the score histogram and counters kept between calls only
+// guide the selection - a stale histogram from a call of another shape costs
+// time, not correctness.
 #include <mutex>
 
 #include "cskv_internal.cuh"
 
 namespace {
 
-// 8 MiB: one fp32 score per visible entry per query row, e.g. one
-// 1,048,576-token sequence (262,144 CSA entries) or 8 rows of 65,536 tokens.
+// 8 MiB.  A request fits when cskv_indexer_workspace_size(B, Tq, max_entries,
+// k) <= 8 MiB: one query row at a 1,048,576-token context (262,144 CSA
+// entries, k = 1,024) needs 1,131,776 bytes, so up to 7 such rows fit; a row
+// at 65,536 tokens (16,384 entries, k = 512) needs 148,512 bytes, up to 56
+// rows.
 constexpr size_t kScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) unsigned char g_indexer_scratch[kScratchBytes];
 

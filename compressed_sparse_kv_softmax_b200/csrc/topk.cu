@@ -156,29 +156,55 @@ __device__ void find_threshold_bin2(const Bins &bins, int nbins, int target, int
   __syncthreads();
 }
 
+// A row with a NaN score (a scoring CTA that gave up marks its entries so,
+// and NaN inputs give NaN scores) has no ranking: every slot of the row
+// reads -1 / NaN and the event is recorded.
+__device__ void write_failed_row(int k, int32_t *__restrict__ oi, float *__restrict__ os,
+                                 unsigned int *status) {
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    oi[i] = -1;
+    if (os) os[i] = __int_as_float(0x7fffffff);
+  }
+  if (threadIdx.x == 0) record_event(status, CSKV_DEV_ROW_FAILED);
+}
+
 // Whole-row exact top-k by one CTA (any blockDim multiple of 32).
 // (not inlined: inside the multi-CTA selection it is the rarely taken
 // fall-back, kept out of the hot code's instruction stream)
 __device__ __noinline__ void topk_row_single_cta(const float *__restrict__ s, long long n, int k,
-                                    int32_t *__restrict__ oi, float *__restrict__ os) {
+                                    int32_t *__restrict__ oi, float *__restrict__ os,
+                                    unsigned int *status) {
   __shared__ int hist[256];
   __shared__ int scan_scratch[33];
   const int tid = threadIdx.x;
   uint32_t thr = 0;
   int take_eq = 0;
   const bool all = n <= k;
-  if (!all) {
+  if (all) {
+    bool nan = false;
+    for (long long j = tid; j < n; j += blockDim.x) nan |= isnan(s[j]);
+    if (__syncthreads_or(nan)) {
+      write_failed_row(k, oi, os, status);
+      return;
+    }
+  } else {
     uint32_t prefix = 0, mask = 0;
     int remaining = k;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
       for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
       __syncthreads();
+      bool nan = false;
       for (long long j = tid; j < n; j += blockDim.x) {
-        const uint32_t key = score_key(s[j]);
+        const float sv = s[j];
+        nan |= isnan(sv);
+        const uint32_t key = score_key(sv);
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
       }
-      __syncthreads();
+      if (__syncthreads_or(nan)) {      // (only the first pass can see one)
+        write_failed_row(k, oi, os, status);
+        return;
+      }
       __shared__ int s_bin, s_above;
       if (tid == 0) { s_bin = 0; s_above = 0; }
       find_threshold_bin([&](int i) { return hist[i]; }, 256, remaining, scan_scratch, &s_bin,
@@ -261,9 +287,6 @@ constexpr int kSelPer = 8;                        // consecutive entries per thr
 constexpr int kSelChunk = kSelThreads * kSelPer;  // entries per CTA and pass
 constexpr int kMaxK = 4096;
 constexpr int kTieCap = kTopkBins;                // exact ties held in the histogram's space
-// Spins of the row barrier before it gives up (each backs off ~0.1-1 us, so
-// the limit is seconds: far beyond any legitimate wait, which is microseconds).
-constexpr uint32_t kBarrierSpins = 1u << 22;
 
 struct SelSmem {
   uint32_t hist[kTopkBins];   // row histogram, then refine bins, then the tie list
@@ -295,13 +318,13 @@ __device__ __forceinline__ void load8(const float *__restrict__ s, long long j0,
 __global__ void __launch_bounds__(1024)
 topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *__restrict__ q_pos,
                  int stride, long long max_entries, int k, int32_t *__restrict__ out_idx,
-                 float *__restrict__ out_score) {
+                 float *__restrict__ out_score, unsigned int *status) {
   pdl_wait();
   pdl_trigger();
   const int row = blockIdx.x;
   const long long n = visible(q_pos, row, stride, max_entries);
   topk_row_single_cta(scores + (long long)row * ld, n, k, out_idx + (long long)row * k,
-                      out_score ? out_score + (long long)row * k : nullptr);
+                      out_score ? out_score + (long long)row * k : nullptr, status);
 }
 
 // kDeep: slices longer than one pass (a CTA per row of a long chunk); the
@@ -310,7 +333,7 @@ template <bool kDeep>
 __global__ void __launch_bounds__(kSelThreads, 1)
 topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int stride,
                    long long max_entries, int k, int32_t *__restrict__ out_idx,
-                   float *__restrict__ out_score) {
+                   float *__restrict__ out_score, unsigned int *status, uint32_t spin_limit) {
   extern __shared__ __align__(16) uint8_t sel_smem_raw[];
   SelSmem &sm = *reinterpret_cast<SelSmem *>(sel_smem_raw);
   pdl_wait();
@@ -344,14 +367,37 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   uint4 *hclear = reinterpret_cast<uint4 *>(w.hist + (size_t)row * kTopkBins);
   if (n <= k) {            // every visible entry is selected, already in order
     if (me == 0) {
-      for (int i = tid; i < k; i += blockDim.x) {
-        oi[i] = i < n ? i : -1;
-        if (os) os[i] = i < n ? s[i] : -__int_as_float(0x7f800000);
+      bool nan = false;
+      for (long long i = tid; i < n; i += blockDim.x) nan |= isnan(s[i]);
+      if (__syncthreads_or(nan)) {
+        write_failed_row(k, oi, os, status);
+      } else {
+        for (int i = tid; i < k; i += blockDim.x) {
+          oi[i] = i < n ? i : -1;
+          if (os) os[i] = i < n ? s[i] : -__int_as_float(0x7f800000);
+        }
       }
       // (the histogram is not read on this path)
       for (int i = tid; i < kTopkBins / 4; i += blockDim.x) hclear[i] = make_uint4(0, 0, 0, 0);
     }
     return;
+  }
+
+  // ---- 0. a histogram with counts in the NaN / infinity bins (a scoring CTA
+  // gave up, or the inputs hold NaN): the row's first CTA checks every score
+  // in the whole-row path; the last CTA to pass here clears the histogram
+  {
+    bool extreme = false;
+#pragma unroll
+    for (int e = 0; e < kHPer; ++e) extreme |= hv[e] != 0u && topk_extreme_bin(tid + e * kSelThreads);
+    if (__syncthreads_or(extreme)) {
+      if (tid == 0) sm.state = atomicAdd(&w.ctr[(size_t)row * 4 + 1], 1u) == (uint32_t)nsplit - 1;
+      __syncthreads();
+      if (sm.state)
+        for (int i = tid; i < kTopkBins / 4; i += blockDim.x) hclear[i] = make_uint4(0, 0, 0, 0);
+      if (me == 0) topk_row_single_cta(s, n, k, oi, os, status);
+      return;
+    }
   }
 
   // ---- 1. threshold bucket b*, this slice's winners and candidates
@@ -434,9 +480,9 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     int state = 0;
     uint32_t spins = 0;
     while (ld_acquire_u32(&ctr[1]) < (uint32_t)nsplit) {
-      if (++spins > kBarrierSpins) {
+      if (++spins > spin_limit) {
         state = 1;
-        atomicOr(w.err, 2);
+        record_event(status, CSKV_DEV_TOPK_BARRIER);
         break;
       }
       __nanosleep(64);
@@ -446,8 +492,9 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   }
   __syncthreads();
   // every CTA of the row has read the histogram before arriving (a CTA that
-  // gave up waiting selects from the scores alone)
-  if (me == 0)
+  // gave up waiting selects from the scores alone and leaves the histogram:
+  // a stale one costs the next call time, not correctness)
+  if (me == 0 && sm.state == 0)
     for (int i = tid; i < kTopkBins / 4; i += blockDim.x) hclear[i] = make_uint4(0, 0, 0, 0);
   const int n_cand = sm.n_cand;
   const int r = k - above;             // candidates still to take
@@ -645,19 +692,19 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   }
   // inconsistent histogram or candidate overflow (never expected with the
   // scoring kernel's histogram): the row's first CTA selects the whole row
-  if (me == 0) topk_row_single_cta(s, n, k, oi, os);
+  if (me == 0) topk_row_single_cta(s, n, k, oi, os, status);
 }
 
 void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,
                       long long max_entries, int k, int rows, int32_t *out_idx,
-                      float *out_score, cudaStream_t st) {
+                      float *out_score, unsigned int *status, cudaStream_t st) {
   launch_pdl(topk_rows_kernel, dim3(rows), dim3(1024), 0, st, scores, ld, q_pos, stride,
-             max_entries, k, out_idx, out_score);
+             max_entries, k, out_idx, out_score, status);
 }
 
 int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
                        long long max_entries, int k, int rows, int32_t *out_idx,
-                       float *out_score, cudaStream_t st) {
+                       float *out_score, unsigned int *status, cudaStream_t st) {
   if (k > kMaxK) return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(SelSmem);
   int dev = 0, sms = 148;
@@ -675,7 +722,7 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
   auto kernel = per > kSelChunk ? topk_select_kernel<true> : topk_select_kernel<false>;
   if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   launch_pdl(kernel, dim3((unsigned)splits, (unsigned)rows), dim3(kSelThreads), smem, st, w,
-             q_pos, stride, max_entries, k, out_idx, out_score);
+             q_pos, stride, max_entries, k, out_idx, out_score, status, topk_barrier_spins());
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
 }
 

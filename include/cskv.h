@@ -57,7 +57,26 @@ enum {
   CSKV_ERR_UNSUPPORTED = -2,  /* valid but not implemented combination of formats/dims */
   CSKV_ERR_CUDA = -3,         /* a kernel launch failed */
   CSKV_ERR_WORKSPACE = -4,    /* ws is NULL, misaligned or smaller than required */
-  CSKV_ERR_SCRATCH_LIMIT = -5 /* request larger than indexer_topk_noalloc's fixed scratch */
+  CSKV_ERR_SCRATCH_LIMIT = -5, /* request larger than indexer_topk_noalloc's fixed scratch */
+  CSKV_ERR_DEVICE = -6         /* cskv_check_device_errors: a kernel recorded an event below */
+};
+
+/*
+ * Device-side events (bits of the sticky per-device status word that
+ * cskv_check_device_errors reads).  Every wait inside a kernel is bounded
+ * (seconds, far beyond any legitimate wait); when one runs out the kernel
+ * records the event, leaves the affected results visibly invalid and
+ * returns instead of hanging.
+ */
+enum {
+  CSKV_DEV_INDEXER_WAIT = 1,  /* a scoring CTA gave up waiting on its copy / MMA pipeline;
+                                 its scores read NaN and its rows are reported failed */
+  CSKV_DEV_TOPK_BARRIER = 2,  /* the selection's per-row meeting point timed out; the row was
+                                 selected by one CTA from its scores (result unchanged) */
+  CSKV_DEV_ATTN_WAIT = 4,     /* an attention CTA gave up waiting on its copies / MMAs;
+                                 the affected rows' lse is NaN */
+  CSKV_DEV_ROW_FAILED = 8     /* the selection met a row with a NaN score; that row's
+                                 out_idx is all -1 and its out_score all NaN */
 };
 
 enum {
@@ -207,11 +226,15 @@ size_t cskv_indexer_workspace_size(int B, int Tq, int64_t max_entries, int k);
  *  - The first call on a device looks the array's address up (once per
  *    device, with that device current); make that first call before any
  *    stream capture.
- *  - Requests whose workspace (cskv_indexer_workspace_size) exceeds the array
- *    return CSKV_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *  - A request fits when cskv_indexer_workspace_size(B, Tq, max_entries, k)
+ *    <= cskv_noalloc_scratch_bytes(): e.g. up to 7 query rows at a
+ *    1,048,576-token context (k = 1,024), or 56 rows at 65,536 tokens
+ *    (k = 512).  Larger requests return CSKV_ERR_SCRATCH_LIMIT before
+ *    anything is enqueued.
  *  - All calls share the array: calls that may overlap on the GPU (other
  *    streams or host threads on the same device) race and must be serialised
- *    by the caller.  Nothing in the array needs to start at zero.
+ *    by the caller.  Nothing in the array needs to start at zero, and calls
+ *    of different shapes may follow one another.
  *  - It allocates nothing (no cudaMalloc / cudaFree or allocating library call).
  */
 int indexer_topk_noalloc(int B, int Tq, const int64_t *q_pos,
@@ -265,6 +288,27 @@ int hybrid_attn_prefill(int B, int Tq, const int64_t *q_pos, const void *q, int 
                         float *out, float *lse, void *ws, size_t ws_bytes, cskv_stream_t stream);
 
 size_t cskv_attn_workspace_size(int B, int Tq, int Hq, int Dv, int64_t max_entries, int window);
+
+/*
+ * cskv_check_device_errors - waits for `stream` to finish, then reads and
+ * clears the current device's sticky status word: the CSKV_DEV_* events that
+ * kernels of this library recorded on the device since the last read (from
+ * any stream).  Writes the bits to *events (may be NULL) and returns CSKV_OK
+ * when none was recorded, CSKV_ERR_DEVICE when some were, CSKV_ERR_CUDA when
+ * the synchronisation or the read failed.  Not for use inside stream capture.
+ */
+int cskv_check_device_errors(cskv_stream_t stream, uint32_t *events);
+
+/*
+ * cskv_debug_topk_barrier_spins - sets how many times a CTA of the multi-CTA
+ * top-k selection polls its row's meeting point before it gives up (default
+ * 4,194,304, i.e. seconds), and returns the previous setting.  For tests of
+ * the failure path: with 0 a CTA that arrives before the others gives up at
+ * once, the row's first CTA then selects the whole row from its scores (the
+ * result is the same) and CSKV_DEV_TOPK_BARRIER is recorded.  Affects calls
+ * made afterwards in this process, on every device.
+ */
+uint32_t cskv_debug_topk_barrier_spins(uint32_t spins);
 
 /* Static text for a status code. */
 const char *cskv_error_string(int status);

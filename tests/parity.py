@@ -20,11 +20,14 @@ import oracle as O
 
 TOPK_REL = 1e-3
 ATTN_REL = 2e-3
-# Natural-log units.  The tensor-core path rounds dequantised K/V and the
-# probabilities to fp16 (unit roundoff 2^-11); a logit over D = 512 dims then
-# carries an error of about sm_scale * 2^-11 * ||q|| * ||K|| / sqrt(D) ~ 5e-4,
-# and lse inherits at most the largest logit error.
-LSE_TOL = 2e-3
+# Natural-log units, the survey's bound.  Both attention paths keep about 22
+# significant bits in every product: the CUDA-core path computes in fp32, the
+# tensor-core path splits every operand that is not exact in FP16 into FP16
+# hi + lo parts (relative error ~2^-22) and accumulates in fp32.  A logit
+# sm_scale * q . k over D = 512 dims with |q|, |k| ~ sqrt(D) then carries an
+# error of order 2^-22 * sm_scale * |q| |k| ~ 1e-5 at the largest logits, and
+# lse = m + log(sum) inherits at most that plus the fp32 rounding of the sum.
+LSE_TOL = 1e-4
 # Float32 evaluation error of a pooled value c = sum_r a_r x_r, relative to
 # its magnitude scale m = sum_r a_r |x_r|: the sum itself contributes about
 # pool * 2^-24 * m, and an error dg in a gate logit g_r = w . k + b (D terms,

@@ -177,3 +177,58 @@ def test_layer_compress_tiny_uniform_gate_equals_mean():
     for j, row in zip(res["j"], res["k"]):
         pos = O.pool_positions(int(j), 8, 4)
         assert np.allclose(row, ring[pos % ring.shape[0]].mean(axis=0), rtol=1e-13, atol=1e-13)
+
+
+def _bf16_bits_to_float(bits: int) -> float:
+    # a BF16 value is the upper half of an IEEE binary32 word
+    import struct
+    return struct.unpack("<f", struct.pack("<I", (int(bits) & 0xFFFF) << 16))[0]
+
+
+def _kv_entry_brute_force(codes, scales, rope, b, j):
+    """One cache entry of the FP8 + BF16 KV layout read value by value: dims
+    0 .. 447 are E4M3 codes times the scale of their 64-dim block, dims
+    448 .. 511 the BF16 RoPE part."""
+    tab = O.e4m3_value_table()
+    d_nope, d_rope = codes.shape[2], rope.shape[2]
+    out = []
+    for d in range(d_nope):
+        out.append(tab[int(codes[b, j, d])] * float(scales[b, j, d // 64]))
+    for r in range(d_rope):
+        out.append(_bf16_bits_to_float(rope[b, j, r]))
+    return np.array(out)
+
+
+def test_dequant_slots_kv_layout_brute_force():
+    # the compressed KV cache entry of the measured workloads: 448 E4M3 dims
+    # with seven fp32 block scales (scale plane padded to eight columns), then
+    # 64 BF16 RoPE dims.  Planted mistakes (RoPE part first, scale columns
+    # shifted by one block, the pad column used) must all disagree.
+    rng = np.random.default_rng(11)
+    B, n, d_nope, d_rope = 2, 5, 448, 64
+    codes = rng.integers(0, 256, size=(B, n, d_nope)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x01     # no NaN codes
+    scales = rng.uniform(0.25, 4.0, size=(B, n, 8))
+    scales[:, :, 7] = np.nan                 # the pad column is never read
+    rope_vals = rng.normal(size=(B, n, d_rope))
+    rope = torch.tensor(rope_vals, dtype=torch.float32).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+    cache = {"fmt": "e4m3", "d_nope": d_nope, "d_rope": d_rope, "data": codes, "scale": scales,
+             "rope": rope}
+    slots = [3, 0, 4]
+    got = O.dequant_slots(cache, 1, slots)
+    assert got.shape == (3, d_nope + d_rope)
+    for r, j in enumerate(slots):
+        want = _kv_entry_brute_force(codes, scales, rope, 1, j)
+        assert np.array_equal(got[r], want), f"slot {j}"
+        # planted mistakes that a wrong oracle could make
+        rope_first = np.concatenate([want[d_nope:], want[:d_nope]])
+        assert not np.array_equal(got[r], rope_first)
+        tab = O.e4m3_value_table()
+        shifted = np.array([tab[codes[1, j, d]] * scales[1, j, min(d // 64 + 1, 6)]
+                            for d in range(d_nope)])
+        assert not np.array_equal(got[r, :d_nope], shifted)
+        assert np.all(np.isfinite(got[r]))    # the NaN pad scale is not used
+    # the BF16 part is exactly torch's bfloat16 value of the stored bits
+    ref_rope = torch.tensor(rope.view(np.int16)).view(torch.bfloat16).double().numpy()
+    assert np.array_equal(got[:, d_nope:], ref_rope[1, slots])
