@@ -176,30 +176,36 @@ class Replica:
         self.hca = HCALayer(self.hca_L)
         self.sched = sched
 
-    def step(self, s, mark=None, pos=None, split_select=True):
-        """Enqueue decode step s of the window on the current stream; mark(i)
-        records an event between calls (i = 0 before indexer_score, 1 after
-        it).  indexer_score + indexer_select is the indexer_topk call (one call
-        when split_select is False).  pos = (q_pos, ctx_len, t_begin, t_end)
-        device tensors replace the schedule's."""
+    def step(self, s, hook=None, pos=None, split_select=True):
+        """Enqueue decode step s of the window on the current stream.
+        hook(name) runs before each call (names in CALLS) and hook("end")
+        after the last.  indexer_score + indexer_select is the indexer_topk
+        call (one call, "indexer_topk", when split_select is False).
+        pos = (q_pos, ctx_len, t_begin, t_end) device tensors replace the
+        schedule's."""
         sc = self.sched
         q_pos, ctx, tb, te = pos if pos is not None else (sc.q_pos[s], sc.ctx[s], sc.tb[s],
                                                           sc.te[s])
+        mark = hook or (lambda name: None)
         if sc.csa_fires[s]:
+            mark("csa_compress")
             self.csa.compress(tb, te, 1)
         if split_select:
-            if mark:
-                mark(0)
+            mark("indexer_score")
             self.csa.select(q_pos, phase="score")
-            if mark:
-                mark(1)
+            mark("indexer_select")
             self.csa.select(q_pos, phase="pick")
         else:
+            mark("indexer_topk")
             self.csa.select(q_pos)
+        mark("csa_attention")
         self.csa.attend(pos=ctx)
         if sc.hca_fires[s]:
+            mark("hca_compress")
             self.hca.compress(tb, te, 1)
+        mark("hca_attention")
         self.hca.attend(pos=ctx)
+        mark("end")
 
 
 def _rt():
@@ -214,7 +220,9 @@ def _ok(res, what):
     return res[1] if isinstance(res, tuple) and len(res) == 2 else res
 
 
-EVENT_EVERY = 16  # steps between in-graph event pairs (each record node stalls the stream)
+EVENT_EVERY = 2   # steps between in-graph event pairs around the indexer scoring call
+CALLS = ("csa_compress", "indexer_score", "indexer_select", "csa_attention", "hca_compress",
+         "hca_attention")
 
 
 class StepGraph:
@@ -244,6 +252,14 @@ class StepGraph:
             _ok(rt.cudaStreamWaitEvent(side, f, 0), "fork wait")
             _ok(rt.cudaEventRecordWithFlags(ev, side, rt.cudaEventRecordExternal), "record")
 
+        def hook_for(ev):
+            def hook(name):
+                if name == "indexer_score":
+                    mark_on_side(ev[0])
+                elif name == "indexer_select":
+                    mark_on_side(ev[1])
+            return hook
+
         with torch.cuda.stream(stream):
             _ok(rt.cudaStreamBeginCapture(
                 sh, rt.cudaStreamCaptureMode.cudaStreamCaptureModeThreadLocal), "capture")
@@ -252,8 +268,7 @@ class StepGraph:
                 if i % EVENT_EVERY:
                     rep.step((i0 + i) % PERIOD)
                     continue
-                ev = self.events[i // EVENT_EVERY]
-                rep.step((i0 + i) % PERIOD, mark=lambda m, ev=ev: mark_on_side(ev[m]))
+                rep.step((i0 + i) % PERIOD, hook=hook_for(self.events[i // EVENT_EVERY]))
             # join the side stream back before the capture ends
             j = next(forks)
             _ok(rt.cudaEventRecord(j, side), "join")
@@ -284,6 +299,43 @@ class StepGraph:
         return [_ok(rt.cudaEventElapsedTime(a, b), "elapsed") for a, b in self.events]
 
 
+class CallGraph:
+    """CUDA graph of G decode steps with an event recorded on the step's own
+    stream before every call and after the last one: each call then runs on
+    its own (its kernels start once the previous call has finished), and
+    consecutive events give its duration.  Replayed after the timed region;
+    every replay adds one sample per call and step."""
+
+    def __init__(self, replicas, G, stream, i0=0):
+        rt = _rt()
+        self.sh = rt.cudaStream_t(stream.cuda_stream)
+        self.marks = []          # (name, event) in stream order
+        with torch.cuda.stream(stream):
+            _ok(rt.cudaStreamBeginCapture(
+                self.sh, rt.cudaStreamCaptureMode.cudaStreamCaptureModeThreadLocal), "capture")
+
+            def hook(name):
+                ev = _ok(rt.cudaEventCreate(), "event")
+                _ok(rt.cudaEventRecordWithFlags(ev, self.sh, rt.cudaEventRecordExternal),
+                    "record")
+                self.marks.append((name, ev))
+
+            for i in range(G):
+                replicas[(i0 + i) % len(replicas)].step((i0 + i) % PERIOD, hook=hook)
+            self.graph = _ok(rt.cudaStreamEndCapture(self.sh), "end capture")
+        self.exec = _ok(rt.cudaGraphInstantiate(self.graph, 0), "instantiate")
+
+    def run(self, samples):
+        """Replay once and append each call's duration (ms) to samples[name]."""
+        rt = _rt()
+        _ok(rt.cudaGraphLaunch(self.exec, self.sh), "graph launch")
+        _ok(rt.cudaStreamSynchronize(self.sh), "sync")
+        for (name, a), (_, b) in zip(self.marks, self.marks[1:]):
+            if name != "end":
+                samples.setdefault(name, []).append(
+                    _ok(rt.cudaEventElapsedTime(a, b), "elapsed"))
+
+
 def _ik_scales(wl):
     """fp32 scales per indexer key or query head: one per vector in the
     per-vector layout, else one per 64 dims."""
@@ -301,22 +353,55 @@ def indexer_bytes(wl):
     return wl.B * (n_c * per_entry + q)
 
 
-def step_bytes(wl):
-    """Algorithmic HBM bytes of one decode step (both layers), compression
-    averaged over the 128-step window (32 CSA entries and 1 HCA entry)."""
+def call_bytes(wl):
+    """Algorithmic bytes of one call of each kind in a decode step: what the
+    definition must read and write once (a KV entry is 448 FP8 codes, 7 fp32
+    block scales and 64 BF16 RoPE values = 604 bytes; an indexer key 128 codes
+    and one or two scales).  The selection's scores live in L2."""
     entry = wl.d_nope + 2 * wl.d_rope + 4 * (wl.d_nope // 64)
     ik = wl.d_I + 4 * _ik_scales(wl)
+    n_c = wl.T // wl.csa_stride
     n_h = wl.T // wl.hca_stride
     q = wl.Hq * wl.D * 2
     out = wl.Hq * wl.D * 4 + wl.Hq * 4
-    csa = indexer_bytes(wl) + wl.B * (4 * wl.k + (wl.k + wl.window) * entry + q + out)
-    hca = wl.B * ((n_h + wl.window) * entry + q + out)
-    compress = wl.B * ((PERIOD // wl.csa_stride) * (wl.csa_pool * (entry + ik) + entry + ik)
-                       + (PERIOD // wl.hca_stride) * (wl.hca_pool * entry + entry)) / PERIOD
-    return int(csa + hca + compress)
+    return {
+        "csa_compress": wl.B * (wl.csa_pool * (entry + ik) + entry + ik) + 4 * (wl.D + wl.csa_pool),
+        "indexer_score": indexer_bytes(wl),
+        "indexer_select": wl.B * (4 * n_c + 8 * wl.k),
+        "csa_attention": wl.B * (4 * wl.k + (wl.k + wl.window) * entry + q + out),
+        "hca_compress": wl.B * (wl.hca_pool * entry + entry) + 4 * (wl.D + wl.hca_pool),
+        "hca_attention": wl.B * ((n_h + wl.window) * entry + q + out),
+    }
 
 
-def _time_decode(args, wl, rank, world, dev, steps, seed0, clocks=True):
+def step_bytes(wl):
+    """Algorithmic HBM bytes of one decode step (both layers), compression
+    averaged over the 128-step window (32 CSA entries and 1 HCA entry)."""
+    cb = call_bytes(wl)
+    fixed = sum(cb[n] for n in ("indexer_score", "csa_attention", "hca_attention"))
+    fixed += wl.B * 4 * wl.k          # the selection's output (its scores stay in L2)
+    compress = ((PERIOD // wl.csa_stride) * cb["csa_compress"]
+                + (PERIOD // wl.hca_stride) * cb["hca_compress"]) / PERIOD
+    return int(fixed + compress)
+
+
+def per_call_report(wl, samples, peak):
+    """Per-call mean duration and achieved bytes/s against the HBM peak."""
+    cb = call_bytes(wl)
+    out = {}
+    for name in CALLS:
+        v = samples.get(name)
+        if not v:
+            continue
+        us = float(np.mean(v)) * 1e3
+        gbs = cb[name] / (us * 1e-6) / 1e9
+        out[name] = {"us": round(us, 3), "us_median": round(float(np.median(v)) * 1e3, 3),
+                     "samples": len(v), "algorithmic_bytes": int(cb[name]),
+                     "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    return out
+
+
+def _time_decode(args, wl, rank, world, dev, steps, seed0, clocks=True, call_replays=None):
     """Build the rotating replicas of `wl`, warm up, capture the step graph and
     time exactly `steps` steps (max over ranks).  Returns the timing record."""
     per_rep_bytes = step_bytes(wl)
@@ -364,7 +449,18 @@ def _time_decode(args, wl, rank, world, dev, steps, seed0, clocks=True):
         torch.distributed.barrier()
     clk = sampler.stop() if sampler else None
     ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
-    return {"ms": ms, "steps": n_launch * G + rest, "idx_ms": float(np.mean(graph.indexer_ms())),
+    idx = graph.indexer_ms()
+    # every call on its own: events before and after each call of PERIOD steps
+    # (each replica set in turn, so the inputs still come from HBM), replayed
+    calls = {}
+    n_rep = args.call_replays if call_replays is None else call_replays
+    if n_rep > 0:
+        cg = CallGraph(replicas, PERIOD, stream)
+        for _ in range(n_rep):
+            cg.run(calls)
+        del cg
+    return {"ms": ms, "steps": n_launch * G + rest, "idx_ms": float(np.mean(idx)),
+            "idx_samples": len(idx), "calls": calls,
             "clocks": clk, "replicas": replicas, "R": R, "sched": sched,
             "per_rep_bytes": per_rep_bytes,
             "launches": graph.kernels * n_launch + (tail.kernels if tail else 0)}
@@ -374,7 +470,8 @@ def _other_layout(args, wl, rank, world, dev):
     """The same step with the other FP8 indexer scale layout, timed briefly:
     the layout comparison rides along with the headline number."""
     other = wl.with_(ik_fmt="e4m3" if wl.ik_fmt == "e4m3vec" else "e4m3vec")
-    t = _time_decode(args, other, rank, world, dev, args.alt_steps, 5000, clocks=False)
+    t = _time_decode(args, other, rank, world, dev, args.alt_steps, 5000, clocks=False,
+                     call_replays=0)
     ib = indexer_bytes(other)
     peak, _ = _peaks()
     achieved = ib / (t["idx_ms"] / 1e3) / 1e9
@@ -410,11 +507,13 @@ def run_ours(args, rank, world, dev):
                           "call, one launch)",
                 "peak_kind": f"{peak_kind} HBM copy bandwidth (burst)",
                 "algorithmic_bytes_per_launch": ib, "avg_launch_us": round(idx_ms * 1e3, 3),
-                "timed_launches": f"every {EVENT_EVERY}th step of the last graph replay, "
+                "samples": t["idx_samples"],
+                "timed_launches": f"every {EVENT_EVERY}nd step of the last timed graph replay, "
                                   f"events on a side stream (no serialisation of the step)"}
-    traffic = _profile_traffic(args.workload) if wl.ik_fmt == "e4m3vec" else None
+    traffic = _profile_traffic("indexer_tc_kernel", wl)
     if traffic is not None:
         roofline["traffic"] = traffic
+    kernels = per_call_report(wl, t["calls"], peak)
 
     res = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
            "steps": steps_done, "warmup": args.warmup, "ms_per_step": ms / steps_done,
@@ -432,6 +531,12 @@ def run_ours(args, rank, world, dev):
                             f"touched per cycle (> 4x L2)",
                       "step_bytes": per_rep_bytes},
            "roofline": roofline,
+           "kernels": {"per_call": kernels,
+                       "how": f"each call alone (events before and after it on the step's "
+                              f"stream), {args.call_replays} replays of a {PERIOD}-step graph "
+                              f"over the rotating replicas; frac = algorithmic bytes / time / "
+                              f"{peak_kind} HBM copy bandwidth (the selection's scores are "
+                              f"L2-resident)"},
            "gpu_launches": t["launches"],
            "clocks": clocks}
     del t
@@ -440,27 +545,24 @@ def run_ours(args, rank, world, dev):
     return res, replicas, wl
 
 
-_TRAFFIC_SOURCES = ["indexer.cu", "indexer_tc.cu", "topk_common.cuh", "sm100.cuh", "cskv_internal.cuh"]
-
-
-def _profile_traffic(workload):
-    """DRAM bytes per indexer scoring launch from the committed ncu summary, when
-    the kernel sources still hash to the ones the counters were taken on
-    (null otherwise: the counters describe another build)."""
+def _profile_traffic(kernel, wl):
+    """DRAM bytes per launch of `kernel` on this workload from the committed
+    ncu record (profiles/ncu_traffic.json), when the kernel's sources still
+    hash to the ones the counters were taken on; None otherwise (the
+    counters describe another build)."""
     import hashlib
-    import re
-    p = os.path.join(ROOT, "profiles", f"indexer_tc_{workload}_decode.md")
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
-    text = open(p).read()
-    m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
-    m_h = re.search(r"^traffic_sources_sha256_16:\s*([0-9a-f]+)", text, re.M)
-    if not (m_t and m_h):
+    rec = json.load(open(p)).get(kernel)
+    if not rec or rec.get("workload") != wl.name or rec.get("ik_fmt", wl.ik_fmt) != wl.ik_fmt:
         return None
     h = hashlib.sha256()
-    for f in _TRAFFIC_SOURCES:
+    for f in rec["sources"]:
         h.update(open(os.path.join(ROOT, "compressed_sparse_kv_softmax_b200", "csrc", f), "rb").read())
-    return int(m_t.group(1)) if h.hexdigest()[:16] == m_h.group(1) else None
+    if h.hexdigest()[:16] != rec["sources_sha256_16"]:
+        return None
+    return int(rec["dram_bytes_per_launch"])
 
 
 def _pack(tensors, device, pin=False):
@@ -477,54 +579,74 @@ def _pack(tensors, device, pin=False):
 
 
 def run_e2e(args, replicas, wl, dev, world):
-    """Same metric through the public API with per-step host<->device copies:
-    the new token's raw KV and indexer key (into their ring slots), q, the
-    indexer query and scales, head weights and the step's positions go in from
-    pinned host memory; out and lse of both layers come back.  The step's
-    small inputs sit in one contiguous buffer (one copy), the outputs too."""
+    """Same metric through the public API with per-step host<->device copies.
+    Every step: one host->device copy of the step's inputs from pinned host
+    memory (both layers' queries, the indexer query, its scales and head
+    weights, the positions, and the new token's raw KV and indexer key), the
+    cskv_ring_store call that appends that token to the step's rings, the
+    layer calls (csa_compress, indexer_topk, hybrid_attn_decode, hca_compress,
+    hybrid_attn_decode), and one device->host copy of both layers' outputs.
+    Steps rotate over the same replicas as the timed graph (HBM-resident
+    inputs, more than 4x L2), eager calls on one stream."""
+    import compressed_sparse_kv_softmax_b200 as C
     K = max(3, min(args.steps, args.e2e_steps))
-    rep = replicas[0]
-    sc = rep.sched
-    cl, hl = rep.csa_L, rep.hca_L
-    cap = cl["ring_k"]["cap"]
+    sc = replicas[0].sched
+    cl0, hl0 = replicas[0].csa_L, replicas[0].hca_L
+    cap = cl0["ring_k"]["cap"]
 
-    def ring_slots(s):
+    def token(L, key, s):
+        # the new token of position T0 + s: its ring slot's planes, as a
+        # one-slot cache per sequence
         slot = (sc.T0 + s) % cap
-        ins = [Ld["ring_k"][key][:, slot] for Ld in (cl, hl) for key in ("data", "scale", "rope")]
-        return ins + [cl["ring_ik"]["data"][:, slot], cl["ring_ik"]["scale"][:, slot]]
+        c = L[key]
+        return [c[p][:, slot:slot + 1] for p in ("data", "scale", "rope") if c.get(p) is not None]
 
-    # the step's small inputs: both layers' queries, the indexer query, its
-    # scales and head weights, and the positions; the layers read them from
-    # views of one device buffer
-    small = [cl["q"], hl["q"], cl["q_ik"], cl["q_ik_scale"], cl["head_w"], sc.q_pos[0],
-             sc.ctx[0], sc.tb[0], sc.te[0]]
-    dev_buf, views = _pack(small, dev)
-    for v, t in zip(views, small):
-        v.copy_(t)
-    cl["q"], hl["q"], cl["q_ik"], cl["q_ik_scale"], cl["head_w"] = views[:5]
-    pos = tuple(views[5:])
+    def small(s):
+        return ([cl0["q"], hl0["q"], cl0["q_ik"], cl0["q_ik_scale"], cl0["head_w"], sc.q_pos[s],
+                 sc.ctx[s], sc.tb[s], sc.te[s]] + token(cl0, "ring_k", s) + token(hl0, "ring_k", s)
+                + token(cl0, "ring_ik", s))
+
+    dev_buf, views = _pack(small(0), dev)
+    q_c, q_h, q_ik, q_ik_s, head_w, q_pos, ctx, tb, te = views[:9]
+    tok = views[9:]
+
+    def one_slot(c, planes):
+        d = {k: c[k] for k in ("fmt", "d_nope", "d_rope")}
+        d.update(ring=False, cap=1, data=planes[0], scale=planes[1],
+                 rope=planes[2] if len(planes) > 2 else None)
+        return d
+
+    src = [one_slot(cl0["ring_k"], tok[0:3]), one_slot(hl0["ring_k"], tok[3:6]),
+           one_slot(cl0["ring_ik"], tok[6:8])]
+    src = [C.cache_struct(c) for c in src]
+    # every replica's layers read the step's inputs from the staging views and
+    # write their outputs into one output buffer
+    out_buf, out_views = _pack([replicas[0].csa.out, replicas[0].csa.lse, replicas[0].hca.out,
+                                replicas[0].hca.lse], dev)
+    rings = []
+    for rep in replicas:
+        cl, hl = rep.csa_L, rep.hca_L
+        cl["q"], hl["q"], cl["q_ik"], cl["q_ik_scale"], cl["head_w"] = q_c, q_h, q_ik, q_ik_s, head_w
+        rep.csa.out, rep.csa.lse, rep.hca.out, rep.hca.lse = out_views
+        rings.append([rep.csa.cs["ring_k"], rep.hca.cs["ring_k"], rep.csa.cs["ring_ik"]])
     host_small = []
     for s in range(PERIOD):
-        hb, hv = _pack(small, "cpu", pin=True)
-        for v, t in zip(hv, [cl["q"], hl["q"], cl["q_ik"], cl["q_ik_scale"], cl["head_w"],
-                             sc.q_pos[s], sc.ctx[s], sc.tb[s], sc.te[s]]):
+        hb, hv = _pack(small(s), "cpu", pin=True)
+        for v, t in zip(hv, small(s)):
             v.copy_(t.cpu())
         host_small.append(hb)
-    dev_ring = [ring_slots(s) for s in range(PERIOD)]
-    host_ring = [[t.detach().cpu().pin_memory() for t in ins] for ins in dev_ring]
-    # outputs of both layers in one buffer
-    out_buf, out_views = _pack([rep.csa.out, rep.csa.lse, rep.hca.out, rep.hca.lse], dev)
-    rep.csa.out, rep.csa.lse, rep.hca.out, rep.hca.lse = out_views
     host_out = torch.empty(out_buf.shape, dtype=torch.uint8, pin_memory=True)
-    bi = host_small[0].numel() + sum(t.numel() * t.element_size() for t in host_ring[0])
+    bi = host_small[0].numel()
     bo = host_out.numel()
     stream = torch.cuda.Stream(device=dev)
+    pos = (q_pos, ctx, tb, te)
+    R = len(replicas)
 
     def one(i):
         s = i % PERIOD
+        rep = replicas[i % R]
         dev_buf.copy_(host_small[s], non_blocking=True)
-        for d, h in zip(dev_ring[s], host_ring[s]):
-            d.copy_(h, non_blocking=True)
+        C.ring_store(wl.B, tb, src, rings[i % R])
         rep.step(s, pos=pos, split_select=False)
         host_out.copy_(out_buf, non_blocking=True)
 
@@ -545,10 +667,11 @@ def run_e2e(args, replicas, wl, dev, world):
     ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
     return {"value": round(whole_job_rate(wl.B * K, ms, world), 2), "unit": UNIT,
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "steps": K,
-            "path": "eager public API calls (no graph: csa_compress, indexer_topk, "
-                    "hybrid_attn_decode, hca_compress, hybrid_attn_decode), single replica, "
-                    "same decode window; per step one copy of the small inputs, 8 ring-slot "
-                    "copies, one copy of both layers' outputs"}
+            "path": f"eager public API calls on one stream (cskv_ring_store, csa_compress, "
+                    f"indexer_topk, hybrid_attn_decode, hca_compress, hybrid_attn_decode), "
+                    f"{R} rotating replicas as in the timed region; per step one pinned "
+                    f"host->device copy of all inputs and one device->host copy of both "
+                    f"layers' outputs"}
 
 
 # ------------------------------------------------------------- the oracle
@@ -785,6 +908,8 @@ def main():
     ap.add_argument("--tq", type=int, default=0,
                     help="prefill: new tokens per sequence (0: the workload's chunk); a "
                          "shorter chunk is a smaller case of the same step, for profiling")
+    ap.add_argument("--call-replays", type=int, default=4,
+                    help="replays of the per-call timing graph (0: skip)")
     ap.add_argument("--alt-steps", type=int, default=4096,
                     help="steps timed with the other indexer layout (0: skip)")
     args = ap.parse_args()

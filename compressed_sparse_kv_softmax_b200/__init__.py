@@ -62,6 +62,8 @@ _lib.indexer_topk_noalloc.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC, _I, _
                                       _P, _P]
 _lib.indexer_topk_noalloc.restype = _I
 _lib.cskv_noalloc_scratch_bytes.restype = _SZ
+_lib.cskv_ring_store.argtypes = [_I, _P, _I, ctypes.POINTER(_PC), ctypes.POINTER(_PC), _P]
+_lib.cskv_ring_store.restype = _I
 _lib.cskv_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
 _lib.cskv_check_device_errors.restype = _I
 _lib.cskv_debug_topk_barrier_spins.argtypes = [ctypes.c_uint32]
@@ -128,6 +130,17 @@ def _stream(stream):
         return ctypes.c_void_p(stream)
     import torch
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def ring_store(B, pos, src, ring, stream=None):
+    """Copies each sequence's new token (slot 0 of every cache in `src`) into
+    slot pos[b] % cap of the matching raw ring in `ring` (lists of caches)."""
+    ss = [cache_struct(c) for c in src]
+    rs = [cache_struct(c) for c in ring]
+    n = len(ss)
+    sp = (_PC * n)(*[ctypes.pointer(c) for c in ss])
+    rp = (_PC * n)(*[ctypes.pointer(c) for c in rs])
+    _check(_lib.cskv_ring_store(B, _ptr(pos), n, sp, rp, _stream(stream)), "cskv_ring_store")
 
 
 def indexer_workspace_size(B, Tq, max_entries, k) -> int:

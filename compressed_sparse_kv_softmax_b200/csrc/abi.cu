@@ -206,6 +206,22 @@ int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
                          stride, out_k, out_v, nullptr, stream);
 }
 
+int cskv_ring_store(int B, const int64_t *pos, int n, const cskv_cache *const *src,
+                    const cskv_cache *const *ring, cskv_stream_t stream) {
+  if (B < 0 || B > 65535 || n < 1 || n > 8) return CSKV_ERR_ARG;
+  if (B == 0) return CSKV_OK;
+  if (!pos || !src || !ring) return CSKV_ERR_ARG;
+  Cache s[8], r[8];
+  for (int i = 0; i < n; ++i) {
+    CSKV_TRY(check_cache(src[i], 0));
+    CSKV_TRY(check_cache(ring[i], 1));
+    if (!same_layout(src[i], ring[i])) return CSKV_ERR_ARG;
+    s[i] = to_dev(src[i]);
+    r[i] = to_dev(ring[i]);
+  }
+  return launch_ring_store(B, pos, n, s, r, (cudaStream_t)stream);
+}
+
 size_t cskv_indexer_workspace_size(int B, int Tq, int64_t max_entries, int k) {
   if (B <= 0 || Tq <= 0 || max_entries < 0) return 0;
   return indexer_ws_bytes(B, Tq, max_entries, k);

@@ -95,10 +95,16 @@ __host__ __device__ inline ScaleSpan scale_span(long long g0, long long rows, in
   return sp;
 }
 
-// Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
+// Order-preserving map of an fp32 score to uint32 (larger score -> larger key):
+// negative values have every bit flipped, others only the sign bit, so
+// -inf < finite < +inf, with NaN patterns beyond the infinities of their
+// sign (the canonical NaN of fp32 arithmetic is positive).  Written
+// branch-free with an arithmetic shift: the equivalent select on the sign bit
+// was measured to map NaN to its own bit pattern (the key of -0.0's
+// neighbourhood) in this toolchain's code for sm_100a.
 __device__ __forceinline__ uint32_t score_key(float s) {
-  uint32_t u = __float_as_uint(s);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const uint32_t u = __float_as_uint(s);
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -188,6 +194,9 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
                     const float *gate_w, const float *gate_b, int pool, int stride,
                     const Cache &out_k, const Cache &out_v, const Cache &out_ik,
                     cudaStream_t st);
+
+int launch_ring_store(int B, const int64_t *pos, int n, const Cache *src, const Cache *ring,
+                      cudaStream_t st);
 
 struct IndexerArgs {
   int B, Tq, H_I, d_I, stride, k;

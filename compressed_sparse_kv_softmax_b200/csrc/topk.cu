@@ -691,8 +691,11 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
     return;
   }
   // inconsistent histogram or candidate overflow (never expected with the
-  // scoring kernel's histogram): the row's first CTA selects the whole row
-  if (me == 0) topk_row_single_cta(s, n, k, oi, os, status);
+  // scoring kernel's histogram): the row's first CTA selects the whole row.
+  // A CTA that gave up at the meeting point cannot know whether the others
+  // write their slices, so it selects the whole row too (every writer of a
+  // slot writes the same exact value).
+  if (me == 0 || sm.state != 0) topk_row_single_cta(s, n, k, oi, os, status);
 }
 
 void launch_topk_rows(const float *scores, long long ld, const int64_t *q_pos, int stride,

@@ -153,6 +153,24 @@ int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
                  const cskv_cache *out_k, const cskv_cache *out_v, cskv_stream_t stream);
 
 /*
+ * cskv_ring_store - appends one new raw token per sequence to raw-token
+ * rings: for each ring i and sequence b, the token held in slot 0 of
+ * sequence b of src[i] (a cache of cap >= 1 slots per sequence, ring = 0)
+ * is copied into slot pos[b] % cap of ring[i] (ring = 1), every plane
+ * (codes, scales, RoPE) byte for byte.  This is the cache append that
+ * precedes csa_compress / hca_compress and the window's attention; the pages
+ * keep the last 128 raw tokens for the sliding window («Chinas
+ * KI-Unabhaengigkeit?: Bei Deepseek V4 haben kleine Aenderungen grosse
+ * Wirkung», "Komprimierte Erinnerung fuer laengere Kontexte").
+ *   pos       : [B] device int64, position of each sequence's new token.
+ *   n         : number of (src, ring) pairs, 1 <= n <= 8; each pair has one
+ *               layout (fmt, d_nope, d_rope) and its planes' alignments.
+ * No ring may also be another pair's ring or source.
+ */
+int cskv_ring_store(int B, const int64_t *pos, int n, const cskv_cache *const *src,
+                    const cskv_cache *const *ring, cskv_stream_t stream);
+
+/*
  * indexer_topk - lightning-indexer scores of every visible CSA entry and the
  * top-k selection per query row.
  *   s_j = sum_h head_w[h] * max(0, q_ik[h] . k_ik[j])       (per query row)

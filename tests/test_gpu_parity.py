@@ -132,7 +132,7 @@ def test_indexer_any_scale_plane_layout(C, ik_fmt, pad_cols, Tq):
         wide[..., : sc.shape[2]] = sc
         Ld["comp_ik"]["scale"] = wide[..., : sc.shape[2]]
     layer = _run_indexer(C, Ld)
-    rows = sample_rows(wl.B, wl.Tq, n=12)
+    rows = sample_rows(wl.B, wl.Tq)
     ref = O.layer_indexer_topk(L, wl.k, rows=rows)
     idx = layer.idx.cpu().numpy()
     for (b, t), (ridx, rs) in ref.items():
@@ -487,3 +487,42 @@ def test_end_to_end_tiny_pipeline(C):
             (ro, rl), = O.layer_attention(Lo, sel=None).values()
             check_attention(out[0, 0].cpu().numpy(), lse[0, 0].cpu().numpy(), ro, rl,
                             where="e2e hca")
+
+
+# ---------------------------------------------------------------- ring store
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e4m3vec", "f32"])
+def test_ring_store_appends_each_sequence_token(C, fmt):
+    # byte work: the ring slot pos % cap of every sequence holds exactly the
+    # new token's bytes afterwards, every other slot is untouched
+    B, cap = 3, 128
+    g = torch.Generator(device="cpu").manual_seed(5)
+    d_nope, d_rope = (448, 64) if fmt == "e4m3" else ((128, 0) if fmt == "e4m3vec" else (64, 64))
+
+    def cache(n, ring):
+        c = {"fmt": fmt, "d_nope": d_nope, "d_rope": d_rope, "ring": ring, "cap": n}
+        if fmt == "f32":
+            c["data"] = torch.randn(B, n, d_nope + d_rope, generator=g)
+        else:
+            c["data"] = torch.randint(0, 255, (B, n, d_nope), dtype=torch.uint8, generator=g)
+            nb = 8 if fmt == "e4m3" else 1
+            c["scale"] = torch.rand(B, n, nb, generator=g)
+            if d_rope:
+                c["rope"] = torch.randn(B, n, d_rope, generator=g).to(torch.bfloat16)
+        return c
+
+    ring, src = cache(cap, True), cache(1, False)
+    pos = torch.tensor([5, 127 + 128 * 9, 1_048_575], dtype=torch.int64)
+    ring_d = to_device(ring)
+    C.ring_store(B, pos.cuda(), [to_device(src)], [ring_d])
+    torch.cuda.synchronize()
+    slots = O.ring_slots(pos.numpy(), cap)
+    for p in ("data", "scale", "rope"):
+        if p not in ring:
+            continue
+        want = ring[p].clone()
+        for b in range(B):
+            want[b, slots[b]] = src[p][b, 0]
+        got = ring_d[p].cpu()
+        assert torch.equal(got.view(torch.uint8) if got.dtype != torch.uint8 else got,
+                           want.view(torch.uint8) if want.dtype != torch.uint8 else want), p

@@ -43,8 +43,8 @@ def test_noalloc_matches_workspace_entry_point_twice():
     ref.select()
     torch.cuda.synchronize()
     want = (ref.idx.cpu().numpy(), ref.score.cpu().numpy())
-    # a call of another shape (many rows of one sequence, other entry count)
-    wl2 = W.get("parity_prefill")
+    # a call of another shape (40 rows of one sequence, other entry count)
+    wl2 = W.get("parity_prefill").with_(Tq=40)
     Ld2 = to_device(W.make_csa_layer(wl2))
     ref2 = CSALayer(Ld2)
     ref2.select()
