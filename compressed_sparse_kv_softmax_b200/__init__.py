@@ -68,6 +68,8 @@ _lib.cskv_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32)]
 _lib.cskv_check_device_errors.restype = _I
 _lib.cskv_debug_topk_barrier_spins.argtypes = [ctypes.c_uint32]
 _lib.cskv_debug_topk_barrier_spins.restype = ctypes.c_uint32
+_lib.cskv_debug_indexer_stall.argtypes = [ctypes.c_uint32]
+_lib.cskv_debug_indexer_stall.restype = ctypes.c_uint32
 _lib.cskv_error_string.argtypes = [_I]
 _lib.cskv_error_string.restype = ctypes.c_char_p
 _lib.cskv_version.restype = _I
@@ -261,6 +263,13 @@ def debug_topk_barrier_spins(spins: int) -> int:
     """Polls of the multi-CTA selection's row meeting point before a CTA
     gives up (tests of the failure path); returns the previous setting."""
     return int(_lib.cskv_debug_topk_barrier_spins(int(spins)))
+
+
+def debug_indexer_stall(polls: int) -> int:
+    """Test hook of the failure path (see cskv_debug_indexer_stall): with
+    polls > 0 the first scoring CTA misses a tile and its waits run out after
+    `polls` polls; 0 switches it off.  Returns the previous setting."""
+    return int(_lib.cskv_debug_indexer_stall(int(polls)))
 
 
 def error_string(status: int) -> str:

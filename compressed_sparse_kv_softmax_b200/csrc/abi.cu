@@ -182,6 +182,7 @@ int indexer_common(int phases, int B, int Tq, const int64_t *q_pos, const void *
   a.ws = ws; a.ws_bytes = ws_bytes;
   a.status = device_status_word();
   if (!a.status) return CSKV_ERR_CUDA;
+  a.stall_polls = indexer_stall_polls();
   return launch_indexer_topk(a, phases, (cudaStream_t)stream);
 }
 

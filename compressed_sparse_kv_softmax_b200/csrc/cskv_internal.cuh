@@ -183,6 +183,9 @@ unsigned int *device_status_word();
 __device__ __forceinline__ void record_event(unsigned int *status, unsigned int bit) {
   if (status) atomicOr(status, bit);
 }
+// Test hook (cskv_debug_indexer_stall): mbarrier polls that bound every wait
+// of a scoring launch whose first CTA leaves out its first tile (0: off).
+uint32_t indexer_stall_polls();
 // Polls of the multi-CTA selection's row meeting point before a CTA gives up
 // (each poll backs off ~0.1-1 us, so the default is seconds).
 constexpr uint32_t kDefaultBarrierSpins = 1u << 22;
@@ -207,6 +210,7 @@ struct IndexerArgs {
   int32_t *out_idx; float *out_score;
   void *ws; size_t ws_bytes;
   unsigned int *status;    // device status word
+  uint32_t stall_polls;    // test hook: 0, or the wait bound of a stalled first CTA
 };
 size_t indexer_ws_bytes(int B, int Tq, long long max_entries, int k);
 // phases of an indexer call: scoring (with the selection histogram) and the

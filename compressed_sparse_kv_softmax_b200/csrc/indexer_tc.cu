@@ -121,6 +121,10 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   __syncthreads();                 // barriers initialised, TMEM address published
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // wait bound (test hook: a short one, and CTA 0 of row 0 leaves out its
+  // first tile, so that its waits run out with nothing in flight)
+  const uint32_t lim = a.stall_polls ? a.stall_polls : kWaitLimit;
+  const bool drop_first = a.stall_polls && blockIdx.x == 0 && row == 0;
   pdl_wait();                      // global memory from here on
   pdl_trigger();
   // the selection's per-row counters start at zero (the selection runs after
@@ -176,6 +180,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
     const long long total_rows = (long long)a.B * a.ik.cap;
     if (elect_one()) {
       auto issue = [&](int i) {
+        if (drop_first && i == 0) return;
         const int s = i % kStages;
         const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
         const long long g0 = (long long)b * a.ik.cap + j0;    // first row of the tile
@@ -199,7 +204,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       for (int i = spec; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages;
         const uint32_t ph = (i / kStages) & 1;
-        if (!mbar_wait(&sm.empty[s], ph ^ 1)) {
+        if (!mbar_wait(&sm.empty[s], ph ^ 1, lim)) {
           record_abort(sm);
           break;
         }
@@ -208,7 +213,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       }
       // never leave while a copy into this CTA's shared memory is in flight
       for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_wait(&sm.full[i % kStages], (i / kStages) & 1);
+        mbar_wait(&sm.full[i % kStages], (i / kStages) & 1, lim);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -217,11 +222,11 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       int done = 0;
       for (int i = 0; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages, acc = i % kAcc;
-        if (i >= kAcc && !mbar_wait(&sm.acc_empty[acc], ((i / kAcc) & 1) ^ 1)) {
+        if (i >= kAcc && !mbar_wait(&sm.acc_empty[acc], ((i / kAcc) & 1) ^ 1, lim)) {
           record_abort(sm);
           break;
         }
-        if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
+        if (!mbar_wait(&sm.full[s], (i / kStages) & 1, lim)) {
           record_abort(sm);
           break;
         }
@@ -244,7 +249,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       }
       // every MMA of this CTA has finished before TMEM is released
       mma_commit(&sm.mma_done);
-      if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm);
+      if (!mbar_wait(&sm.mma_done, 0, lim)) record_abort(sm);
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: the warpgroups take tiles in turn
@@ -260,7 +265,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       const int acc = i % kAcc;
       const int s = i % kStages;
       const long long j = (long long)(blockIdx.x + i * gridDim.x) * kTile + r;
-      if (!mbar_wait(&sm.acc_full[acc], (i / kAcc) & 1)) {
+      if (!mbar_wait(&sm.acc_full[acc], (i / kAcc) & 1, lim)) {
         record_abort(sm);
         break;
       }
@@ -269,7 +274,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       // before this warpgroup arrives on its empty barrier, so the wait on
       // the stage's full barrier (for visibility of the copy) returns at once.
       // An odd last row of the whole cache came without them: plain load.
-      mbar_wait(&sm.full[s], (i / kStages) & 1);
+      mbar_wait(&sm.full[s], (i / kStages) & 1, lim);
       float sk0 = 1.f, sk1 = 0.f;            // (rows past n: score not stored)
       if (j < n) {
         const long long g = (long long)b * a.ik.cap + j;

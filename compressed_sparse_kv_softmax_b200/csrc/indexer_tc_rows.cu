@@ -156,6 +156,13 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
   __syncthreads();                 // barriers initialised, TMEM address published
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // wait bound (test hook: short waits, and the first CTA leaves out its
+  // first tile, so that its waits run out with nothing in flight)
+  const uint32_t lim = a.stall_polls ? a.stall_polls : kWaitLimit;
+  const bool drop_first = a.stall_polls && blockIdx.x == 0 && blockIdx.y == 0;
+  auto wait_long = [&](uint64_t *bar, uint32_t parity) {
+    return a.stall_polls ? mbar_wait(bar, parity, lim) : mbar_wait_sleep(bar, parity);
+  };
   pdl_wait();                      // global memory from here on
   pdl_trigger();
   // the selection's per-row counters start at zero (the selection runs after
@@ -214,6 +221,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       const uint64_t keep = policy_evict_last();
       const long long total_rows = (long long)a.B * a.ik.cap;
       auto issue = [&](int i) {
+        if (drop_first && i == 0) return;
         const int s = i % kStages;
         const long long j0 = ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile;
         const long long g0 = (long long)b * a.ik.cap + j0;     // first cache row of the tile
@@ -238,7 +246,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       const int my_tiles = tiles_of(nmax);
       for (int i = spec; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages;
-        if (!mbar_wait_sleep(&sm.empty[s], ((i / kStages) & 1) ^ 1)) {
+        if (!wait_long(&sm.empty[s], ((i / kStages) & 1) ^ 1)) {
           record_abort(sm);
           break;
         }
@@ -247,7 +255,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       }
       // never leave while a copy into this CTA's shared memory is in flight
       for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_wait(&sm.full[i % kStages], (i / kStages) & 1);
+        mbar_wait(&sm.full[i % kStages], (i / kStages) & 1, lim);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -258,7 +266,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       const uint32_t qa = smem_addr(sm.q);
       for (int i = 0; i < my_tiles && !sm.abort; ++i) {
         const int s = i % kStages;
-        if (!mbar_wait_sleep(&sm.full[s], (i / kStages) & 1)) {
+        if (!wait_long(&sm.full[s], (i / kStages) & 1)) {
           record_abort(sm);
           break;
         }
@@ -266,7 +274,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
         bool ok = true;
         for (int h = 0; h < halves; ++h) {
           // the epilogue has drained this half's accumulator of the last tile
-          if (i > 0 && !mbar_wait_sleep(&sm.acc_empty[h], (i - 1) & 1)) {
+          if (i > 0 && !wait_long(&sm.acc_empty[h], (i - 1) & 1)) {
             record_abort(sm);
             ok = false;
             break;
@@ -284,7 +292,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       }
       // every MMA of this CTA has finished before TMEM is released
       mma_commit(&sm.mma_done);
-      if (!mbar_wait(&sm.mma_done, 0)) record_abort(sm);
+      if (!mbar_wait(&sm.mma_done, 0, lim)) record_abort(sm);
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: warpgroup eg takes row eg of each half
@@ -310,7 +318,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       const int j = jt + r;
       // the tile's scales arrived with its keys (the stage is not refilled
       // before this warp arrives on its empty barrier)
-      if (!mbar_wait_sleep(&sm.full[s], (i / kStages) & 1)) {
+      if (!wait_long(&sm.full[s], (i / kStages) & 1)) {
         record_abort(sm);
         break;
       }
@@ -330,7 +338,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       if (lane == 0) mbar_arrive(&sm.empty[s]);
       bool stop = false;
       for (int h = 0; h < halves; ++h) {
-        if (!mbar_wait_sleep(&sm.acc_full[h], i & 1)) {
+        if (!wait_long(&sm.acc_full[h], i & 1)) {
           record_abort(sm);
           stop = true;
           break;

@@ -1,4 +1,5 @@
-// Sticky per-device status word and the test knob of the top-k meeting point.
+// Sticky per-device status word and the test hooks of the failure paths (the
+// selection's meeting-point poll limit, a stalled scoring CTA).
 //
 // Every wait inside a kernel of the library is bounded.  When one runs out,
 // the kernel ORs a CSKV_DEV_* bit into this word, marks its results invalid
@@ -23,6 +24,7 @@ __global__ void status_take_kernel() { g_status_taken = atomicExch(&g_status, 0u
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned int *g_status_ptr[kMaxDevices] = {};
+std::atomic<uint32_t> g_indexer_stall{0};
 std::atomic<uint32_t> g_barrier_spins{kDefaultBarrierSpins};
 
 }  // namespace
@@ -45,6 +47,7 @@ unsigned int *device_status_word() {
   return g_status_ptr[dev];
 }
 
+uint32_t indexer_stall_polls() { return g_indexer_stall.load(std::memory_order_relaxed); }
 uint32_t topk_barrier_spins() { return g_barrier_spins.load(std::memory_order_relaxed); }
 
 }  // namespace cskv
@@ -72,6 +75,10 @@ int cskv_check_device_errors(cskv_stream_t stream, uint32_t *events) {
 
 uint32_t cskv_debug_topk_barrier_spins(uint32_t spins) {
   return cskv::g_barrier_spins.exchange(spins);
+}
+
+uint32_t cskv_debug_indexer_stall(uint32_t polls) {
+  return cskv::g_indexer_stall.exchange(polls);
 }
 
 }  // extern "C"

@@ -72,7 +72,8 @@ enum {
   CSKV_DEV_INDEXER_WAIT = 1,  /* a scoring CTA gave up waiting on its copy / MMA pipeline;
                                  its scores read NaN and its rows are reported failed */
   CSKV_DEV_TOPK_BARRIER = 2,  /* the selection's per-row meeting point timed out; the row was
-                                 selected by one CTA from its scores (result unchanged) */
+                                 selected from its scores by each CTA that gave up
+                                 (result unchanged) */
   CSKV_DEV_ATTN_WAIT = 4,     /* an attention CTA gave up waiting on its copies / MMAs;
                                  the affected rows' lse is NaN */
   CSKV_DEV_ROW_FAILED = 8     /* the selection met a row with a NaN score; that row's
@@ -320,13 +321,27 @@ int cskv_check_device_errors(cskv_stream_t stream, uint32_t *events);
 /*
  * cskv_debug_topk_barrier_spins - sets how many times a CTA of the multi-CTA
  * top-k selection polls its row's meeting point before it gives up (default
- * 4,194,304, i.e. seconds), and returns the previous setting.  For tests of
+ * 4,194,304, i.e. seconds), and returns the previous setting.  Test hook of
  * the failure path: with 0 a CTA that arrives before the others gives up at
- * once, the row's first CTA then selects the whole row from its scores (the
- * result is the same) and CSKV_DEV_TOPK_BARRIER is recorded.  Affects calls
- * made afterwards in this process, on every device.
+ * once and selects the whole row from its scores (the result is the same)
+ * and CSKV_DEV_TOPK_BARRIER is recorded.  Affects later calls in this
+ * process, on every device.
  */
 uint32_t cskv_debug_topk_barrier_spins(uint32_t spins);
+
+/*
+ * cskv_debug_indexer_stall - test hook of the failure path.  With polls > 0,
+ * every later tensor-core scoring launch in this process leaves out the copy
+ * of the first key tile of its first CTA and bounds
+ * every wait of its kernel to `polls` mbarrier polls instead of seconds: that
+ * CTA's waits for the missing tile run out, nothing it issued is left in
+ * flight, it writes NaN into its score slots, and the selection reports its
+ * query rows as failed (row 0; with several query rows per sequence, the
+ * group of up to 8 rows of sequence 0 that the CTA scores), recording
+ * CSKV_DEV_INDEXER_WAIT and CSKV_DEV_ROW_FAILED.
+ * polls = 0 switches it off (the default).  Returns the previous setting.
+ */
+uint32_t cskv_debug_indexer_stall(uint32_t polls);
 
 /* Static text for a status code. */
 const char *cskv_error_string(int status);

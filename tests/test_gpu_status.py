@@ -1,9 +1,10 @@
 """Device-side failure reporting, made to happen without a GPU fault: the
 top-k meeting point is given a poll limit of zero (a CTA that arrives first
-gives up at once), and a NaN head weight makes one query row unrankable.
-The kernels must return, record the event in the device status word, and
-leave either the exact result (the meeting point) or a row visibly marked
-failed (NaN scores)."""
+gives up at once), a test hook makes the first scoring CTA miss one key tile
+(nothing is left in flight) so that its bounded waits run out, and a NaN
+head weight makes one query row unrankable.  The kernels must return, record the event in the
+device status word, and leave the affected row visibly failed (-1 indices,
+NaN scores) and every other row exact."""
 import numpy as np
 import pytest
 import torch
@@ -60,6 +61,42 @@ def test_topk_meeting_point_timeout_keeps_the_result_exact(C):
     torch.cuda.synchronize()
     idx = layer.idx.cpu().numpy()
     for (b, t), (ridx, rs) in ref.items():
+        check_topk(idx[b, t], ridx, rs, where=f"row {(b, t)}")
+    assert C.check_device_errors() == 0
+
+
+@pytest.mark.parametrize("Tq", [1, 4])
+def test_scoring_wait_runs_out_and_the_row_is_reported(C, Tq):
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    # the hook makes the first scoring CTA miss its first key tile and bounds
+    # its waits to a few thousand polls: the kernel returns, the CTA's scores
+    # read NaN, its query rows are reported failed (row 0; with several rows
+    # per sequence, the CTA's group: every row of sequence 0 here), the
+    # other rows are exact
+    wl = W.get("parity_decode").with_(Tq=Tq, prefill=Tq > 1)
+    L = W.make_csa_layer(wl)
+    layer = CSALayer(to_device(L))
+    rows = [(b, t) for b in range(wl.B) for t in range(wl.Tq)]
+    failed = [(0, t) for t in range(wl.Tq)]
+    ref = O.layer_indexer_topk(L, wl.k, rows=[r for r in rows if r not in failed])
+    old = C.debug_indexer_stall(4096)
+    try:
+        layer.select()
+        torch.cuda.synchronize()
+    finally:
+        C.debug_indexer_stall(old)
+    idx, sc = layer.idx.cpu().numpy(), layer.score.cpu().numpy()
+    for b, t in failed:
+        assert (idx[b, t] == -1).all() and np.isnan(sc[b, t]).all(), (b, t)
+    for (b, t), (ridx, rs) in ref.items():
+        check_topk(idx[b, t], ridx, rs, where=f"row {(b, t)} beside a stalled one")
+    assert C.check_device_errors() == C.DEV_INDEXER_WAIT | C.DEV_ROW_FAILED
+    # the hook off: every row exact, nothing recorded
+    layer.select()
+    torch.cuda.synchronize()
+    idx = layer.idx.cpu().numpy()
+    ref0 = O.layer_indexer_topk(L, wl.k, rows=failed)
+    for (b, t), (ridx, rs) in ref0.items():
         check_topk(idx[b, t], ridx, rs, where=f"row {(b, t)}")
     assert C.check_device_errors() == 0
 
