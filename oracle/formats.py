@@ -85,3 +85,102 @@ def bf16_encode(x) -> np.ndarray:
     q = np.where(np.abs(q) > bf16_max, np.copysign(np.inf, x), q)
     q = np.where(np.isnan(x), np.nan, q)
     return (q.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+# ------------------------------------------------------------------- MXFP4 ---
+#
+# The lightning indexer runs in FP4 («DeepSeek-V4: 1 Million Token Context
+# endlich nutzbar», section "Hybrid Attention: CSA und HCA"); the 4-bit
+# format named for DeepSeek-V4's attention is MXFP4 («Chinas
+# KI-Unabhaengigkeit?: Bei Deepseek V4 haben kleine Aenderungen grosse
+# Wirkung», introduction) and F8_E8M0 is among its stored types («DeepSeek-V4
+# Pro und Flash ...», "Modelldetails").  MXFP4 as defined by the OCP
+# Microscaling Formats (MX) Specification v1.0: blocks of 32 elements share
+# one E8M0 scale; each element is FP4 E2M1.
+#   E2M1: 1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit; exponent
+#         field 0 is subnormal (value m/2); no infinities or NaN; magnitudes
+#         0, 0.5, 1, 1.5, 2, 3, 4, 6.
+#   E8M0: an unsigned 8-bit exponent, value 2^(e - 127); e = 255 is NaN.
+# Storage here: two E2M1 codes per byte, the even element in the low nibble.
+
+E2M1_MAX = 6.0
+MX_BLOCK = 32
+
+
+def e2m1_value_table() -> np.ndarray:
+    """Value of each of the 16 E2M1 codes, from the bit-field definition."""
+    vals = np.empty(16, dtype=np.float64)
+    for code in range(16):
+        sign = -1.0 if code & 0x8 else 1.0
+        e = (code >> 1) & 0x3
+        m = code & 0x1
+        vals[code] = sign * ((m / 2.0) if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1))
+    return vals
+
+
+_E2M1 = e2m1_value_table()
+_E2M1_POS = _E2M1[:8].copy()            # codes 0..7, strictly increasing
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    return _E2M1[np.asarray(codes, dtype=np.uint8) & 0xF]
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """Round to the nearest E2M1 value, ties to the even code, saturating to
+    +-6; the sign is kept (negative values that round to zero give 0x8)."""
+    x = np.asarray(x, dtype=np.float64)
+    m = np.minimum(np.abs(x), E2M1_MAX)
+    hi = np.clip(np.searchsorted(_E2M1_POS, m, side="left"), 0, 7)
+    lo = np.clip(hi - 1, 0, 7)
+    d_lo = m - _E2M1_POS[lo]
+    d_hi = _E2M1_POS[hi] - m
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(m == _E2M1_POS[hi], hi, code)
+    return (code.astype(np.uint8) | (np.signbit(x).astype(np.uint8) << 3)).astype(np.uint8)
+
+
+def e8m0_decode(e) -> np.ndarray:
+    e = np.asarray(e, dtype=np.int64)
+    return np.where(e == 255, np.nan, np.ldexp(1.0, (e - 127).astype(np.int64)))
+
+
+def mxfp4_pack(codes) -> np.ndarray:
+    """[..., d] E2M1 codes -> [..., d/2] bytes, element 2i in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
+
+
+def mxfp4_unpack(packed) -> np.ndarray:
+    """[..., d/2] bytes -> [..., d] E2M1 codes."""
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def mxfp4_decode(packed, exps) -> np.ndarray:
+    """Values of MXFP4 vectors: [..., d/2] packed codes, [..., d/32] E8M0
+    exponents -> float64 [..., d]."""
+    v = e2m1_decode(mxfp4_unpack(packed))
+    s = e8m0_decode(exps)
+    return v * np.repeat(s, MX_BLOCK, axis=-1)[..., : v.shape[-1]]
+
+
+def mxfp4_quantize(x):
+    """MXFP4 encoding of float64 vectors [..., d] (d a multiple of 32), the
+    OCP MX conversion: per block, the shared exponent is
+    X = floor(log2(amax)) - 2 (2 = the largest E2M1 exponent), clamped to the
+    E8M0 range, and every element is E2M1(x / 2^X) rounded to nearest even
+    and saturated.  READING: an all-zero block takes exponent 0 (byte 127).
+    Returns (packed codes [..., d/2] uint8, E8M0 bytes [..., d/32] uint8)."""
+    x = np.asarray(x, dtype=np.float64)
+    blocks = x.reshape(x.shape[:-1] + (x.shape[-1] // MX_BLOCK, MX_BLOCK))
+    amax = np.max(np.abs(blocks), axis=-1)
+    with np.errstate(divide="ignore"):
+        X = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2, 0.0)
+    X = np.clip(X, -127, 127)
+    codes = e2m1_encode(blocks / np.ldexp(1.0, X.astype(np.int64))[..., None])
+    return mxfp4_pack(codes.reshape(x.shape)), (X + 127).astype(np.uint8)

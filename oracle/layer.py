@@ -9,7 +9,8 @@ from __future__ import annotations
 import numpy as np
 
 from .method import (attend, dequant_slots, indexer_scores, n_entries, pool_entries,
-                     requantize, ring_slots, scale_block, topk, window_positions)
+                     requantize, requantize_mxfp4, ring_slots, scale_block, topk,
+                     window_positions)
 
 
 def _np(t):
@@ -35,6 +36,10 @@ def _q_ik(L, b, t):
     q = _np(L["q_ik"])[b, t].astype(np.float64)
     if L["q_ik_scale"] is None:
         return q
+    if L["comp_ik"]["fmt"] == "mxfp4":
+        from .formats import mxfp4_decode
+        d_I = L["comp_ik"]["d_nope"]
+        return mxfp4_decode(_np(L["q_ik"])[b, t], _np(L["q_ik_scale"])[b, t][:, : d_I // 32])
     from .formats import e4m3_decode
     sc = _np(L["q_ik_scale"])[b, t].astype(np.float64)       # [H_I][cols]
     d_I = q.shape[-1]
@@ -90,6 +95,11 @@ def layer_compress(L, t_begin, t_end):
             for name, cache in (("k", ring_k), ("ik", ring_ik)):
                 if name in r and cache is not None and len(js):
                     d_nope = cache["d_nope"]
+                    if cache["fmt"] == "mxfp4":
+                        # FP4 indexer keys: packed E2M1 codes, E8M0 exponents
+                        codes, exps = requantize_mxfp4(r[name])
+                        r[name + "_codes"], r[name + "_scales"] = codes, exps
+                        continue
                     codes, scales, rope = requantize(r[name], d_nope,
                                                      scale_block(cache["fmt"], d_nope))
                     r[name + "_codes"], r[name + "_scales"], r[name + "_rope"] = codes, scales, rope

@@ -17,7 +17,8 @@ from __future__ import annotations
 
 import numpy as np
 
-from .formats import E4M3_MAX, bf16_decode, bf16_encode, e4m3_decode, e4m3_encode
+from .formats import (E4M3_MAX, bf16_decode, bf16_encode, e4m3_decode, e4m3_encode,
+                      mxfp4_decode, mxfp4_quantize)
 
 
 # ---------------------------------------------------------------- pooling ---
@@ -111,6 +112,13 @@ def requantize(c: np.ndarray, d_nope: int, block: int = 64):
     return codes, scales, rope
 
 
+def requantize_mxfp4(c: np.ndarray):
+    """Store pooled indexer keys in the MXFP4 layout (the FP4 lightning
+    indexer): packed E2M1 codes and one E8M0 exponent per 32 dims, the OCP MX
+    conversion (see formats.mxfp4_quantize)."""
+    return mxfp4_quantize(np.asarray(c, dtype=np.float64))
+
+
 # ---------------------------------------------------------------- indexer ---
 
 def indexer_scores(q_ik: np.ndarray, head_w: np.ndarray, k_ik: np.ndarray) -> np.ndarray:
@@ -190,6 +198,10 @@ def dequant_slots(cache: dict, b: int, slots) -> np.ndarray:
     slots = np.asarray(slots, dtype=np.int64)
     if cache["fmt"] == "f32":
         return cache["data"][b, slots].astype(np.float64)
+    if cache["fmt"] == "mxfp4":
+        # packed E2M1 codes and one E8M0 exponent per 32 dims (no RoPE part)
+        d_nope = cache["d_nope"]
+        return mxfp4_decode(cache["data"][b, slots], cache["scale"][b, slots][:, : d_nope // 32])
     d_nope, d_rope = cache["d_nope"], cache["d_rope"]
     block = scale_block(cache["fmt"], d_nope)
     nb = (d_nope + block - 1) // block

@@ -27,7 +27,8 @@ class Workload:
     Hq: int = 64           # query heads sharing one KV head (MQA)
     fmt: str = "e4m3"      # "e4m3": FP8 E4M3 + per-64 fp32 scales + BF16 RoPE dims; "f32"
     ik_fmt: str = "e4m3vec"  # indexer keys / queries: "e4m3vec" (one fp32 scale per
-                             # vector) or "e4m3" (per-64 blocks); f32 workloads: "f32"
+                             # vector), "e4m3" (per-64 blocks) or "mxfp4" (FP4 E2M1 with
+                             # an E8M0 exponent per 32 dims); f32 workloads: "f32"
     d_nope: int = 448
     d_rope: int = 64
     separate_v: bool = False   # f32 tiny workload keeps separate K and V

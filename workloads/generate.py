@@ -76,10 +76,33 @@ def _fp8_planes(rng: _Rng, lead, d_nope: int, scale_pad: int, block: int = 64):
     return codes, scale
 
 
+# E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (codes 0..7) and the midpoints
+# between them: a draw is stored as the code of the interval it falls in
+_E2M1_EDGES = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def _mxfp4_planes(rng: _Rng, lead, d: int):
+    """FP4 (MXFP4) vectors: per element a draw y ~ N(0, 4) stored as the E2M1
+    code of its magnitude interval (magnitudes above 5 read 6) with its sign,
+    two codes per byte (even element in the low nibble); per 32 elements an
+    E8M0 exponent byte 126 + U{-1, 0, 1} (scale 2^-2 .. 2^0).  The values are
+    those of N(0,1)-like activations in the OCP MX layout.
+    Returns (packed uint8 [*lead, d/2], exponents uint8 [*lead, d/32])."""
+    y = rng.normal(*lead, d, std=2.0)
+    mag = torch.bucketize(y.abs(), _E2M1_EDGES.to(y.device))
+    codes = (mag | ((y < 0).to(mag.dtype) << 3)).to(torch.uint8)
+    packed = codes[..., 0::2] | (codes[..., 1::2] << 4)
+    exps = (126 + rng.integers(-1, 2, *lead, d // 32)).to(torch.uint8)
+    return packed, exps
+
+
 def _cache(rng: _Rng, wl: Workload, B: int, n: int, *, d_nope: int, d_rope: int,
            fmt: str, scale_pad: int, ring: bool):
     """A cache of n slots per sequence in the workload's storage format."""
     c = {"fmt": fmt, "d_nope": d_nope, "d_rope": d_rope, "ring": ring, "cap": n}
+    if fmt == "mxfp4":
+        c["data"], c["scale"] = _mxfp4_planes(rng, (B, n), d_nope)
+        return c
     if fmt == "f32":
         c["data"] = rng.normal(B, n, d_nope + d_rope)
     else:
@@ -99,6 +122,8 @@ def _poison_ring(c: dict, t_end: int):
     dead = torch.arange(live, cap)  # slots p % cap for p in [t_end-cap, 0) map here when t_end < cap
     if c["fmt"] == "f32":
         c["data"][:, dead] = float("nan")
+    elif c["fmt"] == "mxfp4":
+        c["scale"][:, dead] = 255          # the E8M0 NaN
     else:
         c["scale"][:, dead] = float("nan")
         if "rope" in c:
@@ -170,6 +195,8 @@ def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
     if wl.fmt == "f32":
         L["q_ik"] = rng.normal(wl.B, wl.Tq, wl.H_I, wl.d_I)
         L["q_ik_scale"] = None
+    elif ik_fmt == "mxfp4":
+        L["q_ik"], L["q_ik_scale"] = _mxfp4_planes(rng, (wl.B, wl.Tq, wl.H_I), wl.d_I)
     else:
         L["q_ik"], L["q_ik_scale"] = _fp8_planes(rng, (wl.B, wl.Tq, wl.H_I), wl.d_I, 1,
                                                  wl.d_I if ik_fmt == "e4m3vec" else 64)
@@ -187,6 +214,10 @@ def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
                 continue
             if wl.fmt == "f32":
                 L["comp_ik"]["data"][b, j] = L["q_ik"][b, 0, hstar] * 4.0
+            elif ik_fmt == "mxfp4":
+                # the head's codes, every block exponent 2 higher (x4)
+                L["comp_ik"]["data"][b, j] = L["q_ik"][b, 0, hstar]
+                L["comp_ik"]["scale"][b, j] = L["q_ik_scale"][b, 0, hstar] + 2
             else:
                 L["comp_ik"]["data"][b, j] = L["q_ik"][b, 0, hstar]
                 nbq = L["q_ik_scale"].shape[-1]
