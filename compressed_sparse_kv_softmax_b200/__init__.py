@@ -28,8 +28,8 @@ OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_SCRATCH_LIMIT, ERR_DE
     0, -1, -2, -3, -4, -5, -6)
 # device-side events (bits of cskv_check_device_errors)
 DEV_INDEXER_WAIT, DEV_TOPK_BARRIER, DEV_ATTN_WAIT, DEV_ROW_FAILED = 1, 2, 4, 8
-FMT_F32, FMT_E4M3_BF16, FMT_E4M3_VEC = 0, 1, 2
-_FMT = {"f32": FMT_F32, "e4m3": FMT_E4M3_BF16, "e4m3vec": FMT_E4M3_VEC}
+FMT_F32, FMT_E4M3_BF16, FMT_E4M3_VEC, FMT_MXFP4 = 0, 1, 2, 3
+_FMT = {"f32": FMT_F32, "e4m3": FMT_E4M3_BF16, "e4m3vec": FMT_E4M3_VEC, "mxfp4": FMT_MXFP4}
 
 
 class CskvCache(ctypes.Structure):

@@ -24,6 +24,15 @@ int check_cache(const cskv_cache *c, int ring) {
     if (c->data_stride < 4LL * (c->d_nope + c->d_rope)) return CSKV_ERR_ARG;
     return CSKV_OK;
   }
+  if (c->fmt == CSKV_FMT_MXFP4) {
+    // packed E2M1 codes, one E8M0 byte per 32 dims (whole 4-byte groups)
+    if (c->d_nope < 128 || c->d_nope % 128 || c->d_rope) return CSKV_ERR_UNSUPPORTED;
+    if (c->data_stride < c->d_nope / 2) return CSKV_ERR_ARG;
+    if (!c->scale || !aligned16(c->scale) || c->scale_stride % 4 ||
+        c->scale_stride < c->d_nope / 32)
+      return CSKV_ERR_ARG;
+    return CSKV_OK;
+  }
   if (c->fmt != CSKV_FMT_E4M3_BF16 && c->fmt != CSKV_FMT_E4M3_VEC) return CSKV_ERR_UNSUPPORTED;
   if (c->d_nope < 64 || c->d_nope % 64) return CSKV_ERR_UNSUPPORTED;
   if (c->fmt == CSKV_FMT_E4M3_VEC && c->d_rope) return CSKV_ERR_UNSUPPORTED;
@@ -165,7 +174,8 @@ int indexer_common(int phases, int B, int Tq, const int64_t *q_pos, const void *
   if (!q_pos || !q_ik || !head_w || !out_idx || !aligned16(q_ik)) return CSKV_ERR_ARG;
   CSKV_TRY(check_cache(ik, 0));
   if (ik->d_rope != 0 || ik->d_nope != d_I || max_entries > ik->cap) return CSKV_ERR_ARG;
-  if (ik->fmt == CSKV_FMT_E4M3_BF16 || ik->fmt == CSKV_FMT_E4M3_VEC) {
+  if (ik->fmt == CSKV_FMT_E4M3_BF16 || ik->fmt == CSKV_FMT_E4M3_VEC ||
+      ik->fmt == CSKV_FMT_MXFP4) {
     if (!q_ik_scale) return CSKV_ERR_ARG;
   } else if (q_ik_scale) {
     return CSKV_ERR_ARG;

@@ -33,12 +33,43 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
+// E2M1 code of x: round to nearest, ties to the even code, saturate to +-6
+// (the comparisons put each tie on the even side), sign in bit 3
+__device__ __forceinline__ uint32_t e2m1_encode(float x) {
+  const float m = fabsf(x);
+  const uint32_t c = (m > 0.25f) + (m >= 0.75f) + (m > 1.25f) + (m >= 1.75f) + (m > 2.5f) +
+                     (m >= 3.5f) + (m > 5.0f);
+  return c | (signbit(x) ? 8u : 0u);
+}
+
+// MXFP4 store of one warp's 32-dim block: the OCP MX shared exponent
+// X = floor(log2 amax) - 2 (0 for an all-zero block), every element
+// E2M1(x / 2^X), two codes per byte (even element in the low nibble)
+__device__ __forceinline__ void store_mxfp4_block(uint8_t *codes, uint8_t *exps, int blk,
+                                                  float v) {
+  const int lane = threadIdx.x & 31;
+  const float amax = warp_max(fabsf(v));
+  int X = amax > 0.f ? ilogbf(amax) - 2 : 0;
+  X = X < -127 ? -127 : (X > 127 ? 127 : X);
+  const uint32_t c = e2m1_encode(ldexpf(v, -X));
+  const uint32_t hi = __shfl_down_sync(0xffffffffu, c, 1);
+  if (!(lane & 1)) codes[blk * 16 + (lane >> 1)] = (uint8_t)(c | (hi << 4));
+  if (lane == 0) exps[blk] = (uint8_t)(X + 127);
+}
+
 __device__ __noinline__ void store_entry(const Cache &out, int b, long long j,
                                         const float *pooled, int D) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (out.fmt == CSKV_FMT_F32) {
     float *dst = reinterpret_cast<float *>(out.data + out.row(b, j) * out.data_stride);
     for (int d = tid; d < D; d += kThreads) dst[d] = pooled[d];
+    return;
+  }
+  if (out.fmt == CSKV_FMT_MXFP4) {
+    uint8_t *codes = out.data + out.row(b, j) * out.data_stride;
+    uint8_t *exps = out.scale + out.row(b, j) * out.scale_stride;
+    for (int blk = warp; blk < (out.d_nope >> 5); blk += kWarps)
+      store_mxfp4_block(codes, exps, blk, pooled[blk * 32 + lane]);
     return;
   }
   uint8_t *codes = out.data + out.row(b, j) * out.data_stride;
@@ -168,9 +199,9 @@ __host__ __device__ inline SlotLayout slot_layout(const Cache &c) {
     l.scale_off = l.rope_off = l.bytes = round16(l.data_bytes);
     return l;
   }
-  l.data_bytes = c.d_nope;
-  l.scale_off = round16(c.d_nope);
-  l.rope_off = l.scale_off + round16(4 * c.n_scales());
+  l.data_bytes = c.data_bytes();
+  l.scale_off = round16(l.data_bytes);
+  l.rope_off = l.scale_off + round16(c.scale_bytes());
   l.bytes = l.rope_off + round16(2 * c.d_rope);
   return l;
 }
@@ -216,8 +247,7 @@ __device__ __noinline__ void stage_window(const Cache &c, const SlotLayout &l, c
     uint8_t *dst = buf + (size_t)r * l.bytes;
     stage_bytes(dst, c.data + row * c.data_stride, l.data_bytes, lane, 32);
     if (c.fmt != CSKV_FMT_F32) {
-      stage_bytes(dst + l.scale_off, c.scale + row * c.scale_stride, 4 * c.n_scales(), lane,
-                  32);
+      stage_bytes(dst + l.scale_off, c.scale + row * c.scale_stride, c.scale_bytes(), lane, 32);
       if (c.d_rope)
         stage_bytes(dst + l.rope_off, c.rope + row * c.rope_stride, 2 * c.d_rope, lane, 32);
     }
@@ -227,6 +257,8 @@ __device__ __noinline__ void stage_window(const Cache &c, const SlotLayout &l, c
 __device__ __forceinline__ float staged_value(const Cache &c, const SlotLayout &l,
                                               const uint8_t *slot, int d) {
   if (c.fmt == CSKV_FMT_F32) return reinterpret_cast<const float *>(slot)[d];
+  if (c.fmt == CSKV_FMT_MXFP4)
+    return mxfp4_value(slot[d >> 1] >> ((d & 1) << 2), slot[l.scale_off + (d >> 5)]);
   if (d < c.d_nope)
     return e4m3_decode(slot[d]) *
            reinterpret_cast<const float *>(slot + l.scale_off)[c.fmt == CSKV_FMT_E4M3_VEC ? 0 : d >> 6];
@@ -244,6 +276,18 @@ __device__ __noinline__ void pool_staged(const Cache &c, const SlotLayout &l, co
       float acc = 0.f;
       for (int r = r0; r < pool; ++r)
         acc = fmaf(a[r], reinterpret_cast<const float *>(buf + (size_t)r * bytes)[d], acc);
+      pooled[d] = acc;
+    }
+    return;
+  }
+  if (c.fmt == CSKV_FMT_MXFP4) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      float acc = 0.f;
+      for (int r = r0; r < pool; ++r) {
+        const uint8_t *slot = buf + (size_t)r * bytes;
+        acc = fmaf(a[r], mxfp4_value(slot[d >> 1] >> ((d & 1) << 2), slot[l.scale_off + (d >> 5)]),
+                   acc);
+      }
       pooled[d] = acc;
     }
     return;

@@ -13,6 +13,18 @@
 
 namespace cskv {
 
+// FP4 E2M1 (low 4 bits of `code`) times the E8M0 scale 2^(e - 127); e = 255
+// (the E8M0 NaN) gives NaN.  E2M1: sign, 2 exponent bits (bias 1), 1 mantissa
+// bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+__host__ __device__ __forceinline__ float e2m1_decode(uint32_t code) {
+  const uint32_t m = code & 7u;
+  const float mag = m < 2 ? 0.5f * (float)m : (float)(2u + (m & 1u)) * (float)(1u << ((m >> 1) - 1)) * 0.5f;
+  return (code & 8u) ? -mag : mag;
+}
+__device__ __forceinline__ float mxfp4_value(uint32_t code, uint8_t e) {
+  return e == 255 ? __int_as_float(0x7fffffff) : ldexpf(e2m1_decode(code), (int)e - 127);
+}
+
 // Device-side view of a cskv_cache (passed to kernels by value).
 struct Cache {
   int fmt, d_nope, d_rope, ring;
@@ -22,9 +34,21 @@ struct Cache {
   uint8_t *rope; long long rope_stride;
 
   __host__ __device__ int dims() const { return d_nope + d_rope; }
-  // fp32 scales per slot and the dims each covers
-  __host__ __device__ int n_scales() const { return fmt == CSKV_FMT_E4M3_VEC ? 1 : d_nope >> 6; }
-  __host__ __device__ int scale_block() const { return fmt == CSKV_FMT_E4M3_VEC ? d_nope : 64; }
+  // scales per slot, the dims each covers, and the bytes they take
+  // (fp32 scales; one E8M0 byte per 32 dims for MXFP4)
+  __host__ __device__ int n_scales() const {
+    return fmt == CSKV_FMT_E4M3_VEC ? 1 : (fmt == CSKV_FMT_MXFP4 ? d_nope >> 5 : d_nope >> 6);
+  }
+  __host__ __device__ int scale_block() const {
+    return fmt == CSKV_FMT_E4M3_VEC ? d_nope : (fmt == CSKV_FMT_MXFP4 ? 32 : 64);
+  }
+  __host__ __device__ int scale_bytes() const {
+    return fmt == CSKV_FMT_MXFP4 ? n_scales() : 4 * n_scales();
+  }
+  // bytes of the data plane that a slot's values take
+  __host__ __device__ int data_bytes() const {
+    return fmt == CSKV_FMT_F32 ? 4 * dims() : (fmt == CSKV_FMT_MXFP4 ? d_nope >> 1 : d_nope);
+  }
   __host__ __device__ long long row(int b, long long slot) const {
     return (long long)b * cap + slot;
   }
@@ -43,6 +67,9 @@ struct Cache {
   __device__ float value(int b, long long slot, int d) const {
     if (fmt == CSKV_FMT_F32)
       return reinterpret_cast<const float *>(data_ptr(b, slot))[d];
+    if (fmt == CSKV_FMT_MXFP4)
+      return mxfp4_value(data_ptr(b, slot)[d >> 1] >> ((d & 1) << 2),
+                         (scale + row(b, slot) * scale_stride)[d >> 5]);
     if (d < d_nope) {
       __nv_fp8_e4m3 c;
       c.__x = data_ptr(b, slot)[d];

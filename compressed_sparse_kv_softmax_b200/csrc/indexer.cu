@@ -23,6 +23,9 @@ int launch_topk_select(const IndexerWs &w, const int64_t *q_pos, int stride,
                        long long max_entries, int k, int rows, int32_t *out_idx,
                        float *out_score, unsigned int *status, cudaStream_t st);
 bool indexer_tc_supported(const IndexerArgs &a);
+bool indexer_mxf4_supported(const IndexerArgs &a);
+int launch_indexer_mxf4(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
+                        uint32_t *ctr, cudaStream_t st);
 int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
                       uint32_t *ctr, cudaStream_t st);
 int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint32_t *hist,
@@ -52,6 +55,11 @@ indexer_score_kernel(IndexerArgs a, float *__restrict__ scores, long long ld) {
   for (int i = tid; i < H * dI; i += blockDim.x) {
     if (a.ik.fmt == CSKV_FMT_F32) {
       q[i] = reinterpret_cast<const float *>(a.q_ik)[qoff + i];
+    } else if (a.ik.fmt == CSKV_FMT_MXFP4) {
+      // packed codes of head i / dI, dim i % dI; one E8M0 byte per 32 dims
+      const uint8_t code = reinterpret_cast<const uint8_t *>(a.q_ik)[(qoff + i) >> 1];
+      const uint8_t *ex = reinterpret_cast<const uint8_t *>(a.q_ik_scale);
+      q[i] = mxfp4_value(code >> (((qoff + i) & 1) << 2), ex[(qoff + i) >> 5]);
     } else {
       const int h = i / dI, d = i % dI;
       // query scales follow the keys' layout: per 64 dims, or one per head
@@ -95,7 +103,8 @@ int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st) {
   if (rows == 0) return CSKV_OK;
   const IndexerWs w = indexer_ws_layout(a.ws, rows, a.max_entries, a.k, nullptr);
   const bool score = phases & kIndexerScore, select = phases & kIndexerSelect;
-  if (a.max_entries > 0 && indexer_tc_supported(a)) {
+  const bool mxf4 = a.max_entries > 0 && indexer_mxf4_supported(a);
+  if (a.max_entries > 0 && (mxf4 || indexer_tc_supported(a))) {
     // tensor-core scoring builds the score histogram the multi-CTA selection
     // uses.  The histogram only guides the selection (every count it implies
     // is checked against the scores, and a row whose counts disagree is
@@ -105,8 +114,10 @@ int launch_indexer_topk(const IndexerArgs &a, int phases, cudaStream_t st) {
     // scoring kernel clears the selection's counters.
     if (score) {
       // several query rows per sequence share each key tile; one row streams alone
-      int rc = launch_indexer_rows(a, w.scores, w.ld, w.hist, w.ctr, st);
-      if (rc == CSKV_ERR_UNSUPPORTED)
+      // (FP4 keys: one query row per CTA group, block-scaled MMAs)
+      int rc = mxf4 ? launch_indexer_mxf4(a, w.scores, w.ld, w.hist, w.ctr, st)
+                    : launch_indexer_rows(a, w.scores, w.ld, w.hist, w.ctr, st);
+      if (!mxf4 && rc == CSKV_ERR_UNSUPPORTED)
         rc = launch_indexer_tc(a, w.scores, w.ld, w.hist, w.ctr, st);
       if (rc != CSKV_OK) return rc;
     }

@@ -444,7 +444,11 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+}  // namespace
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (nullptr
+// when unavailable)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void *p = nullptr;
@@ -459,7 +463,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-}  // namespace
 
 bool indexer_tc_supported(const IndexerArgs &a) {
   const bool vec = a.ik.fmt == CSKV_FMT_E4M3_VEC;
@@ -471,11 +474,11 @@ bool indexer_tc_supported(const IndexerArgs &a) {
   int dev = 0, major = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  return major == 10 && encode_fn() != nullptr;
+  return major == 10 && tensor_map_encode_fn() != nullptr;
 }
 
 bool make_key_tmap(const IndexerArgs &a, CUtensorMap *map) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encode_fn();
   if (!fn) return false;
   // all sequences' key rows as one [B * cap] x 128-byte matrix; 128 x 128 B
   // boxes in the 128-byte swizzle the K-major operand descriptors expect

@@ -215,6 +215,31 @@ __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_
       : "memory");
 }
 
+// Block-scaled MXFP4 MMA: A and B packed FP4 E2M1 (two per byte), K = 64 per
+// instruction with one E8M0 scale per 32 elements of each row of A and B,
+// read from TMEM at sfa / sfb (the top two address bits select the byte of
+// the 32-bit TMEM column where this K step's two scales start).
+__device__ __forceinline__ void mma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy a 32-row x 16-byte matrix from shared memory into TMEM columns
+// [taddr, taddr + 4) of every lane quadrant (lanes r, 32 + r, 64 + r, 96 + r
+// receive row r): the scale-factor layout of the block-scaled MMAs.
+// Asynchronous; ordered before later tcgen05.mma of the same thread.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
 // Arrive on an mbarrier once every previously issued tcgen05.mma of this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -317,6 +342,40 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t addr, uint32_t l
   d |= (uint64_t)1u << 46;
   d |= (uint64_t)2u << 61;
   return d;
+}
+
+// K-major operand tile in the canonical 64-byte-swizzled layout: rows of 64
+// bytes, 8-row atoms 512 bytes apart (16-byte chunk c of row r stored at
+// chunk c ^ ((r >> 1) & 3)).
+__device__ __forceinline__ uint64_t desc_kmajor_sw64(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);          // start address
+  d |= (uint64_t)1u << 16;                         // leading byte offset (16 B, unused)
+  d |= (uint64_t)(512u >> 4) << 32;                // stride byte offset: 8-row atom pitch
+  d |= (uint64_t)1u << 46;                         // descriptor version (sm_100)
+  d |= (uint64_t)4u << 61;                         // 64-byte swizzle
+  return d;
+}
+
+// Unswizzled matrix of 16-byte rows stored one after another (8-row groups
+// 128 bytes apart): the source layout of tmem_cp_32x128b_x4.
+__device__ __forceinline__ uint64_t desc_rows16(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 16;
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;
+}
+
+// Instruction descriptor of the block-scaled MXFP4 MMA: E2M1 A and B, E8M0
+// scales, fp32 accumulator, K-major operands, M x N tile; sf_a / sf_b are
+// the scale bytes this K step starts at (as in the scale TMEM addresses).
+__host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t M, uint32_t N, uint32_t sf_a,
+                                                  uint32_t sf_b) {
+  return (sf_b << 4)               // B scale factor byte
+         | (1u << 7) | (1u << 10)  // A, B: E2M1
+         | ((N >> 3) << 17) | (1u << 23) /* E8M0 scales */ | ((M >> 4) << 24) | (sf_a << 29);
 }
 
 // Instruction descriptor: fp32 accumulator, A/B format codes, K-major or

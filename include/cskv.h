@@ -83,7 +83,8 @@ enum {
 enum {
   CSKV_FMT_F32 = 0,        /* fp32 values, d_nope + d_rope per slot (no scale/rope planes) */
   CSKV_FMT_E4M3_BF16 = 1,  /* d_nope E4M3 codes + d_nope/64 fp32 scales + d_rope BF16 */
-  CSKV_FMT_E4M3_VEC = 2    /* d_nope E4M3 codes + ONE fp32 scale per slot; d_rope = 0 */
+  CSKV_FMT_E4M3_VEC = 2,   /* d_nope E4M3 codes + ONE fp32 scale per slot; d_rope = 0 */
+  CSKV_FMT_MXFP4 = 3       /* d_nope FP4 E2M1 codes, two per byte + d_nope/32 E8M0 bytes; d_rope = 0 */
 };
 
 /*
@@ -96,12 +97,22 @@ enum {
  *                   value[d_nope + r] = BF16(rope[r])          for r < d_rope.
  * E4M3_VEC layout:  value[d] = E4M3(data[d]) * scale[0]        for d < d_nope
  *                   (one scale per vector, no RoPE plane).
- * The lightning-indexer key cache uses either E4M3 layout with d_rope = 0;
- * E4M3_VEC is the one the tensor-core scoring path reads fastest (one
- * accumulator per key and head).
+ * MXFP4 layout (OCP Microscaling MXFP4, blocks of 32):
+ *                   value[d] = E2M1(nibble d of data) * 2^(E[d / 32] - 127),
+ *                   nibble d = bits 4*(d%2) .. 4*(d%2)+3 of byte d/2 (the even
+ *                   element in the low nibble), E = the bytes of the scale
+ *                   plane (the `scale` pointer then addresses uint8 E8M0
+ *                   exponents, 255 = NaN); no RoPE plane.  The FP4 lightning
+ *                   indexer («DeepSeek-V4: 1 Million Token Context endlich
+ *                   nutzbar», "Hybrid Attention: CSA und HCA").
+ * The lightning-indexer key cache uses any of the three E4M3 / MXFP4 layouts
+ * with d_rope = 0; E4M3_VEC and MXFP4 are the ones the tensor-core scoring
+ * path reads fastest (one accumulator per key and head), MXFP4 with half the
+ * bytes.
  * Alignment: data and rope pointers and strides are multiples of 16 bytes;
  * scale pointer 16-byte aligned, scale stride a multiple of 4 bytes and at
- * least 4 * ceil(d_nope / 64) (E4M3_BF16) or 4 (E4M3_VEC).  F32: data pointer and stride multiples of 16.
+ * least 4 * ceil(d_nope / 64) (E4M3_BF16), 4 (E4M3_VEC) or d_nope / 32
+ * (MXFP4, d_nope a multiple of 128).  F32: data pointer and stride multiples of 16.
  */
 typedef struct cskv_cache {
   int32_t fmt;            /* CSKV_FMT_* */
@@ -183,7 +194,9 @@ int cskv_ring_store(int B, const int64_t *pos, int n, const cskv_cache *const *s
  *   q_ik     : [B][Tq][H_I][d_I]; E4M3 codes when ik->fmt is E4M3_BF16 (with
  *              q_ik_scale [B][Tq][H_I][d_I/64] fp32) or E4M3_VEC (with
  *              q_ik_scale [B][Tq][H_I], one fp32 scale per head), fp32 when
- *              ik->fmt is F32 (q_ik_scale NULL).
+ *              ik->fmt is F32 (q_ik_scale NULL); MXFP4: [B][Tq][H_I][d_I/2]
+ *              packed E2M1 codes with q_ik_scale pointing to [B][Tq][H_I][d_I/32]
+ *              E8M0 bytes.  16-byte aligned.
  *   head_w   : [B][Tq][H_I] fp32.
  *   ik       : indexer-key cache (ring = 0, d_nope = d_I, d_rope = 0).
  *   k        : selections per row, 1 <= k <= 4096.

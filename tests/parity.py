@@ -128,3 +128,32 @@ def check_compressed_e4m3(cache, b, js, ref_vals, ref_mag, d_nope, where=""):
         check_codes(rope, ref_vals[:, d_nope:], O.bf16_encode, O.bf16_decode,
                     POOL_EPS * ref_mag[:, d_nope:], where=where + " bf16")
     return exact, float(np.max(serr)) if serr.size else 0.0
+
+
+def check_compressed_mxfp4(cache, b, js, ref_vals, ref_mag, d_nope, where=""):
+    """MXFP4 entries (packed E2M1 codes, one E8M0 exponent per 32 dims):
+    every block's exponent X must be floor(log2 amax) - 2 for an amax inside
+    the float32 evaluation band of the oracle's block maximum, and every code
+    the E2M1 rounding of a value inside the band of the oracle's value divided
+    by 2^X; at least 99.9% of the codes equal the oracle's own rounding."""
+    js = np.asarray(js)
+    packed = cache["data"][b, js].cpu().numpy()
+    exps = cache["scale"][b, js][:, : d_nope // 32].cpu().numpy().astype(np.int64)
+    X = exps - 127
+    y = ref_vals[:, :d_nope].reshape(len(js), d_nope // 32, 32)
+    dy = POOL_EPS * ref_mag[:, :d_nope].reshape(len(js), d_nope // 32, 32)
+    amax = np.max(np.abs(y), axis=2)
+    band = np.max(dy, axis=2)
+
+    def shared_x(a):
+        with np.errstate(divide="ignore"):
+            return np.where(a > 0, np.floor(np.log2(np.where(a > 0, a, 1.0))) - 2, 0.0)
+    x_lo, x_hi = shared_x(np.maximum(amax - band, 0.0)), shared_x(amax + band)
+    x_lo = np.where(amax - band <= 0, np.minimum(x_lo, 0), x_lo)
+    ok = (X >= np.minimum(x_lo, x_hi)) & (X <= np.maximum(x_lo, x_hi))
+    assert np.all(ok), f"{where}: {np.sum(~ok)} block exponents outside the band"
+    s = np.ldexp(1.0, X)[:, :, None]
+    codes = O.mxfp4_unpack(packed).reshape(len(js), d_nope // 32, 32)
+    exact = check_codes(codes.reshape(-1), (y / s).reshape(-1), O.e2m1_encode, O.e2m1_decode,
+                        (dy / s).reshape(-1), where=where + " e2m1")
+    return exact

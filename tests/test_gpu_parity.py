@@ -8,7 +8,8 @@ import torch
 import oracle as O
 import workloads as W
 from gpu_common import require_gpu, sample_rows, to_device
-from parity import check_attention, check_compressed_e4m3, check_pooled_f32, check_topk
+from parity import (check_attention, check_compressed_e4m3, check_compressed_mxfp4,
+                    check_pooled_f32, check_topk)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,7 +50,8 @@ def test_compress_f32_tiny(C, kind, span):
         check_pooled_f32(got, ref[name], ref[name + "_mag"], where=f"{kind} {name}")
 
 
-@pytest.mark.parametrize("kind,ik_fmt", [("csa", "e4m3vec"), ("csa", "e4m3"), ("hca", "e4m3vec")])
+@pytest.mark.parametrize("kind,ik_fmt", [("csa", "e4m3vec"), ("csa", "e4m3"), ("hca", "e4m3vec"),
+                                         ("csa", "mxfp4")])
 def test_compress_e4m3_parity_decode(C, kind, ik_fmt):
     wl = W.get("parity_decode").with_(ik_fmt=ik_fmt)
     mk = W.make_csa_layer if kind == "csa" else W.make_hca_layer
@@ -65,7 +67,10 @@ def test_compress_e4m3_parity_decode(C, kind, ik_fmt):
             continue
         check_compressed_e4m3(Ld["comp_k"], b, r["j"], r["k"], r["k_mag"], wl.d_nope,
                               where=f"{kind} b{b} kv")
-        if "ik" in r:
+        if "ik" in r and ik_fmt == "mxfp4":
+            check_compressed_mxfp4(Ld["comp_ik"], b, r["j"], r["ik"], r["ik_mag"], wl.d_I,
+                                   where=f"b{b} ik")
+        elif "ik" in r:
             check_compressed_e4m3(Ld["comp_ik"], b, r["j"], r["ik"], r["ik_mag"], wl.d_I,
                                   where=f"b{b} ik")
         n_checked += len(r["j"])
@@ -95,7 +100,8 @@ def _run_indexer(C, Ld, k=None):
 
 @pytest.mark.parametrize("name,ik_fmt", [("tiny", "f32"), ("parity_decode", "e4m3vec"),
                                          ("parity_prefill", "e4m3vec"),
-                                         ("parity_decode", "e4m3"), ("parity_prefill", "e4m3")])
+                                         ("parity_decode", "e4m3"), ("parity_prefill", "e4m3"),
+                                         ("parity_decode", "mxfp4"), ("parity_prefill", "mxfp4")])
 def test_indexer_topk(C, name, ik_fmt):
     # both FP8 indexer layouts: one scale per vector, and one per 64 dims
     wl = W.get(name)
@@ -115,7 +121,7 @@ def test_indexer_topk(C, name, ik_fmt):
 
 
 @pytest.mark.parametrize("ik_fmt,pad_cols", [("e4m3vec", 0), ("e4m3vec", 2), ("e4m3", 0),
-                                              ("e4m3", 4)])
+                                              ("e4m3", 4), ("mxfp4", 0), ("mxfp4", 8)])
 @pytest.mark.parametrize("Tq", [1, 5])
 def test_indexer_any_scale_plane_layout(C, ik_fmt, pad_cols, Tq):
     # 3 sequences of 2,499 entries: with 4 or 8 scale bytes per entry every
@@ -128,7 +134,8 @@ def test_indexer_any_scale_plane_layout(C, ik_fmt, pad_cols, Tq):
     Ld = to_device(L)
     if pad_cols:
         sc = Ld["comp_ik"]["scale"]
-        wide = torch.full((*sc.shape[:2], pad_cols), float("nan"), device="cuda")
+        fill = float("nan") if sc.is_floating_point() else 255      # (255: the E8M0 NaN)
+        wide = torch.full((*sc.shape[:2], pad_cols), fill, dtype=sc.dtype, device="cuda")
         wide[..., : sc.shape[2]] = sc
         Ld["comp_ik"]["scale"] = wide[..., : sc.shape[2]]
     layer = _run_indexer(C, Ld)

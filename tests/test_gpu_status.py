@@ -65,15 +65,15 @@ def test_topk_meeting_point_timeout_keeps_the_result_exact(C):
     assert C.check_device_errors() == 0
 
 
-@pytest.mark.parametrize("Tq", [1, 4])
-def test_scoring_wait_runs_out_and_the_row_is_reported(C, Tq):
+@pytest.mark.parametrize("Tq,ik_fmt", [(1, "e4m3vec"), (4, "e4m3vec"), (1, "mxfp4")])
+def test_scoring_wait_runs_out_and_the_row_is_reported(C, Tq, ik_fmt):
     from compressed_sparse_kv_softmax_b200.layer import CSALayer
     # the hook makes the first scoring CTA miss its first key tile and bounds
     # its waits to a few thousand polls: the kernel returns, the CTA's scores
     # read NaN, its query rows are reported failed (row 0; with several rows
     # per sequence, the CTA's group: every row of sequence 0 here), the
     # other rows are exact
-    wl = W.get("parity_decode").with_(Tq=Tq, prefill=Tq > 1)
+    wl = W.get("parity_decode").with_(Tq=Tq, prefill=Tq > 1, ik_fmt=ik_fmt)
     L = W.make_csa_layer(wl)
     layer = CSALayer(to_device(L))
     rows = [(b, t) for b in range(wl.B) for t in range(wl.Tq)]
