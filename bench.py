@@ -336,21 +336,21 @@ class CallGraph:
                     _ok(rt.cudaEventElapsedTime(a, b), "elapsed"))
 
 
-def _ik_scales(wl):
-    """fp32 scales per indexer key or query head: one per vector in the
-    per-vector layout, else one per 64 dims."""
-    return 1 if wl.ik_fmt == "e4m3vec" else wl.d_I // 64
+def ik_key_bytes(wl):
+    """Bytes of one indexer key: FP8 codes and one fp32 scale per vector or
+    per 64 dims, or MXFP4 codes (two per byte) and one E8M0 byte per 32 dims."""
+    if wl.ik_fmt == "mxfp4":
+        return wl.d_I // 2 + wl.d_I // 32
+    return wl.d_I + 4 * (1 if wl.ik_fmt == "e4m3vec" else wl.d_I // 64)
 
 
 def indexer_bytes(wl):
     """Algorithmic HBM bytes of one indexer scoring launch: every visible CSA
-    entry's FP8 indexer key (d_I bytes) and its fp32 scale(s), the FP8 query
-    heads with their scales and the head weights.  (The scores, 4 bytes per
-    entry, stay in L2 for the selection.)"""
+    entry's indexer key, the query heads in the same layout and the head
+    weights.  (The scores, 4 bytes per entry, stay in L2 for the selection.)"""
     n_c = wl.T // wl.csa_stride
-    per_entry = wl.d_I + 4 * _ik_scales(wl)
-    q = wl.H_I * wl.d_I + 4 * wl.H_I * _ik_scales(wl) + 4 * wl.H_I
-    return wl.B * (n_c * per_entry + q)
+    q = wl.H_I * ik_key_bytes(wl) + 4 * wl.H_I
+    return wl.B * (n_c * ik_key_bytes(wl) + q)
 
 
 def call_bytes(wl):
@@ -359,7 +359,7 @@ def call_bytes(wl):
     block scales and 64 BF16 RoPE values = 604 bytes; an indexer key 128 codes
     and one or two scales).  The selection's scores live in L2."""
     entry = wl.d_nope + 2 * wl.d_rope + 4 * (wl.d_nope // 64)
-    ik = wl.d_I + 4 * _ik_scales(wl)
+    ik = ik_key_bytes(wl)
     n_c = wl.T // wl.csa_stride
     n_h = wl.T // wl.hca_stride
     q = wl.Hq * wl.D * 2
@@ -466,27 +466,35 @@ def _time_decode(args, wl, rank, world, dev, steps, seed0, clocks=True, call_rep
             "launches": graph.kernels * n_launch + (tail.kernels if tail else 0)}
 
 
-def _other_layout(args, wl, rank, world, dev):
-    """The same step with the other FP8 indexer scale layout, timed briefly:
-    the layout comparison rides along with the headline number."""
-    other = wl.with_(ik_fmt="e4m3" if wl.ik_fmt == "e4m3vec" else "e4m3vec")
-    t = _time_decode(args, other, rank, world, dev, args.alt_steps, 5000, clocks=False,
-                     call_replays=0)
-    ib = indexer_bytes(other)
+def _other_layouts(args, wl, rank, world, dev):
+    """The same step with each other indexer layout (FP8 with the other scale
+    granularity, FP4 MXFP4), timed briefly: the layout comparison rides along
+    with the headline number."""
     peak, _ = _peaks()
-    achieved = ib / (t["idx_ms"] / 1e3) / 1e9
-    out = {"indexer_scales": _scales_text(other),
-           "value": round(other.B * t["steps"] * world / (t["ms"] / 1e3), 2), "unit": UNIT,
-           "steps": t["steps"], "ms_per_step": t["ms"] / t["steps"],
-           "indexer_score_us": round(t["idx_ms"] * 1e3, 3),
-           "indexer_algorithmic_bytes": ib, "indexer_frac": round(achieved / peak, 4)}
-    del t
-    torch.cuda.empty_cache()
+    out = []
+    for fmt in ("e4m3vec", "e4m3", "mxfp4"):
+        if fmt == wl.ik_fmt:
+            continue
+        other = wl.with_(ik_fmt=fmt)
+        t = _time_decode(args, other, rank, world, dev, args.alt_steps, 5000, clocks=False,
+                         call_replays=0)
+        ib = indexer_bytes(other)
+        achieved = ib / (t["idx_ms"] / 1e3) / 1e9
+        out.append({"indexer_layout": fmt, "indexer_scales": _scales_text(other),
+                    "value": round(other.B * t["steps"] * world / (t["ms"] / 1e3), 2),
+                    "unit": UNIT, "steps": t["steps"], "ms_per_step": t["ms"] / t["steps"],
+                    "indexer_score_us": round(t["idx_ms"] * 1e3, 3),
+                    "indexer_samples": t["idx_samples"],
+                    "indexer_algorithmic_bytes": ib, "indexer_frac": round(achieved / peak, 4)})
+        del t
+        torch.cuda.empty_cache()
     return out
 
 
 def _scales_text(wl):
-    return "one fp32 per key / query head" if wl.ik_fmt == "e4m3vec" else "one fp32 per 64 dims"
+    return {"e4m3vec": "FP8 E4M3, one fp32 scale per key / query head",
+            "e4m3": "FP8 E4M3, one fp32 scale per 64 dims",
+            "mxfp4": "FP4 MXFP4: E2M1 codes, one E8M0 exponent per 32 dims"}[wl.ik_fmt]
 
 
 def run_ours(args, rank, world, dev):
@@ -541,7 +549,7 @@ def run_ours(args, rank, world, dev):
            "clocks": clocks}
     del t
     if args.alt_steps > 0:
-        res["other_indexer_layout"] = _other_layout(args, wl, rank, world, dev)
+        res["other_indexer_layouts"] = _other_layouts(args, wl, rank, world, dev)
     return res, replicas, wl
 
 
@@ -606,7 +614,16 @@ def run_e2e(args, replicas, wl, dev, world):
                  sc.ctx[s], sc.tb[s], sc.te[s]] + token(cl0, "ring_k", s) + token(hl0, "ring_k", s)
                 + token(cl0, "ring_ik", s))
 
+    # the step's inputs in pinned host memory, taken before the layers are
+    # pointed at the staging buffer
+    host_small = []
+    for s in range(PERIOD):
+        hb, hv = _pack(small(s), "cpu", pin=True)
+        for v, t in zip(hv, small(s)):
+            v.copy_(t.cpu())
+        host_small.append(hb)
     dev_buf, views = _pack(small(0), dev)
+    dev_buf.copy_(host_small[0])
     q_c, q_h, q_ik, q_ik_s, head_w, q_pos, ctx, tb, te = views[:9]
     tok = views[9:]
 
@@ -629,12 +646,6 @@ def run_e2e(args, replicas, wl, dev, world):
         cl["q"], hl["q"], cl["q_ik"], cl["q_ik_scale"], cl["head_w"] = q_c, q_h, q_ik, q_ik_s, head_w
         rep.csa.out, rep.csa.lse, rep.hca.out, rep.hca.lse = out_views
         rings.append([rep.csa.cs["ring_k"], rep.hca.cs["ring_k"], rep.csa.cs["ring_ik"]])
-    host_small = []
-    for s in range(PERIOD):
-        hb, hv = _pack(small(s), "cpu", pin=True)
-        for v, t in zip(hv, small(s)):
-            v.copy_(t.cpu())
-        host_small.append(hb)
     host_out = torch.empty(out_buf.shape, dtype=torch.uint8, pin_memory=True)
     bi = host_small[0].numel()
     bo = host_out.numel()
@@ -888,6 +899,41 @@ def run_prefill(args, rank, world, dev):
     return res
 
 
+def run_other_workloads(args, rank, world, dev):
+    """The batched decode workloads (Flash-like B = 8 at 65,536 tokens, k =
+    512; Pro-like B = 4 at 131,072 tokens, k = 1,024) and the 8,192-token
+    chunked prefill on a 1M context, each timed briefly the same way as the
+    headline (decode: graph replays over rotating replicas, per-call times;
+    prefill: events around each call).  Reported beside the headline, not as
+    it."""
+    import argparse as _ap
+    peak, _ = _peaks()
+    out = {}
+    for name in ("flash", "pro"):
+        wl = W.get(name).with_(ik_fmt=args.ik_fmt)
+        a = _ap.Namespace(**vars(args))
+        a.warmup = max(3, min(args.warmup, 10))
+        t = _time_decode(a, wl, rank, world, dev, args.other_steps, 7000, clocks=False,
+                         call_replays=1)
+        ib = indexer_bytes(wl)
+        out[name] = {"metric": f"CSA+HCA decode queries/s ({name}: B={wl.B}, ctx {wl.T}, "
+                               f"k={wl.k})",
+                     "value": round(whole_job_rate(wl.B * t["steps"], t["ms"], world), 2),
+                     "unit": UNIT, "steps": t["steps"], "ms_per_step": t["ms"] / t["steps"],
+                     "indexer_score_us": round(t["idx_ms"] * 1e3, 3),
+                     "indexer_frac": round(ib / (t["idx_ms"] / 1e3) / 1e9 / peak, 4),
+                     "per_call": per_call_report(wl, t["calls"], peak)}
+        del t
+        torch.cuda.empty_cache()
+    a = _ap.Namespace(**vars(args))
+    a.workload, a.warmup, a.steps, a.tq = "prefill", 1, 2, 0
+    r = run_prefill(a, rank, world, dev)
+    out["prefill"] = {k: r[k] for k in ("metric", "value", "unit", "steps", "ms_per_step",
+                                        "roofline", "flop", "calls_ms")}
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -903,14 +949,19 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ik-fmt", default="e4m3vec", choices=["e4m3vec", "e4m3"],
-                    help="FP8 indexer scale layout: one scale per vector, or per 64 dims")
+    ap.add_argument("--ik-fmt", default="e4m3vec", choices=["e4m3vec", "e4m3", "mxfp4"],
+                    help="indexer layout: FP8 with one scale per vector or per 64 dims, or "
+                         "FP4 MXFP4")
     ap.add_argument("--tq", type=int, default=0,
                     help="prefill: new tokens per sequence (0: the workload's chunk); a "
                          "shorter chunk is a smaller case of the same step, for profiling")
     ap.add_argument("--call-replays", type=int, default=4,
                     help="replays of the per-call timing graph (0: skip)")
-    ap.add_argument("--alt-steps", type=int, default=4096,
+    ap.add_argument("--other-workloads", type=int, default=1,
+                    help="1: also time the Flash-like and Pro-like batched decode and the "
+                         "chunked prefill (briefly), reported beside the headline")
+    ap.add_argument("--other-steps", type=int, default=1024)
+    ap.add_argument("--alt-steps", type=int, default=2048,
                     help="steps timed with the other indexer layout (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -939,6 +990,10 @@ def main():
     res["e2e"] = run_e2e(args, replicas, wl, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(replicas[0].csa_L, replicas[0].hca_L, args.cpu_budget)
+    del replicas
+    torch.cuda.empty_cache()
+    if args.other_workloads:
+        res["other_workloads"] = run_other_workloads(args, rank, world, dev)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
