@@ -536,7 +536,7 @@ def run_ours(args, rank, world, dev):
                       "global_batch": wl.B * world, "seq_len": wl.T,
                       "parallelism": f"replicas x{world} (weak)",
                       "l2": f"{R} rotating input replicas, {R * per_rep_bytes / 1e6:.0f} MB "
-                            f"touched per cycle (> 4x L2)",
+                            f"touched per cycle ({R * per_rep_bytes / 126e6:.1f}x the 126 MB L2)",
                       "step_bytes": per_rep_bytes},
            "roofline": roofline,
            "kernels": {"per_call": kernels,

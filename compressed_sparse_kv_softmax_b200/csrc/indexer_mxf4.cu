@@ -23,10 +23,11 @@
 // CTA roles (persistent over the row's tiles assigned to the CTA):
 //   warp 0      TMA producer: key tiles (128 rows x 64 B, 64-byte swizzle)
 //               and their exponent words (bulk copy) into a kStages ring
-//   warp 1      MMA issuer: rearranges each tile's exponent words into the
-//               chunk layout, then one thread copies them to TMEM and issues
-//               the two MMAs into one of the accumulator slots
+//   warp 1      MMA issuer: one thread copies each tile's exponent chunk to
+//               TMEM and issues the two MMAs into one of the accumulator slots
 //   warp 2      TMEM allocation
+//   warp 3      rearranges each tile's exponent words into the chunk layout as
+//               soon as the tile lands (running ahead of the MMA issuer)
 //   warps 4-19  four epilogue warpgroups taking tiles in turn: tcgen05.ld,
 //               ReLU, head weights -> score; score histogram for the selection
 // HBM traffic is the key tile stream: 64 B of codes + 4 B of exponents per
@@ -68,7 +69,8 @@ struct __align__(1024) Smem {
   uint32_t kexp[kStages][kTile];          // the tiles' exponent words as copied
   float w[kHeads];
   uint32_t hist[kTopkBins];
-  uint64_t full[kStages], empty[kStages], acc_full[kAcc], acc_empty[kAcc], mma_done;
+  uint64_t full[kStages], empty[kStages], sf_ready[kStages], acc_full[kAcc], acc_empty[kAcc],
+      mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -92,6 +94,7 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.sf_ready[s], 1);
     }
     for (int s = 0; s < kAcc; ++s) {
       mbar_init(&sm.acc_full[s], 1);
@@ -186,26 +189,57 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
         mbar_wait(&sm.full[i % kStages], (i / kStages) & 1, lim);
     }
   } else if (warp == 1) {
-    // ---------------- exponent chunks and MMA issue
+    // ---------------- MMA issue
+    const int my_tiles = tiles_of(visible_n());
+    if (elect_one()) {
+      tmem_cp_32x128b_x4(tmem + kSfbCol, desc_rows16(smem_addr(sm.sfb)));
+      for (int i = 0; i < my_tiles && !sm.abort; ++i) {
+        const int s = i % kStages, acc = i % kAcc;
+        if (i >= kAcc && !mbar_wait(&sm.acc_empty[acc], ((i / kAcc) & 1) ^ 1, lim)) {
+          record_abort(sm);
+          break;
+        }
+        // the tile's keys have landed and its exponent chunk is laid out
+        if (!mbar_wait(&sm.sf_ready[s], (i / kStages) & 1, lim) ||
+            !mbar_wait(&sm.full[s], (i / kStages) & 1, lim)) {
+          record_abort(sm);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + acc * 64, sfa = tmem + kSfaCol + 4 * acc;
+        tmem_cp_32x128b_x4(sfa, desc_rows16(smem_addr(sm.sfa[s])));
+        const uint32_t ka = smem_addr(sm.keys[s]), qa = smem_addr(sm.q);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          // K = 64 codes = 32 bytes per step; its two exponents start at
+          // byte 2 kk of each 32-bit scale column
+          const uint32_t sf = 2u * kk;
+          mma_mxf4(d, desc_kmajor_sw64(ka + 32 * kk), desc_kmajor_sw64(qa + 32 * kk),
+                   idesc_mxf4(kTile, kHeads, sf, sf), sfa | (sf << 30),
+                   (tmem + kSfbCol) | (sf << 30), kk);
+        }
+        mma_commit(&sm.empty[s]);
+        mma_commit(&sm.acc_full[acc]);
+      }
+      // every MMA of this CTA has finished before TMEM is released
+      mma_commit(&sm.mma_done);
+      if (!mbar_wait(&sm.mma_done, 0, lim)) record_abort(sm);
+    }
+  } else if (warp == 3) {
+    // ---------------- exponent chunks: lane r gathers the exponent words of
+    // entries r, 32 + r, 64 + r, 96 + r of each tile (those the bulk copy did
+    // not bring come from global memory) into row r of the tile's chunk
     const int my_tiles = tiles_of(visible_n());
     const long long total_rows = (long long)a.B * a.ik.cap;
     const uint8_t *exp_base = reinterpret_cast<const uint8_t *>(a.ik.scale);
-    if (elect_one()) tmem_cp_32x128b_x4(tmem + kSfbCol, desc_rows16(smem_addr(sm.sfb)));
-    __syncwarp();
     for (int i = 0; i < my_tiles; ++i) {
       // (the stop flag is read once per warp: the loop stays warp-uniform)
       if (__shfl_sync(0xffffffffu, sm.abort, 0)) break;
-      const int s = i % kStages, acc = i % kAcc;
-      bool ok = true;
-      if (i >= kAcc) ok = mbar_wait(&sm.acc_empty[acc], ((i / kAcc) & 1) ^ 1, lim);
-      ok = ok && mbar_wait(&sm.full[s], (i / kStages) & 1, lim);
-      if (!__all_sync(0xffffffffu, ok)) {
+      const int s = i % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[s], (i / kStages) & 1, lim))) {
         if (lane == 0) record_abort(sm);
         break;
       }
-      tc_fence_after();
-      // lane r gathers the exponent words of entries r, 32 + r, 64 + r, 96 + r
-      // (those the bulk copy did not bring come from global memory)
       const long long g0 = (long long)b * a.ik.cap + (long long)(blockIdx.x + i * gridDim.x) * kTile;
       const long long tile_rows = total_rows - g0;
       const ScaleSpan sp =
@@ -225,30 +259,8 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       *reinterpret_cast<uint4 *>(&sm.sfa[s][16 * lane]) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       fence_proxy_async_shared();
       __syncwarp();
-      if (elect_one()) {
-        const uint32_t d = tmem + acc * 64, sfa = tmem + kSfaCol + 4 * acc;
-        tmem_cp_32x128b_x4(sfa, desc_rows16(smem_addr(sm.sfa[s])));
-        const uint32_t ka = smem_addr(sm.keys[s]), qa = smem_addr(sm.q);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          // K = 64 codes = 32 bytes per step; its two exponents start at
-          // byte 2 kk of each 32-bit scale column
-          const uint32_t sf = 2u * kk;
-          mma_mxf4(d, desc_kmajor_sw64(ka + 32 * kk), desc_kmajor_sw64(qa + 32 * kk),
-                   idesc_mxf4(kTile, kHeads, sf, sf), sfa | (sf << 30),
-                   (tmem + kSfbCol) | (sf << 30), kk);
-        }
-        mma_commit(&sm.empty[s]);
-        mma_commit(&sm.acc_full[acc]);
-      }
-      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.sf_ready[s]);
     }
-    // every MMA of this CTA has finished before TMEM is released
-    if (elect_one()) {
-      mma_commit(&sm.mma_done);
-      if (!mbar_wait(&sm.mma_done, 0, lim)) record_abort(sm);
-    }
-    __syncwarp();
   } else if (warp >= 4) {
     // ---------------- epilogue: the warpgroups take tiles in turn
     const long long n = visible_n();
