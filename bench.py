@@ -511,14 +511,14 @@ def run_ours(args, rank, world, dev):
     achieved = ib / (idx_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": None,
-                "kernel": "indexer_tc_kernel (lightning-indexer scoring: the indexer_score "
-                          "call, one launch)",
+                "kernel": f"{_scoring_kernel(wl)} (lightning-indexer scoring: the "
+                          f"indexer_score call, one launch)",
                 "peak_kind": f"{peak_kind} HBM copy bandwidth (burst)",
                 "algorithmic_bytes_per_launch": ib, "avg_launch_us": round(idx_ms * 1e3, 3),
                 "samples": t["idx_samples"],
                 "timed_launches": f"every {EVENT_EVERY}nd step of the last timed graph replay, "
                                   f"events on a side stream (no serialisation of the step)"}
-    traffic = _profile_traffic("indexer_tc_kernel", wl)
+    traffic = _profile_traffic(_scoring_kernel(wl), wl)
     if traffic is not None:
         roofline["traffic"] = traffic
     kernels = per_call_report(wl, t["calls"], peak)
@@ -551,6 +551,15 @@ def run_ours(args, rank, world, dev):
     if args.alt_steps > 0:
         res["other_indexer_layouts"] = _other_layouts(args, wl, rank, world, dev)
     return res, replicas, wl
+
+
+def _scoring_kernel(wl):
+    """The kernel that the indexer_score call launches for this workload."""
+    if wl.ik_fmt == "mxfp4":
+        return "indexer_mxf4_kernel"
+    if wl.Tq > 1 and wl.ik_fmt == "e4m3vec":
+        return "indexer_rows_kernel"
+    return "indexer_tc_kernel"
 
 
 def _profile_traffic(kernel, wl):
@@ -889,8 +898,8 @@ def run_prefill(args, rank, world, dev):
            "roofline": {"bound": "tensor", "achieved": round(idx_tflops, 2),
                         "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                         "frac": round(idx_tflops / fp8_peak, 4), "traffic": None,
-                        "kernel": "indexer_tc_kernel (indexer_score: FP8 scoring of every "
-                                  "visible entry for each new token)",
+                        "kernel": f"{_scoring_kernel(wl)} (indexer_score: scoring of every "
+                                  f"visible entry for each new token)",
                         "peak_kind": f"{peak_kind} sustained bf16 GEMM x 2 (nominal FP8/BF16 "
                                      f"ratio)",
                         "algorithmic_flop_per_launch": idx_flop},
