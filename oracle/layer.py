@@ -9,6 +9,7 @@ from __future__ import annotations
 import numpy as np
 
 from .method import (attend, dequant_slots, indexer_scores, n_entries, pool_entries,
+                     pool_entries_per_channel,
                      requantize, requantize_mxfp4, ring_slots, scale_block, topk,
                      window_positions)
 
@@ -68,6 +69,12 @@ def layer_compress(L, t_begin, t_end):
     ring_ik = as_numpy_cache(L.get("ring_ik"))
     gw = _np(L["gate_w"]).astype(np.float64)
     gb = _np(L["gate_b"]).astype(np.float64)
+    # the per-channel gate variant: gate_b [pool][D] and the indexer keys' own
+    # gate_w_ik [d_I], gate_b_ik [pool][d_I]
+    per_channel = L.get("gate_mode", "scalar") == "channel"
+    if per_channel and ring_ik is not None:
+        gw_ik = _np(L["gate_w_ik"]).astype(np.float64)
+        gb_ik = _np(L["gate_b_ik"]).astype(np.float64)
     res = []
     for b in range(len(t_begin)):
         js = list(range(n_entries(int(t_begin[b]), stride), n_entries(int(t_end[b]), stride)))
@@ -79,16 +86,28 @@ def layer_compress(L, t_begin, t_end):
         names = ["k"]
         if ring_v is not None:
             vals.append(reader(ring_v)); names.append("v")
-        if ring_ik is not None:
+        if ring_ik is not None and not per_channel:
             vals.append(reader(ring_ik)); names.append("ik")
-        pooled, w = pool_entries(reader(ring_k), vals, gw, gb, pool, stride, js)
-        r = {"j": np.asarray(js, dtype=np.int64), "weights": w}
-        for name, arr in zip(names, pooled):
-            r[name] = arr
         # sum_r a_r |x_{p_r}|: the magnitude scale of each pooled sum, which
         # bounds its floating-point evaluation error
         absvals = [(lambda f: (lambda p: np.abs(f(p))))(v) for v in vals]
-        mags, _ = pool_entries(reader(ring_k), absvals, gw, gb, pool, stride, js)
+        if per_channel:
+            # one gate per channel; the indexer keys have gates of their own
+            pooled, w = pool_entries_per_channel(reader(ring_k), vals, gw, gb, pool, stride, js)
+            mags, _ = pool_entries_per_channel(reader(ring_k), absvals, gw, gb, pool, stride, js)
+            if ring_ik is not None:
+                ri = reader(ring_ik)
+                pi, _ = pool_entries_per_channel(ri, [ri], gw_ik, gb_ik, pool, stride, js)
+                mi, _ = pool_entries_per_channel(ri, [lambda p: np.abs(ri(p))], gw_ik, gb_ik,
+                                                 pool, stride, js)
+                names.append("ik")
+                pooled, mags = list(pooled) + pi, list(mags) + mi
+        else:
+            pooled, w = pool_entries(reader(ring_k), vals, gw, gb, pool, stride, js)
+            mags, _ = pool_entries(reader(ring_k), absvals, gw, gb, pool, stride, js)
+        r = {"j": np.asarray(js, dtype=np.int64), "weights": w}
+        for name, arr in zip(names, pooled):
+            r[name] = arr
         for name, arr in zip(names, mags):
             r[name + "_mag"] = arr
         if ring_k["fmt"] != "f32":

@@ -80,6 +80,47 @@ def pool_entries(gate_src, values, gate_w, gate_b, pool: int, stride: int, j_lis
     return [np.asarray(o) for o in outs], np.asarray(weights)
 
 
+def pool_entries_per_channel(gate_src, values, gate_w, gate_b, pool: int, stride: int,
+                             j_list):
+    """Softmax-gated pooling with one gate per channel (the per-channel
+    variant of the gated pooling with learned positional bias [chaosnode]).
+
+    gate_src(p) -> float64 [D]   the key vector of token p (gate input)
+    values: callables v(p) -> float64 [D], pooled channel by channel with the
+            key's weights (K and V of the separate-V layout share D)
+    gate_w: [D]; gate_b: [pool][D].  For entry j and channel c:
+        g_{r,c} = gate_w[c] * k_{p_r}[c] + gate_b[r][c]   over present slots r,
+        a_{.,c} = softmax_r(g_{.,c}),   out[c] = sum_r a_{r,c} v(p_r)[c].
+    READING: each channel's gate reads that channel of the key alone, with a
+    per-slot, per-channel bias; the pages name the softmax gate and the
+    positional bias but not their shapes.
+    Returns (list of pooled arrays [len(j_list)][D] per value, weights
+    [n][pool][D])."""
+    gate_w = np.asarray(gate_w, dtype=np.float64)
+    gate_b = np.asarray(gate_b, dtype=np.float64)
+    outs = [[] for _ in values]
+    weights = []
+    for j in j_list:
+        pos = pool_positions(j, pool, stride)
+        valid = pos >= 0
+        D = gate_w.shape[0]
+        g = np.full((pool, D), -np.inf)
+        for r in range(pool):
+            if valid[r]:
+                g[r] = gate_w * gate_src(int(pos[r])) + gate_b[r]
+        gmax = np.max(g[valid], axis=0)                 # per channel
+        e = np.where(valid[:, None], np.exp(g - gmax[None, :]), 0.0)
+        a = e / e.sum(axis=0, keepdims=True)
+        weights.append(a)
+        for i, v in enumerate(values):
+            acc = np.zeros(D)
+            for r in range(pool):
+                if valid[r]:
+                    acc = acc + a[r] * v(int(pos[r]))
+            outs[i].append(acc)
+    return [np.asarray(o) for o in outs], np.asarray(weights)
+
+
 def scale_block(fmt: str, d_nope: int) -> int:
     """Dims per fp32 scale: 64 for the KV-cache layout ("e4m3"), the whole
     vector for the indexer layout ("e4m3vec": one scale per key or query

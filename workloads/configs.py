@@ -43,6 +43,8 @@ class Workload:
     needles: int = 0
     needle_mode: str = "uniform"   # "uniform" | "loguniform"
     q_prescale: bool = False       # tiny workload: Q already multiplied by 1/sqrt(head dim)
+    gate_mode: str = "scalar"      # "scalar": g_r = w . k + b[r]; "channel": one gate per
+                                   # channel, g_{r,c} = w_c k_c + b[r][c]
     seed: int = 0
 
     @property

@@ -170,6 +170,18 @@ def _plant_kv_needle(cache: dict, b: int, j: int, q_head0: torch.Tensor, rng: _R
     cache["data"][b, j] = e4m3_from_float(v / s.repeat_interleave(64)[:d_nope])
 
 
+def _channel_gates(rng: _Rng, L: dict, D: int, pool: int, d_I):
+    """Parameters of the per-channel gate variant: gate_w [D] and gate_b
+    [pool][D] ~ N(0, 1) (wide enough that the weights are far from uniform),
+    and the indexer keys' own gate_w_ik [d_I], gate_b_ik [pool][d_I]."""
+    L["gate_mode"] = "channel"
+    L["gate_w"] = rng.normal(D)
+    L["gate_b"] = rng.normal(pool, D)
+    if d_I is not None:
+        L["gate_w_ik"] = rng.normal(d_I)
+        L["gate_b_ik"] = rng.normal(pool, d_I)
+
+
 def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap: int | None = None):
     """Inputs of one CSA layer: raw KV / indexer-key rings, the compressed CSA
     cache and indexer-key cache, queries, indexer queries and weights, gates."""
@@ -203,6 +215,8 @@ def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
     L["head_w"] = rng.normal(wl.B, wl.Tq, wl.H_I) / math.sqrt(wl.H_I)
     L["gate_w"] = rng.normal(wl.D, std=0.1)
     L["gate_b"] = rng.normal(wl.csa_pool, std=0.1)
+    if wl.gate_mode == "channel":
+        _channel_gates(rng, L, wl.D, wl.csa_pool, wl.d_I)
     L["pool"], L["stride"] = wl.csa_pool, wl.csa_stride
     L["q_pos"], L["ctx_len"] = _positions(wl, device)
     L["needles"] = _needle_positions(rng, wl, t_end)
@@ -245,6 +259,8 @@ def make_hca_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
     L["q"] = _queries(rng, wl)
     L["gate_w"] = rng.normal(wl.D, std=0.1)
     L["gate_b"] = rng.normal(wl.hca_pool, std=0.1)
+    if wl.gate_mode == "channel":
+        _channel_gates(rng, L, wl.D, wl.hca_pool, None)
     L["pool"], L["stride"] = wl.hca_pool, wl.hca_stride
     L["q_pos"], L["ctx_len"] = _positions(wl, device)
     L["needles"] = _needle_positions(rng, wl, t_end)
