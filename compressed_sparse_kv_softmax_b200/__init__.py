@@ -46,6 +46,10 @@ _I, _I64, _F, _SZ = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_
 
 _lib.csa_compress.argtypes = [_I, _P, _P, _I64, _PC, _PC, _PC, _P, _P, _I, _I, _PC, _PC, _PC, _P]
 _lib.hca_compress.argtypes = [_I, _P, _P, _I64, _PC, _PC, _P, _P, _I, _I, _PC, _PC, _P]
+_lib.csa_compress_channel_gate.argtypes = [_I, _P, _P, _I64, _PC, _PC, _PC, _P, _P, _P, _P, _I,
+                                           _I, _PC, _PC, _PC, _P]
+_lib.hca_compress_channel_gate.argtypes = [_I, _P, _P, _I64, _PC, _PC, _P, _P, _I, _I, _PC, _PC,
+                                           _P]
 _lib.indexer_score.argtypes = _lib.indexer_select.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC,
                                                              _I, _I, _I64, _P, _P, _P, _SZ, _P]
 _lib.indexer_topk.argtypes = [_I, _I, _P, _P, _P, _P, _I, _I, _PC, _I, _I, _I64, _P, _P, _P,
@@ -73,7 +77,8 @@ _lib.cskv_debug_indexer_stall.restype = ctypes.c_uint32
 _lib.cskv_error_string.argtypes = [_I]
 _lib.cskv_error_string.restype = ctypes.c_char_p
 _lib.cskv_version.restype = _I
-for _name in ("csa_compress", "hca_compress", "indexer_topk", "indexer_score", "indexer_select",
+for _name in ("csa_compress", "hca_compress", "csa_compress_channel_gate",
+              "hca_compress_channel_gate", "indexer_topk", "indexer_score", "indexer_select",
               "hybrid_attn_decode", "hybrid_attn_prefill"):
     getattr(_lib, _name).restype = _I
 
@@ -183,6 +188,29 @@ def hca_compress(B, t_begin, t_end, max_new, raw_k, raw_v, gate_w, gate_b, pool,
     _check(_lib.hca_compress(B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]),
                              _ref(cs[1]), _ptr(gate_w), _ptr(gate_b), pool, stride, _ref(cs[2]),
                              _ref(cs[3]), _stream(stream)), "hca_compress")
+
+
+def csa_compress_channel_gate(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b,
+                              gate_w_ik, gate_b_ik, pool, stride, out_k, out_v, out_ik,
+                              stream=None):
+    """csa_compress with one gate per channel: gate_b [pool][D], the indexer
+    keys' own gate_w_ik [d_I] and gate_b_ik [pool][d_I]."""
+    cs = [cache_struct(c) for c in (raw_k, raw_v, raw_ik, out_k, out_v, out_ik)]
+    _check(_lib.csa_compress_channel_gate(B, _ptr(t_begin), _ptr(t_end), int(max_new),
+                                          _ref(cs[0]), _ref(cs[1]), _ref(cs[2]), _ptr(gate_w),
+                                          _ptr(gate_b), _ptr(gate_w_ik), _ptr(gate_b_ik), pool,
+                                          stride, _ref(cs[3]), _ref(cs[4]), _ref(cs[5]),
+                                          _stream(stream)), "csa_compress_channel_gate")
+
+
+def hca_compress_channel_gate(B, t_begin, t_end, max_new, raw_k, raw_v, gate_w, gate_b, pool,
+                              stride, out_k, out_v, stream=None):
+    """hca_compress with one gate per channel: gate_b [pool][D]."""
+    cs = [cache_struct(c) for c in (raw_k, raw_v, out_k, out_v)]
+    _check(_lib.hca_compress_channel_gate(B, _ptr(t_begin), _ptr(t_end), int(max_new),
+                                          _ref(cs[0]), _ref(cs[1]), _ptr(gate_w), _ptr(gate_b),
+                                          pool, stride, _ref(cs[2]), _ref(cs[3]),
+                                          _stream(stream)), "hca_compress_channel_gate")
 
 
 def indexer_topk(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,

@@ -65,9 +65,13 @@ int check_ws(const void *ws, size_t have, size_t need) {
     if (_rc != CSKV_OK) return _rc; \
   } while (0)
 
+// channel = 0: one scalar gate per token (gate_b [pool]); channel = 1: one
+// gate per channel (gate_b [pool][D], the indexer keys with gate_w_ik [d_I]
+// and gate_b_ik [pool][d_I])
 int compress_common(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
                     const cskv_cache *raw_k, const cskv_cache *raw_v, const cskv_cache *raw_ik,
-                    const float *gate_w, const float *gate_b, int pool, int stride,
+                    const float *gate_w, const float *gate_b, const float *gate_w_ik,
+                    const float *gate_b_ik, int channel, int pool, int stride,
                     const cskv_cache *out_k, const cskv_cache *out_v, const cskv_cache *out_ik,
                     cskv_stream_t stream) {
   if (B < 0 || B > 65535 || max_new < 0 || max_new > 0x7fffffffLL) return CSKV_ERR_ARG;
@@ -96,6 +100,16 @@ int compress_common(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
     if (!rings[i]) continue;
     if (rings[i]->cap < (max_new - 1) * (int64_t)stride + pool) return CSKV_ERR_ARG;
     if (outs[i]->cap < max_new) return CSKV_ERR_ARG;
+  }
+  if (channel) {
+    // the value is pooled with the key's per-channel weights: same channels
+    if (raw_v && raw_v->d_nope + raw_v->d_rope != raw_k->d_nope + raw_k->d_rope)
+      return CSKV_ERR_ARG;
+    if (raw_ik && (!gate_w_ik || !gate_b_ik)) return CSKV_ERR_ARG;
+    return launch_compress_channel(B, t_begin, t_end, max_new, to_dev(raw_k), to_dev(raw_v),
+                                   to_dev(raw_ik), gate_w, gate_b, gate_w_ik, gate_b_ik, pool,
+                                   stride, to_dev(out_k), to_dev(out_v), to_dev(out_ik),
+                                   (cudaStream_t)stream);
   }
   return launch_compress(B, t_begin, t_end, max_new, to_dev(raw_k), to_dev(raw_v),
                          to_dev(raw_ik), gate_w, gate_b, pool, stride, to_dev(out_k),
@@ -205,16 +219,35 @@ int csa_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
                  const float *gate_w, const float *gate_b, int pool, int stride,
                  const cskv_cache *out_k, const cskv_cache *out_v, const cskv_cache *out_ik,
                  cskv_stream_t stream) {
-  return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b, pool,
-                         stride, out_k, out_v, out_ik, stream);
+  return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b,
+                         nullptr, nullptr, 0, pool, stride, out_k, out_v, out_ik, stream);
+}
+
+int csa_compress_channel_gate(int B, const int64_t *t_begin, const int64_t *t_end,
+                              int64_t max_new, const cskv_cache *raw_k, const cskv_cache *raw_v,
+                              const cskv_cache *raw_ik, const float *gate_w, const float *gate_b,
+                              const float *gate_w_ik, const float *gate_b_ik, int pool,
+                              int stride, const cskv_cache *out_k, const cskv_cache *out_v,
+                              const cskv_cache *out_ik, cskv_stream_t stream) {
+  return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b,
+                         gate_w_ik, gate_b_ik, 1, pool, stride, out_k, out_v, out_ik, stream);
 }
 
 int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
                  const cskv_cache *raw_k, const cskv_cache *raw_v, const float *gate_w,
                  const float *gate_b, int pool, int stride, const cskv_cache *out_k,
                  const cskv_cache *out_v, cskv_stream_t stream) {
-  return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, nullptr, gate_w, gate_b, pool,
-                         stride, out_k, out_v, nullptr, stream);
+  return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, nullptr, gate_w, gate_b,
+                         nullptr, nullptr, 0, pool, stride, out_k, out_v, nullptr, stream);
+}
+
+int hca_compress_channel_gate(int B, const int64_t *t_begin, const int64_t *t_end,
+                              int64_t max_new, const cskv_cache *raw_k, const cskv_cache *raw_v,
+                              const float *gate_w, const float *gate_b, int pool, int stride,
+                              const cskv_cache *out_k, const cskv_cache *out_v,
+                              cskv_stream_t stream) {
+  return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, nullptr, gate_w, gate_b,
+                         nullptr, nullptr, 1, pool, stride, out_k, out_v, nullptr, stream);
 }
 
 int cskv_ring_store(int B, const int64_t *pos, int n, const cskv_cache *const *src,

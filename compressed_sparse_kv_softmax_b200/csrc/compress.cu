@@ -403,6 +403,100 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   if (raw_ik.data) store_entry(out_ik, b, j, pi, Di);
 }
 
+
+// ---------------------------------------------------------------------------
+// Per-channel gate variant: one softmax over the window's slots for every
+// channel c, with logits g_{r,c} = gate_w[c] * k_{p_r}[c] + gate_b[r][c] read
+// from that channel of the key alone; the value (separate-V layout) is pooled
+// with the key's weights, the indexer keys with gates of their own.  The
+// window is staged in shared memory as above; each thread then runs an online
+// softmax over the slots for its channels (the bias rows come from L2).
+__device__ __noinline__ void pool_channels(const Cache &c, const SlotLayout &l, const uint8_t *buf,
+                                           const Cache *cv, const SlotLayout &lv,
+                                           const uint8_t *bufv, int r0, int pool,
+                                           const float *__restrict__ gw,
+                                           const float *__restrict__ gb, float *pooled,
+                                           float *pooled_v) {
+  const int D = c.dims();
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    const float w = gw[d];
+    float m = -CUDART_INF_F, s = 0.f, acc = 0.f, accv = 0.f;
+    for (int r = r0; r < pool; ++r) {
+      const float x = staged_value(c, l, buf + (size_t)r * l.bytes, d);
+      const float g = fmaf(w, x, gb[(size_t)r * D + d]);
+      if (g > m) {
+        const float f = expf(m - g);       // (m = -inf: f = 0, the sums are 0)
+        s *= f;
+        acc *= f;
+        accv *= f;
+        m = g;
+      }
+      const float e = expf(g - m);
+      s += e;
+      acc = fmaf(e, x, acc);
+      if (cv) accv = fmaf(e, staged_value(*cv, lv, bufv + (size_t)r * lv.bytes, d), accv);
+    }
+    pooled[d] = acc / s;
+    if (cv) pooled_v[d] = accv / s;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+compress_channel_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__ t_end,
+                        Cache raw_k, Cache raw_v, Cache raw_ik, const float *__restrict__ gate_w,
+                        const float *__restrict__ gate_b, const float *__restrict__ gate_w_ik,
+                        const float *__restrict__ gate_b_ik, int pool, int stride, Cache out_k,
+                        Cache out_v, Cache out_ik) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x;
+  const SlotLayout lk = slot_layout(raw_k);
+  const SlotLayout lv = raw_v.data ? slot_layout(raw_v) : lk;
+  const SlotLayout li = raw_ik.data ? slot_layout(raw_ik) : lk;
+  const int D = raw_k.dims();
+  const int Dv = raw_v.data ? raw_v.dims() : 0, Di = raw_ik.data ? raw_ik.dims() : 0;
+  uint8_t *bk = csm;
+  uint8_t *bv = bk + (size_t)pool * lk.bytes;
+  uint8_t *bi = bv + (raw_v.data ? (size_t)pool * lv.bytes : 0);
+  float *pk = reinterpret_cast<float *>(bi + (raw_ik.data ? (size_t)pool * li.bytes : 0));
+  float *pv = pk + round16(D);
+  float *pi = pv + round16(Dv);
+  long long *rows = reinterpret_cast<long long *>(pi + round16(Di));
+  long long *rows_v = rows + pool;
+  long long *rows_i = rows_v + pool;
+
+  const long long j = t_begin[b] / stride + blockIdx.x;
+  // never write past a cache's capacity, whatever the device-side token counts say
+  if (j >= t_end[b] / stride || j < 0 || j >= out_k.cap || (raw_v.data && j >= out_v.cap) ||
+      (raw_ik.data && j >= out_ik.cap))
+    return;
+  const long long first = (long long)stride * (j + 1) - pool;
+  for (int r = tid; r < pool; r += blockDim.x) {
+    const long long p = first + r;
+    rows[r] = p < 0 ? -1 : raw_k.row(b, raw_k.slot_of(p));
+    if (raw_v.data) rows_v[r] = p < 0 ? -1 : raw_v.row(b, raw_v.slot_of(p));
+    if (raw_ik.data) rows_i[r] = p < 0 ? -1 : raw_ik.row(b, raw_ik.slot_of(p));
+  }
+  __syncthreads();
+  stage_window(raw_k, lk, rows, pool, bk);
+  if (raw_v.data) stage_window(raw_v, lv, rows_v, pool, bv);
+  if (raw_ik.data) stage_window(raw_ik, li, rows_i, pool, bi);
+  cp_async_wait_all();
+  __syncthreads();
+
+  const int r0 = first < 0 ? (int)-first : 0;
+  pool_channels(raw_k, lk, bk, raw_v.data ? &raw_v : nullptr, lv, bv, r0, pool, gate_w, gate_b,
+                pk, pv);
+  if (raw_ik.data)
+    pool_channels(raw_ik, li, bi, nullptr, li, bi, r0, pool, gate_w_ik, gate_b_ik, pi, nullptr);
+  __syncthreads();
+  store_entry(out_k, b, j, pk, D);
+  if (raw_v.data) store_entry(out_v, b, j, pv, Dv);
+  if (raw_ik.data) store_entry(out_ik, b, j, pi, Di);
+}
+
 }  // namespace
 
 int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
@@ -436,6 +530,29 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
       return CSKV_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;
+}
+
+int launch_compress_channel(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
+                            const Cache &raw_k, const Cache &raw_v, const Cache &raw_ik,
+                            const float *gate_w, const float *gate_b, const float *gate_w_ik,
+                            const float *gate_b_ik, int pool, int stride, const Cache &out_k,
+                            const Cache &out_v, const Cache &out_ik, cudaStream_t st) {
+  if (max_new == 0 || B == 0) return CSKV_OK;
+  size_t staged = (size_t)pool * slot_layout(raw_k).bytes;
+  if (raw_v.data) staged += (size_t)pool * slot_layout(raw_v).bytes;
+  if (raw_ik.data) staged += (size_t)pool * slot_layout(raw_ik).bytes;
+  const int Dk = raw_k.dims(), Dv = raw_v.data ? raw_v.dims() : 0;
+  const int Di = raw_ik.data ? raw_ik.dims() : 0;
+  const size_t smem = staged + sizeof(float) * (size_t)(round16(Dk) + round16(Dv) + round16(Di)) +
+                      3 * sizeof(long long) * (size_t)pool + 16;
+  // the staged window must fit in shared memory (HCA's 128 FP8 slots: 78 KB)
+  if (smem > 200 * 1024 || !ensure_dynamic_smem(compress_channel_kernel, smem))
+    return CSKV_ERR_UNSUPPORTED;
+  if (launch_pdl(compress_channel_kernel, dim3((unsigned)max_new, (unsigned)B), dim3(kThreads),
+                 smem, st, t_begin, t_end, raw_k, raw_v, raw_ik, gate_w, gate_b, gate_w_ik,
+                 gate_b_ik, pool, stride, out_k, out_v, out_ik) != cudaSuccess)
+    return CSKV_ERR_CUDA;
+  return CSKV_OK;
 }
 
 }  // namespace cskv

@@ -224,6 +224,11 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
                     const float *gate_w, const float *gate_b, int pool, int stride,
                     const Cache &out_k, const Cache &out_v, const Cache &out_ik,
                     cudaStream_t st);
+int launch_compress_channel(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
+                            const Cache &raw_k, const Cache &raw_v, const Cache &raw_ik,
+                            const float *gate_w, const float *gate_b, const float *gate_w_ik,
+                            const float *gate_b_ik, int pool, int stride, const Cache &out_k,
+                            const Cache &out_v, const Cache &out_ik, cudaStream_t st);
 
 int launch_ring_store(int B, const int64_t *pos, int n, const Cache *src, const Cache *ring,
                       cudaStream_t st);

@@ -11,9 +11,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (attn_workspace_size, cache_struct, csa_compress, hca_compress,
-               hybrid_attn_decode, hybrid_attn_prefill, indexer_score, indexer_select,
-               indexer_topk, indexer_workspace_size, workspace)
+from . import (attn_workspace_size, cache_struct, csa_compress, csa_compress_channel_gate,
+               hca_compress, hca_compress_channel_gate, hybrid_attn_decode, hybrid_attn_prefill,
+               indexer_score, indexer_select, indexer_topk, indexer_workspace_size, workspace)
 
 
 def _dims(c):
@@ -56,6 +56,12 @@ class CSALayer:
 
     def compress(self, t_begin, t_end, max_new):
         L, c = self.L, self.cs
+        if L.get("gate_mode", "scalar") == "channel":
+            csa_compress_channel_gate(self.B, t_begin, t_end, max_new, c["ring_k"], c["ring_v"],
+                                      c["ring_ik"], L["gate_w"], L["gate_b"], L.get("gate_w_ik"),
+                                      L.get("gate_b_ik"), L["pool"], L["stride"], c["comp_k"],
+                                      c["comp_v"], c["comp_ik"])
+            return
         csa_compress(self.B, t_begin, t_end, max_new, c["ring_k"], c["ring_v"], c["ring_ik"],
                      L["gate_w"], L["gate_b"], L["pool"], L["stride"], c["comp_k"], c["comp_v"],
                      c["comp_ik"])
@@ -113,8 +119,10 @@ class HCALayer:
 
     def compress(self, t_begin, t_end, max_new):
         L, c = self.L, self.cs
-        hca_compress(self.B, t_begin, t_end, max_new, c["ring_k"], c["ring_v"], L["gate_w"],
-                     L["gate_b"], L["pool"], L["stride"], c["comp_k"], c["comp_v"])
+        fn = (hca_compress_channel_gate if L.get("gate_mode", "scalar") == "channel"
+              else hca_compress)
+        fn(self.B, t_begin, t_end, max_new, c["ring_k"], c["ring_v"], L["gate_w"], L["gate_b"],
+           L["pool"], L["stride"], c["comp_k"], c["comp_v"])
 
     def attend(self, pos=None):
         """Dense hybrid attention; pos overrides q_pos (prefill) or ctx_len (decode)."""

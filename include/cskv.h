@@ -165,6 +165,35 @@ int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
                  const cskv_cache *out_k, const cskv_cache *out_v, cskv_stream_t stream);
 
 /*
+ * csa_compress_channel_gate / hca_compress_channel_gate - the per-channel
+ * gate variant of the same pooling (the pages name a softmax gate with a
+ * learned positional bias, «DeepSeek-V4: 1 Million Token Context endlich
+ * nutzbar», "Hybrid Attention: CSA und HCA", without its shape; this variant
+ * gives every channel its own gate).  For entry j and channel c:
+ *     g_{r,c} = gate_w[c] * k_{p_r}[c] + gate_b[r][c]      (present slots r)
+ *     a_{.,c} = softmax_r(g_{.,c}),   entry[c] = sum_r a_{r,c} x_{p_r}[c]
+ * over the dequantised key k; the value (raw_v, separate-V layout, same
+ * channel count as the key) is pooled with the key's weights; the indexer
+ * keys have gates of their own read from themselves (gate_w_ik [d_I],
+ * gate_b_ik [pool][d_I], both required when raw_ik is given).
+ *   gate_w : [D] fp32.   gate_b : [pool][D] fp32 (row r = slot r).
+ * Everything else (positions, formats, re-quantisation, requirements) as
+ * csa_compress / hca_compress.  The window of every plane is staged in shared
+ * memory: CSKV_ERR_UNSUPPORTED when it does not fit (more than 200 KB).
+ */
+int csa_compress_channel_gate(int B, const int64_t *t_begin, const int64_t *t_end,
+                              int64_t max_new, const cskv_cache *raw_k, const cskv_cache *raw_v,
+                              const cskv_cache *raw_ik, const float *gate_w, const float *gate_b,
+                              const float *gate_w_ik, const float *gate_b_ik, int pool,
+                              int stride, const cskv_cache *out_k, const cskv_cache *out_v,
+                              const cskv_cache *out_ik, cskv_stream_t stream);
+int hca_compress_channel_gate(int B, const int64_t *t_begin, const int64_t *t_end,
+                              int64_t max_new, const cskv_cache *raw_k, const cskv_cache *raw_v,
+                              const float *gate_w, const float *gate_b, int pool, int stride,
+                              const cskv_cache *out_k, const cskv_cache *out_v,
+                              cskv_stream_t stream);
+
+/*
  * cskv_ring_store - appends one new raw token per sequence to raw-token
  * rings: for each ring i and sequence b, the token held in slot 0 of
  * sequence b of src[i] (a cache of cap >= 1 slots per sequence, ring = 0)

@@ -34,10 +34,13 @@ def _run_compress(C, L, Ld, t_begin, t_end, kind):
     return O.layer_compress(L, t_begin, t_end)
 
 
+@pytest.mark.parametrize("gate_mode", ["scalar", "channel"])
 @pytest.mark.parametrize("kind", ["csa", "hca"])
 @pytest.mark.parametrize("span", [1, 4, 300])
-def test_compress_f32_tiny(C, kind, span):
-    wl = W.get("tiny").with_(T=4096 + 7)
+def test_compress_f32_tiny(C, kind, span, gate_mode):
+    # (gate_mode "channel": one softmax gate per channel, separate V pooled
+    # with the key's weights, indexer keys with gates of their own)
+    wl = W.get("tiny").with_(T=4096 + 7, gate_mode=gate_mode)
     mk = W.make_csa_layer if kind == "csa" else W.make_hca_layer
     L = mk(wl, ring_cap=1024)
     Ld = to_device(L)
@@ -50,10 +53,13 @@ def test_compress_f32_tiny(C, kind, span):
         check_pooled_f32(got, ref[name], ref[name + "_mag"], where=f"{kind} {name}")
 
 
-@pytest.mark.parametrize("kind,ik_fmt", [("csa", "e4m3vec"), ("csa", "e4m3"), ("hca", "e4m3vec"),
-                                         ("csa", "mxfp4")])
-def test_compress_e4m3_parity_decode(C, kind, ik_fmt):
-    wl = W.get("parity_decode").with_(ik_fmt=ik_fmt)
+@pytest.mark.parametrize("kind,ik_fmt,gate_mode",
+                         [("csa", "e4m3vec", "scalar"), ("csa", "e4m3", "scalar"),
+                          ("hca", "e4m3vec", "scalar"), ("csa", "mxfp4", "scalar"),
+                          ("csa", "e4m3vec", "channel"), ("hca", "e4m3vec", "channel"),
+                          ("csa", "mxfp4", "channel")])
+def test_compress_e4m3_parity_decode(C, kind, ik_fmt, gate_mode):
+    wl = W.get("parity_decode").with_(ik_fmt=ik_fmt, gate_mode=gate_mode)
     mk = W.make_csa_layer if kind == "csa" else W.make_hca_layer
     L = mk(wl, ring_cap=1024)
     Ld = to_device(L)
@@ -77,9 +83,10 @@ def test_compress_e4m3_parity_decode(C, kind, ik_fmt):
     assert n_checked > 0
 
 
-def test_compress_first_entries_left_edge(C):
+@pytest.mark.parametrize("gate_mode", ["scalar", "channel"])
+def test_compress_first_entries_left_edge(C, gate_mode):
     # the first CSA entries see positions < 0 (absent slots)
-    wl = W.get("parity_decode").with_(T=40, B=1)
+    wl = W.get("parity_decode").with_(T=40, B=1, gate_mode=gate_mode)
     L = W.make_csa_layer(wl, ring_cap=64)
     Ld = to_device(L)
     ref = _run_compress(C, L, Ld, [0], [40], "csa")[0]
