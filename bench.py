@@ -911,7 +911,8 @@ def run_prefill(args, rank, world, dev):
 def run_other_workloads(args, rank, world, dev):
     """The batched decode workloads (Flash-like B = 8 at 65,536 tokens, k =
     512; Pro-like B = 4 at 131,072 tokens, k = 1,024), the 1M-context step
-    with the per-channel gate variant of the compressors, and the 8,192-token
+    with the per-channel gate variant of the compressors and with paged
+    compressed caches (256-entry blocks), and the 8,192-token
     chunked prefill on a 1M context, each timed briefly the same way as the
     headline (decode: graph replays over rotating replicas, per-call times;
     prefill: events around each call).  Reported beside the headline, not as
@@ -919,10 +920,13 @@ def run_other_workloads(args, rank, world, dev):
     import argparse as _ap
     peak, _ = _peaks()
     out = {}
-    for name in ("flash", "pro", "long_channel_gate"):
+    for name in ("flash", "pro", "long_channel_gate", "long_paged"):
         if name == "long_channel_gate":
             # the headline step with the per-channel gate variant of the compressors
             wl = W.get("long").with_(ik_fmt=args.ik_fmt, gate_mode="channel")
+        elif name == "long_paged":
+            # the headline step with its compressed caches paged in 256-entry blocks
+            wl = W.get("long").with_(ik_fmt=args.ik_fmt, page_block=256)
         else:
             wl = W.get(name).with_(ik_fmt=args.ik_fmt)
         a = _ap.Namespace(**vars(args))
@@ -931,7 +935,8 @@ def run_other_workloads(args, rank, world, dev):
                          call_replays=1)
         ib = indexer_bytes(wl)
         out[name] = {"metric": f"CSA+HCA decode queries/s ({name}: B={wl.B}, ctx {wl.T}, "
-                               f"k={wl.k}, gate {wl.gate_mode})",
+                               f"k={wl.k}, gate {wl.gate_mode}, "
+                               f"{'paged %d' % wl.page_block if wl.page_block else 'contiguous'})",
                      "value": round(whole_job_rate(wl.B * t["steps"], t["ms"], world), 2),
                      "unit": UNIT, "steps": t["steps"], "ms_per_step": t["ms"] / t["steps"],
                      "indexer_score_us": round(t["idx_ms"] * 1e3, 3),

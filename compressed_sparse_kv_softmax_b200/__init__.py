@@ -37,7 +37,9 @@ class CskvCache(ctypes.Structure):
                 ("ring", ctypes.c_int32), ("cap", ctypes.c_int64),
                 ("data", ctypes.c_void_p), ("data_stride", ctypes.c_int64),
                 ("scale", ctypes.c_void_p), ("scale_stride", ctypes.c_int64),
-                ("rope", ctypes.c_void_p), ("rope_stride", ctypes.c_int64)]
+                ("rope", ctypes.c_void_p), ("rope_stride", ctypes.c_int64),
+                ("block_table", ctypes.c_void_p), ("block_size", ctypes.c_int64),
+                ("num_blocks", ctypes.c_int64)]
 
 
 _P = ctypes.c_void_p
@@ -105,8 +107,8 @@ def _slot_bytes(t):
 
 def cache_struct(c):
     """C descriptor for a cache given as a dict of planes
-    {"fmt": "f32"|"e4m3"|"e4m3vec", "d_nope", "d_rope", "ring", "cap", "data", "scale",
-    "rope"}
+    {"fmt": "f32"|"e4m3"|"e4m3vec"|"mxfp4", "d_nope", "d_rope", "ring", "cap", "data",
+    "scale", "rope"} and, for a paged cache, "block_table", "block_size", "num_blocks"
     (or None).  A CskvCache is returned as it is: callers that pass the same
     cache every step can build its descriptor once."""
     if c is None or isinstance(c, CskvCache):
@@ -121,6 +123,12 @@ def cache_struct(c):
         s.scale, s.scale_stride = sc.data_ptr(), _slot_bytes(sc)
     if rp is not None:
         s.rope, s.rope_stride = rp.data_ptr(), _slot_bytes(rp)
+    bt = c.get("block_table")
+    if bt is not None:
+        # paged: the planes hold num_blocks x block_size rows shared by all
+        # sequences; block_table [B][cap / block_size] int32
+        s.block_table, s.block_size = bt.data_ptr(), int(c["block_size"])
+        s.num_blocks = int(c["num_blocks"])
     return s
 
 

@@ -19,6 +19,18 @@ int check_cache(const cskv_cache *c, int ring) {
   if (ring >= 0 && c->ring != ring) return CSKV_ERR_ARG;
   if (c->cap < 1 || c->d_nope < 0 || c->d_rope < 0 || c->d_nope + c->d_rope < 1)
     return CSKV_ERR_ARG;
+  // (the device descriptor holds dims in 16 bits and strides in 32)
+  if (c->d_nope > 16384 || c->d_rope > 16384 || c->data_stride < 0 || c->scale_stride < 0 ||
+      c->rope_stride < 0 || c->data_stride >= (1LL << 31) || c->scale_stride >= (1LL << 31) ||
+      c->rope_stride >= (1LL << 31))
+    return CSKV_ERR_ARG;
+  if (c->block_table) {
+    // paged: compressed caches only, power-of-two blocks dividing cap
+    if (c->ring || c->block_size < 1 || (c->block_size & (c->block_size - 1)) ||
+        c->cap % c->block_size || c->num_blocks < 1 || c->num_blocks > (1LL << 31) - 1 ||
+        ((uintptr_t)c->block_table & 3))
+      return CSKV_ERR_ARG;
+  }
   if (!aligned16(c->data) || c->data_stride % 16) return CSKV_ERR_ARG;
   if (c->fmt == CSKV_FMT_F32) {
     if (c->data_stride < 4LL * (c->d_nope + c->d_rope)) return CSKV_ERR_ARG;

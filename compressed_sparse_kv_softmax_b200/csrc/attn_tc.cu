@@ -315,8 +315,10 @@ __device__ __forceinline__ Row row_of(const AttnArgs &a, int row) {
 // dims][64 hi rows, 64 lo rows][128 B, 128-byte swizzle], converted once per
 // call for all query rows of a chunk.  Entries at or past the furthest row's
 // visible count are zero (cache slots past it may hold anything).
+template <bool kPaged>
 __global__ void __launch_bounds__(kThreads)
 key_tiles_kernel(const AttnArgs a, uint8_t *__restrict__ tiles, int tile_units) {
+  constexpr int kRM = kPaged ? kRowAuto : kRowFlat;
   __shared__ long long s_max[kThreads / 32];
   pdl_wait();
   pdl_trigger();
@@ -352,8 +354,8 @@ key_tiles_kernel(const AttnArgs a, uint8_t *__restrict__ tiles, int tile_units) 
     p.code[k] = make_uint4(0, 0, 0, 0);
     p.sc[k] = 0.f;
     if (live && c < kCodeUnits) {
-      p.code[k] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, j)) + c);
-      p.sc[k] = __ldg(src.scale_ptr(b, j) + (c >> 2));
+      p.code[k] = __ldg(reinterpret_cast<const uint4 *>(src.template data_ptr<kRM>(b, j)) + c);
+      p.sc[k] = __ldg(src.template scale_ptr<kRM>(b, j) + (c >> 2));
     }
   }
 #pragma unroll
@@ -361,20 +363,22 @@ key_tiles_kernel(const AttnArgs a, uint8_t *__restrict__ tiles, int tile_units) 
     const int v = code_unit(lane, lg, k);
     p.rope[k] = make_uint4(0, 0, 0, 0);
     if (live && v < kRopeUnits)
-      p.rope[k] = __ldg(reinterpret_cast<const uint4 *>(src.rope_ptr(b, j)) + v);
+      p.rope[k] = __ldg(reinterpret_cast<const uint4 *>(src.template rope_ptr<kRM>(b, j)) + v);
   }
   convert_parts(tiles + ((size_t)b * tile_units + unit) * (8 * kChunkKK), p, my_r, lane, lg);
 }
 
 // kTiles: dense entries come as pre-converted key tiles (chunked prefill);
-// kMulti: a CTA runs several units (the running output may need rescaling).
+// kMulti: a CTA runs several units (the running output may need rescaling);
+// kPaged: the compressed cache may be paged (block table).
 // Separate instantiations keep those paths out of the decode kernel's code
-// (one unit per CTA, gathered or bulk-copied rows).
-template <bool kTiles, bool kMulti>
+// (one unit per CTA, gathered or bulk-copied rows, contiguous cache).
+template <bool kTiles, bool kMulti, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, int units_per_cta,
                int n_splits, float *__restrict__ part_o, float *__restrict__ part_lse,
                const uint8_t *__restrict__ tiles, int tile_units) {
+  constexpr int kRM = kPaged ? kRowAuto : kRowFlat;   // (the window's ring is never paged)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
@@ -450,7 +454,10 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
         reinterpret_cast<const __nv_bfloat16 *>(a.q) + (size_t)row * kHeads * kD;
     // consecutive slots: the window's positions (one or two runs around the
     // ring) or dense compressed entries (one run)
-    const bool runs_ok = !q_ready && dense_rows(src) && !(comp_unit && a.sel);
+    // (paged caches: a unit's run of at most 64 entries stays inside one
+    // block of 64 or more)
+    const bool runs_ok = !q_ready && dense_rows(src) && !(comp_unit && a.sel) &&
+                         (!kPaged || !src.bt || src.bs_log2 >= 6);
     if (kTiles && comp_unit) {
       // dense entries converted once for every row of the call: the unit's
       // key tile arrives whole by bulk copies (the previous unit's MMAs, the
@@ -485,9 +492,11 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
         for (int k = 0; k < 2; ++k) {
           if (n_run[k] <= 0) continue;
           const int r = r_run[k], n = n_run[k];
-          bulk_load(sm.q + r * kDn, src.data_ptr(b, s_run[k]), n * kDn, &sm.gbar);
-          bulk_load(sm.q + kStgScale + r * 32, src.scale_ptr(b, s_run[k]), n * 32, &sm.gbar);
-          bulk_load(sm.q + kStgRope + r * 2 * kDr, src.rope_ptr(b, s_run[k]), n * 2 * kDr,
+          bulk_load(sm.q + r * kDn, src.template data_ptr<kRM>(b, s_run[k]), n * kDn, &sm.gbar);
+          bulk_load(sm.q + kStgScale + r * 32, src.template scale_ptr<kRM>(b, s_run[k]), n * 32,
+                    &sm.gbar);
+          bulk_load(sm.q + kStgRope + r * 2 * kDr, src.template rope_ptr<kRM>(b, s_run[k]),
+                    n * 2 * kDr,
                     &sm.gbar);
         }
       }
@@ -530,8 +539,8 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
         p.code[k] = make_uint4(0, 0, 0, 0);
         p.sc[k] = 0.f;
         if (slot >= 0 && j < kCodeUnits) {
-          p.code[k] = __ldg(reinterpret_cast<const uint4 *>(src.data_ptr(b, slot)) + j);
-          p.sc[k] = __ldg(src.scale_ptr(b, slot) + (j >> 2));
+          p.code[k] = __ldg(reinterpret_cast<const uint4 *>(src.template data_ptr<kRM>(b, slot)) + j);
+          p.sc[k] = __ldg(src.template scale_ptr<kRM>(b, slot) + (j >> 2));
         }
       }
 #pragma unroll
@@ -539,7 +548,7 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
         const int v = code_unit(lane, lg, k);
         p.rope[k] = make_uint4(0, 0, 0, 0);
         if (slot >= 0 && v < kRopeUnits)
-          p.rope[k] = __ldg(reinterpret_cast<const uint4 *>(src.rope_ptr(b, slot)) + v);
+          p.rope[k] = __ldg(reinterpret_cast<const uint4 *>(src.template rope_ptr<kRM>(b, slot)) + v);
       }
       if (!q_ready) {
         stage_q(qg, sm.q);
@@ -772,15 +781,20 @@ int launch_attn_tc(const AttnArgs &a, const AttnPlan &p, float *part_o, float *p
   const size_t tb = attn_tc_tile_bytes(a.B, a.Tq, a.max_entries);
   const bool use_tiles = a.has_comp && !a.sel && p.splits == 1 && p.unit == kKeys && tb &&
                          a.ws && a.ws_bytes >= tb && !((uintptr_t)a.ws & 127);
-  auto kernel = use_tiles ? attn_tc_kernel<true, true>
-                          : (p.per_cta > 1 ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>);
+  // (the compressed cache is the only one that can be paged)
+  const bool paged = a.has_comp && (a.comp_k.bt || a.comp_v.bt);
+  auto kernel = use_tiles ? (paged ? attn_tc_kernel<true, true, true> : attn_tc_kernel<true, true, false>)
+                : p.per_cta > 1
+                    ? (paged ? attn_tc_kernel<false, true, true> : attn_tc_kernel<false, true, false>)
+                    : (paged ? attn_tc_kernel<false, false, true> : attn_tc_kernel<false, false, false>);
   if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   const uint8_t *tiles = nullptr;
   int tile_units = 0;
   if (use_tiles) {
     tile_units = (int)((a.max_entries + kKeys - 1) / kKeys);
-    if (launch_pdl(key_tiles_kernel, dim3((unsigned)tile_units, (unsigned)a.B), dim3(kThreads), 0,
-                   st, a, reinterpret_cast<uint8_t *>(a.ws), tile_units) != cudaSuccess)
+    if (launch_pdl(paged ? key_tiles_kernel<true> : key_tiles_kernel<false>,
+                   dim3((unsigned)tile_units, (unsigned)a.B), dim3(kThreads), 0, st, a,
+                   reinterpret_cast<uint8_t *>(a.ws), tile_units) != cudaSuccess)
       return CSKV_ERR_CUDA;
     tiles = reinterpret_cast<const uint8_t *>(a.ws);
   }

@@ -57,23 +57,27 @@ __device__ __forceinline__ void store_mxfp4_block(uint8_t *codes, uint8_t *exps,
   if (lane == 0) exps[blk] = (uint8_t)(X + 127);
 }
 
+// kPaged: the output cache may be paged (its row comes from the block
+// table); the contiguous instantiation carries no paging code
+template <bool kPaged>
 __device__ __noinline__ void store_entry(const Cache &out, int b, long long j,
                                         const float *pooled, int D) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long orow = out.row<kPaged ? kRowAuto : kRowFlat>(b, j);
   if (out.fmt == CSKV_FMT_F32) {
-    float *dst = reinterpret_cast<float *>(out.data + out.row(b, j) * out.data_stride);
+    float *dst = reinterpret_cast<float *>(out.data + orow * out.data_stride);
     for (int d = tid; d < D; d += kThreads) dst[d] = pooled[d];
     return;
   }
   if (out.fmt == CSKV_FMT_MXFP4) {
-    uint8_t *codes = out.data + out.row(b, j) * out.data_stride;
-    uint8_t *exps = out.scale + out.row(b, j) * out.scale_stride;
+    uint8_t *codes = out.data + orow * out.data_stride;
+    uint8_t *exps = out.scale + orow * out.scale_stride;
     for (int blk = warp; blk < (out.d_nope >> 5); blk += kWarps)
       store_mxfp4_block(codes, exps, blk, pooled[blk * 32 + lane]);
     return;
   }
-  uint8_t *codes = out.data + out.row(b, j) * out.data_stride;
-  float *scales = reinterpret_cast<float *>(out.scale + out.row(b, j) * out.scale_stride);
+  uint8_t *codes = out.data + orow * out.data_stride;
+  float *scales = reinterpret_cast<float *>(out.scale + orow * out.scale_stride);
   if (out.fmt == CSKV_FMT_E4M3_VEC) {
     // one scale for the whole vector: warp 0 finds its amax and encodes
     if (warp == 0) {
@@ -98,7 +102,7 @@ __device__ __noinline__ void store_entry(const Cache &out, int b, long long j,
   }
   if (out.d_rope) {
     __nv_bfloat16 *rope =
-        reinterpret_cast<__nv_bfloat16 *>(out.rope + out.row(b, j) * out.rope_stride);
+        reinterpret_cast<__nv_bfloat16 *>(out.rope + orow * out.rope_stride);
     for (int r = tid; r < out.d_rope; r += kThreads)
       rope[r] = __float2bfloat16_rn(pooled[out.d_nope + r]);
   }
@@ -112,17 +116,20 @@ __device__ void pool_values(const Cache &raw, int b, long long first, int pool, 
     for (int r = 0; r < pool; ++r) {
       const long long p = first + r;
       if (p < 0) continue;
-      acc = fmaf(a[r], raw.value(b, raw.slot_of(p), d), acc);
+      acc = fmaf(a[r], raw.value<kRowFlat>(b, raw.slot_of(p), d), acc);
     }
     pooled[d] = acc;
   }
 }
 
+template <bool kPaged>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__ t_end,
-                Cache raw_k, Cache raw_v, Cache raw_ik, const float *__restrict__ gate_w,
-                const float *__restrict__ gate_b, int pool, int stride, Cache out_k,
-                Cache out_v, Cache out_ik) {
+                Cache raw_k, Cache raw_v,
+                Cache raw_ik, const float *__restrict__ gate_w,
+                const float *__restrict__ gate_b, int pool, int stride,
+                Cache out_k, Cache out_v,
+                Cache out_ik) {
   extern __shared__ float smem[];
   pdl_wait();
   pdl_trigger();
@@ -131,8 +138,12 @@ compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__
   const int b = blockIdx.y;
   const long long j = t_begin[b] / stride + blockIdx.x;
   if (j >= t_end[b] / stride || j < 0) return;
-  // never write past a cache's capacity, whatever the device-side token counts say
+  // never write past a cache's capacity, whatever the device-side token counts
+  // say, nor into a slot that a paged cache's block table leaves without a block
   if (j >= out_k.cap || (raw_v.data && j >= out_v.cap) || (raw_ik.data && j >= out_ik.cap))
+    return;
+  if (kPaged && (!out_k.mapped(b, j) || (raw_v.data && !out_v.mapped(b, j)) ||
+                 (raw_ik.data && !out_ik.mapped(b, j))))
     return;
   const long long first = (long long)stride * (j + 1) - pool;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -144,7 +155,8 @@ compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__
     float acc = 0.f;
     if (p >= 0) {
       const long long slot = raw_k.slot_of(p);
-      for (int d = lane; d < D; d += 32) acc = fmaf(gate_w[d], raw_k.value(b, slot, d), acc);
+      for (int d = lane; d < D; d += 32)
+        acc = fmaf(gate_w[d], raw_k.value<kRowFlat>(b, slot, d), acc);
     }
     acc = warp_sum(acc);
     if (lane == 0) a[r] = p >= 0 ? acc + gate_b[r] : -CUDART_INF_F;
@@ -166,18 +178,18 @@ compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__
 
   pool_values(raw_k, b, first, pool, a, pooled);
   __syncthreads();
-  store_entry(out_k, b, j, pooled, D);
+  store_entry<kPaged>(out_k, b, j, pooled, D);
   __syncthreads();
   if (raw_v.data) {
     pool_values(raw_v, b, first, pool, a, pooled);
     __syncthreads();
-    store_entry(out_v, b, j, pooled, raw_v.dims());
+    store_entry<kPaged>(out_v, b, j, pooled, raw_v.dims());
     __syncthreads();
   }
   if (raw_ik.data) {
     pool_values(raw_ik, b, first, pool, a, pooled);
     __syncthreads();
-    store_entry(out_ik, b, j, pooled, raw_ik.dims());
+    store_entry<kPaged>(out_ik, b, j, pooled, raw_ik.dims());
   }
 }
 
@@ -311,11 +323,37 @@ __device__ __noinline__ void pool_staged(const Cache &c, const SlotLayout &l, co
   }
 }
 
+template <bool kPaged, bool kSmemDesc>
 __global__ void __launch_bounds__(kThreads, 1)
 compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__ t_end,
-                       Cache raw_k, Cache raw_v, Cache raw_ik, const float *__restrict__ gate_w,
-                       const float *__restrict__ gate_b, int pool, int stride, Cache out_k,
-                       Cache out_v, Cache out_ik) {
+                       Cache p_raw_k, Cache p_raw_v,
+                       Cache p_raw_ik, const float *__restrict__ gate_w,
+                       const float *__restrict__ gate_b, int pool, int stride,
+                       Cache p_out_k, Cache p_out_v,
+                       Cache p_out_ik) {
+  // the cache descriptors: for a long pooling window (HCA), once in shared
+  // memory, where the out-of-line helpers read them (a reference to a kernel
+  // parameter makes every thread copy it to local memory, which the many
+  // per-slot reads then pay for); for a short one (CSA) the per-thread copy
+  // costs less than the extra barrier
+  __shared__ Cache s_caches[6];
+  if constexpr (kSmemDesc) {
+    if (threadIdx.x == 0) {
+      s_caches[0] = p_raw_k;
+      s_caches[1] = p_raw_v;
+      s_caches[2] = p_raw_ik;
+      s_caches[3] = p_out_k;
+      s_caches[4] = p_out_v;
+      s_caches[5] = p_out_ik;
+    }
+    __syncthreads();
+  }
+  const Cache &raw_k = kSmemDesc ? s_caches[0] : p_raw_k;
+  const Cache &raw_v = kSmemDesc ? s_caches[1] : p_raw_v;
+  const Cache &raw_ik = kSmemDesc ? s_caches[2] : p_raw_ik;
+  const Cache &out_k = kSmemDesc ? s_caches[3] : p_out_k;
+  const Cache &out_v = kSmemDesc ? s_caches[4] : p_out_v;
+  const Cache &out_ik = kSmemDesc ? s_caches[5] : p_out_ik;
   extern __shared__ __align__(16) uint8_t csm[];
   pdl_wait();
   pdl_trigger();
@@ -347,7 +385,9 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   const long long j = t_begin[b] / stride + blockIdx.x;
   // never write past a cache's capacity, whatever the device-side token counts say
   if (j >= t_end[b] / stride || j < 0 || j >= out_k.cap || (raw_v.data && j >= out_v.cap) ||
-      (raw_ik.data && j >= out_ik.cap)) {
+      (raw_ik.data && j >= out_ik.cap) ||
+      (kPaged && (!out_k.mapped(b, j) || (raw_v.data && !out_v.mapped(b, j)) ||
+                  (raw_ik.data && !out_ik.mapped(b, j))))) {
     cp_async_wait_all();
     return;
   }
@@ -356,9 +396,9 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   // slot rows of the window's positions, one modulo per position
   for (int r = tid; r < pool; r += blockDim.x) {
     const long long p = first + r;
-    rows[r] = p < 0 ? -1 : raw_k.row(b, raw_k.slot_of(p));
-    if (raw_v.data) rows_v[r] = p < 0 ? -1 : raw_v.row(b, raw_v.slot_of(p));
-    if (raw_ik.data) rows_i[r] = p < 0 ? -1 : raw_ik.row(b, raw_ik.slot_of(p));
+    rows[r] = p < 0 ? -1 : raw_k.row<kRowFlat>(b, raw_k.slot_of(p));
+    if (raw_v.data) rows_v[r] = p < 0 ? -1 : raw_v.row<kRowFlat>(b, raw_v.slot_of(p));
+    if (raw_ik.data) rows_i[r] = p < 0 ? -1 : raw_ik.row<kRowFlat>(b, raw_ik.slot_of(p));
   }
   __syncthreads();
   stage_window(raw_k, lk, rows, pool, bk);
@@ -398,9 +438,9 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   if (raw_ik.data) pool_staged(raw_ik, li, bi, first, pool, a, pi);
   __syncthreads();
   // re-quantisation and stores (no shared memory is written from here on)
-  store_entry(out_k, b, j, pk, D);
-  if (raw_v.data) store_entry(out_v, b, j, pv, Dv);
-  if (raw_ik.data) store_entry(out_ik, b, j, pi, Di);
+  store_entry<kPaged>(out_k, b, j, pk, D);
+  if (raw_v.data) store_entry<kPaged>(out_v, b, j, pv, Dv);
+  if (raw_ik.data) store_entry<kPaged>(out_ik, b, j, pi, Di);
 }
 
 
@@ -443,10 +483,12 @@ __device__ __noinline__ void pool_channels(const Cache &c, const SlotLayout &l, 
 
 __global__ void __launch_bounds__(kThreads, 1)
 compress_channel_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__ t_end,
-                        Cache raw_k, Cache raw_v, Cache raw_ik, const float *__restrict__ gate_w,
+                        Cache raw_k, Cache raw_v,
+                        Cache raw_ik, const float *__restrict__ gate_w,
                         const float *__restrict__ gate_b, const float *__restrict__ gate_w_ik,
-                        const float *__restrict__ gate_b_ik, int pool, int stride, Cache out_k,
-                        Cache out_v, Cache out_ik) {
+                        const float *__restrict__ gate_b_ik, int pool, int stride,
+                        Cache out_k, Cache out_v,
+                        Cache out_ik) {
   extern __shared__ __align__(16) uint8_t csm[];
   pdl_wait();
   pdl_trigger();
@@ -470,14 +512,15 @@ compress_channel_kernel(const int64_t *__restrict__ t_begin, const int64_t *__re
   const long long j = t_begin[b] / stride + blockIdx.x;
   // never write past a cache's capacity, whatever the device-side token counts say
   if (j >= t_end[b] / stride || j < 0 || j >= out_k.cap || (raw_v.data && j >= out_v.cap) ||
-      (raw_ik.data && j >= out_ik.cap))
+      (raw_ik.data && j >= out_ik.cap) || !out_k.mapped(b, j) ||
+      (raw_v.data && !out_v.mapped(b, j)) || (raw_ik.data && !out_ik.mapped(b, j)))
     return;
   const long long first = (long long)stride * (j + 1) - pool;
   for (int r = tid; r < pool; r += blockDim.x) {
     const long long p = first + r;
-    rows[r] = p < 0 ? -1 : raw_k.row(b, raw_k.slot_of(p));
-    if (raw_v.data) rows_v[r] = p < 0 ? -1 : raw_v.row(b, raw_v.slot_of(p));
-    if (raw_ik.data) rows_i[r] = p < 0 ? -1 : raw_ik.row(b, raw_ik.slot_of(p));
+    rows[r] = p < 0 ? -1 : raw_k.row<kRowFlat>(b, raw_k.slot_of(p));
+    if (raw_v.data) rows_v[r] = p < 0 ? -1 : raw_v.row<kRowFlat>(b, raw_v.slot_of(p));
+    if (raw_ik.data) rows_i[r] = p < 0 ? -1 : raw_ik.row<kRowFlat>(b, raw_ik.slot_of(p));
   }
   __syncthreads();
   stage_window(raw_k, lk, rows, pool, bk);
@@ -492,9 +535,9 @@ compress_channel_kernel(const int64_t *__restrict__ t_begin, const int64_t *__re
   if (raw_ik.data)
     pool_channels(raw_ik, li, bi, nullptr, li, bi, r0, pool, gate_w_ik, gate_b_ik, pi, nullptr);
   __syncthreads();
-  store_entry(out_k, b, j, pk, D);
-  if (raw_v.data) store_entry(out_v, b, j, pv, Dv);
-  if (raw_ik.data) store_entry(out_ik, b, j, pi, Di);
+  store_entry<true>(out_k, b, j, pk, D);
+  if (raw_v.data) store_entry<true>(out_v, b, j, pv, Dv);
+  if (raw_ik.data) store_entry<true>(out_ik, b, j, pi, Di);
 }
 
 }  // namespace
@@ -518,15 +561,22 @@ int launch_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t
       staged +
       sizeof(float) * (size_t)(2 * round16(Dk) + 2 * round16(pool) + round16(Dv) + round16(Di)) +
       3 * sizeof(long long) * (size_t)pool + 16;
-  if (smem_staged <= 200 * 1024 && ensure_dynamic_smem(compress_staged_kernel, smem_staged)) {
-    if (launch_pdl(compress_staged_kernel, grid, dim3(kThreads), smem_staged, st, t_begin, t_end,
-                   raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride, out_k, out_v,
+  const bool paged = out_k.bt || (raw_v.data && out_v.bt) || (raw_ik.data && out_ik.bt);
+  const bool smem_desc = pool >= 32;
+  auto staged_kernel = paged ? (smem_desc ? compress_staged_kernel<true, true>
+                                          : compress_staged_kernel<true, false>)
+                             : (smem_desc ? compress_staged_kernel<false, true>
+                                          : compress_staged_kernel<false, false>);
+  if (smem_staged <= 200 * 1024 && ensure_dynamic_smem(staged_kernel, smem_staged)) {
+    if (launch_pdl(staged_kernel, grid, dim3(kThreads), smem_staged, st, t_begin, t_end, raw_k,
+                   raw_v, raw_ik, gate_w, gate_b, pool, stride, out_k, out_v,
                    out_ik) != cudaSuccess)
       return CSKV_ERR_CUDA;
   } else {
     const size_t smem = sizeof(float) * (size_t)(pool + dmax);
-    if (launch_pdl(compress_kernel, grid, dim3(kThreads), smem, st, t_begin, t_end, raw_k, raw_v,
-                   raw_ik, gate_w, gate_b, pool, stride, out_k, out_v, out_ik) != cudaSuccess)
+    if (launch_pdl(paged ? compress_kernel<true> : compress_kernel<false>, grid, dim3(kThreads),
+                   smem, st, t_begin, t_end, raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride,
+                   out_k, out_v, out_ik) != cudaSuccess)
       return CSKV_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? CSKV_OK : CSKV_ERR_CUDA;

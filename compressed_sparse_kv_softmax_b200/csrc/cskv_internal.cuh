@@ -26,12 +26,23 @@ __device__ __forceinline__ float mxfp4_value(uint32_t code, uint8_t e) {
 }
 
 // Device-side view of a cskv_cache (passed to kernels by value).
+// How a kernel maps a slot to its plane row: kRowAuto looks at the cache
+// (block table or not), kRowFlat is the contiguous layout only (rings, and
+// the instantiations of the latency-bound kernels that leave paging out so
+// that their code stays as small as before).
+constexpr int kRowAuto = 0, kRowFlat = 1;
+
+// (kept at 72 bytes: kernels that hand a descriptor to an out-of-line
+// helper copy it per thread, and the cold-cache compressor felt every byte)
 struct Cache {
-  int fmt, d_nope, d_rope, ring;
+  int16_t fmt, d_nope, d_rope, ring;
+  int32_t bs_log2, nblk;      // paged layout: 2^bs_log2 slots per block, nblk blocks
   long long cap;
-  uint8_t *data; long long data_stride;
-  uint8_t *scale; long long scale_stride;   // bytes
-  uint8_t *rope; long long rope_stride;
+  uint8_t *data, *scale, *rope;
+  int32_t data_stride, scale_stride, rope_stride;   // bytes
+  // paged layout: bt [B][cap >> bs_log2] physical block ids (nullptr: rows
+  // b * cap + slot)
+  const int32_t *bt;
 
   __host__ __device__ int dims() const { return d_nope + d_rope; }
   // scales per slot, the dims each covers, and the bytes they take
@@ -49,44 +60,82 @@ struct Cache {
   __host__ __device__ int data_bytes() const {
     return fmt == CSKV_FMT_F32 ? 4 * dims() : (fmt == CSKV_FMT_MXFP4 ? d_nope >> 1 : d_nope);
   }
-  __host__ __device__ long long row(int b, long long slot) const {
-    return (long long)b * cap + slot;
+  // plane row of a slot (device: the block table lives in device memory)
+  template <int M = kRowAuto>
+  __device__ long long row(int b, long long slot) const {
+    if (M == kRowFlat || !bt) return (long long)b * cap + slot;
+    long long blk = bt[(long long)b * (cap >> bs_log2) + (slot >> bs_log2)];
+    blk = blk < 0 ? 0 : (blk >= nblk ? nblk - 1 : blk);   // (a bad table stays in bounds)
+    return (blk << bs_log2) + (slot & ((1LL << bs_log2) - 1));
+  }
+  // whether slot s of sequence b has a block (always, unpaged)
+  __device__ bool mapped(int b, long long slot) const {
+    if (!bt) return true;
+    const long long blk = bt[(long long)b * (cap >> bs_log2) + (slot >> bs_log2)];
+    return blk >= 0 && blk < nblk;
+  }
+  // plane row of slot j0 of sequence b, the first of a run of slots that
+  // stays inside one block (paged: j0's block names a block of the planes);
+  // `invalid` when the block table names none (a slot past the sequence's
+  // allocation)
+  __device__ long long run_row0(int b, long long j0, long long invalid) const {
+    if (!bt) return (long long)b * cap + j0;
+    const long long blk = bt[(long long)b * (cap >> bs_log2) + (j0 >> bs_log2)];
+    if (blk < 0 || blk >= nblk) return invalid;
+    return (blk << bs_log2) + (j0 & ((1LL << bs_log2) - 1));
+  }
+  // rows the planes hold (B sequences of cap slots, or the block pool)
+  __host__ __device__ long long plane_rows(int B) const {
+    return bt ? ((long long)nblk << bs_log2) : (long long)B * cap;
   }
   // slot holding token position p (ring) or entry j (compressed cache)
   __host__ __device__ long long slot_of(long long p) const { return ring ? (p % cap) : p; }
+  template <int M = kRowAuto>
   __device__ const uint8_t *data_ptr(int b, long long slot) const {
-    return data + row(b, slot) * data_stride;
+    return data + row<M>(b, slot) * data_stride;
   }
+  template <int M = kRowAuto>
   __device__ const float *scale_ptr(int b, long long slot) const {
-    return reinterpret_cast<const float *>(scale + row(b, slot) * scale_stride);
+    return reinterpret_cast<const float *>(scale + row<M>(b, slot) * scale_stride);
   }
+  template <int M = kRowAuto>
   __device__ const __nv_bfloat16 *rope_ptr(int b, long long slot) const {
-    return reinterpret_cast<const __nv_bfloat16 *>(rope + row(b, slot) * rope_stride);
+    return reinterpret_cast<const __nv_bfloat16 *>(rope + row<M>(b, slot) * rope_stride);
   }
   // dequantised value of dim d of a slot (scalar path)
+  template <int M = kRowAuto>
   __device__ float value(int b, long long slot, int d) const {
-    if (fmt == CSKV_FMT_F32)
-      return reinterpret_cast<const float *>(data_ptr(b, slot))[d];
+    const long long r = row<M>(b, slot);
+    const uint8_t *dp = data + r * data_stride;
+    if (fmt == CSKV_FMT_F32) return reinterpret_cast<const float *>(dp)[d];
     if (fmt == CSKV_FMT_MXFP4)
-      return mxfp4_value(data_ptr(b, slot)[d >> 1] >> ((d & 1) << 2),
-                         (scale + row(b, slot) * scale_stride)[d >> 5]);
+      return mxfp4_value(dp[d >> 1] >> ((d & 1) << 2), (scale + r * scale_stride)[d >> 5]);
     if (d < d_nope) {
       __nv_fp8_e4m3 c;
-      c.__x = data_ptr(b, slot)[d];
-      return float(c) * scale_ptr(b, slot)[fmt == CSKV_FMT_E4M3_VEC ? 0 : d >> 6];
+      c.__x = dp[d];
+      return float(c) *
+             reinterpret_cast<const float *>(scale + r * scale_stride)[fmt == CSKV_FMT_E4M3_VEC ? 0 : d >> 6];
     }
-    return __bfloat162float(rope_ptr(b, slot)[d - d_nope]);
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(rope + r * rope_stride)[d - d_nope]);
   }
 };
 
+static_assert(sizeof(Cache) == 72, "cache descriptor size");
+
+// (field ranges are checked by the ABI: dims < 2^15, strides and blocks < 2^31)
 inline Cache to_dev(const cskv_cache *c) {
   Cache v{};
   if (!c) return v;
-  v.fmt = c->fmt; v.d_nope = c->d_nope; v.d_rope = c->d_rope; v.ring = c->ring;
+  v.fmt = (int16_t)c->fmt; v.d_nope = (int16_t)c->d_nope; v.d_rope = (int16_t)c->d_rope;
+  v.ring = (int16_t)c->ring;
   v.cap = c->cap;
-  v.data = (uint8_t *)c->data; v.data_stride = c->data_stride;
-  v.scale = (uint8_t *)c->scale; v.scale_stride = c->scale_stride;
-  v.rope = (uint8_t *)c->rope; v.rope_stride = c->rope_stride;
+  v.data = (uint8_t *)c->data; v.data_stride = (int32_t)c->data_stride;
+  v.scale = (uint8_t *)c->scale; v.scale_stride = (int32_t)c->scale_stride;
+  v.rope = (uint8_t *)c->rope; v.rope_stride = (int32_t)c->rope_stride;
+  v.bt = c->block_table;
+  v.bs_log2 = 0;
+  while (c->block_table && (1LL << v.bs_log2) < c->block_size) ++v.bs_log2;
+  v.nblk = c->block_table ? (int32_t)c->num_blocks : 0;
   return v;
 }
 

@@ -155,13 +155,15 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
 
   if (warp == 0) {
     // ---------------- TMA producer
-    const long long total_rows = (long long)a.B * a.ik.cap;
+    const long long total_rows = a.ik.plane_rows(a.B);
     if (elect_one()) {
       auto issue = [&](int i) {
         if (drop_first && i == 0) return;
         const int s = i % kStages;
         const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
-        const long long g0 = (long long)b * a.ik.cap + j0;
+        // (paged: inside one block; a tile with no block reads past the
+        // planes, i.e. zeros, and is never used)
+        const long long g0 = a.ik.run_row0(b, j0, total_rows);
         long long rows = total_rows - g0;
         rows = rows < kTile ? rows : kTile;
         const ScaleSpan sp = packed ? scale_span(g0, rows, 4) : ScaleSpan{0, 0, 0};
@@ -230,7 +232,7 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
     // entries r, 32 + r, 64 + r, 96 + r of each tile (those the bulk copy did
     // not bring come from global memory) into row r of the tile's chunk
     const int my_tiles = tiles_of(visible_n());
-    const long long total_rows = (long long)a.B * a.ik.cap;
+    const long long total_rows = a.ik.plane_rows(a.B);
     const uint8_t *exp_base = reinterpret_cast<const uint8_t *>(a.ik.scale);
     for (int i = 0; i < my_tiles; ++i) {
       // (the stop flag is read once per warp: the loop stays warp-uniform)
@@ -240,7 +242,8 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
         if (lane == 0) record_abort(sm);
         break;
       }
-      const long long g0 = (long long)b * a.ik.cap + (long long)(blockIdx.x + i * gridDim.x) * kTile;
+      const long long g0 =
+          a.ik.run_row0(b, (long long)(blockIdx.x + i * gridDim.x) * kTile, total_rows);
       const long long tile_rows = total_rows - g0;
       const ScaleSpan sp =
           packed ? scale_span(g0, tile_rows < kTile ? tile_rows : kTile, 4) : ScaleSpan{0, 0, 0};
@@ -343,7 +346,8 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
 
 bool indexer_mxf4_supported(const IndexerArgs &a) {
   if (a.ik.fmt != CSKV_FMT_MXFP4 || a.d_I != 2 * kRowBytes || a.H_I != kHeads) return false;
-  if ((long long)a.B * a.ik.cap >= (1LL << 31)) return false;
+  if (a.ik.plane_rows(a.B) >= (1LL << 31)) return false;
+  if (a.ik.bt && a.ik.bs_log2 < 7) return false;     // paged: a key tile within one block
   if (((uintptr_t)a.ik.data & 15) || (a.ik.data_stride & 15)) return false;
   if ((uintptr_t)a.q_ik_scale & 3) return false;
   int dev = 0, major = 0;
@@ -356,10 +360,11 @@ int launch_indexer_mxf4(const IndexerArgs &a, float *scores, long long ld, uint3
                         uint32_t *ctr, cudaStream_t st) {
   auto fn = tensor_map_encode_fn();
   if (!fn) return CSKV_ERR_UNSUPPORTED;
-  // all sequences' packed key rows as one [B * cap] x 64-byte matrix;
-  // 128 x 64 B boxes in the 64-byte swizzle the MMA descriptors expect
+  // all packed key rows as one [B * cap] (paged: [blocks * block size]) x
+  // 64-byte matrix; 128 x 64 B boxes in the 64-byte swizzle the MMA
+  // descriptors expect
   CUtensorMap map;
-  cuuint64_t dims[2] = {(cuuint64_t)kRowBytes, (cuuint64_t)((long long)a.B * a.ik.cap)};
+  cuuint64_t dims[2] = {(cuuint64_t)kRowBytes, (cuuint64_t)a.ik.plane_rows(a.B)};
   cuuint64_t strides[1] = {(cuuint64_t)a.ik.data_stride};
   cuuint32_t box[2] = {(cuuint32_t)kRowBytes, (cuuint32_t)kTile};
   cuuint32_t estr[2] = {1, 1};

@@ -177,13 +177,15 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
 
   if (warp == 0) {
     // ---------------- TMA producer
-    const long long total_rows = (long long)a.B * a.ik.cap;
+    const long long total_rows = a.ik.plane_rows(a.B);
     if (elect_one()) {
       auto issue = [&](int i) {
         if (drop_first && i == 0) return;
         const int s = i % kStages;
         const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
-        const long long g0 = (long long)b * a.ik.cap + j0;    // first row of the tile
+        // first row of the tile (paged: inside one block; a tile with no
+        // block reads past the planes, i.e. zeros, and is never used)
+        const long long g0 = a.ik.run_row0(b, j0, total_rows);
         // scales of the rows that exist (the key TMA zero-fills past the end;
         // a bulk copy must not read past it), when the plane is packed
         long long rows = total_rows - g0;
@@ -260,7 +262,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
     const int r = quad * 32 + lane;           // entry within the tile
     float *srow = scores + (size_t)row * ld;
     const uint8_t *scale_base = reinterpret_cast<const uint8_t *>(a.ik.scale);
-    const long long total_rows = (long long)a.B * a.ik.cap;
+    const long long total_rows = a.ik.plane_rows(a.B);
     for (int i = grp; i < my_tiles; i += kEpiGroups) {
       const int acc = i % kAcc;
       const int s = i % kStages;
@@ -277,8 +279,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       mbar_wait(&sm.full[s], (i / kStages) & 1, lim);
       float sk0 = 1.f, sk1 = 0.f;            // (rows past n: score not stored)
       if (j < n) {
-        const long long g = (long long)b * a.ik.cap + j;
-        const long long g0 = g - r, tile_rows = total_rows - g0;   // rows from the tile's first
+        const long long g0 = a.ik.run_row0(b, j - r, 0), g = g0 + r;
+        const long long tile_rows = total_rows - g0;   // rows from the tile's first
         // entries whose scales the stage's bulk copy brought; the rest come
         // by plain loads
         const ScaleSpan sp =
@@ -467,7 +469,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encode_fn() {
 bool indexer_tc_supported(const IndexerArgs &a) {
   const bool vec = a.ik.fmt == CSKV_FMT_E4M3_VEC;
   if ((a.ik.fmt != CSKV_FMT_E4M3_BF16 && !vec) || a.d_I != kDim || a.H_I != kHeads) return false;
-  if ((long long)a.B * a.ik.cap >= (1LL << 31)) return false;
+  if (a.ik.plane_rows(a.B) >= (1LL << 31)) return false;
+  if (a.ik.bt && a.ik.bs_log2 < 7) return false;     // paged: a key tile within one block
   if (((uintptr_t)a.ik.data & 15) || (a.ik.data_stride & 15)) return false;
   // (scales in any stride and alignment: packed planes arrive by bulk copy,
   // others by plain loads; q_ik is 16-byte aligned by the ABI's checks)
@@ -480,9 +483,10 @@ bool indexer_tc_supported(const IndexerArgs &a) {
 bool make_key_tmap(const IndexerArgs &a, CUtensorMap *map) {
   auto fn = tensor_map_encode_fn();
   if (!fn) return false;
-  // all sequences' key rows as one [B * cap] x 128-byte matrix; 128 x 128 B
-  // boxes in the 128-byte swizzle the K-major operand descriptors expect
-  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)((long long)a.B * a.ik.cap)};
+  // all key rows as one [B * cap] (paged: [blocks * block size]) x 128-byte
+  // matrix; 128 x 128 B boxes in the 128-byte swizzle the K-major operand
+  // descriptors expect
+  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)a.ik.plane_rows(a.B)};
   cuuint64_t strides[1] = {(cuuint64_t)a.ik.data_stride};
   cuuint32_t box[2] = {(cuuint32_t)kDim, (cuuint32_t)kTile};
   cuuint32_t estr[2] = {1, 1};

@@ -219,12 +219,14 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
     // ---------------- TMA producer
     if (elect_one()) {
       const uint64_t keep = policy_evict_last();
-      const long long total_rows = (long long)a.B * a.ik.cap;
+      const long long total_rows = a.ik.plane_rows(a.B);
       auto issue = [&](int i) {
         if (drop_first && i == 0) return;
         const int s = i % kStages;
         const long long j0 = ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile;
-        const long long g0 = (long long)b * a.ik.cap + j0;     // first cache row of the tile
+        // first cache row of the tile (paged: inside one block; a tile with no
+        // block reads past the planes, i.e. zeros, and is never used)
+        const long long g0 = a.ik.run_row0(b, j0, total_rows);
         // scales of the rows that exist (the key TMA zero-fills past the end;
         // a bulk copy must not read past it), when the plane is packed
         long long rows = total_rows - g0;
@@ -305,8 +307,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
     nr[0] = (int)sm.n[eg];
     nr[1] = (int)sm.n[kHalfRows + eg];
     const int my_tiles = tiles_of(nmax);
-    const long long total_rows = (long long)a.B * a.ik.cap;
-    const int gb = b * (int)a.ik.cap;
+    const long long total_rows = a.ik.plane_rows(a.B);
     const uint8_t *scale_base = reinterpret_cast<const uint8_t *>(a.ik.scale);
     float *srow0 = scores + (row0 + eg) * ld;
     float *srow1 = scores + (row0 + kHalfRows + eg) * ld;
@@ -325,14 +326,14 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       float sk = 1.f;
       if (j < nmax) {
         // the scales the stage's bulk copy brought, else a plain load
-        const long long g0 = (long long)gb + jt, tile_rows = total_rows - g0;
+        const long long g0 = a.ik.run_row0(b, jt, 0), tile_rows = total_rows - g0;
         const ScaleSpan sp =
             packed ? scale_span(g0, tile_rows < kTile ? tile_rows : kTile, 4) : ScaleSpan{0, 0, 0};
         const uint32_t off = sp.lead + 4u * (uint32_t)r;
         sk = off + 4 <= sp.bytes
                  ? *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(sm.kscale[s]) + off)
                  : __ldg(reinterpret_cast<const float *>(scale_base +
-                                                         ((long long)gb + j) * a.ik.scale_stride));
+                                                         (g0 + r) * a.ik.scale_stride));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);

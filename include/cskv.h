@@ -109,6 +109,18 @@ enum {
  * with d_rope = 0; E4M3_VEC and MXFP4 are the ones the tensor-core scoring
  * path reads fastest (one accumulator per key and head), MXFP4 with half the
  * bytes.
+ * Paged layout (block tables; no counterpart on the pages, a serving-side
+ * storage choice): with block_table != NULL the planes hold num_blocks
+ * blocks of block_size slots shared by all sequences, and slot s of sequence
+ * b lives in physical row
+ *     block_table[b * (cap / block_size) + s / block_size] * block_size
+ *         + s % block_size
+ * of every plane (row r starting at plane + r * plane_stride).  Only for
+ * compressed caches (ring = 0); block_size a power of two dividing cap;
+ * every table entry in [0, num_blocks).  A paged indexer-key cache keeps
+ * the tensor-core scoring path when block_size is a multiple of 128 (each
+ * 128-entry key tile then lies in one block), else the CUDA-core one; the
+ * attention bulk-copies runs of consecutive entries when block_size >= 64.
  * Alignment: data and rope pointers and strides are multiples of 16 bytes;
  * scale pointer 16-byte aligned, scale stride a multiple of 4 bytes and at
  * least 4 * ceil(d_nope / 64) (E4M3_BF16), 4 (E4M3_VEC) or d_nope / 32
@@ -123,6 +135,10 @@ typedef struct cskv_cache {
   void *data;   int64_t data_stride;
   float *scale; int64_t scale_stride;
   void *rope;   int64_t rope_stride;
+  /* Paged layout (compressed caches only; block_table NULL: contiguous) */
+  const int32_t *block_table;  /* device [B][cap / block_size] physical block ids */
+  int64_t block_size;          /* slots per block: a power of two */
+  int64_t num_blocks;          /* blocks the planes hold */
 } cskv_cache;
 
 /*

@@ -25,11 +25,28 @@ def _np(t):
 
 
 def as_numpy_cache(c):
+    """A cache as numpy planes [B][cap][...]; a paged cache (block table) is
+    read back into that form: slot s of sequence b is pool row
+    table[b][s // block_size] * block_size + s % block_size (slots of a
+    logical block without a pool block read as NaN)."""
     if c is None:
         return None
     out = {k: c[k] for k in ("fmt", "d_nope", "d_rope", "ring", "cap")}
     for k in ("data", "scale", "rope"):
         out[k] = _np(c.get(k))
+    if c.get("block_table") is not None:
+        bt = _np(c["block_table"]).astype(np.int64)
+        bs = int(c["block_size"])
+        B, nb = bt.shape
+        rows = (np.maximum(bt, 0)[:, :, None] * bs + np.arange(bs)[None, None, :]).reshape(B, -1)
+        hole = np.repeat(bt < 0, bs, axis=1)
+        for k in ("data", "scale", "rope"):
+            if out[k] is None:
+                continue
+            v = out[k][0][rows]
+            if k == "scale" and np.issubdtype(v.dtype, np.floating):
+                v = np.where(hole[:, :, None], np.nan, v)
+            out[k] = v
     return out
 
 

@@ -150,6 +150,30 @@ def test_argument_errors_are_caught_on_the_host(C):
     ik_vec.data_stride, ik_vec.scale_stride = 128, 0
     assert lib.indexer_topk(*args, R(ik_vec), 4, 1024, 262144, out, None, ws, big,
                             None) == ERR_ARG
+    # paged caches: a paged ring, a block size that is not a power of two or
+    # does not divide cap, no blocks; the per-channel compressor's value ring
+    # with other channels than the key's, its indexer ring without gates
+    paged_ring = _fake_cache(1, cap=16)
+    paged_ring.block_table, paged_ring.block_size, paged_ring.num_blocks = 1 << 36, 16, 4
+    assert lib.csa_compress(1, ctx, ctx, 1, R(paged_ring), None, None, gate, gate, 8, 4, R(comp),
+                            None, None, None) == ERR_ARG
+    for bs, nblk in ((48, 512), (16384, 1), (64, 0)):
+        pc = _fake_cache(0, cap=8192)
+        pc.block_table, pc.block_size, pc.num_blocks = 1 << 36, bs, nblk
+        assert lib.hybrid_attn_decode(1, ctx, q, 64, 0.04, R(pc), None, 128, None, 0, 8192,
+                                      R(ring), None, 128, out, lse, ws, big, None) == ERR_ARG
+    v128 = _fake_cache(1, cap=16, fmt=C.FMT_E4M3_BF16, d_nope=64, d_rope=64)
+    v128_out = _fake_cache(0, cap=8192, fmt=C.FMT_E4M3_BF16, d_nope=64, d_rope=64)
+    assert lib.csa_compress_channel_gate(1, ctx, ctx, 1, R(small_ring), R(v128), None, gate, gate,
+                                         None, None, 8, 4, R(comp), R(v128_out), None,
+                                         None) == ERR_ARG
+    ik_ring = _fake_cache(1, cap=16, fmt=C.FMT_E4M3_VEC, d_nope=128, d_rope=0)
+    ik_out = _fake_cache(0, cap=8192, fmt=C.FMT_E4M3_VEC, d_nope=128, d_rope=0)
+    ik_ring.data_stride = ik_out.data_stride = 128
+    ik_ring.scale_stride = ik_out.scale_stride = 4
+    assert lib.csa_compress_channel_gate(1, ctx, ctx, 1, R(small_ring), None, R(ik_ring), gate,
+                                         gate, None, None, 8, 4, R(comp), None, R(ik_out),
+                                         None) == ERR_ARG
     # zero-sized work is a no-op success without touching the device
     assert lib.csa_compress(1, ctx, ctx, 0, R(ring), None, None, gate, gate, 8, 4, R(comp),
                             None, None, None) == 0

@@ -5,7 +5,8 @@ the method's arithmetic (no pooling, scoring, selection or attention).  Both
 the CUDA path's tests/bench and the CPU oracle consume what it produces.
 """
 from .configs import Workload, WORKLOADS, get
-from .generate import make_csa_layer, make_hca_layer, e4m3_from_float, random_selection
+from .generate import (make_csa_layer, make_hca_layer, e4m3_from_float, random_selection,
+                       page_cache)
 
 __all__ = ["Workload", "WORKLOADS", "get",
-           "make_csa_layer", "make_hca_layer", "e4m3_from_float", "random_selection"]
+           "make_csa_layer", "make_hca_layer", "e4m3_from_float", "random_selection", "page_cache"]

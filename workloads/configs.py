@@ -45,6 +45,8 @@ class Workload:
     q_prescale: bool = False       # tiny workload: Q already multiplied by 1/sqrt(head dim)
     gate_mode: str = "scalar"      # "scalar": g_r = w . k + b[r]; "channel": one gate per
                                    # channel, g_{r,c} = w_c k_c + b[r][c]
+    page_block: int = 0            # > 0: compressed caches paged in blocks of this many
+                                   # entries (shuffled pool + block table)
     seed: int = 0
 
     @property

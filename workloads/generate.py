@@ -237,6 +237,10 @@ def make_csa_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
                 nbq = L["q_ik_scale"].shape[-1]
                 L["comp_ik"]["scale"][b, j, :nbq] = L["q_ik_scale"][b, 0, hstar, :nbq] * 4.0
             _plant_kv_needle(L["comp_k"], b, j, L["q"][b, 0, 0], rng)
+    if wl.page_block:
+        for i, key in enumerate(("comp_k", "comp_v", "comp_ik")):
+            if L.get(key) is not None:
+                L[key] = page_cache(L[key], wl.page_block, seed=wl.seed * 31 + i)
     return L
 
 
@@ -269,6 +273,10 @@ def make_hca_layer(wl: Workload, device="cpu", seed: int | None = None, ring_cap
             j = p // wl.hca_stride
             if j < n_h:
                 _plant_kv_needle(L["comp_k"], b, j, L["q"][b, 0, 0], rng)
+    if wl.page_block:
+        for i, key in enumerate(("comp_k", "comp_v")):
+            if L.get(key) is not None:
+                L[key] = page_cache(L[key], wl.page_block, seed=wl.seed * 31 + 7 + i)
     return L
 
 
@@ -306,3 +314,41 @@ def random_selection(wl: Workload, k: int, seed: int = 17, device="cpu"):
                 out[b, t] = pick.to(torch.int32)
     return out.to(device)
 
+
+def page_cache(c: dict, block_size: int, seed: int = 0, spare_blocks: int = 3,
+               unmapped_tail: int = 0) -> dict:
+    """Paged copy of a compressed cache (ring = 0): every sequence's slots cut
+    into blocks of `block_size`, the blocks placed in a shared pool in a
+    seeded random order (with `spare_blocks` unused blocks), and the block
+    table [B][cap / block_size] int32 that maps logical block (b, i) to its
+    pool block.  The capacity is rounded up to whole blocks (the new slots
+    hold zeros), and `unmapped_tail` further logical blocks per sequence get
+    no pool block (table entry -1), as in a pool that allocates on demand.
+    Storage only: every logical slot keeps its bytes."""
+    assert not c["ring"] and block_size >= 1 and block_size & (block_size - 1) == 0
+    data = c["data"]
+    B, cap = data.shape[0], int(c["cap"])
+    nb = (cap + block_size - 1) // block_size
+    n = B * nb + spare_blocks
+    g = torch.Generator().manual_seed(seed)
+    phys = torch.randperm(n, generator=g)[: B * nb]        # pool block of each logical block
+    out = dict(c)
+    for key in ("data", "scale", "rope"):
+        t = c.get(key)
+        if t is None:
+            continue
+        tail = tuple(t.shape[2:])
+        padded = torch.zeros((B, nb * block_size) + tail, dtype=t.dtype, device=t.device)
+        padded[:, :cap] = t
+        pool = torch.zeros((1, n * block_size) + tail, dtype=t.dtype, device=t.device)
+        pool.view((n, block_size) + tail)[phys.to(t.device)] = \
+            padded.reshape((B * nb, block_size) + tail)
+        out[key] = pool
+    table = phys.view(B, nb).to(torch.int32)
+    if unmapped_tail:
+        table = torch.cat([table, torch.full((B, unmapped_tail), -1, dtype=torch.int32)], 1)
+    out["cap"] = (nb + unmapped_tail) * block_size
+    out["block_table"] = table.to(data.device)
+    out["block_size"] = block_size
+    out["num_blocks"] = n
+    return out
