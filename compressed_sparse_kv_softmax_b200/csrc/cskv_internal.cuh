@@ -26,6 +26,11 @@ __device__ __forceinline__ float mxfp4_value(uint32_t code, uint8_t e) {
 }
 
 // Device-side view of a cskv_cache (passed to kernels by value).
+// Tiles of a paged key cache whose first rows a scoring CTA resolves up front
+// (the producer warp's lanes together, into shared memory), so that no tile
+// waits on its block-table load; later tiles read the table when they come.
+constexpr int kPagedTiles = 64;
+
 // How a kernel maps a slot to its plane row: kRowAuto looks at the cache
 // (block table or not), kRowFlat is the contiguous layout only (rings, and
 // the instantiations of the latency-bound kernels that leave paging out so

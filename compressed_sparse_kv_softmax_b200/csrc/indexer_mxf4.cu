@@ -69,6 +69,7 @@ struct __align__(1024) Smem {
   uint32_t kexp[kStages][kTile];          // the tiles' exponent words as copied
   float w[kHeads];
   uint32_t hist[kTopkBins];
+  long long tile_row[kPagedTiles];        // paged keys: first plane row of this CTA's tiles
   uint64_t full[kStages], empty[kStages], sf_ready[kStages], acc_full[kAcc], acc_empty[kAcc],
       mma_done;
   uint32_t tmem_base;
@@ -153,17 +154,29 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
     asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");   // all warps but the producer
   }
 
+  // first plane row of tile i of this CTA (paged keys: inside one block; a
+  // tile with no block is placed past the planes, i.e. reads zeros, unused)
+  auto tile_row0 = [&](int i) -> long long {
+    const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
+    if (!a.ik.bt) return (long long)b * a.ik.cap + j0;
+    return i < kPagedTiles ? sm.tile_row[i] : a.ik.run_row0(b, j0, a.ik.plane_rows(a.B));
+  };
   if (warp == 0) {
     // ---------------- TMA producer
     const long long total_rows = a.ik.plane_rows(a.B);
+    if (a.ik.bt) {
+      // (read by the other roles after the tiles' barriers)
+      const int nt = min(kPagedTiles, tiles_of(a.max_entries));
+      for (int i = lane; i < nt; i += 32)
+        sm.tile_row[i] = a.ik.run_row0(b, (long long)(blockIdx.x + i * gridDim.x) * kTile,
+                                       total_rows);
+      __syncwarp();
+    }
     if (elect_one()) {
       auto issue = [&](int i) {
         if (drop_first && i == 0) return;
         const int s = i % kStages;
-        const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
-        // (paged: inside one block; a tile with no block reads past the
-        // planes, i.e. zeros, and is never used)
-        const long long g0 = a.ik.run_row0(b, j0, total_rows);
+        const long long g0 = tile_row0(i);
         long long rows = total_rows - g0;
         rows = rows < kTile ? rows : kTile;
         const ScaleSpan sp = packed ? scale_span(g0, rows, 4) : ScaleSpan{0, 0, 0};
@@ -242,8 +255,7 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
         if (lane == 0) record_abort(sm);
         break;
       }
-      const long long g0 =
-          a.ik.run_row0(b, (long long)(blockIdx.x + i * gridDim.x) * kTile, total_rows);
+      const long long g0 = tile_row0(i);
       const long long tile_rows = total_rows - g0;
       const ScaleSpan sp =
           packed ? scale_span(g0, tile_rows < kTile ? tile_rows : kTile, 4) : ScaleSpan{0, 0, 0};

@@ -75,6 +75,7 @@ struct __align__(1024) Smem {
   // per-vector layout: query scale, scale x weight, weight
   float c0[kHeads], c1[kHeads], w[kHeads];
   uint32_t hist[kTopkBins];
+  long long tile_row[kPagedTiles];        // paged keys: first plane row of this CTA's tiles
   uint64_t full[kStages], empty[kStages], acc_full[kMaxAcc], acc_empty[kMaxAcc], mma_done;
   uint32_t tmem_base;
   int abort, qscale_pos;
@@ -175,17 +176,29 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
     asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");   // all warps but the producer
   }
 
+  // first plane row of tile i of this CTA (paged keys: inside one block; a
+  // tile with no block is placed past the planes, i.e. reads zeros, unused)
+  auto tile_row0 = [&](int i) -> long long {
+    const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
+    if (!a.ik.bt) return (long long)b * a.ik.cap + j0;
+    return i < kPagedTiles ? sm.tile_row[i] : a.ik.run_row0(b, j0, a.ik.plane_rows(a.B));
+  };
   if (warp == 0) {
     // ---------------- TMA producer
     const long long total_rows = a.ik.plane_rows(a.B);
+    if (a.ik.bt) {
+      // (read by the other roles after the tiles' barriers)
+      const int nt = min(kPagedTiles, tiles_of(a.max_entries));
+      for (int i = lane; i < nt; i += 32)
+        sm.tile_row[i] = a.ik.run_row0(b, (long long)(blockIdx.x + i * gridDim.x) * kTile,
+                                       total_rows);
+      __syncwarp();
+    }
     if (elect_one()) {
       auto issue = [&](int i) {
         if (drop_first && i == 0) return;
         const int s = i % kStages;
-        const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
-        // first row of the tile (paged: inside one block; a tile with no
-        // block reads past the planes, i.e. zeros, and is never used)
-        const long long g0 = a.ik.run_row0(b, j0, total_rows);
+        const long long g0 = tile_row0(i);       // first row of the tile
         // scales of the rows that exist (the key TMA zero-fills past the end;
         // a bulk copy must not read past it), when the plane is packed
         long long rows = total_rows - g0;
@@ -279,7 +292,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       mbar_wait(&sm.full[s], (i / kStages) & 1, lim);
       float sk0 = 1.f, sk1 = 0.f;            // (rows past n: score not stored)
       if (j < n) {
-        const long long g0 = a.ik.run_row0(b, j - r, 0), g = g0 + r;
+        const long long g0 = tile_row0(i), g = g0 + r;
         const long long tile_rows = total_rows - g0;   // rows from the tile's first
         // entries whose scales the stage's bulk copy brought; the rest come
         // by plain loads

@@ -78,6 +78,7 @@ struct __align__(1024) RowsSmem {
   float c0[kRows][kHeads], c1[kRows][kHeads], w[kRows][kHeads];
   uint32_t hist[kRows][kHistWords];
   long long n[kRows];                          // visible entries per row (0: no row)
+  long long tile_row[kPagedTiles];        // paged keys: first plane row of this CTA's tiles
   uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], mma_done;
   uint32_t tmem_base;
   int abort;
@@ -215,18 +216,30 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
     asm volatile("bar.sync 1, %0;" ::"r"(nt) : "memory");   // all warps but the producer
   }
 
+  // first plane row of tile i of this CTA (paged keys: inside one block; a
+  // tile with no block is placed past the planes, i.e. reads zeros, unused)
+  auto tile_row0 = [&](int i) -> long long {
+    const long long j0 = ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile;
+    if (!a.ik.bt) return (long long)b * a.ik.cap + j0;
+    return i < kPagedTiles ? sm.tile_row[i] : a.ik.run_row0(b, j0, a.ik.plane_rows(a.B));
+  };
   if (warp == 0) {
     // ---------------- TMA producer
+    if (a.ik.bt) {
+      // (read by the other roles after the tiles' barriers)
+      const int nt = min(kPagedTiles, tiles_of(a.max_entries));
+      for (int i = lane; i < nt; i += 32)
+        sm.tile_row[i] = a.ik.run_row0(
+            b, ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile, a.ik.plane_rows(a.B));
+      __syncwarp();
+    }
     if (elect_one()) {
       const uint64_t keep = policy_evict_last();
       const long long total_rows = a.ik.plane_rows(a.B);
       auto issue = [&](int i) {
         if (drop_first && i == 0) return;
         const int s = i % kStages;
-        const long long j0 = ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile;
-        // first cache row of the tile (paged: inside one block; a tile with no
-        // block reads past the planes, i.e. zeros, and is never used)
-        const long long g0 = a.ik.run_row0(b, j0, total_rows);
+        const long long g0 = tile_row0(i);       // first cache row of the tile
         // scales of the rows that exist (the key TMA zero-fills past the end;
         // a bulk copy must not read past it), when the plane is packed
         long long rows = total_rows - g0;
@@ -326,7 +339,7 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       float sk = 1.f;
       if (j < nmax) {
         // the scales the stage's bulk copy brought, else a plain load
-        const long long g0 = a.ik.run_row0(b, jt, 0), tile_rows = total_rows - g0;
+        const long long g0 = tile_row0(i), tile_rows = total_rows - g0;
         const ScaleSpan sp =
             packed ? scale_span(g0, tile_rows < kTile ? tile_rows : kTile, 4) : ScaleSpan{0, 0, 0};
         const uint32_t off = sp.lead + 4u * (uint32_t)r;
