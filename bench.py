@@ -662,15 +662,20 @@ def run_e2e(args, replicas, wl, dev, world):
     pos = (q_pos, ctx, tb, te)
     R = len(replicas)
 
+    stores = []
+
     def one(i):
         s = i % PERIOD
         rep = replicas[i % R]
         dev_buf.copy_(host_small[s], non_blocking=True)
-        C.ring_store(wl.B, tb, src, rings[i % R])
+        stores[i % R]()
         rep.step(s, pos=pos, split_select=False)
         host_out.copy_(out_buf, non_blocking=True)
 
     with torch.cuda.stream(stream):
+        # (the layers and the ring append marshal their arguments once per
+        # set of buffers; a step then costs the host the launches)
+        stores.extend(C.prepare("cskv_ring_store", wl.B, tb, src, r) for r in rings)
         for i in range(3):
             one(i)
     stream.synchronize()
@@ -688,7 +693,8 @@ def run_e2e(args, replicas, wl, dev, world):
     return {"value": round(whole_job_rate(wl.B * K, ms, world), 2), "unit": UNIT,
             "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "steps": K,
             "path": f"eager public API calls on one stream (cskv_ring_store, csa_compress, "
-                    f"indexer_topk, hybrid_attn_decode, hca_compress, hybrid_attn_decode), "
+                    f"indexer_topk, hybrid_attn_decode, hca_compress, hybrid_attn_decode; "
+                    f"arguments marshalled once per buffer set), "
                     f"{R} rotating replicas as in the timed region; per step one pinned "
                     f"host->device copy of all inputs and one device->host copy of both "
                     f"layers' outputs"}

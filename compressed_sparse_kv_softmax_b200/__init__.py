@@ -147,15 +147,19 @@ def _stream(stream):
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def ring_store(B, pos, src, ring, stream=None):
-    """Copies each sequence's new token (slot 0 of every cache in `src`) into
-    slot pos[b] % cap of the matching raw ring in `ring` (lists of caches)."""
+def _ring_store_args(B, pos, src, ring, stream=None):
     ss = [cache_struct(c) for c in src]
     rs = [cache_struct(c) for c in ring]
     n = len(ss)
     sp = (_PC * n)(*[ctypes.pointer(c) for c in ss])
     rp = (_PC * n)(*[ctypes.pointer(c) for c in rs])
-    _check(_lib.cskv_ring_store(B, _ptr(pos), n, sp, rp, _stream(stream)), "cskv_ring_store")
+    return (B, _ptr(pos), n, sp, rp, _stream(stream))
+
+
+def ring_store(B, pos, src, ring, stream=None):
+    """Copies each sequence's new token (slot 0 of every cache in `src`) into
+    slot pos[b] % cap of the matching raw ring in `ring` (lists of caches)."""
+    _check(_lib.cskv_ring_store(*_ring_store_args(B, pos, src, ring, stream)), "cskv_ring_store")
 
 
 def indexer_workspace_size(B, Tq, max_entries, k) -> int:
@@ -181,73 +185,136 @@ def _ws(ws):
     return ctypes.c_void_p(ap), ws.numel() - (ap - p)
 
 
-def csa_compress(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b, pool, stride,
-                 out_k, out_v, out_ik, stream=None):
+# ---- argument marshalling of each call (device pointers, descriptors, sizes)
+
+def _csa_compress_args(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b, pool,
+                       stride, out_k, out_v, out_ik, stream=None):
     cs = [cache_struct(c) for c in (raw_k, raw_v, raw_ik, out_k, out_v, out_ik)]
-    _check(_lib.csa_compress(B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]),
-                             _ref(cs[1]), _ref(cs[2]), _ptr(gate_w), _ptr(gate_b), pool, stride,
-                             _ref(cs[3]), _ref(cs[4]), _ref(cs[5]), _stream(stream)),
-           "csa_compress")
+    return (B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]), _ref(cs[1]), _ref(cs[2]),
+            _ptr(gate_w), _ptr(gate_b), pool, stride, _ref(cs[3]), _ref(cs[4]), _ref(cs[5]),
+            _stream(stream))
 
 
-def hca_compress(B, t_begin, t_end, max_new, raw_k, raw_v, gate_w, gate_b, pool, stride,
-                 out_k, out_v, stream=None):
+def _hca_compress_args(B, t_begin, t_end, max_new, raw_k, raw_v, gate_w, gate_b, pool, stride,
+                       out_k, out_v, stream=None):
     cs = [cache_struct(c) for c in (raw_k, raw_v, out_k, out_v)]
-    _check(_lib.hca_compress(B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]),
-                             _ref(cs[1]), _ptr(gate_w), _ptr(gate_b), pool, stride, _ref(cs[2]),
-                             _ref(cs[3]), _stream(stream)), "hca_compress")
+    return (B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]), _ref(cs[1]),
+            _ptr(gate_w), _ptr(gate_b), pool, stride, _ref(cs[2]), _ref(cs[3]), _stream(stream))
 
 
-def csa_compress_channel_gate(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b,
-                              gate_w_ik, gate_b_ik, pool, stride, out_k, out_v, out_ik,
-                              stream=None):
+def _csa_compress_channel_gate_args(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w,
+                                    gate_b, gate_w_ik, gate_b_ik, pool, stride, out_k, out_v,
+                                    out_ik, stream=None):
+    cs = [cache_struct(c) for c in (raw_k, raw_v, raw_ik, out_k, out_v, out_ik)]
+    return (B, _ptr(t_begin), _ptr(t_end), int(max_new), _ref(cs[0]), _ref(cs[1]), _ref(cs[2]),
+            _ptr(gate_w), _ptr(gate_b), _ptr(gate_w_ik), _ptr(gate_b_ik), pool, stride,
+            _ref(cs[3]), _ref(cs[4]), _ref(cs[5]), _stream(stream))
+
+
+def _indexer_args(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
+                  out_idx, out_score, ws, stream=None):
+    wp, wn = _ws(ws)
+    return (B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w), H_I, d_I,
+            _ikref(ik), stride, k, int(max_entries), _ptr(out_idx), _ptr(out_score), wp, wn,
+            _stream(stream))
+
+
+def _attn_decode_args(B, ctx_len, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
+                      max_entries, win_k, win_v, window, out, lse, ws, stream=None):
+    cs = [cache_struct(c) for c in (comp_k, comp_v, win_k, win_v)]
+    wp, wn = _ws(ws)
+    return (B, _ptr(ctx_len), _ptr(q), Hq, sm_scale, _ref(cs[0]), _ref(cs[1]), comp_stride,
+            _ptr(sel), k, int(max_entries), _ref(cs[2]), _ref(cs[3]), window, _ptr(out),
+            _ptr(lse), wp, wn, _stream(stream))
+
+
+def _attn_prefill_args(B, Tq, q_pos, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
+                       max_entries, win_k, win_v, window, out, lse, ws, stream=None):
+    cs = [cache_struct(c) for c in (comp_k, comp_v, win_k, win_v)]
+    wp, wn = _ws(ws)
+    return (B, Tq, _ptr(q_pos), _ptr(q), Hq, sm_scale, _ref(cs[0]), _ref(cs[1]), comp_stride,
+            _ptr(sel), k, int(max_entries), _ref(cs[2]), _ref(cs[3]), window, _ptr(out),
+            _ptr(lse), wp, wn, _stream(stream))
+
+
+_MARSHAL = {
+    "csa_compress": _csa_compress_args,
+    "hca_compress": _hca_compress_args,
+    "csa_compress_channel_gate": _csa_compress_channel_gate_args,
+    "hca_compress_channel_gate": _hca_compress_args,
+    "indexer_topk": _indexer_args,
+    "indexer_score": _indexer_args,
+    "indexer_select": _indexer_args,
+    "hybrid_attn_decode": _attn_decode_args,
+    "hybrid_attn_prefill": _attn_prefill_args,
+    "cskv_ring_store": _ring_store_args,
+}
+
+
+class PreparedCall:
+    """One library call with its arguments marshalled once.  A decode step
+    repeats the same calls on the same buffers every token: where the
+    tensors' addresses, the cache descriptors and the stream stay fixed, a
+    prepared call skips the marshalling (and calling it is all the host does
+    per launch).  prepare("hybrid_attn_decode", *args) takes the arguments of
+    the function of that name."""
+    __slots__ = ("_fn", "_args", "_name")
+
+    def __init__(self, name, args):
+        self._fn, self._args, self._name = getattr(_lib, name), args, name
+
+    def __call__(self):
+        rc = self._fn(*self._args)
+        if rc != OK:
+            raise CskvError(rc, self._name)
+
+
+def prepare(name, *args, **kw) -> PreparedCall:
+    return PreparedCall(name, _MARSHAL[name](*args, **kw))
+
+
+def csa_compress(*args, **kw):
+    _check(_lib.csa_compress(*_csa_compress_args(*args, **kw)), "csa_compress")
+
+
+def hca_compress(*args, **kw):
+    _check(_lib.hca_compress(*_hca_compress_args(*args, **kw)), "hca_compress")
+
+
+def csa_compress_channel_gate(*args, **kw):
     """csa_compress with one gate per channel: gate_b [pool][D], the indexer
     keys' own gate_w_ik [d_I] and gate_b_ik [pool][d_I]."""
-    cs = [cache_struct(c) for c in (raw_k, raw_v, raw_ik, out_k, out_v, out_ik)]
-    _check(_lib.csa_compress_channel_gate(B, _ptr(t_begin), _ptr(t_end), int(max_new),
-                                          _ref(cs[0]), _ref(cs[1]), _ref(cs[2]), _ptr(gate_w),
-                                          _ptr(gate_b), _ptr(gate_w_ik), _ptr(gate_b_ik), pool,
-                                          stride, _ref(cs[3]), _ref(cs[4]), _ref(cs[5]),
-                                          _stream(stream)), "csa_compress_channel_gate")
+    _check(_lib.csa_compress_channel_gate(*_csa_compress_channel_gate_args(*args, **kw)),
+           "csa_compress_channel_gate")
 
 
-def hca_compress_channel_gate(B, t_begin, t_end, max_new, raw_k, raw_v, gate_w, gate_b, pool,
-                              stride, out_k, out_v, stream=None):
+def hca_compress_channel_gate(*args, **kw):
     """hca_compress with one gate per channel: gate_b [pool][D]."""
-    cs = [cache_struct(c) for c in (raw_k, raw_v, out_k, out_v)]
-    _check(_lib.hca_compress_channel_gate(B, _ptr(t_begin), _ptr(t_end), int(max_new),
-                                          _ref(cs[0]), _ref(cs[1]), _ptr(gate_w), _ptr(gate_b),
-                                          pool, stride, _ref(cs[2]), _ref(cs[3]),
-                                          _stream(stream)), "hca_compress_channel_gate")
+    _check(_lib.hca_compress_channel_gate(*_hca_compress_args(*args, **kw)),
+           "hca_compress_channel_gate")
 
 
 def indexer_topk(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
                  out_idx, out_score, ws, stream=None):
-    wp, wn = _ws(ws)
-    _check(_lib.indexer_topk(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
-                             H_I, d_I, _ikref(ik), stride, k, int(max_entries),
-                             _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
-           "indexer_topk")
+    _check(_lib.indexer_topk(*_indexer_args(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I,
+                                            ik, stride, k, max_entries, out_idx, out_score, ws,
+                                            stream)), "indexer_topk")
 
 
 def indexer_score(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
                   out_idx, out_score, ws, stream=None):
     """First half of indexer_topk: scores and histogram into the workspace."""
-    wp, wn = _ws(ws)
-    _check(_lib.indexer_score(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
-                              H_I, d_I, _ikref(ik), stride, k, int(max_entries),
-                              _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
-           "indexer_score")
+    _check(_lib.indexer_score(*_indexer_args(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I,
+                                             ik, stride, k, max_entries, out_idx, out_score, ws,
+                                             stream)), "indexer_score")
 
 
 def indexer_select(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k, max_entries,
                    out_idx, out_score, ws, stream=None):
     """Second half of indexer_topk: the top-k from the workspace's scores."""
-    wp, wn = _ws(ws)
-    _check(_lib.indexer_select(B, Tq, _ptr(q_pos), _ptr(q_ik), _ptr(q_ik_scale), _ptr(head_w),
-                               H_I, d_I, _ikref(ik), stride, k, int(max_entries),
-                               _ptr(out_idx), _ptr(out_score), wp, wn, _stream(stream)),
-           "indexer_select")
+    _check(_lib.indexer_select(*_indexer_args(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I,
+                                              ik, stride, k, max_entries, out_idx, out_score, ws,
+                                              stream)), "indexer_select")
 
 
 def indexer_topk_noalloc(B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik, stride, k,
@@ -265,24 +332,12 @@ def noalloc_scratch_bytes() -> int:
     return int(_lib.cskv_noalloc_scratch_bytes())
 
 
-def hybrid_attn_decode(B, ctx_len, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
-                       max_entries, win_k, win_v, window, out, lse, ws, stream=None):
-    cs = [cache_struct(c) for c in (comp_k, comp_v, win_k, win_v)]
-    wp, wn = _ws(ws)
-    _check(_lib.hybrid_attn_decode(B, _ptr(ctx_len), _ptr(q), Hq, sm_scale, _ref(cs[0]),
-                                   _ref(cs[1]), comp_stride, _ptr(sel), k, int(max_entries),
-                                   _ref(cs[2]), _ref(cs[3]), window, _ptr(out), _ptr(lse), wp,
-                                   wn, _stream(stream)), "hybrid_attn_decode")
+def hybrid_attn_decode(*args, **kw):
+    _check(_lib.hybrid_attn_decode(*_attn_decode_args(*args, **kw)), "hybrid_attn_decode")
 
 
-def hybrid_attn_prefill(B, Tq, q_pos, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
-                        max_entries, win_k, win_v, window, out, lse, ws, stream=None):
-    cs = [cache_struct(c) for c in (comp_k, comp_v, win_k, win_v)]
-    wp, wn = _ws(ws)
-    _check(_lib.hybrid_attn_prefill(B, Tq, _ptr(q_pos), _ptr(q), Hq, sm_scale, _ref(cs[0]),
-                                    _ref(cs[1]), comp_stride, _ptr(sel), k, int(max_entries),
-                                    _ref(cs[2]), _ref(cs[3]), window, _ptr(out), _ptr(lse), wp,
-                                    wn, _stream(stream)), "hybrid_attn_prefill")
+def hybrid_attn_prefill(*args, **kw):
+    _check(_lib.hybrid_attn_prefill(*_attn_prefill_args(*args, **kw)), "hybrid_attn_prefill")
 
 
 def check_device_errors(stream=None) -> int:

@@ -183,10 +183,33 @@ def test_argument_errors_are_caught_on_the_host(C):
 
 def test_layer_phases_name_the_split_calls(C):
     # CSALayer.select(phase=...) dispatches to the two halves of indexer_topk
+    import inspect
     from compressed_sparse_kv_softmax_b200 import layer
-    assert layer.indexer_score is C.indexer_score
-    assert layer.indexer_select is C.indexer_select
-    assert layer.indexer_topk is C.indexer_topk
+    src = inspect.getsource(layer.CSALayer.select)
+    for name in ("indexer_topk", "indexer_score", "indexer_select"):
+        assert f'"{name}"' in src
+
+
+def test_prepared_calls_marshal_like_the_plain_calls(C):
+    # every call the layers prepare is a library entry point, and a prepared
+    # call holds exactly the arguments the plain function passes
+    import torch
+    for name in C._MARSHAL:
+        assert hasattr(C.lib, name), name
+    t = [torch.zeros(64, dtype=torch.int64) for _ in range(8)]
+    cache = {"fmt": "e4m3vec", "d_nope": 128, "d_rope": 0, "ring": 0, "cap": 16,
+             "data": torch.zeros(1, 16, 128, dtype=torch.uint8),
+             "scale": torch.zeros(1, 16, 1)}
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    args = (1, 1, t[0], t[1], t[2], t[3], 64, 128, cache, 4, 8, 16, t[4], t[5], ws, 7)
+    call = C.prepare("indexer_score", *args)
+    assert call._fn is C.lib.indexer_score
+    plain = C._indexer_args(*args)
+    for a, b in zip(call._args, plain):
+        if isinstance(a, ctypes.c_void_p):
+            assert a.value == b.value
+        elif isinstance(a, (int, float)):
+            assert a == b
 
 
 def test_header_is_plain_c_and_links(tmp_path):
