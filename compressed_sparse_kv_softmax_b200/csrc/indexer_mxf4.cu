@@ -78,6 +78,8 @@ struct __align__(1024) Smem {
 
 __device__ __forceinline__ void record_abort(Smem &sm) { sm.abort = 1; }
 
+// kPaged: the key cache may be paged (block table)
+template <bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                     float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
@@ -158,13 +160,13 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
   // tile with no block is placed past the planes, i.e. reads zeros, unused)
   auto tile_row0 = [&](int i) -> long long {
     const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
-    if (!a.ik.bt) return (long long)b * a.ik.cap + j0;
+    if constexpr (!kPaged) return (long long)b * a.ik.cap + j0;
     return i < kPagedTiles ? sm.tile_row[i] : a.ik.run_row0(b, j0, a.ik.plane_rows(a.B));
   };
   if (warp == 0) {
     // ---------------- TMA producer
     const long long total_rows = a.ik.plane_rows(a.B);
-    if (a.ik.bt) {
+    if (kPaged) {
       // (read by the other roles after the tiles' barriers)
       const int nt = min(kPagedTiles, tiles_of(a.max_entries));
       for (int i = lane; i < nt; i += 32)
@@ -385,7 +387,8 @@ int launch_indexer_mxf4(const IndexerArgs &a, float *scores, long long ld, uint3
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(Smem) + 1024;
-  if (!ensure_dynamic_smem(indexer_mxf4_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+  auto kernel = a.ik.bt ? indexer_mxf4_kernel<true> : indexer_mxf4_kernel<false>;
+  if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -397,8 +400,8 @@ int launch_indexer_mxf4(const IndexerArgs &a, float *scores, long long ld, uint3
   // a packed exponent plane (4 bytes per entry, one after another) comes by
   // bulk copies with the key tiles
   const bool packed = a.ik.scale_stride == 4;
-  return launch_pdl(indexer_mxf4_kernel, dim3((unsigned)splits, (unsigned)rows), dim3(kThreads),
-                    smem, st, a, map, scores, ld, hist, ctr, packed) == cudaSuccess
+  return launch_pdl(kernel, dim3((unsigned)splits, (unsigned)rows), dim3(kThreads), smem, st, a,
+                    map, scores, ld, hist, ctr, packed) == cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;
 }

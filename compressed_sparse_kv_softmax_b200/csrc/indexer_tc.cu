@@ -84,7 +84,9 @@ struct __align__(1024) Smem {
 // A wait ran out: the CTA stops, and its scores are marked failed at the end.
 __device__ __forceinline__ void record_abort(Smem &sm) { sm.abort = 1; }
 
-template <bool kVec>
+// kPaged: the key cache may be paged (block table); the contiguous
+// instantiation carries no block-table code
+template <bool kVec, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                   float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
@@ -180,13 +182,13 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
   // tile with no block is placed past the planes, i.e. reads zeros, unused)
   auto tile_row0 = [&](int i) -> long long {
     const long long j0 = (long long)(blockIdx.x + i * gridDim.x) * kTile;
-    if (!a.ik.bt) return (long long)b * a.ik.cap + j0;
+    if constexpr (!kPaged) return (long long)b * a.ik.cap + j0;
     return i < kPagedTiles ? sm.tile_row[i] : a.ik.run_row0(b, j0, a.ik.plane_rows(a.B));
   };
   if (warp == 0) {
     // ---------------- TMA producer
     const long long total_rows = a.ik.plane_rows(a.B);
-    if (a.ik.bt) {
+    if (kPaged) {
       // (read by the other roles after the tiles' barriers)
       const int nt = min(kPagedTiles, tiles_of(a.max_entries));
       for (int i = lane; i < nt; i += 32)
@@ -514,7 +516,9 @@ int launch_indexer_tc(const IndexerArgs &a, float *scores, long long ld, uint32_
   if (!make_key_tmap(a, &map)) return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(Smem) + 1024;
   const bool vec = a.ik.fmt == CSKV_FMT_E4M3_VEC;
-  auto kernel = vec ? indexer_tc_kernel<true> : indexer_tc_kernel<false>;
+  const bool paged = a.ik.bt != nullptr;
+  auto kernel = vec ? (paged ? indexer_tc_kernel<true, true> : indexer_tc_kernel<true, false>)
+                    : (paged ? indexer_tc_kernel<false, true> : indexer_tc_kernel<false, false>);
   if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -119,6 +119,8 @@ __device__ __forceinline__ float2 row_part(const float (&v)[32], const float *c1
   return make_float2(acc0.x + acc0.y, acc1.x + acc1.y);
 }
 
+// kPaged: the key cache may be paged (block table)
+template <bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
                     float *__restrict__ scores, long long ld, uint32_t *__restrict__ hist_g,
@@ -220,12 +222,12 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
   // tile with no block is placed past the planes, i.e. reads zeros, unused)
   auto tile_row0 = [&](int i) -> long long {
     const long long j0 = ((long long)blockIdx.x + (long long)i * gridDim.x) * kTile;
-    if (!a.ik.bt) return (long long)b * a.ik.cap + j0;
+    if constexpr (!kPaged) return (long long)b * a.ik.cap + j0;
     return i < kPagedTiles ? sm.tile_row[i] : a.ik.run_row0(b, j0, a.ik.plane_rows(a.B));
   };
   if (warp == 0) {
     // ---------------- TMA producer
-    if (a.ik.bt) {
+    if (kPaged) {
       // (read by the other roles after the tiles' barriers)
       const int nt = min(kPagedTiles, tiles_of(a.max_entries));
       for (int i = lane; i < nt; i += 32)
@@ -455,7 +457,8 @@ int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint3
   CUtensorMap map;
   if (!make_key_tmap(a, &map)) return CSKV_ERR_UNSUPPORTED;
   const size_t smem = sizeof(RowsSmem) + 1024;
-  if (!ensure_dynamic_smem(indexer_rows_kernel, smem)) return CSKV_ERR_UNSUPPORTED;
+  auto kernel = a.ik.bt ? indexer_rows_kernel<true> : indexer_rows_kernel<false>;
+  if (!ensure_dynamic_smem(kernel, smem)) return CSKV_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -468,8 +471,8 @@ int launch_indexer_rows(const IndexerArgs &a, float *scores, long long ld, uint3
   if (splits < 1) splits = 1;
   dim3 grid((unsigned)splits, (unsigned)groups);
   const bool packed = a.ik.scale_stride == 4;
-  return launch_pdl(indexer_rows_kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld,
-                    hist, ctr, gps, packed) == cudaSuccess
+  return launch_pdl(kernel, grid, dim3(kThreads), smem, st, a, map, scores, ld, hist, ctr, gps,
+                    packed) == cudaSuccess
              ? CSKV_OK
              : CSKV_ERR_CUDA;
 }
