@@ -734,6 +734,12 @@ def run_e2e(args, replicas, wl, dev, world):
         done[b].record(stream)
 
     with torch.cuda.stream(stream):
+        # every graph runs once before the timed region (its first launch
+        # uploads it), on the inputs of a step of its own pattern
+        for (r, key, b), g in graphs.items():
+            stream.synchronize()
+            host_in[b].copy_(host_small[first[key]])
+            g.replay()
         for i in range(3):
             replay(i)
     stream.synchronize()
