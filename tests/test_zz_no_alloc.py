@@ -55,6 +55,25 @@ def test_noalloc_matches_workspace_entry_point_twice():
     _same(_noalloc(C, wl, Ld, ref.max_entries, ref), want, "noalloc call 2")
 
 
+@pytest.mark.parametrize("ik_fmt,bs", [("e4m3vec", 256), ("mxfp4", 128), ("e4m3vec", 32)])
+def test_noalloc_on_paged_keys_matches_workspace_entry_point(ik_fmt, bs):
+    # a paged indexer-key cache (block table, a tail block without a pool
+    # block) through the fixed scratch: the same selection as with a
+    # workspace (tensor-core scoring for blocks of 128 or more, the CUDA-core
+    # kernel for smaller ones)
+    C = require_gpu()
+    from compressed_sparse_kv_softmax_b200.layer import CSALayer
+    wl = W.get("parity_decode").with_(ik_fmt=ik_fmt)
+    L = W.make_csa_layer(wl)
+    L["comp_ik"] = W.page_cache(L["comp_ik"], bs, seed=bs, unmapped_tail=1)
+    Ld = to_device(L)
+    ref = CSALayer(Ld)
+    ref.select()
+    torch.cuda.synchronize()
+    want = (ref.idx.cpu().numpy(), ref.score.cpu().numpy())
+    _same(_noalloc(C, wl, Ld, ref.max_entries, ref), want, f"noalloc paged {ik_fmt} bs {bs}")
+
+
 def test_noalloc_limit_is_the_workspace_size():
     C = require_gpu()
     wl = W.get("parity_decode")
