@@ -6,6 +6,12 @@ non-zero status raises `CskvError`.  All computation runs in the library's
 CUDA kernels; there is no CPU fallback.  Importing the package without a
 built libcskv.so raises ImportError.
 
+With CSKV_CHECK=1 in the environment the package loads the checked build
+libcskv_check.so instead (same entry points; its kernels test every index
+they read from device memory and record DEV_BOUNDS in the device status word
+when one is out of range).  CSKV_SPLITS=<n> makes the attention use n splits
+per query row (tuning only; read once by the library).
+
 Cache planes follow the C descriptor (include/cskv.h): for B sequences of
 `cap` slots, `data` is [B, cap, ...] with one slot per row; E4M3_BF16 caches
 add `scale` [B, cap, >= d_nope/64] fp32 and `rope` [B, cap, d_rope] bf16.
@@ -16,18 +22,20 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libcskv.so")
+CHECKED = os.environ.get("CSKV_CHECK", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libcskv_check.so" if CHECKED else "libcskv.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m compressed_sparse_kv_softmax_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python compressed_sparse_kv_softmax_b200/build.py"
+        f"{' --check' if CHECKED else ''}`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE, ERR_SCRATCH_LIMIT, ERR_DEVICE = (
     0, -1, -2, -3, -4, -5, -6)
 # device-side events (bits of cskv_check_device_errors)
-DEV_INDEXER_WAIT, DEV_TOPK_BARRIER, DEV_ATTN_WAIT, DEV_ROW_FAILED = 1, 2, 4, 8
+DEV_INDEXER_WAIT, DEV_TOPK_BARRIER, DEV_ATTN_WAIT, DEV_ROW_FAILED, DEV_BOUNDS = 1, 2, 4, 8, 16
 FMT_F32, FMT_E4M3_BF16, FMT_E4M3_VEC, FMT_MXFP4 = 0, 1, 2, 3
 _FMT = {"f32": FMT_F32, "e4m3": FMT_E4M3_BF16, "e4m3vec": FMT_E4M3_VEC, "mxfp4": FMT_MXFP4}
 
@@ -79,6 +87,7 @@ _lib.cskv_debug_indexer_stall.restype = ctypes.c_uint32
 _lib.cskv_error_string.argtypes = [_I]
 _lib.cskv_error_string.restype = ctypes.c_char_p
 _lib.cskv_version.restype = _I
+_lib.cskv_build_checked.restype = _I
 for _name in ("csa_compress", "hca_compress", "csa_compress_channel_gate",
               "hca_compress_channel_gate", "indexer_topk", "indexer_score", "indexer_select",
               "hybrid_attn_decode", "hybrid_attn_prefill"):
@@ -369,6 +378,11 @@ def error_string(status: int) -> str:
 
 def version() -> int:
     return int(_lib.cskv_version())
+
+
+def build_checked() -> bool:
+    """True for the checked build (libcskv_check.so, CSKV_CHECK=1)."""
+    return bool(_lib.cskv_build_checked())
 
 
 lib = _lib

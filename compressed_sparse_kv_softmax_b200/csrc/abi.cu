@@ -2,6 +2,8 @@
 // launchers.  Nothing is enqueued when a check fails.
 #include <cstdint>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "cskv_internal.cuh"
 
 using namespace cskv;
@@ -12,6 +14,17 @@ constexpr int64_t kMaxIndexerRows = 65535;
 namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// An NVTX range named for the entry point around each call (host side: it
+// brackets the checks and the launches, not the kernels' device time); with
+// no profiler attached a push and a pop cost a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
+#define CSKV_RANGE() const NvtxRange nvtx_range_(__func__)
 
 // ring: 1 / 0 required value, -1 either
 int check_cache(const cskv_cache *c, int ring) {
@@ -231,6 +244,7 @@ int csa_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
                  const float *gate_w, const float *gate_b, int pool, int stride,
                  const cskv_cache *out_k, const cskv_cache *out_v, const cskv_cache *out_ik,
                  cskv_stream_t stream) {
+  CSKV_RANGE();
   return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b,
                          nullptr, nullptr, 0, pool, stride, out_k, out_v, out_ik, stream);
 }
@@ -241,6 +255,7 @@ int csa_compress_channel_gate(int B, const int64_t *t_begin, const int64_t *t_en
                               const float *gate_w_ik, const float *gate_b_ik, int pool,
                               int stride, const cskv_cache *out_k, const cskv_cache *out_v,
                               const cskv_cache *out_ik, cskv_stream_t stream) {
+  CSKV_RANGE();
   return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, raw_ik, gate_w, gate_b,
                          gate_w_ik, gate_b_ik, 1, pool, stride, out_k, out_v, out_ik, stream);
 }
@@ -249,6 +264,7 @@ int hca_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t ma
                  const cskv_cache *raw_k, const cskv_cache *raw_v, const float *gate_w,
                  const float *gate_b, int pool, int stride, const cskv_cache *out_k,
                  const cskv_cache *out_v, cskv_stream_t stream) {
+  CSKV_RANGE();
   return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, nullptr, gate_w, gate_b,
                          nullptr, nullptr, 0, pool, stride, out_k, out_v, nullptr, stream);
 }
@@ -258,12 +274,14 @@ int hca_compress_channel_gate(int B, const int64_t *t_begin, const int64_t *t_en
                               const float *gate_w, const float *gate_b, int pool, int stride,
                               const cskv_cache *out_k, const cskv_cache *out_v,
                               cskv_stream_t stream) {
+  CSKV_RANGE();
   return compress_common(B, t_begin, t_end, max_new, raw_k, raw_v, nullptr, gate_w, gate_b,
                          nullptr, nullptr, 1, pool, stride, out_k, out_v, nullptr, stream);
 }
 
 int cskv_ring_store(int B, const int64_t *pos, int n, const cskv_cache *const *src,
                     const cskv_cache *const *ring, cskv_stream_t stream) {
+  CSKV_RANGE();
   if (B < 0 || B > 65535 || n < 1 || n > 8) return CSKV_ERR_ARG;
   if (B == 0) return CSKV_OK;
   if (!pos || !src || !ring) return CSKV_ERR_ARG;
@@ -287,6 +305,7 @@ int indexer_topk(int B, int Tq, const int64_t *q_pos, const void *q_ik, const fl
                  const float *head_w, int H_I, int d_I, const cskv_cache *ik, int stride, int k,
                  int64_t max_entries, int32_t *out_idx, float *out_score, void *ws,
                  size_t ws_bytes, cskv_stream_t stream) {
+  CSKV_RANGE();
   return indexer_common(kIndexerScore | kIndexerSelect, B, Tq, q_pos, q_ik, q_ik_scale, head_w,
                         H_I, d_I, ik, stride, k, max_entries, out_idx, out_score, ws, ws_bytes,
                         stream);
@@ -296,6 +315,7 @@ int indexer_score(int B, int Tq, const int64_t *q_pos, const void *q_ik, const f
                   const float *head_w, int H_I, int d_I, const cskv_cache *ik, int stride, int k,
                   int64_t max_entries, int32_t *out_idx, float *out_score, void *ws,
                   size_t ws_bytes, cskv_stream_t stream) {
+  CSKV_RANGE();
   return indexer_common(kIndexerScore, B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik,
                         stride, k, max_entries, out_idx, out_score, ws, ws_bytes, stream);
 }
@@ -304,6 +324,7 @@ int indexer_select(int B, int Tq, const int64_t *q_pos, const void *q_ik, const 
                    const float *head_w, int H_I, int d_I, const cskv_cache *ik, int stride, int k,
                    int64_t max_entries, int32_t *out_idx, float *out_score, void *ws,
                    size_t ws_bytes, cskv_stream_t stream) {
+  CSKV_RANGE();
   return indexer_common(kIndexerSelect, B, Tq, q_pos, q_ik, q_ik_scale, head_w, H_I, d_I, ik,
                         stride, k, max_entries, out_idx, out_score, ws, ws_bytes, stream);
 }
@@ -318,6 +339,7 @@ int hybrid_attn_decode(int B, const int64_t *ctx_len, const void *q, int Hq, flo
                        const int32_t *sel, int k, int64_t max_entries, const cskv_cache *win_k,
                        const cskv_cache *win_v, int window, float *out, float *lse, void *ws,
                        size_t ws_bytes, cskv_stream_t stream) {
+  CSKV_RANGE();
   return attention_common(B, 1, ctx_len, 1, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
                           max_entries, win_k, win_v, window, out, lse, ws, ws_bytes, stream);
 }
@@ -328,6 +350,7 @@ int hybrid_attn_prefill(int B, int Tq, const int64_t *q_pos, const void *q, int 
                         const cskv_cache *win_k, const cskv_cache *win_v, int window,
                         float *out, float *lse, void *ws, size_t ws_bytes,
                         cskv_stream_t stream) {
+  CSKV_RANGE();
   return attention_common(B, Tq, q_pos, 0, q, Hq, sm_scale, comp_k, comp_v, comp_stride, sel, k,
                           max_entries, win_k, win_v, window, out, lse, ws, ws_bytes, stream);
 }
@@ -348,5 +371,7 @@ const char *cskv_error_string(int status) {
 }
 
 int cskv_version(void) { return 100; }
+
+int cskv_build_checked(void) { return kChecked ? 1 : 0; }
 
 }  // extern "C"

@@ -18,6 +18,8 @@
 // tensor-core kernel in attn_tc.cu.
 #include <math_constants.h>
 
+#include <cstdlib>
+
 #include "cskv_internal.cuh"
 
 namespace cskv {
@@ -52,6 +54,9 @@ __device__ __forceinline__ RowInfo row_info(const AttnArgs &a, int row) {
   } else {
     long long n = (r.pos + 1) / a.comp_stride;
     r.n_comp = n < a.max_entries ? n : a.max_entries;
+    // checked build: the row's visible entries within the host bound and the caches
+    if (kChecked && threadIdx.x == 0)
+      a.comp_k.check(n <= a.max_entries && n <= a.comp_k.cap && n <= a.comp_v.cap);
   }
   r.w_lo = r.pos - a.window + 1;
   if (r.w_lo < 0) r.w_lo = 0;
@@ -104,6 +109,10 @@ attn_units_kernel(AttnArgs a, AttnPlan p, float *__restrict__ part_o,
         if (i < ri.n_comp) {
           const long long j = a.sel ? (long long)a.sel[(long long)row * a.k + i] : i;
           if (j >= 0 && j < a.comp_k.cap && j < a.comp_v.cap) { src = 1; slot = j; }
+          // checked build: a selected entry is -1 or visible to the row
+          if (kChecked && a.sel &&
+              !a.comp_k.check(j == -1 || (src == 1 && j < (ri.pos + 1) / a.comp_stride)))
+            src = 0;
         }
       } else {
         const long long i = (long long)(unit - p.n_comp_units) * kChunk + tid;
@@ -306,12 +315,28 @@ attn_merge_kernel(int Hq, int Dv, int n_chunks, const float *__restrict__ part_o
 
 }  // namespace
 
+// CSKV_SPLITS=<n> in the environment (read once per process): n splits per
+// query row instead of the planned count, for tuning (clipped to the row's
+// units; the workspace sizes follow it, so it has to be set before the first
+// call that sizes a workspace).  0 when unset or not a positive number.
+static long long splits_override() {
+  static const long long v = [] {
+    const char *e = std::getenv("CSKV_SPLITS");
+    if (!e || !*e) return 0LL;
+    char *end = nullptr;
+    const long long n = std::strtoll(e, &end, 10);
+    return (end && *end == '\0' && n > 0) ? n : 0LL;
+  }();
+  return v;
+}
+
 AttnPlan attn_plan(long long rows, long long max_comp, int window, int unit) {
   AttnPlan p;
   p.unit = unit;
   p.n_comp_units = (int)((max_comp + unit - 1) / unit);
   p.n_units = p.n_comp_units + (window + unit - 1) / unit;
   long long splits = (kTargetCtas + rows - 1) / rows;
+  if (splits_override() > 0) splits = splits_override();
   if (splits > p.n_units) splits = p.n_units;
   if (splits < 1) splits = 1;
   p.per_cta = (int)((p.n_units + splits - 1) / splits);

@@ -303,6 +303,8 @@ __device__ __forceinline__ Row row_of(const AttnArgs &a, int row) {
   else {
     const long long n = (r.pos + 1) / a.comp_stride;
     r.n_comp = n < a.max_entries ? n : a.max_entries;
+    // checked build: the row's visible entries within the host bound and the cache
+    if (kChecked && threadIdx.x == 0) a.comp_k.check(n <= a.max_entries && n <= a.comp_k.cap);
   }
   r.w_lo = r.pos - a.window + 1;
   if (r.w_lo < 0) r.w_lo = 0;
@@ -434,6 +436,10 @@ attn_tc_kernel(const AttnArgs a, int unit_keys, int n_comp_units, int n_units, i
         if (comp_unit) {
           const long long j = a.sel ? (long long)a.sel[(long long)row * a.k + i] : i;
           if (j >= 0 && j < src.cap) slot = j;
+          // checked build: a selected entry is -1 or visible to the row
+          if (kChecked && a.sel &&
+              !src.check(j == -1 || (slot >= 0 && j < (R.pos + 1) / a.comp_stride)))
+            slot = -1;
         } else {
           slot = src.slot_of(R.w_lo + i);
         }

@@ -122,6 +122,38 @@ __device__ void pool_values(const Cache &raw, int b, long long first, int pool, 
   }
 }
 
+// Checked build: the device-side token counts of sequence b against the
+// launch and the caches (one thread; nothing in the regular build, whose
+// kernels skip what the tests reject without recording it):
+//  - the grid's max_new entries per sequence cover n(t_end) - n(t_begin);
+//  - entry j lies below every output's cap and has a block in each;
+//  - the first position it pools is still held by every ring (a ring of
+//    cap slots holds positions t_end - cap .. t_end - 1).
+__device__ __forceinline__ void check_entry(const int64_t *t_begin, const int64_t *t_end, int b,
+                                            long long j, int pool, int stride,
+                                            const Cache &raw_k, const Cache &raw_v,
+                                            const Cache &raw_ik, const Cache &out_k,
+                                            const Cache &out_v, const Cache &out_ik) {
+  if constexpr (kChecked) {
+    if (threadIdx.x != 0) return;
+    const long long tb = t_begin[b], te = t_end[b], n_end = te / stride;
+    if (blockIdx.x == gridDim.x - 1) out_k.check(tb / stride + (long long)gridDim.x >= n_end);
+    if (j < 0 || j >= n_end) return;
+    const bool in_cap = out_k.check(j < out_k.cap) && (!raw_v.data || out_v.check(j < out_v.cap)) &&
+                        (!raw_ik.data || out_ik.check(j < out_ik.cap));
+    if (in_cap) {
+      out_k.check(out_k.mapped(b, j));
+      if (raw_v.data) out_v.check(out_v.mapped(b, j));
+      if (raw_ik.data) out_ik.check(out_ik.mapped(b, j));
+    }
+    long long lo = (long long)stride * (j + 1) - pool;
+    lo = lo < 0 ? 0 : lo;
+    raw_k.check(lo > te - 1 - raw_k.cap);
+    if (raw_v.data) raw_v.check(lo > te - 1 - raw_v.cap);
+    if (raw_ik.data) raw_ik.check(lo > te - 1 - raw_ik.cap);
+  }
+}
+
 template <bool kPaged>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__ t_end,
@@ -137,6 +169,7 @@ compress_kernel(const int64_t *__restrict__ t_begin, const int64_t *__restrict__
   float *pooled = smem + pool;     // [max dims]
   const int b = blockIdx.y;
   const long long j = t_begin[b] / stride + blockIdx.x;
+  check_entry(t_begin, t_end, b, j, pool, stride, raw_k, raw_v, raw_ik, out_k, out_v, out_ik);
   if (j >= t_end[b] / stride || j < 0) return;
   // never write past a cache's capacity, whatever the device-side token counts
   // say, nor into a slot that a paged cache's block table leaves without a block
@@ -383,6 +416,7 @@ compress_staged_kernel(const int64_t *__restrict__ t_begin, const int64_t *__res
   stage_bytes(reinterpret_cast<uint8_t *>(gb), reinterpret_cast<const uint8_t *>(gate_b),
               4 * pool, tid, kThreads);
   const long long j = t_begin[b] / stride + blockIdx.x;
+  check_entry(t_begin, t_end, b, j, pool, stride, raw_k, raw_v, raw_ik, out_k, out_v, out_ik);
   // never write past a cache's capacity, whatever the device-side token counts say
   if (j >= t_end[b] / stride || j < 0 || j >= out_k.cap || (raw_v.data && j >= out_v.cap) ||
       (raw_ik.data && j >= out_ik.cap) ||
@@ -510,6 +544,7 @@ compress_channel_kernel(const int64_t *__restrict__ t_begin, const int64_t *__re
   long long *rows_i = rows_v + pool;
 
   const long long j = t_begin[b] / stride + blockIdx.x;
+  check_entry(t_begin, t_end, b, j, pool, stride, raw_k, raw_v, raw_ik, out_k, out_v, out_ik);
   // never write past a cache's capacity, whatever the device-side token counts say
   if (j >= t_end[b] / stride || j < 0 || j >= out_k.cap || (raw_v.data && j >= out_v.cap) ||
       (raw_ik.data && j >= out_ik.cap) || !out_k.mapped(b, j) ||

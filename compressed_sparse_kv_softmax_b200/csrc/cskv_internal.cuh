@@ -25,6 +25,27 @@ __device__ __forceinline__ float mxfp4_value(uint32_t code, uint8_t e) {
   return e == 255 ? __int_as_float(0x7fffffff) : ldexpf(e2m1_decode(code), (int)e - 127);
 }
 
+// Checked build (compiled with -DCSKV_CHECK, libcskv_check.so): every index
+// a kernel takes from device memory (a selected entry, a block-table entry, a
+// position that names a ring slot or a cache entry) is tested against its
+// range before the access; a failed test records CSKV_DEV_BOUNDS in the
+// device status word and the access is left out, as the regular build leaves
+// it out (or keeps it inside the planes) without saying so.
+#ifdef CSKV_CHECK
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+// Sticky per-device status word (status.cu): kernels OR CSKV_DEV_* bits into
+// it when a bounded wait runs out (and, in the checked build, when an index
+// fails its test).  device_status_word() is its device address on the
+// current device (nullptr if the lookup failed).
+unsigned int *device_status_word();
+__device__ __forceinline__ void record_event(unsigned int *status, unsigned int bit) {
+  if (status) atomicOr(status, bit);
+}
+
 // Device-side view of a cskv_cache (passed to kernels by value).
 // Tiles of a paged key cache whose first rows a scoring CTA resolves up front
 // (the producer warp's lanes together, into shared memory), so that no tile
@@ -48,6 +69,17 @@ struct Cache {
   // paged layout: bt [B][cap >> bs_log2] physical block ids (nullptr: rows
   // b * cap + slot)
   const int32_t *bt;
+#ifdef CSKV_CHECK
+  unsigned int *status;       // checked build: where a failed index test is recorded
+#endif
+
+  // checked build: records CSKV_DEV_BOUNDS when `ok` is false; returns `ok`
+  __device__ __forceinline__ bool check(bool ok) const {
+#ifdef CSKV_CHECK
+    if (!ok) record_event(status, CSKV_DEV_BOUNDS);
+#endif
+    return ok;
+  }
 
   __host__ __device__ int dims() const { return d_nope + d_rope; }
   // scales per slot, the dims each covers, and the bytes they take
@@ -70,7 +102,8 @@ struct Cache {
   __device__ long long row(int b, long long slot) const {
     if (M == kRowFlat || !bt) return (long long)b * cap + slot;
     long long blk = bt[(long long)b * (cap >> bs_log2) + (slot >> bs_log2)];
-    blk = blk < 0 ? 0 : (blk >= nblk ? nblk - 1 : blk);   // (a bad table stays in bounds)
+    // (a slot that is read or written has a block; a bad table stays in bounds)
+    if (!check(blk >= 0 && blk < nblk)) blk = blk < 0 ? 0 : nblk - 1;
     return (blk << bs_log2) + (slot & ((1LL << bs_log2) - 1));
   }
   // whether slot s of sequence b has a block (always, unpaged)
@@ -125,7 +158,7 @@ struct Cache {
   }
 };
 
-static_assert(sizeof(Cache) == 72, "cache descriptor size");
+static_assert(sizeof(Cache) == (kChecked ? 80 : 72), "cache descriptor size");
 
 // (field ranges are checked by the ABI: dims < 2^15, strides and blocks < 2^31)
 inline Cache to_dev(const cskv_cache *c) {
@@ -141,6 +174,9 @@ inline Cache to_dev(const cskv_cache *c) {
   v.bs_log2 = 0;
   while (c->block_table && (1LL << v.bs_log2) < c->block_size) ++v.bs_log2;
   v.nblk = c->block_table ? (int32_t)c->num_blocks : 0;
+#ifdef CSKV_CHECK
+  v.status = device_status_word();
+#endif
   return v;
 }
 
@@ -257,13 +293,6 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Sticky per-device status word (status.cu): kernels OR CSKV_DEV_* bits into
-// it when a bounded wait runs out.  device_status_word() is its device
-// address on the current device (nullptr if the lookup failed).
-unsigned int *device_status_word();
-__device__ __forceinline__ void record_event(unsigned int *status, unsigned int bit) {
-  if (status) atomicOr(status, bit);
-}
 // Test hook (cskv_debug_indexer_stall): mbarrier polls that bound every wait
 // of a scoring launch whose first CTA leaves out its first tile (0: off).
 uint32_t indexer_stall_polls();

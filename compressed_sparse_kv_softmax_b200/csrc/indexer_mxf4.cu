@@ -259,6 +259,8 @@ indexer_mxf4_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
       }
       const long long g0 = tile_row0(i);
       const long long tile_rows = total_rows - g0;
+      // (paged: a visible tile without a block reads as zeros past the planes)
+      if (kPaged && lane == 0) a.ik.check(g0 < total_rows);
       const ScaleSpan sp =
           packed ? scale_span(g0, tile_rows < kTile ? tile_rows : kTile, 4) : ScaleSpan{0, 0, 0};
       uint32_t wv[4];

@@ -293,7 +293,9 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tmap,
       // An odd last row of the whole cache came without them: plain load.
       mbar_wait(&sm.full[s], (i / kStages) & 1, lim);
       float sk0 = 1.f, sk1 = 0.f;            // (rows past n: score not stored)
-      if (j < n) {
+      // (paged: a visible tile without a block was read as zeros past the
+      // planes; its scales are not loaded either)
+      if (j < n && (!kPaged || a.ik.check(tile_row0(i) < total_rows))) {
         const long long g0 = tile_row0(i), g = g0 + r;
         const long long tile_rows = total_rows - g0;   // rows from the tile's first
         // entries whose scales the stage's bulk copy brought; the rest come

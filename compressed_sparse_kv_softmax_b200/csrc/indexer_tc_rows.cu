@@ -339,7 +339,9 @@ indexer_rows_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap tma
         break;
       }
       float sk = 1.f;
-      if (j < nmax) {
+      // (paged: a visible tile without a block was read as zeros past the
+      // planes; its scales are not loaded either)
+      if (j < nmax && (!kPaged || a.ik.check(tile_row0(i) < total_rows))) {
         // the scales the stage's bulk copy brought, else a plain load
         const long long g0 = tile_row0(i), tile_rows = total_rows - g0;
         const ScaleSpan sp =

@@ -37,7 +37,9 @@ ring_store_kernel(const RingPairs p, const int64_t *__restrict__ pos) {
   pdl_trigger();
   const int b = blockIdx.x, i = blockIdx.y;
   const Cache &s = p.src[i], &r = p.ring[i];
-  const long long slot = r.slot_of(pos[b]);
+  const long long q = pos[b];
+  if (!r.check(q >= 0)) return;     // (a negative position names no slot)
+  const long long slot = r.slot_of(q);
   const long long rs = r.row(b, slot), ss = s.row(b, 0);
   if (s.fmt == CSKV_FMT_F32) {
     copy_bytes(r.data + rs * r.data_stride, s.data + ss * s.data_stride, 4 * s.dims());

@@ -255,6 +255,17 @@ __device__ __forceinline__ long long visible(const int64_t *q_pos, int row, int 
   return n < 0 ? 0 : n;
 }
 
+// Checked build: a row's visible entries (q_pos + 1) / stride within the
+// host bound max_entries, which the scoring and the selection both stop at
+// (one thread of the row's first CTA; nothing in the regular build)
+__device__ __forceinline__ void check_visible(const int64_t *q_pos, int row, int stride,
+                                              long long max_entries, unsigned int *status) {
+  if constexpr (kChecked) {
+    if (threadIdx.x == 0 && (q_pos[row] + 1) / stride > max_entries)
+      record_event(status, CSKV_DEV_BOUNDS);
+  }
+}
+
 // Ascending bitonic sort of v[0..m) in shared memory, m a power of two.
 template <typename T>
 __device__ void bitonic_sort_smem(T *v, int m) {
@@ -323,6 +334,7 @@ topk_rows_kernel(const float *__restrict__ scores, long long ld, const int64_t *
   pdl_trigger();
   const int row = blockIdx.x;
   const long long n = visible(q_pos, row, stride, max_entries);
+  check_visible(q_pos, row, stride, max_entries, status);
   topk_row_single_cta(scores + (long long)row * ld, n, k, out_idx + (long long)row * k,
                       out_score ? out_score + (long long)row * k : nullptr, status);
 }
@@ -361,6 +373,7 @@ topk_select_kernel(const IndexerWs w, const int64_t *__restrict__ q_pos, int str
   long long n = (pos + 1) / stride;
   if (n > max_entries) n = max_entries;
   if (n < 0) n = 0;
+  if (me == 0) check_visible(q_pos, row, stride, max_entries, status);
 
   // the row's histogram is cleared for the next scoring call once every CTA
   // of the row has read it (here, or past the row barrier below)

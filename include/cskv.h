@@ -76,8 +76,18 @@ enum {
                                  (result unchanged) */
   CSKV_DEV_ATTN_WAIT = 4,     /* an attention CTA gave up waiting on its copies / MMAs;
                                  the affected rows' lse is NaN */
-  CSKV_DEV_ROW_FAILED = 8     /* the selection met a row with a NaN score; that row's
+  CSKV_DEV_ROW_FAILED = 8,    /* the selection met a row with a NaN score; that row's
                                  out_idx is all -1 and its out_score all NaN */
+  CSKV_DEV_BOUNDS = 16        /* checked build only (cskv_build_checked() == 1): an index
+                                 read from device memory failed its range test and the
+                                 access was left out.  The tests: a selected entry is -1 or
+                                 below both the row's visible count and the cache's
+                                 cap; a slot that is read or written has a block in
+                                 [0, num_blocks); a visible row needs no more than
+                                 max_entries entries; a compressor call has no more than
+                                 max_new entries per sequence, each below its caches' cap,
+                                 and reads only positions its rings still hold
+                                 (p > t_end - 1 - ring cap); a ring_store position is >= 0 */
 };
 
 enum {
@@ -400,6 +410,16 @@ uint32_t cskv_debug_topk_barrier_spins(uint32_t spins);
  * polls = 0 switches it off (the default).  Returns the previous setting.
  */
 uint32_t cskv_debug_indexer_stall(uint32_t polls);
+
+/*
+ * cskv_build_checked - 1 for the checked build of the library
+ * (libcskv_check.so, compiled with -DCSKV_CHECK), whose kernels test every
+ * index they read from device memory and record CSKV_DEV_BOUNDS in the status
+ * word when one is out of range; 0 for the regular build, whose kernels leave
+ * such an access out (or keep it inside the planes) without recording it.
+ * Results of valid inputs are the same bits in both builds.
+ */
+int cskv_build_checked(void);
 
 /* Static text for a status code. */
 const char *cskv_error_string(int status);
