@@ -20,7 +20,7 @@ import oracle as O
 
 TOPK_REL = 1e-3
 ATTN_REL = 2e-3
-# Natural-log units, the survey's bound.  Both attention paths keep about 22
+# Natural-log units (1e-4 absolute on lse).  Both attention paths keep about 22
 # significant bits in every product: the CUDA-core path computes in fp32, the
 # tensor-core path splits every operand that is not exact in FP16 into FP16
 # hi + lo parts (relative error ~2^-22) and accumulates in fp32.  A logit
