@@ -4,6 +4,9 @@
   every parity case passes there too, and no valid call records an
   out-of-range index (the suite's conftest reads the status word after each
   GPU test of a checked run).
+* The attention parity cases run again with the split count forced
+  (CSKV_SPLITS=1 and 5), which moves decode rows onto the kernel variants
+  that run several units per CTA.
 * Inputs whose device-side indices break the documented ranges (a selected
   entry past the row's visible count or the cache, a visible slot with a bad
   block-table entry, positions that need more entries than the compressor's
@@ -50,7 +53,8 @@ def test_checked_build_runs_the_gpu_suite(C):
     env = dict(os.environ, CSKV_CHECK="1")
     r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests"), "-m", "gpu",
                         "-x", "-q", "-p", "no:cacheprovider",
-                        "--deselect", "tests/test_gpu_checked.py::test_checked_build_runs_the_gpu_suite"],
+                        "--deselect", "tests/test_gpu_checked.py::test_checked_build_runs_the_gpu_suite",
+                        "--deselect", "tests/test_gpu_checked.py::test_forced_split_counts_keep_parity"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=1800)
     tail = "\n".join((r.stdout + r.stderr).splitlines()[-30:])
     assert r.returncode == 0, tail
@@ -59,6 +63,26 @@ def test_checked_build_runs_the_gpu_suite(C):
     summary = [ln for ln in r.stdout.splitlines() if " passed" in ln][-1]
     assert int(summary.split(" passed")[0].split()[-1]) >= 130, summary
     assert "failed" not in summary and "skipped" not in summary, summary
+
+
+@pytest.mark.parametrize("splits", ["1", "5"])
+def test_forced_split_counts_keep_parity(C, splits):
+    # CSKV_SPLITS (a tuning switch) moves the decode rows onto other kernel
+    # instantiations: one CTA running every unit of a row in sequence, or a
+    # few units per CTA; the attention parity cases must hold there too
+    if os.environ.get("CSKV_SPLITS") or C.build_checked():
+        pytest.skip("runs from the regular build's suite")
+    env = dict(os.environ, CSKV_SPLITS=splits)
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests",
+                                                                     "test_gpu_parity.py"),
+                        "-m", "gpu", "-x", "-q", "-p", "no:cacheprovider", "-k",
+                        "attention or window_only or dense_small or holes or multi_token"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=1200)
+    tail = "\n".join((r.stdout + r.stderr).splitlines()[-30:])
+    assert r.returncode == 0, tail
+    summary = [ln for ln in r.stdout.splitlines() if " passed" in ln][-1]
+    assert int(summary.split(" passed")[0].split()[-1]) >= 10, summary
+    assert "failed" not in summary, summary
 
 
 # ------------------------------------------------------------ bad indices
