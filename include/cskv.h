@@ -172,7 +172,13 @@ typedef struct cskv_cache {
  *       entries read; raw_v and raw_ik may be NULL (K = V; no indexer keys).
  *   out_k, out_v, out_ik : compressed caches (ring = 0) with cap >= n(t_end).
  * Requirements: pool >= stride; cap of each ring >= (max_new - 1) * stride + pool,
- * the span of positions that max_new consecutive entries read.
+ * the span of positions that max_new consecutive entries read (checked on the
+ * host).  The rings must still hold those positions when the call runs: a ring
+ * that already holds tokens up to t_end - 1 keeps positions >= t_end - cap, so
+ * with t_end not a multiple of stride it needs up to stride - 1 more slots
+ * (cap >= max_new * stride + pool - 1 covers every t_end).  The kernels do not
+ * see which positions a ring holds; the checked build records
+ * CSKV_DEV_BOUNDS when an entry's first position is older than t_end - cap.
  */
 int csa_compress(int B, const int64_t *t_begin, const int64_t *t_end, int64_t max_new,
                  const cskv_cache *raw_k, const cskv_cache *raw_v, const cskv_cache *raw_ik,
