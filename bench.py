@@ -850,10 +850,11 @@ def _cpu_layer(L):
     return out
 
 
-def oracle_query(Lc, Lh, frac=1.0):
+def oracle_query(Lc, Lh, frac=1.0, trace=None):
     """One decode query through the oracle: CSA indexer + top-k + sparse
     attention, HCA dense attention.  frac < 1 runs the same steps over the
-    first frac of the compressed entries (a bounded sample of the query)."""
+    first frac of the compressed entries (a bounded sample of the query).
+    trace (a list) receives each sequence's (scores, selection)."""
     import oracle as O
     from oracle.layer import as_numpy_cache, _q, _q_ik
     wl = Lc["wl"]
@@ -866,6 +867,8 @@ def oracle_query(Lc, Lh, frac=1.0):
                              O.dequant_slots(ik, b, np.arange(n_c)))
         k = max(1, int(round(wl.k * frac)))
         idx = O.topk(s, n_c, k)
+        if trace is not None:
+            trace.append((s, idx))
         ck = as_numpy_cache(Lc["comp_k"])
         sel = idx[idx >= 0]
         rk = as_numpy_cache(Lc["ring_k"])
@@ -883,23 +886,78 @@ def oracle_query(Lc, Lh, frac=1.0):
     return res
 
 
-def cpu_baseline(Lc, Lh, budget_s=12.0):
+# the parity rules of the tests: top-k sets equal up to swaps whose oracle
+# scores lie within 1e-3 of the k-th score; attention max|o - o_ref| within
+# 2e-3 of the reference's RMS, |lse - lse_ref| within 1e-4
+TOPK_REL, ATTN_REL, LSE_TOL = 1e-3, 2e-3, 1e-4
+
+
+def cpu_baseline(rep, budget_s=12.0):
     """The oracle as it stands on the host cores, whole queries until the
-    budget is spent (at least one)."""
-    Lc, Lh = _cpu_layer(Lc), _cpu_layer(Lh)
+    budget is spent (at least one).  The first of them is also the parity
+    record of the run: the same query (the replica's own positions) through
+    the library, compared with the oracle by the tests' rules."""
+    import oracle as O
+    from oracle.layer import as_numpy_cache, _q
+    rep.csa.select()
+    out_c, lse_c = rep.csa.attend()
+    out_h, lse_h = rep.hca.attend()
+    torch.cuda.synchronize()
+    g_idx = rep.csa.idx.cpu().numpy()
+    g_c, g_cl = out_c.cpu().double().numpy(), lse_c.cpu().double().numpy()
+    g_h, g_hl = out_h.cpu().double().numpy(), lse_h.cpu().double().numpy()
+    Lc, Lh = _cpu_layer(rep.csa_L), _cpu_layer(rep.hca_L)
     wl = Lc["wl"]
     t0 = time.perf_counter()
     n = 0
+    trace = []
     while True:
-        oracle_query(Lc, Lh)
+        ref = oracle_query(Lc, Lh, trace=trace if n == 0 else None)
+        if n == 0:
+            first = ref
         n += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
+    # parity of the first query (outside the timing above: the record only)
+    swaps, far, err_c, err_h, err_l = 0, 0, 0.0, 0.0, 0.0
+    ck, rk = as_numpy_cache(Lc["comp_k"]), as_numpy_cache(Lc["ring_k"])
+    for b in range(wl.B):
+        s, ridx = trace[b]
+        G = g_idx[b, 0][g_idx[b, 0] >= 0]
+        R = ridx[ridx >= 0]
+        gs, rs = set(G.tolist()), set(R.tolist())
+        kth = s[R[-1]] if R.size else 0.0
+        diff = (gs - rs) | (rs - gs)
+        far += sum(1 for j in diff if abs(s[j] - kth) > TOPK_REL * abs(kth))
+        far += int(len(G) != len(R))
+        swaps += len(gs - rs)
+        # CSA attention over the library's own selection, HCA over every entry
+        pos = int(Lc["q_pos"][b, 0])
+        wpos = O.window_positions(pos, wl.window)
+        comp = O.dequant_slots(ck, b, G)
+        win = O.dequant_slots(rk, b, O.ring_slots(wpos, rk["cap"]))
+        o_c, l_c = O.hybrid_attention(_q(Lc, b, 0), comp, comp, win, win, wl.sm_scale)
+        o_h, l_h = first[2 * b + 1]
+
+        def rel(got, ref_o):
+            return float(np.max(np.abs(got - ref_o)) / np.sqrt(np.mean(ref_o ** 2)))
+        err_c = max(err_c, rel(g_c[b, 0], o_c))
+        err_h = max(err_h, rel(g_h[b, 0], o_h))
+        err_l = max(err_l, float(np.max(np.abs(g_cl[b, 0] - l_c))),
+                    float(np.max(np.abs(g_hl[b, 0] - l_h))))
+    parity = {"query": f"replica 0 at its own position ({int(Lc['q_pos'][0, 0]):,}), "
+                       f"B={wl.B}, both layers, against the oracle's float64",
+              "topk_swaps_near_tie": int(swaps), "topk_far": int(far),
+              "csa_max_err_over_rms": round(err_c, 8), "hca_max_err_over_rms": round(err_h, 8),
+              "max_lse_err": round(err_l, 8),
+              "bounds": {"topk_rel": TOPK_REL, "attn_rel": ATTN_REL, "lse": LSE_TOL},
+              "pass": bool(far == 0 and err_c <= ATTN_REL and err_h <= ATTN_REL
+                           and err_l <= LSE_TOL)}
     return {"value": round(wl.B * n / dt, 4), "unit": UNIT, "cores": _threads(),
             "kind": "oracle",
             "sample": f"{n} whole decode queries (B={wl.B}) of the same workload, "
-                      f"numpy float64, {dt:.1f} s"}
+                      f"numpy float64, {dt:.1f} s"}, parity
 
 
 def run_reference(args, rank, world):
@@ -1140,7 +1198,7 @@ def main():
     res, replicas, wl = run_ours(args, rank, world, dev)
     res["e2e"] = run_e2e(args, replicas, wl, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(replicas[0].csa_L, replicas[0].hca_L, args.cpu_budget)
+        res["cpu_baseline"], res["parity"] = cpu_baseline(replicas[0], args.cpu_budget)
     del replicas
     torch.cuda.empty_cache()
     if args.other_workloads:
