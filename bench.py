@@ -892,36 +892,21 @@ def oracle_query(Lc, Lh, frac=1.0, trace=None):
 TOPK_REL, ATTN_REL, LSE_TOL = 1e-3, 2e-3, 1e-4
 
 
-def cpu_baseline(rep, budget_s=12.0):
-    """The oracle as it stands on the host cores, whole queries until the
-    budget is spent (at least one).  The first of them is also the parity
-    record of the run: the same query (the replica's own positions) through
-    the library, compared with the oracle by the tests' rules."""
+def parity_record(Lc, got, trace, first):
+    """The library's answer to one decode query against the oracle's, under
+    the tests' rules.  got = (idx [B][1][k], CSA out [B][1][H][Dv], CSA lse,
+    HCA out, HCA lse) from the library; trace = the oracle's (scores,
+    selection) per sequence and first = its (out, lse) pairs (CSA, HCA per
+    sequence) for the same query, as oracle_query leaves them."""
     import oracle as O
     from oracle.layer import as_numpy_cache, _q
-    rep.csa.select()
-    out_c, lse_c = rep.csa.attend()
-    out_h, lse_h = rep.hca.attend()
-    torch.cuda.synchronize()
-    g_idx = rep.csa.idx.cpu().numpy()
-    g_c, g_cl = out_c.cpu().double().numpy(), lse_c.cpu().double().numpy()
-    g_h, g_hl = out_h.cpu().double().numpy(), lse_h.cpu().double().numpy()
-    Lc, Lh = _cpu_layer(rep.csa_L), _cpu_layer(rep.hca_L)
+    g_idx, g_c, g_cl, g_h, g_hl = got
     wl = Lc["wl"]
-    t0 = time.perf_counter()
-    n = 0
-    trace = []
-    while True:
-        ref = oracle_query(Lc, Lh, trace=trace if n == 0 else None)
-        if n == 0:
-            first = ref
-        n += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    # parity of the first query (outside the timing above: the record only)
     swaps, far, err_c, err_h, err_l = 0, 0, 0.0, 0.0, 0.0
     ck, rk = as_numpy_cache(Lc["comp_k"]), as_numpy_cache(Lc["ring_k"])
+
+    def rel(out, ref_o):
+        return float(np.max(np.abs(out - ref_o)) / np.sqrt(np.mean(ref_o ** 2)))
     for b in range(wl.B):
         s, ridx = trace[b]
         G = g_idx[b, 0][g_idx[b, 0] >= 0]
@@ -939,21 +924,48 @@ def cpu_baseline(rep, budget_s=12.0):
         win = O.dequant_slots(rk, b, O.ring_slots(wpos, rk["cap"]))
         o_c, l_c = O.hybrid_attention(_q(Lc, b, 0), comp, comp, win, win, wl.sm_scale)
         o_h, l_h = first[2 * b + 1]
-
-        def rel(got, ref_o):
-            return float(np.max(np.abs(got - ref_o)) / np.sqrt(np.mean(ref_o ** 2)))
         err_c = max(err_c, rel(g_c[b, 0], o_c))
         err_h = max(err_h, rel(g_h[b, 0], o_h))
         err_l = max(err_l, float(np.max(np.abs(g_cl[b, 0] - l_c))),
                     float(np.max(np.abs(g_hl[b, 0] - l_h))))
-    parity = {"query": f"replica 0 at its own position ({int(Lc['q_pos'][0, 0]):,}), "
-                       f"B={wl.B}, both layers, against the oracle's float64",
-              "topk_swaps_near_tie": int(swaps), "topk_far": int(far),
-              "csa_max_err_over_rms": round(err_c, 8), "hca_max_err_over_rms": round(err_h, 8),
-              "max_lse_err": round(err_l, 8),
-              "bounds": {"topk_rel": TOPK_REL, "attn_rel": ATTN_REL, "lse": LSE_TOL},
-              "pass": bool(far == 0 and err_c <= ATTN_REL and err_h <= ATTN_REL
-                           and err_l <= LSE_TOL)}
+    return {"query": f"position {int(Lc['q_pos'][0, 0]):,}, B={wl.B}, both layers, against "
+                     f"the oracle's float64",
+            "topk_swaps": int(swaps), "topk_far": int(far),
+            "csa_max_err_over_rms": round(err_c, 8), "hca_max_err_over_rms": round(err_h, 8),
+            "max_lse_err": round(err_l, 8),
+            "bounds": {"topk_rel": TOPK_REL, "attn_rel": ATTN_REL, "lse": LSE_TOL},
+            "pass": bool(far == 0 and err_c <= ATTN_REL and err_h <= ATTN_REL
+                         and err_l <= LSE_TOL)}
+
+
+def cpu_baseline(rep, budget_s=12.0):
+    """The oracle as it stands on the host cores, whole queries until the
+    budget is spent (at least one).  The first of them is also the parity
+    record of the run: the same query (replica 0's own positions) through
+    the library, compared with the oracle by the tests' rules."""
+    rep.csa.select()
+    out_c, lse_c = rep.csa.attend()
+    out_h, lse_h = rep.hca.attend()
+    torch.cuda.synchronize()
+    got = (rep.csa.idx.cpu().numpy(), out_c.cpu().double().numpy(),
+           lse_c.cpu().double().numpy(), out_h.cpu().double().numpy(),
+           lse_h.cpu().double().numpy())
+    Lc, Lh = _cpu_layer(rep.csa_L), _cpu_layer(rep.hca_L)
+    wl = Lc["wl"]
+    t0 = time.perf_counter()
+    n = 0
+    trace = []
+    while True:
+        ref = oracle_query(Lc, Lh, trace=trace if n == 0 else None)
+        if n == 0:
+            first = ref
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    # (the comparison is not part of the timed oracle work)
+    parity = parity_record(Lc, got, trace, first)
+    parity["query"] = "replica 0 at its own " + parity["query"]
     return {"value": round(wl.B * n / dt, 4), "unit": UNIT, "cores": _threads(),
             "kind": "oracle",
             "sample": f"{n} whole decode queries (B={wl.B}) of the same workload, "
