@@ -521,6 +521,7 @@ def run_ours(args, rank, world, dev):
     traffic = _profile_traffic(_scoring_kernel(wl), wl)
     if traffic is not None:
         roofline["traffic"] = traffic
+    roofline["single_launch_floor"] = read_floor(ib, dev, peak)
     kernels = per_call_report(wl, t["calls"], peak)
 
     res = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -580,6 +581,45 @@ def _profile_traffic(kernel, wl):
     if h.hexdigest()[:16] != rec["sources_sha256_16"]:
         return None
     return int(rec["dram_bytes_per_launch"])
+
+
+def read_floor(nbytes, dev, peak, reps=24):
+    """What one launch that only reads `nbytes` reaches on this GPU: torch's
+    fp32 sum over a buffer of that size, rotated over enough buffers that
+    every launch reads HBM (more than 4x the L2).  Timed with CUDA events
+    around each launch alone, and as the mean of launches back to back; both
+    in GB/s and as a fraction of the same peak as the roofline.  A reference
+    for the scoring launch, which reads the same bytes once per call."""
+    n = max(1, int(nbytes) // 4)
+    k = max(4, math.ceil(4 * 126e6 / (4 * n)) + 1)
+    bufs = [torch.randn(n, device=dev) for _ in range(k)]
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for b in bufs:
+            b.sum()
+        stream.synchronize()
+        alone = []
+        for i in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            bufs[i % k].sum()
+            e1.record(stream)
+            stream.synchronize()
+            alone.append(e0.elapsed_time(e1))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(reps):
+            bufs[i % k].sum()
+        e1.record(stream)
+        stream.synchronize()
+        b2b = e0.elapsed_time(e1) / reps
+    del bufs
+    us_alone, us_b2b = float(np.median(alone)) * 1e3, b2b * 1e3
+    gbs = lambda us: 4 * n / (us * 1e-6) / 1e9
+    return {"what": f"torch fp32 sum over {4 * n:,} bytes per launch, {k} buffers rotated "
+                    f"(every launch reads HBM)",
+            "us_alone": round(us_alone, 3), "frac_alone": round(gbs(us_alone) / peak, 4),
+            "us_back_to_back": round(us_b2b, 3), "frac_back_to_back": round(gbs(us_b2b) / peak, 4)}
 
 
 def _pack(tensors, device, pin=False):
