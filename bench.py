@@ -590,8 +590,10 @@ def read_floor(nbytes, dev, peak, reps=24):
     around each launch alone, and as the mean of launches back to back; both
     in GB/s and as a fraction of the same peak as the roofline.  A reference
     for the scoring launch, which reads the same bytes once per call."""
-    n = max(1, int(nbytes) // 4)
-    k = max(4, math.ceil(4 * 126e6 / (4 * n)) + 1)
+    if nbytes < (8 << 20):
+        return {"what": "not measured: under 8 MB per launch (L2-resident scans)"}
+    n = int(nbytes) // 4
+    k = min(64, max(4, math.ceil(4 * 126e6 / (4 * n)) + 1))
     bufs = [torch.randn(n, device=dev) for _ in range(k)]
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
